@@ -1,0 +1,333 @@
+"""Pins for the oracle: facts fixed by the pages or by mathematics, checked without a GPU.
+
+Each test ties one part of ``oracle.wr_oracle`` to something other than itself: a worked
+example printed on the pages, a closed form, an invariant, a brute-force computation on a
+tiny input, or an independent library routine.
+"""
+import json
+import math
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+
+from oracle import wr_oracle as o
+import wr_synth
+
+
+# ---------------------------------------------------------------- pages' worked examples
+
+def test_hadamard_4x4_example(golden_dir):
+    g = json.load(open(os.path.join(golden_dir, "hadamard_4x4.json")))
+    H = o.hadamard(4)
+    assert np.array_equal(H, np.array(g["matrix_times_2"], dtype=np.float64))
+    v = np.array(g["input"])
+    out = (H / 2.0) @ v
+    assert np.allclose(out, g["output"], atol=1e-12)
+    assert math.isclose(float(v @ v), g["sum_of_squares"], rel_tol=1e-12)
+    assert math.isclose(float(out @ out), g["sum_of_squares"], rel_tol=1e-12)
+    small = np.abs(v[1:])
+    assert g["max_ratio_before_min"] <= 3.0 / small.max() + 1e-9
+    assert 3.0 / small.min() <= g["max_ratio_before_max"] + 1e-9
+    # after the rotation the largest value is close to the others
+    assert out.max() / out.min() < 1.3
+
+
+def test_grid_example(golden_dir):
+    g = json.load(open(os.path.join(golden_dir, "grid_example.json")))
+    W = np.zeros((1, 256), dtype=np.float32)
+    W[0, :4] = g["group"]
+    codes, s = o.quantize_odd_grid(W, 2)
+    assert float(s[0, 0]) == 1.0
+    levels = o.code_to_level(codes[0, :4], 2)
+    assert list(levels) == g["expected_levels"]
+    assert set(o.code_to_level(np.arange(4), 2)) == set(g["levels"])
+    # the small values are off by about 1 each, larger than the values themselves
+    err = np.abs(levels[1:] * 1.0 - np.array(g["group"][1:]))
+    assert np.all(err > np.abs(g["group"][1:]))
+
+
+def test_ledger(golden_dir):
+    g = json.load(open(os.path.join(golden_dir, "ledger.json")))
+    mods = wr_synth.QWEN3_4B_LAYER
+    assert len(mods) * wr_synth.QWEN3_4B_LAYERS == g["modules"]
+    weights = sum(K * N for _, K, N, _ in mods)
+    assert round(weights * wr_synth.QWEN3_4B_LAYERS / 1e9, 2) == g["body_weights_billions"]
+    code_bits = sum(K * N * b for _, K, N, b in mods) / weights
+    assert abs(code_bits - g["code_bits_per_weight"]) < 1e-3      # 2.5195 vs the printed 2.520
+    # packed sizes of the layout match the code ledger exactly (N multiple of 16)
+    packed = sum(o.packed_bytes(b, N, K) for _, K, N, b in mods)
+    assert packed * 8 == sum(K * N * b for _, K, N, b in mods)
+
+
+def test_ternary_bits_per_weight():
+    # 5 trits per byte: 1.6 bits per weight when K is a multiple of 320 (K = 2560)
+    assert o.packed_bytes(o.FMT_TERNARY, 16, 2560) * 8 / (16 * 2560) == pytest.approx(1.6)
+    # K = 4096 pads to 4160 trits: 1.625 bits per weight
+    assert o.packed_bytes(o.FMT_TERNARY, 16, 4096) * 8 / (16 * 4096) == pytest.approx(1.625)
+
+
+# ---------------------------------------------------------------- Hadamard and rotation
+
+def _fwht_python(v):
+    """Textbook in-place butterfly, pure Python, unnormalized."""
+    v = list(v)
+    h = 1
+    while h < len(v):
+        for i in range(0, len(v), 2 * h):
+            for j in range(i, i + h):
+                a, b = v[j], v[j + h]
+                v[j], v[j + h] = a + b, a - b
+        h *= 2
+    return v
+
+
+@pytest.mark.parametrize("n", [2, 4, 8, 16, 32, 64, 128])
+def test_hadamard_orthogonal(n):
+    H = o.hadamard(n)
+    assert np.array_equal(H @ H.T, n * np.eye(n))
+
+
+def test_rotation_is_orthogonal_and_matches_butterfly():
+    K = 384
+    signs = wr_synth.sign_bits(7, K)
+    R = o.rotate(np.eye(K), signs).T          # column k = R e_k
+    assert np.allclose(R.T @ R, np.eye(K), atol=1e-13)
+    d = [(-1.0 if (int(signs[k // 32]) >> (k % 32)) & 1 else 1.0) for k in range(K)]
+    rng = np.random.default_rng(3)
+    v = rng.standard_normal(K)
+    ref = []
+    for b in range(K // 128):
+        blk = [v[k] * d[k] for k in range(128 * b, 128 * b + 128)]
+        ref += [t / math.sqrt(128) for t in _fwht_python(blk)]
+    assert np.allclose(o.rotate(v, signs), ref, atol=1e-13)
+
+
+def test_rotation_preserves_products():
+    # W x = (W R^T)(R x): the stored weights are rotated, the input is rotated in-kernel
+    K, N, M = 512, 24, 3
+    signs = wr_synth.sign_bits(11, K)
+    W = wr_synth.weights_fp32(5, N, K).astype(np.float64)
+    x = wr_synth.bf16_bits_to_f32(wr_synth.activations_bf16(6, M, K)).astype(np.float64)
+    y = x @ W.T
+    yr = o.rotate(x, signs) @ o.rotate(W, signs).T
+    assert np.allclose(y, yr, rtol=1e-12, atol=1e-13)
+
+
+def test_sign_vector_bits():
+    w = np.array([0b1011, 0x80000000], dtype=np.uint32)
+    d = o.sign_vector(w, 64)
+    assert list(d[:5]) == [-1, -1, 1, -1, 1]
+    assert d[63] == -1 and d[62] == 1
+
+
+# ---------------------------------------------------------------- scalar conversions
+
+def _fp16_exact_rne(x: Fraction) -> Fraction:
+    """Round a positive rational to fp16 by exact arithmetic (normal and subnormal)."""
+    if x == 0:
+        return Fraction(0)
+    e = math.floor(math.log2(x))
+    while Fraction(2) ** e > x:
+        e -= 1
+    while Fraction(2) ** (e + 1) <= x:
+        e += 1
+    e = max(e, -14)
+    ulp = Fraction(2) ** (e - 10)
+    q = x / ulp
+    fl = math.floor(q)
+    rem = q - fl
+    if rem > Fraction(1, 2) or (rem == Fraction(1, 2) and fl % 2 == 1):
+        fl += 1
+    return fl * ulp
+
+
+def test_fp16_round_matches_exact_rounding():
+    rng = np.random.default_rng(0)
+    vals = list(rng.uniform(1e-6, 1.0, 200)) + [1 + 2 ** -11, 1 + 2 ** -11 + 2 ** -40,
+                                                 3 * 2 ** -20, 0.0612 / 3, 0.02 / 7]
+    for v in vals:
+        exact = _fp16_exact_rne(Fraction(v))
+        assert Fraction(float(o.fp16_round(np.float64(v)))) == exact, v
+
+
+def test_bf16_conversions_match_torch():
+    torch = pytest.importorskip("torch")
+    rng = np.random.default_rng(1)
+    s = rng.uniform(1e-3, 0.1, 4096).astype(np.float16).astype(np.float64)
+    g = rng.integers(-3, 4, 4096) * 2 + 1
+    w = s * g
+    mine = o.f64_to_bf16_bits(w)
+    ref = torch.from_numpy(w).to(torch.float32).to(torch.bfloat16).view(torch.int16).numpy()
+    assert np.array_equal(mine, ref.view(np.uint16))
+    back = o.bf16_bits_to_f64(mine)
+    ref_back = torch.from_numpy(ref).view(torch.bfloat16).to(torch.float64).numpy()
+    assert np.array_equal(back, ref_back)
+
+
+# ---------------------------------------------------------------- quantizer
+
+@pytest.mark.parametrize("bits", [2, 3])
+def test_nearest_point_against_brute_force(bits):
+    L = o.grid_L(bits)
+    W = wr_synth.weights_fp32(21 + bits, 8, 512)
+    codes, s = o.quantize_odd_grid(W, bits)
+    levels = np.arange(-L, L + 1, 2)
+    for n in range(8):
+        for k in range(0, 512, 7):
+            sc = float(s[n, k // 256])
+            absmax = float(np.abs(W[n, (k // 256) * 256:(k // 256 + 1) * 256]).max())
+            assert Fraction(sc) == _fp16_exact_rne(Fraction(absmax) / L)
+            q = float(W[n, k]) / sc
+            dist = np.abs(levels - q)
+            best = levels[dist == dist.min()].max()    # ties go to the larger level
+            assert o.code_to_level(codes[n, k], bits) == best
+
+
+def test_quantizer_special_blocks():
+    W = np.zeros((2, 512), dtype=np.float32)
+    W[1, 256:] = -0.5
+    W[1, 300] = 0.25
+    codes, s = o.quantize_odd_grid(W, 2)
+    assert float(s[0, 0]) == 0.0 and np.all(o.code_to_level(codes[0], 2) == 1)
+    # block of constant -0.5: s = 0.5/3 rounded to fp16, all codes at -3
+    assert float(s[1, 1]) == float(np.float16(0.5 / 3))
+    assert o.code_to_level(codes[1, 257], 2) == -3
+    assert o.code_to_level(codes[1, 300], 2) == 1     # 0.25/s = 1.5 -> nearest odd is 1
+
+
+def test_dequant_hand_examples():
+    codes = np.array([[0, 3] + [1] * 254, [7, 4] + [0] * 254], dtype=np.uint8)
+    s2 = np.array([[0.5]], dtype=np.float16)
+    W = o.dequant(codes[:1, :256] & 3, s2, 2)
+    assert W[0, 0] == -1.5 and W[0, 1] == 1.5 and W[0, 2] == -0.5
+    s3 = np.array([[2.0]], dtype=np.float16)
+    W3 = o.dequant(codes[1:, :256], s3, 3)
+    assert W3[0, 0] == 14.0 and W3[0, 1] == 2.0 and W3[0, 2] == -14.0
+    tiny = np.array([[2.0 ** -24]], dtype=np.float16)       # smallest fp16 subnormal
+    assert o.dequant(codes[1:, :256], tiny, 3)[0, 0] == 7 * 2.0 ** -24
+    assert np.all(o.dequant(codes[1:, :256], np.zeros((1, 1), np.float16), 3) == 0)
+
+
+def test_ternary_quantizer_rules():
+    K, N = 512, 16
+    signs = wr_synth.sign_bits(3, K)
+    W = wr_synth.weights_fp32(4, N, K)
+    codes, alpha, Wr = o.quantize_ternary(W, signs)
+    t = codes.astype(np.int64) - 1
+    for n in range(N):
+        a = np.abs(Wr[n])
+        delta = 0.7 * a.mean()
+        assert np.array_equal(t[n] != 0, a > delta)
+        assert np.array_equal(np.sign(Wr[n])[t[n] != 0], t[n][t[n] != 0])
+        # alpha is the least-squares scale for fixed t (then rounded to fp16)
+        best = float(np.dot(np.abs(Wr[n]), np.abs(t[n])) / np.abs(t[n]).sum())
+        f = lambda al: float(((Wr[n] - al * t[n]) ** 2).sum())
+        assert f(best) <= min(f(best * 1.001), f(best * 0.999))
+        assert float(alpha[n]) == float(np.float16(best))
+
+
+# ---------------------------------------------------------------- contraction
+
+def _brute(x_bits, codes, scales, bits):
+    M, K = x_bits.shape
+    N = codes.shape[0]
+    L = (1 << bits) - 1
+    xf = [[float(v) for v in row] for row in wr_synth.bf16_bits_to_f32(x_bits)]
+    y = [[0.0] * N for _ in range(M)]
+    for m in range(M):
+        for n in range(N):
+            acc = Fraction(0)
+            for k in range(K):
+                g = 2 * int(codes[n, k]) - L
+                acc += Fraction(float(scales[n, k // 256])) * g * Fraction(xf[m][k])
+            y[m][n] = float(acc)
+    return np.array(y)
+
+
+@pytest.mark.parametrize("bits", [2, 3])
+def test_gemm_against_exact_brute_force(bits):
+    M, N, K = 2, 5, 512
+    W = wr_synth.weights_fp32(31, N, K)
+    codes, s = o.quantize_odd_grid(W, bits)
+    x = wr_synth.activations_bf16(32, M, K)
+    y, B = o.gemm_codes(x, codes, s, bits)
+    ref = _brute(x, codes, s, bits)
+    assert np.allclose(y, ref, rtol=1e-13, atol=1e-14)
+    assert np.all(B >= np.abs(y))
+
+
+def test_gemm_special_cases():
+    K, N = 512, 4
+    codes = np.full((N, K), 3, dtype=np.uint8)        # level +3 everywhere (2-bit)
+    s = np.full((N, 2), 0.25, dtype=np.float16)
+    x = wr_synth.activations_bf16(9, 1, K)
+    xf = wr_synth.bf16_bits_to_f32(x).astype(np.float64)
+    y, _ = o.gemm_codes(x, codes, s, 2)
+    assert np.allclose(y, 3 * 0.25 * xf.sum(), rtol=1e-14)
+    # one-hot x picks a column of W
+    W = wr_synth.weights_fp32(10, N, K)
+    codes, s = o.quantize_odd_grid(W, 3)
+    onehot = np.zeros((1, K), dtype=np.uint16)
+    onehot[0, 300] = 0x3F80                             # bf16 1.0
+    y, _ = o.gemm_codes(onehot, codes, s, 3)
+    assert np.array_equal(y[0], o.dequant(codes, s, 3)[:, 300])
+
+
+def test_ternary_gemm_matches_rotation_identity():
+    K, N, M = 640, 16, 2
+    signs = wr_synth.sign_bits(12, K)
+    W = wr_synth.weights_fp32(13, N, K)
+    codes, alpha, _ = o.quantize_ternary(W, signs)
+    x = wr_synth.activations_bf16(14, M, K)
+    y, B = o.gemm_ternary(x, codes, alpha, signs)
+    # same result from the unrotated dense weight R^T (alpha t) applied to plain x
+    Wt = o.dequant_ternary(codes, alpha)
+    R = o.rotate(np.eye(K), signs).T       # column k is R e_k
+    dense = Wt @ R                         # (alpha t) R: the weights in the unrotated basis
+    xf = wr_synth.bf16_bits_to_f32(x).astype(np.float64)
+    assert np.allclose(y, xf @ dense.T, rtol=1e-11, atol=1e-12)
+    assert np.all(B >= np.abs(y) - 1e-12)
+
+
+# ---------------------------------------------------------------- packed layout
+
+def test_pack_golden_vectors(golden_dir):
+    g = json.load(open(os.path.join(golden_dir, "pack_vectors.json")))
+    for case in g["cases"]:
+        fmt, N, K = case["fmt"], case["N"], case["K"]
+        codes = np.full((N, K), case["fill"], dtype=np.uint8)
+        for n, k, c in case["set"]:
+            codes[n, k] = c
+        p = o.pack(fmt, codes)
+        assert p.size == o.packed_bytes(fmt, N, K)
+        for idx, val in case["expect"].items():
+            assert int(p[int(idx)]) == val, (case["fmt"], idx)
+        # every byte not listed holds the fill pattern
+        fillbyte = 121 if fmt == o.FMT_TERNARY else 0
+        listed = {int(i) for i in case["expect"]}
+        others = np.array([i for i in range(p.size) if i not in listed])
+        nz = others[p[others] != fillbyte]
+        assert nz.size == 0, (fmt, nz[:10])
+        assert np.array_equal(o.unpack_codes(fmt, p, N, K), codes)
+
+
+@pytest.mark.parametrize("fmt,levels,N,K", [(2, 4, 48, 768), (3, 8, 40, 512), (1, 3, 35, 700),
+                                             (1, 3, 16, 2560), (2, 4, 1, 256)])
+def test_pack_round_trip(fmt, levels, N, K):
+    rng = np.random.default_rng(fmt * 100 + N)
+    codes = rng.integers(0, levels, (N, K)).astype(np.uint8)
+    p = o.pack(fmt, codes)
+    assert np.array_equal(o.unpack_codes(fmt, p, N, K), codes)
+
+
+def test_pack_is_a_bijection_on_bytes():
+    # Q2/Q3 with N % 16 == 0 use every bit exactly once: distinct code arrays give
+    # distinct byte arrays and the byte count equals the bit count / 8
+    for fmt, b in ((2, 2), (3, 3)):
+        N, K = 16, 256
+        byte, bit = o.code_bit_positions(fmt, N, K)
+        flat = (byte.astype(np.int64) * 8 + bit).ravel()
+        assert np.unique(flat).size == flat.size == N * K * b
+        assert flat.max() < o.packed_bytes(fmt, N, K) * 8
