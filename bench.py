@@ -1,0 +1,464 @@
+#!/usr/bin/env python
+"""Benchmark of the packed-code weight-only GEMV/GEMM on B200 (one JSON line on rank 0).
+
+Headline workload: decode of one token (M = 1) through the 36-layer Qwen3-4B-shaped body,
+252 packed GEMVs back to back (v/up/down at 3 bits, the rest at 2 bits, fp16 block-256
+scales), each module with its own seeded weights and a fresh seeded bf16 input. One step is
+one pass over the body, captured in a CUDA graph. The packed body is 1.18 GB, larger than L2
+(126 MB), so every step streams the weights from HBM.
+
+Extra keys report the other rows of the path on the same synthetic recipe: the M = 8 body,
+single-linear and per-module GEMVs, the prefill GEMM sweep (TFLOP/s), the ternary body and
+the bf16 materializer. `--impl reference` times the fp64 CPU oracle on the host cores on a
+bounded sample of the same workload instead.
+
+Multi-GPU (torchrun): the path needs no exchange; each rank runs its own replica of the
+body, the step time is the max over ranks and `value` is the aggregate over all ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "decode GEMV HBM GB/s (% of 8 TB/s) & tokens/s; prefill GEMM TFLOP/s (% peak)"
+HBM_FALLBACK_GBS, BF16_FALLBACK_TFLOPS = 6650.0, 1590.0
+
+
+def parse_args():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", choices=["wr", "reference"], default="wr")
+    p.add_argument("--layers", type=int, default=36)
+    p.add_argument("--no-extras", action="store_true", help="headline body only")
+    p.add_argument("--cpu-seconds", type=float, default=12.0, help="oracle sample budget")
+    return p.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        d = json.load(open(path))
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), float(d.get("bf16_tflops_sustained", d["bf16_tflops"])), "measured"
+    except Exception:
+        return HBM_FALLBACK_GBS, BF16_FALLBACK_TFLOPS, 1400.0, "fallback"
+
+
+# ------------------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while the timed region runs."""
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid: str | None):
+        self.uuid, self.rows, self.proc = uuid, [], None
+
+    def __enter__(self):
+        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "100"]
+        if self.uuid:
+            cmd += ["-i", self.uuid]
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.rows.append([c.strip() for c in line.split(",")])
+
+    def __exit__(self, *exc):
+        if self.proc:
+            time.sleep(0.2)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in self.rows:
+            try:
+                sm.append(float(r[0]))
+                mx.append(float(r[1]))
+                for i, nm in enumerate(names):
+                    if r[4 + i].lower().startswith("active"):
+                        reasons.add(nm)
+            except Exception:
+                continue
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------------------ workloads
+
+def body_modules(layers: int):
+    import wr_synth
+    for layer in range(layers):
+        for idx, (name, K, N, bits) in enumerate(wr_synth.QWEN3_4B_LAYER):
+            yield layer, idx, name, K, N, bits
+
+
+def build_q_module(wr, torch, seed, N, K, bits):
+    import numpy as np
+    import wr_synth
+    W = wr_synth.weights_fp32(seed, N, K)
+    codes, scales = wr.wr_quantize(bits, W)
+    packed = wr.wr_pack(bits, codes)
+    return (torch.from_numpy(packed).cuda(), torch.from_numpy(scales.view(np.int16)).cuda())
+
+
+def module_bytes(wr, M, N, K, bits):
+    fmt = bits
+    return wr.wr_packed_bytes(fmt, N, K) + N * (K // 256) * 2 + M * K * 2 + M * N * 4
+
+
+def graph_time_ms(torch, fn, steps, warmup, stream, dist=None):
+    """Capture fn() once in a CUDA graph; replay `warmup` times, then time `steps` replays with
+    CUDA events recorded on the stream the replays are launched on, with a barrier and a
+    device synchronize on both sides."""
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(stream):
+        fn()                                   # one eager pass (lazy init outside capture)
+        torch.cuda.synchronize()
+        with torch.cuda.graph(g, stream=stream):
+            fn()
+        for _ in range(warmup):
+            g.replay()
+        torch.cuda.synchronize()
+        if dist:
+            dist.barrier()
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        assert torch.cuda.current_stream() == stream
+        start.record(stream)
+        for _ in range(steps):
+            g.replay()
+        end.record(stream)
+        torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    ms = start.elapsed_time(end)
+    del g
+    return ms
+
+
+def max_over_ranks(torch, dist, v):
+    if not dist:
+        return v
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------------------ reference arm
+
+def cpu_oracle_sample(budget_s: float, M: int = 1):
+    """Time the fp64 oracle on modules of the body, in order, until the budget is used."""
+    import numpy as np
+    import wr_synth
+    from oracle import wr_oracle as o
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([d.get("num_threads", 1) for d in threadpool_info()] + [1])
+    except Exception:
+        cores = os.cpu_count() or 1
+    done_bytes, t_total, mods = 0, 0.0, []
+    for layer, idx, name, K, N, bits in body_modules(36):
+        W = wr_synth.weights_fp32(wr_synth.module_seed(layer, idx), N, K)
+        codes, scales = o.quantize_odd_grid(W, bits)
+        x = wr_synth.activations_bf16(10_000 + 10 * layer + idx, M, K)
+        t0 = time.perf_counter()
+        o.gemm_codes(x, codes, scales, bits)
+        t_total += time.perf_counter() - t0
+        done_bytes += (o.packed_bytes(bits, N, K) + N * (K // 256) * 2 + M * K * 2 + M * N * 4)
+        mods.append(f"L{layer}.{name}")
+        if t_total >= budget_s:
+            break
+    return {"value": done_bytes / t_total / 1e9, "unit": "GB/s", "cores": cores, "kind": "oracle",
+            "sample": f"{len(mods)} body modules at M={M} ({mods[0]}..{mods[-1]}), fp64 dequant + "
+                      f"matmul, {t_total:.1f} s of CPU time"}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    per_step = []
+    for _ in range(args.warmup):
+        cpu_oracle_sample(0.5)
+    for _ in range(args.steps):
+        per_step.append(cpu_oracle_sample(max(0.5, args.cpu_seconds / max(args.steps, 1))))
+    gbs = statistics.median(s["value"] for s in per_step)
+    tokps = gbs * 1e9 / 1_178_984_448
+    cb = dict(per_step[-1])
+    cb["value"] = gbs
+    line = {"impl": "reference", "metric": METRIC, "value": gbs, "unit": "GB/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 / tokps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "tokens_per_s": tokps,
+            "config": {"workload": "qwen3-4b body, 36 layers x 7 packed GEMVs, M=1 (oracle sample)",
+                       "model": "Qwen3-4B-shaped linears", "global_batch": 1, "seq_len": 1,
+                       "parallelism": "replicas"},
+            "cpu_baseline": cb,
+            "e2e": {"value": gbs, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------------------ main arm
+
+def main():
+    args = parse_args()
+    rank, world = int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1))
+    local_rank = int(os.environ.get("LOCAL_RANK", 0))
+    if world > 1:
+        os.environ["CUDA_VISIBLE_DEVICES"] = str(local_rank)
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    import numpy as np
+    import torch
+    import bit_weight_only_wr_b200 as wr
+    import wr_synth
+
+    torch.cuda.set_device(0)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as tdist
+        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                 device_id=torch.device("cuda", 0))
+        dist = tdist
+    hbm_peak, bf16_peak, bf16_sust, peak_kind = peaks()
+    stream = torch.cuda.Stream()
+    uuid = None
+    try:
+        uuid = str(torch.cuda.get_device_properties(0).uuid)
+        uuid = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+    except Exception:
+        pass
+
+    # ---- the body: weights resident in HBM, fresh x per module
+    t_setup = time.time()
+    mods = []
+    for layer, idx, name, K, N, bits in body_modules(args.layers):
+        packed, scales = build_q_module(wr, torch, wr_synth.module_seed(layer, idx), N, K, bits)
+        mods.append(dict(layer=layer, name=name, K=K, N=N, bits=bits, packed=packed, scales=scales))
+    setup_s = time.time() - t_setup
+
+    def body_run(M, steps, warmup, with_e2e):
+        xs_host = [wr_synth.activations_bf16(10_000 + 10 * m["layer"] + i % 7, M, m["K"])
+                   for i, m in enumerate(mods)]
+        x_all = torch.from_numpy(np.concatenate([x.ravel() for x in xs_host]).view(np.int16)).cuda()
+        offs, o_ = [], 0
+        for x in xs_host:
+            offs.append(o_)
+            o_ += x.size
+        y_all = torch.empty(sum(M * m["N"] for m in mods), dtype=torch.float32, device="cuda")
+        yoffs, o_ = [], 0
+        for m in mods:
+            yoffs.append(o_)
+            o_ += M * m["N"]
+        nb = max(wr.wr_gemv_workspace_bytes(M, m["N"], m["K"], m["bits"]) for m in mods)
+        ws = torch.zeros(nb, dtype=torch.uint8, device="cuda")
+        xp, yp = x_all.data_ptr(), y_all.data_ptr()
+
+        def step():
+            for i, m in enumerate(mods):
+                wr.wr_gemv(M, m["N"], m["K"], xp + 2 * offs[i], m["packed"], m["scales"], m["bits"],
+                           yp + 4 * yoffs[i], ws, nb)
+        ms = graph_time_ms(torch, step, steps, warmup, stream, dist) / steps
+        ms = max_over_ranks(torch, dist, ms)
+        nbytes = sum(module_bytes(wr, M, m["N"], m["K"], m["bits"]) for m in mods)
+        out = {"ms": ms, "bytes": nbytes, "gbs": nbytes / ms / 1e6, "launches": len(mods)}
+        if with_e2e:
+            xh = x_all.cpu().pin_memory()
+            yh = torch.empty(y_all.numel(), dtype=torch.float32).pin_memory()
+
+            def e2e_step():
+                x_all.copy_(xh, non_blocking=True)
+                step()
+                yh.copy_(y_all, non_blocking=True)
+            ms_e = graph_time_ms(torch, e2e_step, steps, warmup, stream, dist) / steps
+            ms_e = max_over_ranks(torch, dist, ms_e)
+            out["e2e"] = {"ms": ms_e, "gbs": nbytes / ms_e / 1e6, "h2d": x_all.numel() * 2,
+                          "d2h": y_all.numel() * 4}
+        return out
+
+    with ClockSampler(uuid) as clk:
+        head = body_run(1, args.steps, args.warmup, True)
+    clocks = clk.summary()
+    total_gbs = head["gbs"] * world
+    tokens_per_s = world * 1e3 / head["ms"]
+
+    extras = {}
+    if not args.no_extras:
+        try:
+            extras["body_m8"] = {k: v for k, v in body_run(8, max(5, args.steps // 2), 3, False).items()}
+            extras["body_m8"]["tokens_per_s"] = 8e3 / extras["body_m8"]["ms"]
+        except Exception as e:  # noqa: BLE001
+            extras["body_m8"] = {"error": repr(e)}
+        extras.update(run_extras(args, wr, torch, np, stream, dist, hbm_peak, bf16_peak))
+
+    # the graph holds only GEMV launches: bytes per launch / time per launch = bytes / step time
+    achieved = head["gbs"]
+    roof = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+            "frac": achieved / hbm_peak, "traffic": None, "peak_kind": peak_kind,
+            "kernel": "gemv_q_kernel (2/3-bit decode GEMV)",
+            "note": "average GEMV launch in the M=1 body graph: algorithmic bytes per launch / "
+                    "event-timed duration per launch"}
+    cb = None
+    if rank == 0 and world == 1:
+        try:
+            cb = cpu_oracle_sample(args.cpu_seconds)
+        except Exception as e:  # noqa: BLE001
+            cb = {"error": repr(e)}
+    line = {
+        "metric": METRIC, "value": total_gbs, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": head["ms"], "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "tokens_per_s": tokens_per_s, "pct_of_8TBps": 100.0 * head["gbs"] / 8000.0,
+        "config": {"workload": f"qwen3-4b body, {args.layers} layers x 7 packed GEMVs (v/up/down 3-bit, "
+                               "others 2-bit, fp16 block-256 scales), M=1 decode",
+                   "model": "Qwen3-4B-shaped linears (synthetic, W~N(0,0.02), x~N(0,1) bf16)",
+                   "global_batch": world, "seq_len": 1, "parallelism": f"replicas x{world}",
+                   "l2": "inputs larger than L2 (1.18 GB of packed weights per step)",
+                   "bytes_per_step": head["bytes"], "setup_s": round(setup_s, 1)},
+        "roofline": roof, "cpu_baseline": cb, "clocks": clocks,
+        "e2e": {"value": head["e2e"]["gbs"] * world, "unit": "GB/s",
+                "h2d_bytes_per_step": head["e2e"]["h2d"], "d2h_bytes_per_step": head["e2e"]["d2h"],
+                "ms_per_step": head["e2e"]["ms"]},
+        "gpu_launches": head["launches"] * args.steps,
+        "extras": extras,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def run_extras(args, wr, torch, np, stream, dist, hbm_peak, bf16_peak):
+    """Other rows of the path: per-module GEMVs over rotating copies, single linear, unpack,
+    prefill GEMM sweep and the ternary body."""
+    import wr_synth
+    out = {}
+    l2 = torch.cuda.get_device_properties(0).L2_cache_size
+
+    # config 0: single 2560x2560 2-bit linear, M=1, rotating over >= 3x L2 of distinct copies
+    try:
+        N = K = 2560
+        per = wr.wr_packed_bytes(2, N, K) + N * (K // 256) * 2
+        copies = max(3, int(3 * l2 // per) + 1)
+        base_p, base_s = build_q_module(wr, torch, 0, N, K, 2)
+        ps = [base_p.roll(i * 1024) for i in range(copies)]      # distinct buffers, same statistics
+        x = torch.from_numpy(wr_synth.activations_bf16(1, 1, K).view(np.int16)).cuda()
+        y = torch.empty(1, N, dtype=torch.float32, device="cuda")
+        nb = wr.wr_gemv_workspace_bytes(1, N, K, 2)
+        ws = torch.zeros(nb, dtype=torch.uint8, device="cuda")
+
+        def step():
+            for p in ps:
+                wr.wr_gemv(1, N, K, x, p, base_s, 2, y, ws, nb)
+        ms = graph_time_ms(torch, step, 10, 3, stream) / 10 / copies
+        b = module_bytes(wr, 1, N, K, 2)
+        out["single_linear_2560"] = {"us": ms * 1e3, "gbs": b / ms / 1e6, "bytes": b, "copies": copies}
+    except Exception as e:  # noqa: BLE001
+        out["single_linear_2560"] = {"error": repr(e)}
+
+    # unpack (materializer) on the gate shape, rotating copies
+    try:
+        N, K = 9728, 2560
+        p, s = build_q_module(wr, torch, 7, N, K, 2)
+        w = torch.empty(N, K, dtype=torch.int16, device="cuda")
+
+        def step():
+            wr.wr_unpack_bf16(2, N, K, p, s, w)
+        ms = graph_time_ms(torch, step, 20, 3, stream) / 20
+        b = wr.wr_packed_bytes(2, N, K) + N * (K // 256) * 2 + N * K * 2
+        out["unpack_bf16_gate"] = {"us": ms * 1e3, "gbs": b / ms / 1e6}
+    except Exception as e:  # noqa: BLE001
+        out["unpack_bf16_gate"] = {"error": repr(e)}
+
+    # prefill sweep
+    try:
+        res = {}
+        shapes = [("gate", 2560, 9728, 2), ("up", 2560, 9728, 3), ("down", 9728, 2560, 3)]
+        for name, K, N, bits in shapes:
+            p, s = build_q_module(wr, torch, 5000 + K, N, K, bits)
+            for M in (16, 128, 512, 2048, 4096):
+                x = torch.from_numpy(wr_synth.activations_bf16(M, M, K).view(np.int16)).cuda()
+                y = torch.empty(M, N, dtype=torch.float32, device="cuda")
+                nb = wr.wr_gemm_workspace_bytes(M, N, K, bits)
+                ws = torch.zeros(max(nb, 256), dtype=torch.uint8, device="cuda")
+
+                def step():
+                    wr.wr_gemm(M, N, K, x, p, s, bits, y, ws, nb)
+                reps = 5 if M >= 2048 else 10
+                ms = graph_time_ms(torch, step, reps, 2, stream) / reps
+                tf = 2.0 * M * N * K / ms / 1e9
+                b = module_bytes(wr, M, N, K, bits)
+                res[f"{name}_M{M}"] = {"us": ms * 1e3, "tflops": tf, "pct_bf16_peak": 100 * tf / bf16_peak,
+                                       "gbs": b / ms / 1e6}
+        out["prefill"] = res
+    except Exception as e:  # noqa: BLE001
+        out["prefill"] = {"error": repr(e)}
+
+    # ternary: one layer's 7 shapes at M=1 (rotating over 6 copies of the layer > L2)
+    try:
+        mods = []
+        for idx, (name, K, N, _) in enumerate(wr_synth.QWEN3_4B_LAYER):
+            signs = wr_synth.sign_bits(900 + idx, K)
+            W = wr_synth.weights_fp32(800 + idx, N, K)
+            codes, alpha = wr.wr_quantize_ternary(W, signs)
+            packed = wr.wr_pack(1, codes)
+            mods.append(dict(K=K, N=N, p=torch.from_numpy(packed).cuda(),
+                             a=torch.from_numpy(alpha.view(np.int16)).cuda(),
+                             s=torch.from_numpy(signs.view(np.int32)).cuda()))
+        per_layer = sum(m["p"].numel() for m in mods)
+        copies = max(1, int(3 * l2 // per_layer) + 1)
+        res = {}
+        for M in (1, 512):
+            xs = [torch.from_numpy(wr_synth.activations_bf16(M + i, M, m["K"]).view(np.int16)).cuda()
+                  for i, m in enumerate(mods)]
+            ys = [torch.empty(M, m["N"], dtype=torch.float32, device="cuda") for m in mods]
+            nb = max(wr.wr_gemm_ternary_workspace_bytes(M, m["N"], m["K"]) for m in mods)
+            ws = torch.zeros(nb, dtype=torch.uint8, device="cuda")
+            rolled = [[m["p"].roll(c * 1024) for m in mods] for c in range(copies if M == 1 else 1)]
+
+            def step():
+                for c in range(len(rolled)):
+                    for i, m in enumerate(mods):
+                        wr.wr_gemm_ternary(M, m["N"], m["K"], xs[i], rolled[c][i], m["a"], m["s"], ys[i], ws, nb)
+            reps = 10 if M == 1 else 3
+            ms = graph_time_ms(torch, step, reps, 2, stream) / reps / len(rolled)
+            b = sum(m["p"].numel() + 2 * m["N"] + 4 * ((m["K"] + 31) // 32) + 2 * M * m["K"] + 4 * M * m["N"]
+                    for m in mods)
+            fl = sum(2.0 * M * m["N"] * m["K"] for m in mods)
+            res[f"layer_M{M}"] = {"us": ms * 1e3, "gbs": b / ms / 1e6, "tflops": fl / ms / 1e9,
+                                  "tokens_per_s_layer": M * 1e3 / ms}
+        out["ternary"] = res
+    except Exception as e:  # noqa: BLE001
+        out["ternary"] = {"error": repr(e)}
+    return out
+
+
+if __name__ == "__main__":
+    main()

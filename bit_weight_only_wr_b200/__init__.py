@@ -1,0 +1,187 @@
+"""Python binding of libwr (packed low-bit weight-only GEMV/GEMM for B200).
+
+Argument marshalling only: every function forwards to the C entry point of the same name in
+``libwr.so`` (declared in ``include/wr.h``). Device operands are torch CUDA tensors (or raw
+device addresses as ints); torch supplies device memory and the current stream, nothing else.
+Importing this module fails loudly when the shared library has not been built.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+
+__all__ = [
+    "WR_FMT_TERNARY", "WR_FMT_Q2", "WR_FMT_Q3", "WrError", "LIB_PATH",
+    "wr_abi_version", "wr_status_string", "wr_packed_bytes", "wr_pack", "wr_unpack_codes",
+    "wr_quantize", "wr_quantize_ternary", "wr_unpack_bf16", "wr_gemv_workspace_bytes", "wr_gemv",
+    "wr_gemm_workspace_bytes", "wr_gemm", "wr_gemm_ternary_workspace_bytes", "wr_gemm_ternary",
+    "wr_get_device_error", "exported_symbols",
+]
+
+WR_FMT_TERNARY, WR_FMT_Q2, WR_FMT_Q3 = 1, 2, 3
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libwr.so")
+
+_c_i64, _c_int, _c_size, _vp = ctypes.c_int64, ctypes.c_int, ctypes.c_size_t, ctypes.c_void_p
+
+_SIGNATURES = {
+    "wr_abi_version": (_c_int, []),
+    "wr_status_string": (ctypes.c_char_p, [_c_int]),
+    "wr_packed_bytes": (_c_size, [_c_int, _c_i64, _c_i64]),
+    "wr_pack": (_c_int, [_c_int, _c_i64, _c_i64, _vp, _vp]),
+    "wr_unpack_codes": (_c_int, [_c_int, _c_i64, _c_i64, _vp, _vp]),
+    "wr_quantize": (_c_int, [_c_int, _c_i64, _c_i64, _vp, _vp, _vp]),
+    "wr_quantize_ternary": (_c_int, [_c_i64, _c_i64, _vp, _vp, _vp, _vp]),
+    "wr_unpack_bf16": (_c_int, [_c_int, _c_i64, _c_i64, _vp, _vp, _c_int, _vp, _vp]),
+    "wr_gemv_workspace_bytes": (_c_size, [_c_i64, _c_i64, _c_i64, _c_int]),
+    "wr_gemv": (_c_int, [_c_i64, _c_i64, _c_i64, _vp, _vp, _vp, _c_int, _c_int, _vp, _vp, _c_size, _vp]),
+    "wr_gemm_workspace_bytes": (_c_size, [_c_i64, _c_i64, _c_i64, _c_int]),
+    "wr_gemm": (_c_int, [_c_i64, _c_i64, _c_i64, _vp, _vp, _vp, _c_int, _c_int, _vp, _vp, _c_size, _vp]),
+    "wr_gemm_ternary_workspace_bytes": (_c_size, [_c_i64, _c_i64, _c_i64]),
+    "wr_gemm_ternary": (_c_int, [_c_i64, _c_i64, _c_i64, _vp, _vp, _vp, _vp, _vp, _vp, _c_size, _vp]),
+    "wr_get_device_error": (_c_int, [_vp]),
+}
+
+
+def exported_symbols():
+    """Names of the C entry points this binding expects libwr.so to export."""
+    return sorted(_SIGNATURES)
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"libwr.so not found at {LIB_PATH}; build it with "
+                          "`python bit_weight_only_wr_b200/build.py` (nvcc, sm_100a)")
+    lib = ctypes.CDLL(LIB_PATH)
+    for name, (res, args) in _SIGNATURES.items():
+        fn = getattr(lib, name)
+        fn.restype, fn.argtypes = res, args
+    return lib
+
+
+_lib = _load()
+
+
+class WrError(RuntimeError):
+    def __init__(self, func: str, status: int):
+        super().__init__(f"{func}: {wr_status_string(status)} (status {status})")
+        self.status = status
+
+
+def _check(func: str, st: int) -> None:
+    if st != 0:
+        raise WrError(func, st)
+
+
+def _ptr(t) -> int | None:
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    if isinstance(t, np.ndarray):
+        return t.ctypes.data
+    return t.data_ptr()
+
+
+def _stream(stream) -> int | None:
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def wr_abi_version() -> int:
+    return _lib.wr_abi_version()
+
+
+def wr_status_string(st: int) -> str:
+    return _lib.wr_status_string(st).decode()
+
+
+def wr_packed_bytes(fmt: int, N: int, K: int) -> int:
+    return _lib.wr_packed_bytes(fmt, N, K)
+
+
+def wr_pack(fmt: int, codes: np.ndarray) -> np.ndarray:
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    N, K = codes.shape
+    nb = wr_packed_bytes(fmt, N, K)
+    if nb == 0:
+        raise WrError("wr_pack", 1)
+    out = np.empty(nb, dtype=np.uint8)
+    _check("wr_pack", _lib.wr_pack(fmt, N, K, _ptr(codes), _ptr(out)))
+    return out
+
+
+def wr_unpack_codes(fmt: int, packed: np.ndarray, N: int, K: int) -> np.ndarray:
+    packed = np.ascontiguousarray(packed, dtype=np.uint8)
+    if packed.size < wr_packed_bytes(fmt, N, K):
+        raise WrError("wr_unpack_codes", 1)
+    out = np.empty((N, K), dtype=np.uint8)
+    _check("wr_unpack_codes", _lib.wr_unpack_codes(fmt, N, K, _ptr(packed), _ptr(out)))
+    return out
+
+
+def wr_quantize(bits: int, W: np.ndarray):
+    """fp32 [N, K] -> (codes uint8 [N, K], fp16 scale bits uint16 [N, K/256])."""
+    W = np.ascontiguousarray(W, dtype=np.float32)
+    N, K = W.shape
+    codes = np.empty((N, K), dtype=np.uint8)
+    scales = np.empty((N, max(K // 256, 1)), dtype=np.uint16)
+    _check("wr_quantize", _lib.wr_quantize(bits, N, K, _ptr(W), _ptr(codes), _ptr(scales)))
+    return codes, scales
+
+
+def wr_quantize_ternary(W: np.ndarray, sign_bits: np.ndarray):
+    """fp32 [N, K] and uint32 sign mask -> (codes uint8 [N, K], fp16 alpha bits uint16 [N])."""
+    W = np.ascontiguousarray(W, dtype=np.float32)
+    sign_bits = np.ascontiguousarray(sign_bits, dtype=np.uint32)
+    N, K = W.shape
+    codes = np.empty((N, K), dtype=np.uint8)
+    alpha = np.empty(N, dtype=np.uint16)
+    _check("wr_quantize_ternary",
+           _lib.wr_quantize_ternary(N, K, _ptr(W), _ptr(sign_bits), _ptr(codes), _ptr(alpha)))
+    return codes, alpha
+
+
+def wr_unpack_bf16(fmt: int, N: int, K: int, packed, scales, out, group: int = 256, stream=None) -> None:
+    _check("wr_unpack_bf16", _lib.wr_unpack_bf16(fmt, N, K, _ptr(packed), _ptr(scales), group,
+                                                 _ptr(out), _stream(stream)))
+
+
+def wr_gemv_workspace_bytes(M: int, N: int, K: int, bits: int) -> int:
+    return _lib.wr_gemv_workspace_bytes(M, N, K, bits)
+
+
+def wr_gemv(M: int, N: int, K: int, x, packed, scales, bits: int, y, workspace, workspace_bytes: int,
+            group: int = 256, stream=None) -> None:
+    _check("wr_gemv", _lib.wr_gemv(M, N, K, _ptr(x), _ptr(packed), _ptr(scales), bits, group, _ptr(y),
+                                   _ptr(workspace), workspace_bytes, _stream(stream)))
+
+
+def wr_gemm_workspace_bytes(M: int, N: int, K: int, bits: int) -> int:
+    return _lib.wr_gemm_workspace_bytes(M, N, K, bits)
+
+
+def wr_gemm(M: int, N: int, K: int, x, packed, scales, bits: int, y, workspace, workspace_bytes: int,
+            group: int = 256, stream=None) -> None:
+    _check("wr_gemm", _lib.wr_gemm(M, N, K, _ptr(x), _ptr(packed), _ptr(scales), bits, group, _ptr(y),
+                                   _ptr(workspace), workspace_bytes, _stream(stream)))
+
+
+def wr_gemm_ternary_workspace_bytes(M: int, N: int, K: int) -> int:
+    return _lib.wr_gemm_ternary_workspace_bytes(M, N, K)
+
+
+def wr_gemm_ternary(M: int, N: int, K: int, x, packed, alpha, sign_bits, y, workspace,
+                    workspace_bytes: int, stream=None) -> None:
+    _check("wr_gemm_ternary", _lib.wr_gemm_ternary(M, N, K, _ptr(x), _ptr(packed), _ptr(alpha),
+                                                   _ptr(sign_bits), _ptr(y), _ptr(workspace),
+                                                   workspace_bytes, _stream(stream)))
+
+
+def wr_get_device_error(stream=None) -> int:
+    return _lib.wr_get_device_error(_stream(stream))

@@ -1,0 +1,109 @@
+// Device helpers shared by the libwr kernels: loads, the legacy warp MMA used by the decode
+// GEMV, and the register decoders that turn packed codes into exact bf16 grid values.
+#pragma once
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <stdint.h>
+
+namespace wr {
+
+// ---------------------------------------------------------------- loads
+
+// Streaming 16-byte load: read once, do not keep in L1 (the weights are touched once).
+__device__ __forceinline__ uint4 ld_stream_v4(const void* p) {
+  uint4 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "l"(p));
+  return r;
+}
+
+// Read-only 16-byte load through L1 (activations: shared by every warp of an SM).
+__device__ __forceinline__ uint4 ld_ro_v4(const void* p) {
+  return __ldg(reinterpret_cast<const uint4*>(p));
+}
+
+// ---------------------------------------------------------------- warp MMA
+
+// D += A(16x16, row) * B(16x8, col) with bf16 inputs and fp32 accumulation.
+__device__ __forceinline__ void mma_bf16_16816(float d[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                               uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// ---------------------------------------------------------------- exact code decoders
+//
+// A pair register holds two bf16 weights (low half: even code, high half: odd code).
+// A code field c of width w placed at mantissa bits p..p+w-1 of bf16 1.0 (0x3F80) reads as
+// 1 + c*2^(p-7). One fused multiply-add with power-of-two scale 2^(7-p) and offset
+// -(2^(7-p) + o) yields c - o exactly (the result is a small multiple of 1/2 and the
+// offset has at most 8 significant bits). With o = L/2 the result is g/2 = c - L/2, the
+// grid level halved; with o = 1 (ternary) it is t = c - 1.
+
+constexpr uint32_t kOneBf16x2 = 0x3F803F80u;
+
+__device__ __forceinline__ uint32_t bf16x2_fma(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;
+  asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+
+// bf16x2 constants (both halves equal).
+constexpr uint32_t kB64 = 0x42804280u, kB16 = 0x41804180u, kB4 = 0x40804080u, kB8 = 0x41004100u;
+constexpr uint32_t kBm65_5 = 0xC283C283u, kBm17_5 = 0xC18CC18Cu, kBm5_5 = 0xC0B0C0B0u;  // Q2: o = 1.5
+constexpr uint32_t kBm67_5 = 0xC287C287u, kBm11_5 = 0xC138C138u;                      // Q3: o = 3.5
+constexpr uint32_t kBm65 = 0xC282C282u, kBm17 = 0xC188C188u, kBm5 = 0xC0A0C0A0u;      // ternary: o = 1
+
+// Q2 word -> 8 pair registers of g/2 values. Pair j = codes (2j, 2j+1) at bits 2j, 16+2j.
+__device__ __forceinline__ void decode_q2_word(uint32_t w, uint32_t p[8]) {
+  const uint32_t t0 = w << 1, t1 = w >> 5, t2 = w >> 11;
+  p[0] = bf16x2_fma((t0 & 0x00060006u) | kOneBf16x2, kB64, kBm65_5);
+  p[1] = bf16x2_fma((t0 & 0x00180018u) | kOneBf16x2, kB16, kBm17_5);
+  p[2] = bf16x2_fma((t0 & 0x00600060u) | kOneBf16x2, kB4, kBm5_5);
+  p[3] = bf16x2_fma((t1 & 0x00060006u) | kOneBf16x2, kB64, kBm65_5);
+  p[4] = bf16x2_fma((t1 & 0x00180018u) | kOneBf16x2, kB16, kBm17_5);
+  p[5] = bf16x2_fma((t1 & 0x00600060u) | kOneBf16x2, kB4, kBm5_5);
+  p[6] = bf16x2_fma((t2 & 0x00060006u) | kOneBf16x2, kB64, kBm65_5);
+  p[7] = bf16x2_fma((t2 & 0x00180018u) | kOneBf16x2, kB16, kBm17_5);
+}
+
+// Q3 group (3 words, 32 codes) -> 16 pair registers of g/2 values. Word u holds pairs
+// 5u..5u+4 as 3-bit fields at bits 3j (low half) and 16+3j (high half); pair 15 is spread
+// over bit 15 / bit 31 of the three words.
+__device__ __forceinline__ void decode_q3_group(const uint32_t w[3], uint32_t p[16]) {
+#pragma unroll
+  for (int u = 0; u < 3; ++u) {
+    const uint32_t t0 = w[u] << 1, t1 = w[u] >> 5, t2 = w[u] >> 11;
+    p[5 * u + 0] = bf16x2_fma((t0 & 0x000E000Eu) | kOneBf16x2, kB64, kBm67_5);
+    p[5 * u + 1] = bf16x2_fma((t0 & 0x00700070u) | kOneBf16x2, kB8, kBm11_5);
+    p[5 * u + 2] = bf16x2_fma((t1 & 0x000E000Eu) | kOneBf16x2, kB64, kBm67_5);
+    p[5 * u + 3] = bf16x2_fma((t1 & 0x00700070u) | kOneBf16x2, kB8, kBm11_5);
+    p[5 * u + 4] = bf16x2_fma((t2 & 0x000E000Eu) | kOneBf16x2, kB64, kBm67_5);
+  }
+  const uint32_t s = ((w[0] >> 14) & 0x00020002u) | ((w[1] >> 13) & 0x00040004u) |
+                     ((w[2] >> 12) & 0x00080008u) | kOneBf16x2;
+  p[15] = bf16x2_fma(s, kB64, kBm67_5);
+}
+
+// Ternary: a table entry holds the five trits of one byte as 2-bit codes at bits 1, 3, 5,
+// 9, 11 (entry for the low half) or those +16 (high half). OR-ing a low entry and a high
+// entry gives five pair registers' worth of fields: slots 1, 3, 5 directly, 9 and 11 after
+// a shift by 8.
+__device__ __forceinline__ void decode_trit_pairs(uint32_t e, uint32_t p[5]) {
+  const uint32_t t1 = e >> 8;
+  p[0] = bf16x2_fma((e & 0x00060006u) | kOneBf16x2, kB64, kBm65);
+  p[1] = bf16x2_fma((e & 0x00180018u) | kOneBf16x2, kB16, kBm17);
+  p[2] = bf16x2_fma((e & 0x00600060u) | kOneBf16x2, kB4, kBm5);
+  p[3] = bf16x2_fma((t1 & 0x00060006u) | kOneBf16x2, kB64, kBm65);
+  p[4] = bf16x2_fma((t1 & 0x00180018u) | kOneBf16x2, kB16, kBm17);
+}
+
+__device__ __forceinline__ float half_bits_to_float(uint16_t h) {
+  return __half2float(__ushort_as_half(h));
+}
+
+}  // namespace wr

@@ -1,0 +1,308 @@
+// Host side of libwr: packed-layout writer/reader and the synthetic quantizers.
+//
+// The byte layout is specified in include/wr.h. Here it is produced word by word: each
+// lane's 16-byte chunks are assembled from the code matrix and stored at
+// (32*chunk + lane)*16 inside their unit. The quantizers prepare inputs (codes and fp16
+// scales) from fp32 weights; they are not part of the device path.
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <vector>
+
+#include "wr.h"
+#include "wr_internal.h"
+
+namespace {
+
+constexpr int kTileRows = 16;
+
+inline bool fmt_ok(int fmt) { return fmt == WR_FMT_Q2 || fmt == WR_FMT_Q3 || fmt == WR_FMT_TERNARY; }
+
+struct Geometry {
+  int64_t unit_k;      // codes per unit along K
+  int64_t unit_bytes;  // bytes per unit
+  int64_t tiles;       // ceil(N/16)
+  int64_t units;       // units per tile row
+};
+
+bool geometry(int fmt, int64_t N, int64_t K, Geometry* g) {
+  if (!fmt_ok(fmt) || N <= 0 || K <= 0) return false;
+  if (fmt == WR_FMT_TERNARY) {
+    g->unit_k = 320;   // any K: the last unit is padded with trit 1 (t = 0)
+    g->unit_bytes = 1024;
+  } else {
+    if (K % 256 != 0) return false;
+    g->unit_k = 256;
+    g->unit_bytes = fmt == WR_FMT_Q2 ? 1024 : 1536;
+  }
+  g->tiles = (N + kTileRows - 1) / kTileRows;
+  g->units = (K + g->unit_k - 1) / g->unit_k;
+  return true;
+}
+
+// Byte offset inside a unit of lane-byte `lb` of lane `lane`.
+inline int64_t unit_offset(int lane, int lb) { return (int64_t)(32 * (lb / 16) + lane) * 16 + lb % 16; }
+
+inline void put_word(uint8_t* unit, int lane, int lb, uint32_t w) {
+  const int64_t off = unit_offset(lane, lb);   // lb is a multiple of 4: never crosses a chunk
+  unit[off + 0] = (uint8_t)(w);
+  unit[off + 1] = (uint8_t)(w >> 8);
+  unit[off + 2] = (uint8_t)(w >> 16);
+  unit[off + 3] = (uint8_t)(w >> 24);
+}
+
+inline uint32_t get_word(const uint8_t* unit, int lane, int lb) {
+  const int64_t off = unit_offset(lane, lb);
+  return (uint32_t)unit[off] | ((uint32_t)unit[off + 1] << 8) | ((uint32_t)unit[off + 2] << 16) |
+         ((uint32_t)unit[off + 3] << 24);
+}
+
+// Q2: one row quarter = 4 words of 16 codes; code e of a word at bits 16*(e&1) + 2*(e>>1).
+uint32_t q2_word(const uint8_t* c16) {
+  uint32_t w = 0;
+  for (int e = 0; e < 16; ++e) w |= (uint32_t)(c16[e] & 3u) << (16 * (e & 1) + 2 * (e >> 1));
+  return w;
+}
+void q2_unword(uint32_t w, uint8_t* c16) {
+  for (int e = 0; e < 16; ++e) c16[e] = (uint8_t)((w >> (16 * (e & 1) + 2 * (e >> 1))) & 3u);
+}
+
+// Q3: one 12-byte group = 3 words holding 32 codes. Codes 10u + 2j + h (j = 0..4) of word u
+// at bits 16h + 3j; code 30 + h spread over bit 16h + 15 of words 0, 1, 2.
+void q3_group(const uint8_t* c32, uint32_t w[3]) {
+  for (int u = 0; u < 3; ++u) {
+    uint32_t v = 0;
+    for (int f = 0; f < 10; ++f) v |= (uint32_t)(c32[10 * u + f] & 7u) << (16 * (f & 1) + 3 * (f >> 1));
+    for (int h = 0; h < 2; ++h) v |= (uint32_t)((c32[30 + h] >> u) & 1u) << (16 * h + 15);
+    w[u] = v;
+  }
+}
+void q3_ungroup(const uint32_t w[3], uint8_t* c32) {
+  for (int u = 0; u < 3; ++u)
+    for (int f = 0; f < 10; ++f) c32[10 * u + f] = (uint8_t)((w[u] >> (16 * (f & 1) + 3 * (f >> 1))) & 7u);
+  for (int h = 0; h < 2; ++h) {
+    uint8_t c = 0;
+    for (int u = 0; u < 3; ++u) c |= (uint8_t)(((w[u] >> (16 * h + 15)) & 1u) << u);
+    c32[30 + h] = c;
+  }
+}
+
+// fp16 helpers (host): decode bits exactly; encode a double with one RNE rounding.
+double half_to_double(uint16_t h) {
+  const int e = (h >> 10) & 31, m = h & 1023;
+  double v;
+  if (e == 0) v = std::ldexp((double)m, -24);
+  else if (e == 31) v = m ? NAN : INFINITY;
+  else v = std::ldexp((double)(m + 1024), e - 25);
+  return (h & 0x8000) ? -v : v;
+}
+
+uint16_t double_to_half(double v) {
+  const uint16_t sign = std::signbit(v) ? 0x8000 : 0;
+  const double a = std::fabs(v);
+  if (std::isnan(v)) return 0x7E00;
+  if (a == 0.0) return sign;
+  int ex;
+  std::frexp(a, &ex);          // a = f * 2^ex, f in [0.5, 1)
+  int E = ex - 1;              // a in [2^E, 2^(E+1))
+  if (E < -14) E = -14;        // subnormal range shares the 2^-24 step
+  const double q = std::ldexp(a, 10 - E);   // a / ulp, exact
+  double fl = std::floor(q);
+  const double rem = q - fl;
+  if (rem > 0.5 || (rem == 0.5 && std::fmod(fl, 2.0) == 1.0)) fl += 1.0;
+  int64_t mant = (int64_t)fl;
+  if (mant == 2048) { mant = 1024; E += 1; }
+  if (mant < 1024) return (uint16_t)(sign | mant);            // subnormal (E == -14)
+  if (E + 15 >= 31) return (uint16_t)(sign | 0x7C00);        // overflow to infinity
+  return (uint16_t)(sign | ((E + 15) << 10) | (mant - 1024));
+}
+
+}  // namespace
+
+namespace wr {
+bool packed_geometry(int fmt, int64_t N, int64_t K, int64_t* unit_bytes, int64_t* units, int64_t* tiles) {
+  Geometry g;
+  if (!geometry(fmt, N, K, &g)) return false;
+  if (unit_bytes) *unit_bytes = g.unit_bytes;
+  if (units) *units = g.units;
+  if (tiles) *tiles = g.tiles;
+  return true;
+}
+uint16_t host_double_to_half(double v) { return double_to_half(v); }
+double host_half_to_double(uint16_t h) { return half_to_double(h); }
+}  // namespace wr
+
+extern "C" {
+
+size_t wr_packed_bytes(int fmt, int64_t N, int64_t K) {
+  Geometry g;
+  if (!geometry(fmt, N, K, &g)) return 0;
+  return (size_t)(g.tiles * g.units * g.unit_bytes);
+}
+
+wr_status wr_pack(int fmt, int64_t N, int64_t K, const uint8_t* codes, uint8_t* packed) {
+  Geometry g;
+  if (!geometry(fmt, N, K, &g) || !codes || !packed) return WR_ERR_INVALID_ARG;
+  const uint8_t cmax = fmt == WR_FMT_Q2 ? 3 : fmt == WR_FMT_Q3 ? 7 : 2;
+  bool bad = false;
+#pragma omp parallel for reduction(|| : bad)
+  for (int64_t i = 0; i < N * K; ++i) bad = bad || codes[i] > cmax;
+  if (bad) return WR_ERR_INVALID_ARG;
+
+#pragma omp parallel for collapse(2) schedule(static)
+  for (int64_t tn = 0; tn < g.tiles; ++tn) {
+    for (int64_t u = 0; u < g.units; ++u) {
+      uint8_t* unit = packed + (tn * g.units + u) * g.unit_bytes;
+      for (int lane = 0; lane < 32; ++lane) {
+        const int r0 = lane / 4, q = lane % 4;
+        for (int half = 0; half < 2; ++half) {
+          const int64_t n = tn * kTileRows + r0 + 8 * half;
+          if (fmt == WR_FMT_TERNARY) {
+            for (int beta = 0; beta < 16; ++beta) {
+              int v = 0, p3 = 1;
+              for (int d = 0; d < 5; ++d) {
+                const int64_t k = u * 320 + 80 * q + 5 * beta + d;
+                const int c = (n < N && k < K) ? codes[n * K + k] : 1;
+                v += c * p3;
+                p3 *= 3;
+              }
+              unit[unit_offset(lane, 16 * half + beta)] = (uint8_t)v;
+            }
+          } else {
+            uint8_t c64[64];
+            for (int i = 0; i < 64; ++i) c64[i] = n < N ? codes[n * K + u * 256 + 64 * q + i] : 0;
+            if (fmt == WR_FMT_Q2) {
+              for (int w = 0; w < 4; ++w) put_word(unit, lane, 16 * half + 4 * w, q2_word(c64 + 16 * w));
+            } else {
+              for (int grp = 0; grp < 2; ++grp) {
+                uint32_t w3[3];
+                q3_group(c64 + 32 * grp, w3);
+                for (int uu = 0; uu < 3; ++uu) put_word(unit, lane, 24 * half + 12 * grp + 4 * uu, w3[uu]);
+              }
+            }
+          }
+        }
+      }
+    }
+  }
+  return WR_OK;
+}
+
+wr_status wr_unpack_codes(int fmt, int64_t N, int64_t K, const uint8_t* packed, uint8_t* codes) {
+  Geometry g;
+  if (!geometry(fmt, N, K, &g) || !codes || !packed) return WR_ERR_INVALID_ARG;
+#pragma omp parallel for collapse(2) schedule(static)
+  for (int64_t tn = 0; tn < g.tiles; ++tn) {
+    for (int64_t u = 0; u < g.units; ++u) {
+      const uint8_t* unit = packed + (tn * g.units + u) * g.unit_bytes;
+      for (int lane = 0; lane < 32; ++lane) {
+        const int r0 = lane / 4, q = lane % 4;
+        for (int half = 0; half < 2; ++half) {
+          const int64_t n = tn * kTileRows + r0 + 8 * half;
+          if (n >= N) continue;
+          if (fmt == WR_FMT_TERNARY) {
+            for (int beta = 0; beta < 16; ++beta) {
+              int v = unit[unit_offset(lane, 16 * half + beta)];
+              for (int d = 0; d < 5; ++d) {
+                const int64_t k = u * 320 + 80 * q + 5 * beta + d;
+                if (k < K) codes[n * K + k] = (uint8_t)(v % 3);
+                v /= 3;
+              }
+            }
+          } else {
+            uint8_t c64[64];
+            if (fmt == WR_FMT_Q2) {
+              for (int w = 0; w < 4; ++w) q2_unword(get_word(unit, lane, 16 * half + 4 * w), c64 + 16 * w);
+            } else {
+              for (int grp = 0; grp < 2; ++grp) {
+                uint32_t w3[3];
+                for (int uu = 0; uu < 3; ++uu) w3[uu] = get_word(unit, lane, 24 * half + 12 * grp + 4 * uu);
+                q3_ungroup(w3, c64 + 32 * grp);
+              }
+            }
+            std::memcpy(codes + n * K + u * 256 + 64 * q, c64, 64);
+          }
+        }
+      }
+    }
+  }
+  return WR_OK;
+}
+
+wr_status wr_quantize(int bits, int64_t N, int64_t K, const float* w, uint8_t* codes, uint16_t* scales) {
+  if (bits != 2 && bits != 3) return WR_ERR_UNSUPPORTED;
+  if (N <= 0 || K <= 0 || K % 256 != 0 || !w || !codes || !scales) return WR_ERR_INVALID_ARG;
+  const int L = (1 << bits) - 1;
+  const int64_t nb = K / 256;
+#pragma omp parallel for schedule(static)
+  for (int64_t n = 0; n < N; ++n) {
+    for (int64_t b = 0; b < nb; ++b) {
+      const float* wb = w + n * K + b * 256;
+      double amax = 0.0;
+      for (int i = 0; i < 256; ++i) amax = std::fmax(amax, std::fabs((double)wb[i]));
+      const uint16_t sh = double_to_half(amax / (double)L);
+      scales[n * nb + b] = sh;
+      const double s = half_to_double(sh);
+      for (int i = 0; i < 256; ++i) {
+        int g = 1;
+        if (s > 0.0) {
+          const double qv = (double)wb[i] / s;
+          double gd = 2.0 * std::floor(qv * 0.5) + 1.0;
+          if (gd > L) gd = L;
+          if (gd < -L) gd = -L;
+          g = (int)gd;
+        }
+        codes[n * K + b * 256 + i] = (uint8_t)((g + L) / 2);
+      }
+    }
+  }
+  return WR_OK;
+}
+
+wr_status wr_quantize_ternary(int64_t N, int64_t K, const float* w, const uint32_t* sign_bits,
+                              uint8_t* codes, uint16_t* alpha) {
+  if (N <= 0 || K <= 0 || K % 128 != 0 || !w || !sign_bits || !codes || !alpha) return WR_ERR_INVALID_ARG;
+  const double inv = 1.0 / std::sqrt(128.0);
+#pragma omp parallel
+  {
+    std::vector<double> row((size_t)K);
+#pragma omp for schedule(static)
+    for (int64_t n = 0; n < N; ++n) {
+      // row n of W R^T is R applied to row n of W: signs, then the butterfly, then 1/sqrt(128)
+      for (int64_t k = 0; k < K; ++k) {
+        const bool neg = (sign_bits[k >> 5] >> (k & 31)) & 1u;
+        row[k] = neg ? -(double)w[n * K + k] : (double)w[n * K + k];
+      }
+      for (int64_t b0 = 0; b0 < K; b0 += 128) {
+        double* v = row.data() + b0;
+        for (int h = 1; h < 128; h *= 2)
+          for (int i = 0; i < 128; i += 2 * h)
+            for (int j = i; j < i + h; ++j) {
+              const double a = v[j], c = v[j + h];
+              v[j] = a + c;
+              v[j + h] = a - c;
+            }
+        for (int i = 0; i < 128; ++i) v[i] *= inv;
+      }
+      double sum = 0.0;
+      for (int64_t k = 0; k < K; ++k) sum += std::fabs(row[k]);
+      const double delta = 0.7 * (sum / (double)K);
+      double kept = 0.0;
+      int64_t cnt = 0;
+      for (int64_t k = 0; k < K; ++k) {
+        const double a = std::fabs(row[k]);
+        int t = 0;
+        if (a > delta) {
+          t = row[k] > 0 ? 1 : -1;
+          kept += a;
+          ++cnt;
+        }
+        codes[n * K + k] = (uint8_t)(t + 1);
+      }
+      alpha[n] = double_to_half(cnt > 0 ? kept / (double)cnt : 0.0);
+    }
+  }
+  return WR_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,132 @@
+// Materializer: packed codes + scales -> bf16 weights, bit-exact.
+//
+// The "Qwen3-4B-Wringer-Q2.6" card ("What is in this repo") describes a materializer that
+// expands the container into a bf16 checkpoint, bit-identical across independent re-runs.
+// Here W[n,k] = bf16_RNE(s * g): the fp32 product of an fp16 scale (11 significant bits)
+// and a grid integer (at most 3 bits) is exact, so the one rounding to bf16 is the only one.
+// One warp per packed unit; each lane expands its 64 codes (80 trits) of two rows and
+// writes them as 16-byte stores. The kernel is bound by the 2 bytes/weight it writes.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+#include "gemv.cuh"
+#include "wr.h"
+
+namespace wr {
+namespace {
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  const uint32_t a = __bfloat16_as_ushort(__float2bfloat16_rn(lo));
+  const uint32_t b = __bfloat16_as_ushort(__float2bfloat16_rn(hi));
+  return a | (b << 16);
+}
+
+template <int FMT>
+__global__ void __launch_bounds__(256) unpack_kernel(const uint8_t* __restrict__ packed,
+                                                     const uint16_t* __restrict__ scales, int N,
+                                                     int K, int B, int64_t U,
+                                                     uint16_t* __restrict__ out) {
+  const int lane = threadIdx.x & 31;
+  const int64_t u = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (u >= U) return;
+  constexpr int UB = FMT == WR_FMT_Q3 ? 1536 : 1024;
+  constexpr int kChunks = FMT == WR_FMT_Q3 ? 3 : 2;
+  const uint8_t* base = packed + u * UB;
+  uint32_t wd[4 * kChunks];
+#pragma unroll
+  for (int c = 0; c < kChunks; ++c) {
+    const uint4 v = ld_stream_v4(base + (32 * c + lane) * 16);
+    wd[4 * c + 0] = v.x;
+    wd[4 * c + 1] = v.y;
+    wd[4 * c + 2] = v.z;
+    wd[4 * c + 3] = v.w;
+  }
+  const int64_t tn = u / B, ub = u % B;
+  const int r0 = lane >> 2, q = lane & 3;
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int64_t n = tn * 16 + r0 + 8 * h;
+    if (n >= N) continue;
+    if (FMT == WR_FMT_TERNARY) {
+      const float al = half_bits_to_float(scales[n]);
+      float v[80];
+#pragma unroll
+      for (int beta = 0; beta < 16; ++beta) {
+        uint32_t byte = (wd[4 * h + beta / 4] >> (8 * (beta % 4))) & 0xFFu;
+#pragma unroll
+        for (int d = 0; d < 5; ++d) {
+          v[5 * beta + d] = al * (float)((int)(byte % 3u) - 1);
+          byte /= 3u;
+        }
+      }
+      const int64_t k0 = ub * 320 + 80 * q;
+      uint16_t* dst = out + n * (int64_t)K + k0;
+      if (k0 + 80 <= K) {
+#pragma unroll
+        for (int i = 0; i < 10; ++i) {
+          uint4 st;
+          st.x = pack_bf16x2(v[8 * i + 0], v[8 * i + 1]);
+          st.y = pack_bf16x2(v[8 * i + 2], v[8 * i + 3]);
+          st.z = pack_bf16x2(v[8 * i + 4], v[8 * i + 5]);
+          st.w = pack_bf16x2(v[8 * i + 6], v[8 * i + 7]);
+          *reinterpret_cast<uint4*>(dst + 8 * i) = st;
+        }
+      } else {
+        for (int i = 0; i < 80 && k0 + i < K; ++i) dst[i] = __bfloat16_as_ushort(__float2bfloat16_rn(v[i]));
+      }
+    } else {
+      const float s = half_bits_to_float(scales[n * B + ub]);
+      const int L = FMT == WR_FMT_Q2 ? 3 : 7;
+      int c[64];
+      if (FMT == WR_FMT_Q2) {
+#pragma unroll
+        for (int w = 0; w < 4; ++w)
+#pragma unroll
+          for (int e = 0; e < 16; ++e) c[16 * w + e] = (wd[4 * h + w] >> (16 * (e & 1) + 2 * (e >> 1))) & 3;
+      } else {
+        const uint32_t* rw = wd + 6 * h;
+#pragma unroll
+        for (int g = 0; g < 2; ++g) {
+#pragma unroll
+          for (int uu = 0; uu < 3; ++uu)
+#pragma unroll
+            for (int f = 0; f < 10; ++f)
+              c[32 * g + 10 * uu + f] = (rw[3 * g + uu] >> (16 * (f & 1) + 3 * (f >> 1))) & 7;
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+            int cc = 0;
+#pragma unroll
+            for (int uu = 0; uu < 3; ++uu) cc |= ((rw[3 * g + uu] >> (16 * hh + 15)) & 1) << uu;
+            c[32 * g + 30 + hh] = cc;
+          }
+        }
+      }
+      uint16_t* dst = out + n * (int64_t)K + ub * 256 + 64 * q;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        uint4 st;
+        st.x = pack_bf16x2(s * (float)(2 * c[8 * i + 0] - L), s * (float)(2 * c[8 * i + 1] - L));
+        st.y = pack_bf16x2(s * (float)(2 * c[8 * i + 2] - L), s * (float)(2 * c[8 * i + 3] - L));
+        st.z = pack_bf16x2(s * (float)(2 * c[8 * i + 4] - L), s * (float)(2 * c[8 * i + 5] - L));
+        st.w = pack_bf16x2(s * (float)(2 * c[8 * i + 6] - L), s * (float)(2 * c[8 * i + 7] - L));
+        *reinterpret_cast<uint4*>(dst + 8 * i) = st;
+      }
+    }
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_unpack_bf16(int fmt, const uint8_t* packed, const uint16_t* scales, int N, int K,
+                               int units, uint16_t* w, cudaStream_t stream) {
+  const int64_t tiles = (N + 15) / 16;
+  const int64_t U = tiles * units;
+  const unsigned ctas = (unsigned)((U + 7) / 8);
+  if (fmt == WR_FMT_Q2) unpack_kernel<WR_FMT_Q2><<<ctas, 256, 0, stream>>>(packed, scales, N, K, units, U, w);
+  else if (fmt == WR_FMT_Q3) unpack_kernel<WR_FMT_Q3><<<ctas, 256, 0, stream>>>(packed, scales, N, K, units, U, w);
+  else unpack_kernel<WR_FMT_TERNARY><<<ctas, 256, 0, stream>>>(packed, scales, N, K, units, U, w);
+  return cudaGetLastError();
+}
+
+}  // namespace wr

@@ -1,0 +1,158 @@
+/*
+ * wr.h -- C ABI of libwr: packed low-bit weight-only GEMV/GEMM for B200 (sm_100a).
+ *
+ * What is computed
+ * ----------------
+ * Weights are stored as integer codes on a signed odd grid with one fp16 scale per
+ * 256 weights along K:  W[n,k] = s[n, k/256] * g(c[n,k]),  g(c) = 2c - (2^b - 1),
+ * i.e. {-3,-1,1,3} at b = 2 and {-7,-5,...,5,7} at b = 3.  The 2-bit grid and the
+ * reason it has no zero level are the worked example in "How We Shrank an AI Model by
+ * 85% and Kept 90% of Its Smarts" (section "Why 2 bits is hard"); the container of
+ * "packed codes + fp16 block scales" is described on the "Qwen3-4B-Wringer-Q2.6" model
+ * card ("What is in this repo"), which also states that no kernel consumes it.
+ *
+ * The ternary format (W1.58A16, the Qwen3-4B post-training ternarization article) stores
+ * t in {-1,0,+1} as c = t + 1, five trits per byte, with one fp16 scale alpha per row, in
+ * a basis rotated along K by R = blockdiag((1/sqrt(128)) H_128 D): W x = (W R^T)(R x)
+ * ("How We Shrank...", "Trick 1: rotate the weights first"). H_128 is the Sylvester
+ * Hadamard matrix in natural order, D = diag(d), d_k = -1 where bit k%32 of word k/32 of
+ * the sign mask is set. The library applies R to x inside the call.
+ *
+ * Every GEMV/GEMM computes, for m < M and n < N,
+ *     y[m,n] = sum_b s[n,b] * sum_{k in block b} g[n,k] * x[m,k]          (Q2, Q3)
+ *     y[m,n] = alpha[n] * sum_k t[n,k] * (R x[m,:])[k]                      (ternary)
+ * with x bf16 [M,K] row-major and y fp32 [M,N] row-major (overwritten). Products of the
+ * exact grid integers and x are formed exactly and accumulated in fp32; each 256-block
+ * partial is multiplied by its scale in fp32. R x is kept in fp32 (split into two bf16
+ * terms where tensor cores consume it).
+ *
+ * Packed layout (shared by every kernel; the bytes are what wr_pack writes)
+ * -------------------------------------------------------------------------
+ * Rows are grouped in tiles of 16 (the last tile padded). K is cut in units: 256 codes
+ * for Q2/Q3 (K must be a multiple of 256), 320 trits for ternary (any K, the last unit
+ * padded; the ternary GEMM needs K to be a multiple of 128 for the rotation). The buffer is the sequence of units of tile 0, then of
+ * tile 1, ... ; a unit is UB contiguous bytes: UB = 1024 (Q2), 1536 (Q3), 1024 (ternary).
+ * Inside a unit, lane l = 4*r0 + q (r0 = 0..7, q = 0..3) owns rows r0 and r0+8 of the
+ * tile and the q-th quarter (64 codes, or 80 trits) of the unit's K range. A lane's bytes
+ * are its row-r0 bytes followed by its row-(r0+8) bytes (16 + 16 for Q2, 24 + 24 for Q3,
+ * 16 + 16 for ternary), cut in 16-byte chunks; chunk c of lane l is stored at unit byte
+ * (32*c + l)*16. Multi-byte words below are little-endian uint32.
+ *   Q2: a row quarter is 4 words; code i (0..63) is in word i/16; with e = i%16 it sits
+ *       at bits 16*(e%2) + 2*(e/2) .. +1 (even codes in the low 16 bits, odd in the high).
+ *   Q3: a row quarter is two 12-byte groups (codes 0..31, 32..63), 3 words each. With
+ *       e = i%32: for e < 30, word e/10, f = e%10, bits 16*(f%2) + 3*(f/2) .. +2; code
+ *       30+h (h = 0,1) has its bit j in bit 16*h + 15 of word j.
+ *   Ternary: a row quarter is 16 bytes; trit i is digit i%5 of byte i/5, whose value is
+ *       sum_d c_d * 3^d. Pad trits are c = 1 (t = 0).
+ * Pad rows of Q2/Q3 hold code 0. packed bytes = ceil(N/16) * ceil(K/unit) * UB.
+ *
+ * Conventions
+ * -----------
+ * - Pointers: device pointers unless the name ends in _host. The caller owns every
+ *   buffer; the library allocates nothing and keeps no per-call state.
+ * - Alignment: every pointer must be 16-byte aligned (WR_ERR_INVALID_ARG otherwise).
+ * - stream: a cudaStream_t passed as void* (NULL = legacy default stream). Device calls
+ *   are asynchronous on that stream and never synchronize.
+ * - Errors: arguments are checked synchronously and the call returns before any launch;
+ *   launch failures return WR_ERR_CUDA. Nothing aborts and no exception crosses the ABI.
+ * - Workspace: where a call takes one, it must be at least *_workspace_bytes(...) bytes
+ *   and zero-filled before its first use. Each successful call leaves the parts that must
+ *   start at zero (arrival counters) zero again, so one zeroed buffer serves any number of
+ *   calls issued in stream order. Calls that may run concurrently (different streams) need
+ *   different workspaces.
+ */
+#ifndef WR_H
+#define WR_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  WR_OK = 0,
+  WR_ERR_INVALID_ARG = 1,   /* null/misaligned pointer, bad size or code value */
+  WR_ERR_UNSUPPORTED = 2,   /* valid but unsupported: group != 256, bits not 2/3, ... */
+  WR_ERR_CUDA = 3,          /* a CUDA launch or runtime call failed */
+  WR_ERR_TIMEOUT = 4        /* a bounded device-side wait gave up (see wr_get_device_error) */
+} wr_status;
+
+enum { WR_FMT_TERNARY = 1, WR_FMT_Q2 = 2, WR_FMT_Q3 = 3 };
+
+/* Version of this ABI (incremented on any incompatible change). */
+int wr_abi_version(void);
+
+/* Static description of a status code. */
+const char* wr_status_string(wr_status st);
+
+/* Bytes of the packed buffer for an N x K code matrix in format fmt; 0 on bad arguments. */
+size_t wr_packed_bytes(int fmt, int64_t N, int64_t K);
+
+/* Host packer: codes_host [N,K] uint8 (Q2: 0..3, Q3: 0..7, ternary: 0..2) ->
+ * packed_host (wr_packed_bytes bytes, caller-allocated). Pad bytes are written too.
+ * WR_ERR_INVALID_ARG on a code out of range (nothing is guaranteed about packed_host). */
+wr_status wr_pack(int fmt, int64_t N, int64_t K, const uint8_t* codes_host, uint8_t* packed_host);
+
+/* Host inverse of wr_pack on the real rows and columns: packed_host -> codes_host [N,K]. */
+wr_status wr_unpack_codes(int fmt, int64_t N, int64_t K, const uint8_t* packed_host,
+                          uint8_t* codes_host);
+
+/* Host synthetic quantizer for the odd grid (data preparation, not on the device path).
+ * Per 256-block along K: s = fp16(absmax / L) (L = 2^bits - 1; the division in fp64 and
+ * one rounding to fp16, so the scale is fixed before the codes are chosen, as on the
+ * "Agents-A1-4B-Wringer-Q2.6" card, "Honest caveats"), then the nearest odd level of
+ * w/s (fp64), clamped to [-L, L]; an exact even quotient goes up; s = 0 gives level +1
+ * (nearest-point codes: "Qwen3-4B-Wringer-Q2.6", "Recipe").
+ * w_host fp32 [N,K]; codes_host uint8 [N,K]; scales_host fp16 bits [N, K/256]. */
+wr_status wr_quantize(int bits, int64_t N, int64_t K, const float* w_host, uint8_t* codes_host,
+                      uint16_t* scales_host);
+
+/* Host synthetic ternary quantizer: W' = W R^T (fp64, per 128-block fast Walsh-Hadamard
+ * transform with the sign mask), Delta_n = 0.7 * mean_k |W'[n,k]|, t = sign(W') where
+ * |W'| > Delta_n else 0, alpha_n = fp16(mean |W'| over t != 0) (0 if none); codes c = t+1.
+ * K % 128 == 0. sign_bits_host uint32 [ceil(K/32)]; alpha_host fp16 bits [N]. */
+wr_status wr_quantize_ternary(int64_t N, int64_t K, const float* w_host,
+                              const uint32_t* sign_bits_host, uint8_t* codes_host,
+                              uint16_t* alpha_host);
+
+/* Device materializer: w_bf16 [N,K] = bf16_RNE(s * g) for Q2/Q3 (group must be 256), or
+ * bf16_RNE(alpha_n * t) for ternary (scales = alpha [N], group ignored; the result is in
+ * the rotated basis). Bit-exact; the bf16 checkpoint the "Qwen3-4B-Wringer-Q2.6" card's
+ * materializer produces from the container. */
+wr_status wr_unpack_bf16(int fmt, int64_t N, int64_t K, const void* packed, const uint16_t* scales,
+                         int group, uint16_t* w_bf16, void* stream);
+
+/* Decode GEMV for 1 <= M <= 8 (Q2/Q3, group 256): streams the packed codes once, decodes
+ * them in registers and contracts them on tensor cores. Splits K across warps and combines
+ * the pieces through the workspace (deterministic summation order). */
+size_t wr_gemv_workspace_bytes(int64_t M, int64_t N, int64_t K, int bits);
+wr_status wr_gemv(int64_t M, int64_t N, int64_t K, const uint16_t* x, const void* packed,
+                  const uint16_t* scales, int bits, int group, float* y, void* workspace,
+                  size_t workspace_bytes, void* stream);
+
+/* Prefill GEMM, any M >= 1 (Q2/Q3, group 256): packed tiles are staged in shared memory,
+ * decoded to exact bf16 grid integers and contracted by tcgen05 MMAs into TMEM, one fp32
+ * partial per 256-block, scaled in fp32 by the epilogue. */
+size_t wr_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int bits);
+wr_status wr_gemm(int64_t M, int64_t N, int64_t K, const uint16_t* x, const void* packed,
+                  const uint16_t* scales, int bits, int group, float* y, void* workspace,
+                  size_t workspace_bytes, void* stream);
+
+/* Ternary GEMV/GEMM, any M >= 1: applies the block-128 random-sign Hadamard to x and
+ * contracts with the packed trits; alpha fp16 [N]; sign_bits uint32 [ceil(K/32)]. */
+size_t wr_gemm_ternary_workspace_bytes(int64_t M, int64_t N, int64_t K);
+wr_status wr_gemm_ternary(int64_t M, int64_t N, int64_t K, const uint16_t* x, const void* packed,
+                          const uint16_t* alpha, const uint32_t* sign_bits, float* y,
+                          void* workspace, size_t workspace_bytes, void* stream);
+
+/* Reads and clears the device error word that bounded waits set when they give up
+ * (synchronizes the stream). WR_OK when no wait timed out since the last call. */
+wr_status wr_get_device_error(void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* WR_H */

@@ -1,0 +1,50 @@
+"""Shared set-up of the GPU parity tests: both sides start from the same seeded fp32
+weights and bf16 activations (wr_synth); the library quantizes and packs for the CUDA
+path, the oracle quantizes for itself, and the two code sets are checked to agree."""
+import numpy as np
+
+import wr_synth
+from oracle import wr_oracle as o
+
+
+def torch_mod():
+    import torch
+    return torch
+
+
+def dev(a: np.ndarray):
+    """numpy array -> CUDA tensor with the same bytes (uint16 bit patterns travel as int16)."""
+    torch = torch_mod()
+    if a.dtype == np.uint16:
+        a = a.view(np.int16)
+    elif a.dtype == np.uint32:
+        a = a.view(np.int32)
+    return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+
+def q_case(wr, bits, N, K, seed):
+    W = wr_synth.weights_fp32(seed, N, K)
+    codes, scales = wr.wr_quantize(bits, W)
+    codes_o, scales_o = o.quantize_odd_grid(W, bits)
+    assert np.array_equal(codes, codes_o) and np.array_equal(scales, scales_o.view(np.uint16))
+    packed = wr.wr_pack(bits, codes)
+    return codes_o, scales_o, dev(packed), dev(scales)
+
+
+def t_case(wr, N, K, seed):
+    signs = wr_synth.sign_bits(seed + 1, K)
+    W = wr_synth.weights_fp32(seed, N, K)
+    codes, alpha = wr.wr_quantize_ternary(W, signs)
+    codes_o, alpha_o, _ = o.quantize_ternary(W, signs)
+    assert np.array_equal(codes, codes_o) and np.array_equal(alpha, alpha_o.view(np.uint16))
+    packed = wr.wr_pack(1, codes)
+    return codes_o, alpha_o, signs, dev(packed), dev(alpha), dev(signs)
+
+
+def check_close(y_gpu: np.ndarray, y_ref: np.ndarray, bound: np.ndarray, rel: float = 1e-4):
+    """Per element |y_gpu - y_ref| <= rel * sum_k |w x|; exact zero where the bound is zero."""
+    err = np.abs(y_gpu.astype(np.float64) - y_ref)
+    bad = err > rel * bound
+    assert not bad.any(), (f"{bad.sum()} of {bad.size} elements out of tolerance; "
+                           f"worst err/bound {np.max(err / np.maximum(bound, 1e-300)):.3e}")
+    assert np.all(y_gpu[bound == 0] == 0)

@@ -1,0 +1,120 @@
+"""Host-side checks of libwr (no GPU): exported symbols, the packer against the oracle's
+independent implementation of the layout, the synthetic quantizers against the oracle's,
+and argument validation that must return before any device work."""
+import json
+import os
+import re
+
+import numpy as np
+import pytest
+
+import bit_weight_only_wr_b200 as wr
+import wr_synth
+from oracle import wr_oracle as o
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _header_functions():
+    text = open(os.path.join(ROOT, "include", "wr.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(wr_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_symbol():
+    declared = _header_functions()
+    assert declared == wr.exported_symbols()
+    out = os.popen(f"nm -D --defined-only {wr.LIB_PATH}").read()
+    exported = set(re.findall(r" T (wr_[a-z0-9_]+)", out))
+    missing = [f for f in declared if f not in exported]
+    assert not missing, missing
+    assert wr.wr_abi_version() == 1
+    assert wr.wr_status_string(0) == "ok"
+
+
+@pytest.mark.parametrize("fmt", [2, 3, 1])
+@pytest.mark.parametrize("N,K", [(16, 256), (40, 512), (1, 768), (33, 2560)])
+def test_pack_matches_oracle(fmt, N, K):
+    if fmt == 1 and K % 128:
+        pytest.skip()
+    levels = {1: 3, 2: 4, 3: 8}[fmt]
+    rng = np.random.default_rng(N * 7 + K + fmt)
+    codes = rng.integers(0, levels, (N, K)).astype(np.uint8)
+    assert wr.wr_packed_bytes(fmt, N, K) == o.packed_bytes(fmt, N, K)
+    mine = wr.wr_pack(fmt, codes)
+    ref = o.pack(fmt, codes)
+    assert np.array_equal(mine, ref)
+    assert np.array_equal(wr.wr_unpack_codes(fmt, mine, N, K), codes)
+
+
+def test_pack_golden_vectors_through_library(golden_dir):
+    g = json.load(open(os.path.join(golden_dir, "pack_vectors.json")))
+    for case in g["cases"]:
+        codes = np.full((case["N"], case["K"]), case["fill"], dtype=np.uint8)
+        for n, k, c in case["set"]:
+            codes[n, k] = c
+        p = wr.wr_pack(case["fmt"], codes)
+        for idx, val in case["expect"].items():
+            assert int(p[int(idx)]) == val
+
+
+def test_pack_rejects_bad_codes_and_shapes():
+    with pytest.raises(wr.WrError):
+        wr.wr_pack(2, np.full((16, 256), 4, dtype=np.uint8))
+    with pytest.raises(wr.WrError):
+        wr.wr_pack(1, np.full((16, 256), 3, dtype=np.uint8))
+    assert wr.wr_packed_bytes(2, 16, 100) == 0           # K not a multiple of 256
+    assert wr.wr_packed_bytes(1, 16, 100) == 1024        # ternary: any K, padded to 320 trits
+    assert wr.wr_packed_bytes(7, 16, 256) == 0
+
+
+@pytest.mark.parametrize("bits", [2, 3])
+def test_quantizer_matches_oracle(bits):
+    W = wr_synth.weights_fp32(100 + bits, 64, 1024)
+    W[3, :256] = 0.0                                      # an all-zero block (s = 0)
+    W[5, 300] = 1e-9                                      # tiny values, tiny scale
+    c1, s1 = wr.wr_quantize(bits, W)
+    c2, s2 = o.quantize_odd_grid(W, bits)
+    assert np.array_equal(s1, s2.view(np.uint16))
+    assert np.array_equal(c1, c2)
+
+
+def test_ternary_quantizer_matches_oracle():
+    K = 1280
+    signs = wr_synth.sign_bits(5, K)
+    W = wr_synth.weights_fp32(6, 48, K)
+    c1, a1 = wr.wr_quantize_ternary(W, signs)
+    c2, a2, Wr = o.quantize_ternary(W, signs)
+    assert np.array_equal(a1, a2.view(np.uint16))
+    diff = c1 != c2
+    # the two sides rotate with different summation orders; a code may differ only where
+    # |W'| sits on the threshold to within rounding
+    if diff.any():
+        a = np.abs(Wr)
+        delta = 0.7 * a.mean(axis=1, keepdims=True)
+        assert np.all(np.abs(a - delta)[diff] < 1e-12 * delta.repeat(K, 1)[diff])
+    assert diff.sum() == 0
+
+
+def test_device_calls_reject_bad_arguments_before_launch():
+    # misaligned / null pointers and unsupported configurations return before any CUDA call
+    st = wr._lib.wr_gemv(1, 16, 256, 8, 16, 16, 2, 256, 16, 16, 1 << 20, None)
+    assert st == 1
+    st = wr._lib.wr_gemv(9, 16, 256, 16, 16, 16, 2, 256, 16, 16, 1 << 20, None)   # M > 8
+    assert st == 1
+    st = wr._lib.wr_gemv(1, 16, 256, 16, 16, 16, 4, 256, 16, 16, 1 << 20, None)   # bits
+    assert st == 2
+    st = wr._lib.wr_gemv(1, 16, 256, 16, 16, 16, 2, 128, 16, 16, 1 << 20, None)   # group
+    assert st == 2
+    st = wr._lib.wr_gemv(1, 16, 300, 16, 16, 16, 2, 256, 16, 16, 1 << 20, None)   # K % 256
+    assert st == 1
+    st = wr._lib.wr_gemv(1, 16, 256, 16, 16, 16, 2, 256, 16, 16, 0, None)         # workspace
+    assert st == 1
+    st = wr._lib.wr_gemm(4, 16, 256, 16, 0, 16, 2, 256, 16, 16, 1 << 20, None)    # null packed
+    assert st == 1
+    st = wr._lib.wr_gemm_ternary(4, 16, 200, 16, 16, 16, 16, 16, 16, 1 << 20, None)  # K % 128
+    assert st == 1
+    st = wr._lib.wr_unpack_bf16(2, 16, 256, 16, 16, 64, 16, None)                 # group
+    assert st == 2
+    assert wr.wr_gemv_workspace_bytes(9, 16, 256, 2) == 0
+    assert wr.wr_gemv_workspace_bytes(1, 16, 256, 2) > 0

@@ -1,0 +1,144 @@
+"""GPU parity: the CUDA path against the fp64 oracle, element by element, through the C ABI.
+
+Unpack must be bit-exact; every GEMV/GEMM output must satisfy
+|y_gpu - y_ref| <= 1e-4 * sum_k |w[n,k] x[m,k]| (the bound in the oracle's fp64), and be
+exactly zero where that sum is zero. Shapes span several tiles, ragged N, every M from 1 to 8
+for the decode path, and the Qwen3-4B layer shapes at full size."""
+import numpy as np
+import pytest
+
+import wr_synth
+from oracle import wr_oracle as o
+from gpu_inputs import check_close, dev, q_case, t_case, torch_mod
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def wr():
+    torch = torch_mod()
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import bit_weight_only_wr_b200 as lib
+    return lib
+
+
+def _zeros_ws(nbytes):
+    torch = torch_mod()
+    return torch.zeros(max(nbytes, 256), dtype=torch.uint8, device="cuda")
+
+
+def _run_gemv(wr, bits, x_bits, packed, scales, N, K):
+    torch = torch_mod()
+    M = x_bits.shape[0]
+    x = dev(x_bits)
+    y = torch.full((M, N), float("nan"), dtype=torch.float32, device="cuda")
+    nb = wr.wr_gemv_workspace_bytes(M, N, K, bits)
+    ws = _zeros_ws(nb)
+    wr.wr_gemv(M, N, K, x, packed, scales, bits, y, ws, nb)
+    torch.cuda.synchronize()
+    return y.cpu().numpy(), ws
+
+
+# ---------------------------------------------------------------- unpack (bit-exact)
+
+@pytest.mark.parametrize("bits,N,K", [(2, 40, 512), (2, 2560, 2560), (3, 33, 768), (3, 1024, 2560)])
+def test_unpack_bf16_bit_exact(wr, bits, N, K):
+    torch = torch_mod()
+    codes, scales, packed, s_d = q_case(wr, bits, N, K, seed=N + K + bits)
+    out = torch.zeros((N, K), dtype=torch.int16, device="cuda")
+    wr.wr_unpack_bf16(bits, N, K, packed, s_d, out)
+    torch.cuda.synchronize()
+    ref = o.unpack_bf16(codes, scales, bits)
+    assert np.array_equal(out.cpu().numpy().view(np.uint16), ref)
+
+
+@pytest.mark.parametrize("N,K", [(35, 640), (48, 4096), (16, 9728)])
+def test_unpack_bf16_ternary_bit_exact(wr, N, K):
+    torch = torch_mod()
+    codes, alpha, signs, packed, a_d, _ = t_case(wr, N, K, seed=N + K)
+    out = torch.zeros((N, K), dtype=torch.int16, device="cuda")
+    wr.wr_unpack_bf16(1, N, K, packed, a_d, out)
+    torch.cuda.synchronize()
+    assert np.array_equal(out.cpu().numpy().view(np.uint16), o.unpack_bf16_ternary(codes, alpha))
+
+
+# ---------------------------------------------------------------- decode GEMV
+
+@pytest.mark.parametrize("bits", [2, 3])
+@pytest.mark.parametrize("M", [1, 2, 3, 4, 5, 6, 7, 8])
+def test_gemv_every_m_ragged(wr, bits, M):
+    N, K = 40, 768
+    codes, scales, packed, s_d = q_case(wr, bits, N, K, seed=11 * M + bits)
+    x = wr_synth.activations_bf16(200 + M, M, K)
+    y, _ = _run_gemv(wr, bits, x, packed, s_d, N, K)
+    ref, B = o.gemm_codes(x, codes, scales, bits)
+    check_close(y, ref, B)
+
+
+@pytest.mark.parametrize("bits,N,K,M", [(2, 2560, 2560, 1), (2, 4096, 2560, 8), (3, 1024, 2560, 1),
+                                        (3, 2560, 9728, 1), (3, 2560, 9728, 8), (2, 9728, 2560, 3)])
+def test_gemv_layer_shapes(wr, bits, N, K, M):
+    codes, scales, packed, s_d = q_case(wr, bits, N, K, seed=N * 3 + K + M)
+    x = wr_synth.activations_bf16(300 + M, M, K)
+    y, ws = _run_gemv(wr, bits, x, packed, s_d, N, K)
+    ref, B = o.gemm_codes(x, codes, scales, bits)
+    check_close(y, ref, B)
+    # the arrival counters are back to zero after the call
+    tiles = (N + 15) // 16
+    assert int(ws[: 4 * tiles].view(dtype=torch_mod().int32).abs().sum()) == 0
+
+
+def test_gemv_deterministic(wr):
+    N, K, M = 2560, 9728, 2
+    codes, scales, packed, s_d = q_case(wr, 3, N, K, seed=77)
+    x = wr_synth.activations_bf16(78, M, K)
+    y1, _ = _run_gemv(wr, 3, x, packed, s_d, N, K)
+    y2, _ = _run_gemv(wr, 3, x, packed, s_d, N, K)
+    assert np.array_equal(y1.view(np.uint32), y2.view(np.uint32))
+
+
+def test_gemv_zero_cases(wr):
+    N, K, M = 48, 512, 3
+    codes, scales, packed, s_d = q_case(wr, 2, N, K, seed=5)
+    x = wr_synth.activations_bf16(6, M, K)
+    x[1] = 0                                   # an all-zero token
+    y, _ = _run_gemv(wr, 2, x, packed, s_d, N, K)
+    ref, B = o.gemm_codes(x, codes, scales, 2)
+    check_close(y, ref, B)
+    assert np.all(y[1] == 0)
+    zs = dev(np.zeros_like(scales.view(np.uint16)))   # all scales zero -> y exactly 0
+    y0, _ = _run_gemv(wr, 2, x, packed, zs, N, K)
+    assert np.all(y0 == 0)
+
+
+# ---------------------------------------------------------------- ternary
+
+@pytest.mark.parametrize("M", [1, 2, 4, 5, 8])
+@pytest.mark.parametrize("N,K", [(40, 640), (64, 4096)])
+def test_ternary_gemv(wr, M, N, K):
+    torch = torch_mod()
+    codes, alpha, signs, packed, a_d, s_d = t_case(wr, N, K, seed=N + K + M)
+    x = wr_synth.activations_bf16(400 + M, M, K)
+    y = torch.full((M, N), float("nan"), dtype=torch.float32, device="cuda")
+    nb = wr.wr_gemm_ternary_workspace_bytes(M, N, K)
+    ws = _zeros_ws(nb)
+    wr.wr_gemm_ternary(M, N, K, dev(x), packed, a_d, s_d, y, ws, nb)
+    torch.cuda.synchronize()
+    ref, B = o.gemm_ternary(x, codes, alpha, signs)
+    check_close(y.cpu().numpy(), ref, B)
+
+
+@pytest.mark.parametrize("N,K", [(2560, 9728), (9728, 2560)])
+def test_ternary_gemv_layer_shapes(wr, N, K):
+    torch = torch_mod()
+    codes, alpha, signs, packed, a_d, s_d = t_case(wr, N, K, seed=N + 2 * K)
+    M = 1
+    x = wr_synth.activations_bf16(500, M, K)
+    y = torch.full((M, N), float("nan"), dtype=torch.float32, device="cuda")
+    nb = wr.wr_gemm_ternary_workspace_bytes(M, N, K)
+    ws = _zeros_ws(nb)
+    wr.wr_gemm_ternary(M, N, K, dev(x), packed, a_d, s_d, y, ws, nb)
+    torch.cuda.synchronize()
+    ref, B = o.gemm_ternary(x, codes, alpha, signs)
+    check_close(y.cpu().numpy(), ref, B)
