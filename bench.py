@@ -263,7 +263,7 @@ def main():
         mods.append(dict(layer=layer, name=name, K=K, N=N, bits=bits, packed=packed, scales=scales))
     setup_s = time.time() - t_setup
 
-    def body_run(M, steps, warmup, with_e2e):
+    def body_run(M, steps, warmup, with_e2e, batched=True):
         xs_host = [wr_synth.activations_bf16(10_000 + 10 * m["layer"] + i % 7, M, m["K"])
                    for i, m in enumerate(mods)]
         x_all = torch.from_numpy(np.concatenate([x.ravel() for x in xs_host]).view(np.int16)).cuda()
@@ -276,18 +276,30 @@ def main():
         for m in mods:
             yoffs.append(o_)
             o_ += M * m["N"]
-        nb = max(wr.wr_gemv_workspace_bytes(M, m["N"], m["K"], m["bits"]) for m in mods)
-        ws = torch.zeros(nb, dtype=torch.uint8, device="cuda")
         xp, yp = x_all.data_ptr(), y_all.data_ptr()
+        if batched:
+            # the whole body: one launch of the batched decode GEMV per token
+            arr = wr._problems([(xp + 2 * offs[i], m["packed"], m["scales"], yp + 4 * yoffs[i], m["N"], m["K"],
+                                 m["bits"]) for i, m in enumerate(mods)])
+            nb = wr.wr_gemv_batched_workspace_bytes(M, arr)
+            ws = torch.zeros(nb, dtype=torch.uint8, device="cuda")
+            launches = (len(mods) + 255) // 256
 
-        def step():
-            for i, m in enumerate(mods):
-                wr.wr_gemv(M, m["N"], m["K"], xp + 2 * offs[i], m["packed"], m["scales"], m["bits"],
-                           yp + 4 * yoffs[i], ws, nb)
+            def step():
+                wr.wr_gemv_batched(M, arr, ws, nb)
+        else:
+            nb = max(wr.wr_gemv_workspace_bytes(M, m["N"], m["K"], m["bits"]) for m in mods)
+            ws = torch.zeros(nb, dtype=torch.uint8, device="cuda")
+            launches = len(mods)
+
+            def step():
+                for i, m in enumerate(mods):
+                    wr.wr_gemv(M, m["N"], m["K"], xp + 2 * offs[i], m["packed"], m["scales"], m["bits"],
+                               yp + 4 * yoffs[i], ws, nb)
         ms = graph_time_ms(torch, step, steps, warmup, stream, dist) / steps
         ms = max_over_ranks(torch, dist, ms)
         nbytes = sum(module_bytes(wr, M, m["N"], m["K"], m["bits"]) for m in mods)
-        out = {"ms": ms, "bytes": nbytes, "gbs": nbytes / ms / 1e6, "launches": len(mods)}
+        out = {"ms": ms, "bytes": nbytes, "gbs": nbytes / ms / 1e6, "launches": launches}
         if with_e2e:
             xh = x_all.cpu().pin_memory()
             yh = torch.empty(y_all.numel(), dtype=torch.float32).pin_memory()
@@ -315,15 +327,19 @@ def main():
             extras["body_m8"]["tokens_per_s"] = 8e3 / extras["body_m8"]["ms"]
         except Exception as e:  # noqa: BLE001
             extras["body_m8"] = {"error": repr(e)}
+        try:
+            extras["body_m1_one_call_per_linear"] = body_run(1, max(5, args.steps // 2), 3, False, batched=False)
+        except Exception as e:  # noqa: BLE001
+            extras["body_m1_one_call_per_linear"] = {"error": repr(e)}
         extras.update(run_extras(args, wr, torch, np, stream, dist, hbm_peak, bf16_peak))
 
-    # the graph holds only GEMV launches: bytes per launch / time per launch = bytes / step time
+    # one batched decode launch per step: algorithmic bytes per launch / event-timed launch time
     achieved = head["gbs"]
     roof = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
             "frac": achieved / hbm_peak, "traffic": None, "peak_kind": peak_kind,
-            "kernel": "gemv_q_kernel (2/3-bit decode GEMV)",
-            "note": "average GEMV launch in the M=1 body graph: algorithmic bytes per launch / "
-                    "event-timed duration per launch"}
+            "kernel": "decode_kernel<false> (batched 2/3-bit decode GEMV, tcgen05)",
+            "note": "the M=1 body step is one launch of the batched decode GEMV: algorithmic bytes per "
+                    "launch / event-timed duration per launch"}
     cb = None
     if rank == 0 and world == 1:
         try:
@@ -346,6 +362,7 @@ def main():
                 "h2d_bytes_per_step": head["e2e"]["h2d"], "d2h_bytes_per_step": head["e2e"]["d2h"],
                 "ms_per_step": head["e2e"]["ms"]},
         "gpu_launches": head["launches"] * args.steps,
+        "step": "252 linears (36 layers x 7) in one wr_gemv_batched launch, CUDA graph replay",
         "extras": extras,
     }
     if rank == 0:

@@ -17,13 +17,23 @@ __all__ = [
     "wr_abi_version", "wr_status_string", "wr_packed_bytes", "wr_pack", "wr_unpack_codes",
     "wr_quantize", "wr_quantize_ternary", "wr_unpack_bf16", "wr_gemv_workspace_bytes", "wr_gemv",
     "wr_gemm_workspace_bytes", "wr_gemm", "wr_gemm_ternary_workspace_bytes", "wr_gemm_ternary",
-    "wr_get_device_error", "exported_symbols",
+    "wr_get_device_error", "exported_symbols", "WrGemvProblem", "wr_gemv_batched_workspace_bytes",
+    "wr_gemv_batched",
 ]
 
 WR_FMT_TERNARY, WR_FMT_Q2, WR_FMT_Q3 = 1, 2, 3
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libwr.so")
 
 _c_i64, _c_int, _c_size, _vp = ctypes.c_int64, ctypes.c_int, ctypes.c_size_t, ctypes.c_void_p
+
+class WrGemvProblem(ctypes.Structure):
+    """Mirror of the C struct wr_gemv_problem."""
+    _fields_ = [("x", ctypes.c_void_p), ("packed", ctypes.c_void_p), ("scales", ctypes.c_void_p),
+                ("y", ctypes.c_void_p), ("N", ctypes.c_int64), ("K", ctypes.c_int64),
+                ("bits", ctypes.c_int32), ("reserved", ctypes.c_int32)]
+
+
+_PROBLEMS = ctypes.POINTER(WrGemvProblem)
 
 _SIGNATURES = {
     "wr_abi_version": (_c_int, []),
@@ -36,6 +46,8 @@ _SIGNATURES = {
     "wr_unpack_bf16": (_c_int, [_c_int, _c_i64, _c_i64, _vp, _vp, _c_int, _vp, _vp]),
     "wr_gemv_workspace_bytes": (_c_size, [_c_i64, _c_i64, _c_i64, _c_int]),
     "wr_gemv": (_c_int, [_c_i64, _c_i64, _c_i64, _vp, _vp, _vp, _c_int, _c_int, _vp, _vp, _c_size, _vp]),
+    "wr_gemv_batched_workspace_bytes": (_c_size, [_c_i64, ctypes.c_int32, _PROBLEMS]),
+    "wr_gemv_batched": (_c_int, [_c_i64, ctypes.c_int32, _PROBLEMS, _vp, _c_size, _vp]),
     "wr_gemm_workspace_bytes": (_c_size, [_c_i64, _c_i64, _c_i64, _c_int]),
     "wr_gemm": (_c_int, [_c_i64, _c_i64, _c_i64, _vp, _vp, _vp, _c_int, _c_int, _vp, _vp, _c_size, _vp]),
     "wr_gemm_ternary_workspace_bytes": (_c_size, [_c_i64, _c_i64, _c_i64]),
@@ -160,6 +172,26 @@ def wr_gemv(M: int, N: int, K: int, x, packed, scales, bits: int, y, workspace, 
             group: int = 256, stream=None) -> None:
     _check("wr_gemv", _lib.wr_gemv(M, N, K, _ptr(x), _ptr(packed), _ptr(scales), bits, group, _ptr(y),
                                    _ptr(workspace), workspace_bytes, _stream(stream)))
+
+
+def _problems(problems):
+    """problems: sequence of (x, packed, scales, y, N, K, bits) -> ctypes array."""
+    arr = (WrGemvProblem * len(problems))()
+    for i, (x, packed, scales, y, N, K, bits) in enumerate(problems):
+        arr[i] = WrGemvProblem(_ptr(x), _ptr(packed), _ptr(scales), _ptr(y), N, K, bits, 0)
+    return arr
+
+
+def wr_gemv_batched_workspace_bytes(M: int, problems) -> int:
+    arr = problems if isinstance(problems, ctypes.Array) else _problems(problems)
+    return _lib.wr_gemv_batched_workspace_bytes(M, len(arr), arr)
+
+
+def wr_gemv_batched(M: int, problems, workspace, workspace_bytes: int, stream=None) -> None:
+    """problems: sequence of (x, packed, scales, y, N, K, bits), or a prepared ctypes array."""
+    arr = problems if isinstance(problems, ctypes.Array) else _problems(problems)
+    _check("wr_gemv_batched", _lib.wr_gemv_batched(M, len(arr), arr, _ptr(workspace), workspace_bytes,
+                                                   _stream(stream)))
 
 
 def wr_gemm_workspace_bytes(M: int, N: int, K: int, bits: int) -> int:

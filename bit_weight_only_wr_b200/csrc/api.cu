@@ -8,8 +8,7 @@
 #include <cstdint>
 #include <mutex>
 
-#include "gemm.cuh"
-#include "gemv.cuh"
+#include "tc_kernels.cuh"
 #include "wr.h"
 #include "wr_internal.h"
 
@@ -36,24 +35,17 @@ int sm_count() {
   return cache[dev];
 }
 
-// Workspace of the decode GEMV: [counters: one int per 16-row tile][partials: 2 per warp,
-// 16 x 8 fp32 each][ternary only: R x as two bf16 planes of M x Kp].
-struct GemvWorkspace {
-  size_t counter_off, partial_off, xr_off, total;
-};
-
-GemvWorkspace gemv_workspace(int fmt, int64_t M, int64_t N, int64_t K) {
-  int64_t unit_bytes = 0, units = 0, tiles = 0;
-  wr::packed_geometry(fmt, N, K, &unit_bytes, &units, &tiles);
-  const int64_t U = tiles * units;
-  const int64_t wt = std::min<int64_t>(U, wr::kGemvMaxWarps);
-  GemvWorkspace w;
-  w.counter_off = 0;
-  w.partial_off = align256((size_t)tiles * sizeof(int));
-  w.xr_off = w.partial_off + align256((size_t)(2 * wt) * 128 * sizeof(float));
-  w.total = w.xr_off;
-  if (fmt == WR_FMT_TERNARY) w.total += align256((size_t)(2 * M) * (size_t)(units * 320) * 2);
-  return w;
+int* device_error_word() {
+  static std::mutex mu;
+  static int* cache[64] = {nullptr};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!cache[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_device_error) == cudaSuccess) cache[dev] = static_cast<int*>(p);
+  }
+  return cache[dev];
 }
 
 wr_status check_dims(int64_t M, int64_t N, int64_t K) {
@@ -62,37 +54,168 @@ wr_status check_dims(int64_t M, int64_t N, int64_t K) {
   return WR_OK;
 }
 
-// Launch the GEMV on tokens [0, M) (M <= 8) of already validated operands.
-wr_status run_gemv(int fmt, int M, int N, int K, const uint16_t* x, const uint8_t* packed,
-                   const uint16_t* scales, const uint16_t* alpha, const uint32_t* signs, float* y,
-                   void* workspace, cudaStream_t stream) {
-  int64_t unit_bytes = 0, units = 0, tiles = 0;
-  wr::packed_geometry(fmt, N, K, &unit_bytes, &units, &tiles);
-  const GemvWorkspace ws = gemv_workspace(fmt, M, N, K);
+constexpr int kPlanSMs = 148;   // split heuristics are sized for a 148-SM part (device-independent)
+constexpr int kDecodeTokens = 16;
+
+// ---- decode kernel (M <= 16): work items (problem, 128-row group, block range) and workspace
+// [counters: one int per row group of every problem][split-K partials of problems with P > 1]
+// [ternary only: R x as two bf16 planes of M x Kp].
+struct DecodePlan {
+  wr::DecArgs args;
+  size_t counter_off = 0, partial_off = 0, xr_off = 0, total = 0;
+};
+
+struct ProblemShape {
+  int64_t N, K;
+  int fmt;
+};
+
+void plan_decode(int64_t M, int count, const ProblemShape* shapes, DecodePlan* dp) {
+  wr::DecArgs& a = dp->args;
+  a.count = count;
+  a.M = (int)M;
+  int64_t total_blocks = 0;
+  for (int i = 0; i < count; ++i) {
+    int64_t ub = 0, units = 0, tiles = 0;
+    wr::packed_geometry(shapes[i].fmt, shapes[i].N, shapes[i].K, &ub, &units, &tiles);
+    wr::DecProblem& pr = a.prob[i];
+    pr = wr::DecProblem{};
+    pr.N = (int)shapes[i].N;
+    pr.K = (int)shapes[i].K;
+    pr.B = (int)units;
+    pr.Kp = shapes[i].fmt == WR_FMT_TERNARY ? (int)(units * 320) : (int)shapes[i].K;
+    pr.RG = (int)((shapes[i].N + 127) / 128);
+    pr.bits = shapes[i].fmt == WR_FMT_TERNARY ? 1 : shapes[i].fmt;
+    total_blocks += (int64_t)pr.RG * pr.B;
+  }
+  const int64_t target_items = std::max<int64_t>(2 * kPlanSMs, (total_blocks + 7) / 8);
+  const double bpi = (double)total_blocks / (double)target_items;
+  int items = 0, counters = 0;
+  int64_t partials = 0;
+  size_t xr_bytes = 0;
+  for (int i = 0; i < count; ++i) {
+    wr::DecProblem& pr = a.prob[i];
+    int P = (int)std::lround((double)pr.B / bpi);
+    pr.P = std::max(1, std::min(pr.B, P));
+    pr.item_base = items;
+    pr.counter_base = counters;
+    pr.partial_base = partials;
+    items += pr.RG * pr.P;
+    counters += pr.RG;
+    if (pr.P > 1) partials += (int64_t)pr.RG * pr.P * M * 128;
+    if (shapes[i].fmt == WR_FMT_TERNARY) xr_bytes += align256((size_t)(2 * M) * (size_t)pr.Kp * 2);
+  }
+  a.items = items;
+  dp->counter_off = 0;
+  dp->partial_off = align256((size_t)counters * sizeof(int));
+  dp->xr_off = dp->partial_off + align256((size_t)partials * sizeof(float));
+  dp->total = dp->xr_off + xr_bytes;
+}
+
+wr_status run_decode(DecodePlan& dp, bool ternary, void* workspace, cudaStream_t stream) {
   uint8_t* wsb = static_cast<uint8_t*>(workspace);
-  wr::GemvArgs a{};
-  a.x = x;
+  dp.args.counter = reinterpret_cast<int*>(wsb + dp.counter_off);
+  dp.args.partial = reinterpret_cast<float*>(wsb + dp.partial_off);
+  dp.args.err = device_error_word();
+  const int grid = (int)std::min<int64_t>(dp.args.items, (int64_t)sm_count() * 2);
+  return wr::launch_decode(ternary, dp.args, grid, stream) == cudaSuccess ? WR_OK : WR_ERR_CUDA;
+}
+
+// ---- prefill GEMM kernel (M > 16): 128-row groups x 128-token tiles x K splits; workspace
+// [counters: one int per (row group, token tile)][split-K partials].
+struct GemmPlan {
+  int B = 0, RG = 0, MT = 0, P = 1, items = 0;
+  size_t counter_off = 0, partial_off = 0, total = 0;
+};
+
+GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K) {
+  GemmPlan p;
+  p.B = (int)(K / 256);
+  p.RG = (int)((N + 127) / 128);
+  p.MT = (int)((M + 127) / 128);
+  const int64_t base = (int64_t)p.RG * p.MT;
+  if (base < kPlanSMs) p.P = (int)std::min<int64_t>(p.B, (kPlanSMs + base - 1) / base);
+  p.items = (int)(base * p.P);
+  p.counter_off = 0;
+  p.partial_off = align256((size_t)base * sizeof(int));
+  p.total = p.partial_off + (p.P > 1 ? align256((size_t)base * p.P * 128 * 128 * sizeof(float)) : 0);
+  return p;
+}
+
+wr_status run_gemm(int bits, int M, int N, int K, const uint16_t* x, const uint8_t* packed, const uint16_t* scales,
+                   float* y, void* workspace, cudaStream_t stream) {
+  const GemmPlan p = plan_gemm(M, N, K);
+  uint8_t* wsb = static_cast<uint8_t*>(workspace);
+  wr::TcArgs a{};
   a.packed = packed;
   a.scales = scales;
-  a.row_scale = alpha;
   a.y = y;
-  a.counter = reinterpret_cast<int*>(wsb + ws.counter_off);
-  a.partial = reinterpret_cast<float*>(wsb + ws.partial_off);
+  a.partial = reinterpret_cast<float*>(wsb + p.partial_off);
+  a.counter = reinterpret_cast<int*>(wsb + p.counter_off);
+  a.err = device_error_word();
   a.M = M;
   a.N = N;
   a.K = K;
-  a.B = (int)units;
-  a.U = tiles * units;
-  const int64_t wt_cap = std::min<int64_t>((int64_t)sm_count() * wr::kGemvWarpsPerSM, wr::kGemvMaxWarps);
-  a.Wt = (int)std::min<int64_t>(a.U, wt_cap);
-  if (fmt == WR_FMT_TERNARY) {
-    uint16_t* xr = reinterpret_cast<uint16_t*>(wsb + ws.xr_off);
-    a.xr = xr;
-    if (wr::launch_rotate_x(x, signs, xr, M, K, units * 320, stream) != cudaSuccess) return WR_ERR_CUDA;
+  a.B = p.B;
+  a.RG = p.RG;
+  a.MT = p.MT;
+  a.P = p.P;
+  a.items = p.items;
+  const int grid = (int)std::min<int64_t>(p.items, sm_count());
+  return wr::launch_tc_kernel(bits, 128, a, x, M, K, grid, stream) == cudaSuccess ? WR_OK : WR_ERR_CUDA;
+}
+
+// One Q2/Q3 call of any M.
+size_t q_workspace(int bits, int64_t M, int64_t N, int64_t K) {
+  if (M <= kDecodeTokens) {
+    static thread_local DecodePlan dp;
+    const ProblemShape sh{N, K, bits};
+    plan_decode(M, 1, &sh, &dp);
+    return dp.total;
   }
-  const int wpc = wr::gemv_warps_per_cta();
-  const int ctas = (a.Wt + wpc - 1) / wpc;
-  if (wr::launch_gemv(fmt, a, ctas, stream) != cudaSuccess) return WR_ERR_CUDA;
+  return plan_gemm(M, N, K).total;
+}
+
+wr_status run_q(int bits, int64_t M, int64_t N, int64_t K, const uint16_t* x, const void* packed,
+                const uint16_t* scales, float* y, void* workspace, cudaStream_t stream) {
+  if (M <= kDecodeTokens) {
+    static thread_local DecodePlan dp;
+    const ProblemShape sh{N, K, bits};
+    plan_decode(M, 1, &sh, &dp);
+    dp.args.prob[0].x = x;
+    dp.args.prob[0].packed = static_cast<const uint8_t*>(packed);
+    dp.args.prob[0].scales = scales;
+    dp.args.prob[0].y = y;
+    return run_decode(dp, false, workspace, stream);
+  }
+  return run_gemm(bits, (int)M, (int)N, (int)K, x, static_cast<const uint8_t*>(packed), scales, y, workspace, stream);
+}
+
+// Ternary: 8-token slices through the decode kernel (R x hi and lo fill the 16 MMA columns).
+size_t t_workspace(int64_t M, int64_t N, int64_t K) {
+  static thread_local DecodePlan dp;
+  const ProblemShape sh{N, K, WR_FMT_TERNARY};
+  plan_decode(std::min<int64_t>(M, 8), 1, &sh, &dp);
+  return dp.total;
+}
+
+wr_status run_t(int64_t M, int64_t N, int64_t K, const uint16_t* x, const void* packed, const uint16_t* alpha,
+                const uint32_t* signs, float* y, void* workspace, cudaStream_t stream) {
+  static thread_local DecodePlan dp;
+  for (int64_t m0 = 0; m0 < M; m0 += 8) {
+    const int mm = (int)std::min<int64_t>(8, M - m0);
+    const ProblemShape sh{N, K, WR_FMT_TERNARY};
+    plan_decode(mm, 1, &sh, &dp);
+    uint16_t* xr = reinterpret_cast<uint16_t*>(static_cast<uint8_t*>(workspace) + dp.xr_off);
+    if (wr::launch_rotate_x(x + m0 * K, signs, xr, mm, (int)K, dp.args.prob[0].Kp, stream) != cudaSuccess)
+      return WR_ERR_CUDA;
+    dp.args.prob[0].x = xr;
+    dp.args.prob[0].packed = static_cast<const uint8_t*>(packed);
+    dp.args.prob[0].scales = alpha;
+    dp.args.prob[0].y = y + m0 * N;
+    const wr_status st = run_decode(dp, true, workspace, stream);
+    if (st != WR_OK) return st;
+  }
   return WR_OK;
 }
 
@@ -129,7 +252,7 @@ wr_status wr_unpack_bf16(int fmt, int64_t N, int64_t K, const void* packed, cons
 size_t wr_gemv_workspace_bytes(int64_t M, int64_t N, int64_t K, int bits) {
   if (bits != 2 && bits != 3) return 0;
   if (M < 1 || M > 8 || check_dims(M, N, K) != WR_OK || K % 256 != 0) return 0;
-  return gemv_workspace(bits, M, N, K).total;
+  return q_workspace(bits, M, N, K);
 }
 
 wr_status wr_gemv(int64_t M, int64_t N, int64_t K, const uint16_t* x, const void* packed,
@@ -140,15 +263,61 @@ wr_status wr_gemv(int64_t M, int64_t N, int64_t K, const uint16_t* x, const void
   if (M < 1 || M > 8 || check_dims(M, N, K) != WR_OK || K % 256 != 0) return WR_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(packed) || !aligned16(scales) || !aligned16(y) || !aligned16(workspace))
     return WR_ERR_INVALID_ARG;
-  if (workspace_bytes < gemv_workspace(bits, M, N, K).total) return WR_ERR_INVALID_ARG;
-  return run_gemv(bits, (int)M, (int)N, (int)K, x, static_cast<const uint8_t*>(packed), scales, nullptr,
-                  nullptr, y, workspace, static_cast<cudaStream_t>(stream));
+  if (workspace_bytes < q_workspace(bits, M, N, K)) return WR_ERR_INVALID_ARG;
+  return run_q(bits, M, N, K, x, packed, scales, y, workspace, static_cast<cudaStream_t>(stream));
+}
+
+static bool batch_ok(int64_t M, int32_t count, const wr_gemv_problem* pr) {
+  if (M < 1 || M > 8 || count < 1 || !pr) return false;
+  for (int i = 0; i < count; ++i) {
+    if (pr[i].bits != 2 && pr[i].bits != 3) return false;
+    if (pr[i].reserved != 0 || check_dims(M, pr[i].N, pr[i].K) != WR_OK || pr[i].K % 256 != 0) return false;
+    if (!aligned16(pr[i].x) || !aligned16(pr[i].packed) || !aligned16(pr[i].scales) || !aligned16(pr[i].y))
+      return false;
+  }
+  return true;
+}
+
+size_t wr_gemv_batched_workspace_bytes(int64_t M, int32_t count, const wr_gemv_problem* problems) {
+  if (!batch_ok(M, count, problems)) return 0;
+  size_t total = 0;
+  static thread_local DecodePlan dp;
+  ProblemShape sh[wr::kMaxDecodeProblems];
+  for (int c0 = 0; c0 < count; c0 += wr::kMaxDecodeProblems) {
+    const int n = std::min(count - c0, wr::kMaxDecodeProblems);
+    for (int i = 0; i < n; ++i) sh[i] = ProblemShape{problems[c0 + i].N, problems[c0 + i].K, problems[c0 + i].bits};
+    plan_decode(M, n, sh, &dp);
+    total = std::max(total, dp.total);
+  }
+  return total;
+}
+
+wr_status wr_gemv_batched(int64_t M, int32_t count, const wr_gemv_problem* problems, void* workspace,
+                          size_t workspace_bytes, void* stream) {
+  if (!batch_ok(M, count, problems) || !aligned16(workspace)) return WR_ERR_INVALID_ARG;
+  if (workspace_bytes < wr_gemv_batched_workspace_bytes(M, count, problems)) return WR_ERR_INVALID_ARG;
+  static thread_local DecodePlan dp;
+  ProblemShape sh[wr::kMaxDecodeProblems];
+  for (int c0 = 0; c0 < count; c0 += wr::kMaxDecodeProblems) {
+    const int n = std::min(count - c0, wr::kMaxDecodeProblems);
+    for (int i = 0; i < n; ++i) sh[i] = ProblemShape{problems[c0 + i].N, problems[c0 + i].K, problems[c0 + i].bits};
+    plan_decode(M, n, sh, &dp);
+    for (int i = 0; i < n; ++i) {
+      dp.args.prob[i].x = problems[c0 + i].x;
+      dp.args.prob[i].packed = static_cast<const uint8_t*>(problems[c0 + i].packed);
+      dp.args.prob[i].scales = problems[c0 + i].scales;
+      dp.args.prob[i].y = problems[c0 + i].y;
+    }
+    const wr_status st = run_decode(dp, false, workspace, static_cast<cudaStream_t>(stream));
+    if (st != WR_OK) return st;
+  }
+  return WR_OK;
 }
 
 size_t wr_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int bits) {
   if (bits != 2 && bits != 3) return 0;
   if (check_dims(M, N, K) != WR_OK || K % 256 != 0) return 0;
-  return std::max(wr::gemm_workspace_bytes(M, N, K, bits), gemv_workspace(bits, 8, N, K).total);
+  return q_workspace(bits, M, N, K);
 }
 
 wr_status wr_gemm(int64_t M, int64_t N, int64_t K, const uint16_t* x, const void* packed,
@@ -159,30 +328,13 @@ wr_status wr_gemm(int64_t M, int64_t N, int64_t K, const uint16_t* x, const void
   if (check_dims(M, N, K) != WR_OK || K % 256 != 0) return WR_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(packed) || !aligned16(scales) || !aligned16(y) || !aligned16(workspace))
     return WR_ERR_INVALID_ARG;
-  if (workspace_bytes < wr_gemm_workspace_bytes(M, N, K, bits)) return WR_ERR_INVALID_ARG;
-  const cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (M <= 8)
-    return run_gemv(bits, (int)M, (int)N, (int)K, x, static_cast<const uint8_t*>(packed), scales, nullptr,
-                    nullptr, y, workspace, s);
-  const cudaError_t e = wr::launch_gemm(bits, (int)M, (int)N, (int)K, x, static_cast<const uint8_t*>(packed),
-                                        scales, y, workspace, s);
-  if (e == cudaErrorNotSupported) {
-    // interim path until the tensor-memory kernel covers this shape: 8-token GEMV slices
-    for (int64_t m0 = 0; m0 < M; m0 += 8) {
-      const int mm = (int)std::min<int64_t>(8, M - m0);
-      const wr_status st = run_gemv(bits, mm, (int)N, (int)K, x + m0 * K, static_cast<const uint8_t*>(packed),
-                                    scales, nullptr, nullptr, y + m0 * N, workspace, s);
-      if (st != WR_OK) return st;
-    }
-    return WR_OK;
-  }
-  return e == cudaSuccess ? WR_OK : WR_ERR_CUDA;
+  if (workspace_bytes < q_workspace(bits, M, N, K)) return WR_ERR_INVALID_ARG;
+  return run_q(bits, M, N, K, x, packed, scales, y, workspace, static_cast<cudaStream_t>(stream));
 }
 
 size_t wr_gemm_ternary_workspace_bytes(int64_t M, int64_t N, int64_t K) {
   if (check_dims(M, N, K) != WR_OK || K % 128 != 0) return 0;
-  return std::max(gemv_workspace(WR_FMT_TERNARY, std::min<int64_t>(M, 8), N, K).total,
-                  wr::gemm_ternary_workspace_bytes(M, N, K));
+  return t_workspace(M, N, K);
 }
 
 wr_status wr_gemm_ternary(int64_t M, int64_t N, int64_t K, const uint16_t* x, const void* packed,
@@ -192,24 +344,8 @@ wr_status wr_gemm_ternary(int64_t M, int64_t N, int64_t K, const uint16_t* x, co
   if (!aligned16(x) || !aligned16(packed) || !aligned16(alpha) || !aligned16(sign_bits) || !aligned16(y) ||
       !aligned16(workspace))
     return WR_ERR_INVALID_ARG;
-  if (workspace_bytes < wr_gemm_ternary_workspace_bytes(M, N, K)) return WR_ERR_INVALID_ARG;
-  const cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (M <= 8)
-    return run_gemv(WR_FMT_TERNARY, (int)M, (int)N, (int)K, x, static_cast<const uint8_t*>(packed), nullptr,
-                    alpha, sign_bits, y, workspace, s);
-  const cudaError_t e = wr::launch_gemm_ternary((int)M, (int)N, (int)K, x, static_cast<const uint8_t*>(packed),
-                                                alpha, sign_bits, y, workspace, s);
-  if (e == cudaErrorNotSupported) {
-    for (int64_t m0 = 0; m0 < M; m0 += 8) {
-      const int mm = (int)std::min<int64_t>(8, M - m0);
-      const wr_status st = run_gemv(WR_FMT_TERNARY, mm, (int)N, (int)K, x + m0 * K,
-                                    static_cast<const uint8_t*>(packed), nullptr, alpha, sign_bits, y + m0 * N,
-                                    workspace, s);
-      if (st != WR_OK) return st;
-    }
-    return WR_OK;
-  }
-  return e == cudaSuccess ? WR_OK : WR_ERR_CUDA;
+  if (workspace_bytes < t_workspace(M, N, K)) return WR_ERR_INVALID_ARG;
+  return run_t(M, N, K, x, packed, alpha, sign_bits, y, workspace, static_cast<cudaStream_t>(stream));
 }
 
 wr_status wr_get_device_error(void* stream) {

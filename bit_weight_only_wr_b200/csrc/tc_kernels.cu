@@ -1,0 +1,551 @@
+// Packed-code GEMV/GEMM on tcgen05 tensor cores (sm_100a).
+//
+//   y[m,n] = sum_b s[n,b] sum_{k in b} g[n,k] x[m,k]         (2/3-bit odd grid, fp16 scales)
+//   y[m,n] = alpha[n] sum_k t[n,k] (R x[m,:])[k]             (ternary, rotated basis)
+//
+// One CTA owns 128 weight rows ("row group") at a time; the MMA is D[128 x BN] += A[128 x 16]
+// * B[16 x BN] with the weights as A and BN token columns as B ("swap-AB"), so every TMEM lane
+// is one output row and the per-block scale is a single scalar per lane.
+//
+// Warp roles (320 threads):
+//   warps 0-3  decode: thread t owns row t of the group (TMEM lane t). It reads its row's
+//              packed codes from shared memory, turns them into exact bf16 values (g/2, or t
+//              for ternary) in registers and writes them into tensor memory with tcgen05.st:
+//              A is consumed from TMEM, so the decoded weights never touch shared memory.
+//   warp 8     producer: bulk-copies the packed units of each 256-block (8 x 16-row units) and
+//              TMA-loads the activation tile (128-byte swizzle) into shared-memory rings.
+//   warp 9     allocates TMEM and issues the MMAs (one thread), committing to the barriers
+//              that recycle A buffers, activation stages and accumulators.
+//   warps 4-7  epilogue: per 256-block, load the fp32 partial from TMEM, multiply by 2*s[n,b]
+//              in fp32 and add it to a register running sum (ternary: once per item); at the
+//              end of an item, write y, or combine split-K pieces through the workspace (the
+//              last of the P pieces to arrive adds them in order p = 0..P-1 and writes y).
+// Every wait is bounded: a stuck pipeline records an error code and the CTA unwinds.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+#include "tc_common.cuh"
+#include "tc_kernels.cuh"
+#include "wr.h"
+
+namespace wr {
+namespace {
+
+using namespace tc;
+
+constexpr int kThreads = 320;
+constexpr int kSP = 4;  // packed-unit stages
+constexpr int kSX = 2;  // activation stages (per block)
+
+template <int FMT>
+struct Fmt {
+  static constexpr int kUnitK = FMT == WR_FMT_TERNARY ? 320 : 256;       // K per block
+  static constexpr int kUnitBytes = FMT == WR_FMT_Q3 ? 1536 : 1024;      // bytes per 16-row unit
+  static constexpr int kQuarterCols = FMT == WR_FMT_TERNARY ? 40 : 32;   // TMEM columns per quarter
+  static constexpr int kChunkCols = 2 * kQuarterCols;                   // A buffer (half block)
+  static constexpr int kChunkSteps = kChunkCols / 8;                    // K-steps of 16 per chunk
+};
+
+template <int FMT, int BN>
+struct Layout {
+  static constexpr int kXStage = BN * Fmt<FMT>::kUnitK * 2;              // bytes per activation stage
+  static constexpr int kXAtom = BN * 128;                                // bytes per 64-wide K atom
+  static constexpr int kPStage = 8 * Fmt<FMT>::kUnitBytes;
+  static constexpr int kXOff = 0;
+  static constexpr int kPOff = kXOff + kSX * kXStage;
+  static constexpr int kBarOff = kPOff + kSP * kPStage;
+  // + barriers and alignment slack; the 16-column variant is padded so that at most two CTAs
+  // share an SM (each holds 256 TMEM columns)
+  static constexpr int kSmemRaw = kBarOff + 256 + 1024;
+  static constexpr int kSmem = (BN == 16 && kSmemRaw < 80 * 1024) ? 80 * 1024 : kSmemRaw;
+  static constexpr int kACols = Fmt<FMT>::kChunkCols;
+  static constexpr int kDCol = 2 * kACols;
+  static constexpr int kTmemCols = (kDCol + 2 * BN) <= 256 ? 256 : 512;
+  static constexpr int kTok = FMT == WR_FMT_TERNARY ? BN / 2 : BN;      // tokens per tile
+};
+
+struct Bars {
+  uint64_t pk_full[kSP], pk_empty[kSP], x_full[kSX], x_empty[kSX];
+  uint64_t a_full[2], a_empty[2], d_full[2], d_empty[2];
+  uint32_t tmem_base;
+  int abort_flag;
+  int last_flag;
+};
+
+__device__ __forceinline__ void item_coords(const TcArgs& a, int it, int& rg, int& mt, int& p, int& b0, int& b1) {
+  p = it % a.P;
+  const int t = it / a.P;
+  mt = t % a.MT;
+  rg = t / a.MT;
+  b0 = (int)((int64_t)a.B * p / a.P);
+  b1 = (int)((int64_t)a.B * (p + 1) / a.P);
+}
+
+// ---------------------------------------------------------------- decode helpers (thread = row)
+
+// Q2: the row's quarter q of a unit is 16 bytes at lane chunk (32*half + 4*r0 + q).
+__device__ __forceinline__ void decode_q2_quarter(const uint8_t* unit, int r0, int half, int q, uint32_t v[32]) {
+  const uint4 c = *reinterpret_cast<const uint4*>(unit + (32 * half + 4 * r0 + q) * 16);
+  decode_q2_word(c.x, v + 0);
+  decode_q2_word(c.y, v + 8);
+  decode_q2_word(c.z, v + 16);
+  decode_q2_word(c.w, v + 24);
+}
+
+// Q3: lane l = 4*r0 + q holds 48 bytes in chunks (32c + l)*16; row half h uses lane bytes
+// 24h .. 24h+23, i.e. two 12-byte groups of 3 words.
+__device__ __forceinline__ void decode_q3_quarter(const uint8_t* unit, int r0, int half, int q, uint32_t v[32]) {
+  const int l = 4 * r0 + q;
+  uint32_t w[6];
+  if (half == 0) {
+    const uint4 c0 = *reinterpret_cast<const uint4*>(unit + l * 16);
+    const uint2 c1 = *reinterpret_cast<const uint2*>(unit + (32 + l) * 16);
+    w[0] = c0.x; w[1] = c0.y; w[2] = c0.z; w[3] = c0.w; w[4] = c1.x; w[5] = c1.y;
+  } else {
+    const uint2 c1 = *reinterpret_cast<const uint2*>(unit + (32 + l) * 16 + 8);
+    const uint4 c2 = *reinterpret_cast<const uint4*>(unit + (64 + l) * 16);
+    w[0] = c1.x; w[1] = c1.y; w[2] = c2.x; w[3] = c2.y; w[4] = c2.z; w[5] = c2.w;
+  }
+  decode_q3_group(w, v);
+  decode_q3_group(w + 3, v + 16);
+}
+
+// Ternary: a quarter is 16 bytes = 80 trits; byte pair (2b', 2b'+1) gives pair registers
+// 5b'..5b'+4, pair i = (trit i of byte 2b', trit i of byte 2b'+1).
+__device__ __forceinline__ void decode_t_quarter(const uint8_t* unit, int r0, int half, int q,
+                                                 const uint32_t* lut_lo, const uint32_t* lut_hi, uint32_t v[40]) {
+  const uint4 c = *reinterpret_cast<const uint4*>(unit + (32 * half + 4 * r0 + q) * 16);
+  const uint32_t wv[4] = {c.x, c.y, c.z, c.w};
+#pragma unroll
+  for (int w = 0; w < 4; ++w) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const uint32_t e = lut_lo[(wv[w] >> (16 * h)) & 0xFFu] | lut_hi[(wv[w] >> (16 * h + 8)) & 0xFFu];
+      decode_trit_pairs(e, v + 5 * (2 * w + h));
+    }
+  }
+}
+
+__device__ __forceinline__ uint32_t trit_entry(int v) {
+  const int slot[5] = {1, 3, 5, 9, 11};
+  uint32_t e = 0;
+  for (int d = 0; d < 5; ++d) {
+    e |= (uint32_t)(v % 3) << slot[d];
+    v /= 3;
+  }
+  return e;
+}
+
+// ---------------------------------------------------------------- the kernel
+
+template <int FMT, int BN>
+__global__ void __launch_bounds__(kThreads, BN == 16 ? 2 : 1) tc_kernel(const TcArgs a, const __grid_constant__ CUtensorMap xmap) {
+  using F = Fmt<FMT>;
+  using Ly = Layout<FMT, BN>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* xs = smem + Ly::kXOff;
+  uint8_t* ps = smem + Ly::kPOff;
+  Bars* bars = reinterpret_cast<Bars*>(smem + Ly::kBarOff);
+  __shared__ uint32_t lut_lo[FMT == WR_FMT_TERNARY ? 256 : 1], lut_hi[FMT == WR_FMT_TERNARY ? 256 : 1];
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  volatile int* abort_flag = &bars->abort_flag;
+
+  if (FMT == WR_FMT_TERNARY) {
+    for (int i = threadIdx.x; i < 256; i += kThreads) {
+      const uint32_t e = i < 243 ? trit_entry(i) : 0u;
+      lut_lo[i] = e;
+      lut_hi[i] = e << 16;
+    }
+  }
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kSP; ++i) {
+      mbar_init(&bars->pk_full[i], 1);
+      mbar_init(&bars->pk_empty[i], 4);
+    }
+    for (int i = 0; i < kSX; ++i) {
+      mbar_init(&bars->x_full[i], 1);
+      mbar_init(&bars->x_empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bars->a_full[i], 4);
+      mbar_init(&bars->a_empty[i], 1);
+      mbar_init(&bars->d_full[i], 1);
+      mbar_init(&bars->d_empty[i], 4);
+    }
+    bars->abort_flag = 0;
+    bars->last_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 9) tmem_alloc(&bars->tmem_base, Ly::kTmemCols);
+  fence_before_sync();
+  __syncthreads();
+  fence_after_sync();
+  const uint32_t tmem = bars->tmem_base;
+
+  if (warp == 8) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      prefetch_tensormap(&xmap);
+      uint32_t gb = 0;
+      const int tiles = (a.N + 15) / 16;
+      for (int it = blockIdx.x; it < a.items && !*abort_flag; it += gridDim.x) {
+        int rg, mt, p, b0, b1;
+        item_coords(a, it, rg, mt, p, b0, b1);
+        for (int b = b0; b < b1; ++b, ++gb) {
+          const int sx = gb % kSX;
+          if (!mbar_wait(&bars->x_empty[sx], ((gb / kSX) & 1) ^ 1, abort_flag, a.err, 101)) break;
+          mbar_arrive_expect_tx(&bars->x_full[sx], Ly::kXStage);
+#pragma unroll
+          for (int at = 0; at < F::kUnitK / 64; ++at) {
+            uint8_t* dst = xs + sx * Ly::kXStage + at * Ly::kXAtom;
+            const int k = b * F::kUnitK + 64 * at;
+            if (FMT == WR_FMT_TERNARY) {
+              // two 8-token boxes: hi plane into rows 0..7, lo plane into rows 8..15
+              asm volatile(
+                  "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, "
+                  "%3, %4}], [%5];" ::"r"(smem_u32(dst)),
+                  "l"(&xmap), "r"(k), "r"(mt * 8), "r"(0), "r"(smem_u32(&bars->x_full[sx]))
+                  : "memory");
+              asm volatile(
+                  "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, "
+                  "%3, %4}], [%5];" ::"r"(smem_u32(dst + 8 * 128)),
+                  "l"(&xmap), "r"(k), "r"(mt * 8), "r"(1), "r"(smem_u32(&bars->x_full[sx]))
+                  : "memory");
+            } else {
+              tma_load_2d(dst, &xmap, k, mt * BN, &bars->x_full[sx]);
+            }
+          }
+          const int sp = gb % kSP;
+          if (!mbar_wait(&bars->pk_empty[sp], ((gb / kSP) & 1) ^ 1, abort_flag, a.err, 102)) break;
+          const int ntile = min(8, tiles - rg * 8);
+          mbar_arrive_expect_tx(&bars->pk_full[sp], ntile * F::kUnitBytes);
+          for (int i = 0; i < ntile; ++i) {
+            const uint8_t* src = a.packed + ((int64_t)(rg * 8 + i) * a.B + b) * F::kUnitBytes;
+            bulk_load(ps + sp * Ly::kPStage + i * F::kUnitBytes, src, F::kUnitBytes, &bars->pk_full[sp]);
+          }
+        }
+      }
+    }
+  } else if (warp == 9) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_m128(BN);
+      uint32_t gb = 0, gc = 0, gi = 0;
+      for (int it = blockIdx.x; it < a.items && !*abort_flag; it += gridDim.x, ++gi) {
+        int rg, mt, p, b0, b1;
+        item_coords(a, it, rg, mt, p, b0, b1);
+        bool ok = true;
+        uint32_t dbuf = 0;
+        if (FMT == WR_FMT_TERNARY) {
+          dbuf = gi & 1;
+          ok = mbar_wait(&bars->d_empty[dbuf], ((gi >> 1) & 1) ^ 1, abort_flag, a.err, 201);
+        }
+        for (int b = b0; b < b1 && ok; ++b, ++gb) {
+          if (FMT != WR_FMT_TERNARY) {
+            dbuf = gb & 1;
+            if (!(ok = mbar_wait(&bars->d_empty[dbuf], ((gb >> 1) & 1) ^ 1, abort_flag, a.err, 202))) break;
+          }
+          const int sx = gb % kSX;
+          if (!(ok = mbar_wait(&bars->x_full[sx], (gb / kSX) & 1, abort_flag, a.err, 203))) break;
+          const uint8_t* xst = xs + sx * Ly::kXStage;
+          for (int c = 0; c < 2; ++c, ++gc) {
+            const int sa = gc & 1;
+            if (!(ok = mbar_wait(&bars->a_full[sa], (gc >> 1) & 1, abort_flag, a.err, 204))) break;
+            fence_after_sync();
+#pragma unroll
+            for (int j = 0; j < F::kChunkSteps; ++j) {
+              const int kk = c * (F::kUnitK / 2) + 16 * j;     // K offset inside the block
+              const uint64_t bdesc = smem_desc_sw128(xst + (kk / 64) * Ly::kXAtom + (kk % 64) * 2);
+              const uint32_t acc = (FMT == WR_FMT_TERNARY) ? (uint32_t)(b != b0 || c != 0 || j != 0)
+                                                           : (uint32_t)(c != 0 || j != 0);
+              mma_ts(tmem + Ly::kDCol + dbuf * BN, tmem + sa * Ly::kACols + 8 * j, bdesc, idesc, acc);
+            }
+            mma_commit(&bars->a_empty[sa]);
+          }
+          if (!ok) break;
+          mma_commit(&bars->x_empty[sx]);
+          if (FMT != WR_FMT_TERNARY) mma_commit(&bars->d_full[dbuf]);
+        }
+        if (FMT == WR_FMT_TERNARY && ok) mma_commit(&bars->d_full[dbuf]);
+      }
+    }
+  } else if (warp < 4) {
+    // ------------------------------------------------------------ decode (thread = row)
+    const int t = threadIdx.x;
+    const int tile = t >> 4, r = t & 15, r0 = r & 7, half = r >> 3;
+    const uint32_t lane_addr = (uint32_t)(32 * warp) << 16;
+    uint32_t gb = 0, gc = 0;
+    for (int it = blockIdx.x; it < a.items && !*abort_flag; it += gridDim.x) {
+      int rg, mt, p, b0, b1;
+      item_coords(a, it, rg, mt, p, b0, b1);
+      bool ok = true;
+      for (int b = b0; b < b1; ++b, ++gb) {
+        const int sp = gb % kSP;
+        if (!(ok = mbar_wait(&bars->pk_full[sp], (gb / kSP) & 1, abort_flag, a.err, 301))) break;
+        const uint8_t* unit = ps + sp * Ly::kPStage + tile * F::kUnitBytes;
+        for (int c = 0; c < 2; ++c, ++gc) {
+          const int sa = gc & 1;
+          if (!(ok = mbar_wait(&bars->a_empty[sa], ((gc >> 1) & 1) ^ 1, abort_flag, a.err, 302))) break;
+          fence_after_sync();
+#pragma unroll
+          for (int qq = 0; qq < 2; ++qq) {
+            const int q = 2 * c + qq;
+            const uint32_t col = tmem + lane_addr + sa * Ly::kACols + qq * F::kQuarterCols;
+            if (FMT == WR_FMT_TERNARY) {
+              uint32_t v[40];
+              decode_t_quarter(unit, r0, half, q, lut_lo, lut_hi, v);
+              tmem_st32(col, v);
+              tmem_st8(col + 32, v + 32);
+            } else {
+              uint32_t v[32];
+              if (FMT == WR_FMT_Q2) decode_q2_quarter(unit, r0, half, q, v);
+              else decode_q3_quarter(unit, r0, half, q, v);
+              tmem_st32(col, v);
+            }
+          }
+          tmem_wait_st();
+          fence_before_sync();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bars->a_full[sa]);
+        }
+        if (!ok) break;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->pk_empty[sp]);
+      }
+      if (!ok) break;
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue (warps 4-7, thread = row)
+    constexpr int TOK = Ly::kTok;
+    const int t = threadIdx.x - 128;
+    const uint32_t lane_addr = (uint32_t)(32 * (warp - 4)) << 16;
+    uint32_t gb = 0, gi = 0;
+    for (int it = blockIdx.x; it < a.items && !*abort_flag; it += gridDim.x, ++gi) {
+      int rg, mt, p, b0, b1;
+      item_coords(a, it, rg, mt, p, b0, b1);
+      const int n = rg * 128 + t;
+      float acc[TOK];
+#pragma unroll
+      for (int i = 0; i < TOK; ++i) acc[i] = 0.f;
+      bool ok = true;
+      if (FMT == WR_FMT_TERNARY) {
+        const uint32_t dbuf = gi & 1;
+        gb += b1 - b0;
+        ok = mbar_wait(&bars->d_full[dbuf], (gi >> 1) & 1, abort_flag, a.err, 401);
+        if (ok) {
+          fence_after_sync();
+          float d[16];
+          tmem_ld16(tmem + lane_addr + Ly::kDCol + dbuf * BN, d);
+          tmem_wait_ld();
+          fence_before_sync();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bars->d_empty[dbuf]);
+#pragma unroll
+          for (int i = 0; i < TOK; ++i) acc[i] = d[i] + d[i + 8];
+        }
+      } else {
+        for (int b = b0; b < b1; ++b, ++gb) {
+          const uint32_t dbuf = gb & 1;
+          const float s2 = n < a.N ? 2.f * half_bits_to_float(__ldg(a.scales + (int64_t)n * a.B + b)) : 0.f;
+          if (!(ok = mbar_wait(&bars->d_full[dbuf], (gb >> 1) & 1, abort_flag, a.err, 402))) break;
+          fence_after_sync();
+#pragma unroll
+          for (int c0 = 0; c0 < BN; c0 += 16) {
+            float d[16];
+            tmem_ld16(tmem + lane_addr + Ly::kDCol + dbuf * BN + c0, d);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 16; ++i) acc[c0 + i] = fmaf(s2, d[i], acc[c0 + i]);
+          }
+          fence_before_sync();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bars->d_empty[dbuf]);
+        }
+      }
+      if (!ok) break;
+      // ---- output: direct store, or split-K combine through the workspace
+      const int m0 = mt * TOK;
+      const int mcount = min(TOK, a.M - m0);
+      const float rs = (FMT == WR_FMT_TERNARY && n < a.N) ? half_bits_to_float(__ldg(a.alpha + n)) : 1.f;
+      if (a.P == 1) {
+        if (n < a.N) {
+#pragma unroll
+          for (int i = 0; i < TOK; ++i)
+            if (i < mcount) a.y[(int64_t)(m0 + i) * a.N + n] = rs * acc[i];
+        }
+      } else {
+        const int tileid = rg * a.MT + mt;
+        float* part = a.partial + ((int64_t)tileid * a.P + p) * (TOK * 128);
+#pragma unroll
+        for (int i = 0; i < TOK; ++i)
+          if (i < mcount) part[i * 128 + t] = acc[i];
+        __threadfence();
+        named_bar_sync(1, 128);
+        if (t == 0) bars->last_flag = (atomicAdd(a.counter + tileid, 1) == a.P - 1);
+        named_bar_sync(1, 128);
+        const int last = bars->last_flag;
+        if (last) {
+          __threadfence();
+          float sum[TOK];
+#pragma unroll
+          for (int i = 0; i < TOK; ++i) sum[i] = 0.f;
+          for (int pp = 0; pp < a.P; ++pp) {
+            const float* src = a.partial + ((int64_t)tileid * a.P + pp) * (TOK * 128);
+#pragma unroll
+            for (int i = 0; i < TOK; ++i)
+              if (i < mcount) sum[i] += __ldcg(src + i * 128 + t);
+          }
+          if (n < a.N) {
+#pragma unroll
+            for (int i = 0; i < TOK; ++i)
+              if (i < mcount) a.y[(int64_t)(m0 + i) * a.N + n] = rs * sum[i];
+          }
+          if (t == 0) a.counter[tileid] = 0;
+        }
+        named_bar_sync(1, 128);
+      }
+    }
+  }
+
+  fence_before_sync();
+  __syncthreads();
+  fence_after_sync();
+  if (warp == 9) tmem_dealloc(tmem, Ly::kTmemCols);
+}
+
+// ---------------------------------------------------------------- host side
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+template <int FMT, int BN>
+cudaError_t launch_tc(const TcArgs& a, const void* x_act, int64_t x_rows, int64_t x_k, int grid, cudaStream_t stream) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return cudaErrorNotSupported;
+  CUtensorMap map;
+  CUresult r;
+  if (FMT == WR_FMT_TERNARY) {
+    // R x planes: [2][M][Kp] bf16 -> dims (Kp, M, 2), box (64, 8, 1)
+    const cuuint64_t dims[3] = {(cuuint64_t)x_k, (cuuint64_t)x_rows, 2};
+    const cuuint64_t strides[2] = {(cuuint64_t)x_k * 2, (cuuint64_t)x_k * 2 * x_rows};
+    const cuuint32_t box[3] = {64, 8, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    r = enc(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(x_act), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  } else {
+    const cuuint64_t dims[2] = {(cuuint64_t)x_k, (cuuint64_t)x_rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)x_k * 2};
+    const cuuint32_t box[2] = {64, (cuuint32_t)BN};
+    const cuuint32_t estr[2] = {1, 1};
+    r = enc(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(x_act), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  }
+  if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+  using Ly = Layout<FMT, BN>;
+  auto kern = tc_kernel<FMT, BN>;
+  static bool attr_set = false;
+  if (!attr_set) {
+    const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Ly::kSmem);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  kern<<<grid, kThreads, Ly::kSmem, stream>>>(a, map);
+  return cudaGetLastError();
+}
+
+// R x for the ternary path: one warp per (token, 128-block). x' = (1/sqrt(128)) H (d * x) in
+// fp32, split into hi = bf16(x') and lo = bf16(x' - hi), written as two planes [2][M][Kp] in
+// the K order of the decoded A columns: position 80q + 2P + h of a 320-trit unit holds trit
+// 80q + 5*(2*(P/5) + h) + P%5 (pair P of byte pair P/5; h selects the byte). Pad trits get 0.
+__global__ void rotate_x_kernel(const uint16_t* __restrict__ x, const uint32_t* __restrict__ signs,
+                                uint16_t* __restrict__ xr, int M, int K, int64_t Kp) {
+  const int lane = threadIdx.x & 31;
+  const int64_t item = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int64_t nblk = (Kp + 127) / 128;
+  if (item >= (int64_t)M * nblk) return;
+  const int m = (int)(item / nblk);
+  const int64_t k0 = (item % nblk) * 128;
+  float v[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int64_t k = k0 + 4 * lane + i;
+    float xv = 0.f;
+    if (k < K) {
+      xv = __bfloat162float(__ushort_as_bfloat16(x[(int64_t)m * K + k]));
+      if ((signs[k >> 5] >> (k & 31)) & 1u) xv = -xv;
+    }
+    v[i] = xv;
+  }
+  float t0 = v[0] + v[1], t1 = v[0] - v[1], t2 = v[2] + v[3], t3 = v[2] - v[3];
+  v[0] = t0 + t2; v[2] = t0 - t2; v[1] = t1 + t3; v[3] = t1 - t3;
+#pragma unroll
+  for (int s = 1; s < 32; s <<= 1) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float o = __shfl_xor_sync(0xffffffffu, v[i], s);
+      v[i] = (lane & s) ? o - v[i] : v[i] + o;
+    }
+  }
+  const float inv = 0.08838834764831845f;  // 1/sqrt(128)
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int64_t k = k0 + 4 * lane + i;
+    if (k >= Kp) continue;
+    const float xp = v[i] * inv;
+    const __nv_bfloat16 hi = __float2bfloat16_rn(xp);
+    const __nv_bfloat16 lo = __float2bfloat16_rn(xp - __bfloat162float(hi));
+    const int64_t u = k / 320;
+    const int kk = (int)(k % 320), q = kk / 80, i80 = kk % 80, beta = i80 / 5, dig = i80 % 5;
+    const int P = 5 * (beta >> 1) + dig;
+    const int64_t pos = u * 320 + 80 * q + 2 * P + (beta & 1);
+    xr[(int64_t)m * Kp + pos] = __bfloat16_as_ushort(hi);
+    xr[((int64_t)M + m) * Kp + pos] = __bfloat16_as_ushort(lo);
+  }
+}
+
+}  // namespace
+
+int tc_tmem_cols(int fmt, int bn) {
+  if (fmt == WR_FMT_TERNARY) return Layout<WR_FMT_TERNARY, 16>::kTmemCols;
+  if (bn == 16) return Layout<WR_FMT_Q2, 16>::kTmemCols;
+  return Layout<WR_FMT_Q2, 128>::kTmemCols;
+}
+
+cudaError_t launch_tc_kernel(int fmt, int bn, const TcArgs& a, const void* x_act, int64_t x_rows, int64_t x_k,
+                             int grid, cudaStream_t stream) {
+  if (fmt == WR_FMT_Q2 && bn == 16) return launch_tc<WR_FMT_Q2, 16>(a, x_act, x_rows, x_k, grid, stream);
+  if (fmt == WR_FMT_Q3 && bn == 16) return launch_tc<WR_FMT_Q3, 16>(a, x_act, x_rows, x_k, grid, stream);
+  if (fmt == WR_FMT_Q2 && bn == 128) return launch_tc<WR_FMT_Q2, 128>(a, x_act, x_rows, x_k, grid, stream);
+  if (fmt == WR_FMT_Q3 && bn == 128) return launch_tc<WR_FMT_Q3, 128>(a, x_act, x_rows, x_k, grid, stream);
+  if (fmt == WR_FMT_TERNARY && bn == 16) return launch_tc<WR_FMT_TERNARY, 16>(a, x_act, x_rows, x_k, grid, stream);
+  return cudaErrorNotSupported;
+}
+
+cudaError_t launch_rotate_x(const uint16_t* x, const uint32_t* signs, uint16_t* xr, int M, int K, int64_t Kp,
+                            cudaStream_t stream) {
+  const int64_t items = (int64_t)M * ((Kp + 127) / 128);
+  const int warps = 8;
+  const int64_t ctas = (items + warps - 1) / warps;
+  rotate_x_kernel<<<(unsigned)ctas, warps * 32, 0, stream>>>(x, signs, xr, M, K, Kp);
+  return cudaGetLastError();
+}
+
+}  // namespace wr

@@ -1,0 +1,57 @@
+// Launch interface of the tcgen05 GEMV/GEMM kernels (internal to libwr).
+#pragma once
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace wr {
+
+struct TcArgs {
+  const uint8_t* packed;     // packed units, tile-major
+  const uint16_t* scales;    // fp16 [N, K/256] (Q2/Q3)
+  const uint16_t* alpha;     // fp16 [N] (ternary)
+  float* y;                  // fp32 [M, N]
+  float* partial;            // split-K partials [RG*MT][P][TOK][128]
+  int* counter;              // [RG*MT] arrival counters, zero between calls
+  int* err;                  // device error word (bounded waits)
+  int M, N, K;
+  int B;                     // 256-code (or 320-trit) blocks per row
+  int RG;                    // 128-row groups
+  int MT;                    // token tiles
+  int P;                     // K splits per (row group, token tile)
+  int items;                 // RG * MT * P
+};
+
+// Batched decode GEMV (M <= 16): one launch over up to kMaxDecodeProblems independent problems.
+constexpr int kMaxDecodeProblems = 256;
+
+struct DecProblem {
+  const uint16_t* x;         // bf16 [M, K]; ternary: R x as [2][M][Kp] planes (hi, lo)
+  const uint8_t* packed;     // packed units, tile-major
+  const uint16_t* scales;    // fp16 [N, K/256] (Q2/Q3) or alpha [N] (ternary)
+  float* y;                  // fp32 [M, N]
+  int N, K, Kp;              // Kp: padded K of the ternary planes
+  int B, RG, P, bits;        // blocks per row, 128-row groups, K splits, 2/3 (ternary: 1)
+  int item_base;             // first work item of this problem
+  int counter_base;          // first arrival counter of this problem
+  int64_t partial_base;      // first partial float of this problem
+};
+
+struct DecArgs {
+  int count, M, items, pad;
+  float* partial;
+  int* counter;
+  int* err;
+  DecProblem prob[kMaxDecodeProblems];
+};
+
+cudaError_t launch_decode(bool ternary, const DecArgs& a, int grid, cudaStream_t stream);
+
+int tc_tmem_cols(int fmt, int bn);
+cudaError_t launch_tc_kernel(int fmt, int bn, const TcArgs& a, const void* x_act, int64_t x_rows, int64_t x_k,
+                             int grid, cudaStream_t stream);
+cudaError_t launch_rotate_x(const uint16_t* x, const uint32_t* signs, uint16_t* xr, int M, int K, int64_t Kp,
+                            cudaStream_t stream);
+cudaError_t launch_unpack_bf16(int fmt, const uint8_t* packed, const uint16_t* scales, int N, int K, int units,
+                               uint16_t* w, cudaStream_t stream);
+
+}  // namespace wr

@@ -10,7 +10,7 @@
 #include <cuda_runtime.h>
 
 #include "common.cuh"
-#include "gemv.cuh"
+#include "tc_kernels.cuh"
 #include "wr.h"
 
 namespace wr {

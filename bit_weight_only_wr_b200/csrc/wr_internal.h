@@ -10,9 +10,5 @@ bool packed_geometry(int fmt, int64_t N, int64_t K, int64_t* unit_bytes, int64_t
 uint16_t host_double_to_half(double v);
 double host_half_to_double(uint16_t h);
 
-// Upper bound on GEMV warps: every workspace size is computed with it, so sizes do not
-// depend on the device the call later runs on.
-constexpr int kGemvMaxWarps = 2560;
-constexpr int kGemvWarpsPerSM = 16;
 
 }  // namespace wr

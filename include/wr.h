@@ -132,6 +132,27 @@ wr_status wr_gemv(int64_t M, int64_t N, int64_t K, const uint16_t* x, const void
                   const uint16_t* scales, int bits, int group, float* y, void* workspace,
                   size_t workspace_bytes, void* stream);
 
+/* One problem of a batched decode GEMV (all fields are read on the host during the call). */
+typedef struct {
+  const uint16_t* x;       /* bf16 [M, K] activations (device) */
+  const void* packed;      /* packed codes (device), format Q2 or Q3 as given by bits */
+  const uint16_t* scales;  /* fp16 [N, K/256] block scales (device) */
+  float* y;                /* fp32 [M, N] output (device, overwritten) */
+  int64_t N, K;            /* K % 256 == 0 */
+  int32_t bits;            /* 2 or 3 */
+  int32_t reserved;        /* must be 0 */
+} wr_gemv_problem;
+
+/* Batched decode GEMV: `count` independent problems (2- and 3-bit may be mixed) sharing one
+ * token count 1 <= M <= 8, computed by one persistent launch that streams all their packed
+ * weights back to back, so the fixed latency of a small GEMV is paid once per batch instead
+ * of once per problem (the 252 linears of a 36-layer decoder body fit in one batch of at most
+ * 256 problems; larger batches are split into several launches). Each problem computes what
+ * wr_gemv computes. problems_host is a host array read during the call. */
+size_t wr_gemv_batched_workspace_bytes(int64_t M, int32_t count, const wr_gemv_problem* problems_host);
+wr_status wr_gemv_batched(int64_t M, int32_t count, const wr_gemv_problem* problems_host, void* workspace,
+                          size_t workspace_bytes, void* stream);
+
 /* Prefill GEMM, any M >= 1 (Q2/Q3, group 256): packed tiles are staged in shared memory,
  * decoded to exact bf16 grid integers and contracted by tcgen05 MMAs into TMEM, one fp32
  * partial per 256-block, scaled in fp32 by the epilogue. */

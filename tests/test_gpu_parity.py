@@ -84,9 +84,14 @@ def test_gemv_layer_shapes(wr, bits, N, K, M):
     y, ws = _run_gemv(wr, bits, x, packed, s_d, N, K)
     ref, B = o.gemm_codes(x, codes, scales, bits)
     check_close(y, ref, B)
-    # the arrival counters are back to zero after the call
-    tiles = (N + 15) // 16
-    assert int(ws[: 4 * tiles].view(dtype=torch_mod().int32).abs().sum()) == 0
+    # the same workspace serves further calls (its counters were left at zero)
+    torch = torch_mod()
+    y2 = torch.empty_like(torch.from_numpy(y)).cuda()
+    nb = wr.wr_gemv_workspace_bytes(M, N, K, bits)
+    for _ in range(2):
+        wr.wr_gemv(M, N, K, dev(x), packed, s_d, bits, y2, ws, nb)
+    torch.cuda.synchronize()
+    assert np.array_equal(y2.cpu().numpy().view(np.uint32), y.view(np.uint32))
 
 
 def test_gemv_deterministic(wr):
@@ -114,7 +119,7 @@ def test_gemv_zero_cases(wr):
 
 # ---------------------------------------------------------------- ternary
 
-@pytest.mark.parametrize("M", [1, 2, 4, 5, 8])
+@pytest.mark.parametrize("M", [1, 2, 4, 5, 8, 9, 20])
 @pytest.mark.parametrize("N,K", [(40, 640), (64, 4096)])
 def test_ternary_gemv(wr, M, N, K):
     torch = torch_mod()
@@ -142,3 +147,99 @@ def test_ternary_gemv_layer_shapes(wr, N, K):
     torch.cuda.synchronize()
     ref, B = o.gemm_ternary(x, codes, alpha, signs)
     check_close(y.cpu().numpy(), ref, B)
+
+
+# ---------------------------------------------------------------- prefill GEMM (tcgen05)
+
+def _run_gemm(wr, bits, x_bits, packed, scales, N, K):
+    torch = torch_mod()
+    M = x_bits.shape[0]
+    y = torch.full((M, N), float("nan"), dtype=torch.float32, device="cuda")
+    nb = wr.wr_gemm_workspace_bytes(M, N, K, bits)
+    ws = _zeros_ws(nb)
+    wr.wr_gemm(M, N, K, dev(x_bits), packed, scales, bits, y, ws, nb)
+    torch.cuda.synchronize()
+    return y.cpu().numpy()
+
+
+@pytest.mark.parametrize("bits", [2, 3])
+@pytest.mark.parametrize("M", [9, 16, 17, 100, 128, 129, 300])
+def test_gemm_ragged(wr, bits, M):
+    N, K = 200, 1024
+    codes, scales, packed, s_d = q_case(wr, bits, N, K, seed=13 * M + bits)
+    x = wr_synth.activations_bf16(600 + M, M, K)
+    y = _run_gemm(wr, bits, x, packed, s_d, N, K)
+    ref, B = o.gemm_codes(x, codes, scales, bits)
+    check_close(y, ref, B)
+
+
+@pytest.mark.parametrize("bits,N,K,M", [(2, 9728, 2560, 512), (3, 2560, 9728, 512), (3, 9728, 2560, 16)])
+def test_gemm_layer_shapes(wr, bits, N, K, M):
+    codes, scales, packed, s_d = q_case(wr, bits, N, K, seed=N + K + M + bits)
+    x = wr_synth.activations_bf16(700 + M, M, K)
+    y = _run_gemm(wr, bits, x, packed, s_d, N, K)
+    rows = np.random.default_rng(M).choice(N, 256, replace=False)
+    ref, B = o.gemm_codes(x, codes[rows], scales[rows], bits)
+    check_close(y[:, rows], ref, B)
+
+
+@pytest.mark.parametrize("bits,N,K", [(2, 9728, 2560), (3, 2560, 9728)])
+def test_gemm_full_size_sampled(wr, bits, N, K):
+    """M = 4096 (the largest prefill size): every column of y for 64 sampled rows."""
+    M = 4096
+    codes, scales, packed, s_d = q_case(wr, bits, N, K, seed=N * 7 + K)
+    x = wr_synth.activations_bf16(800, M, K)
+    y = _run_gemm(wr, bits, x, packed, s_d, N, K)
+    rows = np.random.default_rng(1).choice(N, 64, replace=False)
+    ref, B = o.gemm_codes(x, codes[rows], scales[rows], bits)
+    check_close(y[:, rows], ref, B)
+
+
+def test_no_device_error_after_calls(wr):
+    assert wr.wr_get_device_error() == 0
+
+
+# ---------------------------------------------------------------- batched decode GEMV
+
+@pytest.mark.parametrize("M", [1, 3, 8])
+def test_gemv_batched_layer(wr, M):
+    """The 7 linears of one Qwen3-4B layer (mixed 2/3-bit) in one batched launch, twice."""
+    torch = torch_mod()
+    cases, problems, ys = [], [], []
+    for idx, (name, K, N, bits) in enumerate(wr_synth.QWEN3_4B_LAYER):
+        codes, scales, packed, s_d = q_case(wr, bits, N, K, seed=wr_synth.module_seed(0, idx))
+        x = wr_synth.activations_bf16(900 + idx, M, K)
+        xd = dev(x)
+        y = torch.full((M, N), float("nan"), dtype=torch.float32, device="cuda")
+        cases.append((codes, scales, bits, x, xd, packed, s_d))
+        ys.append(y)
+        problems.append((xd, packed, s_d, y, N, K, bits))
+    nb = wr.wr_gemv_batched_workspace_bytes(M, problems)
+    ws = _zeros_ws(nb)
+    for rep in range(2):
+        wr.wr_gemv_batched(M, problems, ws, nb)
+        torch.cuda.synchronize()
+        for (codes, scales, bits, x, *_), y in zip(cases, ys):
+            ref, B = o.gemm_codes(x, codes, scales, bits)
+            check_close(y.cpu().numpy(), ref, B)
+
+
+def test_gemv_batched_ragged_mixed(wr):
+    torch = torch_mod()
+    M = 5
+    shapes = [(40, 512, 2), (300, 768, 3), (16, 256, 2), (129, 2560, 3), (1, 256, 3)]
+    cases, problems = [], []
+    for i, (N, K, bits) in enumerate(shapes):
+        codes, scales, packed, s_d = q_case(wr, bits, N, K, seed=1000 + i)
+        x = wr_synth.activations_bf16(1100 + i, M, K)
+        xd = dev(x)
+        y = torch.full((M, N), float("nan"), dtype=torch.float32, device="cuda")
+        cases.append((codes, scales, bits, x, y))
+        problems.append((xd, packed, s_d, y, N, K, bits))
+    nb = wr.wr_gemv_batched_workspace_bytes(M, problems)
+    ws = _zeros_ws(nb)
+    wr.wr_gemv_batched(M, problems, ws, nb)
+    torch.cuda.synchronize()
+    for codes, scales, bits, x, y in cases:
+        ref, B = o.gemm_codes(x, codes, scales, bits)
+        check_close(y.cpu().numpy(), ref, B)
