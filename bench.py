@@ -41,7 +41,7 @@ def parse_args():
     p.add_argument("--impl", choices=["wr", "reference"], default="wr")
     p.add_argument("--layers", type=int, default=36)
     p.add_argument("--no-extras", action="store_true", help="headline body only")
-    p.add_argument("--cpu-seconds", type=float, default=12.0, help="oracle sample budget")
+    p.add_argument("--cpu-seconds", type=float, default=12.0, help="oracle sample budget (0: no CPU baseline)")
     return p.parse_args()
 
 
@@ -341,7 +341,7 @@ def main():
             "note": "the M=1 body step is one launch of the batched decode GEMV: algorithmic bytes per "
                     "launch / event-timed duration per launch"}
     cb = None
-    if rank == 0 and world == 1:
+    if rank == 0 and world == 1 and args.cpu_seconds > 0:
         try:
             cb = cpu_oracle_sample(args.cpu_seconds)
         except Exception as e:  # noqa: BLE001
