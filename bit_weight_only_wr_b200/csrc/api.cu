@@ -59,10 +59,12 @@ constexpr int kDecodeTokens = 16;
 
 // ---- decode kernel (M <= 16): work items (problem, 128-row group, block range) and workspace
 // [counters: one int per row group of every problem][split-K partials of problems with P > 1]
-// [ternary only: R x as two bf16 planes of M x Kp].
+// [prepared activation tiles: one per block of every problem].
 struct DecodePlan {
   wr::DecArgs args;
-  size_t counter_off = 0, partial_off = 0, xr_off = 0, total = 0;
+  int total_blocks = 0;
+  size_t counter_off = 0, partial_off = 0, xt_off = 0, total = 0;
+  int64_t xt_rel[wr::kMaxDecodeProblems];
 };
 
 struct ProblemShape {
@@ -90,9 +92,8 @@ void plan_decode(int64_t M, int count, const ProblemShape* shapes, DecodePlan* d
   }
   const int64_t target_items = std::max<int64_t>(2 * kPlanSMs, (total_blocks + 7) / 8);
   const double bpi = (double)total_blocks / (double)target_items;
-  int items = 0, counters = 0;
-  int64_t partials = 0;
-  size_t xr_bytes = 0;
+  int items = 0, counters = 0, blocks = 0;
+  int64_t partials = 0, xt_bytes = 0;
   for (int i = 0; i < count; ++i) {
     wr::DecProblem& pr = a.prob[i];
     int P = (int)std::lround((double)pr.B / bpi);
@@ -100,23 +101,36 @@ void plan_decode(int64_t M, int count, const ProblemShape* shapes, DecodePlan* d
     pr.item_base = items;
     pr.counter_base = counters;
     pr.partial_base = partials;
+    pr.xblk_base = blocks;
     items += pr.RG * pr.P;
     counters += pr.RG;
+    blocks += pr.B;
     if (pr.P > 1) partials += (int64_t)pr.RG * pr.P * M * 128;
-    if (shapes[i].fmt == WR_FMT_TERNARY) xr_bytes += align256((size_t)(2 * M) * (size_t)pr.Kp * 2);
+    dp->xt_rel[i] = xt_bytes;
+    xt_bytes += (int64_t)pr.B * wr::xtile_bytes(shapes[i].fmt == WR_FMT_TERNARY, (int)M);
   }
   a.items = items;
+  dp->total_blocks = blocks;
   dp->counter_off = 0;
   dp->partial_off = align256((size_t)counters * sizeof(int));
-  dp->xr_off = dp->partial_off + align256((size_t)partials * sizeof(float));
-  dp->total = dp->xr_off + xr_bytes;
+  dp->xt_off = dp->partial_off + align256((size_t)partials * sizeof(float));
+  dp->total = dp->xt_off + align256((size_t)xt_bytes);
 }
 
-wr_status run_decode(DecodePlan& dp, bool ternary, void* workspace, cudaStream_t stream) {
+// Fills the workspace pointers of a plan (the activation tiles of problem i start at
+// xt_off + xt_rel[i]).
+void bind_workspace(DecodePlan& dp, void* workspace) {
   uint8_t* wsb = static_cast<uint8_t*>(workspace);
   dp.args.counter = reinterpret_cast<int*>(wsb + dp.counter_off);
   dp.args.partial = reinterpret_cast<float*>(wsb + dp.partial_off);
+  for (int i = 0; i < dp.args.count; ++i) dp.args.prob[i].xt = wsb + dp.xt_off + dp.xt_rel[i];
   dp.args.err = device_error_word();
+}
+
+// Q2/Q3: preparation pass, then the decode kernel; ternary: the rotation pass has already
+// written the tiles.
+wr_status run_decode(DecodePlan& dp, bool ternary, cudaStream_t stream) {
+  if (!ternary && wr::launch_prep_x(dp.args, dp.total_blocks, stream) != cudaSuccess) return WR_ERR_CUDA;
   const int grid = (int)std::min<int64_t>(dp.args.items, (int64_t)sm_count() * 2);
   return wr::launch_decode(ternary, dp.args, grid, stream) == cudaSuccess ? WR_OK : WR_ERR_CUDA;
 }
@@ -186,7 +200,8 @@ wr_status run_q(int bits, int64_t M, int64_t N, int64_t K, const uint16_t* x, co
     dp.args.prob[0].packed = static_cast<const uint8_t*>(packed);
     dp.args.prob[0].scales = scales;
     dp.args.prob[0].y = y;
-    return run_decode(dp, false, workspace, stream);
+    bind_workspace(dp, workspace);
+    return run_decode(dp, false, stream);
   }
   return run_gemm(bits, (int)M, (int)N, (int)K, x, static_cast<const uint8_t*>(packed), scales, y, workspace, stream);
 }
@@ -206,14 +221,15 @@ wr_status run_t(int64_t M, int64_t N, int64_t K, const uint16_t* x, const void* 
     const int mm = (int)std::min<int64_t>(8, M - m0);
     const ProblemShape sh{N, K, WR_FMT_TERNARY};
     plan_decode(mm, 1, &sh, &dp);
-    uint16_t* xr = reinterpret_cast<uint16_t*>(static_cast<uint8_t*>(workspace) + dp.xr_off);
-    if (wr::launch_rotate_x(x + m0 * K, signs, xr, mm, (int)K, dp.args.prob[0].Kp, stream) != cudaSuccess)
+    bind_workspace(dp, workspace);
+    if (wr::launch_rotate_x(x + m0 * K, signs, dp.args.prob[0].xt, mm, (int)K, dp.args.prob[0].Kp, stream) !=
+        cudaSuccess)
       return WR_ERR_CUDA;
-    dp.args.prob[0].x = xr;
+    dp.args.prob[0].x = nullptr;
     dp.args.prob[0].packed = static_cast<const uint8_t*>(packed);
     dp.args.prob[0].scales = alpha;
     dp.args.prob[0].y = y + m0 * N;
-    const wr_status st = run_decode(dp, true, workspace, stream);
+    const wr_status st = run_decode(dp, true, stream);
     if (st != WR_OK) return st;
   }
   return WR_OK;
@@ -308,7 +324,8 @@ wr_status wr_gemv_batched(int64_t M, int32_t count, const wr_gemv_problem* probl
       dp.args.prob[i].scales = problems[c0 + i].scales;
       dp.args.prob[i].y = problems[c0 + i].y;
     }
-    const wr_status st = run_decode(dp, false, workspace, static_cast<cudaStream_t>(stream));
+    bind_workspace(dp, workspace);
+    const wr_status st = run_decode(dp, false, static_cast<cudaStream_t>(stream));
     if (st != WR_OK) return st;
   }
   return WR_OK;

@@ -2,8 +2,9 @@
 //
 // The byte layout is specified in include/wr.h. Here it is produced word by word: each
 // lane's 16-byte chunks are assembled from the code matrix and stored at
-// (32*chunk + lane)*16 inside their unit. The quantizers prepare inputs (codes and fp16
+// (32*chunk + lane)*16 inside their unit, and units are placed group by group. The quantizers prepare inputs (codes and fp16
 // scales) from fp32 weights; they are not part of the device path.
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -38,6 +39,14 @@ bool geometry(int fmt, int64_t N, int64_t K, Geometry* g) {
   g->tiles = (N + kTileRows - 1) / kTileRows;
   g->units = (K + g->unit_k - 1) / g->unit_k;
   return true;
+}
+
+// Index of unit (tile tn, block u): tiles come in groups of 8; a group's units are stored
+// block by block and, within a block, tile by tile.
+inline int64_t unit_index(const Geometry& g, int64_t tn, int64_t u) {
+  const int64_t grp = tn / 8;
+  const int64_t tg = std::min<int64_t>(8, g.tiles - 8 * grp);
+  return 8 * grp * g.units + u * tg + tn % 8;
 }
 
 // Byte offset inside a unit of lane-byte `lb` of lane `lane`.
@@ -152,7 +161,7 @@ wr_status wr_pack(int fmt, int64_t N, int64_t K, const uint8_t* codes, uint8_t* 
 #pragma omp parallel for collapse(2) schedule(static)
   for (int64_t tn = 0; tn < g.tiles; ++tn) {
     for (int64_t u = 0; u < g.units; ++u) {
-      uint8_t* unit = packed + (tn * g.units + u) * g.unit_bytes;
+      uint8_t* unit = packed + unit_index(g, tn, u) * g.unit_bytes;
       for (int lane = 0; lane < 32; ++lane) {
         const int r0 = lane / 4, q = lane % 4;
         for (int half = 0; half < 2; ++half) {
@@ -194,7 +203,7 @@ wr_status wr_unpack_codes(int fmt, int64_t N, int64_t K, const uint8_t* packed, 
 #pragma omp parallel for collapse(2) schedule(static)
   for (int64_t tn = 0; tn < g.tiles; ++tn) {
     for (int64_t u = 0; u < g.units; ++u) {
-      const uint8_t* unit = packed + (tn * g.units + u) * g.unit_bytes;
+      const uint8_t* unit = packed + unit_index(g, tn, u) * g.unit_bytes;
       for (int lane = 0; lane < 32; ++lane) {
         const int r0 = lane / 4, q = lane % 4;
         for (int half = 0; half < 2; ++half) {

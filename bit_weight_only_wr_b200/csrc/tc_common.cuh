@@ -27,27 +27,28 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
                : "memory");
 }
+// try_wait with a suspend-time hint: a thread whose phase is not complete sleeps in hardware
+// (up to the hint) instead of spinning.
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
-      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}"
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n selp.u32 %0, 1, 0, p;\n}"
       : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(200000u)
       : "memory");
   return ok != 0;
 }
 
 // Wait for the phase with the given parity to complete. Gives up after a bounded number of
-// polls (seconds of wall time): records `code` in the device error word, raises the CTA's
-// abort flag and returns false. Every waiter also returns false once the flag is up.
+// tries (each suspends for at most 0.2 ms; a few seconds in all): records `code` in the
+// device error word, raises the CTA's abort flag and returns false. Every waiter also
+// returns false once the flag is up.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
                                           int* err_word, int code) {
-  for (uint32_t i = 0; i < (1u << 26); ++i) {
+  if (mbar_try_wait(bar, parity)) return true;
+  for (uint32_t i = 0; i < 20000u; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 255u) == 255u) {
-      if (*abort_flag) return false;
-      __nanosleep(32);
-    }
+    if (*abort_flag) return false;
   }
   *abort_flag = 1;
   if (err_word) atomicCAS(err_word, 0, code);

@@ -222,10 +222,8 @@ __global__ void __launch_bounds__(kThreads, BN == 16 ? 2 : 1) tc_kernel(const Tc
           if (!mbar_wait(&bars->pk_empty[sp], ((gb / kSP) & 1) ^ 1, abort_flag, a.err, 102)) break;
           const int ntile = min(8, tiles - rg * 8);
           mbar_arrive_expect_tx(&bars->pk_full[sp], ntile * F::kUnitBytes);
-          for (int i = 0; i < ntile; ++i) {
-            const uint8_t* src = a.packed + ((int64_t)(rg * 8 + i) * a.B + b) * F::kUnitBytes;
-            bulk_load(ps + sp * Ly::kPStage + i * F::kUnitBytes, src, F::kUnitBytes, &bars->pk_full[sp]);
-          }
+          bulk_load(ps + sp * Ly::kPStage, a.packed + ((int64_t)rg * 8 * a.B + (int64_t)b * ntile) * F::kUnitBytes,
+                    ntile * F::kUnitBytes, &bars->pk_full[sp]);
         }
       }
     }
@@ -472,11 +470,13 @@ cudaError_t launch_tc(const TcArgs& a, const void* x_act, int64_t x_rows, int64_
 }
 
 // R x for the ternary path: one warp per (token, 128-block). x' = (1/sqrt(128)) H (d * x) in
-// fp32, split into hi = bf16(x') and lo = bf16(x' - hi), written as two planes [2][M][Kp] in
-// the K order of the decoded A columns: position 80q + 2P + h of a 320-trit unit holds trit
-// 80q + 5*(2*(P/5) + h) + P%5 (pair P of byte pair P/5; h selects the byte). Pad trits get 0.
+// fp32, split into hi = bf16(x') and lo = bf16(x' - hi). The values are written as the B tiles
+// the decode kernel copies: per 320-trit unit, 5 atoms of 64 positions and 16 rows (2048 B),
+// hi of token m in row m, lo in row 8 + m (128-byte swizzle: 16-byte chunk c of row r at
+// c ^ (r % 8)). Position 80q + 2P + h of a unit holds trit 80q + 5*(2*(P/5) + h) + P%5 (pair P
+// of byte pair P/5; h selects the byte), the K order of the decoded A columns. Pad trits get 0.
 __global__ void rotate_x_kernel(const uint16_t* __restrict__ x, const uint32_t* __restrict__ signs,
-                                uint16_t* __restrict__ xr, int M, int K, int64_t Kp) {
+                                uint8_t* __restrict__ xt, int M, int K, int64_t Kp) {
   const int lane = threadIdx.x & 31;
   const int64_t item = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int64_t nblk = (Kp + 127) / 128;
@@ -515,9 +515,11 @@ __global__ void rotate_x_kernel(const uint16_t* __restrict__ x, const uint32_t* 
     const int64_t u = k / 320;
     const int kk = (int)(k % 320), q = kk / 80, i80 = kk % 80, beta = i80 / 5, dig = i80 % 5;
     const int P = 5 * (beta >> 1) + dig;
-    const int64_t pos = u * 320 + 80 * q + 2 * P + (beta & 1);
-    xr[(int64_t)m * Kp + pos] = __bfloat16_as_ushort(hi);
-    xr[((int64_t)M + m) * Kp + pos] = __bfloat16_as_ushort(lo);
+    const int kp = 80 * q + 2 * P + (beta & 1);
+    const int at = kp >> 6, e = kp & 63;
+    const int64_t off = u * (5 * 2048) + at * 2048 + m * 128 + ((((e >> 3) ^ (m & 7)) << 4) | ((e & 7) << 1));
+    *reinterpret_cast<uint16_t*>(xt + off) = __bfloat16_as_ushort(hi);                 // row m
+    *reinterpret_cast<uint16_t*>(xt + off + 1024) = __bfloat16_as_ushort(lo);          // row 8 + m
   }
 }
 
@@ -539,12 +541,12 @@ cudaError_t launch_tc_kernel(int fmt, int bn, const TcArgs& a, const void* x_act
   return cudaErrorNotSupported;
 }
 
-cudaError_t launch_rotate_x(const uint16_t* x, const uint32_t* signs, uint16_t* xr, int M, int K, int64_t Kp,
+cudaError_t launch_rotate_x(const uint16_t* x, const uint32_t* signs, uint8_t* xt, int M, int K, int64_t Kp,
                             cudaStream_t stream) {
   const int64_t items = (int64_t)M * ((Kp + 127) / 128);
   const int warps = 8;
   const int64_t ctas = (items + warps - 1) / warps;
-  rotate_x_kernel<<<(unsigned)ctas, warps * 32, 0, stream>>>(x, signs, xr, M, K, Kp);
+  rotate_x_kernel<<<(unsigned)ctas, warps * 32, 0, stream>>>(x, signs, xt, M, K, Kp);
   return cudaGetLastError();
 }
 

@@ -25,13 +25,15 @@ struct TcArgs {
 constexpr int kMaxDecodeProblems = 256;
 
 struct DecProblem {
-  const uint16_t* x;         // bf16 [M, K]; ternary: R x as [2][M][Kp] planes (hi, lo)
+  const uint16_t* x;         // bf16 [M, K] activations (Q2/Q3; read by the preparation pass)
+  uint8_t* xt;               // prepared activation tiles of this problem (workspace), one per block
   const uint8_t* packed;     // packed units, tile-major
   const uint16_t* scales;    // fp16 [N, K/256] (Q2/Q3) or alpha [N] (ternary)
   float* y;                  // fp32 [M, N]
   int N, K, Kp;              // Kp: padded K of the ternary planes
   int B, RG, P, bits;        // blocks per row, 128-row groups, K splits, 2/3 (ternary: 1)
   int item_base;             // first work item of this problem
+  int xblk_base;             // first block of this problem in the preparation pass
   int counter_base;          // first arrival counter of this problem
   int64_t partial_base;      // first partial float of this problem
 };
@@ -45,11 +47,23 @@ struct DecArgs {
 };
 
 cudaError_t launch_decode(bool ternary, const DecArgs& a, int grid, cudaStream_t stream);
+cudaError_t launch_prep_x(const DecArgs& a, int total_blocks, cudaStream_t stream);
+
+// One prepared activation tile per block, stored as the exact image of a shared-memory B
+// stage so that one bulk copy moves it: K atoms of 64 positions at a stride of xatom_stride
+// bytes, token row m of an atom at m * 128 with 16-byte chunk c at c ^ (m % 8) (128-byte
+// swizzle). Q2/Q3: 4 atoms, 8 rows per atom for M <= 8 (1024 B) else 16 (2048 B), then 64
+// bytes of per-token corrections; ternary: 5 atoms of 16 rows, rows 0..7 the hi plane of
+// tokens 0..7, rows 8..15 the lo plane. Rows of tokens >= M are never read back as results.
+__host__ __device__ inline int xatom_stride(bool ternary, int M) { return (ternary || M > 8) ? 2048 : 1024; }
+__host__ __device__ inline int64_t xtile_bytes(bool ternary, int M) {
+  return ternary ? (int64_t)5 * 2048 : (int64_t)4 * xatom_stride(false, M) + 64;
+}
 
 int tc_tmem_cols(int fmt, int bn);
 cudaError_t launch_tc_kernel(int fmt, int bn, const TcArgs& a, const void* x_act, int64_t x_rows, int64_t x_k,
                              int grid, cudaStream_t stream);
-cudaError_t launch_rotate_x(const uint16_t* x, const uint32_t* signs, uint16_t* xr, int M, int K, int64_t Kp,
+cudaError_t launch_rotate_x(const uint16_t* x, const uint32_t* signs, uint8_t* xt, int M, int K, int64_t Kp,
                             cudaStream_t stream);
 cudaError_t launch_unpack_bf16(int fmt, const uint8_t* packed, const uint16_t* scales, int N, int K, int units,
                                uint16_t* w, cudaStream_t stream);

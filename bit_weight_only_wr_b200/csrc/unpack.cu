@@ -42,7 +42,12 @@ __global__ void __launch_bounds__(256) unpack_kernel(const uint8_t* __restrict__
     wd[4 * c + 2] = v.z;
     wd[4 * c + 3] = v.w;
   }
-  const int64_t tn = u / B, ub = u % B;
+  // unit u -> (tile, block): groups of 8 tiles, each group's units block by block
+  const int64_t tiles = (N + 15) / 16;
+  const int64_t grp = u / (8 * (int64_t)B);
+  const int64_t tg = min((int64_t)8, tiles - 8 * grp);
+  const int64_t rem = u - grp * 8 * (int64_t)B;
+  const int64_t ub = rem / tg, tn = 8 * grp + rem % tg;
   const int r0 = lane >> 2, q = lane & 3;
 #pragma unroll
   for (int h = 0; h < 2; ++h) {

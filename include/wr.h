@@ -28,10 +28,13 @@
  *
  * Packed layout (shared by every kernel; the bytes are what wr_pack writes)
  * -------------------------------------------------------------------------
- * Rows are grouped in tiles of 16 (the last tile padded). K is cut in units: 256 codes
- * for Q2/Q3 (K must be a multiple of 256), 320 trits for ternary (any K, the last unit
- * padded; the ternary GEMM needs K to be a multiple of 128 for the rotation). The buffer is the sequence of units of tile 0, then of
- * tile 1, ... ; a unit is UB contiguous bytes: UB = 1024 (Q2), 1536 (Q3), 1024 (ternary).
+ * Rows are grouped in tiles of 16 (the last tile padded) and tiles in groups of 8 (the last
+ * group may hold fewer). K is cut in units: 256 codes for Q2/Q3 (K must be a multiple of 256),
+ * 320 trits for ternary (any K, the last unit padded; the ternary GEMM needs K to be a multiple
+ * of 128 for the rotation). A unit is UB contiguous bytes: UB = 1024 (Q2), 1536 (Q3), 1024
+ * (ternary). A group's units are stored block by block and, within a block, tile by tile:
+ * unit (tile t, block b) is number 8*(t/8)*B + b*Tg + t%8, with B units per row of tiles and
+ * Tg = min(8, tiles - 8*(t/8)), so the 8 units that cover 128 rows of one block are adjacent.
  * Inside a unit, lane l = 4*r0 + q (r0 = 0..7, q = 0..3) owns rows r0 and r0+8 of the
  * tile and the q-th quarter (64 codes, or 80 trits) of the unit's K range. A lane's bytes
  * are its row-r0 bytes followed by its row-(r0+8) bytes (16 + 16 for Q2, 24 + 24 for Q3,

@@ -218,9 +218,12 @@ def sign_vector(sign_words: np.ndarray, K: int) -> np.ndarray:
 # --------------------------------------------------------------------------------------
 #
 # Common frame (2-bit, 3-bit and ternary): rows are grouped in tiles of 16 (the last
-# tile padded); the K axis is cut in units (256 codes for Q2/Q3, 320 trits for
-# ternary, the last ternary unit padded). Tiles are stored unit after unit
-# (tile-major), each unit a contiguous byte block. Inside a unit, "lane"
+# tile padded) and tiles in groups of 8 (the last group may hold fewer); the K axis is
+# cut in units (256 codes for Q2/Q3, 320 trits for ternary, the last ternary unit
+# padded). Each unit is a contiguous byte block; a group's units are stored block by
+# block and, within a block, tile by tile: unit (tile t, block b) has index
+# 8*(t//8)*B + b*T_g + t%8, with B units per tile row and T_g = min(8, tiles - 8*(t//8)).
+# Inside a unit, "lane"
 # l = 4*r0 + q (r0 = 0..7, q = 0..3) owns rows r0 and r0 + 8 of the tile and the
 # q-th quarter of the unit's K range; a lane's bytes (row r0's data, then row
 # r0+8's) are cut in 16-byte chunks, and chunk c of lane l sits at unit byte
@@ -254,13 +257,16 @@ def _frame(fmt: int, N: int, K: int):
     n = np.arange(N)[:, None]
     k = np.arange(K)[None, :]
     units = -(-K // ku)
+    tiles = -(-N // TILE_ROWS)
     tn, r = n // TILE_ROWS, n % TILE_ROWS
     u, kk = k // ku, k % ku
     qlen = ku // 4
     q, i = kk // qlen, kk % qlen
     lane = 4 * (r % 8) + q
     half = r // 8
-    base = (tn * units + u) * ub
+    grp = tn // 8
+    tg = np.minimum(8, tiles - 8 * grp)
+    base = (8 * grp * units + u * tg + tn % 8) * ub
     return base, lane, half, i
 
 
