@@ -40,6 +40,7 @@ def parse_args():
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", choices=["wr", "reference"], default="wr")
     p.add_argument("--layers", type=int, default=36)
+    p.add_argument("--tokens", type=int, default=1, help="decode tokens M of the headline body (1..8)")
     p.add_argument("--no-extras", action="store_true", help="headline body only")
     p.add_argument("--cpu-seconds", type=float, default=12.0, help="oracle sample budget (0: no CPU baseline)")
     return p.parse_args()
@@ -315,10 +316,10 @@ def main():
         return out
 
     with ClockSampler(uuid) as clk:
-        head = body_run(1, args.steps, args.warmup, True)
+        head = body_run(args.tokens, args.steps, args.warmup, True)
     clocks = clk.summary()
     total_gbs = head["gbs"] * world
-    tokens_per_s = world * 1e3 / head["ms"]
+    tokens_per_s = world * args.tokens * 1e3 / head["ms"]
 
     extras = {}
     if not args.no_extras:
@@ -352,9 +353,9 @@ def main():
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "tokens_per_s": tokens_per_s, "pct_of_8TBps": 100.0 * head["gbs"] / 8000.0,
         "config": {"workload": f"qwen3-4b body, {args.layers} layers x 7 packed GEMVs (v/up/down 3-bit, "
-                               "others 2-bit, fp16 block-256 scales), M=1 decode",
+                               "others 2-bit, fp16 block-256 scales), M=%d decode" % args.tokens,
                    "model": "Qwen3-4B-shaped linears (synthetic, W~N(0,0.02), x~N(0,1) bf16)",
-                   "global_batch": world, "seq_len": 1, "parallelism": f"replicas x{world}",
+                   "global_batch": world * args.tokens, "seq_len": 1, "parallelism": f"replicas x{world}",
                    "l2": "inputs larger than L2 (1.18 GB of packed weights per step)",
                    "bytes_per_step": head["bytes"], "setup_s": round(setup_s, 1)},
         "roofline": roof, "cpu_baseline": cb, "clocks": clocks,

@@ -55,9 +55,9 @@ wr_status check_dims(int64_t M, int64_t N, int64_t K) {
 }
 
 constexpr int kPlanSMs = 148;   // split heuristics are sized for a 148-SM part (device-independent)
-constexpr int kDecodeTokens = 16;
+constexpr int kDecodeTokens = 8;   // decode kernel: 8 tokens x 4 activation limbs = 32 MMA columns
 
-// ---- decode kernel (M <= 16): work items (problem, 128-row group, block range) and workspace
+// ---- decode kernel (M <= 8): work items (problem, 128-row group, block range) and workspace
 // [counters: one int per row group of every problem][split-K partials of problems with P > 1]
 // [prepared activation tiles: one per block of every problem].
 struct DecodePlan {
@@ -135,7 +135,7 @@ wr_status run_decode(DecodePlan& dp, bool ternary, cudaStream_t stream) {
   return wr::launch_decode(ternary, dp.args, grid, stream) == cudaSuccess ? WR_OK : WR_ERR_CUDA;
 }
 
-// ---- prefill GEMM kernel (M > 16): 128-row groups x 128-token tiles x K splits; workspace
+// ---- prefill GEMM kernel (M > 8): 128-row groups x 128-token tiles x K splits; workspace
 // [counters: one int per (row group, token tile)][split-K partials].
 struct GemmPlan {
   int B = 0, RG = 0, MT = 0, P = 1, items = 0;

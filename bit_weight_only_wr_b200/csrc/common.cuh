@@ -146,6 +146,62 @@ __device__ __forceinline__ int q3_shift(int k) {
   return 7 - ((P == 15 || (P % 5) % 2 == 0) ? 1 : 4);
 }
 
+// ---------------------------------------------------------------- int8 code decoders
+//
+// The integer tensor-core path keeps weights as their unsigned codes c, one byte each; a 32-bit
+// TMEM column holds 4 consecutive K positions of the MMA. The bytes are taken straight out of
+// the packed words, so the K order inside a register is a fixed permutation of the code order;
+// the activation tile is written in the same permuted order (see q2_logical / q3_logical).
+//
+// Q2 word (codes e = 0..15, code e at bits 16*(e&1) + 2*(e>>1)): register s' (0..3) =
+// (w >> 2s') & 0x03030303 holds codes [2s', 2s'+8, 2s'+1, 2s'+9] in bytes 0..3.
+__device__ __forceinline__ void decode_q2_word_i8(uint32_t w, uint32_t r[4]) {
+  r[0] = w & 0x03030303u;
+  r[1] = (w >> 2) & 0x03030303u;
+  r[2] = (w >> 4) & 0x03030303u;
+  r[3] = (w >> 6) & 0x03030303u;
+}
+
+// Q3 group (3 words, codes 10u + 2j + h at bits 16h + 3j; codes 30 + h in bit 16h + 15 of
+// words 0..2) -> 8 registers:
+//   2u:   [10u,   10u+2, 10u+1, 10u+3]     2u+1: [10u+4, 10u+6, 10u+5, 10u+7]   (u = 0, 1, 2)
+//   6:    [8, 18, 9, 19]                   7:    [28, 30, 29, 31]
+__device__ __forceinline__ void decode_q3_group_i8(const uint32_t w[3], uint32_t r[8]) {
+#pragma unroll
+  for (int u = 0; u < 3; ++u) {
+    r[2 * u] = (w[u] & 0x00070007u) | ((w[u] << 5) & 0x07000700u);
+    r[2 * u + 1] = ((w[u] >> 6) & 0x00070007u) | ((w[u] >> 1) & 0x07000700u);
+  }
+  r[6] = ((w[0] >> 12) & 0x00070007u) | ((w[1] >> 4) & 0x07000700u);
+  r[7] = ((w[2] >> 12) & 0x00070007u) | ((w[0] >> 7) & 0x01000100u) | ((w[1] >> 6) & 0x02000200u) |
+         ((w[2] >> 5) & 0x04000400u);
+}
+
+// Code index (within a 256-code block) held at logical K position kl of the decoded block,
+// for the register orders above. Rows of a block are 4 quarters of 64 codes; a quarter is 16
+// registers (Q2: 4 words x 4; Q3: 2 groups x 8).
+__host__ __device__ inline int q2_code_at(int kl) {
+  const int q = kl >> 6, w = (kl >> 4) & 3, sp = (kl >> 2) & 3, byte = kl & 3;
+  const int p = 2 * sp + ((byte & 1) ? 8 : 0) + (byte >> 1);
+  return 64 * q + 16 * w + p;
+}
+__host__ __device__ inline int q3_code_at(int kl) {
+  const int q = kl >> 6, g = (kl >> 5) & 1, reg = (kl >> 2) & 7, byte = kl & 3;
+  int c;
+  if (reg < 6) {
+    const int u = reg >> 1, base = 10 * u + ((reg & 1) ? 4 : 0);
+    const int off[4] = {0, 2, 1, 3};
+    c = base + off[byte];
+  } else if (reg == 6) {
+    const int t[4] = {8, 18, 9, 19};
+    c = t[byte];
+  } else {
+    const int t[4] = {28, 30, 29, 31};
+    c = t[byte];
+  }
+  return 64 * q + 32 * g + c;
+}
+
 __device__ __forceinline__ float half_bits_to_float(uint16_t h) {
   return __half2float(__ushort_as_half(h));
 }

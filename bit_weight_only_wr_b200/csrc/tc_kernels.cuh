@@ -21,7 +21,7 @@ struct TcArgs {
   int items;                 // RG * MT * P
 };
 
-// Batched decode GEMV (M <= 16): one launch over up to kMaxDecodeProblems independent problems.
+// Batched decode GEMV (M <= 8): one launch over up to kMaxDecodeProblems independent problems.
 constexpr int kMaxDecodeProblems = 256;
 
 struct DecProblem {
@@ -49,15 +49,15 @@ struct DecArgs {
 cudaError_t launch_decode(bool ternary, const DecArgs& a, int grid, cudaStream_t stream);
 cudaError_t launch_prep_x(const DecArgs& a, int total_blocks, cudaStream_t stream);
 
-// One prepared activation tile per block, stored as the exact image of a shared-memory B
-// stage so that one bulk copy moves it: K atoms of 64 positions at a stride of xatom_stride
-// bytes, token row m of an atom at m * 128 with 16-byte chunk c at c ^ (m % 8) (128-byte
-// swizzle). Q2/Q3: 4 atoms, 8 rows per atom for M <= 8 (1024 B) else 16 (2048 B), then 64
-// bytes of per-token corrections; ternary: 5 atoms of 16 rows, rows 0..7 the hi plane of
-// tokens 0..7, rows 8..15 the lo plane. Rows of tokens >= M are never read back as results.
-__host__ __device__ inline int xatom_stride(bool ternary, int M) { return (ternary || M > 8) ? 2048 : 1024; }
+// One prepared activation tile per block, stored as the exact image of a shared-memory B stage
+// so that one bulk copy moves it (128-byte swizzle: 16-byte chunk c of a row r at c ^ (r % 8)).
+// 2/3-bit (integer path): two atoms of 128 K positions x xrows rows of int8, limb j of token m in
+// row (xrows/4) j + m, then 256 bytes of corrections: 2^E per token (8 floats) and the limb sums
+// (8 x 4 int32). xrows = 8, 16 or 32 for M <= 2, 4, 8 (the MMA's N).
+// Ternary: 5 atoms of 64 K positions x 16 rows of bf16, hi of token m in row m, lo in 8 + m.
+__host__ __device__ inline int decode_xrows(int M) { return M <= 2 ? 8 : (M <= 4 ? 16 : 32); }
 __host__ __device__ inline int64_t xtile_bytes(bool ternary, int M) {
-  return ternary ? (int64_t)5 * 2048 : (int64_t)4 * xatom_stride(false, M) + 64;
+  return ternary ? (int64_t)5 * 2048 : (int64_t)2 * decode_xrows(M) * 128 + 256;
 }
 
 int tc_tmem_cols(int fmt, int bn);
