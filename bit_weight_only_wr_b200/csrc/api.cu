@@ -130,9 +130,10 @@ void bind_workspace(DecodePlan& dp, void* workspace) {
 // Q2/Q3: preparation pass, then the decode kernel; ternary: the rotation pass has already
 // written the tiles.
 wr_status run_decode(DecodePlan& dp, bool ternary, cudaStream_t stream) {
-  if (!ternary && wr::launch_prep_x(dp.args, dp.total_blocks, stream) != cudaSuccess) return WR_ERR_CUDA;
   const int grid = (int)std::min<int64_t>(dp.args.items, (int64_t)sm_count() * 2);
-  return wr::launch_decode(ternary, dp.args, grid, stream) == cudaSuccess ? WR_OK : WR_ERR_CUDA;
+  if (ternary) return wr::launch_gemv_t(dp.args, grid, stream) == cudaSuccess ? WR_OK : WR_ERR_CUDA;
+  if (wr::launch_prep_x(dp.args, dp.total_blocks, stream) != cudaSuccess) return WR_ERR_CUDA;
+  return wr::launch_gemv_q(dp.args, grid, stream) == cudaSuccess ? WR_OK : WR_ERR_CUDA;
 }
 
 // ---- prefill GEMM kernel (M > 8): 128-row groups x 128-token tiles x K splits; workspace

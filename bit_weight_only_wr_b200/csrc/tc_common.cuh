@@ -27,32 +27,85 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
                : "memory");
 }
-// try_wait with a suspend-time hint: a thread whose phase is not complete sleeps in hardware
-// (up to the hint) instead of spinning.
+// One probe of the phase with the given parity (no suspend-time hint: a hinted try_wait
+// measured about 60% more wake-up latency between warps of one CTA).
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
-      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n selp.u32 %0, 1, 0, p;\n}"
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}"
       : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity), "r"(200000u)
+      : "r"(smem_u32(bar)), "r"(parity)
       : "memory");
   return ok != 0;
 }
 
-// Wait for the phase with the given parity to complete. Gives up after a bounded number of
-// tries (each suspends for at most 0.2 ms; a few seconds in all): records `code` in the
-// device error word, raises the CTA's abort flag and returns false. Every waiter also
-// returns false once the flag is up.
+// The same probe with a suspend-time hint: a thread whose phase is not complete is suspended in
+// hardware (and takes no issue slots) until the phase completes or the hint runs out. Wakes
+// up about 60 ns later than a spinning probe: for roles that wait most of the time and are not
+// on the critical path (producers, the MMA issuer), whose spinning would steal issue slots from
+// the warps that are.
+__device__ __forceinline__ bool mbar_try_wait_suspend(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n selp.u32 %0, 1, 0, p;\n}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(100000u)
+      : "memory");
+  return ok != 0;
+}
+
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Every wait gives up after this long: nothing in these kernels legitimately waits more than
+// microseconds.
+constexpr uint64_t kWaitLimitNs = 1000000000ull;
+
+// Wait for the phase with the given parity to complete. Gives up after kWaitLimitNs: records
+// `code` in the device error word, raises the CTA's abort flag and returns false. Every
+// waiter also returns false once the flag is up.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
                                           int* err_word, int code) {
   if (mbar_try_wait(bar, parity)) return true;
-  for (uint32_t i = 0; i < 20000u; ++i) {
+  const uint64_t t0 = global_ns();
+  for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
-    if (*abort_flag) return false;
+    if ((i & 15u) == 0) {
+      if (*abort_flag) return false;
+      if (global_ns() - t0 > kWaitLimitNs) break;
+    }
   }
   *abort_flag = 1;
   if (err_word) atomicCAS(err_word, 0, code);
   return false;
+}
+
+// mbar_wait for the background roles (see mbar_try_wait_suspend).
+__device__ __forceinline__ bool mbar_wait_bg(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                             int* err_word, int code) {
+  if (mbar_try_wait_suspend(bar, parity)) return true;
+  const uint64_t t0 = global_ns();
+  for (;;) {
+    if (mbar_try_wait_suspend(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if (global_ns() - t0 > kWaitLimitNs) break;
+  }
+  *abort_flag = 1;
+  if (err_word) atomicCAS(err_word, 0, code);
+  return false;
+}
+
+// Bounded wait that ignores the abort flag: used on the way out of an aborted CTA to let
+// copies already in flight land before the CTA exits.
+__device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity) {
+  const uint64_t t0 = global_ns();
+  for (uint32_t i = 0;; ++i) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((i & 15u) == 15u && global_ns() - t0 > kWaitLimitNs) return false;
+  }
 }
 
 // ---------------------------------------------------------------- copies
@@ -130,6 +183,32 @@ __device__ __forceinline__ void mma_ts_i8(uint32_t d_tmem, uint32_t a_tmem, uint
       "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
       " tcgen05.mma.cta_group::1.kind::i8 [%0], [%1], %2, %3, p;\n}" ::"r"(d_tmem),
       "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Warp-wide forms: every lane of the warp executes the call with the same operands (so the
+// descriptor arithmetic stays warp-uniform) and one lane chosen by elect.sync issues the
+// instruction. Issuing from a loop that only lane 0 runs measured about three times slower.
+__device__ __forceinline__ void mma_ts_elect(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                             uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p, e;\n setp.ne.b32 p, %4, 0;\n elect.sync _|e, 0xffffffff;\n"
+      " @e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void mma_ts_i8_elect(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                                uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p, e;\n setp.ne.b32 p, %4, 0;\n elect.sync _|e, 0xffffffff;\n"
+      " @e tcgen05.mma.cta_group::1.kind::i8 [%0], [%1], %2, %3, p;\n}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void mma_commit_elect(uint64_t* bar) {
+  asm volatile(
+      "{\n .reg .pred e;\n elect.sync _|e, 0xffffffff;\n"
+      " @e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n}" ::"r"(smem_u32(bar))
       : "memory");
 }
 

@@ -196,7 +196,7 @@ __global__ void __launch_bounds__(kThreads, BN == 16 ? 2 : 1) tc_kernel(const Tc
         item_coords(a, it, rg, mt, p, b0, b1);
         for (int b = b0; b < b1; ++b, ++gb) {
           const int sx = gb % kSX;
-          if (!mbar_wait(&bars->x_empty[sx], ((gb / kSX) & 1) ^ 1, abort_flag, a.err, 101)) break;
+          if (!mbar_wait_bg(&bars->x_empty[sx], ((gb / kSX) & 1) ^ 1, abort_flag, a.err, 101)) break;
           mbar_arrive_expect_tx(&bars->x_full[sx], Ly::kXStage);
 #pragma unroll
           for (int at = 0; at < F::kUnitK / 64; ++at) {
@@ -219,7 +219,7 @@ __global__ void __launch_bounds__(kThreads, BN == 16 ? 2 : 1) tc_kernel(const Tc
             }
           }
           const int sp = gb % kSP;
-          if (!mbar_wait(&bars->pk_empty[sp], ((gb / kSP) & 1) ^ 1, abort_flag, a.err, 102)) break;
+          if (!mbar_wait_bg(&bars->pk_empty[sp], ((gb / kSP) & 1) ^ 1, abort_flag, a.err, 102)) break;
           const int ntile = min(8, tiles - rg * 8);
           mbar_arrive_expect_tx(&bars->pk_full[sp], ntile * F::kUnitBytes);
           bulk_load(ps + sp * Ly::kPStage, a.packed + ((int64_t)rg * 8 * a.B + (int64_t)b * ntile) * F::kUnitBytes,
@@ -228,47 +228,45 @@ __global__ void __launch_bounds__(kThreads, BN == 16 ? 2 : 1) tc_kernel(const Tc
       }
     }
   } else if (warp == 9) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16_m128(BN);
-      uint32_t gb = 0, gc = 0, gi = 0;
-      for (int it = blockIdx.x; it < a.items && !*abort_flag; it += gridDim.x, ++gi) {
-        int rg, mt, p, b0, b1;
-        item_coords(a, it, rg, mt, p, b0, b1);
-        bool ok = true;
-        uint32_t dbuf = 0;
-        if (FMT == WR_FMT_TERNARY) {
-          dbuf = gi & 1;
-          ok = mbar_wait(&bars->d_empty[dbuf], ((gi >> 1) & 1) ^ 1, abort_flag, a.err, 201);
-        }
-        for (int b = b0; b < b1 && ok; ++b, ++gb) {
-          if (FMT != WR_FMT_TERNARY) {
-            dbuf = gb & 1;
-            if (!(ok = mbar_wait(&bars->d_empty[dbuf], ((gb >> 1) & 1) ^ 1, abort_flag, a.err, 202))) break;
-          }
-          const int sx = gb % kSX;
-          if (!(ok = mbar_wait(&bars->x_full[sx], (gb / kSX) & 1, abort_flag, a.err, 203))) break;
-          const uint8_t* xst = xs + sx * Ly::kXStage;
-          for (int c = 0; c < 2; ++c, ++gc) {
-            const int sa = gc & 1;
-            if (!(ok = mbar_wait(&bars->a_full[sa], (gc >> 1) & 1, abort_flag, a.err, 204))) break;
-            fence_after_sync();
-#pragma unroll
-            for (int j = 0; j < F::kChunkSteps; ++j) {
-              const int kk = c * (F::kUnitK / 2) + 16 * j;     // K offset inside the block
-              const uint64_t bdesc = smem_desc_sw128(xst + (kk / 64) * Ly::kXAtom + (kk % 64) * 2);
-              const uint32_t acc = (FMT == WR_FMT_TERNARY) ? (uint32_t)(b != b0 || c != 0 || j != 0)
-                                                           : (uint32_t)(c != 0 || j != 0);
-              mma_ts(tmem + Ly::kDCol + dbuf * BN, tmem + sa * Ly::kACols + 8 * j, bdesc, idesc, acc);
-            }
-            mma_commit(&bars->a_empty[sa]);
-          }
-          if (!ok) break;
-          mma_commit(&bars->x_empty[sx]);
-          if (FMT != WR_FMT_TERNARY) mma_commit(&bars->d_full[dbuf]);
-        }
-        if (FMT == WR_FMT_TERNARY && ok) mma_commit(&bars->d_full[dbuf]);
+    // ------------------------------------------------------------ MMA issuer (whole warp, one lane issues)
+    constexpr uint32_t idesc = idesc_bf16_m128(BN);
+    uint32_t gb = 0, gc = 0, gi = 0;
+    for (int it = blockIdx.x; it < a.items && !*abort_flag; it += gridDim.x, ++gi) {
+      int rg, mt, p, b0, b1;
+      item_coords(a, it, rg, mt, p, b0, b1);
+      bool ok = true;
+      uint32_t dbuf = 0;
+      if (FMT == WR_FMT_TERNARY) {
+        dbuf = gi & 1;
+        ok = mbar_wait_bg(&bars->d_empty[dbuf], ((gi >> 1) & 1) ^ 1, abort_flag, a.err, 201);
       }
+      for (int b = b0; b < b1 && ok; ++b, ++gb) {
+        if (FMT != WR_FMT_TERNARY) {
+          dbuf = gb & 1;
+          if (!(ok = mbar_wait_bg(&bars->d_empty[dbuf], ((gb >> 1) & 1) ^ 1, abort_flag, a.err, 202))) break;
+        }
+        const int sx = gb % kSX;
+        if (!(ok = mbar_wait_bg(&bars->x_full[sx], (gb / kSX) & 1, abort_flag, a.err, 203))) break;
+        const uint8_t* xst = xs + sx * Ly::kXStage;
+        for (int c = 0; c < 2; ++c, ++gc) {
+          const int sa = gc & 1;
+          if (!(ok = mbar_wait_bg(&bars->a_full[sa], (gc >> 1) & 1, abort_flag, a.err, 204))) break;
+          fence_after_sync();
+#pragma unroll
+          for (int j = 0; j < F::kChunkSteps; ++j) {
+            const int kk = c * (F::kUnitK / 2) + 16 * j;     // K offset inside the block
+            const uint64_t bdesc = smem_desc_sw128(xst + (kk / 64) * Ly::kXAtom + (kk % 64) * 2);
+            const uint32_t acc = (FMT == WR_FMT_TERNARY) ? (uint32_t)(b != b0 || c != 0 || j != 0)
+                                                         : (uint32_t)(c != 0 || j != 0);
+            mma_ts_elect(tmem + Ly::kDCol + dbuf * BN, tmem + sa * Ly::kACols + 8 * j, bdesc, idesc, acc);
+          }
+          mma_commit_elect(&bars->a_empty[sa]);
+        }
+        if (!ok) break;
+        mma_commit_elect(&bars->x_empty[sx]);
+        if (FMT != WR_FMT_TERNARY) mma_commit_elect(&bars->d_full[dbuf]);
+      }
+      if (FMT == WR_FMT_TERNARY && ok) mma_commit_elect(&bars->d_full[dbuf]);
     }
   } else if (warp < 4) {
     // ------------------------------------------------------------ decode (thread = row)

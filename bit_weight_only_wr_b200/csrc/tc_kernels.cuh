@@ -46,14 +46,17 @@ struct DecArgs {
   DecProblem prob[kMaxDecodeProblems];
 };
 
-cudaError_t launch_decode(bool ternary, const DecArgs& a, int grid, cudaStream_t stream);
+// 2/3-bit decode: the preparation pass writes the B tiles, then the GEMV kernel.
 cudaError_t launch_prep_x(const DecArgs& a, int total_blocks, cudaStream_t stream);
+cudaError_t launch_gemv_q(const DecArgs& a, int grid, cudaStream_t stream);
+// Ternary decode (tiles written by launch_rotate_x).
+cudaError_t launch_gemv_t(const DecArgs& a, int grid, cudaStream_t stream);
 
 // One prepared activation tile per block, stored as the exact image of a shared-memory B stage
 // so that one bulk copy moves it (128-byte swizzle: 16-byte chunk c of a row r at c ^ (r % 8)).
-// 2/3-bit (integer path): two atoms of 128 K positions x xrows rows of int8, limb j of token m in
-// row (xrows/4) j + m, then 256 bytes of corrections: 2^E per token (8 floats) and the limb sums
-// (8 x 4 int32). xrows = 8, 16 or 32 for M <= 2, 4, 8 (the MMA's N).
+// 2/3-bit (integer path): two atoms of 128 K positions x xrows rows of int8, limb j of token
+// slot m in row 4m + j, then 256 bytes of corrections: 2^E per slot (8 floats) and per slot and
+// limb 0x4B400000 - L S_j (8 x 4 int32). xrows = 8, 16 or 32 for M <= 2, 4, 8 (the MMA's N).
 // Ternary: 5 atoms of 64 K positions x 16 rows of bf16, hi of token m in row m, lo in 8 + m.
 __host__ __device__ inline int decode_xrows(int M) { return M <= 2 ? 8 : (M <= 4 ? 16 : 32); }
 __host__ __device__ inline int64_t xtile_bytes(bool ternary, int M) {
