@@ -18,10 +18,11 @@ __all__ = [
     "wr_quantize", "wr_quantize_ternary", "wr_unpack_bf16", "wr_gemv_workspace_bytes", "wr_gemv",
     "wr_gemm_workspace_bytes", "wr_gemm", "wr_gemm_ternary_workspace_bytes", "wr_gemm_ternary",
     "wr_get_device_error", "exported_symbols", "WrGemvProblem", "wr_gemv_batched_workspace_bytes",
-    "wr_gemv_batched",
+    "wr_gemv_batched", "wr_gemv_noalloc", "WR_GEMV_NOALLOC_SCRATCH_BYTES",
 ]
 
 WR_FMT_TERNARY, WR_FMT_Q2, WR_FMT_Q3 = 1, 2, 3
+WR_GEMV_NOALLOC_SCRATCH_BYTES = 4 << 20   # mirrors the macro in include/wr.h
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libwr.so")
 
 _c_i64, _c_int, _c_size, _vp = ctypes.c_int64, ctypes.c_int, ctypes.c_size_t, ctypes.c_void_p
@@ -53,6 +54,7 @@ _SIGNATURES = {
     "wr_gemm_ternary_workspace_bytes": (_c_size, [_c_i64, _c_i64, _c_i64]),
     "wr_gemm_ternary": (_c_int, [_c_i64, _c_i64, _c_i64, _vp, _vp, _vp, _vp, _vp, _vp, _c_size, _vp]),
     "wr_get_device_error": (_c_int, [_vp]),
+    "wr_gemv_noalloc": (_c_int, [_c_i64, _c_i64, _c_i64, _vp, _vp, _vp, _c_int, _c_int, _vp, _vp]),
 }
 
 
@@ -172,6 +174,13 @@ def wr_gemv(M: int, N: int, K: int, x, packed, scales, bits: int, y, workspace, 
             group: int = 256, stream=None) -> None:
     _check("wr_gemv", _lib.wr_gemv(M, N, K, _ptr(x), _ptr(packed), _ptr(scales), bits, group, _ptr(y),
                                    _ptr(workspace), workspace_bytes, _stream(stream)))
+
+
+def wr_gemv_noalloc(M: int, N: int, K: int, x, packed, scales, bits: int, y, group: int = 256,
+                    stream=None) -> None:
+    """wr_gemv without a workspace (fixed scratch inside libwr; see include/wr.h)."""
+    _check("wr_gemv_noalloc", _lib.wr_gemv_noalloc(M, N, K, _ptr(x), _ptr(packed), _ptr(scales), bits, group,
+                                                   _ptr(y), _stream(stream)))
 
 
 def _problems(problems):

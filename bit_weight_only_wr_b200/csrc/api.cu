@@ -238,6 +238,37 @@ wr_status run_t(int64_t M, int64_t N, int64_t K, const uint16_t* x, const void* 
 
 }  // namespace
 
+// Scratch of wr_gemv_noalloc: a fixed device array (one per device, zero at module load), so
+// that the entry point needs no allocation and no workspace argument.
+static __device__ __align__(256) uint8_t g_noalloc_scratch[WR_GEMV_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+
+// Device address of the current device's scratch array. Looked up once per device, with that
+// device current (the one-time set-up, which may load the module: keep it outside stream
+// capture); later calls read the cached pointer.
+void* noalloc_scratch(wr_status* st) {
+  static std::mutex mu;
+  static void* cache[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+    *st = WR_ERR_CUDA;
+    return nullptr;
+  }
+  std::lock_guard<std::mutex> lock(mu);
+  if (!cache[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) {
+      *st = WR_ERR_CUDA;
+      return nullptr;
+    }
+    cache[dev] = p;
+  }
+  return cache[dev];
+}
+
+}  // namespace
+
 extern "C" {
 
 int wr_abi_version(void) { return 1; }
@@ -249,6 +280,7 @@ const char* wr_status_string(wr_status st) {
     case WR_ERR_UNSUPPORTED: return "unsupported configuration";
     case WR_ERR_CUDA: return "CUDA error";
     case WR_ERR_TIMEOUT: return "device-side wait timed out";
+    case WR_ERR_TOO_LARGE: return "problem needs more than the fixed scratch of wr_gemv_noalloc";
   }
   return "unknown status";
 }
@@ -282,6 +314,25 @@ wr_status wr_gemv(int64_t M, int64_t N, int64_t K, const uint16_t* x, const void
     return WR_ERR_INVALID_ARG;
   if (workspace_bytes < q_workspace(bits, M, N, K)) return WR_ERR_INVALID_ARG;
   return run_q(bits, M, N, K, x, packed, scales, y, workspace, static_cast<cudaStream_t>(stream));
+}
+
+wr_status wr_gemv_noalloc(int64_t M, int64_t N, int64_t K, const uint16_t* x, const void* packed,
+                          const uint16_t* scales, int bits, int group, float* y, void* stream) {
+  if (bits != 2 && bits != 3) return WR_ERR_UNSUPPORTED;
+  if (group != 256) return WR_ERR_UNSUPPORTED;
+  if (M < 1 || M > 8 || check_dims(M, N, K) != WR_OK || K % 256 != 0) return WR_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(packed) || !aligned16(scales) || !aligned16(y)) return WR_ERR_INVALID_ARG;
+  if (q_workspace(bits, M, N, K) > WR_GEMV_NOALLOC_SCRATCH_BYTES) return WR_ERR_TOO_LARGE;
+  wr_status st = WR_OK;
+  void* scratch = noalloc_scratch(&st);
+  if (scratch == nullptr) return st;
+  // the arrival counters (the first bytes of the plan) must start at zero
+  static thread_local DecodePlan dp;
+  const ProblemShape sh{N, K, bits};
+  plan_decode(M, 1, &sh, &dp);
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (dp.partial_off > 0 && cudaMemsetAsync(scratch, 0, dp.partial_off, s) != cudaSuccess) return WR_ERR_CUDA;
+  return run_q(bits, M, N, K, x, packed, scales, y, scratch, s);
 }
 
 static bool batch_ok(int64_t M, int32_t count, const wr_gemv_problem* pr) {

@@ -79,7 +79,8 @@ typedef enum {
   WR_ERR_INVALID_ARG = 1,   /* null/misaligned pointer, bad size or code value */
   WR_ERR_UNSUPPORTED = 2,   /* valid but unsupported: group != 256, bits not 2/3, ... */
   WR_ERR_CUDA = 3,          /* a CUDA launch or runtime call failed */
-  WR_ERR_TIMEOUT = 4        /* a bounded device-side wait gave up (see wr_get_device_error) */
+  WR_ERR_TIMEOUT = 4,       /* a bounded device-side wait gave up (see wr_get_device_error) */
+  WR_ERR_TOO_LARGE = 5      /* the problem needs more than the fixed scratch of wr_gemv_noalloc */
 } wr_status;
 
 enum { WR_FMT_TERNARY = 1, WR_FMT_Q2 = 2, WR_FMT_Q3 = 3 };
@@ -170,6 +171,28 @@ size_t wr_gemm_ternary_workspace_bytes(int64_t M, int64_t N, int64_t K);
 wr_status wr_gemm_ternary(int64_t M, int64_t N, int64_t K, const uint16_t* x, const void* packed,
                           const uint16_t* alpha, const uint32_t* sign_bits, float* y,
                           void* workspace, size_t workspace_bytes, void* stream);
+
+/* Decode GEMV that allocates nothing and takes no workspace (no counterpart in the paper: a
+ * deployment convenience). For callers that may not allocate device memory or pass a
+ * workspace while they run: code recorded into a CUDA graph whose memory was planned up front,
+ * allocator-free serving loops, and callers that hold no handle to a caching allocator. The
+ * scratch that wr_gemv takes as `workspace` is instead a fixed device array of
+ * WR_GEMV_NOALLOC_SCRATCH_BYTES (4 MiB) inside libwr, one per device.
+ *
+ * Computes exactly what wr_gemv computes (same arguments without workspace/workspace_bytes;
+ * 1 <= M <= 8, bits 2 or 3, group 256, K % 256 == 0, 16-byte aligned device pointers).
+ * Returns WR_ERR_TOO_LARGE, before touching the device, when the problem's scratch need
+ * (wr_gemv_workspace_bytes) exceeds WR_GEMV_NOALLOC_SCRATCH_BYTES; then nothing is launched.
+ *
+ * The first call on a device does a one-time set-up with that device current (it looks up the
+ * address of the scratch array): make that first call before any stream capture begins. Each
+ * call clears the scratch's arrival counters on `stream` (cudaMemsetAsync) and then launches
+ * the same kernels as wr_gemv. All calls on one device share the one scratch array, so calls
+ * that overlap in time (on different streams, or from several host threads) race on it and
+ * give undefined results: serialize them. */
+#define WR_GEMV_NOALLOC_SCRATCH_BYTES ((size_t)4 << 20)
+wr_status wr_gemv_noalloc(int64_t M, int64_t N, int64_t K, const uint16_t* x, const void* packed,
+                          const uint16_t* scales, int bits, int group, float* y, void* stream);
 
 /* Reads and clears the device error word that bounded waits set when they give up
  * (synchronizes the stream). WR_OK when no wait timed out since the last call. */
