@@ -90,7 +90,7 @@ void plan_decode(int64_t M, int count, const ProblemShape* shapes, DecodePlan* d
     pr.bits = shapes[i].fmt == WR_FMT_TERNARY ? 1 : shapes[i].fmt;
     total_blocks += (int64_t)pr.RG * pr.B;
   }
-  const int64_t target_items = std::max<int64_t>(2 * kPlanSMs, (total_blocks + 7) / 8);
+  const int64_t target_items = std::max<int64_t>(3 * kPlanSMs, (total_blocks + 7) / 8);
   const double bpi = (double)total_blocks / (double)target_items;
   int items = 0, counters = 0, blocks = 0;
   int64_t partials = 0, xt_bytes = 0;
@@ -130,8 +130,11 @@ void bind_workspace(DecodePlan& dp, void* workspace) {
 // Q2/Q3: preparation pass, then the decode kernel; ternary: the rotation pass has already
 // written the tiles.
 wr_status run_decode(DecodePlan& dp, bool ternary, cudaStream_t stream) {
-  const int grid = (int)std::min<int64_t>(dp.args.items, (int64_t)sm_count() * 2);
-  if (ternary) return wr::launch_gemv_t(dp.args, grid, stream) == cudaSuccess ? WR_OK : WR_ERR_CUDA;
+  if (ternary) {
+    const int grid = (int)std::min<int64_t>(dp.args.items, (int64_t)sm_count() * 2);
+    return wr::launch_gemv_t(dp.args, grid, stream) == cudaSuccess ? WR_OK : WR_ERR_CUDA;
+  }
+  const int grid = (int)std::min<int64_t>(dp.args.items, (int64_t)sm_count() * wr::gemv_q_ctas_per_sm());
   if (wr::launch_prep_x(dp.args, dp.total_blocks, stream) != cudaSuccess) return WR_ERR_CUDA;
   return wr::launch_gemv_q(dp.args, grid, stream) == cudaSuccess ? WR_OK : WR_ERR_CUDA;
 }

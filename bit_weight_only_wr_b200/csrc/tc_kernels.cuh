@@ -49,6 +49,7 @@ struct DecArgs {
 // 2/3-bit decode: the preparation pass writes the B tiles, then the GEMV kernel.
 cudaError_t launch_prep_x(const DecArgs& a, int total_blocks, cudaStream_t stream);
 cudaError_t launch_gemv_q(const DecArgs& a, int grid, cudaStream_t stream);
+int gemv_q_ctas_per_sm();   // CTAs of the 2/3-bit decode kernel that share an SM
 // Ternary decode (tiles written by launch_rotate_x).
 cudaError_t launch_gemv_t(const DecArgs& a, int grid, cudaStream_t stream);
 
