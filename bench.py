@@ -133,6 +133,19 @@ def module_bytes(wr, M, N, K, bits):
     return wr.wr_packed_bytes(fmt, N, K) + N * (K // 256) * 2 + M * K * 2 + M * N * 4
 
 
+# DRAM traffic of the decode GEMV launch, (dram__bytes_read + dram__bytes_write) / algorithmic
+# bytes, from one ncu capture of the current kernel at that token count (summary and command in
+# profiles/). None: no capture of this kernel version, so no traffic figure is claimed.
+# gemv_q_kernel, three CTAs per SM: M = 1 read 1.18 GB + write 9.70 MB; M = 8 read 1.21 GB + write
+# 53.73 MB, for 1,178,984,448 and 1,223,368,704 algorithmic bytes (ncu prints three digits).
+_TRAFFIC_RATIO = {1: (1.18e9 + 9.70e6) / 1_178_984_448, 8: (1.21e9 + 53.73e6) / 1_223_368_704}
+
+
+def traffic_per_launch(M: int, layers: int, algo_bytes: int):
+    r = _TRAFFIC_RATIO.get(M)
+    return None if r is None else int(r * algo_bytes)
+
+
 def graph_time_ms(torch, fn, steps, warmup, stream, dist=None):
     """Capture fn() once in a CUDA graph; replay `warmup` times, then time `steps` replays with
     CUDA events recorded on the stream the replays are launched on, with a barrier and a
@@ -162,10 +175,11 @@ def graph_time_ms(torch, fn, steps, warmup, stream, dist=None):
     return ms
 
 
-def max_over_ranks(torch, dist, v):
+def max_over_ranks(torch, dist, v, device="cuda"):
+    """The slowest rank's time: every replica's device time, reduced with MAX."""
     if not dist:
         return v
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    t = torch.tensor([v], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
@@ -284,14 +298,14 @@ def main():
                                  m["bits"]) for i, m in enumerate(mods)])
             nb = wr.wr_gemv_batched_workspace_bytes(M, arr)
             ws = torch.zeros(nb, dtype=torch.uint8, device="cuda")
-            launches = (len(mods) + 255) // 256
+            launches = 2 * ((len(mods) + 255) // 256)   # preparation pass + decode GEMV per batch
 
             def step():
                 wr.wr_gemv_batched(M, arr, ws, nb)
         else:
             nb = max(wr.wr_gemv_workspace_bytes(M, m["N"], m["K"], m["bits"]) for m in mods)
             ws = torch.zeros(nb, dtype=torch.uint8, device="cuda")
-            launches = len(mods)
+            launches = 2 * len(mods)
 
             def step():
                 for i, m in enumerate(mods):
@@ -334,13 +348,16 @@ def main():
             extras["body_m1_one_call_per_linear"] = {"error": repr(e)}
         extras.update(run_extras(args, wr, torch, np, stream, dist, hbm_peak, bf16_peak))
 
-    # one batched decode launch per step: algorithmic bytes per launch / event-timed launch time
+    # the step is one wr_gemv_batched call: the preparation pass, then one launch of the decode
+    # GEMV kernel over all 252 problems (about 98% of the step's device time in the ncu launch
+    # list); achieved = algorithmic bytes of the launch / event-timed duration of the whole call
     achieved = head["gbs"]
     roof = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
-            "frac": achieved / hbm_peak, "traffic": None, "peak_kind": peak_kind,
-            "kernel": "decode_kernel<false> (batched 2/3-bit decode GEMV, tcgen05)",
-            "note": "the M=1 body step is one launch of the batched decode GEMV: algorithmic bytes per "
-                    "launch / event-timed duration per launch"}
+            "frac": achieved / hbm_peak, "traffic": traffic_per_launch(args.tokens, args.layers, head["bytes"]),
+            "peak_kind": peak_kind,
+            "kernel": "gemv_q_kernel (batched 2/3-bit decode GEMV on tcgen05 kind::i8), after prep_x_kernel",
+            "note": "algorithmic bytes per launch (packed codes + fp16 scales + bf16 x + fp32 y) / CUDA-event "
+                    "duration of the call (preparation pass + GEMV launch), inside the timed region"}
     cb = None
     if rank == 0 and world == 1 and args.cpu_seconds > 0:
         try:
@@ -363,7 +380,8 @@ def main():
                 "h2d_bytes_per_step": head["e2e"]["h2d"], "d2h_bytes_per_step": head["e2e"]["d2h"],
                 "ms_per_step": head["e2e"]["ms"]},
         "gpu_launches": head["launches"] * args.steps,
-        "step": "252 linears (36 layers x 7) in one wr_gemv_batched launch, CUDA graph replay",
+        "step": f"{7 * args.layers} linears ({args.layers} layers x 7) in one wr_gemv_batched call "
+                "(preparation pass + decode GEMV launch), CUDA graph replay",
         "extras": extras,
     }
     if rank == 0:

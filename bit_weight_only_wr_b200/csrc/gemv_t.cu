@@ -1,9 +1,9 @@
 // Decode GEMV (M <= 8 tokens) for ternary weights on bf16 tensor cores, for one problem or a
 // batch of independent problems.
 //
-// The weights are ternary in a rotated basis ("Bitnet.cpp: Efficient Edge Inference for
-// Ternary LLMs", ternary weights; the random-sign block Hadamard is the rotation of the
-// ternary path): y[m,n] = alpha[n] sum_k t[n,k] (R x[m,:])[k]. The rotation pass has already
+// The weights are ternary (the news item on ternarizing Qwen3-4B to W1.58A16) in a rotated
+// basis ("How We Shrank an AI Model by 85%...", "Trick 1: rotate the weights first": store W R^T,
+// apply R to x): y[m,n] = alpha[n] sum_k t[n,k] (R x[m,:])[k]. The rotation pass has already
 // written, per 320-trit block, R x as hi + lo bf16 parts in B rows m and 8 + m; t is exact in
 // bf16, so the tensor cores see the exact product of t with hi + lo.
 //

@@ -25,8 +25,8 @@ What it defines (citations are to the source pages by title and section):
 * The packed byte layout (defined in ``include/wr.h``), re-implemented here from
   its written specification through explicit per-code index arithmetic.
 
-Readings where the pages are silent are listed in the design doc; the ones that
-change numbers are restated next to the code below.
+Where the pages are silent, the plainest reading is taken; each reading that changes
+numbers is stated next to the code below.
 """
 from __future__ import annotations
 
