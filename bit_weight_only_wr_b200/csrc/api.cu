@@ -55,6 +55,7 @@ wr_status check_dims(int64_t M, int64_t N, int64_t K) {
 }
 
 constexpr int kPlanSMs = 148;   // split heuristics are sized for a 148-SM part (device-independent)
+constexpr int kDecodeGrid = 3 * kPlanSMs;   // 2/3-bit decode: CTAs (block ranges) per launch, at most
 constexpr int kDecodeTokens = 8;   // decode kernel: 8 tokens x 4 activation limbs = 32 MMA columns
 
 // ---- decode kernel (M <= 8): work items (problem, 128-row group, block range) and workspace
@@ -92,8 +93,9 @@ void plan_decode(int64_t M, int count, const ProblemShape* shapes, DecodePlan* d
   }
   const int64_t target_items = std::max<int64_t>(3 * kPlanSMs, (total_blocks + 7) / 8);
   const double bpi = (double)total_blocks / (double)target_items;
+  const bool ternary = count > 0 && shapes[0].fmt == WR_FMT_TERNARY;
   int items = 0, counters = 0, blocks = 0;
-  int64_t partials = 0, xt_bytes = 0;
+  int64_t partials = 0, xt_bytes = 0, block_base = 0;
   for (int i = 0; i < count; ++i) {
     wr::DecProblem& pr = a.prob[i];
     int P = (int)std::lround((double)pr.B / bpi);
@@ -102,14 +104,19 @@ void plan_decode(int64_t M, int count, const ProblemShape* shapes, DecodePlan* d
     pr.counter_base = counters;
     pr.partial_base = partials;
     pr.xblk_base = blocks;
+    pr.block_base = block_base;
     items += pr.RG * pr.P;
     counters += pr.RG;
     blocks += pr.B;
-    if (pr.P > 1) partials += (int64_t)pr.RG * pr.P * M * 128;
+    block_base += (int64_t)pr.RG * pr.B;
+    if (ternary && pr.P > 1) partials += (int64_t)pr.RG * pr.P * M * 128;
     dp->xt_rel[i] = xt_bytes;
-    xt_bytes += (int64_t)pr.B * wr::xtile_bytes(shapes[i].fmt == WR_FMT_TERNARY, (int)M);
+    xt_bytes += (int64_t)pr.B * wr::xtile_bytes(ternary, (int)M);
   }
   a.items = items;
+  a.total = block_base;
+  // 2/3-bit: two partial slots per CTA of the launch (see DecArgs)
+  if (!ternary) partials = 2 * std::min<int64_t>(kDecodeGrid, block_base) * M * 128;
   dp->total_blocks = blocks;
   dp->counter_off = 0;
   dp->partial_off = align256((size_t)counters * sizeof(int));
@@ -134,7 +141,8 @@ wr_status run_decode(DecodePlan& dp, bool ternary, cudaStream_t stream) {
     const int grid = (int)std::min<int64_t>(dp.args.items, (int64_t)sm_count() * 2);
     return wr::launch_gemv_t(dp.args, grid, stream) == cudaSuccess ? WR_OK : WR_ERR_CUDA;
   }
-  const int grid = (int)std::min<int64_t>(dp.args.items, (int64_t)sm_count() * wr::gemv_q_ctas_per_sm());
+  // one contiguous block range per CTA; the partial slots were sized for this grid
+  const int grid = (int)std::min<int64_t>(dp.args.total, kDecodeGrid);
   if (wr::launch_prep_x(dp.args, dp.total_blocks, stream) != cudaSuccess) return WR_ERR_CUDA;
   return wr::launch_gemv_q(dp.args, grid, stream) == cudaSuccess ? WR_OK : WR_ERR_CUDA;
 }

@@ -3,8 +3,9 @@
 //
 // Decoding a token reads every weight once ("How We Shrank an AI Model by 85%...", section
 // "Results": generating a token is mostly reading the weights from memory), so the kernel is a
-// weight stream: each CTA walks a list of work items (problem, 128-row group, range of
-// 256-code blocks) and keeps its copy rings full across item and problem boundaries.
+// weight stream: the batch's blocks (problem by problem, 128-row group by row group, 256-code
+// block by block) are cut into one contiguous range per CTA, so every CTA streams the same
+// number of blocks and keeps its copy rings full across row-group and problem boundaries.
 //
 //   y[m,n] = sum_b s[n,b] sum_{k in b} g[n,k] x[m,k],   g = 2c - L  (L = 3 or 7)
 //
@@ -56,8 +57,7 @@ constexpr int kXOff = 0;                          // 1024-byte aligned (128-byte
 constexpr int kPOff = kXOff + kSX * kXStage;
 constexpr int kCOff = kPOff + kSP * kPStage;
 constexpr int kBarOff = kCOff + kSC * 256;
-constexpr int kBaseOff = kBarOff + 256;           // first work item of every problem (int[256])
-constexpr int kSmem = kBaseOff + 4 * kMaxDecodeProblems + 1024;   // + alignment slack
+constexpr int kSmem = kBarOff + 256 + 1024;        // + alignment slack
 static_assert(kCtasPerSm * (kSmem + 1024) <= 228 * 1024, "three CTAs per SM");
 constexpr int kACol = 0;                          // one block of codes: 256 bytes per lane
 constexpr int kDCol = 64;                         // two accumulators of N <= 32 columns
@@ -76,51 +76,86 @@ struct Bars {
 };
 static_assert(sizeof(Bars) <= 256, "barrier area");
 
-// Position in this CTA's sequence of (item, block) (items blockIdx.x, +gridDim.x, ...), with
-// the per-block fields of the item's problem held in registers: the problem table lives in the
-// kernel parameters, whose constant-cache misses cost hundreds of cycles, so it is read once
-// per item (and once more by the epilogue when the item ends).
-struct Cursor {
-  int it, b, b1, rg, p, pi;
-  int N, B, P, bits;
+// Position in this CTA's contiguous range of the batch's blocks (problem by problem, row group
+// by row group, K block by K block), with the fields of the current problem in registers: the
+// problem table lives in the kernel parameters, whose constant-cache misses cost hundreds of
+// cycles, so it is read only when the range crosses into the next problem.
+struct Pos {
+  int64_t g;            // global block
+  int left;             // blocks left in the range, this one included
+  int pi, rg, b;        // problem, row group, K block
+  int grg;              // global row group (arrival counter index)
+  int N, B, RG, bits;
   const uint8_t* packed;
   const uint8_t* xt;
   const uint16_t* scales;
+  float* y;
 };
 
-__device__ __forceinline__ void cursor_load(Cursor& c, const DecArgs& a, const int* base) {
-  if (c.it >= a.items) return;
+__device__ __forceinline__ int64_t range_start(int64_t T, int c) { return (int64_t)c * T / gridDim.x; }
+// CTA whose range holds global block g: the largest c with range_start(c) <= g
+__device__ __forceinline__ int cta_of(int64_t T, int64_t g) { return (int)(((g + 1) * gridDim.x - 1) / T); }
+
+__device__ __forceinline__ void pos_load(Pos& p, const DecArgs& a) {
+  const DecProblem& pr = a.prob[p.pi];
+  p.N = pr.N;
+  p.B = pr.B;
+  p.RG = pr.RG;
+  p.bits = pr.bits;
+  p.packed = pr.packed;
+  p.xt = pr.xt;
+  p.scales = pr.scales;
+  p.y = pr.y;
+}
+__device__ __forceinline__ Pos pos_start(const DecArgs& a) {
+  Pos p{};
+  p.g = range_start(a.total, blockIdx.x);
+  p.left = (int)(range_start(a.total, blockIdx.x + 1) - p.g);
+  if (p.left <= 0) return p;
   int lo = 0, hi = a.count - 1;
-  while (lo < hi) {  // last problem with item_base <= it
+  while (lo < hi) {  // last problem whose first block is <= g
     const int mid = (lo + hi + 1) >> 1;
-    if (base[mid] <= c.it) lo = mid;
+    if (a.prob[mid].block_base <= p.g) lo = mid;
     else hi = mid - 1;
   }
-  const DecProblem& pr = a.prob[lo];
-  c.pi = lo;
-  c.N = pr.N;
-  c.B = pr.B;
-  c.P = pr.P;
-  c.bits = pr.bits;
-  c.packed = pr.packed;
-  c.xt = pr.xt;
-  c.scales = pr.scales;
-  const int local = c.it - base[lo];
-  c.p = local % c.P;
-  c.rg = local / c.P;
-  c.b = (int)((int64_t)c.B * c.p / c.P);
-  c.b1 = (int)((int64_t)c.B * (c.p + 1) / c.P);
+  p.pi = lo;
+  pos_load(p, a);
+  const int64_t local = p.g - a.prob[lo].block_base;
+  p.rg = (int)(local / p.B);
+  p.b = (int)(local - (int64_t)p.rg * p.B);
+  p.grg = a.prob[lo].counter_base + p.rg;
+  return p;
 }
-__device__ __forceinline__ Cursor cursor_start(const DecArgs& a, const int* base) {
-  Cursor c{};
-  c.it = blockIdx.x;
-  cursor_load(c, a, base);
-  return c;
+__device__ __forceinline__ void pos_next(Pos& p, const DecArgs& a) {
+  ++p.g;
+  if (--p.left <= 0) return;
+  if (++p.b == p.B) {
+    p.b = 0;
+    ++p.grg;
+    if (++p.rg == p.RG) {
+      p.rg = 0;
+      ++p.pi;
+      pos_load(p, a);
+    }
+  }
 }
-__device__ __forceinline__ void cursor_next(Cursor& c, const DecArgs& a, const int* base) {
-  if (++c.b >= c.b1) {
-    c.it += gridDim.x;
-    cursor_load(c, a, base);
+
+// The decode side of the consumers needs only the block's format: a lighter position.
+struct Lite {
+  int left, pi, rg, b, B, RG, bits;
+};
+__device__ __forceinline__ Lite lite_of(const Pos& p) { return Lite{p.left, p.pi, p.rg, p.b, p.B, p.RG, p.bits}; }
+__device__ __forceinline__ void lite_next(Lite& p, const DecArgs& a) {
+  if (--p.left <= 0) return;
+  if (++p.b == p.B) {
+    p.b = 0;
+    if (++p.rg == p.RG) {
+      p.rg = 0;
+      ++p.pi;
+      p.B = a.prob[p.pi].B;
+      p.RG = a.prob[p.pi].RG;
+      p.bits = a.prob[p.pi].bits;
+    }
   }
 }
 
@@ -194,13 +229,11 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_q_kernel(const __gr
   uint8_t* ps = smem + kPOff;
   uint8_t* cs = smem + kCOff;
   Bars* bars = reinterpret_cast<Bars*>(smem + kBarOff);
-  int* base = reinterpret_cast<int*>(smem + kBaseOff);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   volatile int* abort_flag = &bars->abort_flag;
   constexpr int kSlots = XR / 4;       // token slots
   const int M = a.M;
 
-  for (int i = threadIdx.x; i < a.count; i += kThreads) base[i] = a.prob[i].item_base;
   if (threadIdx.x == 0) {
     for (int i = 0; i < kSP; ++i) {
       mbar_init(&bars->pk_full[i], 1);
@@ -231,7 +264,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_q_kernel(const __gr
     if (lane == 0) {
       uint32_t np = 0;
       bool ok = true;
-      for (Cursor c = cursor_start(a, base); c.it < a.items; cursor_next(c, a, base), ++np) {
+      for (Pos c = pos_start(a); c.left > 0; pos_next(c, a), ++np) {
         // the ntile units of this row group and block are adjacent: one copy
         const int ub = c.bits == 2 ? 1024 : 1536;
         const int ntile = min(8, (c.N + 15) / 16 - c.rg * 8);
@@ -252,7 +285,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_q_kernel(const __gr
       constexpr uint32_t xtb = bbytes + 256u;   // prepared tile: B atoms, then corrections
       uint32_t nx = 0, nc = 0;   // B and correction copies issued
       bool ok = true;
-      for (Cursor c = cursor_start(a, base); c.it < a.items; cursor_next(c, a, base)) {
+      for (Pos c = pos_start(a); c.left > 0; pos_next(c, a)) {
         const uint8_t* xsrc = c.xt + (int64_t)c.b * xtb;
         const int sx = nx % kSX, sc = nc % kSC;
         if (!(ok = mbar_wait_bg(&bars->mma_done[sx], ((nx / kSX) & 1) ^ 1, abort_flag, a.err, 102))) break;
@@ -274,9 +307,11 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_q_kernel(const __gr
     const uint64_t bdesc0 = smem_desc_sw128(xs);
     constexpr uint32_t idesc = idesc_i8_m128(XR);
     constexpr uint32_t atom16 = (uint32_t)(XR * 128) >> 4;
+    const int64_t span = range_start(a.total, blockIdx.x + 1) - range_start(a.total, blockIdx.x);
+    const uint32_t nblocks = span > 0 ? (uint32_t)span : 0u;
     uint32_t gm = 0;
     bool ok = true;
-    for (Cursor c = cursor_start(a, base); c.it < a.items; cursor_next(c, a, base), ++gm) {
+    for (; gm < nblocks; ++gm) {
       const int sx = gm % kSX;
       if (!(ok = mbar_wait_bg(&bars->a_full, gm & 1, abort_flag, a.err, 201))) break;
       if (!(ok = mbar_wait_bg(&bars->x_full[sx], (gm / kSX) & 1, abort_flag, a.err, 202))) break;
@@ -308,7 +343,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_q_kernel(const __gr
     };
     // finish block ge (cursor ec): its accumulator (buffer ge % 2, loaded here in chunks of up
     // to 4 token slots), its correction record and its scale
-    auto finish = [&](const Cursor& ec, uint32_t ge, uint16_t sraw) -> bool {
+    auto finish = [&](const Pos& ec, uint32_t ge, uint16_t sraw) -> bool {
       const int sc = ge % kSC;
       if (!mbar_wait(&bars->c_full[sc], (ge / kSC) & 1, abort_flag, a.err, 303)) return false;
       const int4* rec = reinterpret_cast<const int4*>(cs + sc * 256);
@@ -335,34 +370,39 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_q_kernel(const __gr
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->c_empty[sc]);
-      if (ec.b + 1 < ec.b1) return true;
-      // last block of the item: y, or the split-K combine through the workspace
+      if (ec.b + 1 < ec.B && ec.left > 1) return true;
+      // the row group ends here (or this range does): y, or, for a row group that several CTA
+      // ranges share, the combine through the partial slots (the last range to arrive adds
+      // the pieces in range order)
       const int n = ec.rg * 128 + t;
-      float* y = a.prob[ec.pi].y;
-      if (ec.P == 1) {
+      const int64_t T = a.total;
+      const int64_t g0 = ec.g - ec.b;                     // first block of the row group
+      const int c0 = cta_of(T, g0), c1 = cta_of(T, g0 + ec.B - 1);
+      if (c0 == c1) {
         if (n < ec.N) {
 #pragma unroll
           for (int m = 0; m < kSlots; ++m)
-            if (m < M) y[(int64_t)m * ec.N + n] = acc[m];
+            if (m < M) ec.y[(int64_t)m * ec.N + n] = acc[m];
         }
       } else {
-        const int cid = a.prob[ec.pi].counter_base + ec.rg;
-        const int64_t pbase = a.prob[ec.pi].partial_base;
-        float* part = a.partial + pbase + ((int64_t)ec.rg * ec.P + ec.p) * M * 128;
+        // slot 0: the row group began before this range; slot 1: it continues after it
+        const int slot = g0 < range_start(T, blockIdx.x) ? 0 : 1;
+        float* part = a.partial + ((int64_t)2 * blockIdx.x + slot) * M * 128;
 #pragma unroll
         for (int m = 0; m < kSlots; ++m)
           if (m < M) part[m * 128 + t] = acc[m];
         __threadfence();
         if (!group_sync(304)) return false;
-        if (t == 0) bars->last_flag = (atomicAdd(a.counter + cid, 1) == ec.P - 1);
+        if (t == 0) bars->last_flag = (atomicAdd(a.counter + ec.grg, 1) == c1 - c0);
         if (!group_sync(305)) return false;
         if (bars->last_flag) {
           __threadfence();
           float sum[kSlots];
 #pragma unroll
           for (int m = 0; m < kSlots; ++m) sum[m] = 0.f;
-          for (int pp = 0; pp < ec.P; ++pp) {
-            const float* src = a.partial + pbase + ((int64_t)ec.rg * ec.P + pp) * M * 128;
+          for (int c = c0; c <= c1; ++c) {
+            const int sl = g0 < range_start(T, c) ? 0 : 1;
+            const float* src = a.partial + ((int64_t)2 * c + sl) * M * 128;
 #pragma unroll
             for (int m = 0; m < kSlots; ++m)
               if (m < M) sum[m] += __ldcg(src + m * 128 + t);
@@ -370,24 +410,25 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_q_kernel(const __gr
           if (n < ec.N) {
 #pragma unroll
             for (int m = 0; m < kSlots; ++m)
-              if (m < M) y[(int64_t)m * ec.N + n] = sum[m];
+              if (m < M) ec.y[(int64_t)m * ec.N + n] = sum[m];
           }
-          if (t == 0) a.counter[cid] = 0;
+          if (t == 0) a.counter[ec.grg] = 0;
         }
       }
 #pragma unroll
       for (int m = 0; m < kSlots; ++m) acc[m] = 0.f;
       return true;
     };
-    auto scale_of = [&](const Cursor& c) -> uint16_t {
+    auto scale_of = [&](const Pos& c) -> uint16_t {
       const int n = c.rg * 128 + t;
       return n < c.N ? __ldg(c.scales + (int64_t)n * c.B + c.b) : (uint16_t)0;
     };
 
-    Cursor dc = cursor_start(a, base), ec = dc;   // block being decoded, block being finished
+    Pos ec = pos_start(a);     // block being finished
+    Lite dc = lite_of(ec);     // block being decoded
     uint32_t gd = 0;
     bool ok = true;
-    for (; dc.it < a.items; ++gd) {
+    for (; dc.left > 0; ++gd) {
       const uint16_t sraw = gd > 0 ? scale_of(ec) : (uint16_t)0;   // block gd - 1
       const int sp = gd % kSP;
       if (!(ok = mbar_wait(&bars->pk_full[sp], (gd / kSP) & 1, abort_flag, a.err, 301))) break;
@@ -409,10 +450,10 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_q_kernel(const __gr
       fence_before_sync();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->a_full);
-      cursor_next(dc, a, base);
+      lite_next(dc, a);
       if (gd > 0) {
         if (!(ok = finish(ec, gd - 1, sraw))) break;
-        cursor_next(ec, a, base);
+        pos_next(ec, a);
       }
     }
     if (ok && gd > 0) {
@@ -526,7 +567,10 @@ cudaError_t launch_xr(const DecArgs& a, int grid, cudaStream_t stream) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
   if (!set[dev]) {
-    const cudaError_t e = cudaFuncSetAttribute(gemv_q_kernel<XR>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
+    cudaError_t e = cudaFuncSetAttribute(gemv_q_kernel<XR>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
+    // all of the unified L1/shared array as shared memory, so that three CTAs fit
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(gemv_q_kernel<XR>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
     if (e != cudaSuccess) return e;
     set[dev] = true;
   }
@@ -536,6 +580,14 @@ cudaError_t launch_xr(const DecArgs& a, int grid, cudaStream_t stream) {
 }  // namespace
 
 int gemv_q_ctas_per_sm() { return kCtasPerSm; }
+
+int gemv_q_occupancy(int M) {
+  int n = 0;
+  const cudaError_t e = decode_xrows(M) == 8 ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, gemv_q_kernel<8>, kThreads, kSmem)
+                      : decode_xrows(M) == 16 ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, gemv_q_kernel<16>, kThreads, kSmem)
+                                              : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, gemv_q_kernel<32>, kThreads, kSmem);
+  return e == cudaSuccess ? n : -1;
+}
 
 cudaError_t launch_gemv_q(const DecArgs& a, int grid, cudaStream_t stream) {
   switch (decode_xrows(a.M)) {

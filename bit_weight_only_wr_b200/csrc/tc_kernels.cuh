@@ -34,12 +34,19 @@ struct DecProblem {
   int B, RG, P, bits;        // blocks per row, 128-row groups, K splits, 2/3 (ternary: 1)
   int item_base;             // first work item of this problem
   int xblk_base;             // first block of this problem in the preparation pass
-  int counter_base;          // first arrival counter of this problem
-  int64_t partial_base;      // first partial float of this problem
+  int counter_base;          // first arrival counter (row group) of this problem
+  int64_t partial_base;      // first partial float of this problem (ternary items)
+  int64_t block_base;        // first block of this problem in the batch's block sequence (2/3-bit)
 };
 
+// 2/3-bit: the batch's blocks (problem by problem, row group by row group, K block by K block)
+// are cut into gridDim.x contiguous ranges, one per CTA: CTA c takes [c T / G, (c+1) T / G).
+// A row group cut by a range boundary is finished through per-CTA partial slots (two per CTA:
+// the row group that started before the range, and the one that ends after it).
+// Ternary: work items (problem, row group, range of blocks), items c, c + G, ... per CTA.
 struct DecArgs {
   int count, M, items, pad;
+  int64_t total;             // 2/3-bit: blocks of the batch (T)
   float* partial;
   int* counter;
   int* err;
@@ -49,7 +56,8 @@ struct DecArgs {
 // 2/3-bit decode: the preparation pass writes the B tiles, then the GEMV kernel.
 cudaError_t launch_prep_x(const DecArgs& a, int total_blocks, cudaStream_t stream);
 cudaError_t launch_gemv_q(const DecArgs& a, int grid, cudaStream_t stream);
-int gemv_q_ctas_per_sm();   // CTAs of the 2/3-bit decode kernel that share an SM
+int gemv_q_ctas_per_sm();   // CTAs of the 2/3-bit decode kernel that share an SM (by design)
+int gemv_q_occupancy(int M);  // CTAs per SM the runtime reports for it (needs the opt-in smem set)
 // Ternary decode (tiles written by launch_rotate_x).
 cudaError_t launch_gemv_t(const DecArgs& a, int grid, cudaStream_t stream);
 
