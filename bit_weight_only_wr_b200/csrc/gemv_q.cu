@@ -19,17 +19,16 @@
 // multiple of 2^E: at most 2^-30 max|x| per element.
 //
 // A CTA is one small pipeline; three run on every SM so that their latency chains overlap
-// (warp roles, 224 threads):
+// (warp roles, 160 threads):
 //   warps 0-3  consumers, thread = weight row (TMEM lane 32 w + lane). Per block: decode the
 //              row's 256 codes into the A buffer (two 32-column tensor-memory stores), hand it
-//              to the MMA warp, then turn the previous block's accumulator into fp32 partial
-//              dot products times s[n,b] (all tokens of the row).
-//   warp 4     packed-weight producer: per block one bulk copy of the 8 units of the row
-//              group; it runs a full ring ahead of the consumers.
-//   warp 5     activation producer: per block one bulk copy of the prepared B tile and one of
-//              its correction record.
-//   warp 6     allocates tensor memory and issues the 8 MMAs and one commit per block (whole
-//              warp walks the blocks, one elected lane issues).
+//              to the control warp, then turn the previous block's accumulator into fp32
+//              partial dot products times s[n,b] (all tokens of the row).
+//   warp 4     control: allocates tensor memory; issues the bulk copies of the packed weights
+//              (one per block, a ring of kSP blocks ahead), of the prepared B tiles and their
+//              correction records (two blocks ahead), and the 8 MMAs and one commit per block
+//              (the whole warp walks the blocks, one elected lane issues). One warp instead of
+//              three leaves the consumers more registers.
 // Tensor memory (128 columns): one A buffer (64 columns) and two accumulators (32 columns). The
 // store of block i waits for the MMAs of block i - 1; block i's MMAs write accumulator i % 2
 // while the consumers finish block i - 1 from the other one. Every wait is bounded.
@@ -46,7 +45,7 @@ namespace {
 
 using namespace tc;
 
-constexpr int kThreads = 224;
+constexpr int kThreads = 160;
 constexpr int kCtasPerSm = 3;
 constexpr int kSP = 4;   // packed stages: 8 units of up to 1.5 KB
 constexpr int kSX = 2;   // B tiles (up to 2 atoms x 32 rows x 128 bytes); also the MMA-done ring
@@ -253,68 +252,57 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_q_kernel(const __gr
     bars->last_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 6) tmem_alloc(&bars->tmem_base, kTmemCols);
+  if (warp == 4) tmem_alloc(&bars->tmem_base, kTmemCols);
   fence_before_sync();
   __syncthreads();
   fence_after_sync();
   const uint32_t tmem = bars->tmem_base;
 
   if (warp == 4) {
-    // ------------------------------------------------------------ packed-weight producer (one thread)
-    if (lane == 0) {
-      uint32_t np = 0;
-      bool ok = true;
-      for (Pos c = pos_start(a); c.left > 0; pos_next(c, a), ++np) {
-        // the ntile units of this row group and block are adjacent: one copy
-        const int ub = c.bits == 2 ? 1024 : 1536;
-        const int ntile = min(8, (c.N + 15) / 16 - c.rg * 8);
-        const int sp = np % kSP;
-        if (!(ok = mbar_wait_bg(&bars->pk_empty[sp], ((np / kSP) & 1) ^ 1, abort_flag, a.err, 101))) break;
-        mbar_arrive_expect_tx(&bars->pk_full[sp], ntile * ub);
-        bulk_load(ps + sp * kPStage, c.packed + ((int64_t)c.rg * 8 * c.B + (int64_t)c.b * ntile) * ub, ntile * ub,
-                  &bars->pk_full[sp]);
-      }
-      // aborted: let the copies in flight land before the CTA exits
-      if (!ok)
-        for (uint32_t k = np > kSP ? np - kSP : 0; k < np; ++k) mbar_wait_drain(&bars->pk_full[k % kSP], (k / kSP) & 1);
-    }
-  } else if (warp == 5) {
-    // ------------------------------------------------------------ activation producer (one thread)
-    if (lane == 0) {
-      constexpr uint32_t bbytes = 256u * XR;
-      constexpr uint32_t xtb = bbytes + 256u;   // prepared tile: B atoms, then corrections
-      uint32_t nx = 0, nc = 0;   // B and correction copies issued
-      bool ok = true;
-      for (Pos c = pos_start(a); c.left > 0; pos_next(c, a)) {
-        const uint8_t* xsrc = c.xt + (int64_t)c.b * xtb;
-        const int sx = nx % kSX, sc = nc % kSC;
-        if (!(ok = mbar_wait_bg(&bars->mma_done[sx], ((nx / kSX) & 1) ^ 1, abort_flag, a.err, 102))) break;
-        mbar_arrive_expect_tx(&bars->x_full[sx], bbytes);
-        bulk_load(xs + sx * kXStage, xsrc, bbytes, &bars->x_full[sx]);
-        ++nx;
-        if (!(ok = mbar_wait_bg(&bars->c_empty[sc], ((nc / kSC) & 1) ^ 1, abort_flag, a.err, 103))) break;
-        mbar_arrive_expect_tx(&bars->c_full[sc], 256);
-        bulk_load(cs + sc * 256, xsrc + bbytes, 256, &bars->c_full[sc]);
-        ++nc;
-      }
-      if (!ok) {
-        for (uint32_t k = nx > kSX ? nx - kSX : 0; k < nx; ++k) mbar_wait_drain(&bars->x_full[k % kSX], (k / kSX) & 1);
-        for (uint32_t k = nc > kSC ? nc - kSC : 0; k < nc; ++k) mbar_wait_drain(&bars->c_full[k % kSC], (k / kSC) & 1);
-      }
-    }
-  } else if (warp == 6) {
-    // ------------------------------------------------------------ MMA issuer (whole warp, one lane issues)
+    // ------------------------------------------------------------ control warp (whole warp walks the
+    // blocks, one elected lane issues): weight copies kSP blocks ahead, activation copies two ahead,
+    // and the MMAs of each block once the consumers have stored its codes.
+    constexpr uint32_t bbytes = 256u * XR;
+    constexpr uint32_t xtb = bbytes + 256u;   // prepared tile: B atoms, then corrections
     const uint64_t bdesc0 = smem_desc_sw128(xs);
     constexpr uint32_t idesc = idesc_i8_m128(XR);
     constexpr uint32_t atom16 = (uint32_t)(XR * 128) >> 4;
-    const int64_t span = range_start(a.total, blockIdx.x + 1) - range_start(a.total, blockIdx.x);
-    const uint32_t nblocks = span > 0 ? (uint32_t)span : 0u;
-    uint32_t gm = 0;
+    Pos cp = pos_start(a), cx = cp;            // next block to copy: weights, activations
+    const uint32_t nblocks = cp.left > 0 ? (uint32_t)cp.left : 0u;
+    uint32_t np = 0, nx = 0, gm = 0;           // weight copies, activation copies, MMAs issued
     bool ok = true;
+    auto copy_weights = [&]() {                // block np into stage np % kSP (free: caller waited)
+      const int ub = cp.bits == 2 ? 1024 : 1536;
+      const int ntile = min(8, (cp.N + 15) / 16 - cp.rg * 8);
+      const int sp = np % kSP;
+      if (elect_one()) {
+        mbar_arrive_expect_tx(&bars->pk_full[sp], ntile * ub);
+        bulk_load(ps + sp * kPStage, cp.packed + ((int64_t)cp.rg * 8 * cp.B + (int64_t)cp.b * ntile) * ub,
+                  ntile * ub, &bars->pk_full[sp]);
+      }
+      __syncwarp();
+      pos_next(cp, a);
+      ++np;
+    };
+    auto copy_acts = [&]() {                   // block nx: B tile into stage nx % kSX, corrections
+      const uint8_t* xsrc = cx.xt + (int64_t)cx.b * xtb;
+      const int sx = nx % kSX, sc = nx % kSC;
+      if (elect_one()) {
+        mbar_arrive_expect_tx(&bars->x_full[sx], bbytes);
+        bulk_load(xs + sx * kXStage, xsrc, bbytes, &bars->x_full[sx]);
+        mbar_arrive_expect_tx(&bars->c_full[sc], 256);
+        bulk_load(cs + sc * 256, xsrc + bbytes, 256, &bars->c_full[sc]);
+      }
+      __syncwarp();
+      pos_next(cx, a);
+      ++nx;
+    };
+    while (np < nblocks && np < (uint32_t)kSP) copy_weights();   // the rings start empty
+    while (nx < nblocks && nx < (uint32_t)kSX) copy_acts();
     for (; gm < nblocks; ++gm) {
       const int sx = gm % kSX;
-      if (!(ok = mbar_wait_bg(&bars->a_full, gm & 1, abort_flag, a.err, 201))) break;
-      if (!(ok = mbar_wait_bg(&bars->x_full[sx], (gm / kSX) & 1, abort_flag, a.err, 202))) break;
+      if (!(ok = mbar_wait(&bars->a_full, gm & 1, abort_flag, a.err, 201))) break;
+      if (!(ok = mbar_wait(&bars->x_full[sx], (gm / kSX) & 1, abort_flag, a.err, 202))) break;
       fence_after_sync();
       const uint64_t bd = bdesc0 + (uint64_t)((sx * kXStage) >> 4);
 #pragma unroll
@@ -324,9 +312,25 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_q_kernel(const __gr
         mma_ts_i8_elect(tmem + kDCol + (gm & 1) * kDCols, tmem + kACol + 8 * j, bd + off, idesc, j != 0);
       }
       mma_commit_elect(&bars->mma_done[sx]);
+      // the consumers released weight stage gm % kSP before they released block gm to us
+      if (np < nblocks) {
+        if (!(ok = mbar_wait(&bars->pk_empty[np % kSP], ((np / kSP) & 1) ^ 1, abort_flag, a.err, 203))) break;
+        copy_weights();
+      }
+      // activation stage gm % kSX is free once block gm's MMAs are done
+      if (nx < nblocks) {
+        if (!(ok = mbar_wait_bg(&bars->mma_done[nx % kSX], ((nx / kSX) & 1) ^ 1, abort_flag, a.err, 204))) break;
+        if (!(ok = mbar_wait_bg(&bars->c_empty[nx % kSC], ((nx / kSC) & 1) ^ 1, abort_flag, a.err, 205))) break;
+        copy_acts();
+      }
     }
-    // the MMAs already issued finish before tensor memory is released
-    if (!ok && gm > 0) mbar_wait_drain(&bars->mma_done[(gm - 1) % kSX], ((gm - 1) / kSX) & 1);
+    if (!ok) {
+      // aborted: let the copies and MMAs in flight land before the CTA exits
+      for (uint32_t k = np > kSP ? np - kSP : 0; k < np; ++k) mbar_wait_drain(&bars->pk_full[k % kSP], (k / kSP) & 1);
+      for (uint32_t k = nx > kSX ? nx - kSX : 0; k < nx; ++k) mbar_wait_drain(&bars->x_full[k % kSX], (k / kSX) & 1);
+      for (uint32_t k = nx > kSC ? nx - kSC : 0; k < nx; ++k) mbar_wait_drain(&bars->c_full[k % kSC], (k / kSC) & 1);
+      if (gm > 0) mbar_wait_drain(&bars->mma_done[(gm - 1) % kSX], ((gm - 1) / kSX) & 1);
+    }
   } else {
     // ------------------------------------------------------------ consumers (warps 0-3, thread = row)
     const int t = threadIdx.x;                          // row in the row group = TMEM lane
@@ -469,7 +473,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_q_kernel(const __gr
   fence_before_sync();
   __syncthreads();
   fence_after_sync();
-  if (warp == 6) tmem_dealloc(tmem, kTmemCols);
+  if (warp == 4) tmem_dealloc(tmem, kTmemCols);
 }
 
 // Preparation pass: one warp per (problem, block, token slot m < N/4). The block's activations

@@ -186,6 +186,13 @@ __device__ __forceinline__ void mma_ts_i8(uint32_t d_tmem, uint32_t a_tmem, uint
       : "memory");
 }
 
+// True in one lane of the (converged) warp, chosen by elect.sync.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred;
+  asm volatile("{\n .reg .pred p;\n elect.sync _|p, 0xffffffff;\n selp.u32 %0, 1, 0, p;\n}" : "=r"(pred));
+  return pred != 0;
+}
+
 // Warp-wide forms: every lane of the warp executes the call with the same operands (so the
 // descriptor arithmetic stays warp-uniform) and one lane chosen by elect.sync issues the
 // instruction. Issuing from a loop that only lane 0 runs measured about three times slower.
