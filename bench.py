@@ -490,6 +490,24 @@ def run_extras(args, wr, torch, np, stream, dist, hbm_peak, bf16_peak):
             fl = sum(2.0 * M * m["N"] * m["K"] for m in mods)
             res[f"layer_M{M}"] = {"us": ms * 1e3, "gbs": b / ms / 1e6, "tflops": fl / ms / 1e9,
                                   "tokens_per_s_layer": M * 1e3 / ms}
+        # the 36-layer ternary body in one wr_gemv_ternary_batched call per token (36 distinct
+        # copies of the quantized layer, 731 MB, far above L2)
+        body = [(mods[i], m["p"].roll(c * 4096)) for c in range(36) for i, m in enumerate(mods)]
+        for M in (1, 8):
+            xs = [torch.from_numpy(wr_synth.activations_bf16(3000 + j, M, m["K"]).view(np.int16)).cuda()
+                  for j, (m, _) in enumerate(body)]
+            ys = [torch.empty(M, m["N"], dtype=torch.float32, device="cuda") for m, _ in body]
+            arr = wr._tproblems([(xs[j], pk, m["a"], m["s"], ys[j], m["N"], m["K"]) for j, (m, pk) in enumerate(body)])
+            nb = wr.wr_gemv_ternary_batched_workspace_bytes(M, arr)
+            ws = torch.zeros(nb, dtype=torch.uint8, device="cuda")
+
+            def tstep():
+                wr.wr_gemv_ternary_batched(M, arr, ws, nb)
+            ms = graph_time_ms(torch, tstep, 10, 3, stream) / 10
+            b = sum(pk.numel() + 2 * m["N"] + 4 * ((m["K"] + 31) // 32) + 2 * M * m["K"] + 4 * M * m["N"]
+                    for m, pk in body)
+            res[f"body_M{M}"] = {"ms": ms, "bytes": b, "gbs": b / ms / 1e6, "tokens_per_s": M * 1e3 / ms,
+                                 "launches": 2}
         out["ternary"] = res
     except Exception as e:  # noqa: BLE001
         out["ternary"] = {"error": repr(e)}

@@ -18,7 +18,8 @@ __all__ = [
     "wr_quantize", "wr_quantize_ternary", "wr_unpack_bf16", "wr_gemv_workspace_bytes", "wr_gemv",
     "wr_gemm_workspace_bytes", "wr_gemm", "wr_gemm_ternary_workspace_bytes", "wr_gemm_ternary",
     "wr_get_device_error", "exported_symbols", "WrGemvProblem", "wr_gemv_batched_workspace_bytes",
-    "wr_gemv_batched", "wr_gemv_noalloc", "WR_GEMV_NOALLOC_SCRATCH_BYTES",
+    "wr_gemv_batched", "wr_gemv_noalloc", "WR_GEMV_NOALLOC_SCRATCH_BYTES", "WrGemvTernaryProblem",
+    "wr_gemv_ternary_batched_workspace_bytes", "wr_gemv_ternary_batched",
 ]
 
 WR_FMT_TERNARY, WR_FMT_Q2, WR_FMT_Q3 = 1, 2, 3
@@ -35,6 +36,16 @@ class WrGemvProblem(ctypes.Structure):
 
 
 _PROBLEMS = ctypes.POINTER(WrGemvProblem)
+
+
+class WrGemvTernaryProblem(ctypes.Structure):
+    """Mirror of the C struct wr_gemv_ternary_problem."""
+    _fields_ = [("x", ctypes.c_void_p), ("packed", ctypes.c_void_p), ("alpha", ctypes.c_void_p),
+                ("sign_bits", ctypes.c_void_p), ("y", ctypes.c_void_p), ("N", ctypes.c_int64),
+                ("K", ctypes.c_int64)]
+
+
+_TPROBLEMS = ctypes.POINTER(WrGemvTernaryProblem)
 
 _SIGNATURES = {
     "wr_abi_version": (_c_int, []),
@@ -55,6 +66,8 @@ _SIGNATURES = {
     "wr_gemm_ternary": (_c_int, [_c_i64, _c_i64, _c_i64, _vp, _vp, _vp, _vp, _vp, _vp, _c_size, _vp]),
     "wr_get_device_error": (_c_int, [_vp]),
     "wr_gemv_noalloc": (_c_int, [_c_i64, _c_i64, _c_i64, _vp, _vp, _vp, _c_int, _c_int, _vp, _vp]),
+    "wr_gemv_ternary_batched_workspace_bytes": (_c_size, [_c_i64, ctypes.c_int32, _TPROBLEMS]),
+    "wr_gemv_ternary_batched": (_c_int, [_c_i64, ctypes.c_int32, _TPROBLEMS, _vp, _c_size, _vp]),
 }
 
 
@@ -201,6 +214,26 @@ def wr_gemv_batched(M: int, problems, workspace, workspace_bytes: int, stream=No
     arr = problems if isinstance(problems, ctypes.Array) else _problems(problems)
     _check("wr_gemv_batched", _lib.wr_gemv_batched(M, len(arr), arr, _ptr(workspace), workspace_bytes,
                                                    _stream(stream)))
+
+
+def _tproblems(problems):
+    """problems: sequence of (x, packed, alpha, sign_bits, y, N, K) -> ctypes array."""
+    arr = (WrGemvTernaryProblem * len(problems))()
+    for i, (x, packed, alpha, signs, y, N, K) in enumerate(problems):
+        arr[i] = WrGemvTernaryProblem(_ptr(x), _ptr(packed), _ptr(alpha), _ptr(signs), _ptr(y), N, K)
+    return arr
+
+
+def wr_gemv_ternary_batched_workspace_bytes(M: int, problems) -> int:
+    arr = problems if isinstance(problems, ctypes.Array) else _tproblems(problems)
+    return _lib.wr_gemv_ternary_batched_workspace_bytes(M, len(arr), arr)
+
+
+def wr_gemv_ternary_batched(M: int, problems, workspace, workspace_bytes: int, stream=None) -> None:
+    """problems: sequence of (x, packed, alpha, sign_bits, y, N, K), or a prepared ctypes array."""
+    arr = problems if isinstance(problems, ctypes.Array) else _tproblems(problems)
+    _check("wr_gemv_ternary_batched", _lib.wr_gemv_ternary_batched(M, len(arr), arr, _ptr(workspace),
+                                                                   workspace_bytes, _stream(stream)))
 
 
 def wr_gemm_workspace_bytes(M: int, N: int, K: int, bits: int) -> int:

@@ -394,6 +394,61 @@ wr_status wr_gemv_batched(int64_t M, int32_t count, const wr_gemv_problem* probl
   return WR_OK;
 }
 
+static bool tbatch_ok(int64_t M, int32_t count, const wr_gemv_ternary_problem* pr) {
+  if (M < 1 || M > 8 || count < 1 || !pr) return false;
+  for (int i = 0; i < count; ++i) {
+    if (check_dims(M, pr[i].N, pr[i].K) != WR_OK || pr[i].K % 128 != 0) return false;
+    if (!aligned16(pr[i].x) || !aligned16(pr[i].packed) || !aligned16(pr[i].alpha) || !aligned16(pr[i].sign_bits) ||
+        !aligned16(pr[i].y))
+      return false;
+  }
+  return true;
+}
+
+size_t wr_gemv_ternary_batched_workspace_bytes(int64_t M, int32_t count, const wr_gemv_ternary_problem* problems) {
+  if (!tbatch_ok(M, count, problems)) return 0;
+  size_t total = 0;
+  static thread_local DecodePlan dp;
+  ProblemShape sh[wr::kMaxDecodeProblems];
+  for (int c0 = 0; c0 < count; c0 += wr::kMaxDecodeProblems) {
+    const int n = std::min(count - c0, wr::kMaxDecodeProblems);
+    for (int i = 0; i < n; ++i) sh[i] = ProblemShape{problems[c0 + i].N, problems[c0 + i].K, WR_FMT_TERNARY};
+    plan_decode(M, n, sh, &dp);
+    total = std::max(total, dp.total);
+  }
+  return total;
+}
+
+wr_status wr_gemv_ternary_batched(int64_t M, int32_t count, const wr_gemv_ternary_problem* problems,
+                                  void* workspace, size_t workspace_bytes, void* stream) {
+  if (!tbatch_ok(M, count, problems) || !aligned16(workspace)) return WR_ERR_INVALID_ARG;
+  if (workspace_bytes < wr_gemv_ternary_batched_workspace_bytes(M, count, problems)) return WR_ERR_INVALID_ARG;
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  static thread_local DecodePlan dp;
+  ProblemShape sh[wr::kMaxDecodeProblems];
+  for (int c0 = 0; c0 < count; c0 += wr::kMaxDecodeProblems) {
+    const int n = std::min(count - c0, wr::kMaxDecodeProblems);
+    for (int i = 0; i < n; ++i) sh[i] = ProblemShape{problems[c0 + i].N, problems[c0 + i].K, WR_FMT_TERNARY};
+    plan_decode(M, n, sh, &dp);
+    int64_t rot_items = 0;
+    for (int i = 0; i < n; ++i) {
+      wr::DecProblem& pr = dp.args.prob[i];
+      pr.x = problems[c0 + i].x;
+      pr.packed = static_cast<const uint8_t*>(problems[c0 + i].packed);
+      pr.scales = problems[c0 + i].alpha;
+      pr.signs = problems[c0 + i].sign_bits;
+      pr.y = problems[c0 + i].y;
+      pr.xblk_base = (int)rot_items;   // rotation work items: (token, 128-block)
+      rot_items += M * (((int64_t)pr.Kp + 127) / 128);
+    }
+    bind_workspace(dp, workspace);
+    if (wr::launch_rotate_x_batched(dp.args, rot_items, s) != cudaSuccess) return WR_ERR_CUDA;
+    const wr_status st = run_decode(dp, true, s);
+    if (st != WR_OK) return st;
+  }
+  return WR_OK;
+}
+
 size_t wr_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int bits) {
   if (bits != 2 && bits != 3) return 0;
   if (check_dims(M, N, K) != WR_OK || K % 256 != 0) return 0;

@@ -473,14 +473,10 @@ cudaError_t launch_tc(const TcArgs& a, const void* x_act, int64_t x_rows, int64_
 // hi of token m in row m, lo in row 8 + m (128-byte swizzle: 16-byte chunk c of row r at
 // c ^ (r % 8)). Position 80q + 2P + h of a unit holds trit 80q + 5*(2*(P/5) + h) + P%5 (pair P
 // of byte pair P/5; h selects the byte), the K order of the decoded A columns. Pad trits get 0.
-__global__ void rotate_x_kernel(const uint16_t* __restrict__ x, const uint32_t* __restrict__ signs,
-                                uint8_t* __restrict__ xt, int M, int K, int64_t Kp) {
-  const int lane = threadIdx.x & 31;
-  const int64_t item = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  const int64_t nblk = (Kp + 127) / 128;
-  if (item >= (int64_t)M * nblk) return;
-  const int m = (int)(item / nblk);
-  const int64_t k0 = (item % nblk) * 128;
+// One warp: token m, 128-block starting at k0 (lane = 4 consecutive K positions).
+__device__ __forceinline__ void rotate_block(const uint16_t* __restrict__ x, const uint32_t* __restrict__ signs,
+                                             uint8_t* __restrict__ xt, int K, int64_t Kp, int m, int64_t k0,
+                                             int lane) {
   float v[4];
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
@@ -521,6 +517,31 @@ __global__ void rotate_x_kernel(const uint16_t* __restrict__ x, const uint32_t* 
   }
 }
 
+__global__ void rotate_x_kernel(const uint16_t* __restrict__ x, const uint32_t* __restrict__ signs,
+                                uint8_t* __restrict__ xt, int M, int K, int64_t Kp) {
+  const int lane = threadIdx.x & 31;
+  const int64_t item = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int64_t nblk = (Kp + 127) / 128;
+  if (item >= (int64_t)M * nblk) return;
+  rotate_block(x, signs, xt, K, Kp, (int)(item / nblk), (item % nblk) * 128, lane);
+}
+
+// Batched form: work item g -> (problem, token, 128-block) through the problems' first items.
+__global__ void rotate_x_batched_kernel(const __grid_constant__ DecArgs a, int64_t total_items) {
+  const int lane = threadIdx.x & 31;
+  const int64_t g = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (g >= total_items) return;
+  int lo = 0, hi = a.count - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (a.prob[mid].xblk_base <= g) lo = mid;
+    else hi = mid - 1;
+  }
+  const DecProblem& pr = a.prob[lo];
+  const int64_t local = g - pr.xblk_base, nblk = ((int64_t)pr.Kp + 127) / 128;
+  rotate_block(pr.x, pr.signs, pr.xt, pr.K, pr.Kp, (int)(local / nblk), (local % nblk) * 128, lane);
+}
+
 }  // namespace
 
 int tc_tmem_cols(int fmt, int bn) {
@@ -545,6 +566,12 @@ cudaError_t launch_rotate_x(const uint16_t* x, const uint32_t* signs, uint8_t* x
   const int warps = 8;
   const int64_t ctas = (items + warps - 1) / warps;
   rotate_x_kernel<<<(unsigned)ctas, warps * 32, 0, stream>>>(x, signs, xt, M, K, Kp);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_rotate_x_batched(const DecArgs& a, int64_t total_items, cudaStream_t stream) {
+  const int warps = 8;
+  rotate_x_batched_kernel<<<(unsigned)((total_items + warps - 1) / warps), warps * 32, 0, stream>>>(a, total_items);
   return cudaGetLastError();
 }
 

@@ -33,7 +33,9 @@ struct DecProblem {
   int N, K, Kp;              // Kp: padded K of the ternary planes
   int B, RG, P, bits;        // blocks per row, 128-row groups, K splits, 2/3 (ternary: 1)
   int item_base;             // first work item of this problem
-  int xblk_base;             // first block of this problem in the preparation pass
+  int xblk_base;             // 2/3-bit: first block of this problem in the preparation pass;
+                             // ternary: first rotation work item (token, 128-block) of it
+  const uint32_t* signs;     // ternary: random-sign mask of the rotation
   int counter_base;          // first arrival counter (row group) of this problem
   int64_t partial_base;      // first partial float of this problem (ternary items)
   int64_t block_base;        // first block of this problem in the batch's block sequence (2/3-bit)
@@ -77,6 +79,9 @@ cudaError_t launch_tc_kernel(int fmt, int bn, const TcArgs& a, const void* x_act
                              int grid, cudaStream_t stream);
 cudaError_t launch_rotate_x(const uint16_t* x, const uint32_t* signs, uint8_t* xt, int M, int K, int64_t Kp,
                             cudaStream_t stream);
+// The same for every problem of a batch (x, signs, xt, K, Kp per problem; xblk_base = first
+// work item; total_items = M * sum of ceil(Kp / 128)).
+cudaError_t launch_rotate_x_batched(const DecArgs& a, int64_t total_items, cudaStream_t stream);
 cudaError_t launch_unpack_bf16(int fmt, const uint8_t* packed, const uint16_t* scales, int N, int K, int units,
                                uint16_t* w, cudaStream_t stream);
 

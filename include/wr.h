@@ -194,6 +194,26 @@ wr_status wr_gemm_ternary(int64_t M, int64_t N, int64_t K, const uint16_t* x, co
 wr_status wr_gemv_noalloc(int64_t M, int64_t N, int64_t K, const uint16_t* x, const void* packed,
                           const uint16_t* scales, int bits, int group, float* y, void* stream);
 
+/* One problem of a batched ternary decode GEMV (fields read on the host during the call). */
+typedef struct {
+  const uint16_t* x;           /* bf16 [M, K] activations (device) */
+  const void* packed;          /* packed trits (device) */
+  const uint16_t* alpha;       /* fp16 [N] row scales (device) */
+  const uint32_t* sign_bits;   /* uint32 [ceil(K/32)] random-sign mask of the rotation (device) */
+  float* y;                    /* fp32 [M, N] output (device, overwritten) */
+  int64_t N, K;                /* K % 128 == 0 */
+} wr_gemv_ternary_problem;
+
+/* Batched ternary decode GEMV: `count` independent problems sharing one token count
+ * 1 <= M <= 8. One launch applies the block-128 random-sign Hadamard to every problem's x,
+ * one persistent launch contracts them all (at most 256 problems per launch; larger batches
+ * are split). Each problem computes what wr_gemm_ternary computes. problems_host is read
+ * during the call. */
+size_t wr_gemv_ternary_batched_workspace_bytes(int64_t M, int32_t count,
+                                               const wr_gemv_ternary_problem* problems_host);
+wr_status wr_gemv_ternary_batched(int64_t M, int32_t count, const wr_gemv_ternary_problem* problems_host,
+                                  void* workspace, size_t workspace_bytes, void* stream);
+
 /* Reads and clears the device error word that bounded waits set when they give up
  * (synchronizes the stream). WR_OK when no wait timed out since the last call. */
 wr_status wr_get_device_error(void* stream);

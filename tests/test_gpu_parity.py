@@ -243,3 +243,31 @@ def test_gemv_batched_ragged_mixed(wr):
     for codes, scales, bits, x, y in cases:
         ref, B = o.gemm_codes(x, codes, scales, bits)
         check_close(y.cpu().numpy(), ref, B)
+
+
+# ---------------------------------------------------------------- batched ternary decode GEMV
+
+@pytest.mark.parametrize("M", [1, 6])
+def test_ternary_gemv_batched_layer_and_ragged(wr, M):
+    """The 7 Qwen3-4B layer shapes plus ragged ones, ternary, in one batched call, twice."""
+    torch = torch_mod()
+    shapes = [(N, K) for (_, K, N, _) in wr_synth.QWEN3_4B_LAYER] + [(40, 640), (300, 128), (17, 384)]
+    cases, problems = [], []
+    for i, (N, K) in enumerate(shapes):
+        codes, alpha, signs, packed, a_d, s_d = t_case(wr, N, K, seed=2000 + i)
+        x = wr_synth.activations_bf16(2100 + i, M, K)
+        y = torch.full((M, N), float("nan"), dtype=torch.float32, device="cuda")
+        cases.append((codes, alpha, signs, x, y))
+        problems.append((dev(x), packed, a_d, s_d, y, N, K))
+    nb = wr.wr_gemv_ternary_batched_workspace_bytes(M, problems)
+    assert nb > 0
+    ws = _zeros_ws(nb)
+    for rep in range(2):
+        for *_, y in cases:
+            y.fill_(float("nan"))
+        wr.wr_gemv_ternary_batched(M, problems, ws, nb)
+        torch.cuda.synchronize()
+        for codes, alpha, signs, x, y in cases:
+            ref, B = o.gemm_ternary(x, codes, alpha, signs)
+            check_close(y.cpu().numpy(), ref, B)
+    assert wr.wr_get_device_error() == 0
