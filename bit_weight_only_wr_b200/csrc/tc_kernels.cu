@@ -7,17 +7,19 @@
 // * B[16 x BN] with the weights as A and BN token columns as B ("swap-AB"), so every TMEM lane
 // is one output row and the per-block scale is a single scalar per lane.
 //
-// Warp roles (320 threads):
-//   warps 0-3  decode: thread t owns row t of the group (TMEM lane t). It reads its row's
+// Warp roles (576 threads):
+//   warps 0-7  decode: warps w and w + 4 own rows 32 (w % 4) .. + 31 of the group (TMEM lanes)
+//              and take alternate quarters of each half-block chunk. A thread reads its row's
 //              packed codes from shared memory, turns them into exact bf16 values (g/2, or t
 //              for ternary) in registers and writes them into tensor memory with tcgen05.st:
 //              A is consumed from TMEM, so the decoded weights never touch shared memory.
-//   warp 8     producer: bulk-copies the packed units of each 256-block (8 x 16-row units) and
+//   warp 16    producer: bulk-copies the packed units of each 256-block (8 x 16-row units) and
 //              TMA-loads the activation tile (128-byte swizzle) into shared-memory rings.
-//   warp 9     allocates TMEM and issues the MMAs (one thread), committing to the barriers
+//   warp 17    allocates TMEM and issues the MMAs (whole warp, one elected lane), committing to the barriers
 //              that recycle A buffers, activation stages and accumulators.
-//   warps 4-7  epilogue: per 256-block, load the fp32 partial from TMEM, multiply by 2*s[n,b]
-//              in fp32 and add it to a register running sum (ternary: once per item); at the
+//   warps 8-15 epilogue (two per lane quarter, half of the token tile each): per 256-block,
+//              load the fp32 partial from TMEM, multiply by 2*s[n,b] in fp32 and add it to a
+//              register running sum (ternary: once per item); at the
 //              end of an item, write y, or combine split-K pieces through the workspace (the
 //              last of the P pieces to arrive adds them in order p = 0..P-1 and writes y).
 // Every wait is bounded: a stuck pipeline records an error code and the CTA unwinds.
@@ -34,7 +36,7 @@ namespace {
 
 using namespace tc;
 
-constexpr int kThreads = 320;
+constexpr int kThreads = 576;
 constexpr int kSP = 4;  // packed-unit stages
 constexpr int kSX = 2;  // activation stages (per block)
 
@@ -140,7 +142,7 @@ __device__ __forceinline__ uint32_t trit_entry(int v) {
 // ---------------------------------------------------------------- the kernel
 
 template <int FMT, int BN>
-__global__ void __launch_bounds__(kThreads, BN == 16 ? 2 : 1) tc_kernel(const TcArgs a, const __grid_constant__ CUtensorMap xmap) {
+__global__ void __launch_bounds__(kThreads, 1) tc_kernel(const TcArgs a, const __grid_constant__ CUtensorMap xmap) {
   using F = Fmt<FMT>;
   using Ly = Layout<FMT, BN>;
   extern __shared__ uint8_t smem_raw[];
@@ -163,29 +165,29 @@ __global__ void __launch_bounds__(kThreads, BN == 16 ? 2 : 1) tc_kernel(const Tc
   if (threadIdx.x == 0) {
     for (int i = 0; i < kSP; ++i) {
       mbar_init(&bars->pk_full[i], 1);
-      mbar_init(&bars->pk_empty[i], 4);
+      mbar_init(&bars->pk_empty[i], 8);
     }
     for (int i = 0; i < kSX; ++i) {
       mbar_init(&bars->x_full[i], 1);
       mbar_init(&bars->x_empty[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&bars->a_full[i], 4);
+      mbar_init(&bars->a_full[i], 8);
       mbar_init(&bars->a_empty[i], 1);
       mbar_init(&bars->d_full[i], 1);
-      mbar_init(&bars->d_empty[i], 4);
+      mbar_init(&bars->d_empty[i], 8);
     }
     bars->abort_flag = 0;
     bars->last_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 9) tmem_alloc(&bars->tmem_base, Ly::kTmemCols);
+  if (warp == 17) tmem_alloc(&bars->tmem_base, Ly::kTmemCols);
   fence_before_sync();
   __syncthreads();
   fence_after_sync();
   const uint32_t tmem = bars->tmem_base;
 
-  if (warp == 8) {
+  if (warp == 16) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       prefetch_tensormap(&xmap);
@@ -227,7 +229,7 @@ __global__ void __launch_bounds__(kThreads, BN == 16 ? 2 : 1) tc_kernel(const Tc
         }
       }
     }
-  } else if (warp == 9) {
+  } else if (warp == 17) {
     // ------------------------------------------------------------ MMA issuer (whole warp, one lane issues)
     constexpr uint32_t idesc = idesc_bf16_m128(BN);
     uint32_t gb = 0, gc = 0, gi = 0;
@@ -268,11 +270,14 @@ __global__ void __launch_bounds__(kThreads, BN == 16 ? 2 : 1) tc_kernel(const Tc
       }
       if (FMT == WR_FMT_TERNARY && ok) mma_commit_elect(&bars->d_full[dbuf]);
     }
-  } else if (warp < 4) {
+  } else if (warp < 8) {
     // ------------------------------------------------------------ decode (thread = row)
-    const int t = threadIdx.x;
+    // warps w and w + 4 share lane quarter w % 4 (rows 32 (w % 4) ..); group g = w / 4 decodes
+    // quarter g of each half-block chunk, so each row's decode chain is split in two
+    const int g = warp >> 2, lq = warp & 3;
+    const int t = 32 * lq + lane;
     const int tile = t >> 4, r = t & 15, r0 = r & 7, half = r >> 3;
-    const uint32_t lane_addr = (uint32_t)(32 * warp) << 16;
+    const uint32_t lane_addr = (uint32_t)(32 * lq) << 16;
     uint32_t gb = 0, gc = 0;
     for (int it = blockIdx.x; it < a.items && !*abort_flag; it += gridDim.x) {
       int rg, mt, p, b0, b1;
@@ -286,21 +291,18 @@ __global__ void __launch_bounds__(kThreads, BN == 16 ? 2 : 1) tc_kernel(const Tc
           const int sa = gc & 1;
           if (!(ok = mbar_wait(&bars->a_empty[sa], ((gc >> 1) & 1) ^ 1, abort_flag, a.err, 302))) break;
           fence_after_sync();
-#pragma unroll
-          for (int qq = 0; qq < 2; ++qq) {
-            const int q = 2 * c + qq;
-            const uint32_t col = tmem + lane_addr + sa * Ly::kACols + qq * F::kQuarterCols;
-            if (FMT == WR_FMT_TERNARY) {
-              uint32_t v[40];
-              decode_t_quarter(unit, r0, half, q, lut_lo, lut_hi, v);
-              tmem_st32(col, v);
-              tmem_st8(col + 32, v + 32);
-            } else {
-              uint32_t v[32];
-              if (FMT == WR_FMT_Q2) decode_q2_quarter(unit, r0, half, q, v);
-              else decode_q3_quarter(unit, r0, half, q, v);
-              tmem_st32(col, v);
-            }
+          const int q = 2 * c + g;
+          const uint32_t col = tmem + lane_addr + sa * Ly::kACols + g * F::kQuarterCols;
+          if (FMT == WR_FMT_TERNARY) {
+            uint32_t v[40];
+            decode_t_quarter(unit, r0, half, q, lut_lo, lut_hi, v);
+            tmem_st32(col, v);
+            tmem_st8(col + 32, v + 32);
+          } else {
+            uint32_t v[32];
+            if (FMT == WR_FMT_Q2) decode_q2_quarter(unit, r0, half, q, v);
+            else decode_q3_quarter(unit, r0, half, q, v);
+            tmem_st32(col, v);
           }
           tmem_wait_st();
           fence_before_sync();
@@ -314,18 +316,20 @@ __global__ void __launch_bounds__(kThreads, BN == 16 ? 2 : 1) tc_kernel(const Tc
       if (!ok) break;
     }
   } else {
-    // ------------------------------------------------------------ epilogue (warps 4-7, thread = row)
-    constexpr int TOK = Ly::kTok;
-    const int t = threadIdx.x - 128;
-    const uint32_t lane_addr = (uint32_t)(32 * (warp - 4)) << 16;
+    // ------------------------------------------------------------ epilogue (warps 8-15, thread = row)
+    // warps 8 + w and 12 + w share lane quarter w; group e takes tokens e*TH .. e*TH + TH - 1
+    constexpr int TOK = Ly::kTok, TH = TOK / 2;
+    const int e = (warp - 8) >> 2, lq = (warp - 8) & 3;
+    const int t = 32 * lq + lane;
+    const uint32_t lane_addr = (uint32_t)(32 * lq) << 16;
     uint32_t gb = 0, gi = 0;
     for (int it = blockIdx.x; it < a.items && !*abort_flag; it += gridDim.x, ++gi) {
       int rg, mt, p, b0, b1;
       item_coords(a, it, rg, mt, p, b0, b1);
       const int n = rg * 128 + t;
-      float acc[TOK];
+      float acc[TH];
 #pragma unroll
-      for (int i = 0; i < TOK; ++i) acc[i] = 0.f;
+      for (int i = 0; i < TH; ++i) acc[i] = 0.f;
       bool ok = true;
       if (FMT == WR_FMT_TERNARY) {
         const uint32_t dbuf = gi & 1;
@@ -340,7 +344,7 @@ __global__ void __launch_bounds__(kThreads, BN == 16 ? 2 : 1) tc_kernel(const Tc
           __syncwarp();
           if (lane == 0) mbar_arrive(&bars->d_empty[dbuf]);
 #pragma unroll
-          for (int i = 0; i < TOK; ++i) acc[i] = d[i] + d[i + 8];
+          for (int i = 0; i < TH; ++i) acc[i] = d[e * TH + i] + d[e * TH + i + 8];
         }
       } else {
         for (int b = b0; b < b1; ++b, ++gb) {
@@ -349,9 +353,9 @@ __global__ void __launch_bounds__(kThreads, BN == 16 ? 2 : 1) tc_kernel(const Tc
           if (!(ok = mbar_wait(&bars->d_full[dbuf], (gb >> 1) & 1, abort_flag, a.err, 402))) break;
           fence_after_sync();
 #pragma unroll
-          for (int c0 = 0; c0 < BN; c0 += 16) {
+          for (int c0 = 0; c0 < TH; c0 += 16) {
             float d[16];
-            tmem_ld16(tmem + lane_addr + Ly::kDCol + dbuf * BN + c0, d);
+            tmem_ld16(tmem + lane_addr + Ly::kDCol + dbuf * BN + e * TH + c0, d);
             tmem_wait_ld();
 #pragma unroll
             for (int i = 0; i < 16; ++i) acc[c0 + i] = fmaf(s2, d[i], acc[c0 + i]);
@@ -363,45 +367,45 @@ __global__ void __launch_bounds__(kThreads, BN == 16 ? 2 : 1) tc_kernel(const Tc
       }
       if (!ok) break;
       // ---- output: direct store, or split-K combine through the workspace
-      const int m0 = mt * TOK;
-      const int mcount = min(TOK, a.M - m0);
+      const int m0 = mt * TOK + e * TH;
+      const int mcount = max(0, min(TH, a.M - m0));
       const float rs = (FMT == WR_FMT_TERNARY && n < a.N) ? half_bits_to_float(__ldg(a.alpha + n)) : 1.f;
       if (a.P == 1) {
         if (n < a.N) {
 #pragma unroll
-          for (int i = 0; i < TOK; ++i)
+          for (int i = 0; i < TH; ++i)
             if (i < mcount) a.y[(int64_t)(m0 + i) * a.N + n] = rs * acc[i];
         }
       } else {
         const int tileid = rg * a.MT + mt;
-        float* part = a.partial + ((int64_t)tileid * a.P + p) * (TOK * 128);
+        float* part = a.partial + ((int64_t)tileid * a.P + p) * (TOK * 128) + (int64_t)e * TH * 128;
 #pragma unroll
-        for (int i = 0; i < TOK; ++i)
+        for (int i = 0; i < TH; ++i)
           if (i < mcount) part[i * 128 + t] = acc[i];
         __threadfence();
-        named_bar_sync(1, 128);
-        if (t == 0) bars->last_flag = (atomicAdd(a.counter + tileid, 1) == a.P - 1);
-        named_bar_sync(1, 128);
+        named_bar_sync(1, 256);
+        if (threadIdx.x == 256) bars->last_flag = (atomicAdd(a.counter + tileid, 1) == a.P - 1);
+        named_bar_sync(1, 256);
         const int last = bars->last_flag;
         if (last) {
           __threadfence();
-          float sum[TOK];
+          // the pieces in order p = 0 .. P-1 (this one included), into acc
 #pragma unroll
-          for (int i = 0; i < TOK; ++i) sum[i] = 0.f;
+          for (int i = 0; i < TH; ++i) acc[i] = 0.f;
           for (int pp = 0; pp < a.P; ++pp) {
-            const float* src = a.partial + ((int64_t)tileid * a.P + pp) * (TOK * 128);
+            const float* src = a.partial + ((int64_t)tileid * a.P + pp) * (TOK * 128) + (int64_t)e * TH * 128;
 #pragma unroll
-            for (int i = 0; i < TOK; ++i)
-              if (i < mcount) sum[i] += __ldcg(src + i * 128 + t);
+            for (int i = 0; i < TH; ++i)
+              if (i < mcount) acc[i] += __ldcg(src + i * 128 + t);
           }
           if (n < a.N) {
 #pragma unroll
-            for (int i = 0; i < TOK; ++i)
-              if (i < mcount) a.y[(int64_t)(m0 + i) * a.N + n] = rs * sum[i];
+            for (int i = 0; i < TH; ++i)
+              if (i < mcount) a.y[(int64_t)(m0 + i) * a.N + n] = rs * acc[i];
           }
-          if (t == 0) a.counter[tileid] = 0;
+          if (threadIdx.x == 256) a.counter[tileid] = 0;
         }
-        named_bar_sync(1, 128);
+        named_bar_sync(1, 256);
       }
     }
   }
@@ -409,7 +413,7 @@ __global__ void __launch_bounds__(kThreads, BN == 16 ? 2 : 1) tc_kernel(const Tc
   fence_before_sync();
   __syncthreads();
   fence_after_sync();
-  if (warp == 9) tmem_dealloc(tmem, Ly::kTmemCols);
+  if (warp == 17) tmem_dealloc(tmem, Ly::kTmemCols);
 }
 
 // ---------------------------------------------------------------- host side
@@ -552,11 +556,8 @@ int tc_tmem_cols(int fmt, int bn) {
 
 cudaError_t launch_tc_kernel(int fmt, int bn, const TcArgs& a, const void* x_act, int64_t x_rows, int64_t x_k,
                              int grid, cudaStream_t stream) {
-  if (fmt == WR_FMT_Q2 && bn == 16) return launch_tc<WR_FMT_Q2, 16>(a, x_act, x_rows, x_k, grid, stream);
-  if (fmt == WR_FMT_Q3 && bn == 16) return launch_tc<WR_FMT_Q3, 16>(a, x_act, x_rows, x_k, grid, stream);
   if (fmt == WR_FMT_Q2 && bn == 128) return launch_tc<WR_FMT_Q2, 128>(a, x_act, x_rows, x_k, grid, stream);
   if (fmt == WR_FMT_Q3 && bn == 128) return launch_tc<WR_FMT_Q3, 128>(a, x_act, x_rows, x_k, grid, stream);
-  if (fmt == WR_FMT_TERNARY && bn == 16) return launch_tc<WR_FMT_TERNARY, 16>(a, x_act, x_rows, x_k, grid, stream);
   return cudaErrorNotSupported;
 }
 
