@@ -19,19 +19,21 @@
 // multiple of 2^E: at most 2^-30 max|x| per element.
 //
 // A CTA is one small pipeline; three run on every SM so that their latency chains overlap
-// (warp roles, 160 threads):
-//   warps 0-3  consumers, thread = weight row (TMEM lane 32 w + lane). Per block: decode the
-//              row's 256 codes into the A buffer (two 32-column tensor-memory stores), hand it
-//              to the control warp, then turn the previous block's accumulator into fp32
-//              partial dot products times s[n,b] (all tokens of the row).
-//   warp 4     control: allocates tensor memory; issues the bulk copies of the packed weights
+// (warp roles, 288 threads):
+//   warps 0-3  decode, thread = weight row (TMEM lane 32 w + lane): per block, the row's 256
+//              codes into the A buffer (two 32-column tensor-memory stores), then hand it to
+//              the control warp.
+//   warps 4-7  epilogue, thread = row: per block, once its MMAs are done, the integer
+//              accumulator becomes fp32 partial dot products times s[n,b] for all tokens of
+//              the row. Decode and epilogue run in separate warps so that a block costs the
+//              longer of the two chains, not their sum.
+//   warp 8     control: allocates tensor memory; issues the bulk copies of the packed weights
 //              (one per block, a ring of kSP blocks ahead), of the prepared B tiles and their
 //              correction records (two blocks ahead), and the 8 MMAs and one commit per block
-//              (the whole warp walks the blocks, one elected lane issues). One warp instead of
-//              three leaves the consumers more registers.
+//              (the whole warp walks the blocks, one elected lane issues).
 // Tensor memory (128 columns): one A buffer (64 columns) and two accumulators (32 columns). The
 // store of block i waits for the MMAs of block i - 1; block i's MMAs write accumulator i % 2
-// while the consumers finish block i - 1 from the other one. Every wait is bounded.
+// once the epilogue has read block i - 2 from it. Every wait is bounded.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -45,7 +47,7 @@ namespace {
 
 using namespace tc;
 
-constexpr int kThreads = 160;
+constexpr int kThreads = 288;
 constexpr int kCtasPerSm = 3;
 constexpr int kSP = 4;   // packed stages: 8 units of up to 1.5 KB
 constexpr int kSX = 2;   // B tiles (up to 2 atoms x 32 rows x 128 bytes); also the MMA-done ring
@@ -67,7 +69,8 @@ static_assert(kCtasPerSm * kTmemCols <= 512, "tensor memory of an SM");
 struct Bars {
   uint64_t pk_full[kSP], pk_empty[kSP], x_full[kSX], c_full[kSC], c_empty[kSC];
   uint64_t mma_done[kSX];   // block j's MMAs complete: frees B stage j % kSX, A; accumulator holds j
-  uint64_t a_full;          // the consumers have stored block j's codes
+  uint64_t a_full;          // the decode warps have stored block j's codes
+  uint64_t d_empty[2];      // the epilogue warps have read accumulator j % 2
   uint64_t group;           // the 4 consumer warps meet here (bounded, unlike bar.sync)
   uint32_t tmem_base;
   int abort_flag;
@@ -247,18 +250,19 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_q_kernel(const __gr
       mbar_init(&bars->c_empty[i], 4);
     }
     mbar_init(&bars->a_full, 4);
+    for (int i = 0; i < 2; ++i) mbar_init(&bars->d_empty[i], 4);
     mbar_init(&bars->group, 4);
     bars->abort_flag = 0;
     bars->last_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 4) tmem_alloc(&bars->tmem_base, kTmemCols);
+  if (warp == 8) tmem_alloc(&bars->tmem_base, kTmemCols);
   fence_before_sync();
   __syncthreads();
   fence_after_sync();
   const uint32_t tmem = bars->tmem_base;
 
-  if (warp == 4) {
+  if (warp == 8) {
     // ------------------------------------------------------------ control warp (whole warp walks the
     // blocks, one elected lane issues): weight copies kSP blocks ahead, activation copies two ahead,
     // and the MMAs of each block once the consumers have stored its codes.
@@ -303,6 +307,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_q_kernel(const __gr
       const int sx = gm % kSX;
       if (!(ok = mbar_wait(&bars->a_full, gm & 1, abort_flag, a.err, 201))) break;
       if (!(ok = mbar_wait(&bars->x_full[sx], (gm / kSX) & 1, abort_flag, a.err, 202))) break;
+      // accumulator gm % 2 was read by the epilogue warps (block gm - 2)
+      if (!(ok = mbar_wait(&bars->d_empty[gm & 1], ((gm >> 1) & 1) ^ 1, abort_flag, a.err, 206))) break;
       fence_after_sync();
       const uint64_t bd = bdesc0 + (uint64_t)((sx * kXStage) >> 4);
 #pragma unroll
@@ -331,11 +337,40 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_q_kernel(const __gr
       for (uint32_t k = nx > kSC ? nx - kSC : 0; k < nx; ++k) mbar_wait_drain(&bars->c_full[k % kSC], (k / kSC) & 1);
       if (gm > 0) mbar_wait_drain(&bars->mma_done[(gm - 1) % kSX], ((gm - 1) / kSX) & 1);
     }
-  } else {
-    // ------------------------------------------------------------ consumers (warps 0-3, thread = row)
+  } else if (warp < 4) {
+    // ------------------------------------------------------------ decode (warps 0-3, thread = row)
     const int t = threadIdx.x;                          // row in the row group = TMEM lane
     const int tile = t >> 4, r = t & 15, r0 = r & 7, half = r >> 3;
     const uint32_t lane_base = tmem + ((uint32_t)(32 * warp) << 16);
+    Lite dc = lite_of(pos_start(a));
+    for (uint32_t gd = 0; dc.left > 0; ++gd) {
+      const int sp = gd % kSP;
+      if (!mbar_wait(&bars->pk_full[sp], (gd / kSP) & 1, abort_flag, a.err, 301)) break;
+      const uint8_t* unit = ps + sp * kPStage + tile * (dc.bits == 2 ? 1024 : 1536);
+      uint32_t v[32];
+      if (dc.bits == 2) q2_half_i8(unit, r0, half, 0, v);
+      else q3_half_i8(unit, r0, half, 0, v);
+      // the A buffer is free once block gd - 1's MMAs are done
+      if (gd > 0 && !mbar_wait(&bars->mma_done[(gd - 1) % kSX], ((gd - 1) / kSX) & 1, abort_flag, a.err, 302)) break;
+      fence_after_sync();
+      tmem_st32(lane_base + kACol, v);
+      if (dc.bits == 2) q2_half_i8(unit, r0, half, 1, v);
+      else q3_half_i8(unit, r0, half, 1, v);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->pk_empty[sp]);
+      tmem_st32(lane_base + kACol + 32, v);
+      tmem_wait_st();
+      fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->a_full);
+      lite_next(dc, a);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue (warps 4-7, thread = row)
+    // Per block, once its MMAs are done: the integer accumulator becomes fp32 partial dot
+    // products times s[n,b] (all tokens of the row), summed in registers over the row group.
+    const int t = threadIdx.x - 128;
+    const uint32_t lane_base = tmem + ((uint32_t)(32 * (warp - 4)) << 16);
     float acc[kSlots];
 #pragma unroll
     for (int m = 0; m < kSlots; ++m) acc[m] = 0.f;
@@ -345,11 +380,14 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_q_kernel(const __gr
       if (lane == 0) mbar_arrive(&bars->group);
       return mbar_wait(&bars->group, (ng++) & 1, abort_flag, a.err, code);
     };
-    // finish block ge (cursor ec): its accumulator (buffer ge % 2, loaded here in chunks of up
-    // to 4 token slots), its correction record and its scale
-    auto finish = [&](const Pos& ec, uint32_t ge, uint16_t sraw) -> bool {
+    Pos ec = pos_start(a);
+    for (uint32_t ge = 0; ec.left > 0; ++ge) {
+      const int n = ec.rg * 128 + t;
+      const uint16_t sraw = n < ec.N ? __ldg(ec.scales + (int64_t)n * ec.B + ec.b) : (uint16_t)0;
       const int sc = ge % kSC;
-      if (!mbar_wait(&bars->c_full[sc], (ge / kSC) & 1, abort_flag, a.err, 303)) return false;
+      if (!mbar_wait(&bars->mma_done[ge % kSX], (ge / kSX) & 1, abort_flag, a.err, 303)) break;
+      if (!mbar_wait(&bars->c_full[sc], (ge / kSC) & 1, abort_flag, a.err, 304)) break;
+      fence_after_sync();
       const int4* rec = reinterpret_cast<const int4*>(cs + sc * 256);
       const float s = half_bits_to_float(sraw);
       constexpr int kChunk = XR < 16 ? XR : 16;   // columns per load
@@ -372,108 +410,66 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_q_kernel(const __gr
           }
         }
       }
+      fence_before_sync();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->c_empty[sc]);
-      if (ec.b + 1 < ec.B && ec.left > 1) return true;
-      // the row group ends here (or this range does): y, or, for a row group that several CTA
-      // ranges share, the combine through the partial slots (the last range to arrive adds
-      // the pieces in range order)
-      const int n = ec.rg * 128 + t;
-      const int64_t T = a.total;
-      const int64_t g0 = ec.g - ec.b;                     // first block of the row group
-      const int c0 = cta_of(T, g0), c1 = cta_of(T, g0 + ec.B - 1);
-      if (c0 == c1) {
-        if (n < ec.N) {
-#pragma unroll
-          for (int m = 0; m < kSlots; ++m)
-            if (m < M) ec.y[(int64_t)m * ec.N + n] = acc[m];
-        }
-      } else {
-        // slot 0: the row group began before this range; slot 1: it continues after it
-        const int slot = g0 < range_start(T, blockIdx.x) ? 0 : 1;
-        float* part = a.partial + ((int64_t)2 * blockIdx.x + slot) * M * 128;
-#pragma unroll
-        for (int m = 0; m < kSlots; ++m)
-          if (m < M) part[m * 128 + t] = acc[m];
-        __threadfence();
-        if (!group_sync(304)) return false;
-        if (t == 0) bars->last_flag = (atomicAdd(a.counter + ec.grg, 1) == c1 - c0);
-        if (!group_sync(305)) return false;
-        if (bars->last_flag) {
-          __threadfence();
-          float sum[kSlots];
-#pragma unroll
-          for (int m = 0; m < kSlots; ++m) sum[m] = 0.f;
-          for (int c = c0; c <= c1; ++c) {
-            const int sl = g0 < range_start(T, c) ? 0 : 1;
-            const float* src = a.partial + ((int64_t)2 * c + sl) * M * 128;
-#pragma unroll
-            for (int m = 0; m < kSlots; ++m)
-              if (m < M) sum[m] += __ldcg(src + m * 128 + t);
-          }
+      if (lane == 0) {
+        mbar_arrive(&bars->d_empty[ge & 1]);
+        mbar_arrive(&bars->c_empty[sc]);
+      }
+      if (ec.b + 1 == ec.B || ec.left == 1) {
+        // the row group ends here (or this range does): y, or, for a row group that several
+        // CTA ranges share, the combine through the partial slots (the last range to arrive
+        // adds the pieces in range order)
+        const int64_t T = a.total;
+        const int64_t g0 = ec.g - ec.b;                     // first block of the row group
+        const int c0 = cta_of(T, g0), c1 = cta_of(T, g0 + ec.B - 1);
+        if (c0 == c1) {
           if (n < ec.N) {
 #pragma unroll
             for (int m = 0; m < kSlots; ++m)
-              if (m < M) ec.y[(int64_t)m * ec.N + n] = sum[m];
+              if (m < M) ec.y[(int64_t)m * ec.N + n] = acc[m];
           }
-          if (t == 0) a.counter[ec.grg] = 0;
-        }
-      }
+        } else {
+          // slot 0: the row group began before this range; slot 1: it continues after it
+          const int slot = g0 < range_start(T, blockIdx.x) ? 0 : 1;
+          float* part = a.partial + ((int64_t)2 * blockIdx.x + slot) * M * 128;
 #pragma unroll
-      for (int m = 0; m < kSlots; ++m) acc[m] = 0.f;
-      return true;
-    };
-    auto scale_of = [&](const Pos& c) -> uint16_t {
-      const int n = c.rg * 128 + t;
-      return n < c.N ? __ldg(c.scales + (int64_t)n * c.B + c.b) : (uint16_t)0;
-    };
-
-    Pos ec = pos_start(a);     // block being finished
-    Lite dc = lite_of(ec);     // block being decoded
-    uint32_t gd = 0;
-    bool ok = true;
-    for (; dc.left > 0; ++gd) {
-      const uint16_t sraw = gd > 0 ? scale_of(ec) : (uint16_t)0;   // block gd - 1
-      const int sp = gd % kSP;
-      if (!(ok = mbar_wait(&bars->pk_full[sp], (gd / kSP) & 1, abort_flag, a.err, 301))) break;
-      const uint8_t* unit = ps + sp * kPStage + tile * (dc.bits == 2 ? 1024 : 1536);
-      uint32_t v[32];
-      if (dc.bits == 2) q2_half_i8(unit, r0, half, 0, v);
-      else q3_half_i8(unit, r0, half, 0, v);
-      // the A buffer is free (and accumulator (gd - 1) % 2 complete) once block gd - 1's MMAs are done
-      if (gd > 0 && !(ok = mbar_wait(&bars->mma_done[(gd - 1) % kSX], ((gd - 1) / kSX) & 1, abort_flag, a.err, 302)))
-        break;
-      fence_after_sync();
-      tmem_st32(lane_base + kACol, v);
-      if (dc.bits == 2) q2_half_i8(unit, r0, half, 1, v);
-      else q3_half_i8(unit, r0, half, 1, v);
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->pk_empty[sp]);
-      tmem_st32(lane_base + kACol + 32, v);
-      tmem_wait_st();
-      fence_before_sync();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->a_full);
-      lite_next(dc, a);
-      if (gd > 0) {
-        if (!(ok = finish(ec, gd - 1, sraw))) break;
-        pos_next(ec, a);
+          for (int m = 0; m < kSlots; ++m)
+            if (m < M) part[m * 128 + t] = acc[m];
+          __threadfence();
+          if (!group_sync(305)) break;
+          if (t == 0) bars->last_flag = (atomicAdd(a.counter + ec.grg, 1) == c1 - c0);
+          if (!group_sync(306)) break;
+          if (bars->last_flag) {
+            __threadfence();
+#pragma unroll
+            for (int m = 0; m < kSlots; ++m) acc[m] = 0.f;
+            for (int c = c0; c <= c1; ++c) {
+              const int sl = g0 < range_start(T, c) ? 0 : 1;
+              const float* src = a.partial + ((int64_t)2 * c + sl) * M * 128;
+#pragma unroll
+              for (int m = 0; m < kSlots; ++m)
+                if (m < M) acc[m] += __ldcg(src + m * 128 + t);
+            }
+            if (n < ec.N) {
+#pragma unroll
+              for (int m = 0; m < kSlots; ++m)
+                if (m < M) ec.y[(int64_t)m * ec.N + n] = acc[m];
+            }
+            if (t == 0) a.counter[ec.grg] = 0;
+          }
+        }
+#pragma unroll
+        for (int m = 0; m < kSlots; ++m) acc[m] = 0.f;
       }
-    }
-    if (ok && gd > 0) {
-      // the last block
-      const uint16_t sraw = scale_of(ec);
-      if (mbar_wait(&bars->mma_done[(gd - 1) % kSX], ((gd - 1) / kSX) & 1, abort_flag, a.err, 306)) {
-        fence_after_sync();
-        finish(ec, gd - 1, sraw);
-      }
+      pos_next(ec, a);
     }
   }
 
   fence_before_sync();
   __syncthreads();
   fence_after_sync();
-  if (warp == 4) tmem_dealloc(tmem, kTmemCols);
+  if (warp == 8) tmem_dealloc(tmem, kTmemCols);
 }
 
 // Preparation pass: one warp per (problem, block, token slot m < N/4). The block's activations
