@@ -136,9 +136,7 @@ def module_bytes(wr, M, N, K, bits):
 # DRAM traffic of the decode GEMV launch, (dram__bytes_read + dram__bytes_write) / algorithmic
 # bytes, from one ncu capture of the current kernel at that token count (summary and command in
 # profiles/). None: no capture of this kernel version, so no traffic figure is claimed.
-# gemv_q_kernel, three CTAs per SM: M = 1 read 1.18 GB + write 9.70 MB; M = 8 read 1.21 GB + write
-# 53.73 MB, for 1,178,984,448 and 1,223,368,704 algorithmic bytes (ncu prints three digits).
-_TRAFFIC_RATIO = {1: (1.18e9 + 9.70e6) / 1_178_984_448, 8: (1.21e9 + 53.73e6) / 1_223_368_704}
+_TRAFFIC_RATIO = {}   # filled from a capture of the current kernel version
 
 
 def traffic_per_launch(M: int, layers: int, algo_bytes: int):

@@ -19,18 +19,18 @@
 // multiple of 2^E: at most 2^-30 max|x| per element.
 //
 // A CTA is one small pipeline; three run on every SM so that their latency chains overlap
-// (warp roles, 288 threads):
+// (warp roles, 320 threads):
 //   warps 0-3  decode, thread = weight row (TMEM lane 32 w + lane): per block, the row's 256
 //              codes into the A buffer (two 32-column tensor-memory stores), then hand it to
-//              the control warp.
+//              the MMA warp.
 //   warps 4-7  epilogue, thread = row: per block, once its MMAs are done, the integer
 //              accumulator becomes fp32 partial dot products times s[n,b] for all tokens of
 //              the row. Decode and epilogue run in separate warps so that a block costs the
 //              longer of the two chains, not their sum.
-//   warp 8     control: allocates tensor memory; issues the bulk copies of the packed weights
-//              (one per block, a ring of kSP blocks ahead), of the prepared B tiles and their
-//              correction records (two blocks ahead), and the 8 MMAs and one commit per block
-//              (the whole warp walks the blocks, one elected lane issues).
+//   warp 8     copies: the packed weights (one bulk copy per block, a ring of kSP blocks), the
+//              prepared B tiles and their correction records (a ring of kSX blocks).
+//   warp 9     allocates tensor memory and issues the 8 MMAs and one commit per block (the
+//              whole warp walks the blocks, one elected lane issues).
 // Tensor memory (128 columns): one A buffer (64 columns) and two accumulators (32 columns). The
 // store of block i waits for the MMAs of block i - 1; block i's MMAs write accumulator i % 2
 // once the epilogue has read block i - 2 from it. Every wait is bounded.
@@ -47,10 +47,10 @@ namespace {
 
 using namespace tc;
 
-constexpr int kThreads = 288;
+constexpr int kThreads = 320;
 constexpr int kCtasPerSm = 3;
 constexpr int kSP = 4;   // packed stages: 8 units of up to 1.5 KB
-constexpr int kSX = 2;   // B tiles (up to 2 atoms x 32 rows x 128 bytes); also the MMA-done ring
+constexpr int kSX = 3;   // B tiles (up to 2 atoms x 32 rows x 128 bytes); also the MMA-done ring
 constexpr int kSC = 4;   // correction records, 256 bytes
 constexpr int kPStage = 8 * 1536;
 constexpr int kXStage = 8 * 1024;
@@ -256,59 +256,77 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_q_kernel(const __gr
     bars->last_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 8) tmem_alloc(&bars->tmem_base, kTmemCols);
+  if (warp == 9) tmem_alloc(&bars->tmem_base, kTmemCols);
   fence_before_sync();
   __syncthreads();
   fence_after_sync();
   const uint32_t tmem = bars->tmem_base;
 
   if (warp == 8) {
-    // ------------------------------------------------------------ control warp (whole warp walks the
-    // blocks, one elected lane issues): weight copies kSP blocks ahead, activation copies two ahead,
-    // and the MMAs of each block once the consumers have stored its codes.
+    // ------------------------------------------------------------ copy warp (whole warp walks the
+    // blocks, one elected lane issues): packed weights (a ring of kSP blocks), prepared B tiles
+    // and their correction records (a ring of kSX blocks)
     constexpr uint32_t bbytes = 256u * XR;
     constexpr uint32_t xtb = bbytes + 256u;   // prepared tile: B atoms, then corrections
+    Pos cp = pos_start(a), cx = cp;            // next block to copy: weights, activations
+    const uint32_t nblocks = cp.left > 0 ? (uint32_t)cp.left : 0u;
+    uint32_t np = 0, nx = 0;                   // weight copies, activation copies issued
+    bool ok = true;
+    while (ok && (np < nblocks || nx < nblocks)) {
+      if (np < nblocks) {
+        // weight stage np % kSP: free once the decode warps have read block np - kSP
+        const int sp = np % kSP;
+        if (!(ok = mbar_wait_bg(&bars->pk_empty[sp], ((np / kSP) & 1) ^ 1, abort_flag, a.err, 101))) break;
+        const int ub = cp.bits == 2 ? 1024 : 1536;
+        const int ntile = min(8, (cp.N + 15) / 16 - cp.rg * 8);
+        if (elect_one()) {
+          mbar_arrive_expect_tx(&bars->pk_full[sp], ntile * ub);
+          bulk_load(ps + sp * kPStage, cp.packed + ((int64_t)cp.rg * 8 * cp.B + (int64_t)cp.b * ntile) * ub,
+                    ntile * ub, &bars->pk_full[sp]);
+        }
+        __syncwarp();
+        pos_next(cp, a);
+        ++np;
+      }
+      if (nx < nblocks) {
+        // activation stage nx % kSX: free once block nx - kSX's MMAs are done; correction slot
+        // nx % kSC once the epilogue has read block nx - kSC
+        const int sx = nx % kSX, sc = nx % kSC;
+        if (!(ok = mbar_wait_bg(&bars->mma_done[sx], ((nx / kSX) & 1) ^ 1, abort_flag, a.err, 102))) break;
+        if (!(ok = mbar_wait_bg(&bars->c_empty[sc], ((nx / kSC) & 1) ^ 1, abort_flag, a.err, 103))) break;
+        const uint8_t* xsrc = cx.xt + (int64_t)cx.b * xtb;
+        if (elect_one()) {
+          mbar_arrive_expect_tx(&bars->x_full[sx], bbytes);
+          bulk_load(xs + sx * kXStage, xsrc, bbytes, &bars->x_full[sx]);
+          mbar_arrive_expect_tx(&bars->c_full[sc], 256);
+          bulk_load(cs + sc * 256, xsrc + bbytes, 256, &bars->c_full[sc]);
+        }
+        __syncwarp();
+        pos_next(cx, a);
+        ++nx;
+      }
+    }
+    if (!ok) {
+      // aborted: let the copies in flight land before the CTA exits
+      for (uint32_t k = np > kSP ? np - kSP : 0; k < np; ++k) mbar_wait_drain(&bars->pk_full[k % kSP], (k / kSP) & 1);
+      for (uint32_t k = nx > kSX ? nx - kSX : 0; k < nx; ++k) mbar_wait_drain(&bars->x_full[k % kSX], (k / kSX) & 1);
+      for (uint32_t k = nx > kSC ? nx - kSC : 0; k < nx; ++k) mbar_wait_drain(&bars->c_full[k % kSC], (k / kSC) & 1);
+    }
+  } else if (warp == 9) {
+    // ------------------------------------------------------------ MMA warp (whole warp, one lane issues)
     const uint64_t bdesc0 = smem_desc_sw128(xs);
     constexpr uint32_t idesc = idesc_i8_m128(XR);
     constexpr uint32_t atom16 = (uint32_t)(XR * 128) >> 4;
-    Pos cp = pos_start(a), cx = cp;            // next block to copy: weights, activations
-    const uint32_t nblocks = cp.left > 0 ? (uint32_t)cp.left : 0u;
-    uint32_t np = 0, nx = 0, gm = 0;           // weight copies, activation copies, MMAs issued
+    const int64_t span = range_start(a.total, blockIdx.x + 1) - range_start(a.total, blockIdx.x);
+    const uint32_t nblocks = span > 0 ? (uint32_t)span : 0u;
+    uint32_t gm = 0;
     bool ok = true;
-    auto copy_weights = [&]() {                // block np into stage np % kSP (free: caller waited)
-      const int ub = cp.bits == 2 ? 1024 : 1536;
-      const int ntile = min(8, (cp.N + 15) / 16 - cp.rg * 8);
-      const int sp = np % kSP;
-      if (elect_one()) {
-        mbar_arrive_expect_tx(&bars->pk_full[sp], ntile * ub);
-        bulk_load(ps + sp * kPStage, cp.packed + ((int64_t)cp.rg * 8 * cp.B + (int64_t)cp.b * ntile) * ub,
-                  ntile * ub, &bars->pk_full[sp]);
-      }
-      __syncwarp();
-      pos_next(cp, a);
-      ++np;
-    };
-    auto copy_acts = [&]() {                   // block nx: B tile into stage nx % kSX, corrections
-      const uint8_t* xsrc = cx.xt + (int64_t)cx.b * xtb;
-      const int sx = nx % kSX, sc = nx % kSC;
-      if (elect_one()) {
-        mbar_arrive_expect_tx(&bars->x_full[sx], bbytes);
-        bulk_load(xs + sx * kXStage, xsrc, bbytes, &bars->x_full[sx]);
-        mbar_arrive_expect_tx(&bars->c_full[sc], 256);
-        bulk_load(cs + sc * 256, xsrc + bbytes, 256, &bars->c_full[sc]);
-      }
-      __syncwarp();
-      pos_next(cx, a);
-      ++nx;
-    };
-    while (np < nblocks && np < (uint32_t)kSP) copy_weights();   // the rings start empty
-    while (nx < nblocks && nx < (uint32_t)kSX) copy_acts();
     for (; gm < nblocks; ++gm) {
       const int sx = gm % kSX;
       if (!(ok = mbar_wait(&bars->a_full, gm & 1, abort_flag, a.err, 201))) break;
       if (!(ok = mbar_wait(&bars->x_full[sx], (gm / kSX) & 1, abort_flag, a.err, 202))) break;
       // accumulator gm % 2 was read by the epilogue warps (block gm - 2)
-      if (!(ok = mbar_wait(&bars->d_empty[gm & 1], ((gm >> 1) & 1) ^ 1, abort_flag, a.err, 206))) break;
+      if (!(ok = mbar_wait(&bars->d_empty[gm & 1], ((gm >> 1) & 1) ^ 1, abort_flag, a.err, 203))) break;
       fence_after_sync();
       const uint64_t bd = bdesc0 + (uint64_t)((sx * kXStage) >> 4);
 #pragma unroll
@@ -318,25 +336,9 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_q_kernel(const __gr
         mma_ts_i8_elect(tmem + kDCol + (gm & 1) * kDCols, tmem + kACol + 8 * j, bd + off, idesc, j != 0);
       }
       mma_commit_elect(&bars->mma_done[sx]);
-      // the consumers released weight stage gm % kSP before they released block gm to us
-      if (np < nblocks) {
-        if (!(ok = mbar_wait(&bars->pk_empty[np % kSP], ((np / kSP) & 1) ^ 1, abort_flag, a.err, 203))) break;
-        copy_weights();
-      }
-      // activation stage gm % kSX is free once block gm's MMAs are done
-      if (nx < nblocks) {
-        if (!(ok = mbar_wait_bg(&bars->mma_done[nx % kSX], ((nx / kSX) & 1) ^ 1, abort_flag, a.err, 204))) break;
-        if (!(ok = mbar_wait_bg(&bars->c_empty[nx % kSC], ((nx / kSC) & 1) ^ 1, abort_flag, a.err, 205))) break;
-        copy_acts();
-      }
     }
-    if (!ok) {
-      // aborted: let the copies and MMAs in flight land before the CTA exits
-      for (uint32_t k = np > kSP ? np - kSP : 0; k < np; ++k) mbar_wait_drain(&bars->pk_full[k % kSP], (k / kSP) & 1);
-      for (uint32_t k = nx > kSX ? nx - kSX : 0; k < nx; ++k) mbar_wait_drain(&bars->x_full[k % kSX], (k / kSX) & 1);
-      for (uint32_t k = nx > kSC ? nx - kSC : 0; k < nx; ++k) mbar_wait_drain(&bars->c_full[k % kSC], (k / kSC) & 1);
-      if (gm > 0) mbar_wait_drain(&bars->mma_done[(gm - 1) % kSX], ((gm - 1) / kSX) & 1);
-    }
+    // the MMAs already issued finish before tensor memory is released
+    if (!ok && gm > 0) mbar_wait_drain(&bars->mma_done[(gm - 1) % kSX], ((gm - 1) / kSX) & 1);
   } else if (warp < 4) {
     // ------------------------------------------------------------ decode (warps 0-3, thread = row)
     const int t = threadIdx.x;                          // row in the row group = TMEM lane
@@ -380,10 +382,17 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_q_kernel(const __gr
       if (lane == 0) mbar_arrive(&bars->group);
       return mbar_wait(&bars->group, (ng++) & 1, abort_flag, a.err, code);
     };
+    // the scale of the block being finished is loaded one block ahead (its latency is an L2
+    // round trip, longer than the work it would wait for)
+    auto scale_of = [&](const Pos& c) -> uint16_t {
+      const int n = c.rg * 128 + t;
+      return (c.left > 0 && n < c.N) ? __ldg(c.scales + (int64_t)n * c.B + c.b) : (uint16_t)0;
+    };
     Pos ec = pos_start(a);
+    uint16_t snext = scale_of(ec);
     for (uint32_t ge = 0; ec.left > 0; ++ge) {
       const int n = ec.rg * 128 + t;
-      const uint16_t sraw = n < ec.N ? __ldg(ec.scales + (int64_t)n * ec.B + ec.b) : (uint16_t)0;
+      const uint16_t sraw = snext;
       const int sc = ge % kSC;
       if (!mbar_wait(&bars->mma_done[ge % kSX], (ge / kSX) & 1, abort_flag, a.err, 303)) break;
       if (!mbar_wait(&bars->c_full[sc], (ge / kSC) & 1, abort_flag, a.err, 304)) break;
@@ -463,13 +472,14 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_q_kernel(const __gr
         for (int m = 0; m < kSlots; ++m) acc[m] = 0.f;
       }
       pos_next(ec, a);
+      snext = scale_of(ec);
     }
   }
 
   fence_before_sync();
   __syncthreads();
   fence_after_sync();
-  if (warp == 8) tmem_dealloc(tmem, kTmemCols);
+  if (warp == 9) tmem_dealloc(tmem, kTmemCols);
 }
 
 // Preparation pass: one warp per (problem, block, token slot m < N/4). The block's activations
