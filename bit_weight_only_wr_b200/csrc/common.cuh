@@ -149,57 +149,70 @@ __device__ __forceinline__ int q3_shift(int k) {
 // ---------------------------------------------------------------- int8 code decoders
 //
 // The integer tensor-core path keeps weights as their unsigned codes c, one byte each; a 32-bit
-// TMEM column holds 4 consecutive K positions of the MMA. The bytes are taken straight out of
-// the packed words, so the K order inside a register is a fixed permutation of the code order;
-// the activation tile is written in the same permuted order (see q2_logical / q3_logical).
+// TMEM column holds 4 consecutive K positions of the MMA. Each byte is cut out of the packed
+// words by a mask and left where the mask finds it, so byte b of a register holds c * 2^e for a
+// position exponent e (the code sits at bits e .. e + bits - 1 of its byte); the activation of
+// that position is divided by 2^e instead (see the preparation pass of the decode GEMV). The
+// K order inside a register is a fixed permutation of the code order, and the activation tile
+// is written in the same order (q2_code_at / q3_code_at, q2_exp_at / q3_exp_at).
 //
-// Q2 word (codes e = 0..15, code e at bits 16*(e&1) + 2*(e>>1)): register s' (0..3) =
-// (w >> 2s') & 0x03030303 holds codes [2s', 2s'+8, 2s'+1, 2s'+9] in bytes 0..3.
-__device__ __forceinline__ void decode_q2_word_i8(uint32_t w, uint32_t r[4]) {
+// Q2 word (codes e = 0..15, code e at bits 16*(e&1) + 2*(e>>1)): register s = w & (3 << 2s in
+// every byte) holds codes [2s, 2s+8, 2s+1, 2s+9] in bytes 0..3, each times 4^s. One AND each.
+__host__ __device__ __forceinline__ void decode_q2_word_i8(uint32_t w, uint32_t r[4]) {
   r[0] = w & 0x03030303u;
-  r[1] = (w >> 2) & 0x03030303u;
-  r[2] = (w >> 4) & 0x03030303u;
-  r[3] = (w >> 6) & 0x03030303u;
+  r[1] = w & 0x0C0C0C0Cu;
+  r[2] = w & 0x30303030u;
+  r[3] = w & 0xC0C0C0C0u;
 }
 
-// Q3 group (3 words, codes 10u + 2j + h at bits 16h + 3j; codes 30 + h in bit 16h + 15 of
-// words 0..2) -> 8 registers:
-//   2u:   [10u,   10u+2, 10u+1, 10u+3]     2u+1: [10u+4, 10u+6, 10u+5, 10u+7]   (u = 0, 1, 2)
-//   6:    [8, 18, 9, 19]                   7:    [28, 30, 29, 31]
-__device__ __forceinline__ void decode_q3_group_i8(const uint32_t w[3], uint32_t r[8]) {
+// Q3 group (3 words, codes 10u + 2j + h at bits 16h + 3j of word u; codes 30 + h have their
+// bit j in bit 16h + 15 of word j) -> 8 registers (code, exponent per byte):
+//   2u:   [10u,   10u+6, 10u+1, 10u+7]  e = 0,1,0,1   (fields j = 0 and j = 3 of word u)
+//   2u+1: [10u+2, 10u+8, 10u+3, 10u+9]  e = 3,4,3,4   (fields j = 1 and j = 4)
+//   6:    [4, 14, 5, 15]                e = 5         (field j = 2 of words 0 and 1: it
+//   7:    [24, 30, 25, 31]              e = 5          crosses a byte, so it is shifted)
+// Six registers are one AND each; the two others gather the byte-crossing fields and the
+// spread codes 30 and 31 with a few shifts.
+__host__ __device__ __forceinline__ void decode_q3_group_i8(const uint32_t w[3], uint32_t r[8]) {
 #pragma unroll
   for (int u = 0; u < 3; ++u) {
-    r[2 * u] = (w[u] & 0x00070007u) | ((w[u] << 5) & 0x07000700u);
-    r[2 * u + 1] = ((w[u] >> 6) & 0x00070007u) | ((w[u] >> 1) & 0x07000700u);
+    r[2 * u] = w[u] & 0x0E070E07u;
+    r[2 * u + 1] = w[u] & 0x70387038u;
   }
-  r[6] = ((w[0] >> 12) & 0x00070007u) | ((w[1] >> 4) & 0x07000700u);
-  r[7] = ((w[2] >> 12) & 0x00070007u) | ((w[0] >> 7) & 0x01000100u) | ((w[1] >> 6) & 0x02000200u) |
-         ((w[2] >> 5) & 0x04000400u);
+  r[6] = ((w[0] >> 1) & 0x00E000E0u) | ((w[1] << 7) & 0xE000E000u);
+  r[7] = ((w[2] >> 1) & 0x00E000E0u) | ((w[0] >> 2) & 0x20002000u) | ((w[1] >> 1) & 0x40004000u) |
+         (w[2] & 0x80008000u);
 }
 
-// Code index (within a 256-code block) held at logical K position kl of the decoded block,
-// for the register orders above. Rows of a block are 4 quarters of 64 codes; a quarter is 16
-// registers (Q2: 4 words x 4; Q3: 2 groups x 8).
+// Code index (within a 256-code block) held at logical K position kl of the decoded block, and
+// the exponent e of its byte, for the register orders above. Rows of a block are 4 quarters of
+// 64 codes; a quarter is 16 registers (Q2: 4 words x 4; Q3: 2 groups x 8).
 __host__ __device__ inline int q2_code_at(int kl) {
   const int q = kl >> 6, w = (kl >> 4) & 3, sp = (kl >> 2) & 3, byte = kl & 3;
   const int p = 2 * sp + ((byte & 1) ? 8 : 0) + (byte >> 1);
   return 64 * q + 16 * w + p;
 }
+__host__ __device__ inline int q2_exp_at(int kl) { return 2 * ((kl >> 2) & 3); }
 __host__ __device__ inline int q3_code_at(int kl) {
   const int q = kl >> 6, g = (kl >> 5) & 1, reg = (kl >> 2) & 7, byte = kl & 3;
   int c;
   if (reg < 6) {
-    const int u = reg >> 1, base = 10 * u + ((reg & 1) ? 4 : 0);
-    const int off[4] = {0, 2, 1, 3};
-    c = base + off[byte];
+    const int u = reg >> 1;
+    const int lo[4] = {0, 6, 1, 7}, hi[4] = {2, 8, 3, 9};
+    c = 10 * u + ((reg & 1) ? hi[byte] : lo[byte]);
   } else if (reg == 6) {
-    const int t[4] = {8, 18, 9, 19};
+    const int t[4] = {4, 14, 5, 15};
     c = t[byte];
   } else {
-    const int t[4] = {28, 30, 29, 31};
+    const int t[4] = {24, 30, 25, 31};
     c = t[byte];
   }
   return 64 * q + 32 * g + c;
+}
+__host__ __device__ inline int q3_exp_at(int kl) {
+  const int reg = (kl >> 2) & 7, byte = kl & 3;
+  if (reg >= 6) return 5;
+  return ((reg & 1) ? 3 : 0) + (byte & 1);
 }
 
 __device__ __forceinline__ float half_bits_to_float(uint16_t h) {

@@ -9,14 +9,16 @@
 //
 //   y[m,n] = sum_b s[n,b] sum_{k in b} g[n,k] x[m,k],   g = 2c - L  (L = 3 or 7)
 //
-// The weights go to tensor memory as their unsigned codes c (one byte each; kind::i8, K = 32
-// per MMA). The activations of a (token, block) are the integers n_k = x_k / 2^E, with
-// E = exponent(max |x|) - 29, written as four balanced signed bytes d_j (n = sum_j 256^j d_j);
-// limb j of token m is B row 4m + j. Every product and block sum is an exact integer,
-//   D_j[n] = sum_k c[n,k] d_j[k],   sum_k g x = 2^E sum_j 256^j (2 D_j - L S_j),
-// with S_j = sum_k d_j[k]. Limbs 0+1 and 2+3 are combined in int32 (below 2^28 in magnitude),
-// the two halves in fp32. Values below 2^E (more than 2^29 under the block maximum) round to a
-// multiple of 2^E: at most 2^-30 max|x| per element.
+// The weights go to tensor memory as their unsigned codes c, one byte each (kind::i8, K = 32 per
+// MMA), each cut out of the packed words by a mask and left in place in its byte: the byte at
+// K position k holds c_k 2^e_k for a fixed position exponent e_k <= 6. The activations of a
+// (token, block) become the integers n_k = x_k / 2^(E + e_k), E = exponent(max |x|) - 30, written
+// as four balanced signed bytes d_j (n = sum_j 256^j d_j); limb j of token m is B row 4m + j.
+// Every product and limb sum is an exact integer,
+//   D_j[n] = sum_k c[n,k] 2^e_k d_j[k],   sum_k g x = 2^E (sum_j 256^j (2 D_j - L S_j)),
+// with S_j = sum_k 2^e_k d_j[k]; the limbs are combined in fp32. Activations below 2^(E + e_k)
+// (more than 2^24 under the block maximum) round to that step: at most 2^-25 max |x| per
+// element, and the fp32 combination adds a few units of 2^-24 of sum |x| per block.
 //
 // A CTA is one small pipeline; three run on every SM so that their latency chains overlap
 // (warp roles, 320 threads):
@@ -323,19 +325,15 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_q_kernel(const __gr
     bool ok = true;
     for (; gm < nblocks; ++gm) {
       const int sx = gm % kSX;
-      if (!(ok = mbar_wait(&bars->a_full, gm & 1, abort_flag, a.err, 201))) break;
+      // the B tile and the accumulator are normally ready long before the codes: wait for them
+      // first, so that the wait for the A handoff is the last one before the MMAs
       if (!(ok = mbar_wait(&bars->x_full[sx], (gm / kSX) & 1, abort_flag, a.err, 202))) break;
       // accumulator gm % 2 was read by the epilogue warps (block gm - 2)
       if (!(ok = mbar_wait(&bars->d_empty[gm & 1], ((gm >> 1) & 1) ^ 1, abort_flag, a.err, 203))) break;
+      if (!(ok = mbar_wait(&bars->a_full, gm & 1, abort_flag, a.err, 201))) break;
       fence_after_sync();
-      const uint64_t bd = bdesc0 + (uint64_t)((sx * kXStage) >> 4);
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        // K slice j: B atom j / 4 (128 K positions x XR rows), 32-byte step inside it
-        const uint64_t off = (uint64_t)((j >> 2) * atom16 + (((j & 3) * 32) >> 4));
-        mma_ts_i8_elect(tmem + kDCol + (gm & 1) * kDCols, tmem + kACol + 8 * j, bd + off, idesc, j != 0);
-      }
-      mma_commit_elect(&bars->mma_done[sx]);
+      mma8_i8_commit_elect(tmem + kDCol + (gm & 1) * kDCols, tmem + kACol,
+                           bdesc0 + (uint64_t)((sx * kXStage) >> 4), atom16, idesc, &bars->mma_done[sx]);
     }
     // the MMAs already issued finish before tensor memory is released
     if (!ok && gm > 0) mbar_wait_drain(&bars->mma_done[(gm - 1) % kSX], ((gm - 1) / kSX) & 1);
@@ -410,12 +408,13 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_q_kernel(const __gr
         for (int mm = 0; mm < kChunk / 4; ++mm) {
           const int m = c0 / 4 + mm;
           if (m < M) {
-            const int4 c = rec[m];
-            // limbs 0+1 and 2+3 in int32, then the halves in fp32
-            const int v01 = (int)d[4 * mm + 1] * 512 + (int)d[4 * mm] * 2 + c.x;
-            const int v23 = (int)d[4 * mm + 3] * 512 + (int)d[4 * mm + 2] * 2 + c.y;
-            const float v = fmaf((float)v23, 65536.f, (float)v01);
-            acc[m] = fmaf(s * __int_as_float(c.z), v, acc[m]);
+            const int2 c = *reinterpret_cast<const int2*>(rec + m);
+            // 2 sum_j 256^j D_j + C in fp32 (each D_j is exact in fp32: |D_j| < 2^23)
+            float v = fmaf((float)(int)d[4 * mm], 2.f, __int_as_float(c.x));
+            v = fmaf((float)(int)d[4 * mm + 1], 512.f, v);
+            v = fmaf((float)(int)d[4 * mm + 2], 131072.f, v);
+            v = fmaf((float)(int)d[4 * mm + 3], 33554432.f, v);
+            acc[m] = fmaf(s * __int_as_float(c.y), v, acc[m]);
           }
         }
       }
@@ -482,14 +481,14 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_q_kernel(const __gr
   if (warp == 9) tmem_dealloc(tmem, kTmemCols);
 }
 
-// Preparation pass: one warp per (problem, block, token slot m < N/4). The block's activations
-// of token m become integers n_k = x_k / 2^E (E = exponent of the block maximum - 29; values
-// that are not multiples of 2^E round to the nearest, ties to even), split into four balanced
-// signed bytes d_j (n = sum_j 256^j d_j, d_j in [-128, 127]). Limb j goes to B row 4m + j (two
-// atoms of 128 K positions x N rows, 128-byte swizzle) at the logical K position whose A byte
-// holds code k. After the atoms, one 16-byte correction record per slot:
-// {C01, C23, bits of 2^E, 0} with S_j = sum_k d_j[k], C01 = -L (S_0 + 256 S_1) and
-// C23 = -L (S_2 + 256 S_3). Slots m >= M hold zero limbs and a zero factor.
+// Preparation pass: one warp per (problem, block, token slot m < N/4). At the logical K position
+// whose A byte holds c_k * 2^e (code k, position exponent e), the activation of token m becomes
+// the integer n = x_k / 2^(E + e) (E = exponent of the block maximum - 30; values that are not
+// multiples of 2^(E + e) round to the nearest, ties to even), split into four balanced signed
+// bytes d_j (n = sum_j 256^j d_j, d_j in [-128, 127]). Limb j goes to B row 4m + j (two atoms of
+// 128 K positions x N rows, 128-byte swizzle). After the atoms, one 16-byte correction record
+// per slot: {C, bits of 2^E, 0, 0} with S_j = sum_k 2^e_k d_j[k] and C = -L sum_j 256^j S_j in
+// fp32. Slots m >= M hold zero limbs and a zero factor.
 __global__ void __launch_bounds__(256) prep_x_kernel(const __grid_constant__ DecArgs a, int total_blocks) {
   const int lane = threadIdx.x & 31;
   const int M = a.M;
@@ -508,19 +507,18 @@ __global__ void __launch_bounds__(256) prep_x_kernel(const __grid_constant__ Dec
   uint8_t* dst = pr.xt + (int64_t)b * xtile_bytes(false, M);
   // lane l holds logical K positions 8l .. 8l+7 of the decoded block
   float xv[8];
+  int pe[8];   // position exponents: the A byte there holds c * 2^pe
   float amax = 0.f;
-  if (m < M) {
-    const uint16_t* xrow = pr.x + (int64_t)m * pr.K + (int64_t)b * 256;
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      const int kl = 8 * lane + e;
+  for (int e = 0; e < 8; ++e) {
+    const int kl = 8 * lane + e;
+    pe[e] = pr.bits == 2 ? q2_exp_at(kl) : q3_exp_at(kl);
+    xv[e] = 0.f;
+    if (m < M) {
       const int k = pr.bits == 2 ? q2_code_at(kl) : q3_code_at(kl);
-      xv[e] = __bfloat162float(__ushort_as_bfloat16(__ldg(xrow + k)));
+      xv[e] = __bfloat162float(__ushort_as_bfloat16(__ldg(pr.x + (int64_t)m * pr.K + (int64_t)b * 256 + k)));
       amax = fmaxf(amax, fabsf(xv[e]));
     }
-  } else {
-#pragma unroll
-    for (int e = 0; e < 8; ++e) xv[e] = 0.f;
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
@@ -528,16 +526,16 @@ __global__ void __launch_bounds__(256) prep_x_kernel(const __grid_constant__ Dec
   if (amax > 0.f) frexpf(amax, &ex);   // amax in [2^(ex-1), 2^ex)
   const int E = ex - 30;                // |n| < 2^30
   uint32_t lw[4][2] = {{0u, 0u}, {0u, 0u}, {0u, 0u}, {0u, 0u}};
-  int s[4] = {0, 0, 0, 0};
+  int s[4] = {0, 0, 0, 0};                // S_j = sum_k 2^pe_k d_j[k]
 #pragma unroll
   for (int e = 0; e < 8; ++e) {
-    const int n = amax > 0.f ? __float2int_rn(ldexpf(xv[e], -E)) : 0;
+    const int n = amax > 0.f ? __float2int_rn(ldexpf(xv[e], -(E + pe[e]))) : 0;
     int rest = n;
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       const int d = j < 3 ? (int)(int8_t)(rest & 0xFF) : rest;
       rest = (rest - d) >> 8;
-      s[j] += d;
+      s[j] += d * (1 << pe[e]);
       lw[j][e >> 2] |= ((uint32_t)d & 0xFFu) << (8 * (e & 3));
     }
   }
@@ -554,11 +552,12 @@ __global__ void __launch_bounds__(256) prep_x_kernel(const __grid_constant__ Dec
     for (int j = 0; j < 4; ++j) s[j] += __shfl_xor_sync(0xffffffffu, s[j], o);
   }
   if (lane == 0) {
-    // correction record of slot m: C01 = -L (S_0 + 256 S_1), C23 = -L (S_2 + 256 S_3), 2^E
+    // correction record of slot m: C = -L sum_j 256^j S_j (exact in fp64, one rounding to
+    // fp32), then 2^E
     const int L = pr.bits == 2 ? 3 : 7;
     const float f = (m < M && amax > 0.f) ? ldexpf(1.f, E) : 0.f;
-    reinterpret_cast<int4*>(dst + 256 * xrows)[m] =
-        make_int4(-L * (s[0] + 256 * s[1]), -L * (s[2] + 256 * s[3]), __float_as_int(f), 0);
+    const double S = (double)s[0] + 256.0 * s[1] + 65536.0 * s[2] + 16777216.0 * s[3];
+    reinterpret_cast<int4*>(dst + 256 * xrows)[m] = make_int4(__float_as_int((float)(-L * S)), __float_as_int(f), 0, 0);
   }
 }
 
