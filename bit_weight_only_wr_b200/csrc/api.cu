@@ -218,33 +218,77 @@ wr_status run_q(int bits, int64_t M, int64_t N, int64_t K, const uint16_t* x, co
   return run_gemm(bits, (int)M, (int)N, (int)K, x, static_cast<const uint8_t*>(packed), scales, y, workspace, stream);
 }
 
-// Ternary: 8-token slices through the decode kernel (R x hi and lo fill the 16 MMA columns).
+// Ternary. M <= 8: the decode kernel (R x hi and lo fill the MMA columns). M > 8: the prefill
+// GEMM over 128-row groups x 64-token tiles (the hi and lo planes of R x make the 128 MMA
+// columns) x K splits; workspace [counters][split-K partials][R x planes [2][M][Kp] bf16].
+struct TGemmPlan {
+  int B = 0, RG = 0, MT = 0, P = 1, items = 0;
+  int64_t Kp = 0;
+  size_t counter_off = 0, partial_off = 0, planes_off = 0, total = 0;
+};
+constexpr int kTernaryTok = 64;   // tokens per GEMM tile
+
+TGemmPlan plan_gemm_t(int64_t M, int64_t N, int64_t K) {
+  TGemmPlan p;
+  p.B = (int)((K + 319) / 320);
+  p.Kp = (int64_t)p.B * 320;
+  p.RG = (int)((N + 127) / 128);
+  p.MT = (int)((M + kTernaryTok - 1) / kTernaryTok);
+  const int64_t base = (int64_t)p.RG * p.MT;
+  if (base < kPlanSMs) p.P = (int)std::min<int64_t>(p.B, (kPlanSMs + base - 1) / base);
+  p.items = (int)(base * p.P);
+  p.counter_off = 0;
+  p.partial_off = align256((size_t)base * sizeof(int));
+  p.planes_off = p.partial_off + (p.P > 1 ? align256((size_t)base * p.P * kTernaryTok * 128 * sizeof(float)) : 0);
+  p.total = p.planes_off + align256((size_t)2 * M * p.Kp * sizeof(uint16_t));
+  return p;
+}
+
 size_t t_workspace(int64_t M, int64_t N, int64_t K) {
+  if (M > kDecodeTokens) return plan_gemm_t(M, N, K).total;
   static thread_local DecodePlan dp;
   const ProblemShape sh{N, K, WR_FMT_TERNARY};
-  plan_decode(std::min<int64_t>(M, 8), 1, &sh, &dp);
+  plan_decode(M, 1, &sh, &dp);
   return dp.total;
 }
 
 wr_status run_t(int64_t M, int64_t N, int64_t K, const uint16_t* x, const void* packed, const uint16_t* alpha,
                 const uint32_t* signs, float* y, void* workspace, cudaStream_t stream) {
-  static thread_local DecodePlan dp;
-  for (int64_t m0 = 0; m0 < M; m0 += 8) {
-    const int mm = (int)std::min<int64_t>(8, M - m0);
+  if (M <= kDecodeTokens) {
+    static thread_local DecodePlan dp;
     const ProblemShape sh{N, K, WR_FMT_TERNARY};
-    plan_decode(mm, 1, &sh, &dp);
+    plan_decode(M, 1, &sh, &dp);
     bind_workspace(dp, workspace);
-    if (wr::launch_rotate_x(x + m0 * K, signs, dp.args.prob[0].xt, mm, (int)K, dp.args.prob[0].Kp, stream) !=
-        cudaSuccess)
+    if (wr::launch_rotate_x(x, signs, dp.args.prob[0].xt, (int)M, (int)K, dp.args.prob[0].Kp, stream) != cudaSuccess)
       return WR_ERR_CUDA;
     dp.args.prob[0].x = nullptr;
     dp.args.prob[0].packed = static_cast<const uint8_t*>(packed);
     dp.args.prob[0].scales = alpha;
-    dp.args.prob[0].y = y + m0 * N;
-    const wr_status st = run_decode(dp, true, stream);
-    if (st != WR_OK) return st;
+    dp.args.prob[0].y = y;
+    return run_decode(dp, true, stream);
   }
-  return WR_OK;
+  const TGemmPlan p = plan_gemm_t(M, N, K);
+  uint8_t* wsb = static_cast<uint8_t*>(workspace);
+  uint8_t* planes = wsb + p.planes_off;
+  if (wr::launch_rotate_planes(x, signs, planes, (int)M, (int)K, p.Kp, stream) != cudaSuccess) return WR_ERR_CUDA;
+  wr::TcArgs a{};
+  a.packed = static_cast<const uint8_t*>(packed);
+  a.alpha = alpha;
+  a.y = y;
+  a.partial = reinterpret_cast<float*>(wsb + p.partial_off);
+  a.counter = reinterpret_cast<int*>(wsb + p.counter_off);
+  a.err = device_error_word();
+  a.M = (int)M;
+  a.N = (int)N;
+  a.K = (int)K;
+  a.B = p.B;
+  a.RG = p.RG;
+  a.MT = p.MT;
+  a.P = p.P;
+  a.items = p.items;
+  const int grid = (int)std::min<int64_t>(p.items, sm_count());
+  return wr::launch_tc_kernel(WR_FMT_TERNARY, 128, a, planes, M, p.Kp, grid, stream) == cudaSuccess ? WR_OK
+                                                                                                : WR_ERR_CUDA;
 }
 
 }  // namespace

@@ -70,6 +70,7 @@ struct Layout {
 struct Bars {
   uint64_t pk_full[kSP], pk_empty[kSP], x_full[kSX], x_empty[kSX];
   uint64_t a_full[2], a_empty[2], d_full[2], d_empty[2];
+  uint64_t group;   // the 8 epilogue warps meet here (bounded, unlike a named barrier)
   uint32_t tmem_base;
   int abort_flag;
   int last_flag;
@@ -177,6 +178,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const TcArgs a, const _
       mbar_init(&bars->d_full[i], 1);
       mbar_init(&bars->d_empty[i], 8);
     }
+    mbar_init(&bars->group, 8);
     bars->abort_flag = 0;
     bars->last_flag = 0;
     fence_barrier_init();
@@ -205,17 +207,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const TcArgs a, const _
             uint8_t* dst = xs + sx * Ly::kXStage + at * Ly::kXAtom;
             const int k = b * F::kUnitK + 64 * at;
             if (FMT == WR_FMT_TERNARY) {
-              // two 8-token boxes: hi plane into rows 0..7, lo plane into rows 8..15
-              asm volatile(
-                  "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, "
-                  "%3, %4}], [%5];" ::"r"(smem_u32(dst)),
-                  "l"(&xmap), "r"(k), "r"(mt * 8), "r"(0), "r"(smem_u32(&bars->x_full[sx]))
-                  : "memory");
-              asm volatile(
-                  "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, "
-                  "%3, %4}], [%5];" ::"r"(smem_u32(dst + 8 * 128)),
-                  "l"(&xmap), "r"(k), "r"(mt * 8), "r"(1), "r"(smem_u32(&bars->x_full[sx]))
-                  : "memory");
+              // two boxes of kTok tokens: the hi plane of R x into rows 0 .. kTok - 1, the lo
+              // plane into rows kTok .. 2 kTok - 1
+              tma_load_3d(dst, &xmap, k, mt * Ly::kTok, 0, &bars->x_full[sx]);
+              tma_load_3d(dst + Ly::kTok * 128, &xmap, k, mt * Ly::kTok, 1, &bars->x_full[sx]);
             } else {
               tma_load_2d(dst, &xmap, k, mt * BN, &bars->x_full[sx]);
             }
@@ -319,7 +314,14 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const TcArgs a, const _
     // ------------------------------------------------------------ epilogue (warps 8-15, thread = row)
     // warps 8 + w and 12 + w share lane quarter w; group e takes tokens e*TH .. e*TH + TH - 1
     constexpr int TOK = Ly::kTok, TH = TOK / 2;
+    static_assert(TH % 16 == 0, "tokens per epilogue group: a multiple of 16");
     const int e = (warp - 8) >> 2, lq = (warp - 8) & 3;
+    uint32_t ng = 0;   // group barrier phases used
+    auto group_sync = [&](int code) {
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->group);
+      return mbar_wait(&bars->group, (ng++) & 1, abort_flag, a.err, code);
+    };
     const int t = 32 * lq + lane;
     const uint32_t lane_addr = (uint32_t)(32 * lq) << 16;
     uint32_t gb = 0, gi = 0;
@@ -337,14 +339,19 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const TcArgs a, const _
         ok = mbar_wait(&bars->d_full[dbuf], (gi >> 1) & 1, abort_flag, a.err, 401);
         if (ok) {
           fence_after_sync();
-          float d[16];
-          tmem_ld16(tmem + lane_addr + Ly::kDCol + dbuf * BN, d);
-          tmem_wait_ld();
+          // column j < TOK holds token j against the hi plane, column TOK + j against the lo plane
+#pragma unroll
+          for (int c0 = 0; c0 < TH; c0 += 16) {
+            float dh[16], dl[16];
+            tmem_ld16(tmem + lane_addr + Ly::kDCol + dbuf * BN + e * TH + c0, dh);
+            tmem_ld16(tmem + lane_addr + Ly::kDCol + dbuf * BN + TOK + e * TH + c0, dl);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 16; ++i) acc[c0 + i] = dh[i] + dl[i];
+          }
           fence_before_sync();
           __syncwarp();
           if (lane == 0) mbar_arrive(&bars->d_empty[dbuf]);
-#pragma unroll
-          for (int i = 0; i < TH; ++i) acc[i] = d[e * TH + i] + d[e * TH + i + 8];
         }
       } else {
         for (int b = b0; b < b1; ++b, ++gb) {
@@ -383,9 +390,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const TcArgs a, const _
         for (int i = 0; i < TH; ++i)
           if (i < mcount) part[i * 128 + t] = acc[i];
         __threadfence();
-        named_bar_sync(1, 256);
+        if (!group_sync(403)) break;
         if (threadIdx.x == 256) bars->last_flag = (atomicAdd(a.counter + tileid, 1) == a.P - 1);
-        named_bar_sync(1, 256);
+        if (!group_sync(404)) break;
         const int last = bars->last_flag;
         if (last) {
           __threadfence();
@@ -405,7 +412,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const TcArgs a, const _
           }
           if (threadIdx.x == 256) a.counter[tileid] = 0;
         }
-        named_bar_sync(1, 256);
+        if (!group_sync(405)) break;
       }
     }
   }
@@ -441,10 +448,10 @@ cudaError_t launch_tc(const TcArgs& a, const void* x_act, int64_t x_rows, int64_
   CUtensorMap map;
   CUresult r;
   if (FMT == WR_FMT_TERNARY) {
-    // R x planes: [2][M][Kp] bf16 -> dims (Kp, M, 2), box (64, 8, 1)
+    // R x planes: [2][M][Kp] bf16 -> dims (Kp, M, 2), box (64 positions, kTok tokens, 1 plane)
     const cuuint64_t dims[3] = {(cuuint64_t)x_k, (cuuint64_t)x_rows, 2};
     const cuuint64_t strides[2] = {(cuuint64_t)x_k * 2, (cuuint64_t)x_k * 2 * x_rows};
-    const cuuint32_t box[3] = {64, 8, 1};
+    const cuuint32_t box[3] = {64, (cuuint32_t)Layout<FMT, BN>::kTok, 1};
     const cuuint32_t estr[3] = {1, 1, 1};
     r = enc(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(x_act), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -472,14 +479,17 @@ cudaError_t launch_tc(const TcArgs& a, const void* x_act, int64_t x_rows, int64_
 }
 
 // R x for the ternary path: one warp per (token, 128-block). x' = (1/sqrt(128)) H (d * x) in
-// fp32, split into hi = bf16(x') and lo = bf16(x' - hi). The values are written as the B tiles
-// the decode kernel copies: per 320-trit unit, 5 atoms of 64 positions and 16 rows (2048 B),
-// hi of token m in row m, lo in row 8 + m (128-byte swizzle: 16-byte chunk c of row r at
-// c ^ (r % 8)). Position 80q + 2P + h of a unit holds trit 80q + 5*(2*(P/5) + h) + P%5 (pair P
-// of byte pair P/5; h selects the byte), the K order of the decoded A columns. Pad trits get 0.
+// fp32, split into hi = bf16(x') and lo = bf16(x' - hi). Inside each 320-trit unit, position
+// 80q + 2P + h holds trit 80q + 5*(2*(P/5) + h) + P%5 (pair P of byte pair P/5; h selects the
+// byte): the K order of the decoded A columns. Pad trits get 0. Two output forms:
+//   tiles (decode GEMV): the B tiles its copy warp loads, per unit 5 atoms of 64 positions and
+//     16 rows (2048 B), hi of token m in row m, lo in row 8 + m (128-byte swizzle: 16-byte chunk
+//     c of row r at c ^ (r % 8));
+//   planes (prefill GEMM): [2][M][Kp] bf16 row-major, hi then lo, read by TMA.
 // One warp: token m, 128-block starting at k0 (lane = 4 consecutive K positions).
+template <bool PLANES>
 __device__ __forceinline__ void rotate_block(const uint16_t* __restrict__ x, const uint32_t* __restrict__ signs,
-                                             uint8_t* __restrict__ xt, int K, int64_t Kp, int m, int64_t k0,
+                                             uint8_t* __restrict__ xt, int M, int K, int64_t Kp, int m, int64_t k0,
                                              int lane) {
   float v[4];
 #pragma unroll
@@ -514,10 +524,17 @@ __device__ __forceinline__ void rotate_block(const uint16_t* __restrict__ x, con
     const int kk = (int)(k % 320), q = kk / 80, i80 = kk % 80, beta = i80 / 5, dig = i80 % 5;
     const int P = 5 * (beta >> 1) + dig;
     const int kp = 80 * q + 2 * P + (beta & 1);
-    const int at = kp >> 6, e = kp & 63;
-    const int64_t off = u * (5 * 2048) + at * 2048 + m * 128 + ((((e >> 3) ^ (m & 7)) << 4) | ((e & 7) << 1));
-    *reinterpret_cast<uint16_t*>(xt + off) = __bfloat16_as_ushort(hi);                 // row m
-    *reinterpret_cast<uint16_t*>(xt + off + 1024) = __bfloat16_as_ushort(lo);          // row 8 + m
+    if (PLANES) {
+      uint16_t* pl = reinterpret_cast<uint16_t*>(xt);
+      const int64_t off = (int64_t)m * Kp + u * 320 + kp;
+      pl[off] = __bfloat16_as_ushort(hi);
+      pl[(int64_t)M * Kp + off] = __bfloat16_as_ushort(lo);
+    } else {
+      const int at = kp >> 6, e = kp & 63;
+      const int64_t off = u * (5 * 2048) + at * 2048 + m * 128 + ((((e >> 3) ^ (m & 7)) << 4) | ((e & 7) << 1));
+      *reinterpret_cast<uint16_t*>(xt + off) = __bfloat16_as_ushort(hi);                 // row m
+      *reinterpret_cast<uint16_t*>(xt + off + 1024) = __bfloat16_as_ushort(lo);          // row 8 + m
+    }
   }
 }
 
@@ -527,7 +544,17 @@ __global__ void rotate_x_kernel(const uint16_t* __restrict__ x, const uint32_t* 
   const int64_t item = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int64_t nblk = (Kp + 127) / 128;
   if (item >= (int64_t)M * nblk) return;
-  rotate_block(x, signs, xt, K, Kp, (int)(item / nblk), (item % nblk) * 128, lane);
+  rotate_block<false>(x, signs, xt, M, K, Kp, (int)(item / nblk), (item % nblk) * 128, lane);
+}
+
+// The planes form, for the prefill GEMM: planes = [2][M][Kp] bf16 (hi, lo).
+__global__ void rotate_planes_kernel(const uint16_t* __restrict__ x, const uint32_t* __restrict__ signs,
+                                     uint8_t* __restrict__ planes, int M, int K, int64_t Kp) {
+  const int lane = threadIdx.x & 31;
+  const int64_t item = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int64_t nblk = (Kp + 127) / 128;
+  if (item >= (int64_t)M * nblk) return;
+  rotate_block<true>(x, signs, planes, M, K, Kp, (int)(item / nblk), (item % nblk) * 128, lane);
 }
 
 // Batched form: work item g -> (problem, token, 128-block) through the problems' first items.
@@ -543,13 +570,13 @@ __global__ void rotate_x_batched_kernel(const __grid_constant__ DecArgs a, int64
   }
   const DecProblem& pr = a.prob[lo];
   const int64_t local = g - pr.xblk_base, nblk = ((int64_t)pr.Kp + 127) / 128;
-  rotate_block(pr.x, pr.signs, pr.xt, pr.K, pr.Kp, (int)(local / nblk), (local % nblk) * 128, lane);
+  rotate_block<false>(pr.x, pr.signs, pr.xt, 0, pr.K, pr.Kp, (int)(local / nblk), (local % nblk) * 128, lane);
 }
 
 }  // namespace
 
 int tc_tmem_cols(int fmt, int bn) {
-  if (fmt == WR_FMT_TERNARY) return Layout<WR_FMT_TERNARY, 16>::kTmemCols;
+  if (fmt == WR_FMT_TERNARY) return Layout<WR_FMT_TERNARY, 128>::kTmemCols;
   if (bn == 16) return Layout<WR_FMT_Q2, 16>::kTmemCols;
   return Layout<WR_FMT_Q2, 128>::kTmemCols;
 }
@@ -558,6 +585,7 @@ cudaError_t launch_tc_kernel(int fmt, int bn, const TcArgs& a, const void* x_act
                              int grid, cudaStream_t stream) {
   if (fmt == WR_FMT_Q2 && bn == 128) return launch_tc<WR_FMT_Q2, 128>(a, x_act, x_rows, x_k, grid, stream);
   if (fmt == WR_FMT_Q3 && bn == 128) return launch_tc<WR_FMT_Q3, 128>(a, x_act, x_rows, x_k, grid, stream);
+  if (fmt == WR_FMT_TERNARY && bn == 128) return launch_tc<WR_FMT_TERNARY, 128>(a, x_act, x_rows, x_k, grid, stream);
   return cudaErrorNotSupported;
 }
 
@@ -567,6 +595,14 @@ cudaError_t launch_rotate_x(const uint16_t* x, const uint32_t* signs, uint8_t* x
   const int warps = 8;
   const int64_t ctas = (items + warps - 1) / warps;
   rotate_x_kernel<<<(unsigned)ctas, warps * 32, 0, stream>>>(x, signs, xt, M, K, Kp);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_rotate_planes(const uint16_t* x, const uint32_t* signs, uint8_t* planes, int M, int K, int64_t Kp,
+                                 cudaStream_t stream) {
+  const int64_t items = (int64_t)M * ((Kp + 127) / 128);
+  const int warps = 8;
+  rotate_planes_kernel<<<(unsigned)((items + warps - 1) / warps), warps * 32, 0, stream>>>(x, signs, planes, M, K, Kp);
   return cudaGetLastError();
 }
 

@@ -81,6 +81,9 @@ cudaError_t launch_rotate_x(const uint16_t* x, const uint32_t* signs, uint8_t* x
                             cudaStream_t stream);
 // The same for every problem of a batch (x, signs, xt, K, Kp per problem; xblk_base = first
 // work item; total_items = M * sum of ceil(Kp / 128)).
+// R x as two bf16 planes [2][M][Kp] (hi, lo) in the decoded K order, for the prefill GEMM.
+cudaError_t launch_rotate_planes(const uint16_t* x, const uint32_t* signs, uint8_t* planes, int M, int K, int64_t Kp,
+                                 cudaStream_t stream);
 cudaError_t launch_rotate_x_batched(const DecArgs& a, int64_t total_items, cudaStream_t stream);
 cudaError_t launch_unpack_bf16(int fmt, const uint8_t* packed, const uint16_t* scales, int N, int K, int units,
                                uint16_t* w, cudaStream_t stream);

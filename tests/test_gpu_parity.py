@@ -245,6 +245,40 @@ def test_gemv_batched_ragged_mixed(wr):
         check_close(y.cpu().numpy(), ref, B)
 
 
+@pytest.mark.parametrize("M", [64, 65, 129])
+@pytest.mark.parametrize("N,K", [(200, 640), (1024, 2560), (256, 4096)])
+def test_ternary_gemm_prefill(wr, M, N, K):
+    """M > 8 runs the tensor-core prefill GEMM: 64-token tiles, ragged N and M, K splits."""
+    torch = torch_mod()
+    codes, alpha, signs, packed, a_d, s_d = t_case(wr, N, K, seed=7 * N + K + M)
+    x = wr_synth.activations_bf16(600 + M, M, K)
+    y = torch.full((M, N), float("nan"), dtype=torch.float32, device="cuda")
+    nb = wr.wr_gemm_ternary_workspace_bytes(M, N, K)
+    ws = _zeros_ws(nb)
+    for _ in range(2):   # the counters left at zero serve a second call
+        y.fill_(float("nan"))
+        wr.wr_gemm_ternary(M, N, K, dev(x), packed, a_d, s_d, y, ws, nb)
+        torch.cuda.synchronize()
+        ref, B = o.gemm_ternary(x, codes, alpha, signs)
+        check_close(y.cpu().numpy(), ref, B)
+
+
+@pytest.mark.parametrize("N,K", [(9728, 2560), (2560, 9728)])
+def test_ternary_gemm_prefill_m512(wr, N, K):
+    """The bench's M = 512 ternary prefill shapes, every output element against the oracle."""
+    torch = torch_mod()
+    M = 512
+    codes, alpha, signs, packed, a_d, s_d = t_case(wr, N, K, seed=N + 3 * K)
+    x = wr_synth.activations_bf16(700, M, K)
+    y = torch.full((M, N), float("nan"), dtype=torch.float32, device="cuda")
+    nb = wr.wr_gemm_ternary_workspace_bytes(M, N, K)
+    ws = _zeros_ws(nb)
+    wr.wr_gemm_ternary(M, N, K, dev(x), packed, a_d, s_d, y, ws, nb)
+    torch.cuda.synchronize()
+    ref, B = o.gemm_ternary(x, codes, alpha, signs)
+    check_close(y.cpu().numpy(), ref, B)
+
+
 # ---------------------------------------------------------------- batched ternary decode GEMV
 
 @pytest.mark.parametrize("M", [1, 6])
