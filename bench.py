@@ -43,6 +43,8 @@ def parse_args():
     p.add_argument("--tokens", type=int, default=1, help="decode tokens M of the headline body (1..8)")
     p.add_argument("--no-extras", action="store_true", help="headline body only")
     p.add_argument("--cpu-seconds", type=float, default=12.0, help="oracle sample budget (0: no CPU baseline)")
+    p.add_argument("--case", default=None,
+                   help="time one prefill GEMM alone and exit (for profiling): gemm:BITS:M:N:K or tgemm:M:N:K")
     return p.parse_args()
 
 
@@ -270,6 +272,10 @@ def main():
     except Exception:
         pass
 
+    if args.case:
+        run_case(args, wr, torch, np, stream, bf16_peak)
+        return
+
     # ---- the body: weights resident in HBM, fresh x per module
     t_setup = time.time()
     mods = []
@@ -389,6 +395,35 @@ def main():
     if dist:
         dist.barrier()
         dist.destroy_process_group()
+
+
+def run_case(args, wr, torch, np, stream, bf16_peak):
+    """One prefill GEMM shape alone, `--warmup` + `--steps` calls in a graph: a small, single-kernel
+    command for profilers."""
+    import wr_synth
+    kind, *dims = args.case.split(":")
+    if kind == "gemm":
+        bits, M, N, K = (int(v) for v in dims)
+        p, s = build_q_module(wr, torch, 5000 + K, N, K, bits)
+        nb = wr.wr_gemm_workspace_bytes(M, N, K, bits)
+        call = lambda x, y, ws: wr.wr_gemm(M, N, K, x, p, s, bits, y, ws, nb)  # noqa: E731
+    elif kind == "tgemm":
+        M, N, K = (int(v) for v in dims)
+        signs = wr_synth.sign_bits(900, K)
+        codes, alpha = wr.wr_quantize_ternary(wr_synth.weights_fp32(800, N, K), signs)
+        p = torch.from_numpy(wr.wr_pack(1, codes)).cuda()
+        a = torch.from_numpy(alpha.view(np.int16)).cuda()
+        sg = torch.from_numpy(signs.view(np.int32)).cuda()
+        nb = wr.wr_gemm_ternary_workspace_bytes(M, N, K)
+        call = lambda x, y, ws: wr.wr_gemm_ternary(M, N, K, x, p, a, sg, y, ws, nb)  # noqa: E731
+    else:
+        raise SystemExit(f"unknown --case {args.case!r}")
+    x = torch.from_numpy(wr_synth.activations_bf16(M, M, K).view(np.int16)).cuda()
+    y = torch.empty(M, N, dtype=torch.float32, device="cuda")
+    ws = torch.zeros(max(nb, 256), dtype=torch.uint8, device="cuda")
+    ms = graph_time_ms(torch, lambda: call(x, y, ws), args.steps, args.warmup, stream) / args.steps
+    tf = 2.0 * M * N * K / ms / 1e9
+    print(json.dumps({"case": args.case, "us": ms * 1e3, "tflops": tf, "pct_bf16_peak": 100 * tf / bf16_peak}))
 
 
 def run_extras(args, wr, torch, np, stream, dist, hbm_peak, bf16_peak):

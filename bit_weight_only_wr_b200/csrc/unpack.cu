@@ -4,8 +4,9 @@
 // expands the container into a bf16 checkpoint, bit-identical across independent re-runs.
 // Here W[n,k] = bf16_RNE(s * g): the fp32 product of an fp16 scale (11 significant bits)
 // and a grid integer (at most 3 bits) is exact, so the one rounding to bf16 is the only one.
-// One warp per packed unit; each lane expands its 64 codes (80 trits) of two rows and
-// writes them as 16-byte stores. The kernel is bound by the 2 bytes/weight it writes.
+// One warp per packed unit; each lane expands its 64 codes (80 trits) of two rows into shared
+// memory, and the warp writes the unit out in whole-row segments. The kernel is bound by the
+// 2 bytes/weight it writes.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -22,14 +23,31 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return a | (b << 16);
 }
 
+constexpr int kUnpackWarps = 4;   // one packed unit per warp
+
 template <int FMT>
-__global__ void __launch_bounds__(256) unpack_kernel(const uint8_t* __restrict__ packed,
-                                                     const uint16_t* __restrict__ scales, int N,
-                                                     int K, int B, int64_t U,
-                                                     uint16_t* __restrict__ out) {
-  const int lane = threadIdx.x & 31;
-  const int64_t u = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+struct UnpackGeom {
+  static constexpr int kUnitK = FMT == WR_FMT_TERNARY ? 320 : 256;    // K positions per unit
+  static constexpr int kRowBytes = 2 * kUnitK;                          // one staged row of bf16
+  static constexpr int kStride = kRowBytes + 16;                        // padded: rows 4 banks apart
+  static constexpr int kChunks = kRowBytes / 16;                        // 16-byte chunks per row
+};
+
+// One warp per packed unit (16 rows x 256 codes, or x 320 trits). Each lane expands the 64 codes
+// (80 trits) of its two rows into shared memory; the warp then writes the unit row by row, 32
+// lanes x 16 bytes = 512 contiguous bytes per store, so that every global store covers whole
+// 128-byte lines.
+template <int FMT>
+__global__ void __launch_bounds__(32 * kUnpackWarps) unpack_kernel(const uint8_t* __restrict__ packed,
+                                                                  const uint16_t* __restrict__ scales, int N,
+                                                                  int K, int B, int64_t U,
+                                                                  uint16_t* __restrict__ out) {
+  using G = UnpackGeom<FMT>;
+  __shared__ __align__(16) uint8_t stage[kUnpackWarps][16 * G::kStride];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int64_t u = (int64_t)blockIdx.x * kUnpackWarps + warp;
   if (u >= U) return;
+  uint8_t* st = stage[warp];
   constexpr int UB = FMT == WR_FMT_Q3 ? 1536 : 1024;
   constexpr int kChunks = FMT == WR_FMT_Q3 ? 3 : 2;
   const uint8_t* base = packed + u * UB;
@@ -51,10 +69,11 @@ __global__ void __launch_bounds__(256) unpack_kernel(const uint8_t* __restrict__
   const int r0 = lane >> 2, q = lane & 3;
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
-    const int64_t n = tn * 16 + r0 + 8 * h;
-    if (n >= N) continue;
+    const int r = r0 + 8 * h;
+    const int64_t n = tn * 16 + r;
+    uint4* srow = reinterpret_cast<uint4*>(st + r * G::kStride);
     if (FMT == WR_FMT_TERNARY) {
-      const float al = half_bits_to_float(scales[n]);
+      const float al = n < N ? half_bits_to_float(scales[n]) : 0.f;
       float v[80];
 #pragma unroll
       for (int beta = 0; beta < 16; ++beta) {
@@ -65,23 +84,17 @@ __global__ void __launch_bounds__(256) unpack_kernel(const uint8_t* __restrict__
           byte /= 3u;
         }
       }
-      const int64_t k0 = ub * 320 + 80 * q;
-      uint16_t* dst = out + n * (int64_t)K + k0;
-      if (k0 + 80 <= K) {
 #pragma unroll
-        for (int i = 0; i < 10; ++i) {
-          uint4 st;
-          st.x = pack_bf16x2(v[8 * i + 0], v[8 * i + 1]);
-          st.y = pack_bf16x2(v[8 * i + 2], v[8 * i + 3]);
-          st.z = pack_bf16x2(v[8 * i + 4], v[8 * i + 5]);
-          st.w = pack_bf16x2(v[8 * i + 6], v[8 * i + 7]);
-          *reinterpret_cast<uint4*>(dst + 8 * i) = st;
-        }
-      } else {
-        for (int i = 0; i < 80 && k0 + i < K; ++i) dst[i] = __bfloat16_as_ushort(__float2bfloat16_rn(v[i]));
+      for (int i = 0; i < 10; ++i) {
+        uint4 w;
+        w.x = pack_bf16x2(v[8 * i + 0], v[8 * i + 1]);
+        w.y = pack_bf16x2(v[8 * i + 2], v[8 * i + 3]);
+        w.z = pack_bf16x2(v[8 * i + 4], v[8 * i + 5]);
+        w.w = pack_bf16x2(v[8 * i + 6], v[8 * i + 7]);
+        srow[10 * q + i] = w;
       }
     } else {
-      const float s = half_bits_to_float(scales[n * B + ub]);
+      const float s = n < N ? half_bits_to_float(scales[n * B + ub]) : 0.f;
       const int L = FMT == WR_FMT_Q2 ? 3 : 7;
       int c[64];
       if (FMT == WR_FMT_Q2) {
@@ -107,15 +120,35 @@ __global__ void __launch_bounds__(256) unpack_kernel(const uint8_t* __restrict__
           }
         }
       }
-      uint16_t* dst = out + n * (int64_t)K + ub * 256 + 64 * q;
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
-        uint4 st;
-        st.x = pack_bf16x2(s * (float)(2 * c[8 * i + 0] - L), s * (float)(2 * c[8 * i + 1] - L));
-        st.y = pack_bf16x2(s * (float)(2 * c[8 * i + 2] - L), s * (float)(2 * c[8 * i + 3] - L));
-        st.z = pack_bf16x2(s * (float)(2 * c[8 * i + 4] - L), s * (float)(2 * c[8 * i + 5] - L));
-        st.w = pack_bf16x2(s * (float)(2 * c[8 * i + 6] - L), s * (float)(2 * c[8 * i + 7] - L));
-        *reinterpret_cast<uint4*>(dst + 8 * i) = st;
+        uint4 w;
+        w.x = pack_bf16x2(s * (float)(2 * c[8 * i + 0] - L), s * (float)(2 * c[8 * i + 1] - L));
+        w.y = pack_bf16x2(s * (float)(2 * c[8 * i + 2] - L), s * (float)(2 * c[8 * i + 3] - L));
+        w.z = pack_bf16x2(s * (float)(2 * c[8 * i + 4] - L), s * (float)(2 * c[8 * i + 5] - L));
+        w.w = pack_bf16x2(s * (float)(2 * c[8 * i + 6] - L), s * (float)(2 * c[8 * i + 7] - L));
+        srow[8 * q + i] = w;
+      }
+    }
+  }
+  __syncwarp();
+  // row by row: chunk j of row r is K positions k0 + 8j .. k0 + 8j + 7
+  const int64_t k0 = ub * G::kUnitK;
+  const bool vec = (K & 7) == 0;   // rows start 16-byte aligned
+  for (int r = 0; r < 16; ++r) {
+    const int64_t n = tn * 16 + r;
+    if (n >= N) break;
+    uint16_t* orow = out + n * (int64_t)K;
+    const uint4* srow = reinterpret_cast<const uint4*>(st + r * G::kStride);
+    for (int j = lane; j < G::kChunks; j += 32) {
+      const int64_t k = k0 + 8 * j;
+      if (k >= K) break;
+      const uint4 w = srow[j];
+      if (vec && k + 8 <= K) {
+        *reinterpret_cast<uint4*>(orow + k) = w;
+      } else {
+        const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+        for (int e = 0; e < 8 && k + e < K; ++e) orow[k + e] = (uint16_t)(ww[e >> 1] >> (16 * (e & 1)));
       }
     }
   }
@@ -127,10 +160,11 @@ cudaError_t launch_unpack_bf16(int fmt, const uint8_t* packed, const uint16_t* s
                                int units, uint16_t* w, cudaStream_t stream) {
   const int64_t tiles = (N + 15) / 16;
   const int64_t U = tiles * units;
-  const unsigned ctas = (unsigned)((U + 7) / 8);
-  if (fmt == WR_FMT_Q2) unpack_kernel<WR_FMT_Q2><<<ctas, 256, 0, stream>>>(packed, scales, N, K, units, U, w);
-  else if (fmt == WR_FMT_Q3) unpack_kernel<WR_FMT_Q3><<<ctas, 256, 0, stream>>>(packed, scales, N, K, units, U, w);
-  else unpack_kernel<WR_FMT_TERNARY><<<ctas, 256, 0, stream>>>(packed, scales, N, K, units, U, w);
+  const unsigned ctas = (unsigned)((U + kUnpackWarps - 1) / kUnpackWarps);
+  constexpr int th = 32 * kUnpackWarps;
+  if (fmt == WR_FMT_Q2) unpack_kernel<WR_FMT_Q2><<<ctas, th, 0, stream>>>(packed, scales, N, K, units, U, w);
+  else if (fmt == WR_FMT_Q3) unpack_kernel<WR_FMT_Q3><<<ctas, th, 0, stream>>>(packed, scales, N, K, units, U, w);
+  else unpack_kernel<WR_FMT_TERNARY><<<ctas, th, 0, stream>>>(packed, scales, N, K, units, U, w);
   return cudaGetLastError();
 }
 
