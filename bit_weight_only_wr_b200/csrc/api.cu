@@ -147,48 +147,56 @@ wr_status run_decode(DecodePlan& dp, bool ternary, cudaStream_t stream) {
   return wr::launch_gemv_q(dp.args, grid, stream) == cudaSuccess ? WR_OK : WR_ERR_CUDA;
 }
 
-// ---- prefill GEMM kernel (M > 8): 128-row groups x 128-token tiles x K splits; workspace
-// [counters: one int per (row group, token tile)][split-K partials].
+// ---- prefill GEMM kernel (M > 8): 128-row groups x token tiles x K blocks, cut "stream-K" into
+// one contiguous range of (tile, block) pairs per CTA; workspace [counters: one int per tile]
+// [two partial tiles per CTA, for the pieces of tiles cut by range ends].
 struct GemmPlan {
-  int B = 0, RG = 0, MT = 0, P = 1, items = 0;
-  size_t counter_off = 0, partial_off = 0, total = 0;
+  int B = 0, RG = 0, MT = 0, grid = 0;
+  int64_t total = 0, Kp = 0;
+  size_t counter_off = 0, partial_off = 0, planes_off = 0, total_bytes = 0;
 };
 
-GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K) {
+// tok: tokens per tile (128; 64 for ternary, whose R x hi and lo planes fill 128 MMA columns);
+// unit_k: K per block (256; 320 trits for ternary).
+GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, int tok, int unit_k) {
   GemmPlan p;
-  p.B = (int)(K / 256);
+  p.B = (int)((K + unit_k - 1) / unit_k);
+  p.Kp = (int64_t)p.B * unit_k;
   p.RG = (int)((N + 127) / 128);
-  p.MT = (int)((M + 127) / 128);
-  const int64_t base = (int64_t)p.RG * p.MT;
-  if (base < kPlanSMs) p.P = (int)std::min<int64_t>(p.B, (kPlanSMs + base - 1) / base);
-  p.items = (int)(base * p.P);
+  p.MT = (int)((M + tok - 1) / tok);
+  p.total = (int64_t)p.RG * p.MT * p.B;
+  p.grid = (int)std::min<int64_t>(p.total, kPlanSMs);
   p.counter_off = 0;
-  p.partial_off = align256((size_t)base * sizeof(int));
-  p.total = p.partial_off + (p.P > 1 ? align256((size_t)base * p.P * 128 * 128 * sizeof(float)) : 0);
+  p.partial_off = align256((size_t)p.RG * p.MT * sizeof(int));
+  p.planes_off = p.partial_off + align256((size_t)p.grid * 2 * tok * 128 * sizeof(float));
+  p.total_bytes = p.planes_off;
   return p;
+}
+
+wr::TcArgs gemm_args(const GemmPlan& p, int64_t M, int64_t N, int64_t K, void* workspace) {
+  uint8_t* wsb = static_cast<uint8_t*>(workspace);
+  wr::TcArgs a{};
+  a.partial = reinterpret_cast<float*>(wsb + p.partial_off);
+  a.counter = reinterpret_cast<int*>(wsb + p.counter_off);
+  a.err = device_error_word();
+  a.M = (int)M;
+  a.N = (int)N;
+  a.K = (int)K;
+  a.B = p.B;
+  a.RG = p.RG;
+  a.MT = p.MT;
+  a.total = p.total;
+  return a;
 }
 
 wr_status run_gemm(int bits, int M, int N, int K, const uint16_t* x, const uint8_t* packed, const uint16_t* scales,
                    float* y, void* workspace, cudaStream_t stream) {
-  const GemmPlan p = plan_gemm(M, N, K);
-  uint8_t* wsb = static_cast<uint8_t*>(workspace);
-  wr::TcArgs a{};
+  const GemmPlan p = plan_gemm(M, N, K, 128, 256);
+  wr::TcArgs a = gemm_args(p, M, N, K, workspace);
   a.packed = packed;
   a.scales = scales;
   a.y = y;
-  a.partial = reinterpret_cast<float*>(wsb + p.partial_off);
-  a.counter = reinterpret_cast<int*>(wsb + p.counter_off);
-  a.err = device_error_word();
-  a.M = M;
-  a.N = N;
-  a.K = K;
-  a.B = p.B;
-  a.RG = p.RG;
-  a.MT = p.MT;
-  a.P = p.P;
-  a.items = p.items;
-  const int grid = (int)std::min<int64_t>(p.items, sm_count());
-  return wr::launch_tc_kernel(bits, 128, a, x, M, K, grid, stream) == cudaSuccess ? WR_OK : WR_ERR_CUDA;
+  return wr::launch_tc_kernel(bits, 128, a, x, M, K, p.grid, stream) == cudaSuccess ? WR_OK : WR_ERR_CUDA;
 }
 
 // One Q2/Q3 call of any M.
@@ -199,7 +207,7 @@ size_t q_workspace(int bits, int64_t M, int64_t N, int64_t K) {
     plan_decode(M, 1, &sh, &dp);
     return dp.total;
   }
-  return plan_gemm(M, N, K).total;
+  return plan_gemm(M, N, K, 128, 256).total_bytes;
 }
 
 wr_status run_q(int bits, int64_t M, int64_t N, int64_t K, const uint16_t* x, const void* packed,
@@ -219,33 +227,18 @@ wr_status run_q(int bits, int64_t M, int64_t N, int64_t K, const uint16_t* x, co
 }
 
 // Ternary. M <= 8: the decode kernel (R x hi and lo fill the MMA columns). M > 8: the prefill
-// GEMM over 128-row groups x 64-token tiles (the hi and lo planes of R x make the 128 MMA
-// columns) x K splits; workspace [counters][split-K partials][R x planes [2][M][Kp] bf16].
-struct TGemmPlan {
-  int B = 0, RG = 0, MT = 0, P = 1, items = 0;
-  int64_t Kp = 0;
-  size_t counter_off = 0, partial_off = 0, planes_off = 0, total = 0;
-};
+// GEMM over 64-token tiles (the hi and lo planes of R x make the 128 MMA columns); its
+// workspace adds the R x planes [2][M][Kp] bf16 after the GEMM's own.
 constexpr int kTernaryTok = 64;   // tokens per GEMM tile
 
-TGemmPlan plan_gemm_t(int64_t M, int64_t N, int64_t K) {
-  TGemmPlan p;
-  p.B = (int)((K + 319) / 320);
-  p.Kp = (int64_t)p.B * 320;
-  p.RG = (int)((N + 127) / 128);
-  p.MT = (int)((M + kTernaryTok - 1) / kTernaryTok);
-  const int64_t base = (int64_t)p.RG * p.MT;
-  if (base < kPlanSMs) p.P = (int)std::min<int64_t>(p.B, (kPlanSMs + base - 1) / base);
-  p.items = (int)(base * p.P);
-  p.counter_off = 0;
-  p.partial_off = align256((size_t)base * sizeof(int));
-  p.planes_off = p.partial_off + (p.P > 1 ? align256((size_t)base * p.P * kTernaryTok * 128 * sizeof(float)) : 0);
-  p.total = p.planes_off + align256((size_t)2 * M * p.Kp * sizeof(uint16_t));
+GemmPlan plan_gemm_t(int64_t M, int64_t N, int64_t K) {
+  GemmPlan p = plan_gemm(M, N, K, kTernaryTok, 320);
+  p.total_bytes = p.planes_off + align256((size_t)2 * M * p.Kp * sizeof(uint16_t));
   return p;
 }
 
 size_t t_workspace(int64_t M, int64_t N, int64_t K) {
-  if (M > kDecodeTokens) return plan_gemm_t(M, N, K).total;
+  if (M > kDecodeTokens) return plan_gemm_t(M, N, K).total_bytes;
   static thread_local DecodePlan dp;
   const ProblemShape sh{N, K, WR_FMT_TERNARY};
   plan_decode(M, 1, &sh, &dp);
@@ -267,28 +260,15 @@ wr_status run_t(int64_t M, int64_t N, int64_t K, const uint16_t* x, const void* 
     dp.args.prob[0].y = y;
     return run_decode(dp, true, stream);
   }
-  const TGemmPlan p = plan_gemm_t(M, N, K);
-  uint8_t* wsb = static_cast<uint8_t*>(workspace);
-  uint8_t* planes = wsb + p.planes_off;
+  const GemmPlan p = plan_gemm_t(M, N, K);
+  uint8_t* planes = static_cast<uint8_t*>(workspace) + p.planes_off;
   if (wr::launch_rotate_planes(x, signs, planes, (int)M, (int)K, p.Kp, stream) != cudaSuccess) return WR_ERR_CUDA;
-  wr::TcArgs a{};
+  wr::TcArgs a = gemm_args(p, M, N, K, workspace);
   a.packed = static_cast<const uint8_t*>(packed);
   a.alpha = alpha;
   a.y = y;
-  a.partial = reinterpret_cast<float*>(wsb + p.partial_off);
-  a.counter = reinterpret_cast<int*>(wsb + p.counter_off);
-  a.err = device_error_word();
-  a.M = (int)M;
-  a.N = (int)N;
-  a.K = (int)K;
-  a.B = p.B;
-  a.RG = p.RG;
-  a.MT = p.MT;
-  a.P = p.P;
-  a.items = p.items;
-  const int grid = (int)std::min<int64_t>(p.items, sm_count());
-  return wr::launch_tc_kernel(WR_FMT_TERNARY, 128, a, planes, M, p.Kp, grid, stream) == cudaSuccess ? WR_OK
-                                                                                                : WR_ERR_CUDA;
+  return wr::launch_tc_kernel(WR_FMT_TERNARY, 128, a, planes, M, p.Kp, p.grid, stream) == cudaSuccess ? WR_OK
+                                                                                                  : WR_ERR_CUDA;
 }
 
 }  // namespace

@@ -19,9 +19,12 @@
 //              that recycle A buffers, activation stages and accumulators.
 //   warps 8-15 epilogue (two per lane quarter, half of the token tile each): per 256-block,
 //              load the fp32 partial from TMEM, multiply by 2*s[n,b] in fp32 and add it to a
-//              register running sum (ternary: once per item); at the
-//              end of an item, write y, or combine split-K pieces through the workspace (the
-//              last of the P pieces to arrive adds them in order p = 0..P-1 and writes y).
+//              register running sum (ternary: one accumulator per piece of a tile); at the end
+//              of a tile (or of the CTA's range), write y, or, for a tile that several ranges
+//              share, leave the piece in a partial slot (the last piece to arrive adds them in
+//              range order and writes y).
+// Work: the (tile, block) pairs are cut into one contiguous range per CTA ("stream-K"), so that
+// every CTA streams the same number of blocks whatever the tile count.
 // Every wait is bounded: a stuck pipeline records an error code and the CTA unwinds.
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -76,13 +79,48 @@ struct Bars {
   int last_flag;
 };
 
-__device__ __forceinline__ void item_coords(const TcArgs& a, int it, int& rg, int& mt, int& p, int& b0, int& b1) {
-  p = it % a.P;
-  const int t = it / a.P;
-  mt = t % a.MT;
-  rg = t / a.MT;
-  b0 = (int)((int64_t)a.B * p / a.P);
-  b1 = (int)((int64_t)a.B * (p + 1) / a.P);
+// Work is split "stream-K": the batch of (tile, block) pairs, tile-major (tile t = rg * MT + mt,
+// token tiles innermost so that a range reuses one row group's weights from L2), is cut into one
+// contiguous range of blocks per CTA. A tile cut by a range boundary is finished from pieces.
+__device__ __forceinline__ int64_t sk_start(int64_t T, int c) { return (int64_t)c * T / gridDim.x; }
+// CTA whose range holds global block g: the largest c with sk_start(c) <= g
+__device__ __forceinline__ int sk_cta_of(int64_t T, int64_t g) { return (int)(((g + 1) * gridDim.x - 1) / T); }
+
+// Position in this CTA's range, advanced block by block without divisions.
+struct SkPos {
+  int64_t g, g1;      // current global block, end of the range
+  int t;              // tile
+  int b;              // block inside the tile
+  int rg, mt;
+  bool first, last;   // the first / last block of this CTA's piece of the tile
+};
+__device__ __forceinline__ void sk_flags(const TcArgs& a, SkPos& p, bool start) {
+  p.first = start || p.b == 0;
+  p.last = p.b == a.B - 1 || p.g == p.g1 - 1;
+}
+__device__ __forceinline__ SkPos sk_begin(const TcArgs& a) {
+  SkPos p;
+  p.g = sk_start(a.total, blockIdx.x);
+  p.g1 = sk_start(a.total, blockIdx.x + 1);
+  const int64_t t = p.g / a.B;
+  p.t = (int)t;
+  p.b = (int)(p.g - t * a.B);
+  p.rg = p.t / a.MT;
+  p.mt = p.t - p.rg * a.MT;
+  sk_flags(a, p, true);
+  return p;
+}
+__device__ __forceinline__ void sk_next(const TcArgs& a, SkPos& p) {
+  ++p.g;
+  if (++p.b == a.B) {
+    p.b = 0;
+    ++p.t;
+    if (++p.mt == a.MT) {
+      p.mt = 0;
+      ++p.rg;
+    }
+  }
+  sk_flags(a, p, false);
 }
 
 // ---------------------------------------------------------------- decode helpers (thread = row)
@@ -195,75 +233,75 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const TcArgs a, const _
       prefetch_tensormap(&xmap);
       uint32_t gb = 0;
       const int tiles = (a.N + 15) / 16;
-      for (int it = blockIdx.x; it < a.items && !*abort_flag; it += gridDim.x) {
-        int rg, mt, p, b0, b1;
-        item_coords(a, it, rg, mt, p, b0, b1);
-        for (int b = b0; b < b1; ++b, ++gb) {
-          const int sx = gb % kSX;
-          if (!mbar_wait_bg(&bars->x_empty[sx], ((gb / kSX) & 1) ^ 1, abort_flag, a.err, 101)) break;
-          mbar_arrive_expect_tx(&bars->x_full[sx], Ly::kXStage);
+      for (SkPos ps_ = sk_begin(a); ps_.g < ps_.g1 && !*abort_flag; sk_next(a, ps_), ++gb) {
+        const int b = ps_.b, rg = ps_.rg, mt = ps_.mt;
+        const int sx = gb % kSX;
+        if (!mbar_wait_bg(&bars->x_empty[sx], ((gb / kSX) & 1) ^ 1, abort_flag, a.err, 101)) break;
+        mbar_arrive_expect_tx(&bars->x_full[sx], Ly::kXStage);
 #pragma unroll
-          for (int at = 0; at < F::kUnitK / 64; ++at) {
-            uint8_t* dst = xs + sx * Ly::kXStage + at * Ly::kXAtom;
-            const int k = b * F::kUnitK + 64 * at;
-            if (FMT == WR_FMT_TERNARY) {
-              // two boxes of kTok tokens: the hi plane of R x into rows 0 .. kTok - 1, the lo
-              // plane into rows kTok .. 2 kTok - 1
-              tma_load_3d(dst, &xmap, k, mt * Ly::kTok, 0, &bars->x_full[sx]);
-              tma_load_3d(dst + Ly::kTok * 128, &xmap, k, mt * Ly::kTok, 1, &bars->x_full[sx]);
-            } else {
-              tma_load_2d(dst, &xmap, k, mt * BN, &bars->x_full[sx]);
-            }
+        for (int at = 0; at < F::kUnitK / 64; ++at) {
+          uint8_t* dst = xs + sx * Ly::kXStage + at * Ly::kXAtom;
+          const int k = b * F::kUnitK + 64 * at;
+          if (FMT == WR_FMT_TERNARY) {
+            // two boxes of kTok tokens: the hi plane of R x into rows 0 .. kTok - 1, the lo
+            // plane into rows kTok .. 2 kTok - 1
+            tma_load_3d(dst, &xmap, k, mt * Ly::kTok, 0, &bars->x_full[sx]);
+            tma_load_3d(dst + Ly::kTok * 128, &xmap, k, mt * Ly::kTok, 1, &bars->x_full[sx]);
+          } else {
+            tma_load_2d(dst, &xmap, k, mt * BN, &bars->x_full[sx]);
           }
-          const int sp = gb % kSP;
-          if (!mbar_wait_bg(&bars->pk_empty[sp], ((gb / kSP) & 1) ^ 1, abort_flag, a.err, 102)) break;
-          const int ntile = min(8, tiles - rg * 8);
-          mbar_arrive_expect_tx(&bars->pk_full[sp], ntile * F::kUnitBytes);
-          bulk_load(ps + sp * Ly::kPStage, a.packed + ((int64_t)rg * 8 * a.B + (int64_t)b * ntile) * F::kUnitBytes,
-                    ntile * F::kUnitBytes, &bars->pk_full[sp]);
         }
+        const int sp = gb % kSP;
+        if (!mbar_wait_bg(&bars->pk_empty[sp], ((gb / kSP) & 1) ^ 1, abort_flag, a.err, 102)) break;
+        const int ntile = min(8, tiles - rg * 8);
+        mbar_arrive_expect_tx(&bars->pk_full[sp], ntile * F::kUnitBytes);
+        bulk_load(ps + sp * Ly::kPStage, a.packed + ((int64_t)rg * 8 * a.B + (int64_t)b * ntile) * F::kUnitBytes,
+                  ntile * F::kUnitBytes, &bars->pk_full[sp]);
       }
     }
   } else if (warp == 17) {
     // ------------------------------------------------------------ MMA issuer (whole warp, one lane issues)
     constexpr uint32_t idesc = idesc_bf16_m128(BN);
-    uint32_t gb = 0, gc = 0, gi = 0;
-    for (int it = blockIdx.x; it < a.items && !*abort_flag; it += gridDim.x, ++gi) {
-      int rg, mt, p, b0, b1;
-      item_coords(a, it, rg, mt, p, b0, b1);
-      bool ok = true;
-      uint32_t dbuf = 0;
+    uint32_t gb = 0, gc = 0, gp = 0;   // blocks, half-block chunks, pieces (ternary accumulators)
+    bool ok = true;
+    uint32_t dbuf = 0;
+    for (SkPos ps_ = sk_begin(a); ps_.g < ps_.g1 && ok && !*abort_flag; sk_next(a, ps_), ++gb) {
       if (FMT == WR_FMT_TERNARY) {
-        dbuf = gi & 1;
-        ok = mbar_wait_bg(&bars->d_empty[dbuf], ((gi >> 1) & 1) ^ 1, abort_flag, a.err, 201);
-      }
-      for (int b = b0; b < b1 && ok; ++b, ++gb) {
-        if (FMT != WR_FMT_TERNARY) {
-          dbuf = gb & 1;
-          if (!(ok = mbar_wait_bg(&bars->d_empty[dbuf], ((gb >> 1) & 1) ^ 1, abort_flag, a.err, 202))) break;
+        // one accumulator per piece: all its blocks add into it
+        if (ps_.first) {
+          dbuf = gp & 1;
+          if (!(ok = mbar_wait_bg(&bars->d_empty[dbuf], ((gp >> 1) & 1) ^ 1, abort_flag, a.err, 201))) break;
         }
-        const int sx = gb % kSX;
-        if (!(ok = mbar_wait_bg(&bars->x_full[sx], (gb / kSX) & 1, abort_flag, a.err, 203))) break;
-        const uint8_t* xst = xs + sx * Ly::kXStage;
-        for (int c = 0; c < 2; ++c, ++gc) {
-          const int sa = gc & 1;
-          if (!(ok = mbar_wait_bg(&bars->a_full[sa], (gc >> 1) & 1, abort_flag, a.err, 204))) break;
-          fence_after_sync();
+      } else {
+        // one accumulator per block (its scale is applied in the epilogue)
+        dbuf = gb & 1;
+        if (!(ok = mbar_wait_bg(&bars->d_empty[dbuf], ((gb >> 1) & 1) ^ 1, abort_flag, a.err, 202))) break;
+      }
+      const int sx = gb % kSX;
+      if (!(ok = mbar_wait_bg(&bars->x_full[sx], (gb / kSX) & 1, abort_flag, a.err, 203))) break;
+      const uint8_t* xst = xs + sx * Ly::kXStage;
+      for (int c = 0; c < 2; ++c, ++gc) {
+        const int sa = gc & 1;
+        if (!(ok = mbar_wait_bg(&bars->a_full[sa], (gc >> 1) & 1, abort_flag, a.err, 204))) break;
+        fence_after_sync();
 #pragma unroll
-          for (int j = 0; j < F::kChunkSteps; ++j) {
-            const int kk = c * (F::kUnitK / 2) + 16 * j;     // K offset inside the block
-            const uint64_t bdesc = smem_desc_sw128(xst + (kk / 64) * Ly::kXAtom + (kk % 64) * 2);
-            const uint32_t acc = (FMT == WR_FMT_TERNARY) ? (uint32_t)(b != b0 || c != 0 || j != 0)
-                                                         : (uint32_t)(c != 0 || j != 0);
-            mma_ts_elect(tmem + Ly::kDCol + dbuf * BN, tmem + sa * Ly::kACols + 8 * j, bdesc, idesc, acc);
-          }
-          mma_commit_elect(&bars->a_empty[sa]);
+        for (int j = 0; j < F::kChunkSteps; ++j) {
+          const int kk = c * (F::kUnitK / 2) + 16 * j;     // K offset inside the block
+          const uint64_t bdesc = smem_desc_sw128(xst + (kk / 64) * Ly::kXAtom + (kk % 64) * 2);
+          const uint32_t acc = (FMT == WR_FMT_TERNARY) ? (uint32_t)(!ps_.first || c != 0 || j != 0)
+                                                       : (uint32_t)(c != 0 || j != 0);
+          mma_ts_elect(tmem + Ly::kDCol + dbuf * BN, tmem + sa * Ly::kACols + 8 * j, bdesc, idesc, acc);
         }
-        if (!ok) break;
-        mma_commit_elect(&bars->x_empty[sx]);
-        if (FMT != WR_FMT_TERNARY) mma_commit_elect(&bars->d_full[dbuf]);
+        mma_commit_elect(&bars->a_empty[sa]);
       }
-      if (FMT == WR_FMT_TERNARY && ok) mma_commit_elect(&bars->d_full[dbuf]);
+      if (!ok) break;
+      mma_commit_elect(&bars->x_empty[sx]);
+      if (FMT != WR_FMT_TERNARY) {
+        mma_commit_elect(&bars->d_full[dbuf]);
+      } else if (ps_.last) {
+        mma_commit_elect(&bars->d_full[dbuf]);
+        ++gp;
+      }
     }
   } else if (warp < 8) {
     // ------------------------------------------------------------ decode (thread = row)
@@ -274,11 +312,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const TcArgs a, const _
     const int tile = t >> 4, r = t & 15, r0 = r & 7, half = r >> 3;
     const uint32_t lane_addr = (uint32_t)(32 * lq) << 16;
     uint32_t gb = 0, gc = 0;
-    for (int it = blockIdx.x; it < a.items && !*abort_flag; it += gridDim.x) {
-      int rg, mt, p, b0, b1;
-      item_coords(a, it, rg, mt, p, b0, b1);
-      bool ok = true;
-      for (int b = b0; b < b1; ++b, ++gb) {
+    bool ok = true;
+    const int64_t nblk = sk_start(a.total, blockIdx.x + 1) - sk_start(a.total, blockIdx.x);
+    for (int64_t gg = 0; gg < nblk && ok && !*abort_flag; ++gg, ++gb) {
+      {
         const int sp = gb % kSP;
         if (!(ok = mbar_wait(&bars->pk_full[sp], (gb / kSP) & 1, abort_flag, a.err, 301))) break;
         const uint8_t* unit = ps + sp * Ly::kPStage + tile * F::kUnitBytes;
@@ -308,7 +345,6 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const TcArgs a, const _
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars->pk_empty[sp]);
       }
-      if (!ok) break;
     }
   } else {
     // ------------------------------------------------------------ epilogue (warps 8-15, thread = row)
@@ -324,83 +360,86 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const TcArgs a, const _
     };
     const int t = 32 * lq + lane;
     const uint32_t lane_addr = (uint32_t)(32 * lq) << 16;
-    uint32_t gb = 0, gi = 0;
-    for (int it = blockIdx.x; it < a.items && !*abort_flag; it += gridDim.x, ++gi) {
-      int rg, mt, p, b0, b1;
-      item_coords(a, it, rg, mt, p, b0, b1);
-      const int n = rg * 128 + t;
-      float acc[TH];
+    uint32_t gb = 0, gp = 0;   // blocks, pieces (ternary accumulators)
+    const int64_t g0 = sk_start(a.total, blockIdx.x);
+    float acc[TH];
+    bool ok = true;
+    for (SkPos ps_ = sk_begin(a); ps_.g < ps_.g1 && ok; sk_next(a, ps_), ++gb) {
+      const int n = ps_.rg * 128 + t;
+      if (ps_.first) {
 #pragma unroll
-      for (int i = 0; i < TH; ++i) acc[i] = 0.f;
-      bool ok = true;
-      if (FMT == WR_FMT_TERNARY) {
-        const uint32_t dbuf = gi & 1;
-        gb += b1 - b0;
-        ok = mbar_wait(&bars->d_full[dbuf], (gi >> 1) & 1, abort_flag, a.err, 401);
-        if (ok) {
-          fence_after_sync();
-          // column j < TOK holds token j against the hi plane, column TOK + j against the lo plane
-#pragma unroll
-          for (int c0 = 0; c0 < TH; c0 += 16) {
-            float dh[16], dl[16];
-            tmem_ld16(tmem + lane_addr + Ly::kDCol + dbuf * BN + e * TH + c0, dh);
-            tmem_ld16(tmem + lane_addr + Ly::kDCol + dbuf * BN + TOK + e * TH + c0, dl);
-            tmem_wait_ld();
-#pragma unroll
-            for (int i = 0; i < 16; ++i) acc[c0 + i] = dh[i] + dl[i];
-          }
-          fence_before_sync();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&bars->d_empty[dbuf]);
-        }
-      } else {
-        for (int b = b0; b < b1; ++b, ++gb) {
-          const uint32_t dbuf = gb & 1;
-          const float s2 = n < a.N ? 2.f * half_bits_to_float(__ldg(a.scales + (int64_t)n * a.B + b)) : 0.f;
-          if (!(ok = mbar_wait(&bars->d_full[dbuf], (gb >> 1) & 1, abort_flag, a.err, 402))) break;
-          fence_after_sync();
-#pragma unroll
-          for (int c0 = 0; c0 < TH; c0 += 16) {
-            float d[16];
-            tmem_ld16(tmem + lane_addr + Ly::kDCol + dbuf * BN + e * TH + c0, d);
-            tmem_wait_ld();
-#pragma unroll
-            for (int i = 0; i < 16; ++i) acc[c0 + i] = fmaf(s2, d[i], acc[c0 + i]);
-          }
-          fence_before_sync();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&bars->d_empty[dbuf]);
-        }
+        for (int i = 0; i < TH; ++i) acc[i] = 0.f;
       }
-      if (!ok) break;
-      // ---- output: direct store, or split-K combine through the workspace
-      const int m0 = mt * TOK + e * TH;
+      if (FMT == WR_FMT_TERNARY) {
+        if (!ps_.last) continue;
+        // the piece's accumulator: column j < TOK holds token j against the hi plane of R x,
+        // column TOK + j against the lo plane
+        const uint32_t dbuf = gp & 1;
+        ok = mbar_wait(&bars->d_full[dbuf], (gp >> 1) & 1, abort_flag, a.err, 401);
+        ++gp;
+        if (!ok) break;
+        fence_after_sync();
+#pragma unroll
+        for (int c0 = 0; c0 < TH; c0 += 16) {
+          float dh[16], dl[16];
+          tmem_ld16(tmem + lane_addr + Ly::kDCol + dbuf * BN + e * TH + c0, dh);
+          tmem_ld16(tmem + lane_addr + Ly::kDCol + dbuf * BN + TOK + e * TH + c0, dl);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 16; ++i) acc[c0 + i] = dh[i] + dl[i];
+        }
+        fence_before_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->d_empty[dbuf]);
+      } else {
+        const uint32_t dbuf = gb & 1;
+        const float s2 = n < a.N ? 2.f * half_bits_to_float(__ldg(a.scales + (int64_t)n * a.B + ps_.b)) : 0.f;
+        if (!(ok = mbar_wait(&bars->d_full[dbuf], (gb >> 1) & 1, abort_flag, a.err, 402))) break;
+        fence_after_sync();
+#pragma unroll
+        for (int c0 = 0; c0 < TH; c0 += 16) {
+          float d[16];
+          tmem_ld16(tmem + lane_addr + Ly::kDCol + dbuf * BN + e * TH + c0, d);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 16; ++i) acc[c0 + i] = fmaf(s2, d[i], acc[c0 + i]);
+        }
+        fence_before_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->d_empty[dbuf]);
+      }
+      if (!ps_.last) continue;
+      // ---- output: y directly, or, for a tile that several CTA ranges share, the combine
+      // through the partial slots (the last range to arrive adds the pieces in range order)
+      const int m0 = ps_.mt * TOK + e * TH;
       const int mcount = max(0, min(TH, a.M - m0));
       const float rs = (FMT == WR_FMT_TERNARY && n < a.N) ? half_bits_to_float(__ldg(a.alpha + n)) : 1.f;
-      if (a.P == 1) {
+      const int64_t tb = (int64_t)ps_.t * a.B;   // first block of the tile
+      const int c0 = sk_cta_of(a.total, tb), c1 = sk_cta_of(a.total, tb + a.B - 1);
+      if (c0 == c1) {
         if (n < a.N) {
 #pragma unroll
           for (int i = 0; i < TH; ++i)
             if (i < mcount) a.y[(int64_t)(m0 + i) * a.N + n] = rs * acc[i];
         }
       } else {
-        const int tileid = rg * a.MT + mt;
-        float* part = a.partial + ((int64_t)tileid * a.P + p) * (TOK * 128) + (int64_t)e * TH * 128;
+        // slot 0: the tile began before this range; slot 1: it continues after it
+        const int slot = tb < g0 ? 0 : 1;
+        float* part = a.partial + ((int64_t)blockIdx.x * 2 + slot) * (TOK * 128) + (int64_t)e * TH * 128;
 #pragma unroll
         for (int i = 0; i < TH; ++i)
           if (i < mcount) part[i * 128 + t] = acc[i];
         __threadfence();
-        if (!group_sync(403)) break;
-        if (threadIdx.x == 256) bars->last_flag = (atomicAdd(a.counter + tileid, 1) == a.P - 1);
-        if (!group_sync(404)) break;
-        const int last = bars->last_flag;
-        if (last) {
+        if (!(ok = group_sync(403))) break;
+        if (threadIdx.x == 256) bars->last_flag = (atomicAdd(a.counter + ps_.t, 1) == c1 - c0);
+        if (!(ok = group_sync(404))) break;
+        if (bars->last_flag) {
           __threadfence();
-          // the pieces in order p = 0 .. P-1 (this one included), into acc
 #pragma unroll
           for (int i = 0; i < TH; ++i) acc[i] = 0.f;
-          for (int pp = 0; pp < a.P; ++pp) {
-            const float* src = a.partial + ((int64_t)tileid * a.P + pp) * (TOK * 128) + (int64_t)e * TH * 128;
+          for (int c = c0; c <= c1; ++c) {
+            const int sl = tb < sk_start(a.total, c) ? 0 : 1;
+            const float* src = a.partial + ((int64_t)c * 2 + sl) * (TOK * 128) + (int64_t)e * TH * 128;
 #pragma unroll
             for (int i = 0; i < TH; ++i)
               if (i < mcount) acc[i] += __ldcg(src + i * 128 + t);
@@ -410,9 +449,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const TcArgs a, const _
             for (int i = 0; i < TH; ++i)
               if (i < mcount) a.y[(int64_t)(m0 + i) * a.N + n] = rs * acc[i];
           }
-          if (threadIdx.x == 256) a.counter[tileid] = 0;
+          if (threadIdx.x == 256) a.counter[ps_.t] = 0;
         }
-        if (!group_sync(405)) break;
+        if (!(ok = group_sync(405))) break;
       }
     }
   }

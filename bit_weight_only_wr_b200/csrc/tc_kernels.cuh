@@ -10,15 +10,14 @@ struct TcArgs {
   const uint16_t* scales;    // fp16 [N, K/256] (Q2/Q3)
   const uint16_t* alpha;     // fp16 [N] (ternary)
   float* y;                  // fp32 [M, N]
-  float* partial;            // split-K partials [RG*MT][P][TOK][128]
+  float* partial;            // pieces of tiles cut by range ends [grid][2][TOK][128]
   int* counter;              // [RG*MT] arrival counters, zero between calls
   int* err;                  // device error word (bounded waits)
   int M, N, K;
   int B;                     // 256-code (or 320-trit) blocks per row
   int RG;                    // 128-row groups
   int MT;                    // token tiles
-  int P;                     // K splits per (row group, token tile)
-  int items;                 // RG * MT * P
+  int64_t total;             // RG * MT * B (tile, block) pairs, cut into one range per CTA
 };
 
 // Batched decode GEMV (M <= 8): one launch over up to kMaxDecodeProblems independent problems.
