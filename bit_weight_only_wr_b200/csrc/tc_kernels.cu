@@ -42,6 +42,7 @@ using namespace tc;
 constexpr int kThreads = 576;
 constexpr int kSP = 4;  // packed-unit stages
 constexpr int kSX = 2;  // activation stages (per block)
+constexpr int kSA = 3;  // A buffers in tensor memory (half-block chunks)
 
 template <int FMT>
 struct Fmt {
@@ -65,19 +66,21 @@ struct Layout {
   static constexpr int kSmemRaw = kBarOff + 256 + 1024;
   static constexpr int kSmem = (BN == 16 && kSmemRaw < 80 * 1024) ? 80 * 1024 : kSmemRaw;
   static constexpr int kACols = Fmt<FMT>::kChunkCols;
-  static constexpr int kDCol = 2 * kACols;
+  static constexpr int kDCol = kSA * kACols;
   static constexpr int kTmemCols = (kDCol + 2 * BN) <= 256 ? 256 : 512;
+  static_assert(kDCol + 2 * BN <= 512, "tensor memory of the SM");
   static constexpr int kTok = FMT == WR_FMT_TERNARY ? BN / 2 : BN;      // tokens per tile
 };
 
 struct Bars {
   uint64_t pk_full[kSP], pk_empty[kSP], x_full[kSX], x_empty[kSX];
-  uint64_t a_full[2], a_empty[2], d_full[2], d_empty[2];
+  uint64_t a_full[kSA], a_empty[kSA], d_full[2], d_empty[2];
   uint64_t group;   // the 8 epilogue warps meet here (bounded, unlike a named barrier)
   uint32_t tmem_base;
   int abort_flag;
   int last_flag;
 };
+static_assert(sizeof(Bars) <= 256, "barrier area");
 
 // Work is split "stream-K": the batch of (tile, block) pairs, tile-major (tile t = rg * MT + mt,
 // token tiles innermost so that a range reuses one row group's weights from L2), is cut into one
@@ -211,10 +214,12 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const TcArgs a, const _
       mbar_init(&bars->x_empty[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&bars->a_full[i], 8);
-      mbar_init(&bars->a_empty[i], 1);
       mbar_init(&bars->d_full[i], 1);
       mbar_init(&bars->d_empty[i], 8);
+    }
+    for (int i = 0; i < kSA; ++i) {
+      mbar_init(&bars->a_full[i], 8);
+      mbar_init(&bars->a_empty[i], 1);
     }
     mbar_init(&bars->group, 8);
     bars->abort_flag = 0;
@@ -281,8 +286,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const TcArgs a, const _
       if (!(ok = mbar_wait_bg(&bars->x_full[sx], (gb / kSX) & 1, abort_flag, a.err, 203))) break;
       const uint8_t* xst = xs + sx * Ly::kXStage;
       for (int c = 0; c < 2; ++c, ++gc) {
-        const int sa = gc & 1;
-        if (!(ok = mbar_wait_bg(&bars->a_full[sa], (gc >> 1) & 1, abort_flag, a.err, 204))) break;
+        const int sa = gc % kSA;
+        if (!(ok = mbar_wait_bg(&bars->a_full[sa], (gc / kSA) & 1, abort_flag, a.err, 204))) break;
         fence_after_sync();
 #pragma unroll
         for (int j = 0; j < F::kChunkSteps; ++j) {
@@ -320,8 +325,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const TcArgs a, const _
         if (!(ok = mbar_wait(&bars->pk_full[sp], (gb / kSP) & 1, abort_flag, a.err, 301))) break;
         const uint8_t* unit = ps + sp * Ly::kPStage + tile * F::kUnitBytes;
         for (int c = 0; c < 2; ++c, ++gc) {
-          const int sa = gc & 1;
-          if (!(ok = mbar_wait(&bars->a_empty[sa], ((gc >> 1) & 1) ^ 1, abort_flag, a.err, 302))) break;
+          const int sa = gc % kSA;
+          if (!(ok = mbar_wait(&bars->a_empty[sa], ((gc / kSA) & 1) ^ 1, abort_flag, a.err, 302))) break;
           fence_after_sync();
           const int q = 2 * c + g;
           const uint32_t col = tmem + lane_addr + sa * Ly::kACols + g * F::kQuarterCols;
