@@ -19,7 +19,7 @@ __all__ = [
     "wr_gemm_workspace_bytes", "wr_gemm", "wr_gemm_ternary_workspace_bytes", "wr_gemm_ternary",
     "wr_get_device_error", "exported_symbols", "WrGemvProblem", "wr_gemv_batched_workspace_bytes",
     "wr_gemv_batched", "wr_gemv_noalloc", "WR_GEMV_NOALLOC_SCRATCH_BYTES", "WrGemvTernaryProblem",
-    "wr_gemv_ternary_batched_workspace_bytes", "wr_gemv_ternary_batched",
+    "wr_gemv_ternary_batched_workspace_bytes", "wr_gemv_ternary_batched", "wr_selftest_wait_timeout",
 ]
 
 WR_FMT_TERNARY, WR_FMT_Q2, WR_FMT_Q3 = 1, 2, 3
@@ -65,6 +65,7 @@ _SIGNATURES = {
     "wr_gemm_ternary_workspace_bytes": (_c_size, [_c_i64, _c_i64, _c_i64]),
     "wr_gemm_ternary": (_c_int, [_c_i64, _c_i64, _c_i64, _vp, _vp, _vp, _vp, _vp, _vp, _c_size, _vp]),
     "wr_get_device_error": (_c_int, [_vp]),
+    "wr_selftest_wait_timeout": (_c_int, [_vp]),
     "wr_gemv_noalloc": (_c_int, [_c_i64, _c_i64, _c_i64, _vp, _vp, _vp, _c_int, _c_int, _vp, _vp]),
     "wr_gemv_ternary_batched_workspace_bytes": (_c_size, [_c_i64, ctypes.c_int32, _TPROBLEMS]),
     "wr_gemv_ternary_batched": (_c_int, [_c_i64, ctypes.c_int32, _TPROBLEMS, _vp, _c_size, _vp]),
@@ -259,3 +260,8 @@ def wr_gemm_ternary(M: int, N: int, K: int, x, packed, alpha, sign_bits, y, work
 
 def wr_get_device_error(stream=None) -> int:
     return _lib.wr_get_device_error(_stream(stream))
+
+
+def wr_selftest_wait_timeout(stream=None) -> None:
+    """Launch the failure-path self-test (a bounded wait that runs out after one second)."""
+    _check("wr_selftest_wait_timeout", _lib.wr_selftest_wait_timeout(_stream(stream)))

@@ -507,6 +507,12 @@ wr_status wr_gemm_ternary(int64_t M, int64_t N, int64_t K, const uint16_t* x, co
   return run_t(M, N, K, x, packed, alpha, sign_bits, y, workspace, static_cast<cudaStream_t>(stream));
 }
 
+wr_status wr_selftest_wait_timeout(void* stream) {
+  if (wr::launch_selftest_wait_timeout(device_error_word(), static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return WR_ERR_CUDA;
+  return WR_OK;
+}
+
 wr_status wr_get_device_error(void* stream) {
   if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return WR_ERR_CUDA;
   int v = 0;

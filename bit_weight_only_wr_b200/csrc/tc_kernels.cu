@@ -617,7 +617,33 @@ __global__ void rotate_x_batched_kernel(const __grid_constant__ DecArgs a, int64
   rotate_block<false>(pr.x, pr.signs, pr.xt, 0, pr.K, pr.Kp, (int)(local / nblk), (local % nblk) * 128, lane);
 }
 
+// Failure-path self-test: warp 0 waits on a barrier nobody arrives on until the bounded wait
+// gives up (error code 901, abort flag raised); warp 1 waits on another such barrier and
+// leaves on the abort flag (code 902 only if it ran out of time on its own first).
+__global__ void __launch_bounds__(64) selftest_wait_timeout_kernel(int* err_word) {
+  __shared__ __align__(8) uint64_t bar[2];
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar[0], 1);
+    mbar_init(&bar[1], 1);
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  const int warp = threadIdx.x >> 5;
+  if (warp == 0) {
+    mbar_wait(&bar[0], 0, &abort_flag, err_word, 901);
+  } else {
+    mbar_wait(&bar[1], 0, &abort_flag, err_word, 902);
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_selftest_wait_timeout(int* err_word, cudaStream_t stream) {
+  selftest_wait_timeout_kernel<<<1, 64, 0, stream>>>(err_word);
+  return cudaGetLastError();
+}
 
 int tc_tmem_cols(int fmt, int bn) {
   if (fmt == WR_FMT_TERNARY) return Layout<WR_FMT_TERNARY, 128>::kTmemCols;

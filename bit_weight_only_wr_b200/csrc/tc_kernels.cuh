@@ -84,6 +84,8 @@ cudaError_t launch_rotate_x(const uint16_t* x, const uint32_t* signs, uint8_t* x
 cudaError_t launch_rotate_planes(const uint16_t* x, const uint32_t* signs, uint8_t* planes, int M, int K, int64_t Kp,
                                  cudaStream_t stream);
 cudaError_t launch_rotate_x_batched(const DecArgs& a, int64_t total_items, cudaStream_t stream);
+// Failure-path self-test: a bounded wait on a barrier that never completes (see wr.h).
+cudaError_t launch_selftest_wait_timeout(int* err_word, cudaStream_t stream);
 cudaError_t launch_unpack_bf16(int fmt, const uint8_t* packed, const uint16_t* scales, int N, int K, int units,
                                uint16_t* w, cudaStream_t stream);
 

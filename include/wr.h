@@ -218,6 +218,15 @@ wr_status wr_gemv_ternary_batched(int64_t M, int32_t count, const wr_gemv_ternar
  * (synchronizes the stream). WR_OK when no wait timed out since the last call. */
 wr_status wr_get_device_error(void* stream);
 
+/* Self-test of the failure path that every kernel uses (no counterpart in the pages). Launches
+ * one CTA of two warps on `stream`. Warp 0 waits, through the same bounded wait as the
+ * kernels, on an mbarrier that nothing arrives on. After the wait limit (one second) it
+ * records its code in the device error word and raises the CTA's abort flag. Warp 1 waits on
+ * a second such barrier and leaves when it sees the flag. The kernel then returns normally:
+ * nothing faults, traps or hangs, and the context stays usable. Returns WR_OK once launched;
+ * wr_get_device_error(stream) then returns WR_ERR_TIMEOUT (and clears the word). */
+wr_status wr_selftest_wait_timeout(void* stream);
+
 #ifdef __cplusplus
 }
 #endif
