@@ -146,6 +146,10 @@ __device__ __forceinline__ int q3_shift(int k) {
   return 7 - ((P == 15 || (P % 5) % 2 == 0) ? 1 : 4);
 }
 
+// Position of lane l = 4 r0 + q's chunks inside a 32-chunk row of a packed unit (the swizzle
+// of the layout in include/wr.h).
+__host__ __device__ __forceinline__ int lane_pos(int r0, int q) { return 4 * r0 + (q ^ ((r0 >> 1) & 3)); }
+
 // ---------------------------------------------------------------- int8 code decoders
 //
 // The integer tensor-core path keeps weights as their unsigned codes c, one byte each; a 32-bit

@@ -168,7 +168,7 @@ __device__ __forceinline__ void lite_next(Lite& p, const DecArgs& a) {
 __device__ __forceinline__ void q2_half_i8(const uint8_t* unit, int r0, int half, int h, uint32_t v[32]) {
 #pragma unroll
   for (int qq = 0; qq < 2; ++qq) {
-    const uint4 c = *reinterpret_cast<const uint4*>(unit + (32 * half + 4 * r0 + 2 * h + qq) * 16);
+    const uint4 c = *reinterpret_cast<const uint4*>(unit + (32 * half + lane_pos(r0, 2 * h + qq)) * 16);
     decode_q2_word_i8(c.x, v + 16 * qq + 0);
     decode_q2_word_i8(c.y, v + 16 * qq + 4);
     decode_q2_word_i8(c.z, v + 16 * qq + 8);
@@ -179,7 +179,7 @@ __device__ __forceinline__ void q2_half_i8(const uint8_t* unit, int r0, int half
 __device__ __forceinline__ void q3_half_i8(const uint8_t* unit, int r0, int half, int h, uint32_t v[32]) {
 #pragma unroll
   for (int qq = 0; qq < 2; ++qq) {
-    const int l = 4 * r0 + 2 * h + qq;
+    const int l = lane_pos(r0, 2 * h + qq);
     uint32_t w[6];
     if (half == 0) {
       const uint4 c0 = *reinterpret_cast<const uint4*>(unit + l * 16);

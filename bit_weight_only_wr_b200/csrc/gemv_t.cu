@@ -87,7 +87,7 @@ __device__ __forceinline__ Item find_item(const DecArgs& a, int it) {
 // in include/wr.h.
 __device__ __forceinline__ void t_quarter(const uint8_t* unit, int r0, int half, int q, const uint32_t* lut_lo,
                                           const uint32_t* lut_hi, uint32_t v[40]) {
-  const uint4 c = *reinterpret_cast<const uint4*>(unit + (32 * half + 4 * r0 + q) * 16);
+  const uint4 c = *reinterpret_cast<const uint4*>(unit + (32 * half + lane_pos(r0, q)) * 16);
   const uint32_t wv[4] = {c.x, c.y, c.z, c.w};
 #pragma unroll
   for (int w = 0; w < 4; ++w) {

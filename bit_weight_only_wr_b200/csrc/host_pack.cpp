@@ -49,8 +49,12 @@ inline int64_t unit_index(const Geometry& g, int64_t tn, int64_t u) {
   return 8 * grp * g.units + u * tg + tn % 8;
 }
 
-// Byte offset inside a unit of lane-byte `lb` of lane `lane`.
-inline int64_t unit_offset(int lane, int lb) { return (int64_t)(32 * (lb / 16) + lane) * 16 + lb % 16; }
+// Byte offset inside a unit of lane-byte `lb` of lane `lane`: chunk lb / 16 of the lane sits at
+// position lane ^ ((lane >> 3) & 3) of its 32-chunk row, so that the 8 lanes r0 = 0..7 of one
+// quarter land on 8 different 16-byte bank groups.
+inline int64_t unit_offset(int lane, int lb) {
+  return (int64_t)(32 * (lb / 16) + (lane ^ ((lane >> 3) & 3))) * 16 + lb % 16;
+}
 
 inline void put_word(uint8_t* unit, int lane, int lb, uint32_t w) {
   const int64_t off = unit_offset(lane, lb);   // lb is a multiple of 4: never crosses a chunk

@@ -128,19 +128,19 @@ __device__ __forceinline__ void sk_next(const TcArgs& a, SkPos& p) {
 
 // ---------------------------------------------------------------- decode helpers (thread = row)
 
-// Q2: the row's quarter q of a unit is 16 bytes at lane chunk (32*half + 4*r0 + q).
+// Q2: the row's quarter q of a unit is 16 bytes at chunk (32*half + lane_pos(r0, q)).
 __device__ __forceinline__ void decode_q2_quarter(const uint8_t* unit, int r0, int half, int q, uint32_t v[32]) {
-  const uint4 c = *reinterpret_cast<const uint4*>(unit + (32 * half + 4 * r0 + q) * 16);
+  const uint4 c = *reinterpret_cast<const uint4*>(unit + (32 * half + lane_pos(r0, q)) * 16);
   decode_q2_word(c.x, v + 0);
   decode_q2_word(c.y, v + 8);
   decode_q2_word(c.z, v + 16);
   decode_q2_word(c.w, v + 24);
 }
 
-// Q3: lane l = 4*r0 + q holds 48 bytes in chunks (32c + l)*16; row half h uses lane bytes
-// 24h .. 24h+23, i.e. two 12-byte groups of 3 words.
+// Q3: lane 4*r0 + q holds 48 bytes in chunks (32c + lane_pos(r0, q))*16; row half h uses lane
+// bytes 24h .. 24h+23, i.e. two 12-byte groups of 3 words.
 __device__ __forceinline__ void decode_q3_quarter(const uint8_t* unit, int r0, int half, int q, uint32_t v[32]) {
-  const int l = 4 * r0 + q;
+  const int l = lane_pos(r0, q);
   uint32_t w[6];
   if (half == 0) {
     const uint4 c0 = *reinterpret_cast<const uint4*>(unit + l * 16);
@@ -159,7 +159,7 @@ __device__ __forceinline__ void decode_q3_quarter(const uint8_t* unit, int r0, i
 // 5b'..5b'+4, pair i = (trit i of byte 2b', trit i of byte 2b'+1).
 __device__ __forceinline__ void decode_t_quarter(const uint8_t* unit, int r0, int half, int q,
                                                  const uint32_t* lut_lo, const uint32_t* lut_hi, uint32_t v[40]) {
-  const uint4 c = *reinterpret_cast<const uint4*>(unit + (32 * half + 4 * r0 + q) * 16);
+  const uint4 c = *reinterpret_cast<const uint4*>(unit + (32 * half + lane_pos(r0, q)) * 16);
   const uint32_t wv[4] = {c.x, c.y, c.z, c.w};
 #pragma unroll
   for (int w = 0; w < 4; ++w) {

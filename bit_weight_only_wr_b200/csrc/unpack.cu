@@ -66,7 +66,9 @@ __global__ void __launch_bounds__(32 * kUnpackWarps) unpack_kernel(const uint8_t
   const int64_t tg = min((int64_t)8, tiles - 8 * grp);
   const int64_t rem = u - grp * 8 * (int64_t)B;
   const int64_t ub = rem / tg, tn = 8 * grp + rem % tg;
-  const int r0 = lane >> 2, q = lane & 3;
+  // this thread read the chunks at position `lane`, which belong to lane lane ^ ((lane >> 3) & 3)
+  const int ll = lane ^ ((lane >> 3) & 3);
+  const int r0 = ll >> 2, q = ll & 3;
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
     const int r = r0 + 8 * h;

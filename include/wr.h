@@ -39,7 +39,9 @@
  * tile and the q-th quarter (64 codes, or 80 trits) of the unit's K range. A lane's bytes
  * are its row-r0 bytes followed by its row-(r0+8) bytes (16 + 16 for Q2, 24 + 24 for Q3,
  * 16 + 16 for ternary), cut in 16-byte chunks; chunk c of lane l is stored at unit byte
- * (32*c + l)*16. Multi-byte words below are little-endian uint32.
+ * (32*c + (l ^ ((l >> 3) & 3)))*16: the swizzle puts the 8 rows r0 of one quarter in 8
+ * different shared-memory bank groups when one thread reads one row. Multi-byte words below
+ * are little-endian uint32.
  *   Q2: a row quarter is 4 words; code i (0..63) is in word i/16; with e = i%16 it sits
  *       at bits 16*(e%2) + 2*(e/2) .. +1 (even codes in the low 16 bits, odd in the high).
  *   Q3: a row quarter is two 12-byte groups (codes 0..31, 32..63), 3 words each. With

@@ -227,7 +227,7 @@ def sign_vector(sign_words: np.ndarray, K: int) -> np.ndarray:
 # l = 4*r0 + q (r0 = 0..7, q = 0..3) owns rows r0 and r0 + 8 of the tile and the
 # q-th quarter of the unit's K range; a lane's bytes (row r0's data, then row
 # r0+8's) are cut in 16-byte chunks, and chunk c of lane l sits at unit byte
-# (32 * c + l) * 16.
+# (32 * c + (l XOR ((l >> 3) & 3))) * 16.
 
 def _unit_geometry(fmt: int):
     if fmt == FMT_Q2:
@@ -247,7 +247,8 @@ def packed_bytes(fmt: int, N: int, K: int) -> int:
 
 
 def _lane_byte_to_unit_byte(lane: np.ndarray, lane_byte: np.ndarray) -> np.ndarray:
-    return (32 * (lane_byte // 16) + lane) * 16 + lane_byte % 16
+    position = lane ^ ((lane >> 3) & 3)
+    return (32 * (lane_byte // 16) + position) * 16 + lane_byte % 16
 
 
 def _frame(fmt: int, N: int, K: int):
