@@ -140,7 +140,7 @@ def module_bytes(wr, M, N, K, bits):
 # profiles/). None: no capture of this kernel version, so no traffic figure is claimed.
 # current kernel: M = 1 reads 1,207,574,272 and writes 7,993,088 bytes for 1,178,984,448
 # algorithmic; M = 8 reads 1,329,226,752 and writes 39,346,432 for 1,223,368,704
-_TRAFFIC_RATIO = {1: (1_207_889_152 + 7_606_016) / 1_178_984_448, 8: (1_344_171_264 + 38_778_624) / 1_223_368_704}
+_TRAFFIC_RATIO = {1: (1_208_125_184 + 7_661_568) / 1_178_984_448, 8: (1_328_882_944 + 39_116_544) / 1_223_368_704}
 
 
 def traffic_per_launch(M: int, layers: int, algo_bytes: int):
