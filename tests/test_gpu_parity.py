@@ -279,6 +279,56 @@ def test_ternary_gemm_prefill_m512(wr, N, K):
     check_close(y.cpu().numpy(), ref, B)
 
 
+def test_gemv_batched_more_problems_than_one_launch(wr):
+    """300 small mixed 2/3-bit problems in one call: the batch is split over two launches of at
+    most 256 problems, and every problem still matches the oracle."""
+    torch = torch_mod()
+    rng = np.random.default_rng(4242)
+    M = 2
+    problems, refs, keep = [], [], []
+    for i in range(300):
+        N = int(rng.integers(1, 80))
+        K = 256 * int(rng.integers(1, 4))
+        bits = int(rng.integers(2, 4))
+        codes, scales, packed, s_d = q_case(wr, bits, N, K, seed=20000 + i)
+        x = wr_synth.activations_bf16(30000 + i, M, K)
+        xd = dev(x)
+        y = torch.full((M, N), float("nan"), dtype=torch.float32, device="cuda")
+        keep += [xd, packed, s_d]
+        problems.append((xd, packed, s_d, y, N, K, bits))
+        refs.append(o.gemm_codes(x, codes, scales, bits))
+    nb = wr.wr_gemv_batched_workspace_bytes(M, problems)
+    ws = _zeros_ws(nb)
+    wr.wr_gemv_batched(M, problems, ws, nb)
+    torch.cuda.synchronize()
+    for (_, _, _, y, _, _, _), (ref, B) in zip(problems, refs):
+        check_close(y.cpu().numpy(), ref, B)
+    assert wr.wr_get_device_error() == 0
+
+
+def test_ternary_gemv_batched_more_problems_than_one_launch(wr):
+    """270 small ternary problems in one batched call (two launches of at most 256)."""
+    torch = torch_mod()
+    rng = np.random.default_rng(4343)
+    M = 3
+    problems, refs = [], []
+    for i in range(270):
+        N = int(rng.integers(1, 48))
+        K = 128 * int(rng.integers(1, 6))
+        codes, alpha, signs, packed, a_d, s_d = t_case(wr, N, K, seed=40000 + i)
+        x = wr_synth.activations_bf16(50000 + i, M, K)
+        y = torch.full((M, N), float("nan"), dtype=torch.float32, device="cuda")
+        problems.append((dev(x), packed, a_d, s_d, y, N, K))
+        refs.append(o.gemm_ternary(x, codes, alpha, signs))
+    nb = wr.wr_gemv_ternary_batched_workspace_bytes(M, problems)
+    ws = _zeros_ws(nb)
+    wr.wr_gemv_ternary_batched(M, problems, ws, nb)
+    torch.cuda.synchronize()
+    for (_, _, _, _, y, _, _), (ref, B) in zip(problems, refs):
+        check_close(y.cpu().numpy(), ref, B)
+    assert wr.wr_get_device_error() == 0
+
+
 # ---------------------------------------------------------------- batched ternary decode GEMV
 
 @pytest.mark.parametrize("M", [1, 6])
