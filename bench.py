@@ -44,7 +44,7 @@ def parse_args():
     p.add_argument("--no-extras", action="store_true", help="headline body only")
     p.add_argument("--cpu-seconds", type=float, default=12.0, help="oracle sample budget (0: no CPU baseline)")
     p.add_argument("--case", default=None,
-                   help="time one prefill GEMM alone and exit (for profiling): gemm:BITS:M:N:K or tgemm:M:N:K")
+                   help="time one case alone and exit (for profiling): gemm:BITS:M:N:K, tgemm:M:N:K, or the ternary batched body tbody:M:LAYERS")
     return p.parse_args()
 
 
@@ -416,6 +416,27 @@ def run_case(args, wr, torch, np, stream, bf16_peak):
         sg = torch.from_numpy(signs.view(np.int32)).cuda()
         nb = wr.wr_gemm_ternary_workspace_bytes(M, N, K)
         call = lambda x, y, ws: wr.wr_gemm_ternary(M, N, K, x, p, a, sg, y, ws, nb)  # noqa: E731
+    elif kind == "tbody":
+        # the ternary body: `layers` copies of one quantized layer's 7 linears, one batched call
+        M, layers = (int(v) for v in dims)
+        mods = []
+        for idx, (_, K, N, _) in enumerate(wr_synth.QWEN3_4B_LAYER):
+            signs = wr_synth.sign_bits(900 + idx, K)
+            codes, alpha = wr.wr_quantize_ternary(wr_synth.weights_fp32(800 + idx, N, K), signs)
+            mods.append((K, N, torch.from_numpy(wr.wr_pack(1, codes)).cuda(),
+                         torch.from_numpy(alpha.view(np.int16)).cuda(), torch.from_numpy(signs.view(np.int32)).cuda()))
+        body = [(K, N, p.roll(c * 4096), a, sg) for c in range(layers) for (K, N, p, a, sg) in mods]
+        xs = [torch.from_numpy(wr_synth.activations_bf16(3000 + j, M, K).view(np.int16)).cuda()
+              for j, (K, _, _, _, _) in enumerate(body)]
+        ys = [torch.empty(M, N, dtype=torch.float32, device="cuda") for (_, N, _, _, _) in body]
+        arr = wr._tproblems([(xs[j], p, a, sg, ys[j], N, K) for j, (K, N, p, a, sg) in enumerate(body)])
+        nb = wr.wr_gemv_ternary_batched_workspace_bytes(M, arr)
+        ws = torch.zeros(nb, dtype=torch.uint8, device="cuda")
+        ms = graph_time_ms(torch, lambda: wr.wr_gemv_ternary_batched(M, arr, ws, nb), args.steps, args.warmup,
+                           stream) / args.steps
+        b = sum(p.numel() + 2 * N + 4 * ((K + 31) // 32) + 2 * M * K + 4 * M * N for (K, N, p, _, _) in body)
+        print(json.dumps({"case": args.case, "us": ms * 1e3, "gbs": b / ms / 1e6, "bytes": b}))
+        return
     else:
         raise SystemExit(f"unknown --case {args.case!r}")
     x = torch.from_numpy(wr_synth.activations_bf16(M, M, K).view(np.int16)).cuda()
