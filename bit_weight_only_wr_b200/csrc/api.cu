@@ -58,9 +58,11 @@ constexpr int kPlanSMs = 148;   // split heuristics are sized for a 148-SM part 
 constexpr int kDecodeGrid = 3 * kPlanSMs;   // 2/3-bit decode: CTAs (block ranges) per launch, at most
 constexpr int kDecodeTokens = 8;   // decode kernel: 8 tokens x 4 activation limbs = 32 MMA columns
 
-// ---- decode kernel (M <= 8): work items (problem, 128-row group, block range) and workspace
-// [counters: one int per row group of every problem][split-K partials of problems with P > 1]
-// [prepared activation tiles: one per block of every problem].
+// ---- decode kernels (M <= 8) and workspace [counters: one int per row group of every problem]
+// [partials][prepared activation tiles: one per block of every problem]. 2/3-bit: the batch's
+// blocks are cut into one contiguous range per CTA, and the partials are two 128-row slots per
+// CTA for the row groups that two ranges share. Ternary: work items (problem, 128-row group,
+// block range), with split-K partials for problems cut into P > 1 pieces.
 struct DecodePlan {
   wr::DecArgs args;
   int total_blocks = 0;

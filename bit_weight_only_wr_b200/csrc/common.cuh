@@ -1,5 +1,5 @@
-// Device helpers shared by the libwr kernels: loads, the legacy warp MMA used by the decode
-// GEMV, and the register decoders that turn packed codes into exact bf16 grid values.
+// Device helpers shared by the libwr kernels: loads and the register decoders that turn
+// packed codes into exact bf16 grid values or integer codes.
 #pragma once
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -16,23 +16,6 @@ __device__ __forceinline__ uint4 ld_stream_v4(const void* p) {
                : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
                : "l"(p));
   return r;
-}
-
-// Read-only 16-byte load through L1 (activations: shared by every warp of an SM).
-__device__ __forceinline__ uint4 ld_ro_v4(const void* p) {
-  return __ldg(reinterpret_cast<const uint4*>(p));
-}
-
-// ---------------------------------------------------------------- warp MMA
-
-// D += A(16x16, row) * B(16x8, col) with bf16 inputs and fp32 accumulation.
-__device__ __forceinline__ void mma_bf16_16816(float d[4], uint32_t a0, uint32_t a1, uint32_t a2,
-                                               uint32_t a3, uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
-      "{%8,%9}, {%0,%1,%2,%3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
 // ---------------------------------------------------------------- exact code decoders
@@ -100,50 +83,6 @@ __device__ __forceinline__ void decode_trit_pairs(uint32_t e, uint32_t p[5]) {
   p[2] = bf16x2_fma((e & 0x00600060u) | kOneBf16x2, kB4, kBm5);
   p[3] = bf16x2_fma((t1 & 0x00060006u) | kOneBf16x2, kB64, kBm65);
   p[4] = bf16x2_fma((t1 & 0x00180018u) | kOneBf16x2, kB16, kBm17);
-}
-
-// Raw decoders for the tensor-memory path: every pair register is bf16 1.0 with the code
-// field OR-ed into its mantissa, i.e. the value 1 + c * 2^(p-7) for a field at bit p. The
-// power-of-two factor 2^(7-p) is applied to the matching activation instead, and the
-// constant part is removed once per block: with x'_k = x_k 2^(7-p_k),
-//   sum_k (1 + c_k 2^(p_k-7)) x'_k = sum_k x'_k + sum_k c_k x_k,
-// so sum_k g_k x_k = 2 (D - C) with C = sum_k x'_k + (L/2) sum_k x_k. Each product is exact
-// (8-bit significands); the offset costs a few bits of the fp32 accumulator only.
-// Slot positions: Q2 pairs j = 0..7 of a word sit at p = 1,3,5,1,3,5,1,3; Q3 pairs 5u+j of a
-// group at p = 1,4,1,4,1 and pair 15 at p = 1.
-__device__ __forceinline__ void decode_q2_word_raw(uint32_t w, uint32_t p[8]) {
-  const uint32_t t0 = w << 1, t1 = w >> 5, t2 = w >> 11;
-  p[0] = (t0 & 0x00060006u) | kOneBf16x2;
-  p[1] = (t0 & 0x00180018u) | kOneBf16x2;
-  p[2] = (t0 & 0x00600060u) | kOneBf16x2;
-  p[3] = (t1 & 0x00060006u) | kOneBf16x2;
-  p[4] = (t1 & 0x00180018u) | kOneBf16x2;
-  p[5] = (t1 & 0x00600060u) | kOneBf16x2;
-  p[6] = (t2 & 0x00060006u) | kOneBf16x2;
-  p[7] = (t2 & 0x00180018u) | kOneBf16x2;
-}
-
-__device__ __forceinline__ void decode_q3_group_raw(const uint32_t w[3], uint32_t p[16]) {
-#pragma unroll
-  for (int u = 0; u < 3; ++u) {
-    const uint32_t t0 = w[u] << 1, t1 = w[u] >> 5, t2 = w[u] >> 11;
-    p[5 * u + 0] = (t0 & 0x000E000Eu) | kOneBf16x2;
-    p[5 * u + 1] = (t0 & 0x00700070u) | kOneBf16x2;
-    p[5 * u + 2] = (t1 & 0x000E000Eu) | kOneBf16x2;
-    p[5 * u + 3] = (t1 & 0x00700070u) | kOneBf16x2;
-    p[5 * u + 4] = (t2 & 0x000E000Eu) | kOneBf16x2;
-  }
-  p[15] = ((w[0] >> 14) & 0x00020002u) | ((w[1] >> 13) & 0x00040004u) | ((w[2] >> 12) & 0x00080008u) | kOneBf16x2;
-}
-
-// log2 of the activation factor 2^(7-p) for position k (within a 256-block) of a Q2/Q3 row.
-__device__ __forceinline__ int q2_shift(int k) {
-  const int j = (k & 15) >> 1;
-  return 7 - (j % 3 == 0 ? 1 : (j % 3 == 1 ? 3 : 5));
-}
-__device__ __forceinline__ int q3_shift(int k) {
-  const int P = (k & 31) >> 1;
-  return 7 - ((P == 15 || (P % 5) % 2 == 0) ? 1 : 4);
 }
 
 // Position of lane l = 4 r0 + q's chunks inside a 32-chunk row of a packed unit (the swizzle

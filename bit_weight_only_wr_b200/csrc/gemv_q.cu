@@ -588,16 +588,6 @@ cudaError_t launch_xr(const DecArgs& a, int grid, cudaStream_t stream) {
 }
 }  // namespace
 
-int gemv_q_ctas_per_sm() { return kCtasPerSm; }
-
-int gemv_q_occupancy(int M) {
-  int n = 0;
-  const cudaError_t e = decode_xrows(M) == 8 ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, gemv_q_kernel<8>, kThreads, kSmem)
-                      : decode_xrows(M) == 16 ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, gemv_q_kernel<16>, kThreads, kSmem)
-                                              : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, gemv_q_kernel<32>, kThreads, kSmem);
-  return e == cudaSuccess ? n : -1;
-}
-
 cudaError_t launch_gemv_q(const DecArgs& a, int grid, cudaStream_t stream) {
   switch (decode_xrows(a.M)) {
     case 8: return launch_xr<8>(a, grid, stream);

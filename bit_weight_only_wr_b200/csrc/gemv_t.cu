@@ -16,7 +16,8 @@
 //              stores the bf16 values to A buffer g.
 //   warp 12    producer: per block one bulk copy for the 8 packed units of the row group and
 //              one for the activation tile.
-//   warp 13    allocates TMEM and issues the MMAs from one thread (10 per half block).
+//   warp 13    allocates TMEM and issues the MMAs (10 per half block; the whole warp walks the
+//              blocks and one elected lane issues).
 //   warps 8-11 epilogue: hi + lo columns summed, times alpha; then y, or a split-K combine
 //              through the workspace (the last of the P pieces to arrive adds them in order).
 // Every wait is bounded.

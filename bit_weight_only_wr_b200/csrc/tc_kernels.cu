@@ -61,10 +61,7 @@ struct Layout {
   static constexpr int kXOff = 0;
   static constexpr int kPOff = kXOff + kSX * kXStage;
   static constexpr int kBarOff = kPOff + kSP * kPStage;
-  // + barriers and alignment slack; the 16-column variant is padded so that at most two CTAs
-  // share an SM (each holds 256 TMEM columns)
-  static constexpr int kSmemRaw = kBarOff + 256 + 1024;
-  static constexpr int kSmem = (BN == 16 && kSmemRaw < 80 * 1024) ? 80 * 1024 : kSmemRaw;
+  static constexpr int kSmem = kBarOff + 256 + 1024;   // + barriers and alignment slack
   static constexpr int kACols = Fmt<FMT>::kChunkCols;
   static constexpr int kDCol = kSA * kACols;
   static constexpr int kTmemCols = (kDCol + 2 * BN) <= 256 ? 256 : 512;
@@ -643,12 +640,6 @@ __global__ void __launch_bounds__(64) selftest_wait_timeout_kernel(int* err_word
 cudaError_t launch_selftest_wait_timeout(int* err_word, cudaStream_t stream) {
   selftest_wait_timeout_kernel<<<1, 64, 0, stream>>>(err_word);
   return cudaGetLastError();
-}
-
-int tc_tmem_cols(int fmt, int bn) {
-  if (fmt == WR_FMT_TERNARY) return Layout<WR_FMT_TERNARY, 128>::kTmemCols;
-  if (bn == 16) return Layout<WR_FMT_Q2, 16>::kTmemCols;
-  return Layout<WR_FMT_Q2, 128>::kTmemCols;
 }
 
 cudaError_t launch_tc_kernel(int fmt, int bn, const TcArgs& a, const void* x_act, int64_t x_rows, int64_t x_k,

@@ -57,8 +57,6 @@ struct DecArgs {
 // 2/3-bit decode: the preparation pass writes the B tiles, then the GEMV kernel.
 cudaError_t launch_prep_x(const DecArgs& a, int total_blocks, cudaStream_t stream);
 cudaError_t launch_gemv_q(const DecArgs& a, int grid, cudaStream_t stream);
-int gemv_q_ctas_per_sm();   // CTAs of the 2/3-bit decode kernel that share an SM (by design)
-int gemv_q_occupancy(int M);  // CTAs per SM the runtime reports for it (needs the opt-in smem set)
 // Ternary decode (tiles written by launch_rotate_x).
 cudaError_t launch_gemv_t(const DecArgs& a, int grid, cudaStream_t stream);
 
@@ -73,7 +71,6 @@ __host__ __device__ inline int64_t xtile_bytes(bool ternary, int M) {
   return ternary ? (int64_t)5 * 2048 : (int64_t)2 * decode_xrows(M) * 128 + 256;
 }
 
-int tc_tmem_cols(int fmt, int bn);
 cudaError_t launch_tc_kernel(int fmt, int bn, const TcArgs& a, const void* x_act, int64_t x_rows, int64_t x_k,
                              int grid, cudaStream_t stream);
 cudaError_t launch_rotate_x(const uint16_t* x, const uint32_t* signs, uint8_t* xt, int M, int K, int64_t Kp,
