@@ -489,6 +489,24 @@ def run_extras(args, wr, torch, np, stream, dist, hbm_peak, bf16_peak):
     except Exception as e:  # noqa: BLE001
         out["unpack_bf16_gate"] = {"error": repr(e)}
 
+    # device quantizer + packer (fp32 W -> packed codes + fp16 scales) on the gate and up shapes
+    try:
+        res = {}
+        for name, bits in (("gate", 2), ("up", 3)):
+            N, K = 9728, 2560
+            W = torch.from_numpy(wr_synth.weights_fp32(7 + bits, N, K)).cuda()
+            pk = torch.empty(wr.wr_packed_bytes(bits, N, K), dtype=torch.uint8, device="cuda")
+            sc = torch.empty(N * (K // 256), dtype=torch.int16, device="cuda")
+
+            def step():
+                wr.wr_quantize_pack(bits, N, K, W, pk, sc)
+            ms = graph_time_ms(torch, step, 20, 3, stream) / 20
+            b = 4 * N * K + wr.wr_packed_bytes(bits, N, K) + 2 * N * (K // 256)
+            res[name] = {"us": ms * 1e3, "gbs": b / ms / 1e6, "bytes": b}
+        out["quantize_pack"] = res
+    except Exception as e:  # noqa: BLE001
+        out["quantize_pack"] = {"error": repr(e)}
+
     # prefill sweep
     try:
         res = {}

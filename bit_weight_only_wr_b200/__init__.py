@@ -20,6 +20,7 @@ __all__ = [
     "wr_get_device_error", "exported_symbols", "WrGemvProblem", "wr_gemv_batched_workspace_bytes",
     "wr_gemv_batched", "wr_gemv_noalloc", "WR_GEMV_NOALLOC_SCRATCH_BYTES", "WrGemvTernaryProblem",
     "wr_gemv_ternary_batched_workspace_bytes", "wr_gemv_ternary_batched", "wr_selftest_wait_timeout",
+    "wr_quantize_pack",
 ]
 
 WR_FMT_TERNARY, WR_FMT_Q2, WR_FMT_Q3 = 1, 2, 3
@@ -66,6 +67,7 @@ _SIGNATURES = {
     "wr_gemm_ternary": (_c_int, [_c_i64, _c_i64, _c_i64, _vp, _vp, _vp, _vp, _vp, _vp, _c_size, _vp]),
     "wr_get_device_error": (_c_int, [_vp]),
     "wr_selftest_wait_timeout": (_c_int, [_vp]),
+    "wr_quantize_pack": (_c_int, [_c_int, _c_i64, _c_i64, _vp, _vp, _vp, _vp]),
     "wr_gemv_noalloc": (_c_int, [_c_i64, _c_i64, _c_i64, _vp, _vp, _vp, _c_int, _c_int, _vp, _vp]),
     "wr_gemv_ternary_batched_workspace_bytes": (_c_size, [_c_i64, ctypes.c_int32, _TPROBLEMS]),
     "wr_gemv_ternary_batched": (_c_int, [_c_i64, ctypes.c_int32, _TPROBLEMS, _vp, _c_size, _vp]),
@@ -260,6 +262,13 @@ def wr_gemm_ternary(M: int, N: int, K: int, x, packed, alpha, sign_bits, y, work
 
 def wr_get_device_error(stream=None) -> int:
     return _lib.wr_get_device_error(_stream(stream))
+
+
+def wr_quantize_pack(bits: int, N: int, K: int, w, packed, scales, stream=None) -> None:
+    """Device quantizer + packer: fp32 W [N, K] (device) -> packed codes and fp16 block scales
+    (device), bit-identical with wr_quantize + wr_pack."""
+    _check("wr_quantize_pack", _lib.wr_quantize_pack(bits, N, K, _ptr(w), _ptr(packed), _ptr(scales),
+                                                     _stream(stream)))
 
 
 def wr_selftest_wait_timeout(stream=None) -> None:

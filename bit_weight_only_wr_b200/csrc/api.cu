@@ -509,6 +509,17 @@ wr_status wr_gemm_ternary(int64_t M, int64_t N, int64_t K, const uint16_t* x, co
   return run_t(M, N, K, x, packed, alpha, sign_bits, y, workspace, static_cast<cudaStream_t>(stream));
 }
 
+wr_status wr_quantize_pack(int bits, int64_t N, int64_t K, const float* w, void* packed, uint16_t* scales,
+                           void* stream) {
+  if (bits != 2 && bits != 3) return WR_ERR_UNSUPPORTED;
+  if (check_dims(1, N, K) != WR_OK || K % 256 != 0) return WR_ERR_INVALID_ARG;
+  if (!aligned16(w) || !aligned16(packed) || !aligned16(scales)) return WR_ERR_INVALID_ARG;
+  return wr::launch_quantize_pack(bits, w, (int)N, (int)K, static_cast<uint8_t*>(packed), scales,
+                                  static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? WR_OK
+             : WR_ERR_CUDA;
+}
+
 wr_status wr_selftest_wait_timeout(void* stream) {
   if (wr::launch_selftest_wait_timeout(device_error_word(), static_cast<cudaStream_t>(stream)) != cudaSuccess)
     return WR_ERR_CUDA;

@@ -81,6 +81,9 @@ cudaError_t launch_rotate_x(const uint16_t* x, const uint32_t* signs, uint8_t* x
 cudaError_t launch_rotate_planes(const uint16_t* x, const uint32_t* signs, uint8_t* planes, int M, int K, int64_t Kp,
                                  cudaStream_t stream);
 cudaError_t launch_rotate_x_batched(const DecArgs& a, int64_t total_items, cudaStream_t stream);
+// Device quantizer + packer for the 2/3-bit odd grid (quantize.cu).
+cudaError_t launch_quantize_pack(int bits, const float* w, int N, int K, uint8_t* packed, uint16_t* scales,
+                                 cudaStream_t stream);
 // Failure-path self-test: a bounded wait on a barrier that never completes (see wr.h).
 cudaError_t launch_selftest_wait_timeout(int* err_word, cudaStream_t stream);
 cudaError_t launch_unpack_bf16(int fmt, const uint8_t* packed, const uint16_t* scales, int N, int K, int units,

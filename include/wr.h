@@ -115,6 +115,15 @@ wr_status wr_unpack_codes(int fmt, int64_t N, int64_t K, const uint8_t* packed_h
 wr_status wr_quantize(int bits, int64_t N, int64_t K, const float* w_host, uint8_t* codes_host,
                       uint16_t* scales_host);
 
+/* Device quantizer + packer for the 2/3-bit odd grid: computes on the GPU exactly what
+ * wr_quantize followed by wr_pack computes on the host (bit-identical scales and packed bytes),
+ * in one pass over W. w [N,K] fp32 row-major, packed (wr_packed_bytes(bits, N, K) bytes) and
+ * scales fp16 bits [N, K/256] are device pointers (16-byte aligned); K % 256 == 0. The code of
+ * each weight is decided by exact comparisons of w with m*s for the even m between the levels,
+ * which is the decision of the fp64 quotient. Asynchronous on `stream`. */
+wr_status wr_quantize_pack(int bits, int64_t N, int64_t K, const float* w, void* packed, uint16_t* scales,
+                           void* stream);
+
 /* Host synthetic ternary quantizer: W' = W R^T (fp64, per 128-block fast Walsh-Hadamard
  * transform with the sign mask), Delta_n = 0.7 * mean_k |W'[n,k]|, t = sign(W') where
  * |W'| > Delta_n else 0, alpha_n = fp16(mean |W'| over t != 0) (0 if none); codes c = t+1.

@@ -329,6 +329,48 @@ def test_ternary_gemv_batched_more_problems_than_one_launch(wr):
     assert wr.wr_get_device_error() == 0
 
 
+# ---------------------------------------------------------------- device quantizer + packer
+
+def _edge_weights(N, K, seed):
+    """Seeded N(0, 0.02) weights with edge blocks planted: all zeros, ties on the even
+    boundaries (w = m s exactly), negative zeros, tiny blocks whose scale underflows to 0 in
+    fp16, and huge blocks whose scale overflows to inf."""
+    W = wr_synth.weights_fp32(seed, N, K).copy()
+    if N >= 6 and K >= 512:
+        W[0, 0:256] = 0.0
+        s = np.float32(0.125)                     # absmax 3 s -> s exact in fp16 for both grids
+        W[1, 0:256] = np.float32(0.0)
+        W[1, 0:8] = np.array([3, -3, 2, -2, 0, 1, -1, 2], np.float32) * s
+        W[1, 256:512] = np.float32(7.0) * s * np.sign(np.arange(256) - 127.5).astype(np.float32)
+        W[1, 256:262] = np.array([4, -4, 6, -6, 2, -2], np.float32) * s
+        W[2, 0:256] = np.float32(-0.0)
+        W[2, 0] = np.float32(1e-3)
+        W[3, 0:256] = np.float32(1e-9)             # absmax / L underflows fp16 -> s = 0
+        W[4, 0:256] = np.float32(3e5)              # absmax / L overflows fp16 -> s = inf
+        W[5, 256:512] *= np.float32(1e-4)
+    return W
+
+
+@pytest.mark.filterwarnings("ignore:overflow encountered in cast")   # the planted fp16 overflow
+@pytest.mark.parametrize("bits", [2, 3])
+@pytest.mark.parametrize("N,K", [(16, 256), (37, 768), (130, 2560), (6, 512)])
+def test_quantize_pack_bit_exact(wr, bits, N, K):
+    """wr_quantize_pack on the GPU gives the oracle's codes and scales, packed, byte for byte,
+    and the same bytes as the host quantizer and packer."""
+    torch = torch_mod()
+    W = _edge_weights(N, K, seed=60 + N + bits)
+    pk = torch.zeros(wr.wr_packed_bytes(bits, N, K), dtype=torch.uint8, device="cuda")
+    sc = torch.zeros(N * (K // 256), dtype=torch.int16, device="cuda")
+    wr.wr_quantize_pack(bits, N, K, dev(W), pk, sc)
+    torch.cuda.synchronize()
+    codes_o, s_o = o.quantize_odd_grid(W, bits)
+    assert np.array_equal(sc.cpu().numpy().view(np.uint16).reshape(N, K // 256), s_o.view(np.uint16))
+    assert np.array_equal(pk.cpu().numpy(), o.pack(bits, codes_o))
+    codes_h, s_h = wr.wr_quantize(bits, W)
+    assert np.array_equal(pk.cpu().numpy(), wr.wr_pack(bits, codes_h))
+    assert wr.wr_get_device_error() == 0
+
+
 # ---------------------------------------------------------------- batched ternary decode GEMV
 
 @pytest.mark.parametrize("M", [1, 6])
