@@ -20,6 +20,11 @@ What it defines (citations are to the source pages by title and section):
   block-128 random-sign Hadamard R: W x = (W R^T)(R x)
   ("How We Shrank...", "Trick 1: rotate the weights first"; the Qwen3-4B
   ternarization article for W1.58A16).
+* A 2-bit trellis-coded format ("How We Shrank...", "Trick 3: trellis coding"): the
+  encoder carries a state from one weight to the next, the state picks a coset of the
+  levels, the written bits pick a value inside it and set the next state, and a Viterbi
+  search finds the cheapest path. The pages give the 2-state, 1-bit toy in full; the
+  format here is its 2-bit form: 8 odd levels, state = low bit of the previous symbol.
 * The contraction y[m, n] = sum_k W[n, k] x[m, k] in fp64, and the bound
   B[m, n] = sum_k |W[n, k] x[m, k]| used for the per-element tolerance.
 * The packed byte layout (defined in ``include/wr.h``), re-implemented here from
@@ -40,6 +45,7 @@ TILE_ROWS = 16
 FMT_TERNARY = 1
 FMT_Q2 = 2
 FMT_Q3 = 3
+FMT_T2 = 4   # 2-bit trellis-coded: 2-bit symbols in the Q2 layout, 8 odd levels
 
 
 # --------------------------------------------------------------------------------------
@@ -106,6 +112,115 @@ def quantize_odd_grid(W: np.ndarray, bits: int):
     g = np.clip(g, -L, L).astype(np.int64)
     codes = ((g + L) // 2).astype(np.uint8).reshape(N, K)
     return codes, s16
+
+
+# --------------------------------------------------------------------------------------
+# Trellis coding ("How We Shrank...", "Trick 3: trellis coding")
+# --------------------------------------------------------------------------------------
+#
+# The toy on that page: four levels in two cosets, state 0 may use {-1.5, 0.5} and state 1
+# {-0.5, 1.5}; bit 0 picks the lower value, bit 1 the higher, and the bit written becomes the
+# next state. In general form, with `values` the 2^(k+1) levels in ascending order and k bits
+# written per weight: state s may use values[2u + s] for u in [0, 2^k), and the next state is
+# the low bit of u. At k = 1 this is the toy exactly. The 2-bit format below is k = 2 over the
+# 8 odd levels {-7, ..., 7} * s, with the state reset to 0 at the start of every 256-block so
+# that blocks decode on their own. (Reading: the pages also name an 8-state set-partitioned
+# trellis over 4-weight symbols but give no tables for it; the 2-state scalar trellis is the
+# one they specify completely.)
+
+def trellis_level_index(symbols: np.ndarray, state0: int = 0) -> np.ndarray:
+    """Level index 2 u_i + state_i of each step (last axis), state_{i+1} = u_i & 1."""
+    u = np.asarray(symbols, dtype=np.int64)
+    state = np.empty_like(u)
+    state[..., 0] = state0
+    state[..., 1:] = u[..., :-1] & 1
+    return 2 * u + state
+
+
+def trellis_greedy(targets, values, k: int, state0: int = 0):
+    """Greedy encoding: at each step the nearest value the current state allows (a tie takes
+    the lower symbol). Returns (symbols, squared error)."""
+    values = np.asarray(values, dtype=np.float64)
+    state, out, err = state0, [], 0.0
+    for t in np.asarray(targets, dtype=np.float64):
+        cand = [(float(t - values[2 * u + state]) ** 2, u) for u in range(1 << k)]
+        e, u = min(cand)
+        out.append(u)
+        err += e
+        state = u & 1
+    return np.array(out, dtype=np.int64), err
+
+
+def trellis_viterbi(targets: np.ndarray, values: np.ndarray, k: int, state0: int = 0):
+    """Minimum squared-error path (the Viterbi algorithm: for every state, the cheapest path
+    ending there). targets [..., n] (several independent sequences along the leading axes),
+    values [..., 2^(k+1)] ascending (broadcast against the leading axes). Ties go to the
+    lower (state, symbol) pair and, at the end, the lower final state.
+    Returns (symbols int64 [..., n], cost float64 [...])."""
+    t = np.asarray(targets, dtype=np.float64)
+    v = np.asarray(values, dtype=np.float64)
+    lead, n = t.shape[:-1], t.shape[-1]
+    v = np.broadcast_to(v, lead + v.shape[-1:])
+    U = 1 << k
+    inf = np.inf
+    cost = np.full(lead + (2,), inf)
+    cost[..., state0] = 0.0
+    back_s = np.zeros(lead + (n, 2), dtype=np.int64)
+    back_u = np.zeros(lead + (n, 2), dtype=np.int64)
+    for i in range(n):
+        ti = t[..., i]
+        new = np.full(lead + (2,), inf)
+        bs = np.zeros(lead + (2,), dtype=np.int64)
+        bu = np.zeros(lead + (2,), dtype=np.int64)
+        for s in range(2):
+            for u in range(U):
+                d = ti - v[..., 2 * u + s]
+                c = cost[..., s] + d * d
+                nxt = u & 1
+                better = c < new[..., nxt]
+                new[..., nxt] = np.where(better, c, new[..., nxt])
+                bs[..., nxt] = np.where(better, s, bs[..., nxt])
+                bu[..., nxt] = np.where(better, u, bu[..., nxt])
+        cost = new
+        back_s[..., i, :] = bs
+        back_u[..., i, :] = bu
+    final = np.argmin(cost, axis=-1)
+    best = np.take_along_axis(cost, final[..., None], axis=-1)[..., 0]
+    sym = np.zeros(lead + (n,), dtype=np.int64)
+    st = final
+    for i in range(n - 1, -1, -1):
+        sym[..., i] = np.take_along_axis(back_u[..., i, :], st[..., None], axis=-1)[..., 0]
+        st = np.take_along_axis(back_s[..., i, :], st[..., None], axis=-1)[..., 0]
+    return sym, best
+
+
+def quantize_trellis2(W: np.ndarray):
+    """The 2-bit trellis-coded format: per 256-block, s = fp16(absmax / 7) (fp64 division,
+    one rounding), levels s * {-7, -5, ..., 7}, symbols u in [0, 4) by the Viterbi search
+    (state 0 at the block start), so the level index is c3 = 2 u + state and the weight
+    s * (2 c3 - 7). Returns (symbols uint8 [N, K], scales float16 [N, K/256])."""
+    W = np.asarray(W, dtype=np.float32)
+    N, K = W.shape
+    assert K % BLOCK == 0
+    Wb = W.astype(np.float64).reshape(N, K // BLOCK, BLOCK)
+    s16 = fp16_round(np.abs(Wb).max(axis=2) / 7.0)
+    levels = np.arange(-7, 8, 2, dtype=np.float64)
+    vals = s16.astype(np.float64)[:, :, None] * levels
+    sym, _ = trellis_viterbi(Wb, vals, 2)
+    return sym.reshape(N, K).astype(np.uint8), s16
+
+
+def dequant_trellis2(symbols: np.ndarray, scales: np.ndarray) -> np.ndarray:
+    """W = s * (2 c3 - 7) with c3 = 2 u + state, the state restarting at every 256-block."""
+    u = np.asarray(symbols, dtype=np.int64)
+    N, K = u.shape
+    c3 = trellis_level_index(u.reshape(N, K // BLOCK, BLOCK)).reshape(N, K)
+    s = np.repeat(np.asarray(scales, dtype=np.float64), BLOCK, axis=1)
+    return s * (2 * c3 - 7).astype(np.float64)
+
+
+def gemm_trellis2(x_bits, symbols, scales):
+    return gemm(x_bits, dequant_trellis2(symbols, scales))
 
 
 def rotate(v: np.ndarray, sign_words: np.ndarray) -> np.ndarray:

@@ -331,3 +331,74 @@ def test_pack_is_a_bijection_on_bytes():
         flat = (byte.astype(np.int64) * 8 + bit).ravel()
         assert np.unique(flat).size == flat.size == N * K * b
         assert flat.max() < o.packed_bytes(fmt, N, K) * 8
+
+
+# ---------------------------------------------------------------- trellis coding
+
+def test_trellis_toy_matches_the_page(golden_dir):
+    """The page's 1-bit toy: greedy and best-path picks, states and squared errors, and the
+    plain 1-bit rounding it is compared with."""
+    g = json.load(open(os.path.join(golden_dir, "trellis_toy.json")))
+    vals, t, k = np.array(g["values"]), np.array(g["targets"]), g["bits"]
+    u_g, e_g = o.trellis_greedy(t, vals, k)
+    idx_g = o.trellis_level_index(u_g)
+    assert np.allclose(vals[idx_g], g["greedy"]["picks"])
+    assert list(idx_g & 1) == g["greedy"]["states"]           # the level's coset is the state
+    assert abs(e_g - g["greedy"]["squared_error"]) < 1e-9
+    u_v, e_v = o.trellis_viterbi(t, vals, k)
+    idx_v = o.trellis_level_index(u_v)
+    assert np.allclose(vals[idx_v], g["best_path"]["picks"])
+    assert list(idx_v & 1) == g["best_path"]["states"]
+    assert abs(float(e_v) - g["best_path"]["squared_error"]) < 1e-9
+    lv = np.array(g["plain_one_bit_rounding"]["levels"])
+    plain = ((t[:, None] - lv[None, :]) ** 2).min(axis=1).sum()
+    assert abs(plain - g["plain_one_bit_rounding"]["squared_error"]) < 1e-9
+
+
+@pytest.mark.parametrize("k", [1, 2])
+def test_trellis_viterbi_is_the_brute_force_optimum(k):
+    """On short random sequences the Viterbi path costs exactly the minimum over all U^n
+    symbol sequences, and its symbols reach that cost."""
+    import itertools
+    rng = np.random.default_rng(11 + k)
+    U = 1 << k
+    for _ in range(40):
+        n = int(rng.integers(1, 6))
+        vals = np.sort(rng.normal(size=2 * U))
+        t = rng.normal(size=n)
+        best = min(
+            sum((t[i] - vals[idx]) ** 2 for i, idx in enumerate(o.trellis_level_index(np.array(seq))))
+            for seq in itertools.product(range(U), repeat=n))
+        u, c = o.trellis_viterbi(t, vals, k)
+        idx = o.trellis_level_index(u)
+        assert abs(float(c) - best) < 1e-12
+        assert abs(float(((t - vals[idx]) ** 2).sum()) - best) < 1e-12
+        _, cg = o.trellis_greedy(t, vals, k)
+        assert float(c) <= cg + 1e-12
+
+
+def test_trellis2_quantizer_invariants():
+    """The 2-bit trellis format: symbols in [0, 4), the level index 2u + state restarts at
+    every block, the weights lie on s * {-7..7 odd}, its squared error is never above the
+    greedy encoding of the same block, and over the matrix it is below that of the 4-level
+    nearest-point grid, which stores the same 2 bits per weight."""
+    W = wr_synth.weights_fp32(5, 8, 512)
+    u, s = o.quantize_trellis2(W)
+    assert u.dtype == np.uint8 and u.max() <= 3
+    Wd = o.dequant_trellis2(u, s)
+    sb = np.repeat(s.astype(np.float64), 256, axis=1)
+    lv = Wd / np.where(sb > 0, sb, 1.0)
+    assert np.all(np.isin(np.round(lv), np.arange(-7, 8, 2))) and np.allclose(lv, np.round(lv))
+    # block restart: the first weight of every block takes an even level index (state 0)
+    c3 = (np.round(lv).astype(int) + 7) // 2
+    assert np.all(c3[:, ::256] % 2 == 0)
+    err_t = ((W.astype(np.float64) - Wd) ** 2).reshape(8, 2, 256).sum(axis=2)
+    levels = np.arange(-7, 8, 2, dtype=np.float64)
+    for n in range(8):
+        for b in range(2):
+            vals = float(s[n, b]) * levels
+            _, eg = o.trellis_greedy(W[n, 256 * b:256 * (b + 1)].astype(np.float64), vals, 2)
+            assert err_t[n, b] <= eg + 1e-12
+    c2, s2 = o.quantize_odd_grid(W, 2)
+    err_q2 = ((W.astype(np.float64) - o.dequant(c2, s2, 2)) ** 2).sum()
+    assert err_t.sum() < err_q2
