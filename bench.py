@@ -489,6 +489,33 @@ def run_extras(args, wr, torch, np, stream, dist, hbm_peak, bf16_peak):
     except Exception as e:  # noqa: BLE001
         out["unpack_bf16_gate"] = {"error": repr(e)}
 
+    # the 2-bit trellis-coded format: one layer's 7 linears encoded once (Viterbi, host), the
+    # 36-layer body made of 36 distinct byte copies, one batched decode GEMV call per token
+    try:
+        res = {}
+        tmods = []
+        for idx, (name, K, N, _) in enumerate(wr_synth.QWEN3_4B_LAYER):
+            sym, sc = wr.wr_quantize_trellis(wr_synth.weights_fp32(600 + idx, N, K))
+            tmods.append((K, N, torch.from_numpy(wr.wr_pack(wr.WR_FMT_T2, sym)).cuda(),
+                          torch.from_numpy(sc.view(np.int16)).cuda()))
+        body = [(K, N, p.roll(c * 4096), sc) for c in range(36) for (K, N, p, sc) in tmods]
+        for M in (1, 8):
+            xs = [torch.from_numpy(wr_synth.activations_bf16(5000 + j, M, K).view(np.int16)).cuda()
+                  for j, (K, _, _, _) in enumerate(body)]
+            ys = [torch.empty(M, N, dtype=torch.float32, device="cuda") for (_, N, _, _) in body]
+            arr = wr._problems([(xs[j], p, sc, ys[j], N, K, wr.WR_FMT_T2) for j, (K, N, p, sc) in enumerate(body)])
+            nb = wr.wr_gemv_batched_workspace_bytes(M, arr)
+            ws = torch.zeros(nb, dtype=torch.uint8, device="cuda")
+
+            def tstep():
+                wr.wr_gemv_batched(M, arr, ws, nb)
+            ms = graph_time_ms(torch, tstep, 10, 3, stream) / 10
+            b = sum(p.numel() + 2 * N * (K // 256) + 2 * M * K + 4 * M * N for (K, N, p, _) in body)
+            res[f"body_M{M}"] = {"ms": ms, "bytes": b, "gbs": b / ms / 1e6, "tokens_per_s": M * 1e3 / ms}
+        out["trellis2"] = res
+    except Exception as e:  # noqa: BLE001
+        out["trellis2"] = {"error": repr(e)}
+
     # device quantizer + packer (fp32 W -> packed codes + fp16 scales) on the gate and up shapes
     try:
         res = {}

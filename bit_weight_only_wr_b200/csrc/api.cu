@@ -324,7 +324,7 @@ const char* wr_status_string(wr_status st) {
 
 wr_status wr_unpack_bf16(int fmt, int64_t N, int64_t K, const void* packed, const uint16_t* scales,
                          int group, uint16_t* w_bf16, void* stream) {
-  if (fmt != WR_FMT_Q2 && fmt != WR_FMT_Q3 && fmt != WR_FMT_TERNARY) return WR_ERR_UNSUPPORTED;
+  if (fmt != WR_FMT_Q2 && fmt != WR_FMT_Q3 && fmt != WR_FMT_TERNARY && fmt != WR_FMT_T2) return WR_ERR_UNSUPPORTED;
   if (check_dims(1, N, K) != WR_OK) return WR_ERR_INVALID_ARG;
   if (fmt != WR_FMT_TERNARY && group != 256) return WR_ERR_UNSUPPORTED;
   int64_t ub = 0, units = 0, tiles = 0;
@@ -336,7 +336,7 @@ wr_status wr_unpack_bf16(int fmt, int64_t N, int64_t K, const void* packed, cons
 }
 
 size_t wr_gemv_workspace_bytes(int64_t M, int64_t N, int64_t K, int bits) {
-  if (bits != 2 && bits != 3) return 0;
+  if (bits != 2 && bits != 3 && bits != WR_FMT_T2) return 0;
   if (M < 1 || M > 8 || check_dims(M, N, K) != WR_OK || K % 256 != 0) return 0;
   return q_workspace(bits, M, N, K);
 }
@@ -344,7 +344,7 @@ size_t wr_gemv_workspace_bytes(int64_t M, int64_t N, int64_t K, int bits) {
 wr_status wr_gemv(int64_t M, int64_t N, int64_t K, const uint16_t* x, const void* packed,
                   const uint16_t* scales, int bits, int group, float* y, void* workspace,
                   size_t workspace_bytes, void* stream) {
-  if (bits != 2 && bits != 3) return WR_ERR_UNSUPPORTED;
+  if (bits != 2 && bits != 3 && bits != WR_FMT_T2) return WR_ERR_UNSUPPORTED;
   if (group != 256) return WR_ERR_UNSUPPORTED;
   if (M < 1 || M > 8 || check_dims(M, N, K) != WR_OK || K % 256 != 0) return WR_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(packed) || !aligned16(scales) || !aligned16(y) || !aligned16(workspace))
@@ -355,7 +355,7 @@ wr_status wr_gemv(int64_t M, int64_t N, int64_t K, const uint16_t* x, const void
 
 wr_status wr_gemv_noalloc(int64_t M, int64_t N, int64_t K, const uint16_t* x, const void* packed,
                           const uint16_t* scales, int bits, int group, float* y, void* stream) {
-  if (bits != 2 && bits != 3) return WR_ERR_UNSUPPORTED;
+  if (bits != 2 && bits != 3 && bits != WR_FMT_T2) return WR_ERR_UNSUPPORTED;
   if (group != 256) return WR_ERR_UNSUPPORTED;
   if (M < 1 || M > 8 || check_dims(M, N, K) != WR_OK || K % 256 != 0) return WR_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(packed) || !aligned16(scales) || !aligned16(y)) return WR_ERR_INVALID_ARG;
@@ -375,7 +375,7 @@ wr_status wr_gemv_noalloc(int64_t M, int64_t N, int64_t K, const uint16_t* x, co
 static bool batch_ok(int64_t M, int32_t count, const wr_gemv_problem* pr) {
   if (M < 1 || M > 8 || count < 1 || !pr) return false;
   for (int i = 0; i < count; ++i) {
-    if (pr[i].bits != 2 && pr[i].bits != 3) return false;
+    if (pr[i].bits != 2 && pr[i].bits != 3 && pr[i].bits != WR_FMT_T2) return false;
     if (pr[i].reserved != 0 || check_dims(M, pr[i].N, pr[i].K) != WR_OK || pr[i].K % 256 != 0) return false;
     if (!aligned16(pr[i].x) || !aligned16(pr[i].packed) || !aligned16(pr[i].scales) || !aligned16(pr[i].y))
       return false;

@@ -127,6 +127,23 @@ __host__ __device__ __forceinline__ void decode_q3_group_i8(const uint32_t w[3],
          (w[2] & 0x80008000u);
 }
 
+// 2-bit trellis-coded word (the Q2 word layout holding symbols u, code e at bits
+// 16*(e&1) + 2*(e>>1)): the level index of code e is c3 = 2 u_e + p_e, with p_e the low bit of
+// the previous symbol (of code e - 1; of the previous word's code 15 for e = 0, given in
+// `carry`, which returns this word's code-15 low bit). P holds p_e at each field's low bit:
+// odd codes take the low bit of the even code in the same slot, even codes that of the odd
+// code one slot down. Register s holds codes [2s, 2s+8, 2s+1, 2s+9] as (2 u + p) * 2^e,
+// e = 0, 1, 3, 5 for s = 0..3 (u stays in place; p is masked in one bit below it).
+__host__ __device__ __forceinline__ void decode_t2_word_i8(uint32_t w, uint32_t& carry, uint32_t r[4]) {
+  const uint32_t P = ((w << 16) & 0x55550000u) | ((w >> 14) & 0x00005554u) | carry;
+  carry = (w >> 30) & 1u;
+  const uint32_t P1 = P >> 1;
+  r[0] = ((w & 0x03030303u) << 1) | (P & 0x01010101u);
+  r[1] = (w & 0x0C0C0C0Cu) | (P1 & 0x02020202u);
+  r[2] = (w & 0x30303030u) | (P1 & 0x08080808u);
+  r[3] = (w & 0xC0C0C0C0u) | (P1 & 0x20202020u);
+}
+
 // Code index (within a 256-code block) held at logical K position kl of the decoded block, and
 // the exponent e of its byte, for the register orders above. Rows of a block are 4 quarters of
 // 64 codes; a quarter is 16 registers (Q2: 4 words x 4; Q3: 2 groups x 8).
@@ -136,6 +153,11 @@ __host__ __device__ inline int q2_code_at(int kl) {
   return 64 * q + 16 * w + p;
 }
 __host__ __device__ inline int q2_exp_at(int kl) { return 2 * ((kl >> 2) & 3); }
+// The trellis format uses the Q2 K order; its bytes hold (2u + p) * 2^e, e = 0, 1, 3, 5.
+__host__ __device__ inline int t2_exp_at(int kl) {
+  const int sp = (kl >> 2) & 3;
+  return sp == 0 ? 0 : 2 * sp - 1;
+}
 __host__ __device__ inline int q3_code_at(int kl) {
   const int q = kl >> 6, g = (kl >> 5) & 1, reg = (kl >> 2) & 7, byte = kl & 3;
   int c;

@@ -20,6 +20,11 @@
 // (more than 2^24 under the block maximum) round to that step: at most 2^-25 max |x| per
 // element, and the fp32 combination adds a few units of 2^-24 of sum |x| per block.
 //
+// The 2-bit trellis-coded format (WR_FMT_T2) runs through the same kernel: its symbols are
+// stored like Q2 codes, and the decode warps turn each into the level index 2 u + p (p = the
+// low bit of the previous symbol in the row, carried word by word) before the MMA, so the
+// MMA sees 8 levels (L = 7), as for Q3.
+//
 // A CTA is one small pipeline; three run on every SM so that their latency chains overlap
 // (warp roles, 320 threads):
 //   warps 0-3  decode, thread = weight row (TMEM lane 32 w + lane): per block, the row's 256
@@ -176,6 +181,20 @@ __device__ __forceinline__ void q2_half_i8(const uint8_t* unit, int r0, int half
   }
 }
 
+// The trellis-coded format: the Q2 words, with the low bit of the previous symbol carried
+// through the row in code order (quarter by quarter, word by word).
+__device__ __forceinline__ void t2_half_i8(const uint8_t* unit, int r0, int half, int h, uint32_t v[32],
+                                           uint32_t& carry) {
+#pragma unroll
+  for (int qq = 0; qq < 2; ++qq) {
+    const uint4 c = *reinterpret_cast<const uint4*>(unit + (32 * half + lane_pos(r0, 2 * h + qq)) * 16);
+    decode_t2_word_i8(c.x, carry, v + 16 * qq + 0);
+    decode_t2_word_i8(c.y, carry, v + 16 * qq + 4);
+    decode_t2_word_i8(c.z, carry, v + 16 * qq + 8);
+    decode_t2_word_i8(c.w, carry, v + 16 * qq + 12);
+  }
+}
+
 __device__ __forceinline__ void q3_half_i8(const uint8_t* unit, int r0, int half, int h, uint32_t v[32]) {
 #pragma unroll
   for (int qq = 0; qq < 2; ++qq) {
@@ -279,7 +298,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_q_kernel(const __gr
         // weight stage np % kSP: free once the decode warps have read block np - kSP
         const int sp = np % kSP;
         if (!(ok = mbar_wait_bg(&bars->pk_empty[sp], ((np / kSP) & 1) ^ 1, abort_flag, a.err, 101))) break;
-        const int ub = cp.bits == 2 ? 1024 : 1536;
+        const int ub = cp.bits == 3 ? 1536 : 1024;
         const int ntile = min(8, (cp.N + 15) / 16 - cp.rg * 8);
         if (elect_one()) {
           mbar_arrive_expect_tx(&bars->pk_full[sp], ntile * ub);
@@ -346,16 +365,19 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_q_kernel(const __gr
     for (uint32_t gd = 0; dc.left > 0; ++gd) {
       const int sp = gd % kSP;
       if (!mbar_wait(&bars->pk_full[sp], (gd / kSP) & 1, abort_flag, a.err, 301)) break;
-      const uint8_t* unit = ps + sp * kPStage + tile * (dc.bits == 2 ? 1024 : 1536);
+      const uint8_t* unit = ps + sp * kPStage + tile * (dc.bits == 3 ? 1536 : 1024);
       uint32_t v[32];
+      uint32_t carry = 0;   // trellis state at the block start
       if (dc.bits == 2) q2_half_i8(unit, r0, half, 0, v);
-      else q3_half_i8(unit, r0, half, 0, v);
+      else if (dc.bits == 3) q3_half_i8(unit, r0, half, 0, v);
+      else t2_half_i8(unit, r0, half, 0, v, carry);
       // the A buffer is free once block gd - 1's MMAs are done
       if (gd > 0 && !mbar_wait(&bars->mma_done[(gd - 1) % kSX], ((gd - 1) / kSX) & 1, abort_flag, a.err, 302)) break;
       fence_after_sync();
       tmem_st32(lane_base + kACol, v);
       if (dc.bits == 2) q2_half_i8(unit, r0, half, 1, v);
-      else q3_half_i8(unit, r0, half, 1, v);
+      else if (dc.bits == 3) q3_half_i8(unit, r0, half, 1, v);
+      else t2_half_i8(unit, r0, half, 1, v, carry);
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->pk_empty[sp]);
       tmem_st32(lane_base + kACol + 32, v);
@@ -512,10 +534,10 @@ __global__ void __launch_bounds__(256) prep_x_kernel(const __grid_constant__ Dec
 #pragma unroll
   for (int e = 0; e < 8; ++e) {
     const int kl = 8 * lane + e;
-    pe[e] = pr.bits == 2 ? q2_exp_at(kl) : q3_exp_at(kl);
+    pe[e] = pr.bits == 2 ? q2_exp_at(kl) : (pr.bits == 3 ? q3_exp_at(kl) : t2_exp_at(kl));
     xv[e] = 0.f;
     if (m < M) {
-      const int k = pr.bits == 2 ? q2_code_at(kl) : q3_code_at(kl);
+      const int k = pr.bits == 3 ? q3_code_at(kl) : q2_code_at(kl);
       xv[e] = __bfloat162float(__ushort_as_bfloat16(__ldg(pr.x + (int64_t)m * pr.K + (int64_t)b * 256 + k)));
       amax = fmaxf(amax, fabsf(xv[e]));
     }

@@ -8,6 +8,7 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <limits>
 #include <vector>
 
 #include "wr.h"
@@ -17,7 +18,11 @@ namespace {
 
 constexpr int kTileRows = 16;
 
-inline bool fmt_ok(int fmt) { return fmt == WR_FMT_Q2 || fmt == WR_FMT_Q3 || fmt == WR_FMT_TERNARY; }
+inline bool fmt_ok(int fmt) {
+  return fmt == WR_FMT_Q2 || fmt == WR_FMT_Q3 || fmt == WR_FMT_TERNARY || fmt == WR_FMT_T2;
+}
+// 2-bit symbol formats share the Q2 words: Q2 codes and the trellis format's symbols.
+inline bool two_bit(int fmt) { return fmt == WR_FMT_Q2 || fmt == WR_FMT_T2; }
 
 struct Geometry {
   int64_t unit_k;      // codes per unit along K
@@ -34,7 +39,7 @@ bool geometry(int fmt, int64_t N, int64_t K, Geometry* g) {
   } else {
     if (K % 256 != 0) return false;
     g->unit_k = 256;
-    g->unit_bytes = fmt == WR_FMT_Q2 ? 1024 : 1536;
+    g->unit_bytes = fmt == WR_FMT_Q3 ? 1536 : 1024;
   }
   g->tiles = (N + kTileRows - 1) / kTileRows;
   g->units = (K + g->unit_k - 1) / g->unit_k;
@@ -156,7 +161,7 @@ size_t wr_packed_bytes(int fmt, int64_t N, int64_t K) {
 wr_status wr_pack(int fmt, int64_t N, int64_t K, const uint8_t* codes, uint8_t* packed) {
   Geometry g;
   if (!geometry(fmt, N, K, &g) || !codes || !packed) return WR_ERR_INVALID_ARG;
-  const uint8_t cmax = fmt == WR_FMT_Q2 ? 3 : fmt == WR_FMT_Q3 ? 7 : 2;
+  const uint8_t cmax = two_bit(fmt) ? 3 : fmt == WR_FMT_Q3 ? 7 : 2;
   bool bad = false;
 #pragma omp parallel for reduction(|| : bad)
   for (int64_t i = 0; i < N * K; ++i) bad = bad || codes[i] > cmax;
@@ -184,7 +189,7 @@ wr_status wr_pack(int fmt, int64_t N, int64_t K, const uint8_t* codes, uint8_t* 
           } else {
             uint8_t c64[64];
             for (int i = 0; i < 64; ++i) c64[i] = n < N ? codes[n * K + u * 256 + 64 * q + i] : 0;
-            if (fmt == WR_FMT_Q2) {
+            if (two_bit(fmt)) {
               for (int w = 0; w < 4; ++w) put_word(unit, lane, 16 * half + 4 * w, q2_word(c64 + 16 * w));
             } else {
               for (int grp = 0; grp < 2; ++grp) {
@@ -224,7 +229,7 @@ wr_status wr_unpack_codes(int fmt, int64_t N, int64_t K, const uint8_t* packed, 
             }
           } else {
             uint8_t c64[64];
-            if (fmt == WR_FMT_Q2) {
+            if (two_bit(fmt)) {
               for (int w = 0; w < 4; ++w) q2_unword(get_word(unit, lane, 16 * half + 4 * w), c64 + 16 * w);
             } else {
               for (int grp = 0; grp < 2; ++grp) {
@@ -266,6 +271,60 @@ wr_status wr_quantize(int bits, int64_t N, int64_t K, const float* w, uint8_t* c
           g = (int)gd;
         }
         codes[n * K + b * 256 + i] = (uint8_t)((g + L) / 2);
+      }
+    }
+  }
+  return WR_OK;
+}
+
+// The 2-bit trellis-coded format: per 256-block, s = fp16(absmax / 7), levels s * {-7..7 odd};
+// state s may use level index 2u + s (u in [0, 4)) and the next state is u & 1; the Viterbi
+// search (state 0 at the block start) keeps, for each state, the cheapest path ending there.
+// Ties go to the lower (state, symbol) pair and, at the end, the lower final state.
+wr_status wr_quantize_trellis(int64_t N, int64_t K, const float* w, uint8_t* codes, uint16_t* scales) {
+  if (N <= 0 || K <= 0 || K % 256 != 0 || !w || !codes || !scales) return WR_ERR_INVALID_ARG;
+  const int64_t nb = K / 256;
+#pragma omp parallel for schedule(static)
+  for (int64_t n = 0; n < N; ++n) {
+    std::vector<uint8_t> bs(256 * 2), bu(256 * 2);
+    for (int64_t b = 0; b < nb; ++b) {
+      const float* wb = w + n * K + b * 256;
+      double amax = 0.0;
+      for (int i = 0; i < 256; ++i) amax = std::fmax(amax, std::fabs((double)wb[i]));
+      const uint16_t sh = double_to_half(amax / 7.0);
+      scales[n * nb + b] = sh;
+      const double s = half_to_double(sh);
+      double val[8];
+      for (int l = 0; l < 8; ++l) val[l] = s * (double)(2 * l - 7);
+      const double inf = std::numeric_limits<double>::infinity();
+      double cost[2] = {0.0, inf};
+      for (int i = 0; i < 256; ++i) {
+        const double t = (double)wb[i];
+        double nc[2] = {inf, inf};
+        uint8_t ns[2] = {0, 0}, nu[2] = {0, 0};
+        for (int st = 0; st < 2; ++st) {
+          for (int u = 0; u < 4; ++u) {
+            const double d = t - val[2 * u + st];
+            const double c = cost[st] + d * d;
+            const int nx = u & 1;
+            if (c < nc[nx]) {
+              nc[nx] = c;
+              ns[nx] = (uint8_t)st;
+              nu[nx] = (uint8_t)u;
+            }
+          }
+        }
+        cost[0] = nc[0];
+        cost[1] = nc[1];
+        bs[2 * i] = ns[0];
+        bs[2 * i + 1] = ns[1];
+        bu[2 * i] = nu[0];
+        bu[2 * i + 1] = nu[1];
+      }
+      int st = cost[1] < cost[0] ? 1 : 0;
+      for (int i = 255; i >= 0; --i) {
+        codes[n * K + b * 256 + i] = bu[2 * i + st];
+        st = bs[2 * i + st];
       }
     }
   }

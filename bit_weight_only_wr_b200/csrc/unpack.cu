@@ -99,7 +99,7 @@ __global__ void __launch_bounds__(32 * kUnpackWarps) unpack_kernel(const uint8_t
       const float s = n < N ? half_bits_to_float(scales[n * B + ub]) : 0.f;
       const int L = FMT == WR_FMT_Q2 ? 3 : 7;
       int c[64];
-      if (FMT == WR_FMT_Q2) {
+      if (FMT == WR_FMT_Q2 || FMT == WR_FMT_T2) {
 #pragma unroll
         for (int w = 0; w < 4; ++w)
 #pragma unroll
@@ -120,6 +120,19 @@ __global__ void __launch_bounds__(32 * kUnpackWarps) unpack_kernel(const uint8_t
             for (int uu = 0; uu < 3; ++uu) cc |= ((rw[3 * g + uu] >> (16 * hh + 15)) & 1) << uu;
             c[32 * g + 30 + hh] = cc;
           }
+        }
+      }
+      if (FMT == WR_FMT_T2) {
+        // trellis: level index 2u + (low bit of the previous symbol); the previous symbol of
+        // this quarter's first code is the last of quarter q - 1 of the same row (another
+        // lane), and 0 at the block start
+        const uint32_t prev = __shfl_sync(0xffffffffu, (uint32_t)c[63] & 1u, lane_pos(r0, (q + 3) & 3));
+        int p = q == 0 ? 0 : (int)prev;
+#pragma unroll
+        for (int i = 0; i < 64; ++i) {
+          const int u = c[i];
+          c[i] = 2 * u + p;
+          p = u & 1;
         }
       }
 #pragma unroll
@@ -166,6 +179,7 @@ cudaError_t launch_unpack_bf16(int fmt, const uint8_t* packed, const uint16_t* s
   constexpr int th = 32 * kUnpackWarps;
   if (fmt == WR_FMT_Q2) unpack_kernel<WR_FMT_Q2><<<ctas, th, 0, stream>>>(packed, scales, N, K, units, U, w);
   else if (fmt == WR_FMT_Q3) unpack_kernel<WR_FMT_Q3><<<ctas, th, 0, stream>>>(packed, scales, N, K, units, U, w);
+  else if (fmt == WR_FMT_T2) unpack_kernel<WR_FMT_T2><<<ctas, th, 0, stream>>>(packed, scales, N, K, units, U, w);
   else unpack_kernel<WR_FMT_TERNARY><<<ctas, th, 0, stream>>>(packed, scales, N, K, units, U, w);
   return cudaGetLastError();
 }

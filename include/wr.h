@@ -85,7 +85,17 @@ typedef enum {
   WR_ERR_TOO_LARGE = 5      /* the problem needs more than the fixed scratch of wr_gemv_noalloc */
 } wr_status;
 
-enum { WR_FMT_TERNARY = 1, WR_FMT_Q2 = 2, WR_FMT_Q3 = 3 };
+enum { WR_FMT_TERNARY = 1, WR_FMT_Q2 = 2, WR_FMT_Q3 = 3, WR_FMT_T2 = 4 };
+
+/* WR_FMT_T2, the 2-bit trellis-coded format ("How We Shrank...", "Trick 3: trellis coding"):
+ * symbols u in [0, 4) are stored exactly like Q2 codes (same packed layout, same bytes), with
+ * fp16 scales per 256-block, but they select among the 8 odd levels {-7..7} * s through a
+ * 2-state trellis: at step i of a block the state is the low bit of u_(i-1) (0 at the block
+ * start), the level index is c3 = 2 u_i + state and the weight is s * (2 c3 - 7). This is the
+ * pages' 1-bit toy (two cosets of four levels, the written bit is the next state) written
+ * with 2 bits per weight. The codes come from wr_quantize_trellis (a Viterbi search). The
+ * decode GEMV (wr_gemv, wr_gemv_batched, wr_gemv_noalloc with bits = WR_FMT_T2) and
+ * wr_unpack_bf16 accept it; the prefill GEMM (M > 8) does not (WR_ERR_UNSUPPORTED). */
 
 /* Version of this ABI (incremented on any incompatible change). */
 int wr_abi_version(void);
@@ -123,6 +133,13 @@ wr_status wr_quantize(int bits, int64_t N, int64_t K, const float* w_host, uint8
  * which is the decision of the fp64 quotient. Asynchronous on `stream`. */
 wr_status wr_quantize_pack(int bits, int64_t N, int64_t K, const float* w, void* packed, uint16_t* scales,
                            void* stream);
+
+/* Host trellis encoder for WR_FMT_T2: per 256-block s = fp16(absmax / 7) (fp64 division, one
+ * rounding), then the symbol sequence of least squared error under the trellis (Viterbi; ties
+ * go to the lower state and symbol). w_host fp32 [N,K]; codes_host uint8 [N,K] (symbols
+ * 0..3, packed with wr_pack(WR_FMT_T2, ...)); scales_host fp16 bits [N, K/256]; K % 256 == 0. */
+wr_status wr_quantize_trellis(int64_t N, int64_t K, const float* w_host, uint8_t* codes_host,
+                              uint16_t* scales_host);
 
 /* Host synthetic ternary quantizer: W' = W R^T (fp64, per 128-block fast Walsh-Hadamard
  * transform with the sign mask), Delta_n = 0.7 * mean_k |W'[n,k]|, t = sign(W') where

@@ -79,6 +79,29 @@ def test_quantizer_matches_oracle(bits):
     assert np.array_equal(c1, c2)
 
 
+def test_trellis_quantizer_matches_oracle():
+    """The library's Viterbi encoder for the 2-bit trellis format picks the oracle's symbols
+    and scales, bit for bit (same fp64 arithmetic, same tie order)."""
+    W = wr_synth.weights_fp32(321, 48, 1024)
+    W[3, :256] = 0.0                                      # an all-zero block (s = 0)
+    W[5, 256:512] *= np.float32(1e-6)                     # a tiny block
+    c1, s1 = wr.wr_quantize_trellis(W)
+    c2, s2 = o.quantize_trellis2(W)
+    assert np.array_equal(s1, s2.view(np.uint16))
+    assert np.array_equal(c1, c2)
+
+
+@pytest.mark.parametrize("N,K", [(16, 256), (37, 768)])
+def test_trellis_format_packs_like_q2(N, K):
+    """WR_FMT_T2 stores its 2-bit symbols in the Q2 layout: same size, same bytes."""
+    rng = np.random.default_rng(N + K)
+    sym = rng.integers(0, 4, (N, K)).astype(np.uint8)
+    assert wr.wr_packed_bytes(wr.WR_FMT_T2, N, K) == wr.wr_packed_bytes(2, N, K)
+    p = wr.wr_pack(wr.WR_FMT_T2, sym)
+    assert np.array_equal(p, o.pack(o.FMT_Q2, sym))
+    assert np.array_equal(wr.wr_unpack_codes(wr.WR_FMT_T2, p, N, K), sym)
+
+
 def test_ternary_quantizer_matches_oracle():
     K = 1280
     signs = wr_synth.sign_bits(5, K)
@@ -102,7 +125,9 @@ def test_device_calls_reject_bad_arguments_before_launch():
     assert st == 1
     st = wr._lib.wr_gemv(9, 16, 256, 16, 16, 16, 2, 256, 16, 16, 1 << 20, None)   # M > 8
     assert st == 1
-    st = wr._lib.wr_gemv(1, 16, 256, 16, 16, 16, 4, 256, 16, 16, 1 << 20, None)   # bits
+    st = wr._lib.wr_gemv(1, 16, 256, 16, 16, 16, 5, 256, 16, 16, 1 << 20, None)   # bits
+    assert st == 2
+    st = wr._lib.wr_gemm(16, 16, 256, 16, 16, 16, 4, 256, 16, 16, 1 << 20, None)  # trellis, M > 8
     assert st == 2
     st = wr._lib.wr_gemv(1, 16, 256, 16, 16, 16, 2, 128, 16, 16, 1 << 20, None)   # group
     assert st == 2

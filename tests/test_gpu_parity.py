@@ -329,6 +329,67 @@ def test_ternary_gemv_batched_more_problems_than_one_launch(wr):
     assert wr.wr_get_device_error() == 0
 
 
+# ---------------------------------------------------------------- trellis-coded 2-bit format
+
+def tr_case(wr, N, K, seed):
+    W = wr_synth.weights_fp32(seed, N, K)
+    sym, sc = wr.wr_quantize_trellis(W)
+    sym_o, sc_o = o.quantize_trellis2(W)
+    assert np.array_equal(sym, sym_o) and np.array_equal(sc, sc_o.view(np.uint16))
+    return sym_o, sc_o, dev(wr.wr_pack(wr.WR_FMT_T2, sym)), dev(sc)
+
+
+@pytest.mark.parametrize("M", [1, 3, 8])
+@pytest.mark.parametrize("N,K", [(40, 512), (129, 768), (300, 2560)])
+def test_trellis_gemv(wr, M, N, K):
+    """Decode GEMV on the 2-bit trellis-coded format (bits = WR_FMT_T2) against the oracle's
+    decode of the same symbols."""
+    torch = torch_mod()
+    sym, sc, packed, s_d = tr_case(wr, N, K, seed=N + K + M)
+    x = wr_synth.activations_bf16(800 + M, M, K)
+    y = torch.full((M, N), float("nan"), dtype=torch.float32, device="cuda")
+    nb = wr.wr_gemv_workspace_bytes(M, N, K, wr.WR_FMT_T2)
+    ws = _zeros_ws(nb)
+    wr.wr_gemv(M, N, K, dev(x), packed, s_d, wr.WR_FMT_T2, y, ws, nb)
+    torch.cuda.synchronize()
+    ref, B = o.gemm_trellis2(x, sym, sc)
+    check_close(y.cpu().numpy(), ref, B)
+    assert wr.wr_get_device_error() == 0
+
+
+def test_trellis_in_a_mixed_batch(wr):
+    """Q2, Q3 and trellis problems in one batched launch."""
+    torch = torch_mod()
+    M = 4
+    problems, refs = [], []
+    for i, (N, K, fmt) in enumerate([(64, 512, 4), (100, 768, 2), (40, 256, 3), (200, 2560, 4)]):
+        x = wr_synth.activations_bf16(900 + i, M, K)
+        if fmt == 4:
+            sym, sc, packed, s_d = tr_case(wr, N, K, seed=70 + i)
+            refs.append(o.gemm_trellis2(x, sym, sc))
+        else:
+            codes, scales, packed, s_d = q_case(wr, fmt, N, K, seed=70 + i)
+            refs.append(o.gemm_codes(x, codes, scales, fmt))
+        y = torch.full((M, N), float("nan"), dtype=torch.float32, device="cuda")
+        problems.append((dev(x), packed, s_d, y, N, K, fmt))
+    nb = wr.wr_gemv_batched_workspace_bytes(M, problems)
+    ws = _zeros_ws(nb)
+    wr.wr_gemv_batched(M, problems, ws, nb)
+    torch.cuda.synchronize()
+    for (_, _, _, y, _, _, _), (ref, B) in zip(problems, refs):
+        check_close(y.cpu().numpy(), ref, B)
+
+
+@pytest.mark.parametrize("N,K", [(16, 256), (45, 768)])
+def test_trellis_unpack_bf16_bit_exact(wr, N, K):
+    torch = torch_mod()
+    sym, sc, packed, s_d = tr_case(wr, N, K, seed=3 * N + K)
+    out = torch.empty(N, K, dtype=torch.int16, device="cuda")
+    wr.wr_unpack_bf16(wr.WR_FMT_T2, N, K, packed, s_d, out)
+    torch.cuda.synchronize()
+    assert np.array_equal(out.cpu().numpy().view(np.uint16), o.f64_to_bf16_bits(o.dequant_trellis2(sym, sc)))
+
+
 # ---------------------------------------------------------------- device quantizer + packer
 
 def _edge_weights(N, K, seed):
