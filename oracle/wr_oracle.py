@@ -25,6 +25,9 @@ What it defines (citations are to the source pages by title and section):
   levels, the written bits pick a value inside it and set the next state, and a Viterbi
   search finds the cheapest path. The pages give the 2-state, 1-bit toy in full; the
   format here is its 2-bit form: 8 odd levels, state = low bit of the previous symbol.
+* Two-level int8 block scales ("Agents-A1-4B-Wringer-Q2.6", "What is in this repo":
+  packed codes with fp16 or int8 block scales): s[n, b] = d_n q[n, b], an fp16 scale per
+  row times an int8 multiplier 0..127 per 256-block.
 * The contraction y[m, n] = sum_k W[n, k] x[m, k] in fp64, and the bound
   B[m, n] = sum_k |W[n, k] x[m, k]| used for the per-element tolerance.
 * The packed byte layout (defined in ``include/wr.h``), re-implemented here from
@@ -112,6 +115,50 @@ def quantize_odd_grid(W: np.ndarray, bits: int):
     g = np.clip(g, -L, L).astype(np.int64)
     codes = ((g + L) // 2).astype(np.uint8).reshape(N, K)
     return codes, s16
+
+
+S8_QMAX = 127   # int8 block multipliers of the two-level scales take the values 0..127
+
+
+def quantize_odd_grid_s8(W: np.ndarray, bits: int):
+    """Nearest-point codes on the b-bit odd grid with int8 block scales.
+
+    The "Agents-A1-4B-Wringer-Q2.6" card ("What is in this repo") lists a container of
+    packed codes with fp16 or int8 block scales and says no more about the int8 form.
+    Reading: an int8 block scale is a multiplier of a wider per-row scale. Per row n:
+    A_n = max_k |w[n, k]|; d_n = fp16(A_n / (127 L)) (fp64 division, one rounding,
+    saturated to the largest finite fp16). Per 256-block b with absmax a_b:
+    q[n, b] = the integer nearest to a_b / (L d_n) (ties to even), clamped to [0, 127]
+    (0 when d_n = 0). The block scale is s[n, b] = d_n q[n, b] (exact in fp32: at most
+    11 + 7 significant bits), and the codes are the nearest odd levels of w / s exactly
+    as in quantize_odd_grid (an exact even quotient goes up, s == 0 gives g = +1).
+    Returns (codes uint8 [N, K], d float16 [N], q int8 [N, K/256])."""
+    W = np.asarray(W, dtype=np.float32)
+    N, K = W.shape
+    assert K % BLOCK == 0
+    L = grid_L(bits)
+    Wb = W.astype(np.float64).reshape(N, K // BLOCK, BLOCK)
+    absmax = np.abs(Wb).max(axis=2)                      # a_b * L, per block
+    A = absmax.max(axis=1)                               # row absmax
+    with np.errstate(over="ignore"):
+        d16 = fp16_round(A / (S8_QMAX * L))
+    d16 = np.minimum(d16, np.float16(np.finfo(np.float16).max))
+    d = d16.astype(np.float64)[:, None]
+    with np.errstate(divide="ignore", invalid="ignore"):
+        qf = np.where(d > 0, np.rint(absmax / (L * np.where(d > 0, d, 1.0))), 0.0)
+    q = np.clip(qf, 0, S8_QMAX).astype(np.int8)
+    s = (d * q.astype(np.float64))[:, :, None]
+    with np.errstate(divide="ignore", invalid="ignore"):
+        r = np.where(s > 0, Wb / np.where(s > 0, s, 1.0), 0.0)
+    g = 2.0 * np.floor(r / 2.0) + 1.0
+    g = np.clip(g, -L, L).astype(np.int64)
+    codes = ((g + L) // 2).astype(np.uint8).reshape(N, K)
+    return codes, d16, q
+
+
+def s8_block_scales(d: np.ndarray, q: np.ndarray) -> np.ndarray:
+    """s[n, b] = d_n * q[n, b] in fp64 (exact)."""
+    return np.asarray(d, dtype=np.float16).astype(np.float64)[:, None] * np.asarray(q, dtype=np.int64)
 
 
 # --------------------------------------------------------------------------------------
@@ -270,6 +317,34 @@ def dequant(codes: np.ndarray, scales: np.ndarray, bits: int) -> np.ndarray:
     g = code_to_level(codes, bits).astype(np.float64)
     s = np.asarray(scales, dtype=np.float16).astype(np.float64)
     return (g.reshape(N, K // BLOCK, BLOCK) * s[:, :, None]).reshape(N, K)
+
+
+def dequant_s8(codes: np.ndarray, d: np.ndarray, q: np.ndarray, bits: int) -> np.ndarray:
+    """W[n, k] = d_n q[n, k // 256] g(c[n, k]) in fp64 (two-level scales)."""
+    codes = np.asarray(codes)
+    N, K = codes.shape
+    g = code_to_level(codes, bits).astype(np.float64)
+    s = s8_block_scales(d, q)
+    return (g.reshape(N, K // BLOCK, BLOCK) * s[:, :, None]).reshape(N, K)
+
+
+def dequant_trellis2_s8(symbols: np.ndarray, d: np.ndarray, q: np.ndarray) -> np.ndarray:
+    """The trellis format with two-level scales: W = d_n q[n, b] (2 c3 - 7)."""
+    symbols = np.asarray(symbols)
+    N, K = symbols.shape
+    c3 = trellis_level_index(symbols.reshape(N * (K // BLOCK), BLOCK)).reshape(N, K)
+    g = code_to_level(c3, 3).astype(np.float64)
+    return (g.reshape(N, K // BLOCK, BLOCK) * s8_block_scales(d, q)[:, :, None]).reshape(N, K)
+
+
+def unpack_bf16_s8(codes: np.ndarray, d: np.ndarray, q: np.ndarray, bits: int) -> np.ndarray:
+    """The bf16 materialization with two-level scales: bf16_RNE(d q g), one rounding."""
+    return f64_to_bf16_bits(dequant_s8(codes, d, q, bits))
+
+
+def gemm_codes_s8(x_bits, codes, d, q, bits):
+    """y[m, n] = sum_b d_n q[n, b] sum_{k in b} g[n, k] x[m, k]."""
+    return gemm(x_bits, dequant_s8(codes, d, q, bits))
 
 
 def dequant_ternary(codes: np.ndarray, alpha: np.ndarray) -> np.ndarray:

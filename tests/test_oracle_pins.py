@@ -197,6 +197,88 @@ def test_quantizer_special_blocks():
     assert o.code_to_level(codes[1, 300], 2) == 1     # 0.25/s = 1.5 -> nearest odd is 1
 
 
+# ---------------------------------------------------------------- two-level int8 block scales
+
+def _nearest_int_ties_even(x: Fraction, lo: int, hi: int) -> int:
+    """Brute force over the integers lo..hi: the nearest to x, ties to the even one."""
+    best = None
+    for j in range(lo, hi + 1):
+        dist = abs(Fraction(j) - x)
+        if best is None or dist < best[0] or (dist == best[0] and j % 2 == 0):
+            best = (dist, j)
+    return best[1]
+
+
+@pytest.mark.parametrize("bits", [2, 3])
+def test_s8_scales_against_exact_arithmetic(bits):
+    L = o.grid_L(bits)
+    W = wr_synth.weights_fp32(31 + bits, 6, 1024)
+    W[2] *= np.linspace(0.05, 1.0, 1024, dtype=np.float32)   # blocks of very different absmax
+    codes, d, q = o.quantize_odd_grid_s8(W, bits)
+    assert d.dtype == np.float16 and q.dtype == np.int8 and q.shape == (6, 4)
+    levels = np.arange(-L, L + 1, 2)
+    for n in range(6):
+        A = max(Fraction(float(v)) for v in np.abs(W[n]))
+        assert Fraction(float(d[n])) == _fp16_exact_rne(A / (127 * L))
+        dn = Fraction(float(d[n]))
+        for b in range(4):
+            a = max(Fraction(float(v)) for v in np.abs(W[n, 256 * b:256 * (b + 1)]))
+            assert int(q[n, b]) == _nearest_int_ties_even(a / (L * dn), 0, 127)
+        # the block that holds the row maximum gets the full multiplier
+        assert q[n].max() == 127
+        s = o.s8_block_scales(d, q)
+        for k in range(0, 1024, 11):
+            r = float(W[n, k]) / float(s[n, k // 256])
+            dist = np.abs(levels - r)
+            assert o.code_to_level(codes[n, k], bits) == levels[dist == dist.min()].max()
+
+
+def test_s8_closed_form_row():
+    # Q2 (L = 3). Block 0's absmax 127*3*2^-8 makes d = 2^-8 exactly; blocks 1 and 2 have
+    # absmax 3*2^-8 times 10.5 and 11.5, exact ties that go to the even multipliers 10 and 12;
+    # block 3's absmax is 0.4 * 3 * 2^-8, whose multiplier rounds to 0 (s = 0, all codes +1).
+    u = 2.0 ** -8
+    W = np.zeros((3, 1024), dtype=np.float32)
+    W[0, 0] = 127 * 3 * u
+    W[0, 256] = 3 * u * 10.5
+    W[0, 257] = -0.05
+    W[0, 512] = -3 * u * 11.5
+    W[0, 768] = 0.4 * 3 * u
+    W[2, 5] = 1.0e9                      # d saturates at the largest finite fp16
+    codes, d, q = o.quantize_odd_grid_s8(W, 2)
+    assert float(d[0]) == u
+    assert q[0].tolist() == [127, 10, 12, 0]
+    g = o.code_to_level(codes[0], 2)
+    assert g[0] == 3 and g[256] == 3     # 0.123046875 / (10 u) = 3.15 -> level 3
+    assert g[257] == -1                  # -0.05 / (10 u) = -1.28 -> level -1
+    assert g[512] == -3 and np.all(g[768:] == 1)
+    # all-zero row: d = 0, q = 0, every code at level +1
+    assert float(d[1]) == 0.0 and np.all(q[1] == 0) and np.all(o.code_to_level(codes[1], 2) == 1)
+    assert float(d[2]) == 65504.0 and q[2, 0] == 127 and o.code_to_level(codes[2, 5], 2) == 3
+    assert q[2, 1] == 0
+
+
+def test_s8_dequant_hand_examples():
+    codes = np.zeros((2, 512), dtype=np.uint8)
+    codes[0, :2] = [0, 3]
+    codes[1, 256:258] = [7, 2]
+    d = np.array([0.5, 2.0 ** -10], dtype=np.float16)
+    q = np.array([[3, 1], [0, 100]], dtype=np.int8)
+    W2 = o.dequant_s8(codes, d, q, 2)
+    assert W2[0, 0] == -4.5 and W2[0, 1] == 4.5 and W2[0, 256] == -1.5 and np.all(W2[1, :256] == 0)
+    W3 = o.dequant_s8(codes, d, q, 3)
+    assert W3[1, 256] == 7 * 100 * 2.0 ** -10 and W3[1, 257] == -3 * 100 * 2.0 ** -10
+    # bf16 of 700 * 2^-10 = 0.68359375 is exact (8 significant bits)
+    bits = o.unpack_bf16_s8(codes, d, q, 3)
+    assert o.bf16_bits_to_f64(bits[1, 256]) == 0.68359375
+    # trellis symbols with two-level scales match the fp16-scale definition when d q is the scale
+    sym = np.random.default_rng(5).integers(0, 4, size=(2, 512)).astype(np.uint8)
+    dd = np.array([1.0, 0.25], dtype=np.float16)
+    qq = np.array([[5, 7], [9, 127]], dtype=np.int8)
+    ref = o.dequant_trellis2(sym, o.s8_block_scales(dd, qq))
+    assert np.array_equal(o.dequant_trellis2_s8(sym, dd, qq), ref)
+
+
 def test_dequant_hand_examples():
     codes = np.array([[0, 3] + [1] * 254, [7, 4] + [0] * 254], dtype=np.uint8)
     s2 = np.array([[0.5]], dtype=np.float16)
