@@ -516,6 +516,39 @@ def run_extras(args, wr, torch, np, stream, dist, hbm_peak, bf16_peak):
     except Exception as e:  # noqa: BLE001
         out["trellis2"] = {"error": repr(e)}
 
+    # int8 block scales (fp16 row scale times an int8 multiplier per 256-block): one layer's 7
+    # linears quantized once by the device quantizer, the 36-layer body made of 36 distinct byte
+    # copies, one batched decode GEMV call per token
+    try:
+        res = {}
+        smods = []
+        for idx, (name, K, N, bits) in enumerate(wr_synth.QWEN3_4B_LAYER):
+            fmt = bits | wr.WR_SCALES_I8
+            W = torch.from_numpy(wr_synth.weights_fp32(700 + idx, N, K)).cuda()
+            pk = torch.empty(wr.wr_packed_bytes(bits, N, K), dtype=torch.uint8, device="cuda")
+            rec = torch.zeros(wr.wr_scales_bytes(fmt, N, K), dtype=torch.uint8, device="cuda")
+            wr.wr_quantize_pack(fmt, N, K, W, pk, rec)
+            torch.cuda.synchronize()
+            del W
+            smods.append((K, N, fmt, pk, rec))
+        body = [(K, N, fmt, p.roll(c * 4096), r.clone()) for c in range(36) for (K, N, fmt, p, r) in smods]
+        for M in (1, 8):
+            xs = [torch.from_numpy(wr_synth.activations_bf16(6000 + j, M, K).view(np.int16)).cuda()
+                  for j, (K, _, _, _, _) in enumerate(body)]
+            ys = [torch.empty(M, N, dtype=torch.float32, device="cuda") for (_, N, _, _, _) in body]
+            arr = wr._problems([(xs[j], p, r, ys[j], N, K, fmt) for j, (K, N, fmt, p, r) in enumerate(body)])
+            nb = wr.wr_gemv_batched_workspace_bytes(M, arr)
+            ws = torch.zeros(nb, dtype=torch.uint8, device="cuda")
+
+            def sstep():
+                wr.wr_gemv_batched(M, arr, ws, nb)
+            ms = graph_time_ms(torch, sstep, 10, 3, stream) / 10
+            b = sum(p.numel() + 2 * N + N * (K // 256) + 2 * M * K + 4 * M * N for (K, N, _, p, _) in body)
+            res[f"body_M{M}"] = {"ms": ms, "bytes": b, "gbs": b / ms / 1e6, "tokens_per_s": M * 1e3 / ms}
+        out["scales_i8"] = res
+    except Exception as e:  # noqa: BLE001
+        out["scales_i8"] = {"error": repr(e)}
+
     # device quantizer + packer (fp32 W -> packed codes + fp16 scales) on the gate and up shapes
     try:
         res = {}
@@ -530,6 +563,15 @@ def run_extras(args, wr, torch, np, stream, dist, hbm_peak, bf16_peak):
             ms = graph_time_ms(torch, step, 20, 3, stream) / 20
             b = 4 * N * K + wr.wr_packed_bytes(bits, N, K) + 2 * N * (K // 256)
             res[name] = {"us": ms * 1e3, "gbs": b / ms / 1e6, "bytes": b}
+            # int8 block scales: a row pass over W, then the pack pass (W is read twice)
+            fmt = bits | wr.WR_SCALES_I8
+            rec = torch.zeros(wr.wr_scales_bytes(fmt, N, K), dtype=torch.uint8, device="cuda")
+
+            def step8():
+                wr.wr_quantize_pack(fmt, N, K, W, pk, rec)
+            ms = graph_time_ms(torch, step8, 20, 3, stream) / 20
+            b = 4 * N * K + wr.wr_packed_bytes(bits, N, K) + 2 * N + N * (K // 256)
+            res[name + "_i8"] = {"us": ms * 1e3, "gbs": b / ms / 1e6, "bytes": b, "w_reads": 2}
         out["quantize_pack"] = res
     except Exception as e:  # noqa: BLE001
         out["quantize_pack"] = {"error": repr(e)}

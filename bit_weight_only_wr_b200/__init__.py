@@ -20,10 +20,11 @@ __all__ = [
     "wr_get_device_error", "exported_symbols", "WrGemvProblem", "wr_gemv_batched_workspace_bytes",
     "wr_gemv_batched", "wr_gemv_noalloc", "WR_GEMV_NOALLOC_SCRATCH_BYTES", "WrGemvTernaryProblem",
     "wr_gemv_ternary_batched_workspace_bytes", "wr_gemv_ternary_batched", "wr_selftest_wait_timeout",
-    "wr_quantize_pack", "wr_quantize_trellis", "WR_FMT_T2",
+    "wr_quantize_pack", "wr_quantize_trellis", "WR_FMT_T2", "WR_SCALES_I8", "wr_scales_bytes",
 ]
 
 WR_FMT_TERNARY, WR_FMT_Q2, WR_FMT_Q3, WR_FMT_T2 = 1, 2, 3, 4
+WR_SCALES_I8 = 0x100   # OR'd into a format code: int8 block scales (the scale record of include/wr.h)
 WR_GEMV_NOALLOC_SCRATCH_BYTES = 4 << 20   # mirrors the macro in include/wr.h
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libwr.so")
 
@@ -52,6 +53,7 @@ _SIGNATURES = {
     "wr_abi_version": (_c_int, []),
     "wr_status_string": (ctypes.c_char_p, [_c_int]),
     "wr_packed_bytes": (_c_size, [_c_int, _c_i64, _c_i64]),
+    "wr_scales_bytes": (_c_size, [_c_int, _c_i64, _c_i64]),
     "wr_pack": (_c_int, [_c_int, _c_i64, _c_i64, _vp, _vp]),
     "wr_unpack_codes": (_c_int, [_c_int, _c_i64, _c_i64, _vp, _vp]),
     "wr_quantize": (_c_int, [_c_int, _c_i64, _c_i64, _vp, _vp, _vp]),
@@ -136,6 +138,10 @@ def wr_packed_bytes(fmt: int, N: int, K: int) -> int:
     return _lib.wr_packed_bytes(fmt, N, K)
 
 
+def wr_scales_bytes(fmt: int, N: int, K: int) -> int:
+    return _lib.wr_scales_bytes(fmt, N, K)
+
+
 def wr_pack(fmt: int, codes: np.ndarray) -> np.ndarray:
     codes = np.ascontiguousarray(codes, dtype=np.uint8)
     N, K = codes.shape
@@ -157,11 +163,15 @@ def wr_unpack_codes(fmt: int, packed: np.ndarray, N: int, K: int) -> np.ndarray:
 
 
 def wr_quantize(bits: int, W: np.ndarray):
-    """fp32 [N, K] -> (codes uint8 [N, K], fp16 scale bits uint16 [N, K/256])."""
+    """fp32 [N, K] -> (codes uint8 [N, K], fp16 scale bits uint16 [N, K/256]); with
+    bits | WR_SCALES_I8 the scales are the int8 scale record (uint8 [wr_scales_bytes])."""
     W = np.ascontiguousarray(W, dtype=np.float32)
     N, K = W.shape
     codes = np.empty((N, K), dtype=np.uint8)
-    scales = np.empty((N, max(K // 256, 1)), dtype=np.uint16)
+    if bits & WR_SCALES_I8:
+        scales = np.zeros(max(wr_scales_bytes(bits, N, K), 16), dtype=np.uint8)
+    else:
+        scales = np.empty((N, max(K // 256, 1)), dtype=np.uint16)
     _check("wr_quantize", _lib.wr_quantize(bits, N, K, _ptr(W), _ptr(codes), _ptr(scales)))
     return codes, scales
 

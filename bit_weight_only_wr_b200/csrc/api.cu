@@ -54,6 +54,22 @@ wr_status check_dims(int64_t M, int64_t N, int64_t K) {
   return WR_OK;
 }
 
+// The format argument of the 2/3-bit calls: a base format, optionally | WR_SCALES_I8.
+struct QFmt {
+  int base;
+  bool s8;
+};
+inline bool split_fmt(int fmt, bool allow_t2, QFmt* f) {
+  f->s8 = (fmt & WR_SCALES_I8) != 0;
+  f->base = fmt & ~WR_SCALES_I8;
+  return f->base == WR_FMT_Q2 || f->base == WR_FMT_Q3 || (allow_t2 && f->base == WR_FMT_T2);
+}
+// The int8 multipliers of an int8 scale record (null for fp16 scales).
+inline const int8_t* scale_q_of(const QFmt& f, const uint16_t* scales, int64_t N) {
+  return f.s8 ? reinterpret_cast<const int8_t*>(reinterpret_cast<const uint8_t*>(scales) + wr::s8_q_offset(N))
+              : nullptr;
+}
+
 constexpr int kPlanSMs = 148;   // split heuristics are sized for a 148-SM part (device-independent)
 constexpr int kDecodeGrid = 3 * kPlanSMs;   // 2/3-bit decode: CTAs (block ranges) per launch, at most
 constexpr int kDecodeTokens = 8;   // decode kernel: 8 tokens x 4 activation limbs = 32 MMA columns
@@ -192,11 +208,12 @@ wr::TcArgs gemm_args(const GemmPlan& p, int64_t M, int64_t N, int64_t K, void* w
 }
 
 wr_status run_gemm(int bits, int M, int N, int K, const uint16_t* x, const uint8_t* packed, const uint16_t* scales,
-                   float* y, void* workspace, cudaStream_t stream) {
+                   const int8_t* scale_q, float* y, void* workspace, cudaStream_t stream) {
   const GemmPlan p = plan_gemm(M, N, K, 128, 256);
   wr::TcArgs a = gemm_args(p, M, N, K, workspace);
   a.packed = packed;
   a.scales = scales;
+  a.scale_q = scale_q;
   a.y = y;
   return wr::launch_tc_kernel(bits, 128, a, x, M, K, p.grid, stream) == cudaSuccess ? WR_OK : WR_ERR_CUDA;
 }
@@ -213,7 +230,7 @@ size_t q_workspace(int bits, int64_t M, int64_t N, int64_t K) {
 }
 
 wr_status run_q(int bits, int64_t M, int64_t N, int64_t K, const uint16_t* x, const void* packed,
-                const uint16_t* scales, float* y, void* workspace, cudaStream_t stream) {
+                const uint16_t* scales, const int8_t* scale_q, float* y, void* workspace, cudaStream_t stream) {
   if (M <= kDecodeTokens) {
     static thread_local DecodePlan dp;
     const ProblemShape sh{N, K, bits};
@@ -221,11 +238,13 @@ wr_status run_q(int bits, int64_t M, int64_t N, int64_t K, const uint16_t* x, co
     dp.args.prob[0].x = x;
     dp.args.prob[0].packed = static_cast<const uint8_t*>(packed);
     dp.args.prob[0].scales = scales;
+    dp.args.prob[0].scale_q = scale_q;
     dp.args.prob[0].y = y;
     bind_workspace(dp, workspace);
     return run_decode(dp, false, stream);
   }
-  return run_gemm(bits, (int)M, (int)N, (int)K, x, static_cast<const uint8_t*>(packed), scales, y, workspace, stream);
+  return run_gemm(bits, (int)M, (int)N, (int)K, x, static_cast<const uint8_t*>(packed), scales, scale_q, y, workspace,
+                  stream);
 }
 
 // Ternary. M <= 8: the decode kernel (R x hi and lo fill the MMA columns). M > 8: the prefill
@@ -324,41 +343,51 @@ const char* wr_status_string(wr_status st) {
 
 wr_status wr_unpack_bf16(int fmt, int64_t N, int64_t K, const void* packed, const uint16_t* scales,
                          int group, uint16_t* w_bf16, void* stream) {
-  if (fmt != WR_FMT_Q2 && fmt != WR_FMT_Q3 && fmt != WR_FMT_TERNARY && fmt != WR_FMT_T2) return WR_ERR_UNSUPPORTED;
+  QFmt f{};
+  if (!split_fmt(fmt, true, &f) && fmt != WR_FMT_TERNARY) return WR_ERR_UNSUPPORTED;
+  if (fmt == WR_FMT_TERNARY) f = QFmt{WR_FMT_TERNARY, false};
+  fmt = f.base;
   if (check_dims(1, N, K) != WR_OK) return WR_ERR_INVALID_ARG;
   if (fmt != WR_FMT_TERNARY && group != 256) return WR_ERR_UNSUPPORTED;
   int64_t ub = 0, units = 0, tiles = 0;
   if (!wr::packed_geometry(fmt, N, K, &ub, &units, &tiles)) return WR_ERR_INVALID_ARG;
   if (!aligned16(packed) || !aligned16(scales) || !aligned16(w_bf16)) return WR_ERR_INVALID_ARG;
-  const cudaError_t e = wr::launch_unpack_bf16(fmt, static_cast<const uint8_t*>(packed), scales, (int)N,
-                                               (int)K, (int)units, w_bf16, static_cast<cudaStream_t>(stream));
+  const cudaError_t e = wr::launch_unpack_bf16(fmt, static_cast<const uint8_t*>(packed), scales,
+                                               scale_q_of(f, scales, N), (int)N, (int)K, (int)units, w_bf16,
+                                               static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? WR_OK : WR_ERR_CUDA;
 }
 
 size_t wr_gemv_workspace_bytes(int64_t M, int64_t N, int64_t K, int bits) {
-  if (bits != 2 && bits != 3 && bits != WR_FMT_T2) return 0;
+  QFmt f{};
+  if (!split_fmt(bits, true, &f)) return 0;
   if (M < 1 || M > 8 || check_dims(M, N, K) != WR_OK || K % 256 != 0) return 0;
-  return q_workspace(bits, M, N, K);
+  return q_workspace(f.base, M, N, K);
 }
 
 wr_status wr_gemv(int64_t M, int64_t N, int64_t K, const uint16_t* x, const void* packed,
                   const uint16_t* scales, int bits, int group, float* y, void* workspace,
                   size_t workspace_bytes, void* stream) {
-  if (bits != 2 && bits != 3 && bits != WR_FMT_T2) return WR_ERR_UNSUPPORTED;
+  QFmt f{};
+  if (!split_fmt(bits, true, &f)) return WR_ERR_UNSUPPORTED;
   if (group != 256) return WR_ERR_UNSUPPORTED;
   if (M < 1 || M > 8 || check_dims(M, N, K) != WR_OK || K % 256 != 0) return WR_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(packed) || !aligned16(scales) || !aligned16(y) || !aligned16(workspace))
     return WR_ERR_INVALID_ARG;
-  if (workspace_bytes < q_workspace(bits, M, N, K)) return WR_ERR_INVALID_ARG;
-  return run_q(bits, M, N, K, x, packed, scales, y, workspace, static_cast<cudaStream_t>(stream));
+  if (workspace_bytes < q_workspace(f.base, M, N, K)) return WR_ERR_INVALID_ARG;
+  return run_q(f.base, M, N, K, x, packed, scales, scale_q_of(f, scales, N), y, workspace,
+               static_cast<cudaStream_t>(stream));
 }
 
 wr_status wr_gemv_noalloc(int64_t M, int64_t N, int64_t K, const uint16_t* x, const void* packed,
                           const uint16_t* scales, int bits, int group, float* y, void* stream) {
-  if (bits != 2 && bits != 3 && bits != WR_FMT_T2) return WR_ERR_UNSUPPORTED;
+  QFmt f{};
+  if (!split_fmt(bits, true, &f)) return WR_ERR_UNSUPPORTED;
+  bits = f.base;
   if (group != 256) return WR_ERR_UNSUPPORTED;
   if (M < 1 || M > 8 || check_dims(M, N, K) != WR_OK || K % 256 != 0) return WR_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(packed) || !aligned16(scales) || !aligned16(y)) return WR_ERR_INVALID_ARG;
+  const int8_t* scale_q = scale_q_of(f, scales, N);
   if (q_workspace(bits, M, N, K) > WR_GEMV_NOALLOC_SCRATCH_BYTES) return WR_ERR_TOO_LARGE;
   wr_status st = WR_OK;
   void* scratch = noalloc_scratch(&st);
@@ -369,13 +398,14 @@ wr_status wr_gemv_noalloc(int64_t M, int64_t N, int64_t K, const uint16_t* x, co
   plan_decode(M, 1, &sh, &dp);
   const cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (dp.partial_off > 0 && cudaMemsetAsync(scratch, 0, dp.partial_off, s) != cudaSuccess) return WR_ERR_CUDA;
-  return run_q(bits, M, N, K, x, packed, scales, y, scratch, s);
+  return run_q(bits, M, N, K, x, packed, scales, scale_q, y, scratch, s);
 }
 
 static bool batch_ok(int64_t M, int32_t count, const wr_gemv_problem* pr) {
   if (M < 1 || M > 8 || count < 1 || !pr) return false;
   for (int i = 0; i < count; ++i) {
-    if (pr[i].bits != 2 && pr[i].bits != 3 && pr[i].bits != WR_FMT_T2) return false;
+    QFmt f{};
+    if (!split_fmt(pr[i].bits, true, &f)) return false;
     if (pr[i].reserved != 0 || check_dims(M, pr[i].N, pr[i].K) != WR_OK || pr[i].K % 256 != 0) return false;
     if (!aligned16(pr[i].x) || !aligned16(pr[i].packed) || !aligned16(pr[i].scales) || !aligned16(pr[i].y))
       return false;
@@ -390,7 +420,8 @@ size_t wr_gemv_batched_workspace_bytes(int64_t M, int32_t count, const wr_gemv_p
   ProblemShape sh[wr::kMaxDecodeProblems];
   for (int c0 = 0; c0 < count; c0 += wr::kMaxDecodeProblems) {
     const int n = std::min(count - c0, wr::kMaxDecodeProblems);
-    for (int i = 0; i < n; ++i) sh[i] = ProblemShape{problems[c0 + i].N, problems[c0 + i].K, problems[c0 + i].bits};
+    for (int i = 0; i < n; ++i)
+      sh[i] = ProblemShape{problems[c0 + i].N, problems[c0 + i].K, problems[c0 + i].bits & ~WR_SCALES_I8};
     plan_decode(M, n, sh, &dp);
     total = std::max(total, dp.total);
   }
@@ -405,12 +436,17 @@ wr_status wr_gemv_batched(int64_t M, int32_t count, const wr_gemv_problem* probl
   ProblemShape sh[wr::kMaxDecodeProblems];
   for (int c0 = 0; c0 < count; c0 += wr::kMaxDecodeProblems) {
     const int n = std::min(count - c0, wr::kMaxDecodeProblems);
-    for (int i = 0; i < n; ++i) sh[i] = ProblemShape{problems[c0 + i].N, problems[c0 + i].K, problems[c0 + i].bits};
+    for (int i = 0; i < n; ++i)
+      sh[i] = ProblemShape{problems[c0 + i].N, problems[c0 + i].K, problems[c0 + i].bits & ~WR_SCALES_I8};
     plan_decode(M, n, sh, &dp);
     for (int i = 0; i < n; ++i) {
-      dp.args.prob[i].x = problems[c0 + i].x;
-      dp.args.prob[i].packed = static_cast<const uint8_t*>(problems[c0 + i].packed);
-      dp.args.prob[i].scales = problems[c0 + i].scales;
+      const wr_gemv_problem& pi = problems[c0 + i];
+      QFmt f{};
+      split_fmt(pi.bits, true, &f);
+      dp.args.prob[i].x = pi.x;
+      dp.args.prob[i].packed = static_cast<const uint8_t*>(pi.packed);
+      dp.args.prob[i].scales = pi.scales;
+      dp.args.prob[i].scale_q = scale_q_of(f, pi.scales, pi.N);
       dp.args.prob[i].y = problems[c0 + i].y;
     }
     bind_workspace(dp, workspace);
@@ -476,21 +512,24 @@ wr_status wr_gemv_ternary_batched(int64_t M, int32_t count, const wr_gemv_ternar
 }
 
 size_t wr_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int bits) {
-  if (bits != 2 && bits != 3) return 0;
+  QFmt f{};
+  if (!split_fmt(bits, false, &f)) return 0;
   if (check_dims(M, N, K) != WR_OK || K % 256 != 0) return 0;
-  return q_workspace(bits, M, N, K);
+  return q_workspace(f.base, M, N, K);
 }
 
 wr_status wr_gemm(int64_t M, int64_t N, int64_t K, const uint16_t* x, const void* packed,
                   const uint16_t* scales, int bits, int group, float* y, void* workspace,
                   size_t workspace_bytes, void* stream) {
-  if (bits != 2 && bits != 3) return WR_ERR_UNSUPPORTED;
+  QFmt f{};
+  if (!split_fmt(bits, false, &f)) return WR_ERR_UNSUPPORTED;
   if (group != 256) return WR_ERR_UNSUPPORTED;
   if (check_dims(M, N, K) != WR_OK || K % 256 != 0) return WR_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(packed) || !aligned16(scales) || !aligned16(y) || !aligned16(workspace))
     return WR_ERR_INVALID_ARG;
-  if (workspace_bytes < q_workspace(bits, M, N, K)) return WR_ERR_INVALID_ARG;
-  return run_q(bits, M, N, K, x, packed, scales, y, workspace, static_cast<cudaStream_t>(stream));
+  if (workspace_bytes < q_workspace(f.base, M, N, K)) return WR_ERR_INVALID_ARG;
+  return run_q(f.base, M, N, K, x, packed, scales, scale_q_of(f, scales, N), y, workspace,
+               static_cast<cudaStream_t>(stream));
 }
 
 size_t wr_gemm_ternary_workspace_bytes(int64_t M, int64_t N, int64_t K) {
@@ -511,10 +550,12 @@ wr_status wr_gemm_ternary(int64_t M, int64_t N, int64_t K, const uint16_t* x, co
 
 wr_status wr_quantize_pack(int bits, int64_t N, int64_t K, const float* w, void* packed, uint16_t* scales,
                            void* stream) {
-  if (bits != 2 && bits != 3) return WR_ERR_UNSUPPORTED;
+  QFmt f{};
+  if (!split_fmt(bits, false, &f)) return WR_ERR_UNSUPPORTED;
   if (check_dims(1, N, K) != WR_OK || K % 256 != 0) return WR_ERR_INVALID_ARG;
   if (!aligned16(w) || !aligned16(packed) || !aligned16(scales)) return WR_ERR_INVALID_ARG;
-  return wr::launch_quantize_pack(bits, w, (int)N, (int)K, static_cast<uint8_t*>(packed), scales,
+  int8_t* scale_q = const_cast<int8_t*>(scale_q_of(f, scales, N));
+  return wr::launch_quantize_pack(f.base, w, (int)N, (int)K, static_cast<uint8_t*>(packed), scales, scale_q,
                                   static_cast<cudaStream_t>(stream)) == cudaSuccess
              ? WR_OK
              : WR_ERR_CUDA;

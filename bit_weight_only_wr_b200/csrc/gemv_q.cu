@@ -98,6 +98,7 @@ struct Pos {
   const uint8_t* packed;
   const uint8_t* xt;
   const uint16_t* scales;
+  const int8_t* scale_q;
   float* y;
 };
 
@@ -114,6 +115,7 @@ __device__ __forceinline__ void pos_load(Pos& p, const DecArgs& a) {
   p.packed = pr.packed;
   p.xt = pr.xt;
   p.scales = pr.scales;
+  p.scale_q = pr.scale_q;
   p.y = pr.y;
 }
 __device__ __forceinline__ Pos pos_start(const DecArgs& a) {
@@ -244,7 +246,10 @@ __device__ __forceinline__ void tmem_wait_ld_regs(uint32_t (&r)[NC]) {
   for (int i = 0; i < NC; ++i) asm volatile("" : "+r"(r[i]));
 }
 
-template <int XR>   // MMA N: 4 limb rows per token slot (8, 16 or 32 for M <= 2, 4, 8)
+// XR: MMA N, 4 limb rows per token slot (8, 16 or 32 for M <= 2, 4, 8). kAll: the batch holds
+// trellis-coded problems or int8 block scales; without them the decode and epilogue warps keep
+// only the Q2/Q3 branches and the fp16 scale load.
+template <int XR, bool kAll>
 __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_q_kernel(const __grid_constant__ DecArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -369,14 +374,14 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_q_kernel(const __gr
       uint32_t v[32];
       uint32_t carry = 0;   // trellis state at the block start
       if (dc.bits == 2) q2_half_i8(unit, r0, half, 0, v);
-      else if (dc.bits == 3) q3_half_i8(unit, r0, half, 0, v);
+      else if (!kAll || dc.bits == 3) q3_half_i8(unit, r0, half, 0, v);
       else t2_half_i8(unit, r0, half, 0, v, carry);
       // the A buffer is free once block gd - 1's MMAs are done
       if (gd > 0 && !mbar_wait(&bars->mma_done[(gd - 1) % kSX], ((gd - 1) / kSX) & 1, abort_flag, a.err, 302)) break;
       fence_after_sync();
       tmem_st32(lane_base + kACol, v);
       if (dc.bits == 2) q2_half_i8(unit, r0, half, 1, v);
-      else if (dc.bits == 3) q3_half_i8(unit, r0, half, 1, v);
+      else if (!kAll || dc.bits == 3) q3_half_i8(unit, r0, half, 1, v);
       else t2_half_i8(unit, r0, half, 1, v, carry);
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->pk_empty[sp]);
@@ -403,22 +408,32 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_q_kernel(const __gr
       return mbar_wait(&bars->group, (ng++) & 1, abort_flag, a.err, code);
     };
     // the scale of the block being finished is loaded one block ahead (its latency is an L2
-    // round trip, longer than the work it would wait for)
-    auto scale_of = [&](const Pos& c) -> uint16_t {
+    // round trip, longer than the work it would wait for): the fp16 scale with multiplier 1,
+    // or the row scale d and the int8 multiplier q (s = d q, exact in fp32)
+    auto scale_of = [&](const Pos& c, int& qv) -> uint16_t {
       const int n = c.rg * 128 + t;
-      return (c.left > 0 && n < c.N) ? __ldg(c.scales + (int64_t)n * c.B + c.b) : (uint16_t)0;
+      qv = 0;
+      if (c.left <= 0 || n >= c.N) return (uint16_t)0;
+      if (!kAll || c.scale_q == nullptr) {
+        qv = 1;
+        return __ldg(c.scales + (int64_t)n * c.B + c.b);
+      }
+      qv = __ldg(c.scale_q + (int64_t)n * c.B + c.b);
+      return __ldg(c.scales + n);
     };
     Pos ec = pos_start(a);
-    uint16_t snext = scale_of(ec);
+    int qnext = 0;
+    uint16_t snext = scale_of(ec, qnext);
     for (uint32_t ge = 0; ec.left > 0; ++ge) {
       const int n = ec.rg * 128 + t;
       const uint16_t sraw = snext;
+      const int qraw = qnext;
       const int sc = ge % kSC;
       if (!mbar_wait(&bars->mma_done[ge % kSX], (ge / kSX) & 1, abort_flag, a.err, 303)) break;
       if (!mbar_wait(&bars->c_full[sc], (ge / kSC) & 1, abort_flag, a.err, 304)) break;
       fence_after_sync();
       const int4* rec = reinterpret_cast<const int4*>(cs + sc * 256);
-      const float s = half_bits_to_float(sraw);
+      const float s = kAll ? half_bits_to_float(sraw) * (float)qraw : half_bits_to_float(sraw);
       constexpr int kChunk = XR < 16 ? XR : 16;   // columns per load
 #pragma unroll
       for (int c0 = 0; c0 < XR; c0 += kChunk) {
@@ -493,7 +508,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_q_kernel(const __gr
         for (int m = 0; m < kSlots; ++m) acc[m] = 0.f;
       }
       pos_next(ec, a);
-      snext = scale_of(ec);
+      snext = scale_of(ec, qnext);
     }
   }
 
@@ -592,30 +607,38 @@ cudaError_t launch_prep_x(const DecArgs& a, int total_blocks, cudaStream_t strea
 }
 
 namespace {
-template <int XR>
+template <int XR, bool kAll>
 cudaError_t launch_xr(const DecArgs& a, int grid, cudaStream_t stream) {
   static bool set[64] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
   if (!set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(gemv_q_kernel<XR>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
+    cudaError_t e =
+        cudaFuncSetAttribute(gemv_q_kernel<XR, kAll>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
     // all of the unified L1/shared array as shared memory, so that three CTAs fit
     if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(gemv_q_kernel<XR>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+      e = cudaFuncSetAttribute(gemv_q_kernel<XR, kAll>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
     if (e != cudaSuccess) return e;
     set[dev] = true;
   }
-  gemv_q_kernel<XR><<<grid, kThreads, kSmem, stream>>>(a);
+  gemv_q_kernel<XR, kAll><<<grid, kThreads, kSmem, stream>>>(a);
   return cudaGetLastError();
+}
+
+template <bool kAll>
+cudaError_t launch_feat(const DecArgs& a, int grid, cudaStream_t stream) {
+  switch (decode_xrows(a.M)) {
+    case 8: return launch_xr<8, kAll>(a, grid, stream);
+    case 16: return launch_xr<16, kAll>(a, grid, stream);
+    default: return launch_xr<32, kAll>(a, grid, stream);
+  }
 }
 }  // namespace
 
 cudaError_t launch_gemv_q(const DecArgs& a, int grid, cudaStream_t stream) {
-  switch (decode_xrows(a.M)) {
-    case 8: return launch_xr<8>(a, grid, stream);
-    case 16: return launch_xr<16>(a, grid, stream);
-    default: return launch_xr<32>(a, grid, stream);
-  }
+  bool all = false;
+  for (int i = 0; i < a.count; ++i) all = all || a.prob[i].bits == WR_FMT_T2 || a.prob[i].scale_q != nullptr;
+  return all ? launch_feat<true>(a, grid, stream) : launch_feat<false>(a, grid, stream);
 }
 
 }  // namespace wr

@@ -247,20 +247,53 @@ wr_status wr_unpack_codes(int fmt, int64_t N, int64_t K, const uint8_t* packed, 
   return WR_OK;
 }
 
+size_t wr_scales_bytes(int fmt, int64_t N, int64_t K) {
+  const bool s8 = (fmt & WR_SCALES_I8) != 0;
+  const int base = fmt & ~WR_SCALES_I8;
+  Geometry g;
+  if (!geometry(base, N, K, &g)) return 0;
+  if (base == WR_FMT_TERNARY) return s8 ? 0 : (size_t)(2 * N);
+  const int64_t nb = K / 256;
+  return s8 ? (size_t)(wr::s8_q_offset(N) + N * nb) : (size_t)(2 * N * nb);
+}
+
 wr_status wr_quantize(int bits, int64_t N, int64_t K, const float* w, uint8_t* codes, uint16_t* scales) {
+  const bool s8 = (bits & WR_SCALES_I8) != 0;
+  bits &= ~WR_SCALES_I8;
   if (bits != 2 && bits != 3) return WR_ERR_UNSUPPORTED;
   if (N <= 0 || K <= 0 || K % 256 != 0 || !w || !codes || !scales) return WR_ERR_INVALID_ARG;
   const int L = (1 << bits) - 1;
   const int64_t nb = K / 256;
+  // int8 scale record: d fp16 [N] at byte 0, q int8 [N, nb] from byte s8_q_offset(N)
+  int8_t* qrec = s8 ? reinterpret_cast<int8_t*>(reinterpret_cast<uint8_t*>(scales) + wr::s8_q_offset(N)) : nullptr;
 #pragma omp parallel for schedule(static)
   for (int64_t n = 0; n < N; ++n) {
+    double d = 0.0;
+    if (s8) {
+      // d_n = fp16(A_n / (127 L)), saturated to the largest finite fp16
+      double A = 0.0;
+      for (int64_t k = 0; k < K; ++k) A = std::fmax(A, std::fabs((double)w[n * K + k]));
+      uint16_t dh = double_to_half(A / (double)(127 * L));
+      if ((dh & 0x7FFFu) >= 0x7C00u) dh = 0x7BFFu;
+      scales[n] = dh;
+      d = half_to_double(dh);
+    }
     for (int64_t b = 0; b < nb; ++b) {
       const float* wb = w + n * K + b * 256;
       double amax = 0.0;
       for (int i = 0; i < 256; ++i) amax = std::fmax(amax, std::fabs((double)wb[i]));
-      const uint16_t sh = double_to_half(amax / (double)L);
-      scales[n * nb + b] = sh;
-      const double s = half_to_double(sh);
+      double s;
+      if (s8) {
+        // q = nearest integer to amax / (L d) (ties to even under the default rounding mode)
+        double qv = d > 0.0 ? std::nearbyint(amax / ((double)L * d)) : 0.0;
+        qv = std::min(127.0, std::max(0.0, qv));
+        qrec[n * nb + b] = (int8_t)qv;
+        s = d * qv;
+      } else {
+        const uint16_t sh = double_to_half(amax / (double)L);
+        scales[n * nb + b] = sh;
+        s = half_to_double(sh);
+      }
       for (int i = 0; i < 256; ++i) {
         int g = 1;
         if (s > 0.0) {

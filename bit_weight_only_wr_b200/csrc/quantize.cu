@@ -18,6 +18,13 @@
 // quarter q of rows r0 and r0 + 8, the 4 lanes of a row find the block's absmax by two
 // shuffles, and each lane writes its own 16-byte chunks of the unit (see the packed layout in
 // include/wr.h). W is read once, with 16-byte loads.
+//
+// Int8 block scales (the "Agents-A1-4B-Wringer-Q2.6" card, "What is in this repo": fp16 / int8
+// block scales): a first pass finds each row's absmax A and writes d = fp16(A / (127 L))
+// (fp64 division, one rounding, saturated to 65504); the pack pass then takes
+// q = rint(absmax / (L d)) in fp64 (ties to even), clamped to [0, 127], and chooses the codes
+// against s = d q, exact in fp32 (at most 18 significant bits, so m s stays exact too). W is
+// read twice on this path.
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
@@ -28,12 +35,34 @@
 namespace wr {
 namespace {
 
-constexpr int kQWarps = 8;   // units per CTA
+constexpr int kQWarps = 8;   // units (rows, for the row pass) per CTA
 
-template <int BITS>
+// Row pass of the int8 form: d[n] = fp16(max_k |w[n,k]| / (127 L)), saturated to 65504.
+__global__ void __launch_bounds__(32 * kQWarps) row_scale_kernel(const float* __restrict__ w, int N, int K, int L,
+                                                                 uint16_t* __restrict__ d) {
+  const int lane = threadIdx.x & 31;
+  const int64_t n = (int64_t)blockIdx.x * kQWarps + (threadIdx.x >> 5);
+  if (n >= N) return;   // whole warps leave together
+  const float4* src = reinterpret_cast<const float4*>(w + n * (int64_t)K);
+  float am = 0.f;
+  for (int i = lane; i < K / 4; i += 32) {
+    const float4 f = __ldg(src + i);
+    am = fmaxf(am, fmaxf(fmaxf(fabsf(f.x), fabsf(f.y)), fmaxf(fabsf(f.z), fabsf(f.w))));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
+  if (lane == 0) {
+    uint16_t h = __half_as_ushort(__double2half((double)am / (double)(127 * L)));
+    if ((h & 0x7FFFu) >= 0x7C00u) h = 0x7BFFu;
+    d[n] = h;
+  }
+}
+
+template <int BITS, bool S8>
 __global__ void __launch_bounds__(32 * kQWarps) quantize_pack_kernel(const float* __restrict__ w, int N, int K,
                                                                     int B, int64_t U, uint8_t* __restrict__ packed,
-                                                                    uint16_t* __restrict__ scales) {
+                                                                    uint16_t* __restrict__ scales,
+                                                                    int8_t* __restrict__ scale_q) {
   constexpr int L = (1 << BITS) - 1;
   constexpr int UB = BITS == 2 ? 1024 : 1536;
   const int lane = threadIdx.x & 31;
@@ -72,9 +101,19 @@ __global__ void __launch_bounds__(32 * kQWarps) quantize_pack_kernel(const float
     for (int i = 0; i < 64; ++i) am = fmaxf(am, fabsf(v[i]));
     am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 1));
     am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 2));
-    const __half sh = __double2half((double)am / (double)L);
-    const float s = __half2float(sh);
-    if (real && q == 0) scales[n * (int64_t)B + ub] = __half_as_ushort(sh);
+    float s;
+    if (S8) {
+      // d was written by the row pass (an earlier launch on the same stream)
+      const double d = real ? (double)__half2float(__ushort_as_half(scales[n])) : 0.0;
+      double qv = d > 0.0 ? rint((double)am / ((double)L * d)) : 0.0;
+      qv = fmin(127.0, fmax(0.0, qv));
+      if (real && q == 0) scale_q[n * (int64_t)B + ub] = (int8_t)qv;
+      s = (float)(d * qv);
+    } else {
+      const __half sh = __double2half((double)am / (double)L);
+      s = __half2float(sh);
+      if (real && q == 0) scales[n * (int64_t)B + ub] = __half_as_ushort(sh);
+    }
     const bool unit_level = !(s > 0.f) || isinf(s);   // s = 0 or inf: level +1
     // code of weight i (pad rows: code 0)
     auto code = [&](int i) -> uint32_t {
@@ -126,12 +165,19 @@ __global__ void __launch_bounds__(32 * kQWarps) quantize_pack_kernel(const float
 }  // namespace
 
 cudaError_t launch_quantize_pack(int bits, const float* w, int N, int K, uint8_t* packed, uint16_t* scales,
-                                 cudaStream_t stream) {
+                                 int8_t* scale_q, cudaStream_t stream) {
   const int B = K / 256;
   const int64_t U = (int64_t)((N + 15) / 16) * B;
   const unsigned ctas = (unsigned)((U + kQWarps - 1) / kQWarps);
-  if (bits == 2) quantize_pack_kernel<2><<<ctas, 32 * kQWarps, 0, stream>>>(w, N, K, B, U, packed, scales);
-  else quantize_pack_kernel<3><<<ctas, 32 * kQWarps, 0, stream>>>(w, N, K, B, U, packed, scales);
+  constexpr int th = 32 * kQWarps;
+  if (scale_q != nullptr) {
+    row_scale_kernel<<<(unsigned)((N + kQWarps - 1) / kQWarps), th, 0, stream>>>(w, N, K, (1 << bits) - 1, scales);
+    if (bits == 2) quantize_pack_kernel<2, true><<<ctas, th, 0, stream>>>(w, N, K, B, U, packed, scales, scale_q);
+    else quantize_pack_kernel<3, true><<<ctas, th, 0, stream>>>(w, N, K, B, U, packed, scales, scale_q);
+  } else {
+    if (bits == 2) quantize_pack_kernel<2, false><<<ctas, th, 0, stream>>>(w, N, K, B, U, packed, scales, nullptr);
+    else quantize_pack_kernel<3, false><<<ctas, th, 0, stream>>>(w, N, K, B, U, packed, scales, nullptr);
+  }
   return cudaGetLastError();
 }
 

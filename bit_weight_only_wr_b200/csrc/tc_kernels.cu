@@ -1,6 +1,6 @@
 // Packed-code GEMV/GEMM on tcgen05 tensor cores (sm_100a).
 //
-//   y[m,n] = sum_b s[n,b] sum_{k in b} g[n,k] x[m,k]         (2/3-bit odd grid, fp16 scales)
+//   y[m,n] = sum_b s[n,b] sum_{k in b} g[n,k] x[m,k]         (2/3-bit odd grid, fp16 or int8 scales)
 //   y[m,n] = alpha[n] sum_k t[n,k] (R x[m,:])[k]             (ternary, rotated basis)
 //
 // One CTA owns 128 weight rows ("row group") at a time; the MMA is D[128 x BN] += A[128 x 16]
@@ -395,7 +395,12 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const TcArgs a, const _
         if (lane == 0) mbar_arrive(&bars->d_empty[dbuf]);
       } else {
         const uint32_t dbuf = gb & 1;
-        const float s2 = n < a.N ? 2.f * half_bits_to_float(__ldg(a.scales + (int64_t)n * a.B + ps_.b)) : 0.f;
+        // 2 s: the fp16 block scale, or d_n q[n,b] (exact in fp32)
+        const float s2 = n >= a.N ? 0.f
+                         : a.scale_q == nullptr
+                             ? 2.f * half_bits_to_float(__ldg(a.scales + (int64_t)n * a.B + ps_.b))
+                             : 2.f * half_bits_to_float(__ldg(a.scales + n)) *
+                                   (float)__ldg(a.scale_q + (int64_t)n * a.B + ps_.b);
         if (!(ok = mbar_wait(&bars->d_full[dbuf], (gb >> 1) & 1, abort_flag, a.err, 402))) break;
         fence_after_sync();
 #pragma unroll

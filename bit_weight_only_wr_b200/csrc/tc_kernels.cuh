@@ -7,7 +7,8 @@ namespace wr {
 
 struct TcArgs {
   const uint8_t* packed;     // packed units, tile-major
-  const uint16_t* scales;    // fp16 [N, K/256] (Q2/Q3)
+  const uint16_t* scales;    // fp16 [N, K/256] (Q2/Q3), or fp16 [N] row scales d with scale_q
+  const int8_t* scale_q;     // int8 [N, K/256] block multipliers (s = d q), or null: fp16 scales
   const uint16_t* alpha;     // fp16 [N] (ternary)
   float* y;                  // fp32 [M, N]
   float* partial;            // pieces of tiles cut by range ends [grid][2][TOK][128]
@@ -27,7 +28,8 @@ struct DecProblem {
   const uint16_t* x;         // bf16 [M, K] activations (Q2/Q3; read by the preparation pass)
   uint8_t* xt;               // prepared activation tiles of this problem (workspace), one per block
   const uint8_t* packed;     // packed units, tile-major
-  const uint16_t* scales;    // fp16 [N, K/256] (Q2/Q3) or alpha [N] (ternary)
+  const uint16_t* scales;    // fp16 [N, K/256] (Q2/Q3) or alpha [N] (ternary); d [N] with scale_q
+  const int8_t* scale_q;     // int8 [N, K/256] block multipliers (s = d q), or null: fp16 scales
   float* y;                  // fp32 [M, N]
   int N, K, Kp;              // Kp: padded K of the ternary planes
   int B, RG, P, bits;        // blocks per row, 128-row groups, K splits, 2/3 (ternary: 1)
@@ -81,12 +83,16 @@ cudaError_t launch_rotate_x(const uint16_t* x, const uint32_t* signs, uint8_t* x
 cudaError_t launch_rotate_planes(const uint16_t* x, const uint32_t* signs, uint8_t* planes, int M, int K, int64_t Kp,
                                  cudaStream_t stream);
 cudaError_t launch_rotate_x_batched(const DecArgs& a, int64_t total_items, cudaStream_t stream);
-// Device quantizer + packer for the 2/3-bit odd grid (quantize.cu).
+// Device quantizer + packer for the 2/3-bit odd grid (quantize.cu). scale_q null: fp16 block
+// scales [N, K/256] in `scales`; else the int8 form: fp16 row scales d [N] in `scales` and the
+// int8 multipliers [N, K/256] in scale_q.
 cudaError_t launch_quantize_pack(int bits, const float* w, int N, int K, uint8_t* packed, uint16_t* scales,
-                                 cudaStream_t stream);
+                                 int8_t* scale_q, cudaStream_t stream);
 // Failure-path self-test: a bounded wait on a barrier that never completes (see wr.h).
 cudaError_t launch_selftest_wait_timeout(int* err_word, cudaStream_t stream);
-cudaError_t launch_unpack_bf16(int fmt, const uint8_t* packed, const uint16_t* scales, int N, int K, int units,
-                               uint16_t* w, cudaStream_t stream);
+// scales: fp16 [N, K/256] (alpha [N] for ternary), or the fp16 row scales d when scale_q (int8
+// [N, K/256] multipliers) is not null.
+cudaError_t launch_unpack_bf16(int fmt, const uint8_t* packed, const uint16_t* scales, const int8_t* scale_q, int N,
+                               int K, int units, uint16_t* w, cudaStream_t stream);
 
 }  // namespace wr

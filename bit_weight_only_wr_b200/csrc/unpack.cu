@@ -2,8 +2,9 @@
 //
 // The "Qwen3-4B-Wringer-Q2.6" card ("What is in this repo") describes a materializer that
 // expands the container into a bf16 checkpoint, bit-identical across independent re-runs.
-// Here W[n,k] = bf16_RNE(s * g): the fp32 product of an fp16 scale (11 significant bits)
-// and a grid integer (at most 3 bits) is exact, so the one rounding to bf16 is the only one.
+// Here W[n,k] = bf16_RNE(s * g): the fp32 product of an fp16 scale (11 significant bits; 18 for
+// the int8 form d q) and a grid integer (at most 3 bits) is exact, so the one rounding to bf16
+// is the only one.
 // One warp per packed unit; each lane expands its 64 codes (80 trits) of two rows into shared
 // memory, and the warp writes the unit out in whole-row segments. The kernel is bound by the
 // 2 bytes/weight it writes.
@@ -39,7 +40,8 @@ struct UnpackGeom {
 // 128-byte lines.
 template <int FMT>
 __global__ void __launch_bounds__(32 * kUnpackWarps) unpack_kernel(const uint8_t* __restrict__ packed,
-                                                                  const uint16_t* __restrict__ scales, int N,
+                                                                  const uint16_t* __restrict__ scales,
+                                                                  const int8_t* __restrict__ scale_q, int N,
                                                                   int K, int B, int64_t U,
                                                                   uint16_t* __restrict__ out) {
   using G = UnpackGeom<FMT>;
@@ -96,7 +98,10 @@ __global__ void __launch_bounds__(32 * kUnpackWarps) unpack_kernel(const uint8_t
         srow[10 * q + i] = w;
       }
     } else {
-      const float s = n < N ? half_bits_to_float(scales[n * B + ub]) : 0.f;
+      // the fp16 block scale, or d_n q[n,b]: exact in fp32, so s * g stays exact
+      const float s = n >= N ? 0.f
+                      : scale_q == nullptr ? half_bits_to_float(scales[n * B + ub])
+                                           : half_bits_to_float(scales[n]) * (float)scale_q[n * B + ub];
       const int L = FMT == WR_FMT_Q2 ? 3 : 7;
       int c[64];
       if (FMT == WR_FMT_Q2 || FMT == WR_FMT_T2) {
@@ -171,16 +176,16 @@ __global__ void __launch_bounds__(32 * kUnpackWarps) unpack_kernel(const uint8_t
 
 }  // namespace
 
-cudaError_t launch_unpack_bf16(int fmt, const uint8_t* packed, const uint16_t* scales, int N, int K,
-                               int units, uint16_t* w, cudaStream_t stream) {
+cudaError_t launch_unpack_bf16(int fmt, const uint8_t* packed, const uint16_t* scales, const int8_t* scale_q, int N,
+                               int K, int units, uint16_t* w, cudaStream_t stream) {
   const int64_t tiles = (N + 15) / 16;
   const int64_t U = tiles * units;
   const unsigned ctas = (unsigned)((U + kUnpackWarps - 1) / kUnpackWarps);
   constexpr int th = 32 * kUnpackWarps;
-  if (fmt == WR_FMT_Q2) unpack_kernel<WR_FMT_Q2><<<ctas, th, 0, stream>>>(packed, scales, N, K, units, U, w);
-  else if (fmt == WR_FMT_Q3) unpack_kernel<WR_FMT_Q3><<<ctas, th, 0, stream>>>(packed, scales, N, K, units, U, w);
-  else if (fmt == WR_FMT_T2) unpack_kernel<WR_FMT_T2><<<ctas, th, 0, stream>>>(packed, scales, N, K, units, U, w);
-  else unpack_kernel<WR_FMT_TERNARY><<<ctas, th, 0, stream>>>(packed, scales, N, K, units, U, w);
+  if (fmt == WR_FMT_Q2) unpack_kernel<WR_FMT_Q2><<<ctas, th, 0, stream>>>(packed, scales, scale_q, N, K, units, U, w);
+  else if (fmt == WR_FMT_Q3) unpack_kernel<WR_FMT_Q3><<<ctas, th, 0, stream>>>(packed, scales, scale_q, N, K, units, U, w);
+  else if (fmt == WR_FMT_T2) unpack_kernel<WR_FMT_T2><<<ctas, th, 0, stream>>>(packed, scales, scale_q, N, K, units, U, w);
+  else unpack_kernel<WR_FMT_TERNARY><<<ctas, th, 0, stream>>>(packed, scales, nullptr, N, K, units, U, w);
   return cudaGetLastError();
 }
 

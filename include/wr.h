@@ -97,6 +97,28 @@ enum { WR_FMT_TERNARY = 1, WR_FMT_Q2 = 2, WR_FMT_Q3 = 3, WR_FMT_T2 = 4 };
  * decode GEMV (wr_gemv, wr_gemv_batched, wr_gemv_noalloc with bits = WR_FMT_T2) and
  * wr_unpack_bf16 accept it; the prefill GEMM (M > 8) does not (WR_ERR_UNSUPPORTED). */
 
+/* Int8 block scales (the "Agents-A1-4B-Wringer-Q2.6" card, "What is in this repo": a container
+ * of packed codes with fp16 or int8 block scales). WR_SCALES_I8 is OR'd into the format code
+ * (the `bits` or `fmt` argument, or wr_gemv_problem.bits) of Q2, Q3 and T2; the codes and their
+ * packed bytes are unchanged, only the `scales` argument changes meaning: it points to a scale
+ * record of wr_scales_bytes() bytes,
+ *     bytes [0, 2N)          d: fp16 [N], one scale per row,
+ *     bytes [R, R + N*K/256) q: int8 [N, K/256] row-major, values 0..127, R = 16*ceil(2N/16),
+ * and the block scale is s[n,b] = d[n] * q[n,b], formed exactly in fp32 (at most 11 + 7
+ * significant bits), after which every call computes what it computes with fp16 scales s.
+ * wr_quantize(bits | WR_SCALES_I8, ...) writes such a record: d_n = fp16(max_k |w[n,k]| /
+ * (127 L)) (fp64 division, one rounding, saturated to 65504), q = the integer nearest to
+ * absmax_b / (L d_n) (ties to even) clamped to [0, 127] (0 where d_n = 0). Accepted by
+ * wr_quantize, wr_quantize_pack, wr_unpack_bf16, wr_gemv, wr_gemv_noalloc, wr_gemv_batched,
+ * wr_gemm and their *_workspace_bytes; wr_packed_bytes, wr_pack and wr_unpack_codes take the
+ * format without it. Scales: 8 bits per 256 weights plus 16 bits per row, instead of 16 per
+ * 256 weights. */
+enum { WR_SCALES_I8 = 0x100 };
+
+/* Bytes of the scale buffer of an N x K matrix: fp16 [N, K/256] for Q2/Q3/T2, fp16 [N] for
+ * ternary, the record above with WR_SCALES_I8; 0 on bad arguments. */
+size_t wr_scales_bytes(int fmt, int64_t N, int64_t K);
+
 /* Version of this ABI (incremented on any incompatible change). */
 int wr_abi_version(void);
 
@@ -124,6 +146,8 @@ wr_status wr_unpack_codes(int fmt, int64_t N, int64_t K, const uint8_t* packed_h
  * w_host fp32 [N,K]; codes_host uint8 [N,K]; scales_host fp16 bits [N, K/256]. */
 wr_status wr_quantize(int bits, int64_t N, int64_t K, const float* w_host, uint8_t* codes_host,
                       uint16_t* scales_host);
+/* (With bits | WR_SCALES_I8, scales_host receives the int8 scale record described above and
+ * the codes are chosen against s = d q.) */
 
 /* Device quantizer + packer for the 2/3-bit odd grid: computes on the GPU exactly what
  * wr_quantize followed by wr_pack computes on the host (bit-identical scales and packed bytes),
@@ -168,10 +192,10 @@ wr_status wr_gemv(int64_t M, int64_t N, int64_t K, const uint16_t* x, const void
 typedef struct {
   const uint16_t* x;       /* bf16 [M, K] activations (device) */
   const void* packed;      /* packed codes (device), format Q2 or Q3 as given by bits */
-  const uint16_t* scales;  /* fp16 [N, K/256] block scales (device) */
+  const uint16_t* scales;  /* fp16 [N, K/256] block scales, or the int8 scale record (device) */
   float* y;                /* fp32 [M, N] output (device, overwritten) */
   int64_t N, K;            /* K % 256 == 0 */
-  int32_t bits;            /* 2 or 3 */
+  int32_t bits;            /* 2, 3 or WR_FMT_T2, optionally | WR_SCALES_I8 */
   int32_t reserved;        /* must be 0 */
 } wr_gemv_problem;
 

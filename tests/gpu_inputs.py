@@ -41,6 +41,32 @@ def t_case(wr, N, K, seed):
     return codes_o, alpha_o, signs, dev(packed), dev(alpha), dev(signs)
 
 
+def s8_record(d, q):
+    """Int8 scale record of include/wr.h from d (fp16 [N]) and q (int8 [N, B]): d at byte 0,
+    q from byte 16 * ceil(2N / 16)."""
+    d = np.asarray(d, dtype=np.float16)
+    q = np.ascontiguousarray(q, dtype=np.int8)
+    N = d.shape[0]
+    off = (2 * N + 15) // 16 * 16
+    rec = np.zeros(max(off + q.size, 16), dtype=np.uint8)
+    rec[:2 * N] = d.view(np.uint8)
+    rec[off:off + q.size] = q.reshape(-1).view(np.uint8)
+    return rec
+
+
+def s8_case(wr, bits, N, K, seed, W=None):
+    """Codes with int8 block scales: the library's quantizer checked against the oracle's;
+    returns (codes, d, q, packed on the device, scale record on the device)."""
+    if W is None:
+        W = wr_synth.weights_fp32(seed, N, K)
+    fmt = bits | wr.WR_SCALES_I8
+    codes, rec = wr.wr_quantize(fmt, W)
+    codes_o, d_o, q_o = o.quantize_odd_grid_s8(W, bits)
+    nrec = wr.wr_scales_bytes(fmt, N, K)
+    assert np.array_equal(codes, codes_o) and np.array_equal(rec[:nrec], s8_record(d_o, q_o)[:nrec])
+    return codes_o, d_o, q_o, dev(wr.wr_pack(bits, codes)), dev(rec)
+
+
 def check_close(y_gpu: np.ndarray, y_ref: np.ndarray, bound: np.ndarray, rel: float = 1e-4):
     """Per element |y_gpu - y_ref| <= rel * sum_k |w x|; exact zero where the bound is zero."""
     err = np.abs(y_gpu.astype(np.float64) - y_ref)

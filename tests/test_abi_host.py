@@ -11,6 +11,7 @@ import pytest
 import bit_weight_only_wr_b200 as wr
 import wr_synth
 from oracle import wr_oracle as o
+from gpu_inputs import s8_record
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
@@ -79,6 +80,34 @@ def test_quantizer_matches_oracle(bits):
     assert np.array_equal(c1, c2)
 
 
+@pytest.mark.parametrize("bits", [2, 3])
+@pytest.mark.parametrize("N,K", [(64, 1024), (7, 256), (33, 2560)])
+def test_s8_quantizer_matches_oracle(bits, N, K):
+    """Int8 block scales: the library's quantizer writes the oracle's d, q and codes, bit for bit."""
+    W = wr_synth.weights_fp32(200 + bits + N, N, K)
+    W[min(3, N - 1), :256] = 0.0                          # an all-zero block (q = 0)
+    if N > 5:
+        W[5] *= np.float32(1e-30)                         # d subnormal in fp16 (or zero)
+        W[4, 7] = 3.0e9                                   # d saturates at 65504
+    fmt = bits | wr.WR_SCALES_I8
+    assert wr.wr_scales_bytes(fmt, N, K) == (2 * N + 15) // 16 * 16 + N * (K // 256)
+    c1, rec = wr.wr_quantize(fmt, W)
+    c2, d, q = o.quantize_odd_grid_s8(W, bits)
+    assert np.array_equal(rec[:wr.wr_scales_bytes(fmt, N, K)], s8_record(d, q)[:wr.wr_scales_bytes(fmt, N, K)])
+    assert np.array_equal(c1, c2)
+
+
+def test_scales_bytes():
+    assert wr.wr_scales_bytes(2, 16, 512) == 2 * 16 * 2
+    assert wr.wr_scales_bytes(3 | wr.WR_SCALES_I8, 16, 512) == 32 + 16 * 2
+    assert wr.wr_scales_bytes(wr.WR_FMT_T2 | wr.WR_SCALES_I8, 9, 256) == 32 + 9
+    assert wr.wr_scales_bytes(1, 10, 300) == 20                 # ternary alpha [N]
+    assert wr.wr_scales_bytes(1 | wr.WR_SCALES_I8, 10, 300) == 0
+    assert wr.wr_scales_bytes(2, 16, 100) == 0
+    # packed codes do not depend on the scale form: the packer takes the base format
+    assert wr.wr_packed_bytes(2 | wr.WR_SCALES_I8, 16, 256) == 0
+
+
 def test_trellis_quantizer_matches_oracle():
     """The library's Viterbi encoder for the 2-bit trellis format picks the oracle's symbols
     and scales, bit for bit (same fp64 arithmetic, same tie order)."""
@@ -141,5 +170,18 @@ def test_device_calls_reject_bad_arguments_before_launch():
     assert st == 1
     st = wr._lib.wr_unpack_bf16(2, 16, 256, 16, 16, 64, 16, None)                 # group
     assert st == 2
+    i8 = wr.WR_SCALES_I8
+    st = wr._lib.wr_gemv(1, 16, 256, 16, 16, 16, 5 | i8, 256, 16, 16, 1 << 20, None)   # bits
+    assert st == 2
+    st = wr._lib.wr_gemm(16, 16, 256, 16, 16, 16, 4 | i8, 256, 16, 16, 1 << 20, None)  # trellis, M > 8
+    assert st == 2
+    st = wr._lib.wr_gemv(1, 16, 256, 16, 16, 8, 2 | i8, 256, 16, 16, 1 << 20, None)    # misaligned record
+    assert st == 1
+    st = wr._lib.wr_unpack_bf16(1 | i8, 16, 320, 16, 16, 256, 16, None)           # ternary has no int8 form
+    assert st == 2
+    st = wr._lib.wr_quantize_pack(wr.WR_FMT_T2 | i8, 16, 256, 16, 16, 16, None)
+    assert st == 2
+    assert wr.wr_gemv_workspace_bytes(1, 16, 256, 3 | i8) == wr.wr_gemv_workspace_bytes(1, 16, 256, 3)
+    assert wr.wr_gemm_workspace_bytes(64, 16, 256, 2 | i8) == wr.wr_gemm_workspace_bytes(64, 16, 256, 2)
     assert wr.wr_gemv_workspace_bytes(9, 16, 256, 2) == 0
     assert wr.wr_gemv_workspace_bytes(1, 16, 256, 2) > 0
