@@ -82,6 +82,7 @@ constexpr int kDecodeTokens = 8;   // decode kernel: 8 tokens x 4 activation lim
 struct DecodePlan {
   wr::DecArgs args;
   int total_blocks = 0;
+  int grid = 0;   // 2/3-bit: CTAs (block ranges) of the decode launch
   size_t counter_off = 0, partial_off = 0, xt_off = 0, total = 0;
   int64_t xt_rel[wr::kMaxDecodeProblems];
 };
@@ -113,7 +114,7 @@ void plan_decode(int64_t M, int count, const ProblemShape* shapes, DecodePlan* d
   const double bpi = (double)total_blocks / (double)target_items;
   const bool ternary = count > 0 && shapes[0].fmt == WR_FMT_TERNARY;
   int items = 0, counters = 0, blocks = 0;
-  int64_t partials = 0, xt_bytes = 0, block_base = 0;
+  int64_t partials = 0, xt_bytes = 0, block_base = 0, cost_base = 0;
   for (int i = 0; i < count; ++i) {
     wr::DecProblem& pr = a.prob[i];
     int P = (int)std::lround((double)pr.B / bpi);
@@ -123,18 +124,23 @@ void plan_decode(int64_t M, int count, const ProblemShape* shapes, DecodePlan* d
     pr.partial_base = partials;
     pr.xblk_base = blocks;
     pr.block_base = block_base;
+    pr.cost_base = cost_base;
     items += pr.RG * pr.P;
     counters += pr.RG;
     blocks += pr.B;
     block_base += (int64_t)pr.RG * pr.B;
+    if (!ternary) cost_base += (int64_t)pr.RG * pr.B * wr::block_cost(pr.bits);
     if (ternary && pr.P > 1) partials += (int64_t)pr.RG * pr.P * M * 128;
     dp->xt_rel[i] = xt_bytes;
     xt_bytes += (int64_t)pr.B * wr::xtile_bytes(ternary, (int)M);
   }
   a.items = items;
   a.total = block_base;
-  // 2/3-bit: two partial slots per CTA of the launch (see DecArgs)
-  if (!ternary) partials = 2 * std::min<int64_t>(kDecodeGrid, block_base) * M * 128;
+  a.total_cost = cost_base;
+  // 2/3-bit: ranges of at least the largest block cost, so that each holds a block; two partial
+  // slots per CTA of the launch (see DecArgs)
+  dp->grid = (int)std::max<int64_t>(1, std::min<int64_t>(kDecodeGrid, cost_base / wr::block_cost(3)));
+  if (!ternary) partials = 2 * (int64_t)dp->grid * M * 128;
   dp->total_blocks = blocks;
   dp->counter_off = 0;
   dp->partial_off = align256((size_t)counters * sizeof(int));
@@ -160,9 +166,8 @@ wr_status run_decode(DecodePlan& dp, bool ternary, cudaStream_t stream) {
     return wr::launch_gemv_t(dp.args, grid, stream) == cudaSuccess ? WR_OK : WR_ERR_CUDA;
   }
   // one contiguous block range per CTA; the partial slots were sized for this grid
-  const int grid = (int)std::min<int64_t>(dp.args.total, kDecodeGrid);
   if (wr::launch_prep_x(dp.args, dp.total_blocks, stream) != cudaSuccess) return WR_ERR_CUDA;
-  return wr::launch_gemv_q(dp.args, grid, stream) == cudaSuccess ? WR_OK : WR_ERR_CUDA;
+  return wr::launch_gemv_q(dp.args, dp.grid, stream) == cudaSuccess ? WR_OK : WR_ERR_CUDA;
 }
 
 // ---- prefill GEMM kernel (M > 8): 128-row groups x token tiles x K blocks, cut "stream-K" into

@@ -31,25 +31,33 @@ struct DecProblem {
   const uint16_t* scales;    // fp16 [N, K/256] (Q2/Q3) or alpha [N] (ternary); d [N] with scale_q
   const int8_t* scale_q;     // int8 [N, K/256] block multipliers (s = d q), or null: fp16 scales
   float* y;                  // fp32 [M, N]
+  const uint32_t* signs;     // ternary: random-sign mask of the rotation
+  int64_t partial_base;      // first partial float of this problem (ternary items)
+  int64_t block_base;        // first block of this problem in the batch's block sequence (2/3-bit)
+  int64_t cost_base;         // cost (block_cost units) of the batch's blocks before this problem
   int N, K, Kp;              // Kp: padded K of the ternary planes
-  int B, RG, P, bits;        // blocks per row, 128-row groups, K splits, 2/3 (ternary: 1)
+  int B, RG, P, bits;        // blocks per row, 128-row groups, K splits, 2/3/T2 (ternary: 1)
   int item_base;             // first work item of this problem
   int xblk_base;             // 2/3-bit: first block of this problem in the preparation pass;
                              // ternary: first rotation work item (token, 128-block) of it
-  const uint32_t* signs;     // ternary: random-sign mask of the rotation
   int counter_base;          // first arrival counter (row group) of this problem
-  int64_t partial_base;      // first partial float of this problem (ternary items)
-  int64_t block_base;        // first block of this problem in the batch's block sequence (2/3-bit)
 };
 
+// Relative decode-GEMV time of one 128 x 256 block, by format: a 3-bit (or trellis) block takes
+// about 1.3 times a 2-bit one (its weights are 1.5 times the bytes, its decode is longer). The
+// block ranges of the CTAs are cut by this cost so that they finish together.
+__host__ __device__ inline int64_t block_cost(int bits) { return bits == 2 ? 10 : 13; }
+
 // 2/3-bit: the batch's blocks (problem by problem, row group by row group, K block by K block)
-// are cut into gridDim.x contiguous ranges, one per CTA: CTA c takes [c T / G, (c+1) T / G).
+// are cut into gridDim.x contiguous ranges, one per CTA: CTA c takes the blocks whose cost
+// before them (in block_cost units) lies in [c C / G, (c+1) C / G).
 // A row group cut by a range boundary is finished through per-CTA partial slots (two per CTA:
 // the row group that started before the range, and the one that ends after it).
 // Ternary: work items (problem, row group, range of blocks), items c, c + G, ... per CTA.
 struct DecArgs {
   int count, M, items, pad;
   int64_t total;             // 2/3-bit: blocks of the batch (T)
+  int64_t total_cost;        // 2/3-bit: their summed block_cost (C)
   float* partial;
   int* counter;
   int* err;
