@@ -138,9 +138,9 @@ def module_bytes(wr, M, N, K, bits):
 # DRAM traffic of the decode GEMV launch, (dram__bytes_read + dram__bytes_write) / algorithmic
 # bytes, from one ncu capture of the current kernel at that token count (summary and command in
 # profiles/). None: no capture of this kernel version, so no traffic figure is claimed.
-# current kernel: M = 1 reads 1,207,574,272 and writes 7,993,088 bytes for 1,178,984,448
-# algorithmic; M = 8 reads 1,329,226,752 and writes 39,346,432 for 1,223,368,704
-_TRAFFIC_RATIO = {1: (1_208_125_184 + 7_661_568) / 1_178_984_448, 8: (1_328_882_944 + 39_116_544) / 1_223_368_704}
+# current kernel: M = 1 reads 1,205,202,688 and writes 7,539,968 bytes for 1,178,984,448
+# algorithmic; M = 8 reads 1,320,538,624 and writes 40,161,024 for 1,223,368,704
+_TRAFFIC_RATIO = {1: (1_205_202_688 + 7_539_968) / 1_178_984_448, 8: (1_320_538_624 + 40_161_024) / 1_223_368_704}
 
 
 def traffic_per_launch(M: int, layers: int, algo_bytes: int):

@@ -129,7 +129,7 @@ void plan_decode(int64_t M, int count, const ProblemShape* shapes, DecodePlan* d
     counters += pr.RG;
     blocks += pr.B;
     block_base += (int64_t)pr.RG * pr.B;
-    if (!ternary) cost_base += (int64_t)pr.RG * pr.B * wr::block_cost(pr.bits);
+    if (!ternary) cost_base += (int64_t)pr.RG * pr.B * wr::block_cost(pr.bits, (int)M);
     if (ternary && pr.P > 1) partials += (int64_t)pr.RG * pr.P * M * 128;
     dp->xt_rel[i] = xt_bytes;
     xt_bytes += (int64_t)pr.B * wr::xtile_bytes(ternary, (int)M);
@@ -139,7 +139,7 @@ void plan_decode(int64_t M, int count, const ProblemShape* shapes, DecodePlan* d
   a.total_cost = cost_base;
   // 2/3-bit: ranges of at least the largest block cost, so that each holds a block; two partial
   // slots per CTA of the launch (see DecArgs)
-  dp->grid = (int)std::max<int64_t>(1, std::min<int64_t>(kDecodeGrid, cost_base / wr::block_cost(3)));
+  dp->grid = (int)std::max<int64_t>(1, std::min<int64_t>(kDecodeGrid, cost_base / wr::block_cost(3, (int)M)));
   if (!ternary) partials = 2 * (int64_t)dp->grid * M * 128;
   dp->total_blocks = blocks;
   dp->counter_off = 0;

@@ -106,8 +106,8 @@ struct Pos {
 // it is at least that. The host sizes the grid so that every range holds at least one block.
 __device__ __forceinline__ int64_t cost_start(const DecArgs& a, int c) { return (int64_t)c * a.total_cost / gridDim.x; }
 // First block at or after cost position cs, for a cs inside problem pr (or at its end)
-__device__ __forceinline__ int64_t range_start_in(const DecProblem& pr, int64_t cs) {
-  const int64_t w = block_cost(pr.bits), d = cs - pr.cost_base;
+__device__ __forceinline__ int64_t range_start_in(const DecProblem& pr, int M, int64_t cs) {
+  const int64_t w = block_cost(pr.bits, M), d = cs - pr.cost_base;
   return pr.block_base + (d > 0 ? (d + w - 1) / w : 0);
 }
 __device__ __forceinline__ int64_t range_start(const DecArgs& a, int c) {
@@ -118,12 +118,12 @@ __device__ __forceinline__ int64_t range_start(const DecArgs& a, int c) {
     if (a.prob[mid].cost_base <= cs) lo = mid;
     else hi = mid - 1;
   }
-  return range_start_in(a.prob[lo], cs);
+  return range_start_in(a.prob[lo], a.M, cs);
 }
 // CTA whose range holds global block g of problem pr: the largest c with cost_start(c) <= the
 // cost before g
 __device__ __forceinline__ int cta_of(const DecArgs& a, const DecProblem& pr, int64_t g) {
-  const int64_t x = pr.cost_base + (g - pr.block_base) * block_cost(pr.bits);
+  const int64_t x = pr.cost_base + (g - pr.block_base) * block_cost(pr.bits, a.M);
   return (int)(((x + 1) * gridDim.x - 1) / a.total_cost);
 }
 
@@ -497,7 +497,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_q_kernel(const __gr
           }
         } else {
           // slot 0: the row group began before this range; slot 1: it continues after it
-          const int slot = g0 < range_start_in(pr, cost_start(a, blockIdx.x)) ? 0 : 1;
+          const int slot = g0 < range_start_in(pr, M, cost_start(a, blockIdx.x)) ? 0 : 1;
           float* part = a.partial + ((int64_t)2 * blockIdx.x + slot) * M * 128;
 #pragma unroll
           for (int m = 0; m < kSlots; ++m)
@@ -511,7 +511,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_q_kernel(const __gr
 #pragma unroll
             for (int m = 0; m < kSlots; ++m) acc[m] = 0.f;
             for (int c = c0; c <= c1; ++c) {
-              const int sl = g0 < range_start_in(pr, cost_start(a, c)) ? 0 : 1;
+              const int sl = g0 < range_start_in(pr, M, cost_start(a, c)) ? 0 : 1;
               const float* src = a.partial + ((int64_t)2 * c + sl) * M * 128;
 #pragma unroll
               for (int m = 0; m < kSlots; ++m)

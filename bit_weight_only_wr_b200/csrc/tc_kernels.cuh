@@ -43,10 +43,14 @@ struct DecProblem {
   int counter_base;          // first arrival counter (row group) of this problem
 };
 
-// Relative decode-GEMV time of one 128 x 256 block, by format: a 3-bit (or trellis) block takes
-// about 1.3 times a 2-bit one (its weights are 1.5 times the bytes, its decode is longer). The
-// block ranges of the CTAs are cut by this cost so that they finish together.
-__host__ __device__ inline int64_t block_cost(int bits) { return bits == 2 ? 10 : 13; }
+// Relative decode-GEMV time of one 128 x 256 block, by format and token count: a 3-bit (or
+// trellis) block takes about 1.3 times a 2-bit one at M <= 2 and 1.2 times at M = 8 (its weights
+// are 1.5 times the bytes and its decode is longer; the per-block work that does not depend on
+// the format grows with M). The block ranges of the CTAs are cut by this cost so that they
+// finish together; the ratios are the best of a sweep on the 36-layer body.
+__host__ __device__ inline int64_t block_cost(int bits, int M) {
+  return bits == 2 ? 20 : (M <= 2 ? 26 : (M <= 4 ? 25 : 24));
+}
 
 // 2/3-bit: the batch's blocks (problem by problem, row group by row group, K block by K block)
 // are cut into gridDim.x contiguous ranges, one per CTA: CTA c takes the blocks whose cost
