@@ -173,16 +173,18 @@ wr_status wr_quantize_ternary(int64_t N, int64_t K, const float* w_host,
                               const uint32_t* sign_bits_host, uint8_t* codes_host,
                               uint16_t* alpha_host);
 
-/* Device materializer: w_bf16 [N,K] = bf16_RNE(s * g) for Q2/Q3 (group must be 256), or
- * bf16_RNE(alpha_n * t) for ternary (scales = alpha [N], group ignored; the result is in
- * the rotated basis). Bit-exact; the bf16 checkpoint the "Qwen3-4B-Wringer-Q2.6" card's
- * materializer produces from the container. */
+/* Device materializer: w_bf16 [N,K] = bf16_RNE(s * g) for Q2, Q3 and T2, optionally
+ * | WR_SCALES_I8 (group must be 256), or bf16_RNE(alpha_n * t) for ternary (scales = alpha [N],
+ * group ignored; the result is in the rotated basis). Bit-exact; the bf16 checkpoint the
+ * "Qwen3-4B-Wringer-Q2.6" card's materializer produces from the container. */
 wr_status wr_unpack_bf16(int fmt, int64_t N, int64_t K, const void* packed, const uint16_t* scales,
                          int group, uint16_t* w_bf16, void* stream);
 
-/* Decode GEMV for 1 <= M <= 8 (Q2/Q3, group 256): streams the packed codes once, decodes
- * them in registers and contracts them on tensor cores. Splits K across warps and combines
- * the pieces through the workspace (deterministic summation order). */
+/* Decode GEMV for 1 <= M <= 8 (bits = 2, 3 or WR_FMT_T2, optionally | WR_SCALES_I8; group 256):
+ * streams the packed codes once, decodes them in registers and contracts them on tensor cores.
+ * The 128-row x 256-code blocks are cut into one contiguous range per CTA; a row group that
+ * several ranges share is combined through the workspace in range order, so the result is the
+ * same bits on every run. */
 size_t wr_gemv_workspace_bytes(int64_t M, int64_t N, int64_t K, int bits);
 wr_status wr_gemv(int64_t M, int64_t N, int64_t K, const uint16_t* x, const void* packed,
                   const uint16_t* scales, int bits, int group, float* y, void* workspace,
@@ -209,9 +211,10 @@ size_t wr_gemv_batched_workspace_bytes(int64_t M, int32_t count, const wr_gemv_p
 wr_status wr_gemv_batched(int64_t M, int32_t count, const wr_gemv_problem* problems_host, void* workspace,
                           size_t workspace_bytes, void* stream);
 
-/* Prefill GEMM, any M >= 1 (Q2/Q3, group 256): packed tiles are staged in shared memory,
- * decoded to exact bf16 grid integers and contracted by tcgen05 MMAs into TMEM, one fp32
- * partial per 256-block, scaled in fp32 by the epilogue. */
+/* Prefill GEMM, any M >= 1 (bits = 2 or 3, optionally | WR_SCALES_I8; group 256; M <= 8 runs
+ * the decode GEMV): packed tiles are staged in shared memory, decoded to exact bf16 grid
+ * integers and contracted by tcgen05 MMAs into TMEM, one fp32 partial per 256-block, scaled in
+ * fp32 by the epilogue. */
 size_t wr_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int bits);
 wr_status wr_gemm(int64_t M, int64_t N, int64_t K, const uint16_t* x, const void* packed,
                   const uint16_t* scales, int bits, int group, float* y, void* workspace,
