@@ -245,6 +245,33 @@ def test_gemv_batched_ragged_mixed(wr):
         check_close(y.cpu().numpy(), ref, B)
 
 
+@pytest.mark.parametrize("M", [1, 3, 8])
+def test_gemv_row_group_shared_by_many_ranges(wr, M):
+    """Long rows: one 128-row group of 600 blocks (2-bit) and one of 400 blocks (3-bit) in one
+    batch, so that the cost-cut block ranges give every CTA one or two blocks and a single row
+    group is finished by hundreds of ranges through the partial slots (the last to arrive adds
+    them in range order); then a ragged 3-bit problem after them. Run twice (the arrival
+    counters must be back at zero)."""
+    torch = torch_mod()
+    shapes = [(100, 256 * 600, 2), (128, 256 * 400, 3), (37, 768, 3)]
+    cases, problems = [], []
+    for i, (N, K, bits) in enumerate(shapes):
+        codes, scales, packed, s_d = q_case(wr, bits, N, K, seed=1500 + i)
+        x = wr_synth.activations_bf16(1600 + i, M, K)
+        y = torch.full((M, N), float("nan"), dtype=torch.float32, device="cuda")
+        cases.append((codes, scales, bits, x, y))
+        problems.append((dev(x), packed, s_d, y, N, K, bits))
+    nb = wr.wr_gemv_batched_workspace_bytes(M, problems)
+    ws = _zeros_ws(nb)
+    for _ in range(2):
+        wr.wr_gemv_batched(M, problems, ws, nb)
+        torch.cuda.synchronize()
+        for codes, scales, bits, x, y in cases:
+            ref, B = o.gemm_codes(x, codes, scales, bits)
+            check_close(y.cpu().numpy(), ref, B)
+    assert wr.wr_get_device_error() == 0
+
+
 @pytest.mark.parametrize("M", [64, 65, 129])
 @pytest.mark.parametrize("N,K", [(200, 640), (1024, 2560), (256, 4096)])
 def test_ternary_gemm_prefill(wr, M, N, K):
