@@ -76,8 +76,8 @@ constexpr int kDecodeTokens = 8;   // decode kernel: 8 tokens x 4 activation lim
 
 // ---- decode kernels (M <= 8) and workspace [counters: one int per row group of every problem]
 // [partials][prepared activation tiles: one per block of every problem]. 2/3-bit: the batch's
-// blocks are cut into one contiguous range per CTA, and the partials are two 128-row slots per
-// CTA for the row groups that two ranges share. Ternary: work items (problem, 128-row group,
+// blocks are cut into one contiguous range of equal cost per CTA, and the partials are two
+// 128-row slots per CTA for the row groups that several ranges share. Ternary: work items (problem, 128-row group,
 // block range), with split-K partials for problems cut into P > 1 pieces.
 struct DecodePlan {
   wr::DecArgs args;

@@ -4,8 +4,9 @@
 // Decoding a token reads every weight once ("How We Shrank an AI Model by 85%...", section
 // "Results": generating a token is mostly reading the weights from memory), so the kernel is a
 // weight stream: the batch's blocks (problem by problem, 128-row group by row group, 256-code
-// block by block) are cut into one contiguous range per CTA, so every CTA streams the same
-// number of blocks and keeps its copy rings full across row-group and problem boundaries.
+// block by block) are cut into one contiguous range per CTA, of equal cost (a 3-bit block weighs
+// more than a 2-bit one: block_cost), so that the CTAs finish together, each keeping its copy
+// rings full across row-group and problem boundaries.
 //
 //   y[m,n] = sum_b s[n,b] sum_{k in b} g[n,k] x[m,k],   g = 2c - L  (L = 3 or 7)
 //
