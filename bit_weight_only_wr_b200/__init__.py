@@ -288,7 +288,8 @@ def wr_get_device_error(stream=None) -> int:
 
 def wr_quantize_pack(bits: int, N: int, K: int, w, packed, scales, stream=None) -> None:
     """Device quantizer + packer: fp32 W [N, K] (device) -> packed codes and fp16 block scales
-    (device), bit-identical with wr_quantize + wr_pack."""
+    (device), bit-identical with wr_quantize + wr_pack; with bits | WR_SCALES_I8, `scales` is
+    the int8 scale record (wr_scales_bytes bytes)."""
     _check("wr_quantize_pack", _lib.wr_quantize_pack(bits, N, K, _ptr(w), _ptr(packed), _ptr(scales),
                                                      _stream(stream)))
 
