@@ -114,7 +114,7 @@ void plan_decode(int64_t M, int count, const ProblemShape* shapes, DecodePlan* d
   const double bpi = (double)total_blocks / (double)target_items;
   const bool ternary = count > 0 && shapes[0].fmt == WR_FMT_TERNARY;
   int items = 0, counters = 0, blocks = 0;
-  int64_t partials = 0, xt_bytes = 0, block_base = 0, cost_base = 0;
+  int64_t partials = 0, xt_bytes = 0, block_base = 0, cost_base = 0, max_cost = 1;
   for (int i = 0; i < count; ++i) {
     wr::DecProblem& pr = a.prob[i];
     int P = (int)std::lround((double)pr.B / bpi);
@@ -129,7 +129,10 @@ void plan_decode(int64_t M, int count, const ProblemShape* shapes, DecodePlan* d
     counters += pr.RG;
     blocks += pr.B;
     block_base += (int64_t)pr.RG * pr.B;
-    if (!ternary) cost_base += (int64_t)pr.RG * pr.B * wr::block_cost(pr.bits, (int)M);
+    if (!ternary) {
+      cost_base += (int64_t)pr.RG * pr.B * wr::block_cost(pr.bits, (int)M);
+      max_cost = std::max(max_cost, wr::block_cost(pr.bits, (int)M));
+    }
     if (ternary && pr.P > 1) partials += (int64_t)pr.RG * pr.P * M * 128;
     dp->xt_rel[i] = xt_bytes;
     xt_bytes += (int64_t)pr.B * wr::xtile_bytes(ternary, (int)M);
@@ -137,9 +140,10 @@ void plan_decode(int64_t M, int count, const ProblemShape* shapes, DecodePlan* d
   a.items = items;
   a.total = block_base;
   a.total_cost = cost_base;
-  // 2/3-bit: ranges of at least the largest block cost, so that each holds a block; two partial
-  // slots per CTA of the launch (see DecArgs)
-  dp->grid = (int)std::max<int64_t>(1, std::min<int64_t>(kDecodeGrid, cost_base / wr::block_cost(3, (int)M)));
+  // 2/3-bit: ranges of at least the largest block cost in the batch, so that each holds a block
+  // (one block per CTA for a small single-format batch); two partial slots per CTA of the
+  // launch (see DecArgs)
+  dp->grid = (int)std::max<int64_t>(1, std::min<int64_t>(kDecodeGrid, cost_base / max_cost));
   if (!ternary) partials = 2 * (int64_t)dp->grid * M * 128;
   dp->total_blocks = blocks;
   dp->counter_off = 0;
