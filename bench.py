@@ -355,7 +355,7 @@ def main():
         extras.update(run_extras(args, wr, torch, np, stream, dist, hbm_peak, bf16_peak))
 
     # the step is one wr_gemv_batched call: the preparation pass, then one launch of the decode
-    # GEMV kernel over all 252 problems (about 98% of the step's device time in the ncu launch
+    # GEMV kernel over all 252 problems (about 96% of the two kernels' time in the ncu launch
     # list); achieved = algorithmic bytes of the launch / event-timed duration of the whole call
     achieved = head["gbs"]
     roof = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
