@@ -21,6 +21,7 @@ __all__ = [
     "wr_gemv_batched", "wr_gemv_noalloc", "WR_GEMV_NOALLOC_SCRATCH_BYTES", "WrGemvTernaryProblem",
     "wr_gemv_ternary_batched_workspace_bytes", "wr_gemv_ternary_batched", "wr_selftest_wait_timeout",
     "wr_quantize_pack", "wr_quantize_trellis", "WR_FMT_T2", "WR_SCALES_I8", "wr_scales_bytes",
+    "wr_gemv_batched_plan",
 ]
 
 WR_FMT_TERNARY, WR_FMT_Q2, WR_FMT_Q3, WR_FMT_T2 = 1, 2, 3, 4
@@ -64,6 +65,7 @@ _SIGNATURES = {
     "wr_gemv": (_c_int, [_c_i64, _c_i64, _c_i64, _vp, _vp, _vp, _c_int, _c_int, _vp, _vp, _c_size, _vp]),
     "wr_gemv_batched_workspace_bytes": (_c_size, [_c_i64, ctypes.c_int32, _PROBLEMS]),
     "wr_gemv_batched": (_c_int, [_c_i64, ctypes.c_int32, _PROBLEMS, _vp, _c_size, _vp]),
+    "wr_gemv_batched_plan": (_c_int, [_c_i64, ctypes.c_int32, _PROBLEMS, _vp, _vp, ctypes.c_int32]),
     "wr_gemm_workspace_bytes": (_c_size, [_c_i64, _c_i64, _c_i64, _c_int]),
     "wr_gemm": (_c_int, [_c_i64, _c_i64, _c_i64, _vp, _vp, _vp, _c_int, _c_int, _vp, _vp, _c_size, _vp]),
     "wr_gemm_ternary_workspace_bytes": (_c_size, [_c_i64, _c_i64, _c_i64]),
@@ -232,6 +234,18 @@ def _problems(problems):
 def wr_gemv_batched_workspace_bytes(M: int, problems) -> int:
     arr = problems if isinstance(problems, ctypes.Array) else _problems(problems)
     return _lib.wr_gemv_batched_workspace_bytes(M, len(arr), arr)
+
+
+def wr_gemv_batched_plan(M: int, problems):
+    """(grid, range_starts int64 [grid + 1]): the CTA block ranges of one batched decode launch
+    (problems as for wr_gemv_batched; only their shapes and formats are read)."""
+    arr = problems if isinstance(problems, ctypes.Array) else _problems(problems)
+    grid = ctypes.c_int32(0)
+    _check("wr_gemv_batched_plan", _lib.wr_gemv_batched_plan(M, len(arr), arr, ctypes.addressof(grid), None, 0))
+    starts = np.zeros(grid.value + 1, dtype=np.int64)
+    _check("wr_gemv_batched_plan", _lib.wr_gemv_batched_plan(M, len(arr), arr, ctypes.addressof(grid),
+                                                             _ptr(starts), grid.value + 1))
+    return grid.value, starts
 
 
 def wr_gemv_batched(M: int, problems, workspace, workspace_bytes: int, stream=None) -> None:

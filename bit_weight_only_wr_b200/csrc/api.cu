@@ -422,6 +422,26 @@ static bool batch_ok(int64_t M, int32_t count, const wr_gemv_problem* pr) {
   return true;
 }
 
+wr_status wr_gemv_batched_plan(int64_t M, int32_t count, const wr_gemv_problem* problems, int32_t* grid,
+                               int64_t* range_starts, int32_t range_starts_len) {
+  if (M < 1 || M > 8 || count < 1 || count > wr::kMaxDecodeProblems || !problems || !grid) return WR_ERR_INVALID_ARG;
+  ProblemShape sh[wr::kMaxDecodeProblems];
+  for (int i = 0; i < count; ++i) {
+    QFmt f{};
+    if (!split_fmt(problems[i].bits, true, &f)) return WR_ERR_UNSUPPORTED;
+    if (check_dims(M, problems[i].N, problems[i].K) != WR_OK || problems[i].K % 256 != 0) return WR_ERR_INVALID_ARG;
+    sh[i] = ProblemShape{problems[i].N, problems[i].K, f.base};
+  }
+  static thread_local DecodePlan dp;
+  plan_decode(M, count, sh, &dp);
+  *grid = dp.grid;
+  if (range_starts) {
+    if (range_starts_len < dp.grid + 1) return WR_ERR_INVALID_ARG;
+    for (int c = 0; c <= dp.grid; ++c) range_starts[c] = wr::range_start(dp.args, dp.grid, c);
+  }
+  return WR_OK;
+}
+
 size_t wr_gemv_batched_workspace_bytes(int64_t M, int32_t count, const wr_gemv_problem* problems) {
   if (!batch_ok(M, count, problems)) return 0;
   size_t total = 0;

@@ -103,31 +103,6 @@ struct Pos {
   float* y;
 };
 
-// CTA c's range starts at cost c C / G (block_cost units): at the first block whose cost before
-// it is at least that. The host sizes the grid so that every range holds at least one block.
-__device__ __forceinline__ int64_t cost_start(const DecArgs& a, int c) { return (int64_t)c * a.total_cost / gridDim.x; }
-// First block at or after cost position cs, for a cs inside problem pr (or at its end)
-__device__ __forceinline__ int64_t range_start_in(const DecProblem& pr, int M, int64_t cs) {
-  const int64_t w = block_cost(pr.bits, M), d = cs - pr.cost_base;
-  return pr.block_base + (d > 0 ? (d + w - 1) / w : 0);
-}
-__device__ __forceinline__ int64_t range_start(const DecArgs& a, int c) {
-  const int64_t cs = cost_start(a, c);
-  int lo = 0, hi = a.count - 1;
-  while (lo < hi) {  // last problem whose first block's cost position is <= cs
-    const int mid = (lo + hi + 1) >> 1;
-    if (a.prob[mid].cost_base <= cs) lo = mid;
-    else hi = mid - 1;
-  }
-  return range_start_in(a.prob[lo], a.M, cs);
-}
-// CTA whose range holds global block g of problem pr: the largest c with cost_start(c) <= the
-// cost before g
-__device__ __forceinline__ int cta_of(const DecArgs& a, const DecProblem& pr, int64_t g) {
-  const int64_t x = pr.cost_base + (g - pr.block_base) * block_cost(pr.bits, a.M);
-  return (int)(((x + 1) * gridDim.x - 1) / a.total_cost);
-}
-
 __device__ __forceinline__ void pos_load(Pos& p, const DecArgs& a) {
   const DecProblem& pr = a.prob[p.pi];
   p.N = pr.N;
@@ -142,8 +117,9 @@ __device__ __forceinline__ void pos_load(Pos& p, const DecArgs& a) {
 }
 __device__ __forceinline__ Pos pos_start(const DecArgs& a) {
   Pos p{};
-  p.g = range_start(a, blockIdx.x);
-  p.left = (int)(range_start(a, blockIdx.x + 1) - p.g);
+  const int G = (int)gridDim.x;   // the block ranges: range_start in tc_kernels.cuh
+  p.g = range_start(a, G, blockIdx.x);
+  p.left = (int)(range_start(a, G, blockIdx.x + 1) - p.g);
   if (p.left <= 0) return p;
   int lo = 0, hi = a.count - 1;
   while (lo < hi) {  // last problem whose first block is <= g
@@ -365,7 +341,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_q_kernel(const __gr
     const uint64_t bdesc0 = smem_desc_sw128(xs);
     constexpr uint32_t idesc = idesc_i8_m128(XR);
     constexpr uint32_t atom16 = (uint32_t)(XR * 128) >> 4;
-    const int64_t span = range_start(a, blockIdx.x + 1) - range_start(a, blockIdx.x);
+    const int G = (int)gridDim.x;
+    const int64_t span = range_start(a, G, blockIdx.x + 1) - range_start(a, G, blockIdx.x);
     const uint32_t nblocks = span > 0 ? (uint32_t)span : 0u;
     uint32_t gm = 0;
     bool ok = true;
@@ -489,7 +466,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_q_kernel(const __gr
         // adds the pieces in range order)
         const DecProblem& pr = a.prob[ec.pi];
         const int64_t g0 = ec.g - ec.b;                     // first block of the row group
-        const int c0 = cta_of(a, pr, g0), c1 = cta_of(a, pr, g0 + ec.B - 1);
+        const int G = (int)gridDim.x;
+        const int c0 = range_cta_of(a, G, pr, g0), c1 = range_cta_of(a, G, pr, g0 + ec.B - 1);
         if (c0 == c1) {
           if (n < ec.N) {
 #pragma unroll
@@ -498,7 +476,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_q_kernel(const __gr
           }
         } else {
           // slot 0: the row group began before this range; slot 1: it continues after it
-          const int slot = g0 < range_start_in(pr, M, cost_start(a, blockIdx.x)) ? 0 : 1;
+          const int slot = g0 < range_start_in(pr, M, range_cost_start(a, G, blockIdx.x)) ? 0 : 1;
           float* part = a.partial + ((int64_t)2 * blockIdx.x + slot) * M * 128;
 #pragma unroll
           for (int m = 0; m < kSlots; ++m)
@@ -512,7 +490,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_q_kernel(const __gr
 #pragma unroll
             for (int m = 0; m < kSlots; ++m) acc[m] = 0.f;
             for (int c = c0; c <= c1; ++c) {
-              const int sl = g0 < range_start_in(pr, M, cost_start(a, c)) ? 0 : 1;
+              const int sl = g0 < range_start_in(pr, M, range_cost_start(a, G, c)) ? 0 : 1;
               const float* src = a.partial + ((int64_t)2 * c + sl) * M * 128;
 #pragma unroll
               for (int m = 0; m < kSlots; ++m)

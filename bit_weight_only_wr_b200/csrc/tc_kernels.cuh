@@ -68,6 +68,36 @@ struct DecArgs {
   DecProblem prob[kMaxDecodeProblems];
 };
 
+// Block ranges of the 2/3-bit decode GEMV, used by the kernel (G = gridDim.x) and by the host
+// planner: CTA c of G starts at cost position c C / G (block_cost units, C = total_cost), at the
+// first block whose cost before it is at least that. The host sizes G so that every range holds
+// at least one block (C / G is at least the largest block cost in the batch).
+__host__ __device__ inline int64_t range_cost_start(const DecArgs& a, int G, int c) {
+  return (int64_t)c * a.total_cost / G;
+}
+// First block at or after cost position cs, for a cs inside problem pr (or at its end)
+__host__ __device__ inline int64_t range_start_in(const DecProblem& pr, int M, int64_t cs) {
+  const int64_t w = block_cost(pr.bits, M), d = cs - pr.cost_base;
+  return pr.block_base + (d > 0 ? (d + w - 1) / w : 0);
+}
+// First block of CTA c's range (c = G: the end of the batch)
+__host__ __device__ inline int64_t range_start(const DecArgs& a, int G, int c) {
+  const int64_t cs = range_cost_start(a, G, c);
+  int lo = 0, hi = a.count - 1;
+  while (lo < hi) {  // last problem whose first block's cost position is <= cs
+    const int mid = (lo + hi + 1) >> 1;
+    if (a.prob[mid].cost_base <= cs) lo = mid;
+    else hi = mid - 1;
+  }
+  return range_start_in(a.prob[lo], a.M, cs);
+}
+// CTA whose range holds global block g of problem pr: the largest c with
+// range_cost_start(c) <= the cost before g
+__host__ __device__ inline int range_cta_of(const DecArgs& a, int G, const DecProblem& pr, int64_t g) {
+  const int64_t x = pr.cost_base + (g - pr.block_base) * block_cost(pr.bits, a.M);
+  return (int)(((x + 1) * G - 1) / a.total_cost);
+}
+
 // 2/3-bit decode: the preparation pass writes the B tiles, then the GEMV kernel.
 cudaError_t launch_prep_x(const DecArgs& a, int total_blocks, cudaStream_t stream);
 cudaError_t launch_gemv_q(const DecArgs& a, int grid, cudaStream_t stream);

@@ -208,6 +208,15 @@ typedef struct {
  * 256 problems; larger batches are split into several launches). Each problem computes what
  * wr_gemv computes. problems_host is a host array read during the call. */
 size_t wr_gemv_batched_workspace_bytes(int64_t M, int32_t count, const wr_gemv_problem* problems_host);
+/* The work split of one batched decode launch (count <= 256 problems), computed on the host
+ * with the launch's own arithmetic, for inspection and tests: *grid receives the number of CTAs;
+ * if range_starts is not NULL it receives grid + 1 entries (range_starts_len at least that), the
+ * first block of each CTA's range in the batch's block sequence (problem by problem, 128-row
+ * group by row group, 256-code block by block), then the total block count. Ranges are cut by
+ * an estimated cost per block (a 3-bit or trellis block weighs more than a 2-bit one) and each
+ * holds at least one block. Only the shapes and formats of problems_host are read. */
+wr_status wr_gemv_batched_plan(int64_t M, int32_t count, const wr_gemv_problem* problems_host, int32_t* grid,
+                               int64_t* range_starts, int32_t range_starts_len);
 wr_status wr_gemv_batched(int64_t M, int32_t count, const wr_gemv_problem* problems_host, void* workspace,
                           size_t workspace_bytes, void* stream);
 

@@ -185,3 +185,50 @@ def test_device_calls_reject_bad_arguments_before_launch():
     assert wr.wr_gemm_workspace_bytes(64, 16, 256, 2 | i8) == wr.wr_gemm_workspace_bytes(64, 16, 256, 2)
     assert wr.wr_gemv_workspace_bytes(9, 16, 256, 2) == 0
     assert wr.wr_gemv_workspace_bytes(1, 16, 256, 2) > 0
+
+
+def _block_cost(fmt, M):
+    """Relative cost of one 128 x 256 block in the decode GEMV's work split, as include/wr.h and
+    the launch describe it: a 3-bit or trellis block weighs more than a 2-bit one."""
+    base = fmt & ~wr.WR_SCALES_I8
+    return 20 if base == 2 else (26 if M <= 2 else (25 if M <= 4 else 24))
+
+
+def _check_plan(M, shapes):
+    probs = [(None, None, None, None, N, K, fmt) for (N, K, fmt) in shapes]
+    G, starts = wr.wr_gemv_batched_plan(M, probs)
+    costs = []
+    for N, K, fmt in shapes:
+        costs += [_block_cost(fmt, M)] * (((N + 127) // 128) * (K // 256))
+    T = len(costs)
+    assert 1 <= G <= 444 and starts[0] == 0 and starts[G] == T
+    assert np.all(np.diff(starts) >= 1), "every CTA range holds at least one block"
+    # the ranges partition the blocks by cost: each range's cost is within one block of C / G
+    cum = np.concatenate([[0], np.cumsum(costs)])
+    rc = cum[starts[1:]] - cum[starts[:-1]]
+    C, wmax = cum[-1], max(costs)
+    assert np.all(rc <= C / G + wmax) and np.all(rc >= C / G - wmax)
+    return G, starts
+
+
+def test_decode_plan_of_the_qwen3_body():
+    import wr_synth
+    shapes = [(N, K, bits) for _ in range(36) for (_, K, N, bits) in wr_synth.QWEN3_4B_LAYER]
+    for M in (1, 3, 8):
+        G, _ = _check_plan(M, shapes)
+        assert G == 444
+    # a small single-format batch runs one block per CTA
+    G, starts = _check_plan(1, [(2560, 2560, 2)])
+    assert G == 200 and np.array_equal(starts, np.arange(201))
+
+
+def test_decode_plan_random_batches():
+    rng = np.random.default_rng(7)
+    fmts = [2, 3, wr.WR_FMT_T2, 2 | wr.WR_SCALES_I8, 3 | wr.WR_SCALES_I8]
+    for _ in range(300):
+        n = int(rng.integers(1, 24))
+        shapes = [(int(rng.integers(1, 3000)), 256 * int(rng.integers(1, 48)), int(rng.choice(fmts)))
+                  for _ in range(n)]
+        _check_plan(int(rng.integers(1, 9)), shapes)
+    with pytest.raises(wr.WrError):
+        wr.wr_gemv_batched_plan(9, [(None, None, None, None, 16, 256, 2)])
