@@ -313,19 +313,24 @@ def test_ternary_quantizer_rules():
 # ---------------------------------------------------------------- contraction
 
 def _brute(x_bits, codes, scales, bits):
+    """Exact rational y[m, n] = sum_k s g x and bound[m, n] = sum_k |s g x|, term by term."""
     M, K = x_bits.shape
     N = codes.shape[0]
     L = (1 << bits) - 1
     xf = [[float(v) for v in row] for row in wr_synth.bf16_bits_to_f32(x_bits)]
     y = [[0.0] * N for _ in range(M)]
+    bound = [[Fraction(0)] * N for _ in range(M)]
     for m in range(M):
         for n in range(N):
-            acc = Fraction(0)
+            acc, mag = Fraction(0), Fraction(0)
             for k in range(K):
                 g = 2 * int(codes[n, k]) - L
-                acc += Fraction(float(scales[n, k // 256])) * g * Fraction(xf[m][k])
+                term = Fraction(float(scales[n, k // 256])) * g * Fraction(xf[m][k])
+                acc += term
+                mag += abs(term)
             y[m][n] = float(acc)
-    return np.array(y)
+            bound[m][n] = mag
+    return np.array(y), bound
 
 
 @pytest.mark.parametrize("bits", [2, 3])
@@ -335,9 +340,31 @@ def test_gemm_against_exact_brute_force(bits):
     codes, s = o.quantize_odd_grid(W, bits)
     x = wr_synth.activations_bf16(32, M, K)
     y, B = o.gemm_codes(x, codes, s, bits)
-    ref = _brute(x, codes, s, bits)
+    ref, ref_bound = _brute(x, codes, s, bits)
     assert np.allclose(y, ref, rtol=1e-13, atol=1e-14)
+    # the tolerance bound is exactly sum_k |w x| of the same (m, n): not a looser product of
+    # norms, not summed over another axis
+    for m in range(M):
+        for n in range(N):
+            assert math.isclose(float(B[m, n]), float(ref_bound[m][n]), rel_tol=1e-13)
     assert np.all(B >= np.abs(y))
+
+
+def test_gemm_bound_hand_example():
+    # one 256-block, 2-bit: s = 0.5, codes 0, 3, 1, 2 (g = -3, 3, -1, 1) on x = 1, 2, -4, 8
+    # y = 0.5 (-3 + 6 + 4 + 8) = 7.5 ;  bound = 0.5 (3 + 6 + 4 + 8) = 10.5 ; a second row with
+    # all codes 3 on the same x gives 0.5 * 3 * 7 = 10.5 and bound 0.5 * 3 * 15 = 22.5
+    codes = np.full((2, 256), 1, dtype=np.uint8)
+    codes[0, :4] = [0, 3, 1, 2]
+    codes[1, :4] = [3, 3, 3, 3]
+    codes[:, 4:] = 1
+    s = np.full((2, 1), 0.5, dtype=np.float16)
+    xv = np.zeros((1, 256), dtype=np.float32)
+    xv[0, :4] = [1, 2, -4, 8]
+    x = wr_synth.f32_to_bf16_bits(xv)
+    y, B = o.gemm_codes(x, codes, s, 2)
+    assert y[0, 0] == 7.5 and B[0, 0] == 10.5
+    assert y[0, 1] == 10.5 and B[0, 1] == 22.5
 
 
 def test_gemm_special_cases():
@@ -355,6 +382,49 @@ def test_gemm_special_cases():
     onehot[0, 300] = 0x3F80                             # bf16 1.0
     y, _ = o.gemm_codes(onehot, codes, s, 3)
     assert np.array_equal(y[0], o.dequant(codes, s, 3)[:, 300])
+
+
+def test_dequant_ternary_hand_example():
+    # N = 2 rows, K = 3 positions (N != K, so a broadcast along the wrong axis shows):
+    # codes 0, 1, 2 stand for t = -1, 0, +1 and alpha is one scale per ROW
+    codes = np.array([[0, 1, 2], [2, 2, 0]], dtype=np.uint8)
+    alpha = np.array([0.5, 3.0], dtype=np.float16)
+    W = o.dequant_ternary(codes, alpha)
+    assert W.shape == (2, 3)
+    assert W.tolist() == [[-0.5, 0.0, 0.5], [3.0, 3.0, -3.0]]
+
+
+def _hadamard_entry(a, b):
+    """Sylvester Hadamard entry in closed form: (-1)^popcount(a & b)."""
+    return -1.0 if bin(a & b).count("1") % 2 else 1.0
+
+
+def test_ternary_gemm_against_closed_form_brute_force():
+    # (R x)[k] = (1/sqrt(128)) sum_{j in k's block} (-1)^popcount(k%128 & j%128) d_j x_j, with
+    # d_j = -1 where bit j of the sign mask is set; y = alpha_n sum_k (c - 1) (R x)[k] and
+    # bound = sum_k |alpha_n (c - 1)| |(R x)[k]|, written out element by element
+    K, N, M = 256, 3, 2
+    signs = wr_synth.sign_bits(40, K)
+    rng = np.random.default_rng(41)
+    codes = rng.integers(0, 3, size=(N, K)).astype(np.uint8)
+    alpha = np.array([0.25, 1.5, 0.0625], dtype=np.float16)
+    x = wr_synth.activations_bf16(42, M, K)
+    xf = wr_synth.bf16_bits_to_f32(x).astype(np.float64)
+    d = [(-1.0 if (int(signs[j // 32]) >> (j % 32)) & 1 else 1.0) for j in range(K)]
+    xr = np.zeros((M, K))
+    for m in range(M):
+        for k in range(K):
+            b0 = (k // 128) * 128
+            xr[m, k] = sum(_hadamard_entry(k - b0, j - b0) * d[j] * xf[m, j]
+                           for j in range(b0, b0 + 128)) / math.sqrt(128)
+    y, B = o.gemm_ternary(x, codes, alpha, signs)
+    for m in range(M):
+        for n in range(N):
+            a = float(alpha[n])
+            ref = sum(a * (int(codes[n, k]) - 1) * xr[m, k] for k in range(K))
+            mag = sum(abs(a * (int(codes[n, k]) - 1)) * abs(xr[m, k]) for k in range(K))
+            assert math.isclose(y[m, n], ref, rel_tol=1e-12, abs_tol=1e-12)
+            assert math.isclose(B[m, n], mag, rel_tol=1e-12)
 
 
 def test_ternary_gemm_matches_rotation_identity():
