@@ -180,7 +180,7 @@ wr_status run_decode(DecodePlan& dp, bool ternary, cudaStream_t stream) {
 struct GemmPlan {
   int B = 0, RG = 0, MT = 0, grid = 0;
   int64_t total = 0, Kp = 0;
-  size_t counter_off = 0, partial_off = 0, planes_off = 0, total_bytes = 0;
+  size_t counter_off = 0, partial_off = 0, planes_off = 0, tokex_off = 0, total_bytes = 0;
 };
 
 // tok: tokens per tile (128; 64 for ternary, whose R x hi and lo planes fill 128 MMA columns);
@@ -263,7 +263,8 @@ constexpr int kTernaryTok = 64;   // tokens per GEMM tile
 
 GemmPlan plan_gemm_t(int64_t M, int64_t N, int64_t K) {
   GemmPlan p = plan_gemm(M, N, K, kTernaryTok, 320);
-  p.total_bytes = p.planes_off + align256((size_t)2 * M * p.Kp * sizeof(uint16_t));
+  p.tokex_off = p.planes_off + align256((size_t)2 * M * p.Kp * sizeof(uint16_t));
+  p.total_bytes = p.tokex_off + align256((size_t)M * sizeof(int));
   return p;
 }
 
@@ -292,8 +293,11 @@ wr_status run_t(int64_t M, int64_t N, int64_t K, const uint16_t* x, const void* 
   }
   const GemmPlan p = plan_gemm_t(M, N, K);
   uint8_t* planes = static_cast<uint8_t*>(workspace) + p.planes_off;
-  if (wr::launch_rotate_planes(x, signs, planes, (int)M, (int)K, p.Kp, stream) != cudaSuccess) return WR_ERR_CUDA;
+  int* tok_ex = reinterpret_cast<int*>(static_cast<uint8_t*>(workspace) + p.tokex_off);
+  if (wr::launch_rotate_planes(x, signs, planes, (int)M, (int)K, p.Kp, tok_ex, stream) != cudaSuccess)
+    return WR_ERR_CUDA;
   wr::TcArgs a = gemm_args(p, M, N, K, workspace);
+  a.tok_ex = tok_ex;
   a.packed = static_cast<const uint8_t*>(packed);
   a.alpha = alpha;
   a.y = y;

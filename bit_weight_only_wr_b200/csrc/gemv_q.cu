@@ -433,6 +433,9 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_q_kernel(const __gr
       fence_after_sync();
       const int4* rec = reinterpret_cast<const int4*>(cs + sc * 256);
       const float s = kAll ? half_bits_to_float(sraw) * (float)qraw : half_bits_to_float(sraw);
+      // 2^E = f f2 with f a normal fp32 power of two and f2 = 2^-j (0 <= j <= 36): s f2 is exact
+      // and normal, (s f2) v rounds once, and the last multiply by f rounds once more, gradually
+      // into the subnormal range where the block's activations are that small
       constexpr int kChunk = XR < 16 ? XR : 16;   // columns per load
 #pragma unroll
       for (int c0 = 0; c0 < XR; c0 += kChunk) {
@@ -444,13 +447,13 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_q_kernel(const __gr
         for (int mm = 0; mm < kChunk / 4; ++mm) {
           const int m = c0 / 4 + mm;
           if (m < M) {
-            const int2 c = *reinterpret_cast<const int2*>(rec + m);
+            const int4 c = rec[m];
             // 2 sum_j 256^j D_j + C in fp32 (each D_j is exact in fp32: |D_j| < 2^23)
             float v = fmaf((float)(int)d[4 * mm], 2.f, __int_as_float(c.x));
             v = fmaf((float)(int)d[4 * mm + 1], 512.f, v);
             v = fmaf((float)(int)d[4 * mm + 2], 131072.f, v);
             v = fmaf((float)(int)d[4 * mm + 3], 33554432.f, v);
-            acc[m] = fmaf(s * __int_as_float(c.y), v, acc[m]);
+            acc[m] = fmaf((s * __int_as_float(c.z)) * v, __int_as_float(c.y), acc[m]);
           }
         }
       }
@@ -525,7 +528,10 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_q_kernel(const __gr
 // bytes d_j (n = sum_j 256^j d_j, d_j in [-128, 127]). Limb j goes to B row 4m + j (two atoms of
 // 128 K positions x N rows, 128-byte swizzle). After the atoms, one 16-byte correction record
 // per slot: {C, bits of 2^E, 0, 0} with S_j = sum_k 2^e_k d_j[k] and C = -L sum_j 256^j S_j in
-// fp32. Slots m >= M hold zero limbs and a zero factor.
+// fp32. The factor 2^E is stored as two powers of two, f = 2^max(E, -126) (normal) and
+// f2 = 2^(E - max(E, -126)) >= 2^-36, so that no product in the epilogue leaves the normal range
+// before its last multiply (E reaches -162 for subnormal bf16 activations). Slots m >= M hold zero
+// limbs and a zero factor.
 __global__ void __launch_bounds__(256) prep_x_kernel(const __grid_constant__ DecArgs a, int total_blocks) {
   const int lane = threadIdx.x & 31;
   const int M = a.M;
@@ -590,11 +596,14 @@ __global__ void __launch_bounds__(256) prep_x_kernel(const __grid_constant__ Dec
   }
   if (lane == 0) {
     // correction record of slot m: C = -L sum_j 256^j S_j (exact in fp64, one rounding to
-    // fp32), then 2^E
+    // fp32), then 2^E as the two factors f and f2
     const int L = pr.bits == 2 ? 3 : 7;
-    const float f = (m < M && amax > 0.f) ? ldexpf(1.f, E) : 0.f;
+    const int Ehi = max(E, -126);
+    const float f = (m < M && amax > 0.f) ? ldexpf(1.f, Ehi) : 0.f;
+    const float f2 = ldexpf(1.f, E - Ehi);
     const double S = (double)s[0] + 256.0 * s[1] + 65536.0 * s[2] + 16777216.0 * s[3];
-    reinterpret_cast<int4*>(dst + 256 * xrows)[m] = make_int4(__float_as_int((float)(-L * S)), __float_as_int(f), 0, 0);
+    reinterpret_cast<int4*>(dst + 256 * xrows)[m] =
+        make_int4(__float_as_int((float)(-L * S)), __float_as_int(f), __float_as_int(f2), 0);
   }
 }
 

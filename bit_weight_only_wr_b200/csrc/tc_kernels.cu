@@ -178,6 +178,12 @@ __device__ __forceinline__ uint32_t trit_entry(int v) {
   return e;
 }
 
+// Output value of token m: the ternary planes hold token m scaled by 2^-tok_ex[m], undone here
+// (one rounding, gradual into fp32's subnormal range).
+__device__ __forceinline__ float out_value(const TcArgs& a, float v, int m) {
+  return a.tok_ex ? ldexpf(v, a.tok_ex[m]) : v;
+}
+
 // ---------------------------------------------------------------- the kernel
 
 template <int FMT, int BN>
@@ -427,7 +433,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const TcArgs a, const _
         if (n < a.N) {
 #pragma unroll
           for (int i = 0; i < TH; ++i)
-            if (i < mcount) a.y[(int64_t)(m0 + i) * a.N + n] = rs * acc[i];
+            if (i < mcount) a.y[(int64_t)(m0 + i) * a.N + n] = out_value(a, rs * acc[i], m0 + i);
         }
       } else {
         // slot 0: the tile began before this range; slot 1: it continues after it
@@ -454,7 +460,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const TcArgs a, const _
           if (n < a.N) {
 #pragma unroll
             for (int i = 0; i < TH; ++i)
-              if (i < mcount) a.y[(int64_t)(m0 + i) * a.N + n] = rs * acc[i];
+              if (i < mcount) a.y[(int64_t)(m0 + i) * a.N + n] = out_value(a, rs * acc[i], m0 + i);
           }
           if (threadIdx.x == 256) a.counter[ps_.t] = 0;
         }
@@ -533,10 +539,13 @@ cudaError_t launch_tc(const TcArgs& a, const void* x_act, int64_t x_rows, int64_
 //     c of row r at c ^ (r % 8));
 //   planes (prefill GEMM): [2][M][Kp] bf16 row-major, hi then lo, read by TMA.
 // One warp: token m, 128-block starting at k0 (lane = 4 consecutive K positions).
+// The planes form scales token m by 2^-tok_ex[m] first (exact), so that its hi and lo parts stay
+// in bf16's normal range whatever the magnitude of x; the GEMM epilogue multiplies the token's
+// results by 2^tok_ex[m].
 template <bool PLANES>
 __device__ __forceinline__ void rotate_block(const uint16_t* __restrict__ x, const uint32_t* __restrict__ signs,
                                              uint8_t* __restrict__ xt, int M, int K, int64_t Kp, int m, int64_t k0,
-                                             int lane) {
+                                             int lane, int scale_ex = 0) {
   float v[4];
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
@@ -545,6 +554,7 @@ __device__ __forceinline__ void rotate_block(const uint16_t* __restrict__ x, con
     if (k < K) {
       xv = __bfloat162float(__ushort_as_bfloat16(x[(int64_t)m * K + k]));
       if ((signs[k >> 5] >> (k & 31)) & 1u) xv = -xv;
+      if (PLANES) xv = ldexpf(xv, -scale_ex);
     }
     v[i] = xv;
   }
@@ -593,14 +603,33 @@ __global__ void rotate_x_kernel(const uint16_t* __restrict__ x, const uint32_t* 
   rotate_block<false>(x, signs, xt, M, K, Kp, (int)(item / nblk), (item % nblk) * 128, lane);
 }
 
-// The planes form, for the prefill GEMM: planes = [2][M][Kp] bf16 (hi, lo).
+// The planes form, for the prefill GEMM: planes = [2][M][Kp] bf16 (hi, lo), token m scaled by
+// 2^-tok_ex[m].
 __global__ void rotate_planes_kernel(const uint16_t* __restrict__ x, const uint32_t* __restrict__ signs,
-                                     uint8_t* __restrict__ planes, int M, int K, int64_t Kp) {
+                                     uint8_t* __restrict__ planes, int M, int K, int64_t Kp,
+                                     const int* __restrict__ tok_ex) {
   const int lane = threadIdx.x & 31;
   const int64_t item = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int64_t nblk = (Kp + 127) / 128;
   if (item >= (int64_t)M * nblk) return;
-  rotate_block<true>(x, signs, planes, M, K, Kp, (int)(item / nblk), (item % nblk) * 128, lane);
+  const int m = (int)(item / nblk);
+  rotate_block<true>(x, signs, planes, M, K, Kp, m, (item % nblk) * 128, lane, tok_ex[m]);
+}
+
+// Per-token exponent of the ternary prefill GEMM: tok_ex[m] = e with max_k |x[m,k]| in
+// [2^(e-1), 2^e) (0 for an all-zero token). One warp per token.
+__global__ void token_exponent_kernel(const uint16_t* __restrict__ x, int M, int K, int* __restrict__ tok_ex) {
+  const int lane = threadIdx.x & 31;
+  const int m = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (m >= M) return;
+  float amax = 0.f;
+  for (int k = lane; k < K; k += 32)
+    amax = fmaxf(amax, fabsf(__bfloat162float(__ushort_as_bfloat16(x[(int64_t)m * K + k]))));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  int ex = 0;
+  if (amax > 0.f) frexpf(amax, &ex);
+  if (lane == 0) tok_ex[m] = ex;
 }
 
 // Batched form: work item g -> (problem, token, 128-block) through the problems' first items.
@@ -665,10 +694,12 @@ cudaError_t launch_rotate_x(const uint16_t* x, const uint32_t* signs, uint8_t* x
 }
 
 cudaError_t launch_rotate_planes(const uint16_t* x, const uint32_t* signs, uint8_t* planes, int M, int K, int64_t Kp,
-                                 cudaStream_t stream) {
-  const int64_t items = (int64_t)M * ((Kp + 127) / 128);
+                                 int* tok_ex, cudaStream_t stream) {
   const int warps = 8;
-  rotate_planes_kernel<<<(unsigned)((items + warps - 1) / warps), warps * 32, 0, stream>>>(x, signs, planes, M, K, Kp);
+  token_exponent_kernel<<<(unsigned)((M + warps - 1) / warps), warps * 32, 0, stream>>>(x, M, K, tok_ex);
+  const int64_t items = (int64_t)M * ((Kp + 127) / 128);
+  rotate_planes_kernel<<<(unsigned)((items + warps - 1) / warps), warps * 32, 0, stream>>>(x, signs, planes, M, K, Kp,
+                                                                                         tok_ex);
   return cudaGetLastError();
 }
 

@@ -14,6 +14,7 @@ struct TcArgs {
   float* partial;            // pieces of tiles cut by range ends [grid][2][TOK][128]
   int* counter;              // [RG*MT] arrival counters, zero between calls
   int* err;                  // device error word (bounded waits)
+  const int* tok_ex;         // ternary: per-token exponent of the scaled R x planes (y *= 2^tok_ex)
   int M, N, K;
   int B;                     // 256-code (or 320-trit) blocks per row
   int RG;                    // 128-row groups
@@ -122,8 +123,10 @@ cudaError_t launch_rotate_x(const uint16_t* x, const uint32_t* signs, uint8_t* x
 // The same for every problem of a batch (x, signs, xt, K, Kp per problem; xblk_base = first
 // work item; total_items = M * sum of ceil(Kp / 128)).
 // R x as two bf16 planes [2][M][Kp] (hi, lo) in the decoded K order, for the prefill GEMM.
+// Token m is scaled by 2^-tok_ex[m] (tok_ex [M] int, written first by a per-token pass: the
+// exponent of the token's largest |x|), so that tiny and huge tokens keep full precision.
 cudaError_t launch_rotate_planes(const uint16_t* x, const uint32_t* signs, uint8_t* planes, int M, int K, int64_t Kp,
-                                 cudaStream_t stream);
+                                 int* tok_ex, cudaStream_t stream);
 cudaError_t launch_rotate_x_batched(const DecArgs& a, int64_t total_items, cudaStream_t stream);
 // Device quantizer + packer for the 2/3-bit odd grid (quantize.cu). scale_q null: fp16 block
 // scales [N, K/256] in `scales`; else the int8 form: fp16 row scales d [N] in `scales` and the

@@ -244,7 +244,8 @@ wr_status wr_gemm_ternary(int64_t M, int64_t N, int64_t K, const uint16_t* x, co
  * WR_GEMV_NOALLOC_SCRATCH_BYTES (4 MiB) inside libwr, one per device.
  *
  * Computes exactly what wr_gemv computes (same arguments without workspace/workspace_bytes;
- * 1 <= M <= 8, bits 2 or 3, group 256, K % 256 == 0, 16-byte aligned device pointers).
+ * 1 <= M <= 8, bits 2, 3 or WR_FMT_T2, each optionally | WR_SCALES_I8, group 256, K % 256 == 0,
+ * 16-byte aligned device pointers).
  * Returns WR_ERR_TOO_LARGE, before touching the device, when the problem's scratch need
  * (wr_gemv_workspace_bytes) exceeds WR_GEMV_NOALLOC_SCRATCH_BYTES; then nothing is launched.
  *

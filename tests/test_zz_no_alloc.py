@@ -11,7 +11,7 @@ import pytest
 
 import wr_synth
 from oracle import wr_oracle as o
-from gpu_inputs import check_close, dev, q_case, torch_mod
+from gpu_inputs import check_close, dev, q_case, s8_case, torch_mod
 
 
 def test_too_large_rejected_before_device_work():
@@ -60,6 +60,52 @@ def test_noalloc_matches_workspace_path(bits, N, K, M):
     assert wr.wr_get_device_error() == 0
 
     y_ref, bound = o.gemm_codes(x_bits, codes, scales_h, bits)
+    y_ws = y_ws.cpu().numpy()
+    check_close(y_ws, y_ref, bound)
+    for y in outs:
+        check_close(y, y_ref, bound)
+        assert np.all(np.abs(y.astype(np.float64) - y_ws) <= 1e-4 * bound)
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("fmt_name,N,K,M", [
+    ("t2", 300, 2560, 1),        # trellis-coded 2-bit symbols
+    ("q3_i8", 1024, 2560, 4),    # 3-bit codes with int8 block scales
+    ("q2_i8", 129, 768, 8),      # 2-bit codes with int8 block scales, ragged N
+])
+def test_noalloc_trellis_and_int8_scales(fmt_name, N, K, M):
+    """The formats wr_gemv accepts besides plain Q2/Q3 (WR_FMT_T2, | WR_SCALES_I8), through the
+    no-allocation entry point: agreement with wr_gemv and with the oracle on two calls in a row."""
+    torch = torch_mod()
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import bit_weight_only_wr_b200 as wr
+    seed = 7100 + N + M
+    x_bits = wr_synth.activations_bf16(seed + 1, M, K)
+    x = dev(x_bits)
+    if fmt_name == "t2":
+        fmt = wr.WR_FMT_T2
+        sym, sc = wr.wr_quantize_trellis(wr_synth.weights_fp32(seed, N, K))
+        packed, scales = dev(wr.wr_pack(fmt, sym)), dev(sc)
+        y_ref, bound = o.gemm_trellis2(x_bits, sym, sc.view(np.float16))
+    else:
+        bits = 3 if fmt_name == "q3_i8" else 2
+        fmt = bits | wr.WR_SCALES_I8
+        codes, d, q, packed, scales = s8_case(wr, bits, N, K, seed)
+        y_ref, bound = o.gemm_codes_s8(x_bits, codes, d, q, bits)
+    assert wr.wr_gemv_workspace_bytes(M, N, K, fmt) <= wr.WR_GEMV_NOALLOC_SCRATCH_BYTES
+
+    y_ws = torch.full((M, N), float("nan"), dtype=torch.float32, device="cuda")
+    nb = wr.wr_gemv_workspace_bytes(M, N, K, fmt)
+    ws = torch.zeros(max(nb, 256), dtype=torch.uint8, device="cuda")
+    wr.wr_gemv(M, N, K, x, packed, scales, fmt, y_ws, ws, nb)
+    outs = []
+    for _ in range(2):
+        y = torch.full((M, N), float("nan"), dtype=torch.float32, device="cuda")
+        wr.wr_gemv_noalloc(M, N, K, x, packed, scales, fmt, y)
+        torch.cuda.synchronize()
+        outs.append(y.cpu().numpy())
+    assert wr.wr_get_device_error() == 0
     y_ws = y_ws.cpu().numpy()
     check_close(y_ws, y_ref, bound)
     for y in outs:
