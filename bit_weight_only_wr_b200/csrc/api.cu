@@ -21,20 +21,6 @@ __device__ int g_device_error = 0;
 inline bool aligned16(const void* p) { return p && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 inline size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
 
-int sm_count() {
-  static std::mutex mu;
-  static int cache[64] = {0};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
-  std::lock_guard<std::mutex> lock(mu);
-  if (cache[dev] == 0) {
-    int v = 0;
-    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) v = 148;
-    cache[dev] = v;
-  }
-  return cache[dev];
-}
-
 int* device_error_word() {
   static std::mutex mu;
   static int* cache[64] = {nullptr};
@@ -71,18 +57,16 @@ inline const int8_t* scale_q_of(const QFmt& f, const uint16_t* scales, int64_t N
 }
 
 constexpr int kPlanSMs = 148;   // split heuristics are sized for a 148-SM part (device-independent)
-constexpr int kDecodeGrid = 3 * kPlanSMs;   // 2/3-bit decode: CTAs (block ranges) per launch, at most
 constexpr int kDecodeTokens = 8;   // decode kernel: 8 tokens x 4 activation limbs = 32 MMA columns
 
-// ---- decode kernels (M <= 8) and workspace [counters: one int per row group of every problem]
-// [partials][prepared activation tiles: one per block of every problem]. 2/3-bit: the batch's
-// blocks are cut into one contiguous range of equal cost per CTA, and the partials are two
-// 128-row slots per CTA for the row groups that several ranges share. Ternary: work items (problem, 128-row group,
-// block range), with split-K partials for problems cut into P > 1 pieces.
+// ---- decode kernel (M <= 8) and workspace [counters: one int per row group of every problem]
+// [partials][prepared activation tiles: one per block of every problem]. The batch's blocks are
+// cut into one contiguous range of equal cost per CTA, and the partials are two 128-row slots per
+// CTA for the row groups that several ranges share. A batch is all 2/3-bit or all ternary.
 struct DecodePlan {
   wr::DecArgs args;
-  int total_blocks = 0;
-  int grid = 0;   // 2/3-bit: CTAs (block ranges) of the decode launch
+  int total_blocks = 0;   // K blocks of all problems (work of the preparation pass, per token slot)
+  int grid = 0;           // CTAs (block ranges) of the decode launch
   size_t counter_off = 0, partial_off = 0, xt_off = 0, total = 0;
   int64_t xt_rel[wr::kMaxDecodeProblems];
 };
@@ -96,7 +80,9 @@ void plan_decode(int64_t M, int count, const ProblemShape* shapes, DecodePlan* d
   wr::DecArgs& a = dp->args;
   a.count = count;
   a.M = (int)M;
-  int64_t total_blocks = 0;
+  const bool ternary = count > 0 && shapes[0].fmt == WR_FMT_TERNARY;
+  int counters = 0, blocks = 0;
+  int64_t xt_bytes = 0, block_base = 0, cost_base = 0, max_cost = 1;
   for (int i = 0; i < count; ++i) {
     int64_t ub = 0, units = 0, tiles = 0;
     wr::packed_geometry(shapes[i].fmt, shapes[i].N, shapes[i].K, &ub, &units, &tiles);
@@ -105,46 +91,29 @@ void plan_decode(int64_t M, int count, const ProblemShape* shapes, DecodePlan* d
     pr.N = (int)shapes[i].N;
     pr.K = (int)shapes[i].K;
     pr.B = (int)units;
-    pr.Kp = shapes[i].fmt == WR_FMT_TERNARY ? (int)(units * 320) : (int)shapes[i].K;
+    pr.Kp = ternary ? (int)(units * 320) : (int)shapes[i].K;
     pr.RG = (int)((shapes[i].N + 127) / 128);
-    pr.bits = shapes[i].fmt == WR_FMT_TERNARY ? 1 : shapes[i].fmt;
-    total_blocks += (int64_t)pr.RG * pr.B;
-  }
-  const int64_t target_items = std::max<int64_t>(3 * kPlanSMs, (total_blocks + 7) / 8);
-  const double bpi = (double)total_blocks / (double)target_items;
-  const bool ternary = count > 0 && shapes[0].fmt == WR_FMT_TERNARY;
-  int items = 0, counters = 0, blocks = 0;
-  int64_t partials = 0, xt_bytes = 0, block_base = 0, cost_base = 0, max_cost = 1;
-  for (int i = 0; i < count; ++i) {
-    wr::DecProblem& pr = a.prob[i];
-    int P = (int)std::lround((double)pr.B / bpi);
-    pr.P = std::max(1, std::min(pr.B, P));
-    pr.item_base = items;
+    pr.bits = ternary ? 1 : shapes[i].fmt;
     pr.counter_base = counters;
-    pr.partial_base = partials;
     pr.xblk_base = blocks;
     pr.block_base = block_base;
     pr.cost_base = cost_base;
-    items += pr.RG * pr.P;
     counters += pr.RG;
     blocks += pr.B;
     block_base += (int64_t)pr.RG * pr.B;
-    if (!ternary) {
-      cost_base += (int64_t)pr.RG * pr.B * wr::block_cost(pr.bits, (int)M);
-      max_cost = std::max(max_cost, wr::block_cost(pr.bits, (int)M));
-    }
-    if (ternary && pr.P > 1) partials += (int64_t)pr.RG * pr.P * M * 128;
+    cost_base += (int64_t)pr.RG * pr.B * wr::block_cost(pr.bits, (int)M);
+    max_cost = std::max(max_cost, wr::block_cost(pr.bits, (int)M));
     dp->xt_rel[i] = xt_bytes;
     xt_bytes += (int64_t)pr.B * wr::xtile_bytes(ternary, (int)M);
   }
-  a.items = items;
   a.total = block_base;
   a.total_cost = cost_base;
-  // 2/3-bit: ranges of at least the largest block cost in the batch, so that each holds a block
-  // (one block per CTA for a small single-format batch); two partial slots per CTA of the
-  // launch (see DecArgs)
-  dp->grid = (int)std::max<int64_t>(1, std::min<int64_t>(kDecodeGrid, cost_base / max_cost));
-  if (!ternary) partials = 2 * (int64_t)dp->grid * M * 128;
+  // ranges of at least the largest block cost in the batch, so that each holds a block (one
+  // block per CTA for a small single-format batch), at most one wave of CTAs; two partial slots
+  // per CTA of the launch (see DecArgs)
+  const int64_t wave = (int64_t)wr::decode_ctas_per_sm(ternary, (int)M) * kPlanSMs;
+  dp->grid = (int)std::max<int64_t>(1, std::min<int64_t>(wave, cost_base / max_cost));
+  const int64_t partials = 2 * (int64_t)dp->grid * M * 128;
   dp->total_blocks = blocks;
   dp->counter_off = 0;
   dp->partial_off = align256((size_t)counters * sizeof(int));
@@ -162,14 +131,9 @@ void bind_workspace(DecodePlan& dp, void* workspace) {
   dp.args.err = device_error_word();
 }
 
-// Q2/Q3: preparation pass, then the decode kernel; ternary: the rotation pass has already
-// written the tiles.
-wr_status run_decode(DecodePlan& dp, bool ternary, cudaStream_t stream) {
-  if (ternary) {
-    const int grid = (int)std::min<int64_t>(dp.args.items, (int64_t)sm_count() * 2);
-    return wr::launch_gemv_t(dp.args, grid, stream) == cudaSuccess ? WR_OK : WR_ERR_CUDA;
-  }
-  // one contiguous block range per CTA; the partial slots were sized for this grid
+// The preparation pass (for ternary, with the rotation), then the decode kernel over one
+// contiguous block range per CTA (the partial slots were sized for this grid).
+wr_status run_decode(DecodePlan& dp, cudaStream_t stream) {
   if (wr::launch_prep_x(dp.args, dp.total_blocks, stream) != cudaSuccess) return WR_ERR_CUDA;
   return wr::launch_gemv_q(dp.args, dp.grid, stream) == cudaSuccess ? WR_OK : WR_ERR_CUDA;
 }
@@ -250,15 +214,15 @@ wr_status run_q(int bits, int64_t M, int64_t N, int64_t K, const uint16_t* x, co
     dp.args.prob[0].scale_q = scale_q;
     dp.args.prob[0].y = y;
     bind_workspace(dp, workspace);
-    return run_decode(dp, false, stream);
+    return run_decode(dp, stream);
   }
   return run_gemm(bits, (int)M, (int)N, (int)K, x, static_cast<const uint8_t*>(packed), scales, scale_q, y, workspace,
                   stream);
 }
 
-// Ternary. M <= 8: the decode kernel (R x hi and lo fill the MMA columns). M > 8: the prefill
-// GEMM over 64-token tiles (the hi and lo planes of R x make the 128 MMA columns); its
-// workspace adds the R x planes [2][M][Kp] bf16 after the GEMM's own.
+// Ternary. M <= 8: the decode kernel (its preparation pass applies the rotation). M > 8: the
+// prefill GEMM over 64-token tiles (the hi and lo planes of R x make the 128 MMA columns); its
+// workspace adds the R x planes [2][M][Kp] bf16 and the per-token exponents after the GEMM's own.
 constexpr int kTernaryTok = 64;   // tokens per GEMM tile
 
 GemmPlan plan_gemm_t(int64_t M, int64_t N, int64_t K) {
@@ -283,13 +247,12 @@ wr_status run_t(int64_t M, int64_t N, int64_t K, const uint16_t* x, const void* 
     const ProblemShape sh{N, K, WR_FMT_TERNARY};
     plan_decode(M, 1, &sh, &dp);
     bind_workspace(dp, workspace);
-    if (wr::launch_rotate_x(x, signs, dp.args.prob[0].xt, (int)M, (int)K, dp.args.prob[0].Kp, stream) != cudaSuccess)
-      return WR_ERR_CUDA;
-    dp.args.prob[0].x = nullptr;
+    dp.args.prob[0].x = x;
+    dp.args.prob[0].signs = signs;
     dp.args.prob[0].packed = static_cast<const uint8_t*>(packed);
     dp.args.prob[0].scales = alpha;
     dp.args.prob[0].y = y;
-    return run_decode(dp, true, stream);
+    return run_decode(dp, stream);
   }
   const GemmPlan p = plan_gemm_t(M, N, K);
   uint8_t* planes = static_cast<uint8_t*>(workspace) + p.planes_off;
@@ -483,7 +446,7 @@ wr_status wr_gemv_batched(int64_t M, int32_t count, const wr_gemv_problem* probl
       dp.args.prob[i].y = problems[c0 + i].y;
     }
     bind_workspace(dp, workspace);
-    const wr_status st = run_decode(dp, false, static_cast<cudaStream_t>(stream));
+    const wr_status st = run_decode(dp, static_cast<cudaStream_t>(stream));
     if (st != WR_OK) return st;
   }
   return WR_OK;
@@ -525,7 +488,6 @@ wr_status wr_gemv_ternary_batched(int64_t M, int32_t count, const wr_gemv_ternar
     const int n = std::min(count - c0, wr::kMaxDecodeProblems);
     for (int i = 0; i < n; ++i) sh[i] = ProblemShape{problems[c0 + i].N, problems[c0 + i].K, WR_FMT_TERNARY};
     plan_decode(M, n, sh, &dp);
-    int64_t rot_items = 0;
     for (int i = 0; i < n; ++i) {
       wr::DecProblem& pr = dp.args.prob[i];
       pr.x = problems[c0 + i].x;
@@ -533,12 +495,9 @@ wr_status wr_gemv_ternary_batched(int64_t M, int32_t count, const wr_gemv_ternar
       pr.scales = problems[c0 + i].alpha;
       pr.signs = problems[c0 + i].sign_bits;
       pr.y = problems[c0 + i].y;
-      pr.xblk_base = (int)rot_items;   // rotation work items: (token, 128-block)
-      rot_items += M * (((int64_t)pr.Kp + 127) / 128);
     }
     bind_workspace(dp, workspace);
-    if (wr::launch_rotate_x_batched(dp.args, rot_items, s) != cudaSuccess) return WR_ERR_CUDA;
-    const wr_status st = run_decode(dp, true, s);
+    const wr_status st = run_decode(dp, s);
     if (st != WR_OK) return st;
   }
   return WR_OK;

@@ -56,23 +56,37 @@ namespace {
 using namespace tc;
 
 constexpr int kThreads = 320;
-constexpr int kCtasPerSm = 3;
-constexpr int kSP = 4;   // packed stages: 8 units of up to 1.5 KB
-constexpr int kSX = 3;   // B tiles (up to 2 atoms x 32 rows x 128 bytes); also the MMA-done ring
+constexpr int kSP = 4;   // packed stages: the 8 units of a row group's block
+constexpr int kSX = 3;   // B tiles; also the MMA-done ring
 constexpr int kSC = 4;   // correction records, 256 bytes
-constexpr int kPStage = 8 * 1536;
-constexpr int kXStage = 8 * 1024;
-constexpr int kXOff = 0;                          // 1024-byte aligned (128-byte swizzle atoms)
-constexpr int kPOff = kXOff + kSX * kXStage;
-constexpr int kCOff = kPOff + kSP * kPStage;
-constexpr int kBarOff = kCOff + kSC * 256;
-constexpr int kSmem = kBarOff + 256 + 1024;        // + alignment slack
-static_assert(kCtasPerSm * (kSmem + 1024) <= 228 * 1024, "three CTAs per SM");
-constexpr int kACol = 0;                          // one block of codes: 256 bytes per lane
-constexpr int kDCol = 64;                         // two accumulators of N <= 32 columns
-constexpr int kDCols = 32;
-constexpr int kTmemCols = 128;
-static_assert(kCtasPerSm * kTmemCols <= 512, "tensor memory of an SM");
+
+// The three forms of the kernel: a batch of Q2/Q3 problems with fp16 scales (the lean form), a
+// batch that also holds trellis-coded problems or int8 block scales, and a ternary batch.
+enum { kModeLean = 0, kModeAll = 1, kModeTern = 2 };
+
+// Shared-memory and tensor-memory layout of one form. Q2/Q3: a block is 256 codes (A: 64 columns,
+// B: two atoms of 128 K positions). Ternary: a block is one 320-trit unit (A: 80 columns, B: three
+// atoms, the last half used), plus a 243-entry decode table replicated per lane (31 KB), so a CTA
+// needs more room; at MMA N = 16 or 32 two CTAs share an SM.
+template <int XR, int MODE>
+struct Cfg {
+  static constexpr bool kT = MODE == kModeTern;
+  static constexpr int kCtas = (kT && XR > 8) ? 2 : 3;
+  static constexpr int kPStage = 8 * (kT ? 1024 : 1536);
+  static constexpr int kXStage = kT ? 3 * XR * 128 : 8 * 1024;   // 1024-byte multiples (swizzle atoms)
+  static constexpr int kXOff = 0;
+  static constexpr int kPOff = kXOff + kSX * kXStage;
+  static constexpr int kCOff = kPOff + kSP * kPStage;
+  static constexpr int kBarOff = kCOff + kSC * 256;
+  static constexpr int kSmem = kBarOff + 256 + 1024;   // + alignment slack
+  static constexpr int kLutWords = kT ? 243 * 32 : 1;
+  static constexpr int kACol = 0;
+  static constexpr int kDCol = kT ? 96 : 64;           // two accumulators after the A buffer
+  static constexpr int kDCols = kT ? XR : 32;
+  static constexpr int kTmemCols = kDCol + 2 * kDCols <= 128 ? 128 : 256;
+  static_assert(kCtas * (kSmem + 4 * kLutWords + 1024) <= 228 * 1024, "CTAs per SM by shared memory");
+  static_assert(kCtas * kTmemCols <= 512, "tensor memory of an SM");
+};
 
 struct Bars {
   uint64_t pk_full[kSP], pk_empty[kSP], x_full[kSX], c_full[kSC], c_empty[kSC];
@@ -214,6 +228,56 @@ __device__ __forceinline__ void q3_half_i8(const uint8_t* unit, int r0, int half
   }
 }
 
+// Ternary quarter q (80 trits: 16 base-3 bytes v = sum_d c_d 3^d) of a row, as 20 A registers of
+// signed bytes. The 4 packed words themselves, each byte flipped to v - 128 (one XOR), fill A
+// columns 4q .. 4q+3; the first four digits of each byte, as t_d = c_d - 1, come from a 243-entry
+// table (one copy per lane, so the 32 lookups of a warp hit 32 different banks) and fill columns
+// 16 + 16q + j (byte j). With the activations arranged to match (the preparation pass), byte j
+// contributes (v - 128) n_v + sum_{d<4} t_d (n_d - 3^d n_v) = sum_{d<4} t_d n_d + 81 t_4 n_v - 7 n_v,
+// since v - 128 = sum_{d<=4} 3^d t_d - 7: its fifth trit through n_v, the activation of that trit
+// divided by 81, and a constant 7 n_v that the correction record adds back in integers.
+__device__ __forceinline__ void tern_quarter_i8(const uint8_t* unit, int r0, int half, int q, const uint32_t* lut,
+                                                int lane, uint32_t raw[4], uint32_t lv[16]) {
+  const uint4 c = *reinterpret_cast<const uint4*>(unit + (32 * half + lane_pos(r0, q)) * 16);
+  const uint32_t w[4] = {c.x, c.y, c.z, c.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) raw[i] = w[i] ^ 0x80808080u;
+#pragma unroll
+  for (int j = 0; j < 16; ++j) lv[j] = lut[(((w[j >> 2] >> (8 * (j & 3))) & 0xFFu) << 5) | (uint32_t)lane];
+}
+
+// The 10 K slices of one 320-trit block and their commit, issued by one elected lane: A slice j is
+// the 8 columns at a_tmem + 8 j; B slice j is at byte 32 (j % 4) of atom j / 4 (atom16 = the atom
+// size in 16-byte units); the first slice overwrites D.
+__device__ __forceinline__ void mma10_i8_commit_elect(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                                      uint32_t atom16, uint32_t idesc, uint64_t* bar) {
+  const uint64_t b4 = b_desc + atom16, b8 = b_desc + 2 * atom16;
+  asm volatile(
+      "{\n .reg .pred e;\n elect.sync _|e, 0xffffffff;\n"
+      " @e tcgen05.mma.cta_group::1.kind::i8 [%0], [%1], %2, %3, 0;\n"
+      " @e tcgen05.mma.cta_group::1.kind::i8 [%0], [%4], %5, %3, 1;\n"
+      " @e tcgen05.mma.cta_group::1.kind::i8 [%0], [%6], %7, %3, 1;\n"
+      " @e tcgen05.mma.cta_group::1.kind::i8 [%0], [%8], %9, %3, 1;\n"
+      " @e tcgen05.mma.cta_group::1.kind::i8 [%0], [%10], %11, %3, 1;\n"
+      " @e tcgen05.mma.cta_group::1.kind::i8 [%0], [%12], %13, %3, 1;\n"
+      " @e tcgen05.mma.cta_group::1.kind::i8 [%0], [%14], %15, %3, 1;\n"
+      " @e tcgen05.mma.cta_group::1.kind::i8 [%0], [%16], %17, %3, 1;\n"
+      " @e tcgen05.mma.cta_group::1.kind::i8 [%0], [%18], %19, %3, 1;\n"
+      " @e tcgen05.mma.cta_group::1.kind::i8 [%0], [%20], %21, %3, 1;\n"
+      " @e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%22];\n}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(a_tmem + 8), "l"(b_desc + 2), "r"(a_tmem + 16), "l"(b_desc + 4),
+      "r"(a_tmem + 24), "l"(b_desc + 6), "r"(a_tmem + 32), "l"(b4), "r"(a_tmem + 40), "l"(b4 + 2), "r"(a_tmem + 48),
+      "l"(b4 + 4), "r"(a_tmem + 56), "l"(b4 + 6), "r"(a_tmem + 64), "l"(b8), "r"(a_tmem + 72), "l"(b8 + 2),
+      "r"(smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_st4(uint32_t taddr, const uint32_t* v) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1, %2, %3, %4};" ::"r"(taddr), "r"(v[0]), "r"(v[1]),
+               "r"(v[2]), "r"(v[3])
+               : "memory");
+}
+
 // tcgen05.ld of NC (8, 16 or 32) raw 32-bit columns; the values are valid after
 // tmem_wait_ld_regs on the same array, which names them so that no use is scheduled earlier.
 template <int NC>
@@ -244,21 +308,40 @@ __device__ __forceinline__ void tmem_wait_ld_regs(uint32_t (&r)[NC]) {
   for (int i = 0; i < NC; ++i) asm volatile("" : "+r"(r[i]));
 }
 
-// XR: MMA N, 4 limb rows per token slot (8, 16 or 32 for M <= 2, 4, 8). kAll: the batch holds
-// trellis-coded problems or int8 block scales; without them the decode and epilogue warps keep
-// only the Q2/Q3 branches and the fp16 scale load.
-template <int XR, bool kAll>
-__global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_q_kernel(const __grid_constant__ DecArgs a) {
+// XR: MMA N, 4 limb rows per token slot (8, 16 or 32 for M <= 2, 4, 8). MODE: kModeLean keeps
+// only the Q2/Q3 decode branches and the fp16 scale load; kModeAll adds the trellis decode and
+// int8 block scales; kModeTern is the ternary batch (its decode table, 320-trit blocks, signed A).
+template <int XR, int MODE>
+__global__ void __launch_bounds__(kThreads, Cfg<XR, MODE>::kCtas) gemv_q_kernel(const __grid_constant__ DecArgs a) {
+  using C = Cfg<XR, MODE>;
+  constexpr bool kAll = MODE == kModeAll;
+  constexpr bool kT = C::kT;
   extern __shared__ uint8_t smem_raw[];
+  __shared__ uint32_t tlut[C::kLutWords];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* xs = smem + kXOff;
-  uint8_t* ps = smem + kPOff;
-  uint8_t* cs = smem + kCOff;
-  Bars* bars = reinterpret_cast<Bars*>(smem + kBarOff);
+  uint8_t* xs = smem + C::kXOff;
+  uint8_t* ps = smem + C::kPOff;
+  uint8_t* cs = smem + C::kCOff;
+  Bars* bars = reinterpret_cast<Bars*>(smem + C::kBarOff);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   volatile int* abort_flag = &bars->abort_flag;
   constexpr int kSlots = XR / 4;       // token slots
   const int M = a.M;
+
+  if constexpr (kT) {
+    // decode table: entry v holds t_d = c_d - 1 (d = 0..3) of the base-3 byte v as signed bytes,
+    // one copy per lane (word 32 v + lane)
+    for (int i = threadIdx.x; i < 243 * 32; i += kThreads) {
+      int v = i >> 5;
+      uint32_t e = 0;
+#pragma unroll
+      for (int d = 0; d < 4; ++d) {
+        e |= (uint32_t)(uint8_t)(int8_t)(v % 3 - 1) << (8 * d);
+        v /= 3;
+      }
+      tlut[i] = e;
+    }
+  }
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kSP; ++i) {
@@ -280,7 +363,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_q_kernel(const __gr
     bars->last_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 9) tmem_alloc(&bars->tmem_base, kTmemCols);
+  if (warp == 9) tmem_alloc(&bars->tmem_base, C::kTmemCols);
   fence_before_sync();
   __syncthreads();
   fence_after_sync();
@@ -290,7 +373,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_q_kernel(const __gr
     // ------------------------------------------------------------ copy warp (whole warp walks the
     // blocks, one elected lane issues): packed weights (a ring of kSP blocks), prepared B tiles
     // and their correction records (a ring of kSX blocks)
-    constexpr uint32_t bbytes = 256u * XR;
+    constexpr uint32_t bbytes = (kT ? 384u : 256u) * XR;
     constexpr uint32_t xtb = bbytes + 256u;   // prepared tile: B atoms, then corrections
     Pos cp = pos_start(a), cx = cp;            // next block to copy: weights, activations
     const uint32_t nblocks = cp.left > 0 ? (uint32_t)cp.left : 0u;
@@ -305,7 +388,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_q_kernel(const __gr
         const int ntile = min(8, (cp.N + 15) / 16 - cp.rg * 8);
         if (elect_one()) {
           mbar_arrive_expect_tx(&bars->pk_full[sp], ntile * ub);
-          bulk_load(ps + sp * kPStage, cp.packed + ((int64_t)cp.rg * 8 * cp.B + (int64_t)cp.b * ntile) * ub,
+          bulk_load(ps + sp * C::kPStage, cp.packed + ((int64_t)cp.rg * 8 * cp.B + (int64_t)cp.b * ntile) * ub,
                     ntile * ub, &bars->pk_full[sp]);
         }
         __syncwarp();
@@ -321,7 +404,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_q_kernel(const __gr
         const uint8_t* xsrc = cx.xt + (int64_t)cx.b * xtb;
         if (elect_one()) {
           mbar_arrive_expect_tx(&bars->x_full[sx], bbytes);
-          bulk_load(xs + sx * kXStage, xsrc, bbytes, &bars->x_full[sx]);
+          bulk_load(xs + sx * C::kXStage, xsrc, bbytes, &bars->x_full[sx]);
           mbar_arrive_expect_tx(&bars->c_full[sc], 256);
           bulk_load(cs + sc * 256, xsrc + bbytes, 256, &bars->c_full[sc]);
         }
@@ -339,7 +422,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_q_kernel(const __gr
   } else if (warp == 9) {
     // ------------------------------------------------------------ MMA warp (whole warp, one lane issues)
     const uint64_t bdesc0 = smem_desc_sw128(xs);
-    constexpr uint32_t idesc = idesc_i8_m128(XR);
+    constexpr uint32_t idesc = kT ? idesc_i8s_m128(XR) : idesc_i8_m128(XR);
     constexpr uint32_t atom16 = (uint32_t)(XR * 128) >> 4;
     const int G = (int)gridDim.x;
     const int64_t span = range_start(a, G, blockIdx.x + 1) - range_start(a, G, blockIdx.x);
@@ -355,8 +438,12 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_q_kernel(const __gr
       if (!(ok = mbar_wait(&bars->d_empty[gm & 1], ((gm >> 1) & 1) ^ 1, abort_flag, a.err, 203))) break;
       if (!(ok = mbar_wait(&bars->a_full, gm & 1, abort_flag, a.err, 201))) break;
       fence_after_sync();
-      mma8_i8_commit_elect(tmem + kDCol + (gm & 1) * kDCols, tmem + kACol,
-                           bdesc0 + (uint64_t)((sx * kXStage) >> 4), atom16, idesc, &bars->mma_done[sx]);
+      if constexpr (kT)
+        mma10_i8_commit_elect(tmem + C::kDCol + (gm & 1) * C::kDCols, tmem + C::kACol,
+                              bdesc0 + (uint64_t)((sx * C::kXStage) >> 4), atom16, idesc, &bars->mma_done[sx]);
+      else
+        mma8_i8_commit_elect(tmem + C::kDCol + (gm & 1) * C::kDCols, tmem + C::kACol,
+                             bdesc0 + (uint64_t)((sx * C::kXStage) >> 4), atom16, idesc, &bars->mma_done[sx]);
     }
     // the MMAs already issued finish before tensor memory is released
     if (!ok && gm > 0) mbar_wait_drain(&bars->mma_done[(gm - 1) % kSX], ((gm - 1) / kSX) & 1);
@@ -369,22 +456,43 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_q_kernel(const __gr
     for (uint32_t gd = 0; dc.left > 0; ++gd) {
       const int sp = gd % kSP;
       if (!mbar_wait(&bars->pk_full[sp], (gd / kSP) & 1, abort_flag, a.err, 301)) break;
-      const uint8_t* unit = ps + sp * kPStage + tile * (dc.bits == 3 ? 1536 : 1024);
-      uint32_t v[32];
-      uint32_t carry = 0;   // trellis state at the block start
-      if (dc.bits == 2) q2_half_i8(unit, r0, half, 0, v);
-      else if (!kAll || dc.bits == 3) q3_half_i8(unit, r0, half, 0, v);
-      else t2_half_i8(unit, r0, half, 0, v, carry);
-      // the A buffer is free once block gd - 1's MMAs are done
-      if (gd > 0 && !mbar_wait(&bars->mma_done[(gd - 1) % kSX], ((gd - 1) / kSX) & 1, abort_flag, a.err, 302)) break;
-      fence_after_sync();
-      tmem_st32(lane_base + kACol, v);
-      if (dc.bits == 2) q2_half_i8(unit, r0, half, 1, v);
-      else if (!kAll || dc.bits == 3) q3_half_i8(unit, r0, half, 1, v);
-      else t2_half_i8(unit, r0, half, 1, v, carry);
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->pk_empty[sp]);
-      tmem_st32(lane_base + kACol + 32, v);
+      if constexpr (kT) {
+        // ternary: four quarters of 20 columns (4 packed words, then 16 table entries), each
+        // stored as soon as it is decoded
+        const uint8_t* unit = ps + sp * C::kPStage + tile * 1024;
+        uint32_t raw[4], lv[16];
+        tern_quarter_i8(unit, r0, half, 0, tlut, lane, raw, lv);
+        // the A buffer is free once block gd - 1's MMAs are done
+        if (gd > 0 && !mbar_wait(&bars->mma_done[(gd - 1) % kSX], ((gd - 1) / kSX) & 1, abort_flag, a.err, 302)) break;
+        fence_after_sync();
+        tmem_st4(lane_base + C::kACol, raw);
+        tmem_st16(lane_base + C::kACol + 16, lv);
+#pragma unroll
+        for (int q = 1; q < 4; ++q) {
+          tern_quarter_i8(unit, r0, half, q, tlut, lane, raw, lv);
+          tmem_st4(lane_base + C::kACol + 4 * q, raw);
+          tmem_st16(lane_base + C::kACol + 16 + 16 * q, lv);
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->pk_empty[sp]);
+      } else {
+        const uint8_t* unit = ps + sp * C::kPStage + tile * (dc.bits == 3 ? 1536 : 1024);
+        uint32_t v[32];
+        uint32_t carry = 0;   // trellis state at the block start
+        if (dc.bits == 2) q2_half_i8(unit, r0, half, 0, v);
+        else if (!kAll || dc.bits == 3) q3_half_i8(unit, r0, half, 0, v);
+        else t2_half_i8(unit, r0, half, 0, v, carry);
+        // the A buffer is free once block gd - 1's MMAs are done
+        if (gd > 0 && !mbar_wait(&bars->mma_done[(gd - 1) % kSX], ((gd - 1) / kSX) & 1, abort_flag, a.err, 302)) break;
+        fence_after_sync();
+        tmem_st32(lane_base + C::kACol, v);
+        if (dc.bits == 2) q2_half_i8(unit, r0, half, 1, v);
+        else if (!kAll || dc.bits == 3) q3_half_i8(unit, r0, half, 1, v);
+        else t2_half_i8(unit, r0, half, 1, v, carry);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->pk_empty[sp]);
+        tmem_st32(lane_base + C::kACol + 32, v);
+      }
       tmem_wait_st();
       fence_before_sync();
       __syncwarp();
@@ -413,6 +521,10 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_q_kernel(const __gr
       const int n = c.rg * 128 + t;
       qv = 0;
       if (c.left <= 0 || n >= c.N) return (uint16_t)0;
+      if (kT) {   // ternary: alpha, one scale per row
+        qv = 1;
+        return __ldg(c.scales + n);
+      }
       if (!kAll || c.scale_q == nullptr) {
         qv = 1;
         return __ldg(c.scales + (int64_t)n * c.B + c.b);
@@ -441,12 +553,21 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_q_kernel(const __gr
       for (int c0 = 0; c0 < XR; c0 += kChunk) {
         if (c0 / 4 >= M) break;
         uint32_t d[kChunk];
-        tmem_ld_raw<kChunk>(lane_base + kDCol + (ge & 1) * kDCols + c0, d);
+        tmem_ld_raw<kChunk>(lane_base + C::kDCol + (ge & 1) * C::kDCols + c0, d);
         tmem_wait_ld_regs<kChunk>(d);
 #pragma unroll
         for (int mm = 0; mm < kChunk / 4; ++mm) {
           const int m = c0 / 4 + mm;
-          if (m < M) {
+          if (kT && m < M) {
+            // ternary: each limb sum plus its integer correction is exact; sum_j 256^j of those
+            // is sum_k t_k n_k, zero when every t of the block is zero
+            const int4 cr = rec[2 * m], ff = rec[2 * m + 1];
+            float v = (float)((int)d[4 * mm] + cr.x);
+            v = fmaf((float)((int)d[4 * mm + 1] + cr.y), 256.f, v);
+            v = fmaf((float)((int)d[4 * mm + 2] + cr.z), 65536.f, v);
+            v = fmaf((float)((int)d[4 * mm + 3] + cr.w), 16777216.f, v);
+            acc[m] = fmaf((s * __int_as_float(ff.y)) * v, __int_as_float(ff.x), acc[m]);
+          } else if (m < M) {
             const int4 c = rec[m];
             // 2 sum_j 256^j D_j + C in fp32 (each D_j is exact in fp32: |D_j| < 2^23)
             float v = fmaf((float)(int)d[4 * mm], 2.f, __int_as_float(c.x));
@@ -518,7 +639,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_q_kernel(const __gr
   fence_before_sync();
   __syncthreads();
   fence_after_sync();
-  if (warp == 9) tmem_dealloc(tmem, kTmemCols);
+  if (warp == 9) tmem_dealloc(tmem, C::kTmemCols);
 }
 
 // Preparation pass: one warp per (problem, block, token slot m < N/4). At the logical K position
@@ -607,47 +728,179 @@ __global__ void __launch_bounds__(256) prep_x_kernel(const __grid_constant__ Dec
   }
 }
 
+// Ternary preparation pass, with the rotation fused in: one warp per (problem, 320-trit unit b,
+// token slot m < N/4). The warp applies R = (1/sqrt(128)) H D to x (fp32, the sign mask first,
+// then a Walsh-Hadamard butterfly: lane l holds positions 4l .. 4l+3 of a 128-block) on the three
+// 128-blocks that the unit overlaps, keeps x' = R x in shared memory, and writes the B tile of the
+// unit in the K order of the decoded A columns (tern_quarter_i8): with E = exponent(max |x'| over
+// the unit) - 30 and n_k = x'_k / 2^E rounded to the nearest integer (|n| < 2^30),
+//   A column 4q + r, byte p        (v-slot of byte j = 4r + p of quarter q):  n_v = x'_(80q+5j+4) / (81 2^E), rounded
+//   A column 16 + 16q + j, byte d  (digit d of byte j of quarter q):           n_(80q+5j+d) - 3^d n_v(j)
+// each as four balanced signed limbs (B rows 4m + limb). Then the correction record of slot m:
+// {7 S_0, 7 S_1, 7 S_2, 7 S_3} (S_j = sum over the v-slots of limb j of n_v), then the two factors
+// of 2^E as in the 2/3-bit record. Every t_k x'_k then reaches the MMA exactly, up to the rounding
+// of n_k (half a unit of 2^E) and, for the fifth trit of a byte, of 81 n_v (40.5 units).
+__global__ void __launch_bounds__(256) prep_t_kernel(const __grid_constant__ DecArgs a, int total_blocks) {
+  __shared__ float xbuf[8][384];
+  const int lane = threadIdx.x & 31, wi = threadIdx.x >> 5;
+  const int M = a.M;
+  const int xrows = decode_xrows(M), slots = xrows >> 2;
+  const int w = blockIdx.x * 8 + wi;
+  if (w >= total_blocks * slots) return;
+  const int gblk = w / slots, m = w - gblk * slots;
+  int lo = 0, hi = a.count - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (a.prob[mid].xblk_base <= gblk) lo = mid;
+    else hi = mid - 1;
+  }
+  const DecProblem& pr = a.prob[lo];
+  const int b = gblk - pr.xblk_base;
+  uint8_t* dst = pr.xt + (int64_t)b * xtile_bytes(true, M);
+  float* xb = xbuf[wi];
+  const int64_t k0 = (int64_t)320 * b;
+  const int64_t hb0 = k0 / 128;   // first 128-block the unit overlaps; the unit starts 0 or 64 into it
+  const float inv = 0.08838834764831845f;   // 1/sqrt(128)
+#pragma unroll
+  for (int h = 0; h < 3; ++h) {
+    const int64_t kb = (hb0 + h) * 128;
+    float v[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int64_t k = kb + 4 * lane + i;
+      float xv = 0.f;
+      if (m < M && k < pr.K) {   // K is a multiple of 128: a 128-block is all in or all out
+        xv = __bfloat162float(__ushort_as_bfloat16(__ldg(pr.x + (int64_t)m * pr.K + k)));
+        if ((__ldg(pr.signs + (k >> 5)) >> (k & 31)) & 1u) xv = -xv;
+      }
+      v[i] = xv;
+    }
+    float t0 = v[0] + v[1], t1 = v[0] - v[1], t2 = v[2] + v[3], t3 = v[2] - v[3];
+    v[0] = t0 + t2; v[2] = t0 - t2; v[1] = t1 + t3; v[3] = t1 - t3;
+#pragma unroll
+    for (int sft = 1; sft < 32; sft <<= 1) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float o = __shfl_xor_sync(0xffffffffu, v[i], sft);
+        v[i] = (lane & sft) ? o - v[i] : v[i] + o;
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) xb[h * 128 + 4 * lane + i] = v[i] * inv;
+  }
+  __syncwarp();
+  const float* xu = xb + (int)(k0 - hb0 * 128);   // x' of unit position u = xu[u], u < 320
+  float amax = 0.f;
+#pragma unroll
+  for (int i = 0; i < 10; ++i) amax = fmaxf(amax, fabsf(xu[lane + 32 * i]));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  int ex = 0;
+  if (amax > 0.f) frexpf(amax, &ex);
+  const int E = ex - 30;
+  const bool live = amax > 0.f;
+  auto n_of = [&](int u) -> int { return live ? __float2int_rn(ldexpf(xu[u], -E)) : 0; };
+  auto nv_of = [&](int u) -> int { return live ? __double2int_rn(ldexp((double)xu[u], -E) / 81.0) : 0; };
+  int sv[4] = {0, 0, 0, 0};
+  for (int g = lane; g < 40; g += 32) {   // 8 consecutive K positions 8g .. 8g+7 of the tile
+    uint32_t lw[4][2] = {{0u, 0u}, {0u, 0u}, {0u, 0u}, {0u, 0u}};
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const int kl = 8 * g + e, col = kl >> 2, p = kl & 3;
+      int bv;
+      bool vslot;
+      if (col < 16) {
+        const int q = col >> 2, j = 4 * (col & 3) + p;
+        bv = nv_of(80 * q + 5 * j + 4);
+        vslot = true;
+      } else {
+        const int q = (col - 16) >> 4, j = (col - 16) & 15;
+        const int pw = p == 0 ? 1 : (p == 1 ? 3 : (p == 2 ? 9 : 27));
+        bv = n_of(80 * q + 5 * j + p) - pw * nv_of(80 * q + 5 * j + 4);
+        vslot = false;
+      }
+      int rest = bv;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int d = j < 3 ? (int)(int8_t)(rest & 0xFF) : rest;
+        rest = (rest - d) >> 8;
+        if (vslot) sv[j] += d;
+        lw[j][e >> 2] |= ((uint32_t)d & 0xFFu) << (8 * (e & 3));
+      }
+    }
+    const int atom = (8 * g) >> 7, within = (8 * g) & 127, chunk = within >> 4, off = within & 15;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int row = 4 * m + j;
+      *reinterpret_cast<uint2*>(dst + atom * xrows * 128 + row * 128 + ((chunk ^ (row & 7)) << 4) + off) =
+          make_uint2(lw[j][0], lw[j][1]);
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) sv[j] += __shfl_xor_sync(0xffffffffu, sv[j], o);
+  }
+  if (lane == 0) {
+    const int Ehi = max(E, -126);
+    const float f = (m < M && live) ? ldexpf(1.f, Ehi) : 0.f;
+    const float f2 = ldexpf(1.f, E - Ehi);
+    int4* rec = reinterpret_cast<int4*>(dst + 3 * xrows * 128);
+    rec[2 * m] = make_int4(7 * sv[0], 7 * sv[1], 7 * sv[2], 7 * sv[3]);
+    rec[2 * m + 1] = make_int4(__float_as_int(f), __float_as_int(f2), 0, 0);
+  }
+}
+
 }  // namespace
 
 cudaError_t launch_prep_x(const DecArgs& a, int total_blocks, cudaStream_t stream) {
   const int warps = total_blocks * (decode_xrows(a.M) >> 2);
-  prep_x_kernel<<<(warps + 7) / 8, 256, 0, stream>>>(a, total_blocks);
+  if (a.count > 0 && a.prob[0].bits == 1)
+    prep_t_kernel<<<(warps + 7) / 8, 256, 0, stream>>>(a, total_blocks);
+  else
+    prep_x_kernel<<<(warps + 7) / 8, 256, 0, stream>>>(a, total_blocks);
   return cudaGetLastError();
 }
 
 namespace {
-template <int XR, bool kAll>
+template <int XR, int MODE>
 cudaError_t launch_xr(const DecArgs& a, int grid, cudaStream_t stream) {
+  using C = Cfg<XR, MODE>;
   static bool set[64] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
   if (!set[dev]) {
-    cudaError_t e =
-        cudaFuncSetAttribute(gemv_q_kernel<XR, kAll>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
-    // all of the unified L1/shared array as shared memory, so that three CTAs fit
+    cudaError_t e = cudaFuncSetAttribute(gemv_q_kernel<XR, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+    // all of the unified L1/shared array as shared memory, so that the CTAs fit
     if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(gemv_q_kernel<XR, kAll>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+      e = cudaFuncSetAttribute(gemv_q_kernel<XR, MODE>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
     if (e != cudaSuccess) return e;
     set[dev] = true;
   }
-  gemv_q_kernel<XR, kAll><<<grid, kThreads, kSmem, stream>>>(a);
+  gemv_q_kernel<XR, MODE><<<grid, kThreads, C::kSmem, stream>>>(a);
   return cudaGetLastError();
 }
 
-template <bool kAll>
-cudaError_t launch_feat(const DecArgs& a, int grid, cudaStream_t stream) {
+template <int MODE>
+cudaError_t launch_mode(const DecArgs& a, int grid, cudaStream_t stream) {
   switch (decode_xrows(a.M)) {
-    case 8: return launch_xr<8, kAll>(a, grid, stream);
-    case 16: return launch_xr<16, kAll>(a, grid, stream);
-    default: return launch_xr<32, kAll>(a, grid, stream);
+    case 8: return launch_xr<8, MODE>(a, grid, stream);
+    case 16: return launch_xr<16, MODE>(a, grid, stream);
+    default: return launch_xr<32, MODE>(a, grid, stream);
   }
 }
 }  // namespace
 
+// A batch is either ternary (every problem) or 2/3-bit; the 2/3-bit form is chosen by whether
+// any problem is trellis-coded or has int8 block scales.
 cudaError_t launch_gemv_q(const DecArgs& a, int grid, cudaStream_t stream) {
+  if (a.count > 0 && a.prob[0].bits == 1) return launch_mode<kModeTern>(a, grid, stream);
   bool all = false;
   for (int i = 0; i < a.count; ++i) all = all || a.prob[i].bits == WR_FMT_T2 || a.prob[i].scale_q != nullptr;
-  return all ? launch_feat<true>(a, grid, stream) : launch_feat<false>(a, grid, stream);
+  return all ? launch_mode<kModeAll>(a, grid, stream) : launch_mode<kModeLean>(a, grid, stream);
 }
+
+// CTAs of one wave of the decode kernel for a batch of this kind on a 148-SM part.
+int decode_ctas_per_sm(bool ternary, int M) { return ternary && decode_xrows(M) > 8 ? 2 : 3; }
 
 }  // namespace wr

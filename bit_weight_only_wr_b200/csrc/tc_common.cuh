@@ -185,6 +185,11 @@ __host__ __device__ constexpr uint32_t idesc_i8_m128(int n) {
   return (2u << 4) | (0u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
 }
 
+// The same with A signed int8 (B signed int8).
+__host__ __device__ constexpr uint32_t idesc_i8s_m128(int n) {
+  return (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
+}
+
 // D[tmem] (+)= A[tmem] * B[smem] with 8-bit integers (K = 32 per instruction).
 __device__ __forceinline__ void mma_ts_i8(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
                                           uint32_t accumulate) {

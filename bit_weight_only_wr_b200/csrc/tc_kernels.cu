@@ -530,22 +530,23 @@ cudaError_t launch_tc(const TcArgs& a, const void* x_act, int64_t x_rows, int64_
   return cudaGetLastError();
 }
 
-// R x for the ternary path: one warp per (token, 128-block). x' = (1/sqrt(128)) H (d * x) in
-// fp32, split into hi = bf16(x') and lo = bf16(x' - hi). Inside each 320-trit unit, position
-// 80q + 2P + h holds trit 80q + 5*(2*(P/5) + h) + P%5 (pair P of byte pair P/5; h selects the
-// byte): the K order of the decoded A columns. Pad trits get 0. Two output forms:
-//   tiles (decode GEMV): the B tiles its copy warp loads, per unit 5 atoms of 64 positions and
-//     16 rows (2048 B), hi of token m in row m, lo in row 8 + m (128-byte swizzle: 16-byte chunk
-//     c of row r at c ^ (r % 8));
-//   planes (prefill GEMM): [2][M][Kp] bf16 row-major, hi then lo, read by TMA.
-// One warp: token m, 128-block starting at k0 (lane = 4 consecutive K positions).
-// The planes form scales token m by 2^-tok_ex[m] first (exact), so that its hi and lo parts stay
-// in bf16's normal range whatever the magnitude of x; the GEMM epilogue multiplies the token's
-// results by 2^tok_ex[m].
-template <bool PLANES>
-__device__ __forceinline__ void rotate_block(const uint16_t* __restrict__ x, const uint32_t* __restrict__ signs,
-                                             uint8_t* __restrict__ xt, int M, int K, int64_t Kp, int m, int64_t k0,
-                                             int lane, int scale_ex = 0) {
+// R x for the ternary prefill GEMM: one warp per (token, 128-block). x' = (1/sqrt(128)) H (d * x)
+// in fp32, token m scaled first by 2^-tok_ex[m] (exact) so that its hi and lo parts stay in bf16's
+// normal range whatever the magnitude of x (the GEMM epilogue multiplies the token's results by
+// 2^tok_ex[m]); then split into hi = bf16(x') and lo = bf16(x' - hi). Inside each 320-trit unit,
+// position 80q + 2P + h holds trit 80q + 5*(2*(P/5) + h) + P%5 (pair P of byte pair P/5; h
+// selects the byte): the K order of the decoded A columns. Pad trits get 0. The planes are
+// [2][M][Kp] bf16 row-major, hi then lo, read by TMA. Lane l holds K positions 4l .. 4l+3.
+__global__ void rotate_planes_kernel(const uint16_t* __restrict__ x, const uint32_t* __restrict__ signs,
+                                     uint8_t* __restrict__ planes, int M, int K, int64_t Kp,
+                                     const int* __restrict__ tok_ex) {
+  const int lane = threadIdx.x & 31;
+  const int64_t item = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int64_t nblk = (Kp + 127) / 128;
+  if (item >= (int64_t)M * nblk) return;
+  const int m = (int)(item / nblk);
+  const int64_t k0 = (item % nblk) * 128;
+  const int scale_ex = tok_ex[m];
   float v[4];
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
@@ -554,7 +555,7 @@ __device__ __forceinline__ void rotate_block(const uint16_t* __restrict__ x, con
     if (k < K) {
       xv = __bfloat162float(__ushort_as_bfloat16(x[(int64_t)m * K + k]));
       if ((signs[k >> 5] >> (k & 31)) & 1u) xv = -xv;
-      if (PLANES) xv = ldexpf(xv, -scale_ex);
+      xv = ldexpf(xv, -scale_ex);
     }
     v[i] = xv;
   }
@@ -580,40 +581,11 @@ __device__ __forceinline__ void rotate_block(const uint16_t* __restrict__ x, con
     const int kk = (int)(k % 320), q = kk / 80, i80 = kk % 80, beta = i80 / 5, dig = i80 % 5;
     const int P = 5 * (beta >> 1) + dig;
     const int kp = 80 * q + 2 * P + (beta & 1);
-    if (PLANES) {
-      uint16_t* pl = reinterpret_cast<uint16_t*>(xt);
-      const int64_t off = (int64_t)m * Kp + u * 320 + kp;
-      pl[off] = __bfloat16_as_ushort(hi);
-      pl[(int64_t)M * Kp + off] = __bfloat16_as_ushort(lo);
-    } else {
-      const int at = kp >> 6, e = kp & 63;
-      const int64_t off = u * (5 * 2048) + at * 2048 + m * 128 + ((((e >> 3) ^ (m & 7)) << 4) | ((e & 7) << 1));
-      *reinterpret_cast<uint16_t*>(xt + off) = __bfloat16_as_ushort(hi);                 // row m
-      *reinterpret_cast<uint16_t*>(xt + off + 1024) = __bfloat16_as_ushort(lo);          // row 8 + m
-    }
+    uint16_t* pl = reinterpret_cast<uint16_t*>(planes);
+    const int64_t off = (int64_t)m * Kp + u * 320 + kp;
+    pl[off] = __bfloat16_as_ushort(hi);
+    pl[(int64_t)M * Kp + off] = __bfloat16_as_ushort(lo);
   }
-}
-
-__global__ void rotate_x_kernel(const uint16_t* __restrict__ x, const uint32_t* __restrict__ signs,
-                                uint8_t* __restrict__ xt, int M, int K, int64_t Kp) {
-  const int lane = threadIdx.x & 31;
-  const int64_t item = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  const int64_t nblk = (Kp + 127) / 128;
-  if (item >= (int64_t)M * nblk) return;
-  rotate_block<false>(x, signs, xt, M, K, Kp, (int)(item / nblk), (item % nblk) * 128, lane);
-}
-
-// The planes form, for the prefill GEMM: planes = [2][M][Kp] bf16 (hi, lo), token m scaled by
-// 2^-tok_ex[m].
-__global__ void rotate_planes_kernel(const uint16_t* __restrict__ x, const uint32_t* __restrict__ signs,
-                                     uint8_t* __restrict__ planes, int M, int K, int64_t Kp,
-                                     const int* __restrict__ tok_ex) {
-  const int lane = threadIdx.x & 31;
-  const int64_t item = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  const int64_t nblk = (Kp + 127) / 128;
-  if (item >= (int64_t)M * nblk) return;
-  const int m = (int)(item / nblk);
-  rotate_block<true>(x, signs, planes, M, K, Kp, m, (item % nblk) * 128, lane, tok_ex[m]);
 }
 
 // Per-token exponent of the ternary prefill GEMM: tok_ex[m] = e with max_k |x[m,k]| in
@@ -630,22 +602,6 @@ __global__ void token_exponent_kernel(const uint16_t* __restrict__ x, int M, int
   int ex = 0;
   if (amax > 0.f) frexpf(amax, &ex);
   if (lane == 0) tok_ex[m] = ex;
-}
-
-// Batched form: work item g -> (problem, token, 128-block) through the problems' first items.
-__global__ void rotate_x_batched_kernel(const __grid_constant__ DecArgs a, int64_t total_items) {
-  const int lane = threadIdx.x & 31;
-  const int64_t g = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  if (g >= total_items) return;
-  int lo = 0, hi = a.count - 1;
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (a.prob[mid].xblk_base <= g) lo = mid;
-    else hi = mid - 1;
-  }
-  const DecProblem& pr = a.prob[lo];
-  const int64_t local = g - pr.xblk_base, nblk = ((int64_t)pr.Kp + 127) / 128;
-  rotate_block<false>(pr.x, pr.signs, pr.xt, 0, pr.K, pr.Kp, (int)(local / nblk), (local % nblk) * 128, lane);
 }
 
 // Failure-path self-test: warp 0 waits on a barrier nobody arrives on until the bounded wait
@@ -684,15 +640,6 @@ cudaError_t launch_tc_kernel(int fmt, int bn, const TcArgs& a, const void* x_act
   return cudaErrorNotSupported;
 }
 
-cudaError_t launch_rotate_x(const uint16_t* x, const uint32_t* signs, uint8_t* xt, int M, int K, int64_t Kp,
-                            cudaStream_t stream) {
-  const int64_t items = (int64_t)M * ((Kp + 127) / 128);
-  const int warps = 8;
-  const int64_t ctas = (items + warps - 1) / warps;
-  rotate_x_kernel<<<(unsigned)ctas, warps * 32, 0, stream>>>(x, signs, xt, M, K, Kp);
-  return cudaGetLastError();
-}
-
 cudaError_t launch_rotate_planes(const uint16_t* x, const uint32_t* signs, uint8_t* planes, int M, int K, int64_t Kp,
                                  int* tok_ex, cudaStream_t stream) {
   const int warps = 8;
@@ -700,12 +647,6 @@ cudaError_t launch_rotate_planes(const uint16_t* x, const uint32_t* signs, uint8
   const int64_t items = (int64_t)M * ((Kp + 127) / 128);
   rotate_planes_kernel<<<(unsigned)((items + warps - 1) / warps), warps * 32, 0, stream>>>(x, signs, planes, M, K, Kp,
                                                                                          tok_ex);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_rotate_x_batched(const DecArgs& a, int64_t total_items, cudaStream_t stream) {
-  const int warps = 8;
-  rotate_x_batched_kernel<<<(unsigned)((total_items + warps - 1) / warps), warps * 32, 0, stream>>>(a, total_items);
   return cudaGetLastError();
 }
 

@@ -26,21 +26,18 @@ struct TcArgs {
 constexpr int kMaxDecodeProblems = 256;
 
 struct DecProblem {
-  const uint16_t* x;         // bf16 [M, K] activations (Q2/Q3; read by the preparation pass)
+  const uint16_t* x;         // bf16 [M, K] activations (read by the preparation pass)
   uint8_t* xt;               // prepared activation tiles of this problem (workspace), one per block
   const uint8_t* packed;     // packed units, tile-major
   const uint16_t* scales;    // fp16 [N, K/256] (Q2/Q3) or alpha [N] (ternary); d [N] with scale_q
   const int8_t* scale_q;     // int8 [N, K/256] block multipliers (s = d q), or null: fp16 scales
   float* y;                  // fp32 [M, N]
   const uint32_t* signs;     // ternary: random-sign mask of the rotation
-  int64_t partial_base;      // first partial float of this problem (ternary items)
-  int64_t block_base;        // first block of this problem in the batch's block sequence (2/3-bit)
+  int64_t block_base;        // first block of this problem in the batch's block sequence
   int64_t cost_base;         // cost (block_cost units) of the batch's blocks before this problem
-  int N, K, Kp;              // Kp: padded K of the ternary planes
-  int B, RG, P, bits;        // blocks per row, 128-row groups, K splits, 2/3/T2 (ternary: 1)
-  int item_base;             // first work item of this problem
-  int xblk_base;             // 2/3-bit: first block of this problem in the preparation pass;
-                             // ternary: first rotation work item (token, 128-block) of it
+  int N, K, Kp;              // Kp: padded K (ternary: a multiple of the 320-trit unit)
+  int B, RG, bits;           // blocks per row, 128-row groups, 2/3/T2 (ternary: 1)
+  int xblk_base;             // first block (K unit) of this problem in the preparation pass
   int counter_base;          // first arrival counter (row group) of this problem
 };
 
@@ -50,19 +47,18 @@ struct DecProblem {
 // the format grows with M). The block ranges of the CTAs are cut by this cost so that they
 // finish together; the ratios are the best of a sweep on the 36-layer body.
 __host__ __device__ inline int64_t block_cost(int bits, int M) {
-  return bits == 2 ? 20 : (M <= 2 ? 26 : (M <= 4 ? 25 : 24));
+  return bits == 2 ? 20 : (bits == 1 ? 32 : (M <= 2 ? 26 : (M <= 4 ? 25 : 24)));
 }
 
-// 2/3-bit: the batch's blocks (problem by problem, row group by row group, K block by K block)
-// are cut into gridDim.x contiguous ranges, one per CTA: CTA c takes the blocks whose cost
-// before them (in block_cost units) lies in [c C / G, (c+1) C / G).
-// A row group cut by a range boundary is finished through per-CTA partial slots (two per CTA:
-// the row group that started before the range, and the one that ends after it).
-// Ternary: work items (problem, row group, range of blocks), items c, c + G, ... per CTA.
+// The batch's blocks (problem by problem, row group by row group, K block by K block) are cut
+// into gridDim.x contiguous ranges, one per CTA: CTA c takes the blocks whose cost before them
+// (in block_cost units) lies in [c C / G, (c+1) C / G). A row group cut by a range boundary is
+// finished through per-CTA partial slots (two per CTA: the row group that started before the
+// range, and the one that ends after it). A batch is all ternary or all 2/3-bit.
 struct DecArgs {
-  int count, M, items, pad;
-  int64_t total;             // 2/3-bit: blocks of the batch (T)
-  int64_t total_cost;        // 2/3-bit: their summed block_cost (C)
+  int count, M;
+  int64_t total;             // blocks of the batch (T)
+  int64_t total_cost;        // their summed block_cost (C)
   float* partial;
   int* counter;
   int* err;
@@ -99,35 +95,31 @@ __host__ __device__ inline int range_cta_of(const DecArgs& a, int G, const DecPr
   return (int)(((x + 1) * G - 1) / a.total_cost);
 }
 
-// 2/3-bit decode: the preparation pass writes the B tiles, then the GEMV kernel.
+// Decode GEMV: the preparation pass writes the B tiles (for a ternary batch it applies the
+// rotation first), then the GEMV kernel.
 cudaError_t launch_prep_x(const DecArgs& a, int total_blocks, cudaStream_t stream);
 cudaError_t launch_gemv_q(const DecArgs& a, int grid, cudaStream_t stream);
-// Ternary decode (tiles written by launch_rotate_x).
-cudaError_t launch_gemv_t(const DecArgs& a, int grid, cudaStream_t stream);
+// CTAs that one SM holds of the decode GEMV kernel for this kind of batch.
+int decode_ctas_per_sm(bool ternary, int M);
 
 // One prepared activation tile per block, stored as the exact image of a shared-memory B stage
-// so that one bulk copy moves it (128-byte swizzle: 16-byte chunk c of a row r at c ^ (r % 8)).
-// 2/3-bit (integer path): two atoms of 128 K positions x xrows rows of int8, limb j of token
-// slot m in row 4m + j, then 256 bytes of corrections: 2^E per slot (8 floats) and per slot and
-// limb 0x4B400000 - L S_j (8 x 4 int32). xrows = 8, 16 or 32 for M <= 2, 4, 8 (the MMA's N).
-// Ternary: 5 atoms of 64 K positions x 16 rows of bf16, hi of token m in row m, lo in 8 + m.
+// so that one bulk copy moves it (128-byte swizzle: 16-byte chunk c of a row r at c ^ (r % 8)):
+// atoms of 128 K positions x xrows rows of int8, limb j of token slot m in row 4m + j (two atoms
+// for a 256-code block, three for a 320-trit unit, the last half used), then a 256-byte
+// correction record (per slot: 2/3-bit {C, f, f2, 0}; ternary {4 limb corrections}, {f, f2, 0, 0}).
+// xrows = 8, 16 or 32 for M <= 2, 4, 8 (the MMA's N).
 __host__ __device__ inline int decode_xrows(int M) { return M <= 2 ? 8 : (M <= 4 ? 16 : 32); }
 __host__ __device__ inline int64_t xtile_bytes(bool ternary, int M) {
-  return ternary ? (int64_t)5 * 2048 : (int64_t)2 * decode_xrows(M) * 128 + 256;
+  return (int64_t)(ternary ? 3 : 2) * decode_xrows(M) * 128 + 256;
 }
 
 cudaError_t launch_tc_kernel(int fmt, int bn, const TcArgs& a, const void* x_act, int64_t x_rows, int64_t x_k,
                              int grid, cudaStream_t stream);
-cudaError_t launch_rotate_x(const uint16_t* x, const uint32_t* signs, uint8_t* xt, int M, int K, int64_t Kp,
-                            cudaStream_t stream);
-// The same for every problem of a batch (x, signs, xt, K, Kp per problem; xblk_base = first
-// work item; total_items = M * sum of ceil(Kp / 128)).
 // R x as two bf16 planes [2][M][Kp] (hi, lo) in the decoded K order, for the prefill GEMM.
 // Token m is scaled by 2^-tok_ex[m] (tok_ex [M] int, written first by a per-token pass: the
 // exponent of the token's largest |x|), so that tiny and huge tokens keep full precision.
 cudaError_t launch_rotate_planes(const uint16_t* x, const uint32_t* signs, uint8_t* planes, int M, int K, int64_t Kp,
                                  int* tok_ex, cudaStream_t stream);
-cudaError_t launch_rotate_x_batched(const DecArgs& a, int64_t total_items, cudaStream_t stream);
 // Device quantizer + packer for the 2/3-bit odd grid (quantize.cu). scale_q null: fp16 block
 // scales [N, K/256] in `scales`; else the int8 form: fp16 row scales d [N] in `scales` and the
 // int8 multipliers [N, K/256] in scale_q.
