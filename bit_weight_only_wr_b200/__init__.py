@@ -65,7 +65,7 @@ _SIGNATURES = {
     "wr_gemv": (_c_int, [_c_i64, _c_i64, _c_i64, _vp, _vp, _vp, _c_int, _c_int, _vp, _vp, _c_size, _vp]),
     "wr_gemv_batched_workspace_bytes": (_c_size, [_c_i64, ctypes.c_int32, _PROBLEMS]),
     "wr_gemv_batched": (_c_int, [_c_i64, ctypes.c_int32, _PROBLEMS, _vp, _c_size, _vp]),
-    "wr_gemv_batched_plan": (_c_int, [_c_i64, ctypes.c_int32, _PROBLEMS, _vp, _vp, ctypes.c_int32]),
+    "wr_gemv_batched_plan": (_c_int, [_c_i64, ctypes.c_int32, _PROBLEMS, _vp, _vp, ctypes.c_int32, _vp]),
     "wr_gemm_workspace_bytes": (_c_size, [_c_i64, _c_i64, _c_i64, _c_int]),
     "wr_gemm": (_c_int, [_c_i64, _c_i64, _c_i64, _vp, _vp, _vp, _c_int, _c_int, _vp, _vp, _c_size, _vp]),
     "wr_gemm_ternary_workspace_bytes": (_c_size, [_c_i64, _c_i64, _c_i64]),
@@ -237,15 +237,17 @@ def wr_gemv_batched_workspace_bytes(M: int, problems) -> int:
 
 
 def wr_gemv_batched_plan(M: int, problems):
-    """(grid, range_starts int64 [grid + 1]): the CTA block ranges of one batched decode launch
-    (problems as for wr_gemv_batched; only their shapes and formats are read)."""
+    """(grid, range_starts int64 [grid + 1], block_costs int64 [count]): the CTA block ranges of
+    one batched decode launch and the per-problem block cost they were cut by (problems as for
+    wr_gemv_batched; only their shapes and formats are read)."""
     arr = problems if isinstance(problems, ctypes.Array) else _problems(problems)
     grid = ctypes.c_int32(0)
-    _check("wr_gemv_batched_plan", _lib.wr_gemv_batched_plan(M, len(arr), arr, ctypes.addressof(grid), None, 0))
+    _check("wr_gemv_batched_plan", _lib.wr_gemv_batched_plan(M, len(arr), arr, ctypes.addressof(grid), None, 0, None))
     starts = np.zeros(grid.value + 1, dtype=np.int64)
+    costs = np.zeros(len(arr), dtype=np.int64)
     _check("wr_gemv_batched_plan", _lib.wr_gemv_batched_plan(M, len(arr), arr, ctypes.addressof(grid),
-                                                             _ptr(starts), grid.value + 1))
-    return grid.value, starts
+                                                             _ptr(starts), grid.value + 1, _ptr(costs)))
+    return grid.value, starts, costs
 
 
 def wr_gemv_batched(M: int, problems, workspace, workspace_bytes: int, stream=None) -> None:

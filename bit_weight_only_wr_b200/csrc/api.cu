@@ -377,12 +377,19 @@ wr_status wr_gemv_noalloc(int64_t M, int64_t N, int64_t K, const uint16_t* x, co
   return run_q(bits, M, N, K, x, packed, scales, scale_q, y, scratch, s);
 }
 
+// Shape and format of one batched problem (what the plan reads); the batched call also checks
+// its pointers.
+static wr_status problem_shape_ok(int64_t M, const wr_gemv_problem& pr) {
+  QFmt f{};
+  if (!split_fmt(pr.bits, true, &f)) return WR_ERR_UNSUPPORTED;
+  if (pr.reserved != 0 || check_dims(M, pr.N, pr.K) != WR_OK || pr.K % 256 != 0) return WR_ERR_INVALID_ARG;
+  return WR_OK;
+}
+
 static bool batch_ok(int64_t M, int32_t count, const wr_gemv_problem* pr) {
   if (M < 1 || M > 8 || count < 1 || !pr) return false;
   for (int i = 0; i < count; ++i) {
-    QFmt f{};
-    if (!split_fmt(pr[i].bits, true, &f)) return false;
-    if (pr[i].reserved != 0 || check_dims(M, pr[i].N, pr[i].K) != WR_OK || pr[i].K % 256 != 0) return false;
+    if (problem_shape_ok(M, pr[i]) != WR_OK) return false;
     if (!aligned16(pr[i].x) || !aligned16(pr[i].packed) || !aligned16(pr[i].scales) || !aligned16(pr[i].y))
       return false;
   }
@@ -390,14 +397,13 @@ static bool batch_ok(int64_t M, int32_t count, const wr_gemv_problem* pr) {
 }
 
 wr_status wr_gemv_batched_plan(int64_t M, int32_t count, const wr_gemv_problem* problems, int32_t* grid,
-                               int64_t* range_starts, int32_t range_starts_len) {
+                               int64_t* range_starts, int32_t range_starts_len, int64_t* block_costs) {
   if (M < 1 || M > 8 || count < 1 || count > wr::kMaxDecodeProblems || !problems || !grid) return WR_ERR_INVALID_ARG;
   ProblemShape sh[wr::kMaxDecodeProblems];
   for (int i = 0; i < count; ++i) {
-    QFmt f{};
-    if (!split_fmt(problems[i].bits, true, &f)) return WR_ERR_UNSUPPORTED;
-    if (check_dims(M, problems[i].N, problems[i].K) != WR_OK || problems[i].K % 256 != 0) return WR_ERR_INVALID_ARG;
-    sh[i] = ProblemShape{problems[i].N, problems[i].K, f.base};
+    const wr_status st = problem_shape_ok(M, problems[i]);
+    if (st != WR_OK) return st;
+    sh[i] = ProblemShape{problems[i].N, problems[i].K, problems[i].bits & ~WR_SCALES_I8};
   }
   static thread_local DecodePlan dp;
   plan_decode(M, count, sh, &dp);
@@ -406,6 +412,8 @@ wr_status wr_gemv_batched_plan(int64_t M, int32_t count, const wr_gemv_problem* 
     if (range_starts_len < dp.grid + 1) return WR_ERR_INVALID_ARG;
     for (int c = 0; c <= dp.grid; ++c) range_starts[c] = wr::range_start(dp.args, dp.grid, c);
   }
+  if (block_costs)
+    for (int i = 0; i < count; ++i) block_costs[i] = wr::block_cost(dp.args.prob[i].bits, (int)M);
   return WR_OK;
 }
 

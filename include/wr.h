@@ -214,9 +214,12 @@ size_t wr_gemv_batched_workspace_bytes(int64_t M, int32_t count, const wr_gemv_p
  * first block of each CTA's range in the batch's block sequence (problem by problem, 128-row
  * group by row group, 256-code block by block), then the total block count. Ranges are cut by
  * an estimated cost per block (a 3-bit or trellis block weighs more than a 2-bit one) and each
- * holds at least one block. Only the shapes and formats of problems_host are read. */
+ * holds at least one block; if block_costs is not NULL it receives that cost for each problem
+ * (count entries, in the units the split uses). Only the shapes and formats of problems_host are
+ * read (pointers may be NULL); a problem that wr_gemv_batched would reject for its shape, format
+ * or reserved field is rejected with the same status. */
 wr_status wr_gemv_batched_plan(int64_t M, int32_t count, const wr_gemv_problem* problems_host, int32_t* grid,
-                               int64_t* range_starts, int32_t range_starts_len);
+                               int64_t* range_starts, int32_t range_starts_len, int64_t* block_costs);
 wr_status wr_gemv_batched(int64_t M, int32_t count, const wr_gemv_problem* problems_host, void* workspace,
                           size_t workspace_bytes, void* stream);
 

@@ -187,28 +187,47 @@ def test_device_calls_reject_bad_arguments_before_launch():
     assert wr.wr_gemv_workspace_bytes(1, 16, 256, 2) > 0
 
 
-def _block_cost(fmt, M):
-    """Relative cost of one 128 x 256 block in the decode GEMV's work split, as include/wr.h and
-    the launch describe it: a 3-bit or trellis block weighs more than a 2-bit one."""
-    base = fmt & ~wr.WR_SCALES_I8
-    return 20 if base == 2 else (26 if M <= 2 else (25 if M <= 4 else 24))
-
-
 def _check_plan(M, shapes):
+    """The ranges partition the batch's blocks, none is empty, and each range's cost (in the
+    per-problem block costs the library reports) is within one block of C / G."""
     probs = [(None, None, None, None, N, K, fmt) for (N, K, fmt) in shapes]
-    G, starts = wr.wr_gemv_batched_plan(M, probs)
+    G, starts, pcost = wr.wr_gemv_batched_plan(M, probs)
+    assert np.all(pcost > 0)
     costs = []
-    for N, K, fmt in shapes:
-        costs += [_block_cost(fmt, M)] * (((N + 127) // 128) * (K // 256))
+    for (N, K, fmt), c in zip(shapes, pcost):
+        costs += [int(c)] * (((N + 127) // 128) * (K // 256))
     T = len(costs)
     assert 1 <= G <= 444 and starts[0] == 0 and starts[G] == T
     assert np.all(np.diff(starts) >= 1), "every CTA range holds at least one block"
-    # the ranges partition the blocks by cost: each range's cost is within one block of C / G
     cum = np.concatenate([[0], np.cumsum(costs)])
     rc = cum[starts[1:]] - cum[starts[:-1]]
     C, wmax = cum[-1], max(costs)
     assert np.all(rc <= C / G + wmax) and np.all(rc >= C / G - wmax)
     return G, starts
+
+
+def test_decode_plan_block_costs_order():
+    # a 3-bit or trellis block is the longer one to decode; int8 scales do not change the cost
+    probs = [(None, None, None, None, 128, 256, f) for f in (2, 3, wr.WR_FMT_T2, 2 | wr.WR_SCALES_I8)]
+    for M in (1, 4, 8):
+        _, _, c = wr.wr_gemv_batched_plan(M, probs)
+        assert c[1] > c[0] and c[2] == c[1] and c[3] == c[0]
+
+
+def test_decode_plan_rejects_what_the_batched_call_rejects():
+    bad = wr._problems([(16, 16, 16, 16, 16, 256, 2)])
+    bad[0].reserved = 1
+    with pytest.raises(wr.WrError) as e:
+        wr.wr_gemv_batched_plan(1, bad)
+    assert e.value.status == 1
+    assert wr._lib.wr_gemv_batched(1, 1, bad, 16, 1 << 20, None) == 1
+    for fields, status in (((16, 300, 2), 1), ((16, 256, 5), 2), ((0, 256, 2), 1)):
+        N, K, fmt = fields
+        p = wr._problems([(16, 16, 16, 16, N, K, fmt)])
+        with pytest.raises(wr.WrError) as e:
+            wr.wr_gemv_batched_plan(1, p)
+        assert e.value.status == status
+        assert wr._lib.wr_gemv_batched(1, 1, p, 16, 1 << 20, None) != 0
 
 
 def test_decode_plan_of_the_qwen3_body():
