@@ -370,6 +370,36 @@ def main():
                           "d2h": y_all.numel() * 4}
         return out
 
+    def dependent_body_run(M, steps, warmup):
+        """The body as a decoder whose layers depend on each other issues it: per layer four
+        calls in order, each a wr_gemv_grouped over the linears that read one input (q/k/v on the
+        attention input, o, gate/up on the MLP input, down), with fresh seeded inputs standing in
+        for the outputs of attention and the MLP activation; no launch spans two layers."""
+        groups = [("qkv", (0, 1, 2)), ("o", (3,)), ("gate_up", (4, 5)), ("down", (6,))]
+        calls, keep, nbytes, nb = [], [], 0, 0
+        for layer in range(args.layers):
+            lm = mods[7 * layer:7 * layer + 7]
+            for gi, (gname, idxs) in enumerate(groups):
+                K = lm[idxs[0]]["K"]
+                x = torch.from_numpy(wr_synth.activations_bf16(20_000 + 10 * layer + gi, M, K).view(np.int16)).cuda()
+                ys = [torch.empty(M, lm[i]["N"], dtype=torch.float32, device="cuda") for i in idxs]
+                arr = wr._gitems([(lm[i]["packed"], lm[i]["scales"], y, lm[i]["N"], lm[i]["bits"])
+                                  for i, y in zip(idxs, ys)])
+                nb = max(nb, wr.wr_gemv_grouped_workspace_bytes(M, K, arr))
+                calls.append((K, x, arr))
+                keep += ys
+                nbytes += 2 * M * K + sum(wr.wr_packed_bytes(lm[i]["bits"], lm[i]["N"], K) + lm[i]["N"] * (K // 256) * 2
+                                          + 4 * M * lm[i]["N"] for i in idxs)
+        ws = torch.zeros(nb, dtype=torch.uint8, device="cuda")
+
+        def step():
+            for K, x, arr in calls:
+                wr.wr_gemv_grouped(M, K, x, arr, ws, nb)
+        ms = graph_time_ms(torch, step, steps, warmup, stream, dist) / steps
+        ms = max_over_ranks(torch, dist, ms)
+        return {"ms": ms, "bytes": nbytes, "gbs": nbytes / ms / 1e6, "frac_of_hbm": nbytes / ms / 1e6 / hbm_peak,
+                "tokens_per_s": M * 1e3 / ms, "calls": len(calls), "launches": 2 * len(calls)}
+
     with ClockSampler(uuid) as clk:
         head = body_run(args.tokens, args.steps, args.warmup, True)
     clocks = clk.summary()
@@ -387,6 +417,11 @@ def main():
             extras["body_m1_one_call_per_linear"] = body_run(1, max(5, args.steps // 2), 3, False, batched=False)
         except Exception as e:  # noqa: BLE001
             extras["body_m1_one_call_per_linear"] = {"error": repr(e)}
+        for M in (1, 8):
+            try:
+                extras[f"body_dependent_grouped_m{M}"] = dependent_body_run(M, max(5, args.steps // 2), 3)
+            except Exception as e:  # noqa: BLE001
+                extras[f"body_dependent_grouped_m{M}"] = {"error": repr(e)}
         extras.update(run_extras(args, wr, torch, np, stream, dist, hbm_peak, bf16_peak))
 
     # the step is one wr_gemv_batched call: the preparation pass, then one launch of the decode

@@ -21,7 +21,7 @@ __all__ = [
     "wr_gemv_batched", "wr_gemv_noalloc", "WR_GEMV_NOALLOC_SCRATCH_BYTES", "WrGemvTernaryProblem",
     "wr_gemv_ternary_batched_workspace_bytes", "wr_gemv_ternary_batched", "wr_selftest_wait_timeout",
     "wr_quantize_pack", "wr_quantize_trellis", "WR_FMT_T2", "WR_SCALES_I8", "wr_scales_bytes",
-    "wr_gemv_batched_plan",
+    "wr_gemv_batched_plan", "WrGemvGroupItem", "wr_gemv_grouped_workspace_bytes", "wr_gemv_grouped",
 ]
 
 WR_FMT_TERNARY, WR_FMT_Q2, WR_FMT_Q3, WR_FMT_T2 = 1, 2, 3, 4
@@ -50,6 +50,15 @@ class WrGemvTernaryProblem(ctypes.Structure):
 
 _TPROBLEMS = ctypes.POINTER(WrGemvTernaryProblem)
 
+
+class WrGemvGroupItem(ctypes.Structure):
+    """Mirror of the C struct wr_gemv_group_item."""
+    _fields_ = [("packed", ctypes.c_void_p), ("scales", ctypes.c_void_p), ("y", ctypes.c_void_p),
+                ("N", ctypes.c_int64), ("bits", ctypes.c_int32), ("reserved", ctypes.c_int32)]
+
+
+_GITEMS = ctypes.POINTER(WrGemvGroupItem)
+
 _SIGNATURES = {
     "wr_abi_version": (_c_int, []),
     "wr_status_string": (ctypes.c_char_p, [_c_int]),
@@ -71,6 +80,8 @@ _SIGNATURES = {
     "wr_gemm_ternary_workspace_bytes": (_c_size, [_c_i64, _c_i64, _c_i64]),
     "wr_gemm_ternary": (_c_int, [_c_i64, _c_i64, _c_i64, _vp, _vp, _vp, _vp, _vp, _vp, _c_size, _vp]),
     "wr_get_device_error": (_c_int, [_vp]),
+    "wr_gemv_grouped_workspace_bytes": (_c_size, [_c_i64, _c_i64, ctypes.c_int32, _GITEMS]),
+    "wr_gemv_grouped": (_c_int, [_c_i64, _c_i64, _vp, ctypes.c_int32, _GITEMS, _vp, _c_size, _vp]),
     "wr_selftest_wait_timeout": (_c_int, [_vp]),
     "wr_quantize_pack": (_c_int, [_c_int, _c_i64, _c_i64, _vp, _vp, _vp, _vp]),
     "wr_gemv_noalloc": (_c_int, [_c_i64, _c_i64, _c_i64, _vp, _vp, _vp, _c_int, _c_int, _vp, _vp]),
@@ -255,6 +266,26 @@ def wr_gemv_batched(M: int, problems, workspace, workspace_bytes: int, stream=No
     arr = problems if isinstance(problems, ctypes.Array) else _problems(problems)
     _check("wr_gemv_batched", _lib.wr_gemv_batched(M, len(arr), arr, _ptr(workspace), workspace_bytes,
                                                    _stream(stream)))
+
+
+def _gitems(items):
+    """items: sequence of (packed, scales, y, N, bits) -> ctypes array."""
+    arr = (WrGemvGroupItem * len(items))()
+    for i, (packed, scales, y, N, bits) in enumerate(items):
+        arr[i] = WrGemvGroupItem(_ptr(packed), _ptr(scales), _ptr(y), N, bits, 0)
+    return arr
+
+
+def wr_gemv_grouped_workspace_bytes(M: int, K: int, items) -> int:
+    arr = items if isinstance(items, ctypes.Array) else _gitems(items)
+    return _lib.wr_gemv_grouped_workspace_bytes(M, K, len(arr), arr)
+
+
+def wr_gemv_grouped(M: int, K: int, x, items, workspace, workspace_bytes: int, stream=None) -> None:
+    """items: sequence of (packed, scales, y, N, bits), or a prepared ctypes array; all read x."""
+    arr = items if isinstance(items, ctypes.Array) else _gitems(items)
+    _check("wr_gemv_grouped", _lib.wr_gemv_grouped(M, K, _ptr(x), len(arr), arr, _ptr(workspace),
+                                                   workspace_bytes, _stream(stream)))
 
 
 def _tproblems(problems):

@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <climits>
 #include <cstdint>
 #include <mutex>
 
@@ -113,6 +114,14 @@ void plan_decode(int64_t M, int count, const ProblemShape* shapes, DecodePlan* d
   // per CTA of the launch (see DecArgs)
   const int64_t wave = (int64_t)wr::decode_ctas_per_sm(ternary, (int)M) * kPlanSMs;
   dp->grid = (int)std::max<int64_t>(1, std::min<int64_t>(wave, cost_base / max_cost));
+  // each CTA's first block and the problem that holds it
+  for (int c = 0, pi = 0; c <= dp->grid; ++c) {
+    const int64_t g = wr::range_start(a, dp->grid, c);
+    a.rs[c] = (int32_t)g;
+    if (c == dp->grid) break;
+    while (pi + 1 < count && a.prob[pi + 1].block_base <= g) ++pi;
+    a.rp[c] = (uint16_t)pi;
+  }
   const int64_t partials = 2 * (int64_t)dp->grid * M * 128;
   dp->total_blocks = blocks;
   dp->counter_off = 0;
@@ -133,9 +142,40 @@ void bind_workspace(DecodePlan& dp, void* workspace) {
 
 // The preparation pass (for ternary, with the rotation), then the decode kernel over one
 // contiguous block range per CTA (the partial slots were sized for this grid).
+//
+// Problems that read the same activations (same x pointer and K; for ternary the same sign mask)
+// through the same tile layout (Q2, Q3, T2 and ternary order and scale K positions differently)
+// share one set of prepared tiles: the preparation pass writes it once, for the first of them
+// (looked up among the last few distinct sets, which is where q/k/v or gate/up sit in a batch).
 wr_status run_decode(DecodePlan& dp, cudaStream_t stream) {
-  if (wr::launch_prep_x(dp.args, dp.total_blocks, stream) != cudaSuccess) return WR_ERR_CUDA;
-  return wr::launch_gemv_q(dp.args, dp.grid, stream) == cudaSuccess ? WR_OK : WR_ERR_CUDA;
+  if (dp.args.total > INT32_MAX) return WR_ERR_INVALID_ARG;   // block indices are 32-bit in the kernel
+  static thread_local wr::DecArgs prep;
+  wr::DecArgs& a = dp.args;
+  prep.count = 0;
+  prep.M = a.M;
+  int blocks = 0;
+  constexpr int kLook = 8;
+  for (int i = 0; i < a.count; ++i) {
+    wr::DecProblem& pi = a.prob[i];
+    int owner = -1;
+    for (int j = prep.count - 1; j >= 0 && j >= prep.count - kLook; --j) {
+      const wr::DecProblem& pj = prep.prob[j];
+      if (pj.x == pi.x && pj.K == pi.K && pj.bits == pi.bits && pj.signs == pi.signs) {
+        owner = j;
+        break;
+      }
+    }
+    if (owner >= 0) {
+      pi.xt = prep.prob[owner].xt;
+    } else {
+      prep.prob[prep.count] = pi;
+      prep.prob[prep.count].xblk_base = blocks;
+      blocks += pi.B;
+      ++prep.count;
+    }
+  }
+  if (wr::launch_prep_x(prep, blocks, stream) != cudaSuccess) return WR_ERR_CUDA;
+  return wr::launch_gemv_q(a, dp.grid, stream) == cudaSuccess ? WR_OK : WR_ERR_CUDA;
 }
 
 // ---- prefill GEMM kernel (M > 8): 128-row groups x token tiles x K blocks, cut "stream-K" into
@@ -458,6 +498,47 @@ wr_status wr_gemv_batched(int64_t M, int32_t count, const wr_gemv_problem* probl
     if (st != WR_OK) return st;
   }
   return WR_OK;
+}
+
+static bool group_ok(int64_t M, int64_t K, int32_t count, const wr_gemv_group_item* it) {
+  if (M < 1 || M > 8 || count < 1 || count > wr::kMaxDecodeProblems || !it) return false;
+  for (int i = 0; i < count; ++i) {
+    QFmt f{};
+    if (!split_fmt(it[i].bits, true, &f)) return false;
+    if (it[i].reserved != 0 || check_dims(M, it[i].N, K) != WR_OK || K % 256 != 0) return false;
+    if (!aligned16(it[i].packed) || !aligned16(it[i].scales) || !aligned16(it[i].y)) return false;
+  }
+  return true;
+}
+
+size_t wr_gemv_grouped_workspace_bytes(int64_t M, int64_t K, int32_t count, const wr_gemv_group_item* items) {
+  if (!group_ok(M, K, count, items)) return 0;
+  static thread_local DecodePlan dp;
+  ProblemShape sh[wr::kMaxDecodeProblems];
+  for (int i = 0; i < count; ++i) sh[i] = ProblemShape{items[i].N, K, items[i].bits & ~WR_SCALES_I8};
+  plan_decode(M, count, sh, &dp);
+  return dp.total;
+}
+
+wr_status wr_gemv_grouped(int64_t M, int64_t K, const uint16_t* x, int32_t count, const wr_gemv_group_item* items,
+                          void* workspace, size_t workspace_bytes, void* stream) {
+  if (!group_ok(M, K, count, items) || !aligned16(x) || !aligned16(workspace)) return WR_ERR_INVALID_ARG;
+  if (workspace_bytes < wr_gemv_grouped_workspace_bytes(M, K, count, items)) return WR_ERR_INVALID_ARG;
+  static thread_local DecodePlan dp;
+  ProblemShape sh[wr::kMaxDecodeProblems];
+  for (int i = 0; i < count; ++i) sh[i] = ProblemShape{items[i].N, K, items[i].bits & ~WR_SCALES_I8};
+  plan_decode(M, count, sh, &dp);
+  for (int i = 0; i < count; ++i) {
+    QFmt f{};
+    split_fmt(items[i].bits, true, &f);
+    dp.args.prob[i].x = x;
+    dp.args.prob[i].packed = static_cast<const uint8_t*>(items[i].packed);
+    dp.args.prob[i].scales = items[i].scales;
+    dp.args.prob[i].scale_q = scale_q_of(f, items[i].scales, items[i].N);
+    dp.args.prob[i].y = items[i].y;
+  }
+  bind_workspace(dp, workspace);
+  return run_decode(dp, static_cast<cudaStream_t>(stream));
 }
 
 static bool tbatch_ok(int64_t M, int32_t count, const wr_gemv_ternary_problem* pr) {

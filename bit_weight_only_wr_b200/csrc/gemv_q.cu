@@ -131,16 +131,12 @@ __device__ __forceinline__ void pos_load(Pos& p, const DecArgs& a) {
 }
 __device__ __forceinline__ Pos pos_start(const DecArgs& a) {
   Pos p{};
-  const int G = (int)gridDim.x;   // the block ranges: range_start in tc_kernels.cuh
-  p.g = range_start(a, G, blockIdx.x);
-  p.left = (int)(range_start(a, G, blockIdx.x + 1) - p.g);
+  // the block ranges (range_start in tc_kernels.cuh) and the problem of each range's first block
+  // come computed from the host, so no role searches the problem table on the way in
+  p.g = a.rs[blockIdx.x];
+  p.left = (int)(a.rs[blockIdx.x + 1] - p.g);
   if (p.left <= 0) return p;
-  int lo = 0, hi = a.count - 1;
-  while (lo < hi) {  // last problem whose first block is <= g
-    const int mid = (lo + hi + 1) >> 1;
-    if (a.prob[mid].block_base <= p.g) lo = mid;
-    else hi = mid - 1;
-  }
+  const int lo = a.rp[blockIdx.x];
   p.pi = lo;
   pos_load(p, a);
   const int64_t local = p.g - a.prob[lo].block_base;
@@ -395,7 +391,11 @@ __global__ void __launch_bounds__(kThreads, Cfg<XR, MODE>::kCtas) gemv_q_kernel(
         pos_next(cp, a);
         ++np;
       }
-      if (nx < nblocks) {
+      if (nx < nblocks && np >= min(nblocks, (uint32_t)kSP)) {
+        // the activation tiles come from the preparation pass, which may still be running (the
+        // kernel is launched as its programmatic dependent): the first weight copies above are
+        // issued before waiting for it
+        if (nx == 0) grid_dependency_wait();
         // activation stage nx % kSX: free once block nx - kSX's MMAs are done; correction slot
         // nx % kSC once the epilogue has read block nx - kSC
         const int sx = nx % kSX, sc = nx % kSC;
@@ -424,8 +424,7 @@ __global__ void __launch_bounds__(kThreads, Cfg<XR, MODE>::kCtas) gemv_q_kernel(
     const uint64_t bdesc0 = smem_desc_sw128(xs);
     constexpr uint32_t idesc = kT ? idesc_i8s_m128(XR) : idesc_i8_m128(XR);
     constexpr uint32_t atom16 = (uint32_t)(XR * 128) >> 4;
-    const int G = (int)gridDim.x;
-    const int64_t span = range_start(a, G, blockIdx.x + 1) - range_start(a, G, blockIdx.x);
+    const int64_t span = (int64_t)a.rs[blockIdx.x + 1] - a.rs[blockIdx.x];
     const uint32_t nblocks = span > 0 ? (uint32_t)span : 0u;
     uint32_t gm = 0;
     bool ok = true;
@@ -600,7 +599,7 @@ __global__ void __launch_bounds__(kThreads, Cfg<XR, MODE>::kCtas) gemv_q_kernel(
           }
         } else {
           // slot 0: the row group began before this range; slot 1: it continues after it
-          const int slot = g0 < range_start_in(pr, M, range_cost_start(a, G, blockIdx.x)) ? 0 : 1;
+          const int slot = g0 < a.rs[blockIdx.x] ? 0 : 1;
           float* part = a.partial + ((int64_t)2 * blockIdx.x + slot) * M * 128;
 #pragma unroll
           for (int m = 0; m < kSlots; ++m)
@@ -614,7 +613,7 @@ __global__ void __launch_bounds__(kThreads, Cfg<XR, MODE>::kCtas) gemv_q_kernel(
 #pragma unroll
             for (int m = 0; m < kSlots; ++m) acc[m] = 0.f;
             for (int c = c0; c <= c1; ++c) {
-              const int sl = g0 < range_start_in(pr, M, range_cost_start(a, G, c)) ? 0 : 1;
+              const int sl = g0 < a.rs[c] ? 0 : 1;
               const float* src = a.partial + ((int64_t)2 * c + sl) * M * 128;
 #pragma unroll
               for (int m = 0; m < kSlots; ++m)
@@ -654,6 +653,7 @@ __global__ void __launch_bounds__(kThreads, Cfg<XR, MODE>::kCtas) gemv_q_kernel(
 // before its last multiply (E reaches -162 for subnormal bf16 activations). Slots m >= M hold zero
 // limbs and a zero factor.
 __global__ void __launch_bounds__(256) prep_x_kernel(const __grid_constant__ DecArgs a, int total_blocks) {
+  grid_launch_dependents();   // the GEMV may start its prologue and weight copies now
   const int lane = threadIdx.x & 31;
   const int M = a.M;
   const int xrows = decode_xrows(M), slots = xrows >> 2;
@@ -741,6 +741,7 @@ __global__ void __launch_bounds__(256) prep_x_kernel(const __grid_constant__ Dec
 // of 2^E as in the 2/3-bit record. Every t_k x'_k then reaches the MMA exactly, up to the rounding
 // of n_k (half a unit of 2^E) and, for the fifth trit of a byte, of 81 n_v (40.5 units).
 __global__ void __launch_bounds__(256) prep_t_kernel(const __grid_constant__ DecArgs a, int total_blocks) {
+  grid_launch_dependents();   // the GEMV may start its prologue and weight copies now
   __shared__ float xbuf[8][384];
   const int lane = threadIdx.x & 31, wi = threadIdx.x >> 5;
   const int M = a.M;
@@ -877,8 +878,18 @@ cudaError_t launch_xr(const DecArgs& a, int grid, cudaStream_t stream) {
     if (e != cudaSuccess) return e;
     set[dev] = true;
   }
-  gemv_q_kernel<XR, MODE><<<grid, kThreads, C::kSmem, stream>>>(a);
-  return cudaGetLastError();
+  // a programmatic dependent of the preparation pass launched just before it on the stream
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = C::kSmem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, gemv_q_kernel<XR, MODE>, a);
 }
 
 template <int MODE>

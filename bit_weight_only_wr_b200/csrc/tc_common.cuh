@@ -136,6 +136,13 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
                : "memory");
 }
 
+// Programmatic dependent launch: a kernel launched with programmatic stream serialization may
+// start while the kernel before it in the stream still runs; it must wait here before it reads
+// anything that kernel writes (a no-op when there is no such dependency). The earlier kernel
+// lets its dependents start with launch_dependents.
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(map) : "memory");
 }

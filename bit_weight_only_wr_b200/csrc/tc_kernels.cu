@@ -179,9 +179,11 @@ __device__ __forceinline__ uint32_t trit_entry(int v) {
 }
 
 // Output value of token m: the ternary planes hold token m scaled by 2^-tok_ex[m], undone here
-// (one rounding, gradual into fp32's subnormal range).
+// (one rounding, gradual into fp32's subnormal range); the 2/3-bit forms read x unscaled.
+template <int FMT>
 __device__ __forceinline__ float out_value(const TcArgs& a, float v, int m) {
-  return a.tok_ex ? ldexpf(v, a.tok_ex[m]) : v;
+  if constexpr (FMT == WR_FMT_TERNARY) return ldexpf(v, a.tok_ex[m]);
+  else return v;
 }
 
 // ---------------------------------------------------------------- the kernel
@@ -433,7 +435,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const TcArgs a, const _
         if (n < a.N) {
 #pragma unroll
           for (int i = 0; i < TH; ++i)
-            if (i < mcount) a.y[(int64_t)(m0 + i) * a.N + n] = out_value(a, rs * acc[i], m0 + i);
+            if (i < mcount) a.y[(int64_t)(m0 + i) * a.N + n] = out_value<FMT>(a, rs * acc[i], m0 + i);
         }
       } else {
         // slot 0: the tile began before this range; slot 1: it continues after it
@@ -460,7 +462,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const TcArgs a, const _
           if (n < a.N) {
 #pragma unroll
             for (int i = 0; i < TH; ++i)
-              if (i < mcount) a.y[(int64_t)(m0 + i) * a.N + n] = out_value(a, rs * acc[i], m0 + i);
+              if (i < mcount) a.y[(int64_t)(m0 + i) * a.N + n] = out_value<FMT>(a, rs * acc[i], m0 + i);
           }
           if (threadIdx.x == 256) a.counter[ps_.t] = 0;
         }
@@ -589,19 +591,34 @@ __global__ void rotate_planes_kernel(const uint16_t* __restrict__ x, const uint3
 }
 
 // Per-token exponent of the ternary prefill GEMM: tok_ex[m] = e with max_k |x[m,k]| in
-// [2^(e-1), 2^e) (0 for an all-zero token). One warp per token.
-__global__ void token_exponent_kernel(const uint16_t* __restrict__ x, int M, int K, int* __restrict__ tok_ex) {
-  const int lane = threadIdx.x & 31;
-  const int m = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  if (m >= M) return;
+// [2^(e-1), 2^e) (0 for an all-zero token). One CTA of 256 threads per token, 16-byte loads of 8
+// activations (K is a multiple of 128, so rows are 256-byte aligned).
+__global__ void __launch_bounds__(256) token_exponent_kernel(const uint16_t* __restrict__ x, int M, int K,
+                                                            int* __restrict__ tok_ex) {
+  __shared__ float wmax[8];
+  const int m = blockIdx.x;
+  const uint4* row = reinterpret_cast<const uint4*>(x + (int64_t)m * K);
   float amax = 0.f;
-  for (int k = lane; k < K; k += 32)
-    amax = fmaxf(amax, fabsf(__bfloat162float(__ushort_as_bfloat16(x[(int64_t)m * K + k]))));
+  for (int i = threadIdx.x; i < K / 8; i += 256) {
+    const uint4 v = __ldg(row + i);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      amax = fmaxf(amax, fabsf(__uint_as_float(w[j] << 16)));
+      amax = fmaxf(amax, fabsf(__uint_as_float(w[j] & 0xFFFF0000u)));
+    }
+  }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-  int ex = 0;
-  if (amax > 0.f) frexpf(amax, &ex);
-  if (lane == 0) tok_ex[m] = ex;
+  if ((threadIdx.x & 31) == 0) wmax[threadIdx.x >> 5] = amax;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    for (int i = 1; i < 8; ++i) amax = fmaxf(amax, wmax[i]);
+    amax = fmaxf(amax, wmax[0]);
+    int ex = 0;
+    if (amax > 0.f) frexpf(amax, &ex);
+    tok_ex[m] = ex;
+  }
 }
 
 // Failure-path self-test: warp 0 waits on a barrier nobody arrives on until the bounded wait
@@ -643,7 +660,7 @@ cudaError_t launch_tc_kernel(int fmt, int bn, const TcArgs& a, const void* x_act
 cudaError_t launch_rotate_planes(const uint16_t* x, const uint32_t* signs, uint8_t* planes, int M, int K, int64_t Kp,
                                  int* tok_ex, cudaStream_t stream) {
   const int warps = 8;
-  token_exponent_kernel<<<(unsigned)((M + warps - 1) / warps), warps * 32, 0, stream>>>(x, M, K, tok_ex);
+  token_exponent_kernel<<<(unsigned)M, 256, 0, stream>>>(x, M, K, tok_ex);
   const int64_t items = (int64_t)M * ((Kp + 127) / 128);
   rotate_planes_kernel<<<(unsigned)((items + warps - 1) / warps), warps * 32, 0, stream>>>(x, signs, planes, M, K, Kp,
                                                                                          tok_ex);

@@ -55,15 +55,20 @@ __host__ __device__ inline int64_t block_cost(int bits, int M) {
 // (in block_cost units) lies in [c C / G, (c+1) C / G). A row group cut by a range boundary is
 // finished through per-CTA partial slots (two per CTA: the row group that started before the
 // range, and the one that ends after it). A batch is all ternary or all 2/3-bit.
+constexpr int kMaxDecodeGrid = 444;   // CTAs of one decode launch, at most (3 per SM of a 148-SM part)
+
 struct DecArgs {
   int count, M;
   int64_t total;             // blocks of the batch (T)
   int64_t total_cost;        // their summed block_cost (C)
+  int32_t rs[kMaxDecodeGrid + 1];   // first block of CTA c's range (range_start, computed on the host)
+  uint16_t rp[kMaxDecodeGrid];      // problem that holds that first block
   float* partial;
   int* counter;
   int* err;
   DecProblem prob[kMaxDecodeProblems];
 };
+static_assert(sizeof(DecArgs) <= 32764, "kernel parameter space");
 
 // Block ranges of the 2/3-bit decode GEMV, used by the kernel (G = gridDim.x) and by the host
 // planner: CTA c of G starts at cost position c C / G (block_cost units, C = total_cost), at the

@@ -223,6 +223,29 @@ wr_status wr_gemv_batched_plan(int64_t M, int32_t count, const wr_gemv_problem* 
 wr_status wr_gemv_batched(int64_t M, int32_t count, const wr_gemv_problem* problems_host, void* workspace,
                           size_t workspace_bytes, void* stream);
 
+/* One weight matrix of a grouped decode GEMV (fields read on the host during the call). */
+typedef struct {
+  const void* packed;      /* packed codes (device) */
+  const uint16_t* scales;  /* fp16 [N, K/256] block scales, or the int8 scale record (device) */
+  float* y;                /* fp32 [M, N] output (device, overwritten) */
+  int64_t N;
+  int32_t bits;            /* 2, 3 or WR_FMT_T2, optionally | WR_SCALES_I8 */
+  int32_t reserved;        /* must be 0 */
+} wr_gemv_group_item;
+
+/* Grouped decode GEMV: `count` (1..256) weight matrices applied to the same activations x
+ * (bf16 [M, K], 1 <= M <= 8, K % 256 == 0), as the linears of a decoder layer that read one input
+ * do: q, k and v read the attention input, gate and up the MLP input ("Qwen3-4B-Wringer-Q2.6",
+ * "Recipe": each layer's seven linears, quantized alike). One preparation pass turns x into
+ * activation tiles once per tile layout (Q2, Q3, T2), then one persistent launch streams all the
+ * weights; each item computes y_i = what wr_gemv computes for (x, packed_i, scales_i). This is the
+ * grouping a decoder whose layers depend on each other can use: layer i+1's inputs exist only
+ * after layer i. items_host is a host array read during the call; the workspace rules are those
+ * of the other calls (wr_gemv_grouped_workspace_bytes, zero-filled before first use). */
+size_t wr_gemv_grouped_workspace_bytes(int64_t M, int64_t K, int32_t count, const wr_gemv_group_item* items_host);
+wr_status wr_gemv_grouped(int64_t M, int64_t K, const uint16_t* x, int32_t count, const wr_gemv_group_item* items_host,
+                          void* workspace, size_t workspace_bytes, void* stream);
+
 /* Prefill GEMM, any M >= 1 (bits = 2 or 3, optionally | WR_SCALES_I8; group 256; M <= 8 runs
  * the decode GEMV): packed tiles are staged in shared memory, decoded to exact bf16 grid
  * integers and contracted by tcgen05 MMAs into TMEM, one fp32 partial per 256-block, scaled in

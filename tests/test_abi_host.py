@@ -251,3 +251,18 @@ def test_decode_plan_random_batches():
         _check_plan(int(rng.integers(1, 9)), shapes)
     with pytest.raises(wr.WrError):
         wr.wr_gemv_batched_plan(9, [(None, None, None, None, 16, 256, 2)])
+
+
+def test_grouped_argument_checks():
+    items = [(16, 16, 16, 16, 2), (16, 16, 16, 1024, 3)]
+    assert wr.wr_gemv_grouped_workspace_bytes(1, 512, items) > 0
+    assert wr.wr_gemv_grouped_workspace_bytes(1, 300, items) == 0          # K % 256
+    assert wr.wr_gemv_grouped_workspace_bytes(9, 512, items) == 0          # M > 8
+    assert wr.wr_gemv_grouped_workspace_bytes(1, 512, [(16, 16, 16, 16, 7)]) == 0
+    arr = wr._gitems(items)
+    arr[1].reserved = 3
+    assert wr.wr_gemv_grouped_workspace_bytes(1, 512, arr) == 0
+    # misaligned x, and a workspace smaller than asked for, are rejected before any launch
+    nb = wr.wr_gemv_grouped_workspace_bytes(1, 512, items)
+    assert wr._lib.wr_gemv_grouped(1, 512, 8, 2, wr._gitems(items), 16, nb, None) == 1
+    assert wr._lib.wr_gemv_grouped(1, 512, 16, 2, wr._gitems(items), 16, nb - 1, None) == 1
