@@ -49,6 +49,7 @@ FMT_TERNARY = 1
 FMT_Q2 = 2
 FMT_Q3 = 3
 FMT_T2 = 4   # 2-bit trellis-coded: 2-bit symbols in the Q2 layout, 8 odd levels
+FMT_T8 = 5   # 8-state trellis over 4-weight symbols: 2-bit codes in the Q2 layout, 8 odd levels
 
 
 # --------------------------------------------------------------------------------------
@@ -380,6 +381,151 @@ def gemm_ternary(x_bits, codes, alpha, sign_words):
     xr = rotate(bf16_bits_to_f64(x_bits), sign_words)
     Wt = dequant_ternary(codes, alpha)
     return xr @ Wt.T, np.abs(xr) @ np.abs(Wt).T
+
+
+# --------------------------------------------------------------------------------------
+# The 8-state trellis over 4-weight symbols ("How We Shrank...", "Trick 3: trellis coding")
+# --------------------------------------------------------------------------------------
+#
+# The page names an 8-state set-partitioned trellis over symbols of 4 weights at about 2 bits
+# per weight, without tables. Reading taken here (the plainest one that keeps the toy's
+# mechanism): the signal set is the 4-vectors of level indices c in [0, 8) on the 8 odd levels
+# {-7..7} * s whose parities sum to an even number (a checkerboard set), partitioned by parity
+# pattern into 8 cosets of 256 points. State s = (s0, s1, s2) selects the coset whose parity
+# pattern is p = (s0, s1, s2, s0 ^ s1 ^ s2); the 8 written bits, four 2-bit codes u_i, pick the
+# point c_i = 2 u_i + p_i; and, as in the toy, a written bit sets the next state: the low bit of
+# u_3 shifts into the state, s' = ((s << 1) | (u_3 & 1)) & 7. The state restarts at 0 at every
+# 256-block. Storage: the codes u are packed exactly like 2-bit codes (2 bits per weight).
+
+def trellis8_parity(state: int):
+    """Parity pattern (p_0, p_1, p_2, p_3) of the coset that state s selects."""
+    s0, s1, s2 = state & 1, (state >> 1) & 1, (state >> 2) & 1
+    return (s0, s1, s2, s0 ^ s1 ^ s2)
+
+
+def trellis8_next(state: int, u3: int) -> int:
+    """The next state: the low bit of the symbol's last code shifted into the state."""
+    return ((state << 1) | (int(u3) & 1)) & 7
+
+
+def trellis8_level_index(codes: np.ndarray, state0: int = 0) -> np.ndarray:
+    """Level indices c = 2 u + p of each weight along the last axis (a multiple of 4 long),
+    running the state machine from state0 symbol by symbol."""
+    u = np.asarray(codes, dtype=np.int64)
+    n = u.shape[-1]
+    assert n % 4 == 0
+    flat = u.reshape(-1, n)
+    out = np.empty_like(flat)
+    for r in range(flat.shape[0]):
+        st = state0
+        for j in range(n // 4):
+            p = trellis8_parity(st)
+            for i in range(4):
+                out[r, 4 * j + i] = 2 * flat[r, 4 * j + i] + p[i]
+            st = trellis8_next(st, flat[r, 4 * j + 3])
+    return out.reshape(u.shape)
+
+
+def trellis8_viterbi(targets: np.ndarray, values: np.ndarray, state0: int = 0):
+    """Minimum squared-error path through the 8-state trellis: targets [..., n] (n a multiple
+    of 4; independent sequences along the leading axes), values [..., 8] ascending (the levels
+    of index 0..7). For each state and the low bit z of the last code, the branch's symbol is the
+    nearest allowed level per weight (u_0..u_2 free, u_3 with u_3 & 1 = z; a tie takes the lower
+    code); each new state keeps the cheaper of its two predecessors (a tie keeps the lower one),
+    and the path ends in the cheapest state (a tie takes the lower). Returns (codes int64
+    [..., n], cost float64 [...])."""
+    t = np.asarray(targets, dtype=np.float64)
+    v = np.asarray(values, dtype=np.float64)
+    lead, n = t.shape[:-1], t.shape[-1]
+    assert n % 4 == 0
+    v = np.broadcast_to(v, lead + v.shape[-1:])
+    nsym = n // 4
+    inf = np.inf
+    cost = np.full(lead + (8,), inf)
+    cost[..., state0] = 0.0
+    back_s = np.zeros(lead + (nsym, 8), dtype=np.int64)
+    back_u = np.zeros(lead + (nsym, 8, 4), dtype=np.int64)
+    for j in range(nsym):
+        tj = t[..., 4 * j:4 * j + 4]
+        # best code and its error for weight i, parity p, optionally restricted to u & 1 = z
+        def best(i, p, z=None):
+            us = [u for u in range(4) if z is None or (u & 1) == z]
+            be = np.full(lead, inf)
+            bu = np.zeros(lead, dtype=np.int64)
+            for u in us:
+                d = tj[..., i] - v[..., 2 * u + p]
+                e = d * d
+                better = e < be
+                be = np.where(better, e, be)
+                bu = np.where(better, u, bu)
+            return be, bu
+        new = np.full(lead + (8,), inf)
+        bs = np.zeros(lead + (8,), dtype=np.int64)
+        bu = np.zeros(lead + (8, 4), dtype=np.int64)
+        for nxt in range(8):
+            z = nxt & 1
+            for s in (nxt >> 1, (nxt >> 1) | 4):       # the two predecessors, lower first
+                p = trellis8_parity(s)
+                e0, u0 = best(0, p[0])
+                e1, u1 = best(1, p[1])
+                e2, u2 = best(2, p[2])
+                e3, u3 = best(3, p[3], z)
+                c = cost[..., s] + e0 + e1 + e2 + e3
+                better = c < new[..., nxt]
+                new[..., nxt] = np.where(better, c, new[..., nxt])
+                bs[..., nxt] = np.where(better, s, bs[..., nxt])
+                for i, ui in enumerate((u0, u1, u2, u3)):
+                    bu[..., nxt, i] = np.where(better, ui, bu[..., nxt, i])
+        cost = new
+        back_s[..., j, :] = bs
+        back_u[..., j, :, :] = bu
+    final = np.argmin(cost, axis=-1)
+    total = np.take_along_axis(cost, final[..., None], axis=-1)[..., 0]
+    codes = np.zeros(lead + (n,), dtype=np.int64)
+    st = final
+    for j in range(nsym - 1, -1, -1):
+        for i in range(4):
+            codes[..., 4 * j + i] = np.take_along_axis(back_u[..., j, :, i], st[..., None], axis=-1)[..., 0]
+        st = np.take_along_axis(back_s[..., j, :], st[..., None], axis=-1)[..., 0]
+    return codes, total
+
+
+def quantize_trellis8(W: np.ndarray):
+    """The 8-state trellis format: per 256-block s = fp16(absmax / 7) (fp64 division, one
+    rounding), levels s * {-7, ..., 7}, codes by trellis8_viterbi from state 0.
+    Returns (codes uint8 [N, K] in [0, 4), scales float16 [N, K/256])."""
+    W = np.asarray(W, dtype=np.float32)
+    N, K = W.shape
+    assert K % BLOCK == 0
+    Wb = W.astype(np.float64).reshape(N, K // BLOCK, BLOCK)
+    s16 = fp16_round(np.abs(Wb).max(axis=2) / 7.0)
+    levels = np.arange(-7, 8, 2, dtype=np.float64)
+    vals = s16.astype(np.float64)[:, :, None] * levels
+    codes, _ = trellis8_viterbi(Wb, vals)
+    return codes.reshape(N, K).astype(np.uint8), s16
+
+
+def dequant_trellis8(codes: np.ndarray, scales: np.ndarray) -> np.ndarray:
+    """W = s * (2 c - 7) with c the level indices of the 8-state trellis (state 0 at every
+    256-block)."""
+    u = np.asarray(codes, dtype=np.int64)
+    N, K = u.shape
+    c = trellis8_level_index(u.reshape(N, K // BLOCK, BLOCK)).reshape(N, K)
+    s = np.repeat(np.asarray(scales, dtype=np.float16).astype(np.float64), BLOCK, axis=1)
+    return s * (2 * c - 7).astype(np.float64)
+
+
+def dequant_trellis8_s8(codes: np.ndarray, d: np.ndarray, q: np.ndarray) -> np.ndarray:
+    """The 8-state trellis format with two-level scales: W = d_n q[n, b] (2 c - 7)."""
+    u = np.asarray(codes, dtype=np.int64)
+    N, K = u.shape
+    c = trellis8_level_index(u.reshape(N, K // BLOCK, BLOCK)).reshape(N, K)
+    g = (2 * c - 7).astype(np.float64)
+    return (g.reshape(N, K // BLOCK, BLOCK) * s8_block_scales(d, q)[:, :, None]).reshape(N, K)
+
+
+def gemm_trellis8(x_bits, codes, scales):
+    return gemm(x_bits, dequant_trellis8(codes, scales))
 
 
 # --------------------------------------------------------------------------------------

@@ -554,3 +554,80 @@ def test_trellis2_quantizer_invariants():
     c2, s2 = o.quantize_odd_grid(W, 2)
     err_q2 = ((W.astype(np.float64) - o.dequant(c2, s2, 2)) ** 2).sum()
     assert err_t.sum() < err_q2
+
+
+# ---------------------------------------------------------------- 8-state trellis (4-weight symbols)
+
+def test_trellis8_state_machine_hand_example():
+    # two symbols: codes [1, 2, 3, 1] from state 0 (parity pattern 0000) give level indices
+    # [2, 4, 6, 2]; the last code's low bit (1) makes the next state 1, whose pattern is
+    # (1, 0, 0, 1): codes [0, 3, 2, 2] give [1, 6, 4, 5]; the next state is (1 << 1 | 0) = 2
+    c = o.trellis8_level_index(np.array([1, 2, 3, 1, 0, 3, 2, 2]))
+    assert c.tolist() == [2, 4, 6, 2, 1, 6, 4, 5]
+    assert o.trellis8_next(1, 2) == 2 and o.trellis8_next(5, 3) == 3 and o.trellis8_next(7, 1) == 7
+    assert [o.trellis8_parity(s) for s in range(8)] == [
+        (0, 0, 0, 0), (1, 0, 0, 1), (0, 1, 0, 1), (1, 1, 0, 0),
+        (0, 0, 1, 1), (1, 0, 1, 0), (0, 1, 1, 0), (1, 1, 1, 1)]
+
+
+def test_trellis8_cosets_are_a_set_partition_of_the_even_parity_vectors():
+    # every state's coset holds 256 points, the 8 cosets are disjoint, and together they are
+    # exactly the 2048 level-index 4-vectors whose parities sum to an even number
+    seen = set()
+    for s in range(8):
+        p = o.trellis8_parity(s)
+        pts = {tuple(2 * u + p[i] for i, u in enumerate(us))
+               for us in np.ndindex(4, 4, 4, 4)}
+        assert len(pts) == 256 and not (pts & seen)
+        seen |= pts
+    even = {v for v in np.ndindex(8, 8, 8, 8) if sum(x & 1 for x in v) % 2 == 0}
+    assert seen == even
+
+
+def _trellis8_cost(t, vals, codes):
+    c = o.trellis8_level_index(codes)
+    return float(((t - vals[c]) ** 2).sum())
+
+
+@pytest.mark.parametrize("nsym", [1, 2])
+def test_trellis8_viterbi_is_the_brute_force_optimum(nsym):
+    rng = np.random.default_rng(50 + nsym)
+    vals = np.arange(-7, 8, 2, dtype=np.float64) * 0.31
+    all_codes = np.array(list(np.ndindex(*([4] * (4 * nsym)))), dtype=np.int64)   # 256^nsym paths
+    lvl = o.trellis8_level_index(all_codes)
+    for _ in range(4):
+        t = rng.normal(0, 1.0, 4 * nsym)
+        brute = ((t[None, :] - vals[lvl]) ** 2).sum(axis=1).min()
+        codes, cost = o.trellis8_viterbi(t, vals)
+        assert math.isclose(float(cost), float(brute), rel_tol=1e-12, abs_tol=1e-12)
+        assert math.isclose(_trellis8_cost(t, vals, codes), float(brute), rel_tol=1e-12, abs_tol=1e-12)
+
+
+def test_trellis8_error_below_the_two_state_trellis_and_the_grid():
+    # on Gaussian weights at the same 2 bits per weight: 8-state < 2-state < 4-level grid
+    W = wr_synth.weights_fp32(55, 8, 1024)
+    codes8, s8 = o.quantize_trellis8(W)
+    sym2, s2 = o.quantize_trellis2(W)
+    q, sq = o.quantize_odd_grid(W, 2)
+    W64 = W.astype(np.float64)
+    e8 = ((W64 - o.dequant_trellis8(codes8, s8)) ** 2).sum()
+    e2 = ((W64 - o.dequant_trellis2(sym2, s2)) ** 2).sum()
+    eq = ((W64 - o.dequant(q, sq, 2)) ** 2).sum()
+    assert e8 < e2 < eq
+    assert codes8.max() <= 3 and np.array_equal(s8, s2)   # same scale rule as the 2-state format
+    # the decoded level indices of each symbol have even parity sum
+    c = o.trellis8_level_index(codes8.reshape(8, 4, 256).astype(np.int64)).reshape(-1, 4)
+    assert np.all((c & 1).sum(axis=1) % 2 == 0)
+
+
+def test_trellis8_dequant_and_s8_form():
+    codes = np.zeros((2, 256), dtype=np.uint8)
+    codes[0, :8] = [1, 2, 3, 1, 0, 3, 2, 2]
+    s = np.array([[0.5], [2.0]], dtype=np.float16)
+    W = o.dequant_trellis8(codes, s)
+    assert W[0, :8].tolist() == [0.5 * (2 * c - 7) for c in (2, 4, 6, 2, 1, 6, 4, 5)]
+    # all-zero codes stay in state 0 (the low bit of u_3 is 0): level index 0 everywhere
+    assert np.all(W[1] == -14.0)
+    d = np.array([0.25, 1.0], dtype=np.float16)
+    qm = np.array([[2], [2]], dtype=np.int8)
+    assert np.array_equal(o.dequant_trellis8_s8(codes, d, qm), o.dequant_trellis8(codes, s))
