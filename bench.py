@@ -138,9 +138,7 @@ def module_bytes(wr, M, N, K, bits):
 # DRAM traffic of the decode GEMV launch, (dram__bytes_read + dram__bytes_write) / algorithmic
 # bytes, from one ncu capture of the current kernel at that token count (summary and command in
 # profiles/). None: no capture of this kernel version, so no traffic figure is claimed.
-# current kernel: M = 1 reads 1,205,202,688 and writes 7,539,968 bytes for 1,178,984,448
-# algorithmic; M = 8 reads 1,320,538,624 and writes 40,161,024 for 1,223,368,704
-_TRAFFIC_RATIO = {1: (1_205_202_688 + 7_539_968) / 1_178_984_448, 8: (1_320_538_624 + 40_161_024) / 1_223_368_704}
+_TRAFFIC_RATIO: dict = {}
 
 
 def traffic_per_launch(M: int, layers: int, algo_bytes: int):
@@ -585,6 +583,33 @@ def run_extras(args, wr, torch, np, stream, dist, hbm_peak, bf16_peak):
         out["trellis2"] = res
     except Exception as e:  # noqa: BLE001
         out["trellis2"] = {"error": repr(e)}
+
+    # the 8-state trellis over 4-weight symbols: one layer's 7 linears encoded once (Viterbi,
+    # host), the 36-layer body made of 36 distinct byte copies, one batched decode GEMV call
+    try:
+        res = {}
+        tmods = []
+        for idx, (name, K, N, _) in enumerate(wr_synth.QWEN3_4B_LAYER):
+            c8, sc = wr.wr_quantize_trellis8(wr_synth.weights_fp32(650 + idx, N, K))
+            tmods.append((K, N, torch.from_numpy(wr.wr_pack(wr.WR_FMT_T8, c8)).cuda(),
+                          torch.from_numpy(sc.view(np.int16)).cuda()))
+        body = [(K, N, p.roll(c * 4096), sc) for c in range(36) for (K, N, p, sc) in tmods]
+        for M in (1, 8):
+            xs = [torch.from_numpy(wr_synth.activations_bf16(5500 + j, M, K).view(np.int16)).cuda()
+                  for j, (K, _, _, _) in enumerate(body)]
+            ys = [torch.empty(M, N, dtype=torch.float32, device="cuda") for (_, N, _, _) in body]
+            arr = wr._problems([(xs[j], p, sc, ys[j], N, K, wr.WR_FMT_T8) for j, (K, N, p, sc) in enumerate(body)])
+            nb = wr.wr_gemv_batched_workspace_bytes(M, arr)
+            ws = torch.zeros(nb, dtype=torch.uint8, device="cuda")
+
+            def t8step():
+                wr.wr_gemv_batched(M, arr, ws, nb)
+            ms = graph_time_ms(torch, t8step, 10, 3, stream) / 10
+            b = sum(p.numel() + 2 * N * (K // 256) + 2 * M * K + 4 * M * N for (K, N, p, _) in body)
+            res[f"body_M{M}"] = {"ms": ms, "bytes": b, "gbs": b / ms / 1e6, "tokens_per_s": M * 1e3 / ms}
+        out["trellis8"] = res
+    except Exception as e:  # noqa: BLE001
+        out["trellis8"] = {"error": repr(e)}
 
     # int8 block scales (fp16 row scale times an int8 multiplier per 256-block): one layer's 7
     # linears quantized once by the device quantizer, the 36-layer body made of 36 distinct byte

@@ -20,11 +20,11 @@ __all__ = [
     "wr_get_device_error", "exported_symbols", "WrGemvProblem", "wr_gemv_batched_workspace_bytes",
     "wr_gemv_batched", "wr_gemv_noalloc", "WR_GEMV_NOALLOC_SCRATCH_BYTES", "WrGemvTernaryProblem",
     "wr_gemv_ternary_batched_workspace_bytes", "wr_gemv_ternary_batched", "wr_selftest_wait_timeout",
-    "wr_quantize_pack", "wr_quantize_trellis", "WR_FMT_T2", "WR_SCALES_I8", "wr_scales_bytes",
+    "wr_quantize_pack", "wr_quantize_trellis", "WR_FMT_T2", "WR_FMT_T8", "wr_quantize_trellis8", "WR_SCALES_I8", "wr_scales_bytes",
     "wr_gemv_batched_plan", "WrGemvGroupItem", "wr_gemv_grouped_workspace_bytes", "wr_gemv_grouped",
 ]
 
-WR_FMT_TERNARY, WR_FMT_Q2, WR_FMT_Q3, WR_FMT_T2 = 1, 2, 3, 4
+WR_FMT_TERNARY, WR_FMT_Q2, WR_FMT_Q3, WR_FMT_T2, WR_FMT_T8 = 1, 2, 3, 4, 5
 WR_SCALES_I8 = 0x100   # OR'd into a format code: int8 block scales (the scale record of include/wr.h)
 WR_GEMV_NOALLOC_SCRATCH_BYTES = 4 << 20   # mirrors the macro in include/wr.h
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libwr.so")
@@ -68,6 +68,7 @@ _SIGNATURES = {
     "wr_unpack_codes": (_c_int, [_c_int, _c_i64, _c_i64, _vp, _vp]),
     "wr_quantize": (_c_int, [_c_int, _c_i64, _c_i64, _vp, _vp, _vp]),
     "wr_quantize_trellis": (_c_int, [_c_i64, _c_i64, _vp, _vp, _vp]),
+    "wr_quantize_trellis8": (_c_int, [_c_i64, _c_i64, _vp, _vp, _vp]),
     "wr_quantize_ternary": (_c_int, [_c_i64, _c_i64, _vp, _vp, _vp, _vp]),
     "wr_unpack_bf16": (_c_int, [_c_int, _c_i64, _c_i64, _vp, _vp, _c_int, _vp, _vp]),
     "wr_gemv_workspace_bytes": (_c_size, [_c_i64, _c_i64, _c_i64, _c_int]),
@@ -197,6 +198,17 @@ def wr_quantize_trellis(W: np.ndarray):
     codes = np.empty((N, K), dtype=np.uint8)
     scales = np.empty((N, max(K // 256, 1)), dtype=np.uint16)
     _check("wr_quantize_trellis", _lib.wr_quantize_trellis(N, K, _ptr(W), _ptr(codes), _ptr(scales)))
+    return codes, scales
+
+
+def wr_quantize_trellis8(W: np.ndarray):
+    """fp32 [N, K] -> (codes uint8 [N, K] of the 8-state trellis format, fp16 scale bits
+    uint16 [N, K/256]); pack the codes with wr_pack(WR_FMT_T8, ...)."""
+    W = np.ascontiguousarray(W, dtype=np.float32)
+    N, K = W.shape
+    codes = np.empty((N, K), dtype=np.uint8)
+    scales = np.empty((N, max(K // 256, 1)), dtype=np.uint16)
+    _check("wr_quantize_trellis8", _lib.wr_quantize_trellis8(N, K, _ptr(W), _ptr(codes), _ptr(scales)))
     return codes, scales
 
 

@@ -49,7 +49,7 @@ struct QFmt {
 inline bool split_fmt(int fmt, bool allow_t2, QFmt* f) {
   f->s8 = (fmt & WR_SCALES_I8) != 0;
   f->base = fmt & ~WR_SCALES_I8;
-  return f->base == WR_FMT_Q2 || f->base == WR_FMT_Q3 || (allow_t2 && f->base == WR_FMT_T2);
+  return f->base == WR_FMT_Q2 || f->base == WR_FMT_Q3 || (allow_t2 && (f->base == WR_FMT_T2 || f->base == WR_FMT_T8));
 }
 // The int8 multipliers of an int8 scale record (null for fp16 scales).
 inline const int8_t* scale_q_of(const QFmt& f, const uint16_t* scales, int64_t N) {

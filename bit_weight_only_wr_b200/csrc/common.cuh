@@ -144,6 +144,26 @@ __host__ __device__ __forceinline__ void decode_t2_word_i8(uint32_t w, uint32_t&
   r[3] = (w & 0xC0C0C0C0u) | (P1 & 0x20202020u);
 }
 
+// 8-state trellis word (WR_FMT_T8; the Q2 word layout, code e at bits 16*(e&1) + 2*(e>>1)): its
+// 16 codes are symbols j = 0..3 of 4 codes each, and code 4j + i has level index 2 u + p_i with
+// (p_0, p_1, p_2, p_3) = (z_(j-1), z_(j-2), z_(j-3), z_(j-1) ^ z_(j-2) ^ z_(j-3)), z_k the low bit of
+// symbol k's last code (the state is the last three z). `carry` holds the previous word's z_0..z_3
+// at bits 2, 6, 10, 14 (0 at the block start) and returns this word's. With X = (this word's z
+// at bits 18 + 4j) | carry, z_k sits at bit 18 + 4k for k = -4..3, and P (each code's parity at
+// its field's low bit) is four shifted copies of X; the registers then come out as for T2.
+__host__ __device__ __forceinline__ void decode_t8_word_i8(uint32_t w, uint32_t& carry, uint32_t r[4]) {
+  const uint32_t zl = (w >> 16) & 0x4444u;
+  const uint32_t X = (zl << 16) | carry;
+  carry = zl;
+  const uint32_t P = ((X >> 14) & 0x1111u) | ((X << 6) & 0x11110000u) | ((X >> 4) & 0x4444u) |
+                     (((X << 4) ^ (X << 8) ^ (X << 12)) & 0x44440000u);
+  const uint32_t P1 = P >> 1;
+  r[0] = ((w & 0x03030303u) << 1) | (P & 0x01010101u);
+  r[1] = (w & 0x0C0C0C0Cu) | (P1 & 0x02020202u);
+  r[2] = (w & 0x30303030u) | (P1 & 0x08080808u);
+  r[3] = (w & 0xC0C0C0C0u) | (P1 & 0x20202020u);
+}
+
 // Code index (within a 256-code block) held at logical K position kl of the decoded block, and
 // the exponent e of its byte, for the register orders above. Rows of a block are 4 quarters of
 // 64 codes; a quarter is 16 registers (Q2: 4 words x 4; Q3: 2 groups x 8).
@@ -153,7 +173,7 @@ __host__ __device__ inline int q2_code_at(int kl) {
   return 64 * q + 16 * w + p;
 }
 __host__ __device__ inline int q2_exp_at(int kl) { return 2 * ((kl >> 2) & 3); }
-// The trellis format uses the Q2 K order; its bytes hold (2u + p) * 2^e, e = 0, 1, 3, 5.
+// The trellis formats use the Q2 K order; their bytes hold (2u + p) * 2^e, e = 0, 1, 3, 5.
 __host__ __device__ inline int t2_exp_at(int kl) {
   const int sp = (kl >> 2) & 3;
   return sp == 0 ? 0 : 2 * sp - 1;

@@ -205,6 +205,20 @@ __device__ __forceinline__ void t2_half_i8(const uint8_t* unit, int r0, int half
   }
 }
 
+// The 8-state trellis format: the Q2 words, with the last three symbols' low bits carried
+// through the row in code order.
+__device__ __forceinline__ void t8_half_i8(const uint8_t* unit, int r0, int half, int h, uint32_t v[32],
+                                           uint32_t& carry) {
+#pragma unroll
+  for (int qq = 0; qq < 2; ++qq) {
+    const uint4 c = *reinterpret_cast<const uint4*>(unit + (32 * half + lane_pos(r0, 2 * h + qq)) * 16);
+    decode_t8_word_i8(c.x, carry, v + 16 * qq + 0);
+    decode_t8_word_i8(c.y, carry, v + 16 * qq + 4);
+    decode_t8_word_i8(c.z, carry, v + 16 * qq + 8);
+    decode_t8_word_i8(c.w, carry, v + 16 * qq + 12);
+  }
+}
+
 __device__ __forceinline__ void q3_half_i8(const uint8_t* unit, int r0, int half, int h, uint32_t v[32]) {
 #pragma unroll
   for (int qq = 0; qq < 2; ++qq) {
@@ -477,17 +491,19 @@ __global__ void __launch_bounds__(kThreads, Cfg<XR, MODE>::kCtas) gemv_q_kernel(
       } else {
         const uint8_t* unit = ps + sp * C::kPStage + tile * (dc.bits == 3 ? 1536 : 1024);
         uint32_t v[32];
-        uint32_t carry = 0;   // trellis state at the block start
+        uint32_t carry = 0;   // trellis state at the block start (both trellis formats)
         if (dc.bits == 2) q2_half_i8(unit, r0, half, 0, v);
         else if (!kAll || dc.bits == 3) q3_half_i8(unit, r0, half, 0, v);
-        else t2_half_i8(unit, r0, half, 0, v, carry);
+        else if (dc.bits == WR_FMT_T2) t2_half_i8(unit, r0, half, 0, v, carry);
+        else t8_half_i8(unit, r0, half, 0, v, carry);
         // the A buffer is free once block gd - 1's MMAs are done
         if (gd > 0 && !mbar_wait(&bars->mma_done[(gd - 1) % kSX], ((gd - 1) / kSX) & 1, abort_flag, a.err, 302)) break;
         fence_after_sync();
         tmem_st32(lane_base + C::kACol, v);
         if (dc.bits == 2) q2_half_i8(unit, r0, half, 1, v);
         else if (!kAll || dc.bits == 3) q3_half_i8(unit, r0, half, 1, v);
-        else t2_half_i8(unit, r0, half, 1, v, carry);
+        else if (dc.bits == WR_FMT_T2) t2_half_i8(unit, r0, half, 1, v, carry);
+        else t8_half_i8(unit, r0, half, 1, v, carry);
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars->pk_empty[sp]);
         tmem_st32(lane_base + C::kACol + 32, v);
@@ -907,7 +923,8 @@ cudaError_t launch_mode(const DecArgs& a, int grid, cudaStream_t stream) {
 cudaError_t launch_gemv_q(const DecArgs& a, int grid, cudaStream_t stream) {
   if (a.count > 0 && a.prob[0].bits == 1) return launch_mode<kModeTern>(a, grid, stream);
   bool all = false;
-  for (int i = 0; i < a.count; ++i) all = all || a.prob[i].bits == WR_FMT_T2 || a.prob[i].scale_q != nullptr;
+  for (int i = 0; i < a.count; ++i)
+    all = all || a.prob[i].bits == WR_FMT_T2 || a.prob[i].bits == WR_FMT_T8 || a.prob[i].scale_q != nullptr;
   return all ? launch_mode<kModeAll>(a, grid, stream) : launch_mode<kModeLean>(a, grid, stream);
 }
 

@@ -19,10 +19,10 @@ namespace {
 constexpr int kTileRows = 16;
 
 inline bool fmt_ok(int fmt) {
-  return fmt == WR_FMT_Q2 || fmt == WR_FMT_Q3 || fmt == WR_FMT_TERNARY || fmt == WR_FMT_T2;
+  return fmt == WR_FMT_Q2 || fmt == WR_FMT_Q3 || fmt == WR_FMT_TERNARY || fmt == WR_FMT_T2 || fmt == WR_FMT_T8;
 }
-// 2-bit symbol formats share the Q2 words: Q2 codes and the trellis format's symbols.
-inline bool two_bit(int fmt) { return fmt == WR_FMT_Q2 || fmt == WR_FMT_T2; }
+// 2-bit symbol formats share the Q2 words: Q2 codes and the trellis formats' codes.
+inline bool two_bit(int fmt) { return fmt == WR_FMT_Q2 || fmt == WR_FMT_T2 || fmt == WR_FMT_T8; }
 
 struct Geometry {
   int64_t unit_k;      // codes per unit along K
@@ -358,6 +358,79 @@ wr_status wr_quantize_trellis(int64_t N, int64_t K, const float* w, uint8_t* cod
       for (int i = 255; i >= 0; --i) {
         codes[n * K + b * 256 + i] = bu[2 * i + st];
         st = bs[2 * i + st];
+      }
+    }
+  }
+  return WR_OK;
+}
+
+// The 8-state trellis over 4-weight symbols: per 256-block s = fp16(absmax / 7), levels
+// s * {-7..7 odd}; state (s0, s1, s2) selects the parity pattern (s0, s1, s2, s0^s1^s2), code u_i
+// of the symbol's weight i gives level index 2 u_i + p_i, and the next state is
+// ((s << 1) | (u_3 & 1)) & 7. Viterbi from state 0: for each next state, its two predecessors
+// (the lower first), each with its nearest allowed symbol (per weight the nearest level, a tie
+// to the lower code; u_3 restricted to the low bit the next state needs); a tie keeps the
+// earlier candidate; the path ends in the cheapest state (a tie to the lower). The branch cost
+// is summed as cost + e_0 + e_1 + e_2 + e_3, in that order.
+wr_status wr_quantize_trellis8(int64_t N, int64_t K, const float* w, uint8_t* codes, uint16_t* scales) {
+  if (N <= 0 || K <= 0 || K % 256 != 0 || !w || !codes || !scales) return WR_ERR_INVALID_ARG;
+  const int64_t nb = K / 256;
+#pragma omp parallel for schedule(static)
+  for (int64_t n = 0; n < N; ++n) {
+    std::vector<uint8_t> bs(64 * 8), bu(64 * 8 * 4);
+    for (int64_t b = 0; b < nb; ++b) {
+      const float* wb = w + n * K + b * 256;
+      double amax = 0.0;
+      for (int i = 0; i < 256; ++i) amax = std::fmax(amax, std::fabs((double)wb[i]));
+      const uint16_t sh = double_to_half(amax / 7.0);
+      scales[n * nb + b] = sh;
+      const double s = half_to_double(sh);
+      double val[8];
+      for (int l = 0; l < 8; ++l) val[l] = s * (double)(2 * l - 7);
+      const double inf = std::numeric_limits<double>::infinity();
+      double cost[8];
+      for (int st = 0; st < 8; ++st) cost[st] = st == 0 ? 0.0 : inf;
+      for (int j = 0; j < 64; ++j) {
+        double t[4];
+        for (int i = 0; i < 4; ++i) t[i] = (double)wb[4 * j + i];
+        double nc[8];
+        for (int st = 0; st < 8; ++st) nc[st] = inf;
+        for (int nx = 0; nx < 8; ++nx) {
+          const int z = nx & 1;
+          for (int pass = 0; pass < 2; ++pass) {
+            const int st = pass ? ((nx >> 1) | 4) : (nx >> 1);
+            const int p[4] = {st & 1, (st >> 1) & 1, (st >> 2) & 1, (st ^ (st >> 1) ^ (st >> 2)) & 1};
+            double e[4];
+            int u[4];
+            for (int i = 0; i < 4; ++i) {
+              e[i] = inf;
+              u[i] = 0;
+              for (int uu = 0; uu < 4; ++uu) {
+                if (i == 3 && (uu & 1) != z) continue;
+                const double d = t[i] - val[2 * uu + p[i]];
+                const double ee = d * d;
+                if (ee < e[i]) {
+                  e[i] = ee;
+                  u[i] = uu;
+                }
+              }
+            }
+            const double c = cost[st] + e[0] + e[1] + e[2] + e[3];
+            if (c < nc[nx]) {
+              nc[nx] = c;
+              bs[8 * j + nx] = (uint8_t)st;
+              for (int i = 0; i < 4; ++i) bu[32 * j + 4 * nx + i] = (uint8_t)u[i];
+            }
+          }
+        }
+        for (int st = 0; st < 8; ++st) cost[st] = nc[st];
+      }
+      int st = 0;
+      for (int k = 1; k < 8; ++k)
+        if (cost[k] < cost[st]) st = k;
+      for (int j = 63; j >= 0; --j) {
+        for (int i = 0; i < 4; ++i) codes[n * K + b * 256 + 4 * j + i] = bu[32 * j + 4 * st + i];
+        st = bs[8 * j + st];
       }
     }
   }

@@ -104,7 +104,7 @@ __global__ void __launch_bounds__(32 * kUnpackWarps) unpack_kernel(const uint8_t
                                            : half_bits_to_float(scales[n]) * (float)scale_q[n * B + ub];
       const int L = FMT == WR_FMT_Q2 ? 3 : 7;
       int c[64];
-      if (FMT == WR_FMT_Q2 || FMT == WR_FMT_T2) {
+      if (FMT == WR_FMT_Q2 || FMT == WR_FMT_T2 || FMT == WR_FMT_T8) {
 #pragma unroll
         for (int w = 0; w < 4; ++w)
 #pragma unroll
@@ -138,6 +138,23 @@ __global__ void __launch_bounds__(32 * kUnpackWarps) unpack_kernel(const uint8_t
           const int u = c[i];
           c[i] = 2 * u + p;
           p = u & 1;
+        }
+      }
+      if (FMT == WR_FMT_T8) {
+        // 8-state trellis: the state entering this quarter is the low bits of the last codes of
+        // quarter q - 1's last three symbols (codes 55, 59, 63 of that lane), 0 at the block start
+        const uint32_t es = (((uint32_t)c[55] & 1u) << 2) | (((uint32_t)c[59] & 1u) << 1) | ((uint32_t)c[63] & 1u);
+        const uint32_t prev = __shfl_sync(0xffffffffu, es, lane_pos(r0, (q + 3) & 3));
+        int st = q == 0 ? 0 : (int)prev;
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const int p0 = st & 1, p1 = (st >> 1) & 1, p2 = (st >> 2) & 1;
+          const int z = c[4 * j + 3] & 1;
+          c[4 * j + 0] = 2 * c[4 * j + 0] + p0;
+          c[4 * j + 1] = 2 * c[4 * j + 1] + p1;
+          c[4 * j + 2] = 2 * c[4 * j + 2] + p2;
+          c[4 * j + 3] = 2 * c[4 * j + 3] + (p0 ^ p1 ^ p2);
+          st = ((st << 1) | z) & 7;
         }
       }
 #pragma unroll
@@ -185,6 +202,7 @@ cudaError_t launch_unpack_bf16(int fmt, const uint8_t* packed, const uint16_t* s
   if (fmt == WR_FMT_Q2) unpack_kernel<WR_FMT_Q2><<<ctas, th, 0, stream>>>(packed, scales, scale_q, N, K, units, U, w);
   else if (fmt == WR_FMT_Q3) unpack_kernel<WR_FMT_Q3><<<ctas, th, 0, stream>>>(packed, scales, scale_q, N, K, units, U, w);
   else if (fmt == WR_FMT_T2) unpack_kernel<WR_FMT_T2><<<ctas, th, 0, stream>>>(packed, scales, scale_q, N, K, units, U, w);
+  else if (fmt == WR_FMT_T8) unpack_kernel<WR_FMT_T8><<<ctas, th, 0, stream>>>(packed, scales, scale_q, N, K, units, U, w);
   else unpack_kernel<WR_FMT_TERNARY><<<ctas, th, 0, stream>>>(packed, scales, nullptr, N, K, units, U, w);
   return cudaGetLastError();
 }

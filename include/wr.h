@@ -85,7 +85,7 @@ typedef enum {
   WR_ERR_TOO_LARGE = 5      /* the problem needs more than the fixed scratch of wr_gemv_noalloc */
 } wr_status;
 
-enum { WR_FMT_TERNARY = 1, WR_FMT_Q2 = 2, WR_FMT_Q3 = 3, WR_FMT_T2 = 4 };
+enum { WR_FMT_TERNARY = 1, WR_FMT_Q2 = 2, WR_FMT_Q3 = 3, WR_FMT_T2 = 4, WR_FMT_T8 = 5 };
 
 /* WR_FMT_T2, the 2-bit trellis-coded format ("How We Shrank...", "Trick 3: trellis coding"):
  * symbols u in [0, 4) are stored exactly like Q2 codes (same packed layout, same bytes), with
@@ -96,6 +96,17 @@ enum { WR_FMT_TERNARY = 1, WR_FMT_Q2 = 2, WR_FMT_Q3 = 3, WR_FMT_T2 = 4 };
  * with 2 bits per weight. The codes come from wr_quantize_trellis (a Viterbi search). The
  * decode GEMV (wr_gemv, wr_gemv_batched, wr_gemv_noalloc with bits = WR_FMT_T2) and
  * wr_unpack_bf16 accept it; the prefill GEMM (M > 8) does not (WR_ERR_UNSUPPORTED). */
+
+/* WR_FMT_T8, the 8-state trellis over symbols of 4 weights at 2 bits per weight ("How We
+ * Shrank...", "Trick 3: trellis coding", which names an 8-state set-partitioned trellis over
+ * 4-weight symbols and gives no tables; this is the reading taken). The codes u in [0, 4) are stored
+ * exactly like Q2 codes (same packed layout and bytes) with fp16 scales per 256-block (or
+ * | WR_SCALES_I8). Consecutive groups of 4 codes along K are symbols. The state (s0, s1, s2), 0 at
+ * every 256-block start, selects the parity pattern p = (s0, s1, s2, s0 ^ s1 ^ s2): weight i of
+ * the symbol has level index c = 2 u_i + p_i and weight s * (2c - 7) on the 8 odd levels; the next
+ * state is ((s << 1) | (u_3 & 1)) & 7. The reachable 4-vectors of level indices are those whose
+ * parities sum to an even number, split by parity pattern into the 8 cosets the states select.
+ * Codes come from wr_quantize_trellis8 (a Viterbi search). Accepted where WR_FMT_T2 is. */
 
 /* Int8 block scales (the "Agents-A1-4B-Wringer-Q2.6" card, "What is in this repo": a container
  * of packed codes with fp16 or int8 block scales). WR_SCALES_I8 is OR'd into the format code
@@ -165,6 +176,15 @@ wr_status wr_quantize_pack(int bits, int64_t N, int64_t K, const float* w, void*
 wr_status wr_quantize_trellis(int64_t N, int64_t K, const float* w_host, uint8_t* codes_host,
                               uint16_t* scales_host);
 
+/* Host encoder for WR_FMT_T8: per 256-block s = fp16(absmax / 7) (fp64 division, one rounding),
+ * then the code sequence of least squared error under the 8-state trellis (Viterbi from state 0;
+ * per weight the nearest allowed level, a tie to the lower code; each state keeps the cheaper of
+ * its two predecessors, a tie to the lower; the path ends in the cheapest state, a tie to the
+ * lower). w_host fp32 [N,K]; codes_host uint8 [N,K] (0..3, packed with wr_pack(WR_FMT_T8, ...));
+ * scales_host fp16 bits [N, K/256]; K % 256 == 0. */
+wr_status wr_quantize_trellis8(int64_t N, int64_t K, const float* w_host, uint8_t* codes_host,
+                               uint16_t* scales_host);
+
 /* Host synthetic ternary quantizer: W' = W R^T (fp64, per 128-block fast Walsh-Hadamard
  * transform with the sign mask), Delta_n = 0.7 * mean_k |W'[n,k]|, t = sign(W') where
  * |W'| > Delta_n else 0, alpha_n = fp16(mean |W'| over t != 0) (0 if none); codes c = t+1.
@@ -173,14 +193,14 @@ wr_status wr_quantize_ternary(int64_t N, int64_t K, const float* w_host,
                               const uint32_t* sign_bits_host, uint8_t* codes_host,
                               uint16_t* alpha_host);
 
-/* Device materializer: w_bf16 [N,K] = bf16_RNE(s * g) for Q2, Q3 and T2, optionally
+/* Device materializer: w_bf16 [N,K] = bf16_RNE(s * g) for Q2, Q3, T2 and T8, optionally
  * | WR_SCALES_I8 (group must be 256), or bf16_RNE(alpha_n * t) for ternary (scales = alpha [N],
  * group ignored; the result is in the rotated basis). Bit-exact; the bf16 checkpoint the
  * "Qwen3-4B-Wringer-Q2.6" card's materializer produces from the container. */
 wr_status wr_unpack_bf16(int fmt, int64_t N, int64_t K, const void* packed, const uint16_t* scales,
                          int group, uint16_t* w_bf16, void* stream);
 
-/* Decode GEMV for 1 <= M <= 8 (bits = 2, 3 or WR_FMT_T2, optionally | WR_SCALES_I8; group 256):
+/* Decode GEMV for 1 <= M <= 8 (bits = 2, 3, WR_FMT_T2 or WR_FMT_T8, optionally | WR_SCALES_I8; group 256):
  * streams the packed codes once, decodes them in registers and contracts them on tensor cores.
  * The 128-row x 256-code blocks are cut into one contiguous range per CTA; a row group that
  * several ranges share is combined through the workspace in range order, so the result is the
@@ -197,7 +217,7 @@ typedef struct {
   const uint16_t* scales;  /* fp16 [N, K/256] block scales, or the int8 scale record (device) */
   float* y;                /* fp32 [M, N] output (device, overwritten) */
   int64_t N, K;            /* K % 256 == 0 */
-  int32_t bits;            /* 2, 3 or WR_FMT_T2, optionally | WR_SCALES_I8 */
+  int32_t bits;            /* 2, 3, WR_FMT_T2 or WR_FMT_T8, optionally | WR_SCALES_I8 */
   int32_t reserved;        /* must be 0 */
 } wr_gemv_problem;
 
@@ -229,7 +249,7 @@ typedef struct {
   const uint16_t* scales;  /* fp16 [N, K/256] block scales, or the int8 scale record (device) */
   float* y;                /* fp32 [M, N] output (device, overwritten) */
   int64_t N;
-  int32_t bits;            /* 2, 3 or WR_FMT_T2, optionally | WR_SCALES_I8 */
+  int32_t bits;            /* 2, 3, WR_FMT_T2 or WR_FMT_T8, optionally | WR_SCALES_I8 */
   int32_t reserved;        /* must be 0 */
 } wr_gemv_group_item;
 
@@ -270,7 +290,7 @@ wr_status wr_gemm_ternary(int64_t M, int64_t N, int64_t K, const uint16_t* x, co
  * WR_GEMV_NOALLOC_SCRATCH_BYTES (4 MiB) inside libwr, one per device.
  *
  * Computes exactly what wr_gemv computes (same arguments without workspace/workspace_bytes;
- * 1 <= M <= 8, bits 2, 3 or WR_FMT_T2, each optionally | WR_SCALES_I8, group 256, K % 256 == 0,
+ * 1 <= M <= 8, bits 2, 3, WR_FMT_T2 or WR_FMT_T8, each optionally | WR_SCALES_I8, group 256, K % 256 == 0,
  * 16-byte aligned device pointers).
  * Returns WR_ERR_TOO_LARGE, before touching the device, when the problem's scratch need
  * (wr_gemv_workspace_bytes) exceeds WR_GEMV_NOALLOC_SCRATCH_BYTES; then nothing is launched.

@@ -120,15 +120,53 @@ def test_trellis_quantizer_matches_oracle():
     assert np.array_equal(c1, c2)
 
 
+def test_trellis8_quantizer_matches_oracle():
+    """The library's Viterbi encoder for the 8-state trellis format picks the oracle's codes and
+    scales, bit for bit (same fp64 arithmetic, same tie order), including all-zero blocks (every
+    branch ties) and blocks built from exact level values."""
+    W = wr_synth.weights_fp32(322, 24, 1024)
+    W[3, :256] = 0.0
+    W[5, 256:512] *= np.float32(1e-6)
+    W[7, :256] = np.float32(0.25) * np.arange(256, dtype=np.float32) % 3 - 1   # many exact ties
+    c1, s1 = wr.wr_quantize_trellis8(W)
+    c2, s2 = o.quantize_trellis8(W)
+    assert np.array_equal(s1, s2.view(np.uint16))
+    assert np.array_equal(c1, c2)
+
+
+def test_trellis8_word_decoder_matches_the_state_machine():
+    """The GEMV's word decoder for the 8-state format, written out here from its definition in
+    include/wr.h as host arithmetic on one packed word at a time, is checked against the oracle's
+    state machine: every code's level index through the parity-bit positions of the word."""
+    rng = np.random.default_rng(9)
+    for trial in range(20):
+        u = rng.integers(0, 4, 64)
+        lvl = o.trellis8_level_index(u)
+        # the 4 words of a 64-code quarter, code e of word t at bits 16*(e&1) + 2*(e>>1)
+        words = [sum(int(u[16 * t + e]) << (16 * (e & 1) + 2 * (e >> 1)) for e in range(16)) for t in range(4)]
+        carry = 0
+        for t, w in enumerate(words):
+            zl = (w >> 16) & 0x4444
+            X = ((zl << 16) | carry) & 0xFFFFFFFF
+            carry = zl
+            P = (((X >> 14) & 0x1111) | ((X << 6) & 0x11110000) | ((X >> 4) & 0x4444)
+                 | (((X << 4) ^ (X << 8) ^ (X << 12)) & 0x44440000))
+            for e in range(16):
+                pos = 16 * (e & 1) + 2 * (e >> 1)
+                c = 2 * ((w >> pos) & 3) + ((P >> pos) & 1)
+                assert c == lvl[16 * t + e], (trial, t, e)
+
+
 @pytest.mark.parametrize("N,K", [(16, 256), (37, 768)])
-def test_trellis_format_packs_like_q2(N, K):
-    """WR_FMT_T2 stores its 2-bit symbols in the Q2 layout: same size, same bytes."""
+@pytest.mark.parametrize("fmt", [4, 5])
+def test_trellis_format_packs_like_q2(N, K, fmt):
+    """WR_FMT_T2 and WR_FMT_T8 store their 2-bit codes in the Q2 layout: same size, same bytes."""
     rng = np.random.default_rng(N + K)
     sym = rng.integers(0, 4, (N, K)).astype(np.uint8)
-    assert wr.wr_packed_bytes(wr.WR_FMT_T2, N, K) == wr.wr_packed_bytes(2, N, K)
-    p = wr.wr_pack(wr.WR_FMT_T2, sym)
+    assert wr.wr_packed_bytes(fmt, N, K) == wr.wr_packed_bytes(2, N, K)
+    p = wr.wr_pack(fmt, sym)
     assert np.array_equal(p, o.pack(o.FMT_Q2, sym))
-    assert np.array_equal(wr.wr_unpack_codes(wr.WR_FMT_T2, p, N, K), sym)
+    assert np.array_equal(wr.wr_unpack_codes(fmt, p, N, K), sym)
 
 
 def test_ternary_quantizer_matches_oracle():
@@ -154,7 +192,7 @@ def test_device_calls_reject_bad_arguments_before_launch():
     assert st == 1
     st = wr._lib.wr_gemv(9, 16, 256, 16, 16, 16, 2, 256, 16, 16, 1 << 20, None)   # M > 8
     assert st == 1
-    st = wr._lib.wr_gemv(1, 16, 256, 16, 16, 16, 5, 256, 16, 16, 1 << 20, None)   # bits
+    st = wr._lib.wr_gemv(1, 16, 256, 16, 16, 16, 6, 256, 16, 16, 1 << 20, None)   # bits
     assert st == 2
     st = wr._lib.wr_gemm(16, 16, 256, 16, 16, 16, 4, 256, 16, 16, 1 << 20, None)  # trellis, M > 8
     assert st == 2
@@ -171,7 +209,7 @@ def test_device_calls_reject_bad_arguments_before_launch():
     st = wr._lib.wr_unpack_bf16(2, 16, 256, 16, 16, 64, 16, None)                 # group
     assert st == 2
     i8 = wr.WR_SCALES_I8
-    st = wr._lib.wr_gemv(1, 16, 256, 16, 16, 16, 5 | i8, 256, 16, 16, 1 << 20, None)   # bits
+    st = wr._lib.wr_gemv(1, 16, 256, 16, 16, 16, 6 | i8, 256, 16, 16, 1 << 20, None)   # bits
     assert st == 2
     st = wr._lib.wr_gemm(16, 16, 256, 16, 16, 16, 4 | i8, 256, 16, 16, 1 << 20, None)  # trellis, M > 8
     assert st == 2
@@ -221,7 +259,7 @@ def test_decode_plan_rejects_what_the_batched_call_rejects():
         wr.wr_gemv_batched_plan(1, bad)
     assert e.value.status == 1
     assert wr._lib.wr_gemv_batched(1, 1, bad, 16, 1 << 20, None) == 1
-    for fields, status in (((16, 300, 2), 1), ((16, 256, 5), 2), ((0, 256, 2), 1)):
+    for fields, status in (((16, 300, 2), 1), ((16, 256, 6), 2), ((0, 256, 2), 1)):
         N, K, fmt = fields
         p = wr._problems([(16, 16, 16, 16, N, K, fmt)])
         with pytest.raises(wr.WrError) as e:

@@ -27,6 +27,10 @@ def _ws(nb):
 
 def _item(wr, kind, N, K, seed):
     """(packed, scales, fmt, reference function of x) for one weight matrix."""
+    if kind == "t8":
+        codes, sc = wr.wr_quantize_trellis8(wr_synth.weights_fp32(seed, N, K))
+        return dev(wr.wr_pack(wr.WR_FMT_T8, codes)), dev(sc), wr.WR_FMT_T8, \
+            (lambda x: o.gemm_trellis8(x, codes, sc.view(np.float16)))
     if kind == "t2":
         sym, sc = wr.wr_quantize_trellis(wr_synth.weights_fp32(seed, N, K))
         return dev(wr.wr_pack(wr.WR_FMT_T2, sym)), dev(sc), wr.WR_FMT_T2, \
@@ -44,7 +48,7 @@ def _item(wr, kind, N, K, seed):
 @pytest.mark.parametrize("group", [
     ("qkv", 2560, [("q2", 4096), ("q2", 1024), ("q3", 1024)]),
     ("gate_up", 2560, [("q2", 9728), ("q3", 9728)]),
-    ("ragged_mixed", 768, [("q3", 129), ("t2", 40), ("q2i8", 300), ("q2", 16), ("q3i8", 200)]),
+    ("ragged_mixed", 768, [("q3", 129), ("t2", 40), ("q2i8", 300), ("q2", 16), ("q3i8", 200), ("t8", 77)]),
 ])
 def test_grouped_matches_oracle(wr, M, group):
     torch = torch_mod()
@@ -98,7 +102,7 @@ def test_grouped_rejects_bad_items(wr):
     y = torch.zeros(1, 16, device="cuda")
     ok = [(16, 16, y, 16, 2)]
     assert wr.wr_gemv_grouped_workspace_bytes(M, K, ok) > 0
-    for bad in ([(16, 16, y, 16, 5)], [(16, 16, y, 0, 2)]):
+    for bad in ([(16, 16, y, 16, 6)], [(16, 16, y, 0, 2)]):
         assert wr.wr_gemv_grouped_workspace_bytes(M, K, bad) == 0
     assert wr.wr_gemv_grouped_workspace_bytes(M, 300, ok) == 0     # K % 256 != 0
     assert wr.wr_gemv_grouped_workspace_bytes(9, K, ok) == 0       # M > 8

@@ -81,6 +81,10 @@ def test_gemv_activation_range_trellis_and_int8_scales(wr, pattern):
     y = _gemv(wr, wr.WR_FMT_T2, x, dev(wr.wr_pack(wr.WR_FMT_T2, sym)), dev(sc), N, K)
     ref, B = o.gemm_trellis2(x, sym, sc.view(np.float16))
     check_close(y, ref, B, floor=fp32_floor(K))
+    c8, sc8 = wr.wr_quantize_trellis8(W)
+    y = _gemv(wr, wr.WR_FMT_T8, x, dev(wr.wr_pack(wr.WR_FMT_T8, c8)), dev(sc8), N, K)
+    ref, B = o.gemm_trellis8(x, c8, sc8.view(np.float16))
+    check_close(y, ref, B, floor=fp32_floor(K))
     codes, d, q, packed, rec = s8_case(wr, 3, N, K, seed=1302)
     y = _gemv(wr, 3 | wr.WR_SCALES_I8, x, packed, rec, N, K)
     ref, B = o.gemm_codes_s8(x, codes, d, q, 3)

@@ -72,6 +72,7 @@ def test_noalloc_matches_workspace_path(bits, N, K, M):
     ("t2", 300, 2560, 1),        # trellis-coded 2-bit symbols
     ("q3_i8", 1024, 2560, 4),    # 3-bit codes with int8 block scales
     ("q2_i8", 129, 768, 8),      # 2-bit codes with int8 block scales, ragged N
+    ("t8", 200, 1024, 2),        # 8-state trellis codes
 ])
 def test_noalloc_trellis_and_int8_scales(fmt_name, N, K, M):
     """The formats wr_gemv accepts besides plain Q2/Q3 (WR_FMT_T2, | WR_SCALES_I8), through the
@@ -83,7 +84,12 @@ def test_noalloc_trellis_and_int8_scales(fmt_name, N, K, M):
     seed = 7100 + N + M
     x_bits = wr_synth.activations_bf16(seed + 1, M, K)
     x = dev(x_bits)
-    if fmt_name == "t2":
+    if fmt_name == "t8":
+        fmt = wr.WR_FMT_T8
+        c8, sc = wr.wr_quantize_trellis8(wr_synth.weights_fp32(seed, N, K))
+        packed, scales = dev(wr.wr_pack(fmt, c8)), dev(sc)
+        y_ref, bound = o.gemm_trellis8(x_bits, c8, sc.view(np.float16))
+    elif fmt_name == "t2":
         fmt = wr.WR_FMT_T2
         sym, sc = wr.wr_quantize_trellis(wr_synth.weights_fp32(seed, N, K))
         packed, scales = dev(wr.wr_pack(fmt, sym)), dev(sc)
