@@ -681,7 +681,7 @@ def run_extras(args, wr, torch, np, stream, dist, hbm_peak, bf16_peak):
             p, s = build_q_module(wr, torch, 5000 + K, N, K, bits)
             R = max(8, int(3 * l2 // p.numel()) + 1)
             ps = [p.roll(i * 1024) for i in range(R)]          # distinct buffers, same format
-            for M in (16, 128, 512, 2048, 4096):
+            for M in (16, 32, 128, 512, 2048, 4096):
                 x = torch.from_numpy(wr_synth.activations_bf16(M, M, K).view(np.int16)).cuda()
                 y = torch.empty(M, N, dtype=torch.float32, device="cuda")
                 nb = wr.wr_gemm_workspace_bytes(M, N, K, bits)

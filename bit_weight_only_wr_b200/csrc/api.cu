@@ -58,9 +58,12 @@ inline const int8_t* scale_q_of(const QFmt& f, const uint16_t* scales, int64_t N
 }
 
 constexpr int kPlanSMs = 148;   // split heuristics are sized for a 148-SM part (device-independent)
-constexpr int kDecodeTokens = 8;   // decode kernel: 8 tokens x 4 activation limbs = 32 MMA columns
+// Token counts the integer decode kernel takes (4 activation limbs per token: up to 128 MMA
+// columns for the 2/3-bit formats, 32 for ternary); larger M goes to the tensor-core GEMM.
+constexpr int kDecodeTokens = wr::kMaxDecodeTokens;
+constexpr int kTernaryDecodeTokens = wr::kMaxTernaryDecodeTokens;
 
-// ---- decode kernel (M <= 8) and workspace [counters: one int per row group of every problem]
+// ---- decode kernel (M <= 32; ternary M <= 8) and workspace [counters: one int per row group of every problem]
 // [partials][prepared activation tiles: one per block of every problem]. The batch's blocks are
 // cut into one contiguous range of equal cost per CTA, and the partials are two 128-row slots per
 // CTA for the row groups that several ranges share. A batch is all 2/3-bit or all ternary.
@@ -178,7 +181,7 @@ wr_status run_decode(DecodePlan& dp, cudaStream_t stream) {
   return wr::launch_gemv_q(a, dp.grid, stream) == cudaSuccess ? WR_OK : WR_ERR_CUDA;
 }
 
-// ---- prefill GEMM kernel (M > 8): 128-row groups x token tiles x K blocks, cut "stream-K" into
+// ---- prefill GEMM kernel (M > 32; ternary M > 8): 128-row groups x token tiles x K blocks, cut "stream-K" into
 // one contiguous range of (tile, block) pairs per CTA; workspace [counters: one int per tile]
 // [two partial tiles per CTA, for the pieces of tiles cut by range ends].
 struct GemmPlan {
@@ -231,9 +234,20 @@ wr_status run_gemm(int bits, int M, int N, int K, const uint16_t* x, const uint8
   return wr::launch_tc_kernel(bits, 128, a, x, M, K, p.grid, stream) == cudaSuccess ? WR_OK : WR_ERR_CUDA;
 }
 
+// Which kernel a 2/3-bit call of M tokens runs. wr_gemv always takes the integer decode kernel
+// (M <= 32). wr_gemm takes it for M <= 8, and for M <= 32 when K <= 4096: there a row group has
+// few K blocks and the decode kernel measured faster than the tensor-core GEMM (gate 2560 -> 9728:
+// 17.8-21.8 against 24.5-28.2 us at M = 9..32); for long K (down 9728 -> 2560) the GEMM is faster
+// at M <= 16, since four int8 limbs per token make the activation tile twice the weights' bytes
+// and a long row group is split over many CTAs.
+bool decode_route(bool gemm, int64_t M, int64_t K) {
+  if (!gemm) return M <= kDecodeTokens;
+  return M <= 8 || (M <= kDecodeTokens && K <= 4096);
+}
+
 // One Q2/Q3 call of any M.
-size_t q_workspace(int bits, int64_t M, int64_t N, int64_t K) {
-  if (M <= kDecodeTokens) {
+size_t q_workspace(int bits, int64_t M, int64_t N, int64_t K, bool gemm) {
+  if (decode_route(gemm, M, K)) {
     static thread_local DecodePlan dp;
     const ProblemShape sh{N, K, bits};
     plan_decode(M, 1, &sh, &dp);
@@ -243,8 +257,9 @@ size_t q_workspace(int bits, int64_t M, int64_t N, int64_t K) {
 }
 
 wr_status run_q(int bits, int64_t M, int64_t N, int64_t K, const uint16_t* x, const void* packed,
-                const uint16_t* scales, const int8_t* scale_q, float* y, void* workspace, cudaStream_t stream) {
-  if (M <= kDecodeTokens) {
+                const uint16_t* scales, const int8_t* scale_q, float* y, void* workspace, cudaStream_t stream,
+                bool gemm) {
+  if (decode_route(gemm, M, K)) {
     static thread_local DecodePlan dp;
     const ProblemShape sh{N, K, bits};
     plan_decode(M, 1, &sh, &dp);
@@ -273,7 +288,7 @@ GemmPlan plan_gemm_t(int64_t M, int64_t N, int64_t K) {
 }
 
 size_t t_workspace(int64_t M, int64_t N, int64_t K) {
-  if (M > kDecodeTokens) return plan_gemm_t(M, N, K).total_bytes;
+  if (M > kTernaryDecodeTokens) return plan_gemm_t(M, N, K).total_bytes;
   static thread_local DecodePlan dp;
   const ProblemShape sh{N, K, WR_FMT_TERNARY};
   plan_decode(M, 1, &sh, &dp);
@@ -282,7 +297,7 @@ size_t t_workspace(int64_t M, int64_t N, int64_t K) {
 
 wr_status run_t(int64_t M, int64_t N, int64_t K, const uint16_t* x, const void* packed, const uint16_t* alpha,
                 const uint32_t* signs, float* y, void* workspace, cudaStream_t stream) {
-  if (M <= kDecodeTokens) {
+  if (M <= kTernaryDecodeTokens) {
     static thread_local DecodePlan dp;
     const ProblemShape sh{N, K, WR_FMT_TERNARY};
     plan_decode(M, 1, &sh, &dp);
@@ -377,8 +392,8 @@ wr_status wr_unpack_bf16(int fmt, int64_t N, int64_t K, const void* packed, cons
 size_t wr_gemv_workspace_bytes(int64_t M, int64_t N, int64_t K, int bits) {
   QFmt f{};
   if (!split_fmt(bits, true, &f)) return 0;
-  if (M < 1 || M > 8 || check_dims(M, N, K) != WR_OK || K % 256 != 0) return 0;
-  return q_workspace(f.base, M, N, K);
+  if (M < 1 || M > kDecodeTokens || check_dims(M, N, K) != WR_OK || K % 256 != 0) return 0;
+  return q_workspace(f.base, M, N, K, false);
 }
 
 wr_status wr_gemv(int64_t M, int64_t N, int64_t K, const uint16_t* x, const void* packed,
@@ -387,12 +402,12 @@ wr_status wr_gemv(int64_t M, int64_t N, int64_t K, const uint16_t* x, const void
   QFmt f{};
   if (!split_fmt(bits, true, &f)) return WR_ERR_UNSUPPORTED;
   if (group != 256) return WR_ERR_UNSUPPORTED;
-  if (M < 1 || M > 8 || check_dims(M, N, K) != WR_OK || K % 256 != 0) return WR_ERR_INVALID_ARG;
+  if (M < 1 || M > kDecodeTokens || check_dims(M, N, K) != WR_OK || K % 256 != 0) return WR_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(packed) || !aligned16(scales) || !aligned16(y) || !aligned16(workspace))
     return WR_ERR_INVALID_ARG;
-  if (workspace_bytes < q_workspace(f.base, M, N, K)) return WR_ERR_INVALID_ARG;
+  if (workspace_bytes < q_workspace(f.base, M, N, K, false)) return WR_ERR_INVALID_ARG;
   return run_q(f.base, M, N, K, x, packed, scales, scale_q_of(f, scales, N), y, workspace,
-               static_cast<cudaStream_t>(stream));
+               static_cast<cudaStream_t>(stream), false);
 }
 
 wr_status wr_gemv_noalloc(int64_t M, int64_t N, int64_t K, const uint16_t* x, const void* packed,
@@ -401,10 +416,10 @@ wr_status wr_gemv_noalloc(int64_t M, int64_t N, int64_t K, const uint16_t* x, co
   if (!split_fmt(bits, true, &f)) return WR_ERR_UNSUPPORTED;
   bits = f.base;
   if (group != 256) return WR_ERR_UNSUPPORTED;
-  if (M < 1 || M > 8 || check_dims(M, N, K) != WR_OK || K % 256 != 0) return WR_ERR_INVALID_ARG;
+  if (M < 1 || M > kDecodeTokens || check_dims(M, N, K) != WR_OK || K % 256 != 0) return WR_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(packed) || !aligned16(scales) || !aligned16(y)) return WR_ERR_INVALID_ARG;
   const int8_t* scale_q = scale_q_of(f, scales, N);
-  if (q_workspace(bits, M, N, K) > WR_GEMV_NOALLOC_SCRATCH_BYTES) return WR_ERR_TOO_LARGE;
+  if (q_workspace(bits, M, N, K, false) > WR_GEMV_NOALLOC_SCRATCH_BYTES) return WR_ERR_TOO_LARGE;
   wr_status st = WR_OK;
   void* scratch = noalloc_scratch(&st);
   if (scratch == nullptr) return st;
@@ -414,7 +429,7 @@ wr_status wr_gemv_noalloc(int64_t M, int64_t N, int64_t K, const uint16_t* x, co
   plan_decode(M, 1, &sh, &dp);
   const cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (dp.partial_off > 0 && cudaMemsetAsync(scratch, 0, dp.partial_off, s) != cudaSuccess) return WR_ERR_CUDA;
-  return run_q(bits, M, N, K, x, packed, scales, scale_q, y, scratch, s);
+  return run_q(bits, M, N, K, x, packed, scales, scale_q, y, scratch, s, false);
 }
 
 // Shape and format of one batched problem (what the plan reads); the batched call also checks
@@ -427,7 +442,7 @@ static wr_status problem_shape_ok(int64_t M, const wr_gemv_problem& pr) {
 }
 
 static bool batch_ok(int64_t M, int32_t count, const wr_gemv_problem* pr) {
-  if (M < 1 || M > 8 || count < 1 || !pr) return false;
+  if (M < 1 || M > kDecodeTokens || count < 1 || !pr) return false;
   for (int i = 0; i < count; ++i) {
     if (problem_shape_ok(M, pr[i]) != WR_OK) return false;
     if (!aligned16(pr[i].x) || !aligned16(pr[i].packed) || !aligned16(pr[i].scales) || !aligned16(pr[i].y))
@@ -438,7 +453,8 @@ static bool batch_ok(int64_t M, int32_t count, const wr_gemv_problem* pr) {
 
 wr_status wr_gemv_batched_plan(int64_t M, int32_t count, const wr_gemv_problem* problems, int32_t* grid,
                                int64_t* range_starts, int32_t range_starts_len, int64_t* block_costs) {
-  if (M < 1 || M > 8 || count < 1 || count > wr::kMaxDecodeProblems || !problems || !grid) return WR_ERR_INVALID_ARG;
+  if (M < 1 || M > kDecodeTokens || count < 1 || count > wr::kMaxDecodeProblems || !problems || !grid)
+    return WR_ERR_INVALID_ARG;
   ProblemShape sh[wr::kMaxDecodeProblems];
   for (int i = 0; i < count; ++i) {
     const wr_status st = problem_shape_ok(M, problems[i]);
@@ -501,7 +517,7 @@ wr_status wr_gemv_batched(int64_t M, int32_t count, const wr_gemv_problem* probl
 }
 
 static bool group_ok(int64_t M, int64_t K, int32_t count, const wr_gemv_group_item* it) {
-  if (M < 1 || M > 8 || count < 1 || count > wr::kMaxDecodeProblems || !it) return false;
+  if (M < 1 || M > kDecodeTokens || count < 1 || count > wr::kMaxDecodeProblems || !it) return false;
   for (int i = 0; i < count; ++i) {
     QFmt f{};
     if (!split_fmt(it[i].bits, true, &f)) return false;
@@ -542,7 +558,7 @@ wr_status wr_gemv_grouped(int64_t M, int64_t K, const uint16_t* x, int32_t count
 }
 
 static bool tbatch_ok(int64_t M, int32_t count, const wr_gemv_ternary_problem* pr) {
-  if (M < 1 || M > 8 || count < 1 || !pr) return false;
+  if (M < 1 || M > kTernaryDecodeTokens || count < 1 || !pr) return false;
   for (int i = 0; i < count; ++i) {
     if (check_dims(M, pr[i].N, pr[i].K) != WR_OK || pr[i].K % 128 != 0) return false;
     if (!aligned16(pr[i].x) || !aligned16(pr[i].packed) || !aligned16(pr[i].alpha) || !aligned16(pr[i].sign_bits) ||
@@ -596,7 +612,7 @@ size_t wr_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int bits) {
   QFmt f{};
   if (!split_fmt(bits, false, &f)) return 0;
   if (check_dims(M, N, K) != WR_OK || K % 256 != 0) return 0;
-  return q_workspace(f.base, M, N, K);
+  return q_workspace(f.base, M, N, K, true);
 }
 
 wr_status wr_gemm(int64_t M, int64_t N, int64_t K, const uint16_t* x, const void* packed,
@@ -608,9 +624,9 @@ wr_status wr_gemm(int64_t M, int64_t N, int64_t K, const uint16_t* x, const void
   if (check_dims(M, N, K) != WR_OK || K % 256 != 0) return WR_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(packed) || !aligned16(scales) || !aligned16(y) || !aligned16(workspace))
     return WR_ERR_INVALID_ARG;
-  if (workspace_bytes < q_workspace(f.base, M, N, K)) return WR_ERR_INVALID_ARG;
+  if (workspace_bytes < q_workspace(f.base, M, N, K, true)) return WR_ERR_INVALID_ARG;
   return run_q(f.base, M, N, K, x, packed, scales, scale_q_of(f, scales, N), y, workspace,
-               static_cast<cudaStream_t>(stream));
+               static_cast<cudaStream_t>(stream), true);
 }
 
 size_t wr_gemm_ternary_workspace_bytes(int64_t M, int64_t N, int64_t K) {

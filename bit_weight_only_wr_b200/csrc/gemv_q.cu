@@ -68,22 +68,25 @@ enum { kModeLean = 0, kModeAll = 1, kModeTern = 2 };
 // B: two atoms of 128 K positions). Ternary: a block is one 320-trit unit (A: 80 columns, B: three
 // atoms, the last half used), plus a 243-entry decode table replicated per lane (31 KB), so a CTA
 // needs more room; at MMA N = 16 or 32 two CTAs share an SM.
+// At MMA N = 64 or 128 (16 or 32 token slots, 2/3-bit forms only) the accumulators and B tiles
+// grow: two CTAs per SM at N = 64 (256 tensor-memory columns), one at N = 128 (512).
 template <int XR, int MODE>
 struct Cfg {
   static constexpr bool kT = MODE == kModeTern;
-  static constexpr int kCtas = (kT && XR > 8) ? 2 : 3;
+  static constexpr int kCtas = kT ? (XR > 8 ? 2 : 3) : (XR <= 32 ? 3 : (XR == 64 ? 2 : 1));
   static constexpr int kPStage = 8 * (kT ? 1024 : 1536);
-  static constexpr int kXStage = kT ? 3 * XR * 128 : 8 * 1024;   // 1024-byte multiples (swizzle atoms)
+  static constexpr int kXStage = kT ? 3 * XR * 128 : (XR <= 32 ? 8 * 1024 : 2 * XR * 128);   // 1024-byte multiples
+  static constexpr int kRec = kT ? 256 : (XR <= 64 ? 256 : 4 * XR);   // correction record per block
   static constexpr int kXOff = 0;
   static constexpr int kPOff = kXOff + kSX * kXStage;
   static constexpr int kCOff = kPOff + kSP * kPStage;
-  static constexpr int kBarOff = kCOff + kSC * 256;
+  static constexpr int kBarOff = kCOff + kSC * kRec;
   static constexpr int kSmem = kBarOff + 256 + 1024;   // + alignment slack
   static constexpr int kLutWords = kT ? 243 * 32 : 1;
   static constexpr int kACol = 0;
   static constexpr int kDCol = kT ? 96 : 64;           // two accumulators after the A buffer
-  static constexpr int kDCols = kT ? XR : 32;
-  static constexpr int kTmemCols = kDCol + 2 * kDCols <= 128 ? 128 : 256;
+  static constexpr int kDCols = kT ? XR : (XR < 32 ? 32 : XR);
+  static constexpr int kTmemCols = kDCol + 2 * kDCols <= 128 ? 128 : (kDCol + 2 * kDCols <= 256 ? 256 : 512);
   static_assert(kCtas * (kSmem + 4 * kLutWords + 1024) <= 228 * 1024, "CTAs per SM by shared memory");
   static_assert(kCtas * kTmemCols <= 512, "tensor memory of an SM");
 };
@@ -384,7 +387,7 @@ __global__ void __launch_bounds__(kThreads, Cfg<XR, MODE>::kCtas) gemv_q_kernel(
     // blocks, one elected lane issues): packed weights (a ring of kSP blocks), prepared B tiles
     // and their correction records (a ring of kSX blocks)
     constexpr uint32_t bbytes = (kT ? 384u : 256u) * XR;
-    constexpr uint32_t xtb = bbytes + 256u;   // prepared tile: B atoms, then corrections
+    constexpr uint32_t xtb = bbytes + (uint32_t)C::kRec;   // prepared tile: B atoms, then corrections
     Pos cp = pos_start(a), cx = cp;            // next block to copy: weights, activations
     const uint32_t nblocks = cp.left > 0 ? (uint32_t)cp.left : 0u;
     uint32_t np = 0, nx = 0;                   // weight copies, activation copies issued
@@ -419,8 +422,8 @@ __global__ void __launch_bounds__(kThreads, Cfg<XR, MODE>::kCtas) gemv_q_kernel(
         if (elect_one()) {
           mbar_arrive_expect_tx(&bars->x_full[sx], bbytes);
           bulk_load(xs + sx * C::kXStage, xsrc, bbytes, &bars->x_full[sx]);
-          mbar_arrive_expect_tx(&bars->c_full[sc], 256);
-          bulk_load(cs + sc * 256, xsrc + bbytes, 256, &bars->c_full[sc]);
+          mbar_arrive_expect_tx(&bars->c_full[sc], C::kRec);
+          bulk_load(cs + sc * C::kRec, xsrc + bbytes, C::kRec, &bars->c_full[sc]);
         }
         __syncwarp();
         pos_next(cx, a);
@@ -558,7 +561,7 @@ __global__ void __launch_bounds__(kThreads, Cfg<XR, MODE>::kCtas) gemv_q_kernel(
       if (!mbar_wait(&bars->mma_done[ge % kSX], (ge / kSX) & 1, abort_flag, a.err, 303)) break;
       if (!mbar_wait(&bars->c_full[sc], (ge / kSC) & 1, abort_flag, a.err, 304)) break;
       fence_after_sync();
-      const int4* rec = reinterpret_cast<const int4*>(cs + sc * 256);
+      const int4* rec = reinterpret_cast<const int4*>(cs + sc * C::kRec);
       const float s = kAll ? half_bits_to_float(sraw) * (float)qraw : half_bits_to_float(sraw);
       // 2^E = f f2 with f a normal fp32 power of two and f2 = 2^-j (0 <= j <= 36): s f2 is exact
       // and normal, (s f2) v rounds once, and the last multiply by f rounds once more, gradually
@@ -913,7 +916,13 @@ cudaError_t launch_mode(const DecArgs& a, int grid, cudaStream_t stream) {
   switch (decode_xrows(a.M)) {
     case 8: return launch_xr<8, MODE>(a, grid, stream);
     case 16: return launch_xr<16, MODE>(a, grid, stream);
-    default: return launch_xr<32, MODE>(a, grid, stream);
+    case 32: return launch_xr<32, MODE>(a, grid, stream);
+    case 64:
+      if constexpr (MODE != kModeTern) return launch_xr<64, MODE>(a, grid, stream);
+      return cudaErrorInvalidValue;
+    default:
+      if constexpr (MODE != kModeTern) return launch_xr<128, MODE>(a, grid, stream);
+      return cudaErrorInvalidValue;
   }
 }
 }  // namespace
@@ -929,6 +938,10 @@ cudaError_t launch_gemv_q(const DecArgs& a, int grid, cudaStream_t stream) {
 }
 
 // CTAs of one wave of the decode kernel for a batch of this kind on a 148-SM part.
-int decode_ctas_per_sm(bool ternary, int M) { return ternary && decode_xrows(M) > 8 ? 2 : 3; }
+int decode_ctas_per_sm(bool ternary, int M) {
+  const int xr = decode_xrows(M);
+  if (ternary) return xr > 8 ? 2 : 3;
+  return xr <= 32 ? 3 : (xr == 64 ? 2 : 1);
+}
 
 }  // namespace wr

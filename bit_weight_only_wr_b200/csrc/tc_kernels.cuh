@@ -22,7 +22,7 @@ struct TcArgs {
   int64_t total;             // RG * MT * B (tile, block) pairs, cut into one range per CTA
 };
 
-// Batched decode GEMV (M <= 8): one launch over up to kMaxDecodeProblems independent problems.
+// Batched decode GEMV (M <= 32): one launch over up to kMaxDecodeProblems independent problems.
 constexpr int kMaxDecodeProblems = 256;
 
 struct DecProblem {
@@ -112,10 +112,19 @@ int decode_ctas_per_sm(bool ternary, int M);
 // atoms of 128 K positions x xrows rows of int8, limb j of token slot m in row 4m + j (two atoms
 // for a 256-code block, three for a 320-trit unit, the last half used), then a 256-byte
 // correction record (per slot: 2/3-bit {C, f, f2, 0}; ternary {4 limb corrections}, {f, f2, 0, 0}).
-// xrows = 8, 16 or 32 for M <= 2, 4, 8 (the MMA's N).
-__host__ __device__ inline int decode_xrows(int M) { return M <= 2 ? 8 : (M <= 4 ? 16 : 32); }
+// xrows = 8, 16, 32, 64 or 128 for M <= 2, 4, 8, 16, 32 (the MMA's N; the ternary form takes M
+// <= 8). The record holds 16 bytes per token slot (2/3-bit) or 32 (ternary), at least 256.
+constexpr int kMaxDecodeTokens = 32;          // 2/3-bit and trellis formats
+constexpr int kMaxTernaryDecodeTokens = 8;
+__host__ __device__ inline int decode_xrows(int M) {
+  return M <= 2 ? 8 : (M <= 4 ? 16 : (M <= 8 ? 32 : (M <= 16 ? 64 : 128)));
+}
+__host__ __device__ inline int decode_rec_bytes(bool ternary, int M) {
+  const int r = (ternary ? 32 : 16) * (decode_xrows(M) / 4);
+  return r < 256 ? 256 : r;
+}
 __host__ __device__ inline int64_t xtile_bytes(bool ternary, int M) {
-  return (int64_t)(ternary ? 3 : 2) * decode_xrows(M) * 128 + 256;
+  return (int64_t)(ternary ? 3 : 2) * decode_xrows(M) * 128 + decode_rec_bytes(ternary, M);
 }
 
 cudaError_t launch_tc_kernel(int fmt, int bn, const TcArgs& a, const void* x_act, int64_t x_rows, int64_t x_k,

@@ -95,7 +95,7 @@ enum { WR_FMT_TERNARY = 1, WR_FMT_Q2 = 2, WR_FMT_Q3 = 3, WR_FMT_T2 = 4, WR_FMT_T
  * pages' 1-bit toy (two cosets of four levels, the written bit is the next state) written
  * with 2 bits per weight. The codes come from wr_quantize_trellis (a Viterbi search). The
  * decode GEMV (wr_gemv, wr_gemv_batched, wr_gemv_noalloc with bits = WR_FMT_T2) and
- * wr_unpack_bf16 accept it; the prefill GEMM (M > 8) does not (WR_ERR_UNSUPPORTED). */
+ * wr_unpack_bf16 accept it; wr_gemm does not (WR_ERR_UNSUPPORTED). */
 
 /* WR_FMT_T8, the 8-state trellis over symbols of 4 weights at 2 bits per weight ("How We
  * Shrank...", "Trick 3: trellis coding", which names an 8-state set-partitioned trellis over
@@ -200,8 +200,9 @@ wr_status wr_quantize_ternary(int64_t N, int64_t K, const float* w_host,
 wr_status wr_unpack_bf16(int fmt, int64_t N, int64_t K, const void* packed, const uint16_t* scales,
                          int group, uint16_t* w_bf16, void* stream);
 
-/* Decode GEMV for 1 <= M <= 8 (bits = 2, 3, WR_FMT_T2 or WR_FMT_T8, optionally | WR_SCALES_I8; group 256):
- * streams the packed codes once, decodes them in registers and contracts them on tensor cores.
+/* Decode GEMV for 1 <= M <= 32 (bits = 2, 3, WR_FMT_T2 or WR_FMT_T8, optionally | WR_SCALES_I8; group 256):
+ * streams the packed codes once, decodes them in registers and contracts them on tensor cores
+ * (kind::i8: four int8 limbs per token, so M <= 2, 4, 8, 16, 32 take 8, 16, 32, 64, 128 MMA columns).
  * The 128-row x 256-code blocks are cut into one contiguous range per CTA; a row group that
  * several ranges share is combined through the workspace in range order, so the result is the
  * same bits on every run. */
@@ -222,7 +223,7 @@ typedef struct {
 } wr_gemv_problem;
 
 /* Batched decode GEMV: `count` independent problems (2- and 3-bit may be mixed) sharing one
- * token count 1 <= M <= 8, computed by one persistent launch that streams all their packed
+ * token count 1 <= M <= 32, computed by one persistent launch that streams all their packed
  * weights back to back, so the fixed latency of a small GEMV is paid once per batch instead
  * of once per problem (the 252 linears of a 36-layer decoder body fit in one batch of at most
  * 256 problems; larger batches are split into several launches). Each problem computes what
@@ -254,7 +255,7 @@ typedef struct {
 } wr_gemv_group_item;
 
 /* Grouped decode GEMV: `count` (1..256) weight matrices applied to the same activations x
- * (bf16 [M, K], 1 <= M <= 8, K % 256 == 0), as the linears of a decoder layer that read one input
+ * (bf16 [M, K], 1 <= M <= 32, K % 256 == 0), as the linears of a decoder layer that read one input
  * do: q, k and v read the attention input, gate and up the MLP input ("Qwen3-4B-Wringer-Q2.6",
  * "Recipe": each layer's seven linears, quantized alike). One preparation pass turns x into
  * activation tiles once per tile layout (Q2, Q3, T2), then one persistent launch streams all the
@@ -266,8 +267,9 @@ size_t wr_gemv_grouped_workspace_bytes(int64_t M, int64_t K, int32_t count, cons
 wr_status wr_gemv_grouped(int64_t M, int64_t K, const uint16_t* x, int32_t count, const wr_gemv_group_item* items_host,
                           void* workspace, size_t workspace_bytes, void* stream);
 
-/* Prefill GEMM, any M >= 1 (bits = 2 or 3, optionally | WR_SCALES_I8; group 256; M <= 8 runs
- * the decode GEMV): packed tiles are staged in shared memory, decoded to exact bf16 grid
+/* Prefill GEMM, any M >= 1 (bits = 2 or 3, optionally | WR_SCALES_I8; group 256). M <= 8, and
+ * M <= 32 when K <= 4096, run the decode GEMV's integer kernel, which measured faster there; the
+ * workspace size follows the same choice (wr_gemm_workspace_bytes). Otherwise: packed tiles are staged in shared memory, decoded to exact bf16 grid
  * integers and contracted by tcgen05 MMAs into TMEM, one fp32 partial per 256-block, scaled in
  * fp32 by the epilogue. */
 size_t wr_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int bits);
@@ -290,7 +292,7 @@ wr_status wr_gemm_ternary(int64_t M, int64_t N, int64_t K, const uint16_t* x, co
  * WR_GEMV_NOALLOC_SCRATCH_BYTES (4 MiB) inside libwr, one per device.
  *
  * Computes exactly what wr_gemv computes (same arguments without workspace/workspace_bytes;
- * 1 <= M <= 8, bits 2, 3, WR_FMT_T2 or WR_FMT_T8, each optionally | WR_SCALES_I8, group 256, K % 256 == 0,
+ * 1 <= M <= 32, bits 2, 3, WR_FMT_T2 or WR_FMT_T8, each optionally | WR_SCALES_I8, group 256, K % 256 == 0,
  * 16-byte aligned device pointers).
  * Returns WR_ERR_TOO_LARGE, before touching the device, when the problem's scratch need
  * (wr_gemv_workspace_bytes) exceeds WR_GEMV_NOALLOC_SCRATCH_BYTES; then nothing is launched.

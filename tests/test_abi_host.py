@@ -190,7 +190,7 @@ def test_device_calls_reject_bad_arguments_before_launch():
     # misaligned / null pointers and unsupported configurations return before any CUDA call
     st = wr._lib.wr_gemv(1, 16, 256, 8, 16, 16, 2, 256, 16, 16, 1 << 20, None)
     assert st == 1
-    st = wr._lib.wr_gemv(9, 16, 256, 16, 16, 16, 2, 256, 16, 16, 1 << 20, None)   # M > 8
+    st = wr._lib.wr_gemv(33, 16, 256, 16, 16, 16, 2, 256, 16, 16, 1 << 20, None)   # M > 32
     assert st == 1
     st = wr._lib.wr_gemv(1, 16, 256, 16, 16, 16, 6, 256, 16, 16, 1 << 20, None)   # bits
     assert st == 2
@@ -221,7 +221,7 @@ def test_device_calls_reject_bad_arguments_before_launch():
     assert st == 2
     assert wr.wr_gemv_workspace_bytes(1, 16, 256, 3 | i8) == wr.wr_gemv_workspace_bytes(1, 16, 256, 3)
     assert wr.wr_gemm_workspace_bytes(64, 16, 256, 2 | i8) == wr.wr_gemm_workspace_bytes(64, 16, 256, 2)
-    assert wr.wr_gemv_workspace_bytes(9, 16, 256, 2) == 0
+    assert wr.wr_gemv_workspace_bytes(33, 16, 256, 2) == 0
     assert wr.wr_gemv_workspace_bytes(1, 16, 256, 2) > 0
 
 
@@ -288,14 +288,14 @@ def test_decode_plan_random_batches():
                   for _ in range(n)]
         _check_plan(int(rng.integers(1, 9)), shapes)
     with pytest.raises(wr.WrError):
-        wr.wr_gemv_batched_plan(9, [(None, None, None, None, 16, 256, 2)])
+        wr.wr_gemv_batched_plan(33, [(None, None, None, None, 16, 256, 2)])
 
 
 def test_grouped_argument_checks():
     items = [(16, 16, 16, 16, 2), (16, 16, 16, 1024, 3)]
     assert wr.wr_gemv_grouped_workspace_bytes(1, 512, items) > 0
     assert wr.wr_gemv_grouped_workspace_bytes(1, 300, items) == 0          # K % 256
-    assert wr.wr_gemv_grouped_workspace_bytes(9, 512, items) == 0          # M > 8
+    assert wr.wr_gemv_grouped_workspace_bytes(33, 512, items) == 0         # M > 32
     assert wr.wr_gemv_grouped_workspace_bytes(1, 512, [(16, 16, 16, 16, 7)]) == 0
     arr = wr._gitems(items)
     arr[1].reserved = 3
@@ -304,3 +304,19 @@ def test_grouped_argument_checks():
     nb = wr.wr_gemv_grouped_workspace_bytes(1, 512, items)
     assert wr._lib.wr_gemv_grouped(1, 512, 8, 2, wr._gitems(items), 16, nb, None) == 1
     assert wr._lib.wr_gemv_grouped(1, 512, 16, 2, wr._gitems(items), 16, nb - 1, None) == 1
+
+
+def test_decode_token_limits():
+    # the 2/3-bit decode path takes up to 32 tokens (128 MMA columns), the ternary one up to 8;
+    # wr_gemm takes any M (the decode kernel up to 32, the tensor-core GEMM above)
+    for M in (1, 8, 9, 16, 17, 32):
+        assert wr.wr_gemv_workspace_bytes(M, 256, 512, 2) > 0
+        # wr_gemm runs the decode kernel (same workspace) for M <= 8, and up to 32 when K <= 4096
+        assert wr.wr_gemm_workspace_bytes(M, 256, 512, 3) == wr.wr_gemv_workspace_bytes(M, 256, 512, 3)
+        if M > 8:
+            assert wr.wr_gemm_workspace_bytes(M, 256, 9728, 3) != wr.wr_gemv_workspace_bytes(M, 256, 9728, 3)
+    assert wr.wr_gemv_workspace_bytes(33, 256, 512, 2) == 0
+    assert wr.wr_gemm_workspace_bytes(33, 256, 512, 2) > 0
+    t = wr._tproblems([(16, 16, 16, 16, 16, 256, 512)])
+    assert wr.wr_gemv_ternary_batched_workspace_bytes(8, t) > 0
+    assert wr.wr_gemv_ternary_batched_workspace_bytes(9, t) == 0

@@ -105,4 +105,4 @@ def test_grouped_rejects_bad_items(wr):
     for bad in ([(16, 16, y, 16, 6)], [(16, 16, y, 0, 2)]):
         assert wr.wr_gemv_grouped_workspace_bytes(M, K, bad) == 0
     assert wr.wr_gemv_grouped_workspace_bytes(M, 300, ok) == 0     # K % 256 != 0
-    assert wr.wr_gemv_grouped_workspace_bytes(9, K, ok) == 0       # M > 8
+    assert wr.wr_gemv_grouped_workspace_bytes(33, K, ok) == 0      # M > 32

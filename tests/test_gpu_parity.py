@@ -485,3 +485,47 @@ def test_ternary_gemv_batched_layer_and_ragged(wr, M):
             ref, B = o.gemm_ternary(x, codes, alpha, signs)
             check_close(y.cpu().numpy(), ref, B)
     assert wr.wr_get_device_error() == 0
+
+
+# ---------------------------------------------------------------- small-M prefill on the decode kernel
+
+@pytest.mark.parametrize("bits", [2, 3])
+@pytest.mark.parametrize("M", [9, 12, 16, 17, 24, 32])
+def test_decode_kernel_up_to_32_tokens(wr, bits, M):
+    """wr_gemv and wr_gemm at 9 <= M <= 32 run the integer decode kernel with 64 or 128 MMA
+    columns; ragged N and several K blocks, against the oracle, both entry points."""
+    torch = torch_mod()
+    N, K = 300, 1280
+    codes, scales, packed, s_d = q_case(wr, bits, N, K, seed=3000 + M + bits)
+    x = wr_synth.activations_bf16(3100 + M, M, K)
+    ref, B = o.gemm_codes(x, codes, scales, bits)
+    y, _ = _run_gemv(wr, bits, x, packed, s_d, N, K)
+    check_close(y, ref, B)
+    check_close(_run_gemm(wr, bits, x, packed, s_d, N, K), ref, B)
+
+
+@pytest.mark.parametrize("bits,N,K,M", [(2, 9728, 2560, 16), (3, 2560, 9728, 32), (3, 9728, 2560, 24)])
+def test_decode_kernel_layer_shapes_small_prefill(wr, bits, N, K, M):
+    codes, scales, packed, s_d = q_case(wr, bits, N, K, seed=3200 + M)
+    x = wr_synth.activations_bf16(3300 + M, M, K)
+    ref, B = o.gemm_codes(x, codes, scales, bits)
+    check_close(_run_gemm(wr, bits, x, packed, s_d, N, K), ref, B)
+
+
+def test_batched_at_16_tokens(wr):
+    torch = torch_mod()
+    M = 16
+    problems, refs = [], []
+    for i, (N, K, bits) in enumerate([(64, 512, 2), (200, 2560, 3), (40, 256, 2), (1024, 2560, 3)]):
+        codes, scales, packed, s_d = q_case(wr, bits, N, K, seed=3400 + i)
+        x = wr_synth.activations_bf16(3410 + i, M, K)
+        refs.append(o.gemm_codes(x, codes, scales, bits))
+        y = torch.full((M, N), float("nan"), dtype=torch.float32, device="cuda")
+        problems.append((dev(x), packed, s_d, y, N, K, bits))
+    nb = wr.wr_gemv_batched_workspace_bytes(M, problems)
+    ws = _zeros_ws(nb)
+    for _ in range(2):
+        wr.wr_gemv_batched(M, problems, ws, nb)
+        torch.cuda.synchronize()
+        for p, (ref, B) in zip(problems, refs):
+            check_close(p[3].cpu().numpy(), ref, B)
