@@ -138,7 +138,10 @@ def module_bytes(wr, M, N, K, bits):
 # DRAM traffic of the decode GEMV launch, (dram__bytes_read + dram__bytes_write) / algorithmic
 # bytes, from one ncu capture of the current kernel at that token count (summary and command in
 # profiles/). None: no capture of this kernel version, so no traffic figure is claimed.
-_TRAFFIC_RATIO: dict = {}
+# current kernel (weights copied with an L2 evict-first policy, activation tiles evict-last):
+# M = 1 reads 1,181,419,520 and writes 3,914,240 bytes for 1,178,984,448 algorithmic; M = 8 reads
+# 1,206,598,656 and writes 14,751,232 for 1,223,368,704 (part of y is still in L2 at the end)
+_TRAFFIC_RATIO = {1: (1_181_419_520 + 3_914_240) / 1_178_984_448, 8: (1_206_598_656 + 14_751_232) / 1_223_368_704}
 
 
 def traffic_per_launch(M: int, layers: int, algo_bytes: int):

@@ -391,6 +391,9 @@ __global__ void __launch_bounds__(kThreads, Cfg<XR, MODE>::kCtas) gemv_q_kernel(
     Pos cp = pos_start(a), cx = cp;            // next block to copy: weights, activations
     const uint32_t nblocks = cp.left > 0 ? (uint32_t)cp.left : 0u;
     uint32_t np = 0, nx = 0;                   // weight copies, activation copies issued
+    // the weights are read once and the activation tiles by every row group of their problem:
+    // keep the tiles in L2 ahead of the weights streaming through it
+    const uint64_t pol_w = l2_policy_evict_first(), pol_x = l2_policy_evict_last();
     bool ok = true;
     while (ok && (np < nblocks || nx < nblocks)) {
       if (np < nblocks) {
@@ -401,8 +404,8 @@ __global__ void __launch_bounds__(kThreads, Cfg<XR, MODE>::kCtas) gemv_q_kernel(
         const int ntile = min(8, (cp.N + 15) / 16 - cp.rg * 8);
         if (elect_one()) {
           mbar_arrive_expect_tx(&bars->pk_full[sp], ntile * ub);
-          bulk_load(ps + sp * C::kPStage, cp.packed + ((int64_t)cp.rg * 8 * cp.B + (int64_t)cp.b * ntile) * ub,
-                    ntile * ub, &bars->pk_full[sp]);
+          bulk_load_hint(ps + sp * C::kPStage, cp.packed + ((int64_t)cp.rg * 8 * cp.B + (int64_t)cp.b * ntile) * ub,
+                         ntile * ub, &bars->pk_full[sp], pol_w);
         }
         __syncwarp();
         pos_next(cp, a);
@@ -421,9 +424,9 @@ __global__ void __launch_bounds__(kThreads, Cfg<XR, MODE>::kCtas) gemv_q_kernel(
         const uint8_t* xsrc = cx.xt + (int64_t)cx.b * xtb;
         if (elect_one()) {
           mbar_arrive_expect_tx(&bars->x_full[sx], bbytes);
-          bulk_load(xs + sx * C::kXStage, xsrc, bbytes, &bars->x_full[sx]);
+          bulk_load_hint(xs + sx * C::kXStage, xsrc, bbytes, &bars->x_full[sx], pol_x);
           mbar_arrive_expect_tx(&bars->c_full[sc], C::kRec);
-          bulk_load(cs + sc * C::kRec, xsrc + bbytes, C::kRec, &bars->c_full[sc]);
+          bulk_load_hint(cs + sc * C::kRec, xsrc + bbytes, C::kRec, &bars->c_full[sc], pol_x);
         }
         __syncwarp();
         pos_next(cx, a);
