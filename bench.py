@@ -30,6 +30,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "decode GEMV HBM GB/s (% of 8 TB/s) & tokens/s; prefill GEMM TFLOP/s (% peak)"
+E2E_QUARTERS = 4   # batched calls the end-to-end step splits the body into, to overlap host copies
 HBM_FALLBACK_GBS, BF16_FALLBACK_TFLOPS = 6650.0, 1590.0
 
 
@@ -358,17 +359,51 @@ def main():
         nbytes = sum(module_bytes(wr, M, m["N"], m["K"], m["bits"]) for m in mods)
         out = {"ms": ms, "bytes": nbytes, "gbs": nbytes / ms / 1e6, "launches": launches}
         if with_e2e:
+            # end to end from pinned host memory: the body in layer quarters, each one batched
+            # call; a quarter's x is copied in and its y copied out on side streams, so that the
+            # host transfers overlap the decode of the other quarters (every step moves all of x
+            # in and all of y out)
             xh = x_all.cpu().pin_memory()
             yh = torch.empty(y_all.numel(), dtype=torch.float32).pin_memory()
+            nq = E2E_QUARTERS
+            per = (len(mods) + nq - 1) // nq
+            quarters = []
+            for q in range(nq):
+                i0, i1 = q * per, min(len(mods), (q + 1) * per)
+                if i0 >= i1:
+                    break
+                xo0, xo1 = offs[i0], (offs[i1] if i1 < len(mods) else x_all.numel())
+                yo0, yo1 = yoffs[i0], (yoffs[i1] if i1 < len(mods) else y_all.numel())
+                arr_q = wr._problems([(xp + 2 * offs[i], mods[i]["packed"], mods[i]["scales"], yp + 4 * yoffs[i],
+                                       mods[i]["N"], mods[i]["K"], mods[i]["bits"]) for i in range(i0, i1)])
+                quarters.append((xo0, xo1, yo0, yo1, arr_q, wr.wr_gemv_batched_workspace_bytes(M, arr_q)))
+            nbq = max(q[5] for q in quarters)
+            wsq = torch.zeros(nbq, dtype=torch.uint8, device="cuda")   # the quarters run in turn on one stream
+            s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+            ev_in = [torch.cuda.Event() for _ in quarters]
+            ev_done = [torch.cuda.Event() for _ in quarters]
 
             def e2e_step():
-                x_all.copy_(xh, non_blocking=True)
-                step()
-                yh.copy_(y_all, non_blocking=True)
+                main = torch.cuda.current_stream()
+                s_in.wait_stream(main)
+                s_out.wait_stream(main)
+                with torch.cuda.stream(s_in):
+                    for (xo0, xo1, *_r), ev in zip(quarters, ev_in):
+                        x_all[xo0:xo1].copy_(xh[xo0:xo1], non_blocking=True)
+                        ev.record(s_in)
+                for (_, _, yo0, yo1, arr_q, _), ei, ed in zip(quarters, ev_in, ev_done):
+                    main.wait_event(ei)
+                    wr.wr_gemv_batched(M, arr_q, wsq, nbq)
+                    ed.record(main)
+                    with torch.cuda.stream(s_out):
+                        s_out.wait_event(ed)
+                        yh[yo0:yo1].copy_(y_all[yo0:yo1], non_blocking=True)
+                main.wait_stream(s_in)
+                main.wait_stream(s_out)
             ms_e = graph_time_ms(torch, e2e_step, steps, warmup, stream, dist) / steps
             ms_e = max_over_ranks(torch, dist, ms_e)
             out["e2e"] = {"ms": ms_e, "gbs": nbytes / ms_e / 1e6, "h2d": x_all.numel() * 2,
-                          "d2h": y_all.numel() * 4}
+                          "d2h": y_all.numel() * 4, "calls": len(quarters)}
         return out
 
     def dependent_body_run(M, steps, warmup):
@@ -414,6 +449,15 @@ def main():
             extras["body_m8"]["tokens_per_s"] = 8e3 / extras["body_m8"]["ms"]
         except Exception as e:  # noqa: BLE001
             extras["body_m8"] = {"error": repr(e)}
+        for M in (16, 32):
+            # a 16- or 32-token chunk through the body, one batched call: the decode kernel's
+            # 64- and 128-column forms
+            try:
+                extras[f"body_m{M}"] = body_run(M, max(5, args.steps // 2), 3, False)
+                extras[f"body_m{M}"]["tokens_per_s"] = M * 1e3 / extras[f"body_m{M}"]["ms"]
+                extras[f"body_m{M}"]["frac_of_hbm"] = extras[f"body_m{M}"]["gbs"] / hbm_peak
+            except Exception as e:  # noqa: BLE001
+                extras[f"body_m{M}"] = {"error": repr(e)}
         try:
             extras["body_m1_one_call_per_linear"] = body_run(1, max(5, args.steps // 2), 3, False, batched=False)
         except Exception as e:  # noqa: BLE001
@@ -455,7 +499,7 @@ def main():
         "roofline": roof, "cpu_baseline": cb, "clocks": clocks,
         "e2e": {"value": head["e2e"]["gbs"] * world, "unit": "GB/s",
                 "h2d_bytes_per_step": head["e2e"]["h2d"], "d2h_bytes_per_step": head["e2e"]["d2h"],
-                "ms_per_step": head["e2e"]["ms"]},
+                "ms_per_step": head["e2e"]["ms"], "calls_per_step": head["e2e"]["calls"]},
         "gpu_launches": head["launches"] * args.steps,
         "step": f"{7 * args.layers} linears ({args.layers} layers x 7) in one wr_gemv_batched call "
                 "(preparation pass + decode GEMV launch), CUDA graph replay",
