@@ -115,7 +115,7 @@ void plan_decode(int64_t M, int count, const ProblemShape* shapes, DecodePlan* d
   // ranges of at least the largest block cost in the batch, so that each holds a block (one
   // block per CTA for a small single-format batch), at most one wave of CTAs; two partial slots
   // per CTA of the launch (see DecArgs)
-  const int64_t wave = (int64_t)wr::decode_ctas_per_sm(ternary, (int)M) * kPlanSMs;
+  const int64_t wave = (int64_t)wr::decode_ctas_per_sm(ternary, (int)M, block_base) * kPlanSMs;
   dp->grid = (int)std::max<int64_t>(1, std::min<int64_t>(wave, cost_base / max_cost));
   // each CTA's first block and the problem that holds it
   for (int c = 0, pi = 0; c <= dp->grid; ++c) {

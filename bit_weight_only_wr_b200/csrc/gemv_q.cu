@@ -41,7 +41,8 @@
 //              whole warp walks the blocks, one elected lane issues).
 // Tensor memory (128 columns): one A buffer (64 columns) and two accumulators (32 columns). The
 // store of block i waits for the MMAs of block i - 1; block i's MMAs write accumulator i % 2
-// once the epilogue has read block i - 2 from it. Every wait is bounded.
+// once the epilogue has read block i - 2 from it (the 32-token form keeps one accumulator, see
+// Cfg). Every wait is bounded.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -56,8 +57,8 @@ namespace {
 using namespace tc;
 
 constexpr int kThreads = 320;
-constexpr int kSP = 4;   // packed stages: the 8 units of a row group's block
-constexpr int kSX = 3;   // B tiles; also the MMA-done ring
+constexpr int kSP = 4;   // packed stages: the 8 units of a row group's block (Cfg::kSPn may be fewer)
+constexpr int kSX = 3;   // B tiles; also the MMA-done ring (Cfg::kSXn may be fewer)
 constexpr int kSC = 4;   // correction records, 256 bytes
 
 // The three forms of the kernel: a batch of Q2/Q3 problems with fp16 scales (the lean form), a
@@ -69,24 +70,37 @@ enum { kModeLean = 0, kModeAll = 1, kModeTern = 2 };
 // atoms, the last half used), plus a 243-entry decode table replicated per lane (31 KB), so a CTA
 // needs more room; at MMA N = 16 or 32 two CTAs share an SM.
 // At MMA N = 64 or 128 (16 or 32 token slots, 2/3-bit forms only) the accumulators and B tiles
-// grow: two CTAs per SM at N = 64 (256 tensor-memory columns), one at N = 128 (512).
-template <int XR, int MODE>
+// grow: two CTAs per SM at N = 64 (256 tensor-memory columns), one at N = 128 (512). For a batch
+// of many blocks the N = 128 form instead keeps one accumulator (ONE: 192 columns, in an
+// allocation of 256) and shallower rings, so that two CTAs share an SM; block i + 1's MMAs then
+// wait for the epilogue to read block i (decode_one_acc picks the form).
+template <int XR, int MODE, bool ONE = false>
 struct Cfg {
   static constexpr bool kT = MODE == kModeTern;
-  static constexpr int kCtas = kT ? (XR > 8 ? 2 : 3) : (XR <= 32 ? 3 : (XR == 64 ? 2 : 1));
+  static constexpr bool kOneAcc = ONE && !kT && XR == 128;
+  static constexpr int kCtas = kT ? (XR > 8 ? 2 : 3) : (XR <= 32 ? 3 : (XR == 64 || kOneAcc ? 2 : 1));
+  static constexpr int kSXn = kOneAcc ? 2 : kSX;   // B-tile stages (and the MMA-done ring)
+  static constexpr int kSPn = kOneAcc ? 3 : kSP;   // weight stages
+  static constexpr int kDBufs = kOneAcc ? 1 : 2;   // accumulators
+  // accumulator of block g, and the parity of the epilogue's read that frees it for block g
+  __device__ static constexpr int dbuf(uint32_t g) { return kDBufs == 2 ? (int)(g & 1u) : 0; }
+  __device__ static constexpr uint32_t dfree_parity(uint32_t g) {
+    return kDBufs == 2 ? (((g >> 1) & 1u) ^ 1u) : ((g & 1u) ^ 1u);
+  }
   static constexpr int kPStage = 8 * (kT ? 1024 : 1536);
   static constexpr int kXStage = kT ? 3 * XR * 128 : (XR <= 32 ? 8 * 1024 : 2 * XR * 128);   // 1024-byte multiples
   static constexpr int kRec = kT ? 256 : (XR <= 64 ? 256 : 4 * XR);   // correction record per block
   static constexpr int kXOff = 0;
-  static constexpr int kPOff = kXOff + kSX * kXStage;
-  static constexpr int kCOff = kPOff + kSP * kPStage;
+  static constexpr int kPOff = kXOff + kSXn * kXStage;
+  static constexpr int kCOff = kPOff + kSPn * kPStage;
   static constexpr int kBarOff = kCOff + kSC * kRec;
   static constexpr int kSmem = kBarOff + 256 + 1024;   // + alignment slack
   static constexpr int kLutWords = kT ? 243 * 32 : 1;
   static constexpr int kACol = 0;
   static constexpr int kDCol = kT ? 96 : 64;           // two accumulators after the A buffer
   static constexpr int kDCols = kT ? XR : (XR < 32 ? 32 : XR);
-  static constexpr int kTmemCols = kDCol + 2 * kDCols <= 128 ? 128 : (kDCol + 2 * kDCols <= 256 ? 256 : 512);
+  static constexpr int kTmemCols =
+      kDCol + kDBufs * kDCols <= 128 ? 128 : (kDCol + kDBufs * kDCols <= 256 ? 256 : 512);
   static_assert(kCtas * (kSmem + 4 * kLutWords + 1024) <= 228 * 1024, "CTAs per SM by shared memory");
   static_assert(kCtas * kTmemCols <= 512, "tensor memory of an SM");
 };
@@ -324,9 +338,10 @@ __device__ __forceinline__ void tmem_wait_ld_regs(uint32_t (&r)[NC]) {
 // XR: MMA N, 4 limb rows per token slot (8, 16 or 32 for M <= 2, 4, 8). MODE: kModeLean keeps
 // only the Q2/Q3 decode branches and the fp16 scale load; kModeAll adds the trellis decode and
 // int8 block scales; kModeTern is the ternary batch (its decode table, 320-trit blocks, signed A).
-template <int XR, int MODE>
-__global__ void __launch_bounds__(kThreads, Cfg<XR, MODE>::kCtas) gemv_q_kernel(const __grid_constant__ DecArgs a) {
-  using C = Cfg<XR, MODE>;
+template <int XR, int MODE, bool ONE>
+__global__ void __launch_bounds__(kThreads, Cfg<XR, MODE, ONE>::kCtas)
+    gemv_q_kernel(const __grid_constant__ DecArgs a) {
+  using C = Cfg<XR, MODE, ONE>;
   constexpr bool kAll = MODE == kModeAll;
   constexpr bool kT = C::kT;
   extern __shared__ uint8_t smem_raw[];
@@ -357,11 +372,11 @@ __global__ void __launch_bounds__(kThreads, Cfg<XR, MODE>::kCtas) gemv_q_kernel(
   }
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kSP; ++i) {
+    for (int i = 0; i < C::kSPn; ++i) {
       mbar_init(&bars->pk_full[i], 1);
       mbar_init(&bars->pk_empty[i], 4);
     }
-    for (int i = 0; i < kSX; ++i) {
+    for (int i = 0; i < C::kSXn; ++i) {
       mbar_init(&bars->x_full[i], 1);
       mbar_init(&bars->mma_done[i], 1);
     }
@@ -384,8 +399,8 @@ __global__ void __launch_bounds__(kThreads, Cfg<XR, MODE>::kCtas) gemv_q_kernel(
 
   if (warp == 8) {
     // ------------------------------------------------------------ copy warp (whole warp walks the
-    // blocks, one elected lane issues): packed weights (a ring of kSP blocks), prepared B tiles
-    // and their correction records (a ring of kSX blocks)
+    // blocks, one elected lane issues): packed weights (a ring of kSPn blocks), prepared B tiles
+    // and their correction records (a ring of kSXn blocks)
     constexpr uint32_t bbytes = (kT ? 384u : 256u) * XR;
     constexpr uint32_t xtb = bbytes + (uint32_t)C::kRec;   // prepared tile: B atoms, then corrections
     Pos cp = pos_start(a), cx = cp;            // next block to copy: weights, activations
@@ -397,9 +412,9 @@ __global__ void __launch_bounds__(kThreads, Cfg<XR, MODE>::kCtas) gemv_q_kernel(
     bool ok = true;
     while (ok && (np < nblocks || nx < nblocks)) {
       if (np < nblocks) {
-        // weight stage np % kSP: free once the decode warps have read block np - kSP
-        const int sp = np % kSP;
-        if (!(ok = mbar_wait_bg(&bars->pk_empty[sp], ((np / kSP) & 1) ^ 1, abort_flag, a.err, 101))) break;
+        // weight stage np % kSPn: free once the decode warps have read block np - kSPn
+        const int sp = np % C::kSPn;
+        if (!(ok = mbar_wait_bg(&bars->pk_empty[sp], ((np / C::kSPn) & 1) ^ 1, abort_flag, a.err, 101))) break;
         const int ub = cp.bits == 3 ? 1536 : 1024;
         const int ntile = min(8, (cp.N + 15) / 16 - cp.rg * 8);
         if (elect_one()) {
@@ -411,15 +426,15 @@ __global__ void __launch_bounds__(kThreads, Cfg<XR, MODE>::kCtas) gemv_q_kernel(
         pos_next(cp, a);
         ++np;
       }
-      if (nx < nblocks && np >= min(nblocks, (uint32_t)kSP)) {
+      if (nx < nblocks && np >= min(nblocks, (uint32_t)C::kSPn)) {
         // the activation tiles come from the preparation pass, which may still be running (the
         // kernel is launched as its programmatic dependent): the first weight copies above are
         // issued before waiting for it
         if (nx == 0) grid_dependency_wait();
-        // activation stage nx % kSX: free once block nx - kSX's MMAs are done; correction slot
+        // activation stage nx % kSXn: free once block nx - kSXn's MMAs are done; correction slot
         // nx % kSC once the epilogue has read block nx - kSC
-        const int sx = nx % kSX, sc = nx % kSC;
-        if (!(ok = mbar_wait_bg(&bars->mma_done[sx], ((nx / kSX) & 1) ^ 1, abort_flag, a.err, 102))) break;
+        const int sx = nx % C::kSXn, sc = nx % kSC;
+        if (!(ok = mbar_wait_bg(&bars->mma_done[sx], ((nx / C::kSXn) & 1) ^ 1, abort_flag, a.err, 102))) break;
         if (!(ok = mbar_wait_bg(&bars->c_empty[sc], ((nx / kSC) & 1) ^ 1, abort_flag, a.err, 103))) break;
         const uint8_t* xsrc = cx.xt + (int64_t)cx.b * xtb;
         if (elect_one()) {
@@ -435,8 +450,10 @@ __global__ void __launch_bounds__(kThreads, Cfg<XR, MODE>::kCtas) gemv_q_kernel(
     }
     if (!ok) {
       // aborted: let the copies in flight land before the CTA exits
-      for (uint32_t k = np > kSP ? np - kSP : 0; k < np; ++k) mbar_wait_drain(&bars->pk_full[k % kSP], (k / kSP) & 1);
-      for (uint32_t k = nx > kSX ? nx - kSX : 0; k < nx; ++k) mbar_wait_drain(&bars->x_full[k % kSX], (k / kSX) & 1);
+      for (uint32_t k = np > C::kSPn ? np - C::kSPn : 0; k < np; ++k)
+        mbar_wait_drain(&bars->pk_full[k % C::kSPn], (k / C::kSPn) & 1);
+      for (uint32_t k = nx > C::kSXn ? nx - C::kSXn : 0; k < nx; ++k)
+        mbar_wait_drain(&bars->x_full[k % C::kSXn], (k / C::kSXn) & 1);
       for (uint32_t k = nx > kSC ? nx - kSC : 0; k < nx; ++k) mbar_wait_drain(&bars->c_full[k % kSC], (k / kSC) & 1);
     }
   } else if (warp == 9) {
@@ -449,23 +466,23 @@ __global__ void __launch_bounds__(kThreads, Cfg<XR, MODE>::kCtas) gemv_q_kernel(
     uint32_t gm = 0;
     bool ok = true;
     for (; gm < nblocks; ++gm) {
-      const int sx = gm % kSX;
+      const int sx = gm % C::kSXn;
       // the B tile and the accumulator are normally ready long before the codes: wait for them
       // first, so that the wait for the A handoff is the last one before the MMAs
-      if (!(ok = mbar_wait(&bars->x_full[sx], (gm / kSX) & 1, abort_flag, a.err, 202))) break;
-      // accumulator gm % 2 was read by the epilogue warps (block gm - 2)
-      if (!(ok = mbar_wait(&bars->d_empty[gm & 1], ((gm >> 1) & 1) ^ 1, abort_flag, a.err, 203))) break;
+      if (!(ok = mbar_wait(&bars->x_full[sx], (gm / C::kSXn) & 1, abort_flag, a.err, 202))) break;
+      // the accumulator of block gm was read by the epilogue warps (block gm - 2, or gm - 1 with one accumulator)
+      if (!(ok = mbar_wait(&bars->d_empty[C::dbuf(gm)], C::dfree_parity(gm), abort_flag, a.err, 203))) break;
       if (!(ok = mbar_wait(&bars->a_full, gm & 1, abort_flag, a.err, 201))) break;
       fence_after_sync();
       if constexpr (kT)
-        mma10_i8_commit_elect(tmem + C::kDCol + (gm & 1) * C::kDCols, tmem + C::kACol,
+        mma10_i8_commit_elect(tmem + C::kDCol + C::dbuf(gm) * C::kDCols, tmem + C::kACol,
                               bdesc0 + (uint64_t)((sx * C::kXStage) >> 4), atom16, idesc, &bars->mma_done[sx]);
       else
-        mma8_i8_commit_elect(tmem + C::kDCol + (gm & 1) * C::kDCols, tmem + C::kACol,
+        mma8_i8_commit_elect(tmem + C::kDCol + C::dbuf(gm) * C::kDCols, tmem + C::kACol,
                              bdesc0 + (uint64_t)((sx * C::kXStage) >> 4), atom16, idesc, &bars->mma_done[sx]);
     }
     // the MMAs already issued finish before tensor memory is released
-    if (!ok && gm > 0) mbar_wait_drain(&bars->mma_done[(gm - 1) % kSX], ((gm - 1) / kSX) & 1);
+    if (!ok && gm > 0) mbar_wait_drain(&bars->mma_done[(gm - 1) % C::kSXn], ((gm - 1) / C::kSXn) & 1);
   } else if (warp < 4) {
     // ------------------------------------------------------------ decode (warps 0-3, thread = row)
     const int t = threadIdx.x;                          // row in the row group = TMEM lane
@@ -473,8 +490,8 @@ __global__ void __launch_bounds__(kThreads, Cfg<XR, MODE>::kCtas) gemv_q_kernel(
     const uint32_t lane_base = tmem + ((uint32_t)(32 * warp) << 16);
     Lite dc = lite_of(pos_start(a));
     for (uint32_t gd = 0; dc.left > 0; ++gd) {
-      const int sp = gd % kSP;
-      if (!mbar_wait(&bars->pk_full[sp], (gd / kSP) & 1, abort_flag, a.err, 301)) break;
+      const int sp = gd % C::kSPn;
+      if (!mbar_wait(&bars->pk_full[sp], (gd / C::kSPn) & 1, abort_flag, a.err, 301)) break;
       if constexpr (kT) {
         // ternary: four quarters of 20 columns (4 packed words, then 16 table entries), each
         // stored as soon as it is decoded
@@ -482,7 +499,9 @@ __global__ void __launch_bounds__(kThreads, Cfg<XR, MODE>::kCtas) gemv_q_kernel(
         uint32_t raw[4], lv[16];
         tern_quarter_i8(unit, r0, half, 0, tlut, lane, raw, lv);
         // the A buffer is free once block gd - 1's MMAs are done
-        if (gd > 0 && !mbar_wait(&bars->mma_done[(gd - 1) % kSX], ((gd - 1) / kSX) & 1, abort_flag, a.err, 302)) break;
+        if (gd > 0 &&
+            !mbar_wait(&bars->mma_done[(gd - 1) % C::kSXn], ((gd - 1) / C::kSXn) & 1, abort_flag, a.err, 302))
+          break;
         fence_after_sync();
         tmem_st4(lane_base + C::kACol, raw);
         tmem_st16(lane_base + C::kACol + 16, lv);
@@ -503,7 +522,9 @@ __global__ void __launch_bounds__(kThreads, Cfg<XR, MODE>::kCtas) gemv_q_kernel(
         else if (dc.bits == WR_FMT_T2) t2_half_i8(unit, r0, half, 0, v, carry);
         else t8_half_i8(unit, r0, half, 0, v, carry);
         // the A buffer is free once block gd - 1's MMAs are done
-        if (gd > 0 && !mbar_wait(&bars->mma_done[(gd - 1) % kSX], ((gd - 1) / kSX) & 1, abort_flag, a.err, 302)) break;
+        if (gd > 0 &&
+            !mbar_wait(&bars->mma_done[(gd - 1) % C::kSXn], ((gd - 1) / C::kSXn) & 1, abort_flag, a.err, 302))
+          break;
         fence_after_sync();
         tmem_st32(lane_base + C::kACol, v);
         if (dc.bits == 2) q2_half_i8(unit, r0, half, 1, v);
@@ -561,7 +582,7 @@ __global__ void __launch_bounds__(kThreads, Cfg<XR, MODE>::kCtas) gemv_q_kernel(
       const uint16_t sraw = snext;
       const int qraw = qnext;
       const int sc = ge % kSC;
-      if (!mbar_wait(&bars->mma_done[ge % kSX], (ge / kSX) & 1, abort_flag, a.err, 303)) break;
+      if (!mbar_wait(&bars->mma_done[ge % C::kSXn], (ge / C::kSXn) & 1, abort_flag, a.err, 303)) break;
       if (!mbar_wait(&bars->c_full[sc], (ge / kSC) & 1, abort_flag, a.err, 304)) break;
       fence_after_sync();
       const int4* rec = reinterpret_cast<const int4*>(cs + sc * C::kRec);
@@ -574,7 +595,7 @@ __global__ void __launch_bounds__(kThreads, Cfg<XR, MODE>::kCtas) gemv_q_kernel(
       for (int c0 = 0; c0 < XR; c0 += kChunk) {
         if (c0 / 4 >= M) break;
         uint32_t d[kChunk];
-        tmem_ld_raw<kChunk>(lane_base + C::kDCol + (ge & 1) * C::kDCols + c0, d);
+        tmem_ld_raw<kChunk>(lane_base + C::kDCol + C::dbuf(ge) * C::kDCols + c0, d);
         tmem_wait_ld_regs<kChunk>(d);
 #pragma unroll
         for (int mm = 0; mm < kChunk / 4; ++mm) {
@@ -602,7 +623,7 @@ __global__ void __launch_bounds__(kThreads, Cfg<XR, MODE>::kCtas) gemv_q_kernel(
       fence_before_sync();
       __syncwarp();
       if (lane == 0) {
-        mbar_arrive(&bars->d_empty[ge & 1]);
+        mbar_arrive(&bars->d_empty[C::dbuf(ge)]);
         mbar_arrive(&bars->c_empty[sc]);
       }
       if (ec.b + 1 == ec.B || ec.left == 1) {
@@ -886,17 +907,17 @@ cudaError_t launch_prep_x(const DecArgs& a, int total_blocks, cudaStream_t strea
 }
 
 namespace {
-template <int XR, int MODE>
+template <int XR, int MODE, bool ONE = false>
 cudaError_t launch_xr(const DecArgs& a, int grid, cudaStream_t stream) {
-  using C = Cfg<XR, MODE>;
+  using C = Cfg<XR, MODE, ONE>;
   static bool set[64] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
   if (!set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(gemv_q_kernel<XR, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+    cudaError_t e = cudaFuncSetAttribute(gemv_q_kernel<XR, MODE, ONE>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
     // all of the unified L1/shared array as shared memory, so that the CTAs fit
     if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(gemv_q_kernel<XR, MODE>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+      e = cudaFuncSetAttribute(gemv_q_kernel<XR, MODE, ONE>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
     if (e != cudaSuccess) return e;
     set[dev] = true;
   }
@@ -911,7 +932,7 @@ cudaError_t launch_xr(const DecArgs& a, int grid, cudaStream_t stream) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, gemv_q_kernel<XR, MODE>, a);
+  return cudaLaunchKernelEx(&cfg, gemv_q_kernel<XR, MODE, ONE>, a);
 }
 
 template <int MODE>
@@ -924,7 +945,10 @@ cudaError_t launch_mode(const DecArgs& a, int grid, cudaStream_t stream) {
       if constexpr (MODE != kModeTern) return launch_xr<64, MODE>(a, grid, stream);
       return cudaErrorInvalidValue;
     default:
-      if constexpr (MODE != kModeTern) return launch_xr<128, MODE>(a, grid, stream);
+      if constexpr (MODE != kModeTern) {
+        if (decode_one_acc(a.M, a.total)) return launch_xr<128, MODE, true>(a, grid, stream);
+        return launch_xr<128, MODE>(a, grid, stream);
+      }
       return cudaErrorInvalidValue;
   }
 }
@@ -941,10 +965,11 @@ cudaError_t launch_gemv_q(const DecArgs& a, int grid, cudaStream_t stream) {
 }
 
 // CTAs of one wave of the decode kernel for a batch of this kind on a 148-SM part.
-int decode_ctas_per_sm(bool ternary, int M) {
+int decode_ctas_per_sm(bool ternary, int M, int64_t total_blocks) {
   const int xr = decode_xrows(M);
   if (ternary) return xr > 8 ? 2 : 3;
-  return xr <= 32 ? 3 : (xr == 64 ? 2 : 1);
+  if (xr <= 32) return 3;
+  return xr == 64 || decode_one_acc(M, total_blocks) ? 2 : 1;
 }
 
 }  // namespace wr

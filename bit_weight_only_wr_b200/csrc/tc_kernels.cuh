@@ -105,7 +105,7 @@ __host__ __device__ inline int range_cta_of(const DecArgs& a, int G, const DecPr
 cudaError_t launch_prep_x(const DecArgs& a, int total_blocks, cudaStream_t stream);
 cudaError_t launch_gemv_q(const DecArgs& a, int grid, cudaStream_t stream);
 // CTAs that one SM holds of the decode GEMV kernel for this kind of batch.
-int decode_ctas_per_sm(bool ternary, int M);
+int decode_ctas_per_sm(bool ternary, int M, int64_t total_blocks);
 
 // One prepared activation tile per block, stored as the exact image of a shared-memory B stage
 // so that one bulk copy moves it (128-byte swizzle: 16-byte chunk c of a row r at c ^ (r % 8)):
@@ -125,6 +125,14 @@ __host__ __device__ inline int decode_rec_bytes(bool ternary, int M) {
 }
 __host__ __device__ inline int64_t xtile_bytes(bool ternary, int M) {
   return (int64_t)(ternary ? 3 : 2) * decode_xrows(M) * 128 + decode_rec_bytes(ternary, M);
+}
+// The 128-column (17..32 token) form of the 2/3-bit decode GEMV runs with one accumulator at two
+// CTAs per SM when the batch holds at least 8 blocks per such CTA (the 36-layer body at M = 32:
+// 1.09 -> 0.89 ms); below that, where the ranges are short and split row groups three or four
+// ways, with two accumulators at one CTA per SM (a 9728 x 2560 linear at M = 32: 21.6 vs 25.0 us).
+constexpr int64_t kOneAccBlocks = 8 * 2 * 148;
+__host__ __device__ inline bool decode_one_acc(int M, int64_t total_blocks) {
+  return decode_xrows(M) == 128 && total_blocks >= kOneAccBlocks;
 }
 
 cudaError_t launch_tc_kernel(int fmt, int bn, const TcArgs& a, const void* x_act, int64_t x_rows, int64_t x_k,

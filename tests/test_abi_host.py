@@ -273,7 +273,13 @@ def test_decode_plan_of_the_qwen3_body():
     shapes = [(N, K, bits) for _ in range(36) for (_, K, N, bits) in wr_synth.QWEN3_4B_LAYER]
     for M in (1, 3, 8):
         G, _ = _check_plan(M, shapes)
-        assert G == 444
+        assert G == 444      # three CTAs per SM of a 148-SM part
+    for M in (9, 16, 17, 32):
+        G, _ = _check_plan(M, shapes)
+        assert G == 296      # the 64- and 128-column forms: two CTAs per SM
+    # a lone 17..32-token linear keeps the two-accumulator form at one CTA per SM
+    G, _ = _check_plan(32, [(9728, 2560, 2)])
+    assert G == 148
     # a small single-format batch runs one block per CTA
     G, starts = _check_plan(1, [(2560, 2560, 2)])
     assert G == 200 and np.array_equal(starts, np.arange(201))

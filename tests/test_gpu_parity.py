@@ -529,3 +529,37 @@ def test_batched_at_16_tokens(wr):
         torch.cuda.synchronize()
         for p, (ref, B) in zip(problems, refs):
             check_close(p[3].cpu().numpy(), ref, B)
+
+
+@pytest.mark.parametrize("M", [24, 32])
+def test_batched_32_token_form_with_one_accumulator(wr, M):
+    """A batch of at least 8 blocks per CTA at 17..32 tokens runs the 128-column form with one
+    accumulator at two CTAs per SM (the plan's grid shows which form runs); all of y against the
+    oracle, twice on one workspace."""
+    torch = torch_mod()
+    shapes = [(9728, 2560, 2), (9728, 2560, 3), (2560, 9728, 3), (4096, 2560, 2)]
+    problems, refs = [], []
+    for i, (N, K, bits) in enumerate(shapes):
+        codes, scales, packed, s_d = q_case(wr, bits, N, K, seed=3500 + i)
+        x = wr_synth.activations_bf16(3510 + i + M, M, K)
+        refs.append(o.gemm_codes(x, codes, scales, bits))
+        y = torch.full((M, N), float("nan"), dtype=torch.float32, device="cuda")
+        problems.append((dev(x), packed, s_d, y, N, K, bits))
+    G, _, _ = wr.wr_gemv_batched_plan(M, problems)
+    assert G == 296
+    nb = wr.wr_gemv_batched_workspace_bytes(M, problems)
+    ws = _zeros_ws(nb)
+    for _ in range(2):
+        wr.wr_gemv_batched(M, problems, ws, nb)
+        torch.cuda.synchronize()
+        for p, (ref, B) in zip(problems, refs):
+            check_close(p[3].cpu().numpy(), ref, B)
+    assert wr.wr_get_device_error() == 0
+
+
+def test_single_32_token_call_keeps_two_accumulators(wr):
+    """A single linear at 32 tokens has too few blocks for the one-accumulator form: one CTA per
+    SM (grid at most 148)."""
+    probs = [(None, None, None, None, 9728, 2560, 2)]
+    G, _, _ = wr.wr_gemv_batched_plan(32, probs)
+    assert G <= 148
