@@ -563,3 +563,46 @@ def test_single_32_token_call_keeps_two_accumulators(wr):
     probs = [(None, None, None, None, 9728, 2560, 2)]
     G, _, _ = wr.wr_gemv_batched_plan(32, probs)
     assert G <= 148
+
+
+def test_batched_32_token_form_with_one_accumulator_all_formats(wr):
+    """The same one-accumulator form in the kernel build that also decodes trellis codes and int8
+    block scales: a batch of random codes in every 2-bit and 3-bit format, large enough for two
+    CTAs per SM at M = 24, all of y against the oracle."""
+    from gpu_inputs import s8_record
+    torch = torch_mod()
+    M = 24
+    rng = np.random.default_rng(3600)
+    spec = [(9728, 2560, "q3i8"), (9728, 2560, "q2"), (2560, 9728, "q3"), (1024, 2560, "q2i8"),
+            (256, 1024, "t8"), (512, 2560, "t2")]
+    problems, refs = [], []
+    for i, (N, K, kind) in enumerate(spec):
+        x = wr_synth.activations_bf16(3610 + i, M, K)
+        bits = 3 if kind.startswith("q3") else 2
+        codes = rng.integers(0, 1 << bits, (N, K)).astype(np.uint8)
+        if kind.endswith("i8"):
+            d = (np.float16(0.01) * (1 + rng.random(N))).astype(np.float16)
+            q = rng.integers(0, 128, (N, K // 256)).astype(np.int8)
+            fmt, s_d = bits | wr.WR_SCALES_I8, dev(s8_record(d, q))
+            ref = o.gemm_codes_s8(x, codes, d, q, bits)
+        else:
+            sc = (np.float16(0.01) * (1 + rng.random((N, K // 256)))).astype(np.float16)
+            s_d = dev(sc.view(np.uint16))
+            if kind == "t8":
+                fmt, ref = wr.WR_FMT_T8, o.gemm_trellis8(x, codes, sc)
+            elif kind == "t2":
+                fmt, ref = wr.WR_FMT_T2, o.gemm_trellis2(x, codes, sc)
+            else:
+                fmt, ref = bits, o.gemm_codes(x, codes, sc, bits)
+        y = torch.full((M, N), float("nan"), dtype=torch.float32, device="cuda")
+        problems.append((dev(x), dev(wr.wr_pack(fmt & 0xFF, codes)), s_d, y, N, K, fmt))
+        refs.append(ref)
+    G, _, _ = wr.wr_gemv_batched_plan(M, problems)
+    assert G == 296
+    nb = wr.wr_gemv_batched_workspace_bytes(M, problems)
+    ws = _zeros_ws(nb)
+    wr.wr_gemv_batched(M, problems, ws, nb)
+    torch.cuda.synchronize()
+    for p, (r, B) in zip(problems, refs):
+        check_close(p[3].cpu().numpy(), r, B)
+    assert wr.wr_get_device_error() == 0
