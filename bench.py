@@ -488,7 +488,9 @@ def main():
     line = {
         "metric": METRIC, "value": total_gbs, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": head["ms"], "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "vs_baseline": None, "dtype": "i8", "data": "synthetic",
+        "dtype_note": "int8 tensor-core products of the codes and four int8 limbs of each bf16 activation, "
+                      "int32 accumulators, fp32 epilogue; y is fp32",
         "tokens_per_s": tokens_per_s, "pct_of_8TBps": 100.0 * head["gbs"] / 8000.0,
         "config": {"workload": f"qwen3-4b body, {args.layers} layers x 7 packed GEMVs (v/up/down 3-bit, "
                                "others 2-bit, fp16 block-256 scales), M=%d decode" % args.tokens,
