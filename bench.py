@@ -145,6 +145,13 @@ def module_bytes(wr, M, N, K, bits):
 _TRAFFIC_RATIO = {1: (1_181_419_520 + 3_914_240) / 1_178_984_448, 8: (1_206_598_656 + 14_751_232) / 1_223_368_704}
 
 
+def split_ranges(n: int, parts: int):
+    """Consecutive index ranges [(i0, i1), ...] that cover range(n) in at most `parts` pieces of
+    ceil(n / parts) (the end-to-end step's batched calls)."""
+    per = (n + parts - 1) // parts
+    return [(i0, min(n, i0 + per)) for i0 in range(0, n, per)] if n > 0 else []
+
+
 def traffic_per_launch(M: int, layers: int, algo_bytes: int):
     r = _TRAFFIC_RATIO.get(M)
     return None if r is None else int(r * algo_bytes)
@@ -365,13 +372,8 @@ def main():
             # in and all of y out)
             xh = x_all.cpu().pin_memory()
             yh = torch.empty(y_all.numel(), dtype=torch.float32).pin_memory()
-            nq = E2E_QUARTERS
-            per = (len(mods) + nq - 1) // nq
             quarters = []
-            for q in range(nq):
-                i0, i1 = q * per, min(len(mods), (q + 1) * per)
-                if i0 >= i1:
-                    break
+            for i0, i1 in split_ranges(len(mods), E2E_QUARTERS):
                 xo0, xo1 = offs[i0], (offs[i1] if i1 < len(mods) else x_all.numel())
                 yo0, yo1 = yoffs[i0], (yoffs[i1] if i1 < len(mods) else y_all.numel())
                 arr_q = wr._problems([(xp + 2 * offs[i], mods[i]["packed"], mods[i]["scales"], yp + 4 * yoffs[i],

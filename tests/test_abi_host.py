@@ -280,6 +280,18 @@ def test_decode_plan_of_the_qwen3_body():
     # a lone 17..32-token linear keeps the two-accumulator form at one CTA per SM
     G, _ = _check_plan(32, [(9728, 2560, 2)])
     assert G == 148
+
+
+def test_decode_plan_switches_the_32_token_form_at_8_blocks_per_cta():
+    # 2368 blocks (8 per CTA at two CTAs per SM of 148) take the one-accumulator form, 2367 not
+    for M in (17, 32):
+        G, _ = _check_plan(M, [(128, 256 * 2368, 2)])
+        assert G == 296
+        G, _ = _check_plan(M, [(128, 256 * 2367, 2)])
+        assert G == 148
+    # the 16-token form is two CTAs per SM whatever the batch
+    G, _ = _check_plan(16, [(128, 256 * 2367, 2)])
+    assert G == 296
     # a small single-format batch runs one block per CTA
     G, starts = _check_plan(1, [(2560, 2560, 2)])
     assert G == 200 and np.array_equal(starts, np.arange(201))

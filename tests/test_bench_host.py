@@ -57,3 +57,15 @@ def test_two_rank_max_and_rank0_only():
         assert p.exitcode == 0
     assert res[0][0] == pytest.approx(2.5) and res[1][0] == pytest.approx(2.5)
     assert res[1][1] == ""
+
+
+def test_end_to_end_split_covers_every_problem_once():
+    sys.path.insert(0, ROOT)
+    import bench
+    for n in (0, 1, 3, 4, 7, 28, 252, 253):
+        for parts in (1, 2, 4, 8):
+            r = bench.split_ranges(n, parts)
+            assert len(r) <= parts
+            assert [i for a, b in r for i in range(a, b)] == list(range(n))
+            assert all(b > a for a, b in r)
+    assert bench.split_ranges(252, 4) == [(0, 63), (63, 126), (126, 189), (189, 252)]
